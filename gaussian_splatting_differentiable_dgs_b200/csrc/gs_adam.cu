@@ -1,0 +1,351 @@
+// Projection backward (stage 2 of the two-stage backward) and Adam.
+//
+// BoundedGS project page, section 02 (A -> B): raster backward first
+// collects the projected-attribute gradients; projection backward runs
+// after the raster buffers are gone.  Section 01: the whole view's gradient
+// is summed before ONE parameter update.  SkipGS paper notes, "loss
+// function / training strategy": gradients reach means, quaternions, scales,
+// opacities and SH coefficients and Adam updates the parameters.
+//
+// The fused variant runs one thread per Gaussian over all n: candidates
+// differentiate their projection and update their parameters in the same
+// pass; non-candidates take the Adam step with a zero gradient.  Parameters,
+// moments and gradients stream through once (24 bytes per float), and the
+// compact 3D gradients are never materialised.
+#include <math.h>
+
+#include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kThreads = 256;
+
+struct BwdCam {
+  double R[9], t[3], fx, fy, campos[3];
+};
+
+struct AdamK {
+  float lr, b1, b2, eps, bc1, bc2;
+};
+
+__device__ __forceinline__ void adam_update(float* __restrict__ p, float* __restrict__ m,
+                                            float* __restrict__ v, int64_t idx, float g,
+                                            const AdamK& a) {
+  const float mm = fmaf(a.b1, m[idx], (1.0f - a.b1) * g);
+  const float vv = fmaf(a.b2, v[idx], (1.0f - a.b2) * g * g);
+  m[idx] = mm;
+  v[idx] = vv;
+  const float mh = mm / a.bc1;
+  const float vh = vv / a.bc2;
+  p[idx] = p[idx] - a.lr * mh / (sqrtf(vh) + a.eps);
+}
+
+// Gradients of one candidate.  `emit(plane, g)` receives every parameter's
+// gradient exactly once, SH planes first, then planes 10 .. 0.
+template <class Emit>
+__device__ __forceinline__ void candidate_grad(const float* __restrict__ P, int64_t n_pad, int64_t i,
+                                               int D, const BwdCam& c, const float* __restrict__ g2,
+                                               const float4 rgb_rec, Emit&& emit) {
+  const double mx = P[i], my = P[n_pad + i], mz = P[2 * n_pad + i];
+  double tc[3];
+#pragma unroll
+  for (int r = 0; r < 3; ++r) tc[r] = c.R[3 * r] * mx + c.R[3 * r + 1] * my + c.R[3 * r + 2] * mz + c.t[r];
+  const double tx = tc[0], ty = tc[1], tz = tc[2];
+  double qw = P[6 * n_pad + i], qx = P[7 * n_pad + i], qy = P[8 * n_pad + i], qz = P[9 * n_pad + i];
+  const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+  qw /= qn; qx /= qn; qy /= qn; qz /= qn;
+  double Rg[9];
+  Rg[0] = 1.0 - 2.0 * (qy * qy + qz * qz); Rg[1] = 2.0 * (qx * qy - qw * qz); Rg[2] = 2.0 * (qx * qz + qw * qy);
+  Rg[3] = 2.0 * (qx * qy + qw * qz); Rg[4] = 1.0 - 2.0 * (qx * qx + qz * qz); Rg[5] = 2.0 * (qy * qz - qw * qx);
+  Rg[6] = 2.0 * (qx * qz - qw * qy); Rg[7] = 2.0 * (qy * qz + qw * qx); Rg[8] = 1.0 - 2.0 * (qx * qx + qy * qy);
+  double sc[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) sc[k] = exp((double)P[(3 + k) * n_pad + i]);
+  double M[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) M[3 * r + k] = Rg[3 * r + k] * sc[k];
+  double Sg[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      Sg[3 * r + k] = M[3 * r] * M[3 * k] + M[3 * r + 1] * M[3 * k + 1] + M[3 * r + 2] * M[3 * k + 2];
+  const double tz2 = tz * tz;
+  const double j00 = c.fx / tz, j02 = -c.fx * tx / tz2, j11 = c.fy / tz, j12 = -c.fy * ty / tz2;
+  double T0[3], T1[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    T0[k] = j00 * c.R[k] + j02 * c.R[6 + k];
+    T1[k] = j11 * c.R[3 + k] + j12 * c.R[6 + k];
+  }
+  double A0[3], A1[3];  // rows of T Sigma
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    A0[k] = T0[0] * Sg[k] + T0[1] * Sg[3 + k] + T0[2] * Sg[6 + k];
+    A1[k] = T1[0] * Sg[k] + T1[1] * Sg[3 + k] + T1[2] * Sg[6 + k];
+  }
+  const double c00 = A0[0] * T0[0] + A0[1] * T0[1] + A0[2] * T0[2] + 0.3;
+  const double c01 = 0.5 * ((A0[0] * T1[0] + A0[1] * T1[1] + A0[2] * T1[2]) +
+                            (A1[0] * T0[0] + A1[1] * T0[1] + A1[2] * T0[2]));
+  const double c11 = A1[0] * T1[0] + A1[1] * T1[1] + A1[2] * T1[2] + 0.3;
+  const double det = c00 * c11 - c01 * c01;
+  const double qa = c11 / det, qb = -c01 / det, qc = c00 / det;  // conic
+
+  const double du = g2[0], dv = g2[1], dA = g2[2], dB = g2[3], dC = g2[4], dO = g2[5];
+  const double dcol[3] = {g2[6], g2[7], g2[8]};
+
+  // conic -> Sigma': dS = -Q Gbar Q,  Gbar = [[dA, dB/2], [dB/2, dC]]
+  const double hB = 0.5 * dB;
+  const double m00 = qa * dA + qb * hB, m01 = qa * hB + qb * dC;
+  const double m10 = qb * dA + qc * hB, m11 = qb * hB + qc * dC;
+  const double G00 = -(m00 * qa + m01 * qb);
+  const double G01 = -(m00 * qb + m01 * qc);
+  const double G11 = -(m10 * qb + m11 * qc);
+  // Sigma' = T Sigma T^T + 0.3 I  ->  dSigma = T^T G T,  dT = 2 G T Sigma
+  double dS[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      dS[3 * r + k] = T0[r] * (G00 * T0[k] + G01 * T1[k]) + T1[r] * (G01 * T0[k] + G11 * T1[k]);
+  double dT0[3], dT1[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    dT0[k] = 2.0 * (G00 * A0[k] + G01 * A1[k]);
+    dT1[k] = 2.0 * (G01 * A0[k] + G11 * A1[k]);
+  }
+  // T = J W
+  const double dJ00 = dT0[0] * c.R[0] + dT0[1] * c.R[1] + dT0[2] * c.R[2];
+  const double dJ02 = dT0[0] * c.R[6] + dT0[1] * c.R[7] + dT0[2] * c.R[8];
+  const double dJ11 = dT1[0] * c.R[3] + dT1[1] * c.R[4] + dT1[2] * c.R[5];
+  const double dJ12 = dT1[0] * c.R[6] + dT1[1] * c.R[7] + dT1[2] * c.R[8];
+  const double tz3 = tz2 * tz;
+  const double dtx = -dJ02 * c.fx / tz2 + du * c.fx / tz;
+  const double dty = -dJ12 * c.fy / tz2 + dv * c.fy / tz;
+  const double dtz = -dJ00 * c.fx / tz2 + dJ02 * 2.0 * c.fx * tx / tz3 - dJ11 * c.fy / tz2 +
+                     dJ12 * 2.0 * c.fy * ty / tz3 - du * c.fx * tx / tz2 - dv * c.fy * ty / tz2;
+  double dmean[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) dmean[k] = c.R[k] * dtx + c.R[3 + k] * dty + c.R[6 + k] * dtz;
+  // Sigma = M M^T,  M = R S
+  double dM[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      dM[3 * r + k] = 2.0 * (dS[3 * r] * M[k] + dS[3 * r + 1] * M[3 + k] + dS[3 * r + 2] * M[6 + k]);
+  double dls[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k)
+    dls[k] = (dM[k] * Rg[k] + dM[3 + k] * Rg[3 + k] + dM[6 + k] * Rg[6 + k]) * sc[k];
+  double gR[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) gR[3 * r + k] = dM[3 * r + k] * sc[k];
+  // rotation of the unit quaternion -> (w, x, y, z)
+  const double gw = 2.0 * (-qz * gR[1] + qy * gR[2] + qz * gR[3] - qx * gR[5] - qy * gR[6] + qx * gR[7]);
+  const double gx = 2.0 * (qy * gR[1] + qz * gR[2] + qy * gR[3] - 2.0 * qx * gR[4] - qw * gR[5] +
+                           qz * gR[6] + qw * gR[7] - 2.0 * qx * gR[8]);
+  const double gy = 2.0 * (-2.0 * qy * gR[0] + qx * gR[1] + qw * gR[2] + qx * gR[3] + qz * gR[5] -
+                           qw * gR[6] + qz * gR[7] - 2.0 * qy * gR[8]);
+  const double gz = 2.0 * (-2.0 * qz * gR[0] - qw * gR[1] + qx * gR[2] + qw * gR[3] - 2.0 * qz * gR[4] +
+                           qy * gR[5] + qx * gR[6] + qy * gR[7]);
+  const double qdot = gw * qw + gx * qx + gy * qy + gz * qz;
+  const double dq[4] = {(gw - qw * qdot) / qn, (gx - qx * qdot) / qn, (gy - qy * qdot) / qn,
+                        (gz - qz * qdot) / qn};
+  // opacity logit
+  const double o = 1.0 / (1.0 + exp(-(double)P[10 * n_pad + i]));
+  const double dlogit = dO * o * (1.0 - o);
+
+  // SH coefficients and the view direction
+  double ex = mx - c.campos[0], ey = my - c.campos[1], ez = mz - c.campos[2];
+  const double en = sqrt(ex * ex + ey * ey + ez * ez);
+  ex /= en; ey /= en; ez /= en;
+  const bool live[3] = {rgb_rec.x > 0.0f, rgb_rec.y > 0.0f, rgb_rec.z > 0.0f};
+  const double kPi = 3.141592653589793;
+  double Y[16], dY[16][3];
+  {
+    const double x = ex, y = ey, z = ez, xx = x * x, yy = y * y, zz = z * z;
+    Y[0] = 0.5 / sqrt(kPi);
+    dY[0][0] = dY[0][1] = dY[0][2] = 0.0;
+    const double k1 = sqrt(3.0 / (4.0 * kPi));
+    Y[1] = -k1 * y; dY[1][0] = 0; dY[1][1] = -k1; dY[1][2] = 0;
+    Y[2] = k1 * z; dY[2][0] = 0; dY[2][1] = 0; dY[2][2] = k1;
+    Y[3] = -k1 * x; dY[3][0] = -k1; dY[3][1] = 0; dY[3][2] = 0;
+    const double k2a = 0.5 * sqrt(15.0 / kPi), k2b = 0.25 * sqrt(5.0 / kPi), k2c = 0.25 * sqrt(15.0 / kPi);
+    Y[4] = k2a * x * y; dY[4][0] = k2a * y; dY[4][1] = k2a * x; dY[4][2] = 0;
+    Y[5] = -k2a * y * z; dY[5][0] = 0; dY[5][1] = -k2a * z; dY[5][2] = -k2a * y;
+    Y[6] = k2b * (2 * zz - xx - yy); dY[6][0] = -2 * k2b * x; dY[6][1] = -2 * k2b * y; dY[6][2] = 4 * k2b * z;
+    Y[7] = -k2a * x * z; dY[7][0] = -k2a * z; dY[7][1] = 0; dY[7][2] = -k2a * x;
+    Y[8] = k2c * (xx - yy); dY[8][0] = 2 * k2c * x; dY[8][1] = -2 * k2c * y; dY[8][2] = 0;
+    const double k3a = 0.25 * sqrt(35.0 / (2.0 * kPi)), k3b = 0.5 * sqrt(105.0 / kPi),
+                 k3c = 0.25 * sqrt(21.0 / (2.0 * kPi)), k3d = 0.25 * sqrt(7.0 / kPi),
+                 k3e = 0.25 * sqrt(105.0 / kPi);
+    Y[9] = -k3a * y * (3 * xx - yy); dY[9][0] = -6 * k3a * x * y; dY[9][1] = -3 * k3a * (xx - yy); dY[9][2] = 0;
+    Y[10] = k3b * x * y * z; dY[10][0] = k3b * y * z; dY[10][1] = k3b * x * z; dY[10][2] = k3b * x * y;
+    Y[11] = -k3c * y * (4 * zz - xx - yy); dY[11][0] = 2 * k3c * x * y;
+    dY[11][1] = -k3c * (4 * zz - xx - 3 * yy); dY[11][2] = -8 * k3c * y * z;
+    Y[12] = k3d * z * (2 * zz - 3 * xx - 3 * yy); dY[12][0] = -6 * k3d * x * z; dY[12][1] = -6 * k3d * y * z;
+    dY[12][2] = k3d * (6 * zz - 3 * xx - 3 * yy);
+    Y[13] = -k3c * x * (4 * zz - xx - yy); dY[13][0] = -k3c * (4 * zz - 3 * xx - yy);
+    dY[13][1] = 2 * k3c * x * y; dY[13][2] = -8 * k3c * x * z;
+    Y[14] = k3e * z * (xx - yy); dY[14][0] = 2 * k3e * x * z; dY[14][1] = -2 * k3e * y * z; dY[14][2] = k3e * (xx - yy);
+    Y[15] = -k3a * x * (xx - 3 * yy); dY[15][0] = -3 * k3a * (xx - yy); dY[15][1] = 6 * k3a * x * y; dY[15][2] = 0;
+  }
+  const int ksh = (D + 1) * (D + 1);
+  double dd[3] = {0.0, 0.0, 0.0};
+  for (int k = 0; k < ksh; ++k) {
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) {
+      const int plane = 11 + 3 * k + ch;
+      double g = 0.0;
+      if (live[ch]) {
+        g = dcol[ch] * Y[k];
+        const double coef = dcol[ch] * (double)P[plane * n_pad + i];
+        dd[0] += coef * dY[k][0];
+        dd[1] += coef * dY[k][1];
+        dd[2] += coef * dY[k][2];
+      }
+      emit(plane, (float)g);
+    }
+  }
+  const double ddot = dd[0] * ex + dd[1] * ey + dd[2] * ez;
+  dmean[0] += (dd[0] - ex * ddot) / en;
+  dmean[1] += (dd[1] - ey * ddot) / en;
+  dmean[2] += (dd[2] - ez * ddot) / en;
+  emit(10, (float)dlogit);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) emit(6 + k, (float)dq[k]);
+#pragma unroll
+  for (int k = 0; k < 3; ++k) emit(3 + k, (float)dls[k]);
+#pragma unroll
+  for (int k = 0; k < 3; ++k) emit(k, (float)dmean[k]);
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_project_bwd(const float* __restrict__ P, int64_t n_pad, int D, BwdCam cam, int64_t n_cand,
+              const int32_t* __restrict__ cand_idx, const float4* __restrict__ rec,
+              const float* __restrict__ g2d, float* __restrict__ g3d, int64_t stride) {
+  const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (j >= n_cand) return;
+  const int64_t i = cand_idx[j];
+  candidate_grad(P, n_pad, i, D, cam, g2d + 12 * j, rec[3 * j + 2],
+                 [&](int plane, float g) { g3d[(int64_t)plane * stride + j] = g; });
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_project_bwd_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
+                   int64_t n, int64_t n_pad, int D, int nP, BwdCam cam,
+                   const int32_t* __restrict__ slot_map, const float4* __restrict__ rec,
+                   const float* __restrict__ g2d, AdamK a) {
+  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (i >= n) return;
+  const int32_t s = slot_map[i];
+  if (s >= 0) {
+    // gradients of the candidate; each plane is updated as soon as its
+    // gradient is known (the SH planes before the mean, which needs the
+    // view-direction term)
+    candidate_grad(P, n_pad, i, D, cam, g2d + 12 * (int64_t)s, rec[3 * (int64_t)s + 2],
+                   [&](int plane, float g) { adam_update(P, m, v, (int64_t)plane * n_pad + i, g, a); });
+  } else {
+    for (int plane = 0; plane < nP; ++plane) adam_update(P, m, v, (int64_t)plane * n_pad + i, 0.0f, a);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
+       const float* __restrict__ g, int64_t g_stride, const int32_t* __restrict__ slot, int64_t n,
+       int64_t n_pad, int nP, AdamK a) {
+  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (i >= n) return;
+  int64_t col = i;
+  bool has = true;
+  if (slot) {
+    const int32_t s = slot[i];
+    has = s >= 0;
+    col = s;
+  }
+  for (int plane = 0; plane < nP; ++plane) {
+    const float gg = has ? g[(int64_t)plane * g_stride + col] : 0.0f;
+    adam_update(P, m, v, (int64_t)plane * n_pad + i, gg, a);
+  }
+}
+
+BwdCam make_cam(const gs_camera* cam) {
+  BwdCam c;
+  for (int k = 0; k < 9; ++k) c.R[k] = cam->R[k];
+  for (int k = 0; k < 3; ++k) c.t[k] = cam->t[k];
+  c.fx = cam->fx;
+  c.fy = cam->fy;
+  for (int k = 0; k < 3; ++k)
+    c.campos[k] = -(c.R[k] * c.t[0] + c.R[3 + k] * c.t[1] + c.R[6 + k] * c.t[2]);
+  return c;
+}
+
+bool make_adam(const gs_adam_args* args, AdamK* a) {
+  if (!args || args->step < 1 || !(args->lr >= 0) || !(args->beta1 >= 0 && args->beta1 < 1) ||
+      !(args->beta2 >= 0 && args->beta2 < 1) || !(args->eps > 0))
+    return false;
+  a->lr = args->lr;
+  a->b1 = args->beta1;
+  a->b2 = args->beta2;
+  a->eps = args->eps;
+  a->bc1 = (float)(1.0 - pow((double)args->beta1, (double)args->step));
+  a->bc2 = (float)(1.0 - pow((double)args->beta2, (double)args->step));
+  return true;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
+                                    const gs_proj* proj, int64_t n_cand, const float* g2d,
+                                    float* g3d, int64_t g3d_stride, float* adam_m, float* adam_v,
+                                    const gs_adam_args* fused, int32_t* dev_status,
+                                    gs_stream stream) {
+  (void)dev_status;
+  if (!model || !cam || !proj || n_cand < 0 || n_cand > proj->capacity) return GS_ERR_ARG;
+  if (model->sh_degree < 0 || model->sh_degree > 3 || model->n_pad < model->n) return GS_ERR_ARG;
+  if (n_cand > 0 && (!g2d || !proj->rec || !aligned(g2d, 16))) return GS_ERR_ARG;
+  const BwdCam c = make_cam(cam);
+  const int D = model->sh_degree;
+  const int nP = 11 + 3 * (D + 1) * (D + 1);
+  cudaStream_t s = to_stream(stream);
+  const float4* rec = reinterpret_cast<const float4*>(proj->rec);
+  if (!fused) {
+    if (n_cand == 0) return GS_OK;
+    if (!g3d || g3d_stride < n_cand || !proj->cand_idx) return GS_ERR_ARG;
+    k_project_bwd<<<(unsigned)((n_cand + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        model->params, model->n_pad, D, c, n_cand, proj->cand_idx, rec, g2d, g3d, g3d_stride);
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+  }
+  AdamK a;
+  if (!make_adam(fused, &a)) return GS_ERR_ARG;
+  if (!adam_m || !adam_v || !proj->slot) return GS_ERR_ARG;
+  if (model->n == 0) return GS_OK;
+  k_project_bwd_adam<<<(unsigned)((model->n + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+      model->params, adam_m, adam_v, model->n, model->n_pad, D, nP, c, proj->slot, rec, g2d, a);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" gs_status gs_adam(float* params, float* m, float* v, const float* g, int64_t g_stride,
+                             const int32_t* slot, int64_t n, int64_t n_pad, int32_t P,
+                             const gs_adam_args* args, gs_stream stream) {
+  AdamK a;
+  if (!make_adam(args, &a) || n < 0 || n_pad < n || P <= 0) return GS_ERR_ARG;
+  if (n == 0) return GS_OK;
+  if (!params || !m || !v || !g) return GS_ERR_ARG;
+  if (!slot && g_stride < n) return GS_ERR_ARG;
+  k_adam<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, to_stream(stream)>>>(
+      params, m, v, g, g_stride, slot, n, n_pad, P, a);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}

@@ -1,0 +1,154 @@
+// Internal helpers of libgs (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gs.h"
+
+#define GS_TRY(expr)                                   \
+  do {                                                 \
+    cudaError_t e_ = (expr);                           \
+    if (e_ != cudaSuccess) return GS_ERR_CUDA;         \
+  } while (0)
+
+#define GS_LAUNCH_CHECK() GS_TRY(cudaGetLastError())
+
+namespace gs {
+
+constexpr int kTile = GS_TILE;
+// Iteration cap of every device spin-wait (each poll sleeps ~64-256 ns),
+// i.e. a bound of roughly a quarter of a second before giving up.
+constexpr int kSpinCap = 1 << 20;
+
+inline cudaStream_t to_stream(gs_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+inline int64_t tiles_x(int32_t w) { return (w + kTile - 1) / kTile; }
+inline int64_t tiles_y(int32_t h) { return (h + kTile - 1) / kTile; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Carves typed sub-buffers out of a caller workspace (256-byte aligned).
+struct Carver {
+  char* base;
+  size_t cap, off;
+  explicit Carver(void* b, size_t c) : base(static_cast<char*>(b)), cap(c), off(0) {}
+  template <class T>
+  T* take(size_t count) {
+    off = round_up(off, 256);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+  bool ok() const { return off <= cap; }
+};
+
+__device__ __forceinline__ void dev_flag(int32_t* st, uint32_t bit) {
+  if (st) atomicOr(reinterpret_cast<unsigned int*>(st), bit);
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// warp / block scans
+// ---------------------------------------------------------------------------
+template <class T>
+__device__ __forceinline__ T warp_inclusive_scan(T v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    T u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+template <class T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Exclusive scan over the block; returns this thread's exclusive prefix and
+// the block total in *total.  `smem` holds NW values.  All threads call it.
+template <class T, int NW>
+__device__ __forceinline__ T block_exclusive_scan(T v, T* smem, T* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  T inc = warp_inclusive_scan(v);
+  if (lane == 31) smem[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    T s = lane < NW ? smem[lane] : T(0);
+    T si = warp_inclusive_scan(s);
+    if (lane < NW) smem[lane] = si - s;  // exclusive warp offsets
+    if (lane == NW - 1) smem[NW] = si;
+  }
+  __syncthreads();
+  T r = smem[w] + inc - v;
+  *total = smem[NW];
+  __syncthreads();
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// decoupled look-back (single-pass ordered scan across blocks)
+// Status word: bits 62..63 flag (1 aggregate, 2 inclusive), bits 0..61 value.
+// Block ids must be handed out in launch order (atomic ticket) so that a
+// block only ever waits on blocks that have already started.
+// ---------------------------------------------------------------------------
+constexpr unsigned long long kFlagAgg = 1ull << 62;
+constexpr unsigned long long kFlagInc = 2ull << 62;
+constexpr unsigned long long kValMask = (1ull << 62) - 1;
+
+// Called by one full warp.  Publishes `agg` for block `b` and returns the
+// exclusive prefix (sum of the aggregates of blocks 0..b-1) to every lane.
+__device__ __forceinline__ int64_t lookback_warp(unsigned long long* status, int64_t b,
+                                                 int64_t agg, int32_t* dev_status) {
+  const int lane = threadIdx.x & 31;
+  if (b == 0) {
+    if (lane == 0) st_relaxed(&status[0], kFlagInc | (unsigned long long)agg);
+    return 0;
+  }
+  if (lane == 0) st_relaxed(&status[b], kFlagAgg | (unsigned long long)agg);
+  int64_t excl = 0;
+  int64_t end = b - 1;  // window covers end, end-1, ..., end-31
+  int spins = 0;
+  while (true) {
+    int64_t j = end - lane;
+    unsigned long long w = j >= 0 ? ld_relaxed(&status[j]) : (kFlagInc);
+    unsigned flag = (unsigned)(w >> 62);
+    // lanes up to (and including) the first inclusive one must be ready
+    unsigned inc_mask = __ballot_sync(0xffffffffu, flag == 2);
+    unsigned ready_mask = __ballot_sync(0xffffffffu, flag != 0);
+    unsigned need = inc_mask ? ((inc_mask & (0u - inc_mask)) << 1) - 1 : 0xffffffffu;
+    if ((ready_mask & need) != need) {
+      if (++spins > kSpinCap) {
+        if (lane == 0) dev_flag(dev_status, GS_DEV_TIMEOUT);
+        break;
+      }
+      __nanosleep(64);
+      continue;
+    }
+    int64_t v = (need >> lane) & 1u ? (int64_t)(w & kValMask) : 0;
+    excl += warp_sum(v);
+    if (inc_mask) break;
+    end -= 32;
+  }
+  if (lane == 0) st_relaxed(&status[b], kFlagInc | (unsigned long long)(excl + agg));
+  return excl;
+}
+
+}  // namespace gs

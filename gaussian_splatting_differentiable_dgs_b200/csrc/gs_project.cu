@@ -1,0 +1,350 @@
+// gs_project: cull + EWA projection of the candidate Gaussians, ordered
+// compaction of the candidates, per-tile intersection counts and their
+// summed-area table.
+//
+// BoundedGS project page, section 02 (C -> D -> E): only Gaussians that can
+// touch the view get projected state ("candidate-index projection").
+// SkipGS paper notes, "loss function / training strategy": the rasteriser
+// projects each Gaussian to a 2D covariance; its colour comes from SH.
+//
+// One thread per Gaussian.  The arithmetic is fp64: the pass reads ~236
+// bytes per candidate from HBM and does a few hundred flops, so fp64 costs
+// nothing here, and it makes every integer decision (cull, tile rect, depth
+// key) independent of fp32 rounding.  The camera-space position, screen
+// position and cull tests use explicitly rounded operations in a fixed order.
+#include <math.h>
+
+#include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kProjThreads = 256;
+
+struct ProjCam {
+  double R[9], t[3];
+  double fx, fy, cx, cy, limx, limy;
+  double campos[3];
+  int32_t W, H, TW, TH;
+};
+
+// Real SH basis, degree <= 3: Y_0 = 1/(2 sqrt(pi)), band l = 1 ordered
+// (m = -1, 0, 1) as (-y, z, -x) sqrt(3/(4 pi)), bands 2 and 3 the homogeneous
+// polynomials with their closed-form normalisations (Condon-Shortley phase).
+__device__ __forceinline__ void sh_basis(double x, double y, double z, int D, double* Y) {
+  const double kPi = 3.141592653589793;
+  Y[0] = 0.5 / sqrt(kPi);
+  if (D < 1) return;
+  const double k1 = sqrt(3.0 / (4.0 * kPi));
+  Y[1] = -k1 * y;
+  Y[2] = k1 * z;
+  Y[3] = -k1 * x;
+  if (D < 2) return;
+  const double xx = x * x, yy = y * y, zz = z * z;
+  const double k2a = 0.5 * sqrt(15.0 / kPi), k2b = 0.25 * sqrt(5.0 / kPi),
+               k2c = 0.25 * sqrt(15.0 / kPi);
+  Y[4] = k2a * x * y;
+  Y[5] = -k2a * y * z;
+  Y[6] = k2b * (2.0 * zz - xx - yy);
+  Y[7] = -k2a * x * z;
+  Y[8] = k2c * (xx - yy);
+  if (D < 3) return;
+  const double k3a = 0.25 * sqrt(35.0 / (2.0 * kPi)), k3b = 0.5 * sqrt(105.0 / kPi),
+               k3c = 0.25 * sqrt(21.0 / (2.0 * kPi)), k3d = 0.25 * sqrt(7.0 / kPi),
+               k3e = 0.25 * sqrt(105.0 / kPi);
+  Y[9] = -k3a * y * (3.0 * xx - yy);
+  Y[10] = k3b * x * y * z;
+  Y[11] = -k3c * y * (4.0 * zz - xx - yy);
+  Y[12] = k3d * z * (2.0 * zz - 3.0 * xx - 3.0 * yy);
+  Y[13] = -k3c * x * (4.0 * zz - xx - yy);
+  Y[14] = k3e * z * (xx - yy);
+  Y[15] = -k3a * x * (xx - 3.0 * yy);
+}
+
+struct ProjOut {
+  float4 r0, r1, r2;
+  short4 rect;
+  uint32_t key;
+};
+
+// Returns true if Gaussian i is a candidate and fills `o`.
+__device__ __forceinline__ bool project_gaussian(const float* __restrict__ P, int64_t n_pad,
+                                                 int64_t i, int D, const ProjCam& c,
+                                                 ProjOut& o, bool& nonfinite) {
+  const double x = P[i], y = P[n_pad + i], z = P[2 * n_pad + i];
+  double tc[3];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+    tc[r] = __dadd_rn(__dadd_rn(__dadd_rn(__dmul_rn(c.R[3 * r], x), __dmul_rn(c.R[3 * r + 1], y)),
+                                __dmul_rn(c.R[3 * r + 2], z)),
+                      c.t[r]);
+  float pv[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) pv[k] = P[(3 + k) * n_pad + i];
+  bool fin = isfinite(x) && isfinite(y) && isfinite(z);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) fin = fin && isfinite(pv[k]);
+  if (!fin) {
+    nonfinite = true;
+    return false;
+  }
+  const double tz = tc[2];
+  if (!(tz > 0.2)) return false;
+  const double xn = __ddiv_rn(tc[0], tz), yn = __ddiv_rn(tc[1], tz);
+  if (fabs(xn) > c.limx || fabs(yn) > c.limy) return false;
+  const double u = __dadd_rn(__dmul_rn(c.fx, xn), c.cx);
+  const double v = __dadd_rn(__dmul_rn(c.fy, yn), c.cy);
+
+  // 3D covariance from the normalised quaternion and the scales
+  double qw = pv[3], qx = pv[4], qy = pv[5], qz = pv[6];
+  const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+  if (!(qn > 0.0)) {
+    nonfinite = true;
+    return false;
+  }
+  qw /= qn; qx /= qn; qy /= qn; qz /= qn;
+  double Rg[9];
+  Rg[0] = 1.0 - 2.0 * (qy * qy + qz * qz); Rg[1] = 2.0 * (qx * qy - qw * qz); Rg[2] = 2.0 * (qx * qz + qw * qy);
+  Rg[3] = 2.0 * (qx * qy + qw * qz); Rg[4] = 1.0 - 2.0 * (qx * qx + qz * qz); Rg[5] = 2.0 * (qy * qz - qw * qx);
+  Rg[6] = 2.0 * (qx * qz - qw * qy); Rg[7] = 2.0 * (qy * qz + qw * qx); Rg[8] = 1.0 - 2.0 * (qx * qx + qy * qy);
+  const double s0 = exp((double)pv[0]), s1 = exp((double)pv[1]), s2 = exp((double)pv[2]);
+  double M[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    M[3 * r] = Rg[3 * r] * s0;
+    M[3 * r + 1] = Rg[3 * r + 1] * s1;
+    M[3 * r + 2] = Rg[3 * r + 2] * s2;
+  }
+  double Sg[6];  // symmetric 3x3: 00 01 02 11 12 22
+  Sg[0] = M[0] * M[0] + M[1] * M[1] + M[2] * M[2];
+  Sg[1] = M[0] * M[3] + M[1] * M[4] + M[2] * M[5];
+  Sg[2] = M[0] * M[6] + M[1] * M[7] + M[2] * M[8];
+  Sg[3] = M[3] * M[3] + M[4] * M[4] + M[5] * M[5];
+  Sg[4] = M[3] * M[6] + M[4] * M[7] + M[5] * M[8];
+  Sg[5] = M[6] * M[6] + M[7] * M[7] + M[8] * M[8];
+  // T = J W, J the perspective Jacobian at t
+  const double j00 = c.fx / tz, j02 = -c.fx * xn / tz;
+  const double j11 = c.fy / tz, j12 = -c.fy * yn / tz;
+  double T0[3], T1[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    T0[k] = j00 * c.R[k] + j02 * c.R[6 + k];
+    T1[k] = j11 * c.R[3 + k] + j12 * c.R[6 + k];
+  }
+  // A = T Sigma (2x3), then Sigma2 = A T^T
+  double A0[3], A1[3];
+  A0[0] = T0[0] * Sg[0] + T0[1] * Sg[1] + T0[2] * Sg[2];
+  A0[1] = T0[0] * Sg[1] + T0[1] * Sg[3] + T0[2] * Sg[4];
+  A0[2] = T0[0] * Sg[2] + T0[1] * Sg[4] + T0[2] * Sg[5];
+  A1[0] = T1[0] * Sg[0] + T1[1] * Sg[1] + T1[2] * Sg[2];
+  A1[1] = T1[0] * Sg[1] + T1[1] * Sg[3] + T1[2] * Sg[4];
+  A1[2] = T1[0] * Sg[2] + T1[1] * Sg[4] + T1[2] * Sg[5];
+  const double c00 = A0[0] * T0[0] + A0[1] * T0[1] + A0[2] * T0[2] + 0.3;
+  const double c01 = 0.5 * ((A0[0] * T1[0] + A0[1] * T1[1] + A0[2] * T1[2]) +
+                            (A1[0] * T0[0] + A1[1] * T0[1] + A1[2] * T0[2]));
+  const double c11 = A1[0] * T1[0] + A1[1] * T1[1] + A1[2] * T1[2] + 0.3;
+  const double det = c00 * c11 - c01 * c01;
+  if (!(det > 0.0)) return false;
+  const double mid = 0.5 * (c00 + c11);
+  const double lam = mid + sqrt(fmax(0.1, mid * mid - det));
+  const double rad = ceil(3.0 * sqrt(lam));
+  const int64_t rx0 = (int64_t)floor((u - rad) / kTile), rx1 = (int64_t)floor((u + rad) / kTile) + 1;
+  const int64_t ry0 = (int64_t)floor((v - rad) / kTile), ry1 = (int64_t)floor((v + rad) / kTile) + 1;
+  const int64_t x0 = rx0 < 0 ? 0 : (rx0 > c.TW ? c.TW : rx0);
+  const int64_t x1 = rx1 < 0 ? 0 : (rx1 > c.TW ? c.TW : rx1);
+  const int64_t y0 = ry0 < 0 ? 0 : (ry0 > c.TH ? c.TH : ry0);
+  const int64_t y1 = ry1 < 0 ? 0 : (ry1 > c.TH ? c.TH : ry1);
+  if (x0 >= x1 || y0 >= y1) return false;
+
+  // colour from SH at the direction camera centre -> mean
+  double dx = x - c.campos[0], dy = y - c.campos[1], dz = z - c.campos[2];
+  const double dn = sqrt(dx * dx + dy * dy + dz * dz);
+  dx /= dn; dy /= dn; dz /= dn;
+  double Y[16];
+  sh_basis(dx, dy, dz, D, Y);
+  const int ksh = (D + 1) * (D + 1);
+  double rgb[3] = {0.5, 0.5, 0.5};
+  for (int k = 0; k < ksh; ++k) {
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) {
+      float s = P[(11 + 3 * k + ch) * n_pad + i];
+      rgb[ch] += (double)s * Y[k];
+    }
+  }
+  const double opac = 1.0 / (1.0 + exp(-(double)pv[7]));
+
+  const float uh = (float)u, vh = (float)v;
+  o.r0 = make_float4(uh, vh, (float)(u - (double)uh), (float)(v - (double)vh));
+  const double a = c11 / det, b = -c01 / det;
+  o.r1 = make_float4((float)(0.5 * a), (float)(b / a), (float)(0.5 / c11), (float)opac);
+  const float depth = (float)tz;
+  o.r2 = make_float4((float)fmax(rgb[0], 0.0), (float)fmax(rgb[1], 0.0), (float)fmax(rgb[2], 0.0), depth);
+  o.rect = make_short4((short)x0, (short)y0, (short)x1, (short)y1);
+  o.key = __float_as_uint(depth);
+  return true;
+}
+
+__global__ void __launch_bounds__(kProjThreads)
+k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, int D, ProjCam cam,
+          int32_t* __restrict__ cand_idx, int32_t* __restrict__ slot_map, float4* __restrict__ rec,
+          short4* __restrict__ rect, uint32_t* __restrict__ depth_key, int32_t* __restrict__ diff,
+          unsigned long long* __restrict__ lb, unsigned int* __restrict__ ticket,
+          int32_t* __restrict__ n_cand, int64_t n_blocks, int64_t capacity, int32_t* dev_status) {
+  __shared__ unsigned int s_b;
+  __shared__ int s_scan[kProjThreads / 32 + 1];
+  __shared__ long long s_prefix;
+  if (threadIdx.x == 0) s_b = atomicAdd(ticket, 1u);
+  __syncthreads();
+  const int64_t b = s_b;
+  const int64_t i = b * kProjThreads + threadIdx.x;
+  ProjOut o;
+  bool nonfinite = false;
+  const bool cand = i < n && project_gaussian(params, n_pad, i, D, cam, o, nonfinite);
+  if (nonfinite) dev_flag(dev_status, GS_DEV_NONFINITE);
+  int total;
+  const int rank = block_exclusive_scan<int, kProjThreads / 32>(cand ? 1 : 0, s_scan, &total);
+  if (threadIdx.x < 32) {
+    int64_t ex = lookback_warp(lb, b, total, dev_status);
+    if (threadIdx.x == 0) s_prefix = ex;
+  }
+  __syncthreads();
+  const int64_t slot = s_prefix + rank;
+  const bool fits = slot < capacity;  // false only after a timed-out look-back
+  if (cand && !fits) dev_flag(dev_status, GS_DEV_BOUNDS);
+  if (i < n) slot_map[i] = (cand && fits) ? (int32_t)slot : -1;
+  if (cand && fits) {
+    cand_idx[slot] = (int32_t)i;
+    rec[3 * slot] = o.r0;
+    rec[3 * slot + 1] = o.r1;
+    rec[3 * slot + 2] = o.r2;
+    rect[slot] = o.rect;
+    depth_key[slot] = o.key;
+    const int64_t s = cam.TW + 1;
+    atomicAdd(&diff[o.rect.y * s + o.rect.x], 1);
+    atomicAdd(&diff[o.rect.y * s + o.rect.z], -1);
+    atomicAdd(&diff[o.rect.w * s + o.rect.x], -1);
+    atomicAdd(&diff[o.rect.w * s + o.rect.z], 1);
+  }
+  if (b == n_blocks - 1 && threadIdx.x == 0) *n_cand = (int32_t)(s_prefix + total);
+}
+
+// Double inclusive prefix along x of each row (y < TH, x < TW).
+__global__ void __launch_bounds__(256)
+k_sat_rows(const int32_t* __restrict__ diff, int64_t* __restrict__ tmp, int TW, int TH) {
+  __shared__ long long s_scan[9];
+  const int y = blockIdx.x;
+  long long c1 = 0, c2 = 0;
+  for (int x0 = 0; x0 < TW; x0 += 256) {
+    const int x = x0 + threadIdx.x;
+    long long v = x < TW ? (long long)diff[(int64_t)y * (TW + 1) + x] : 0;
+    long long t;
+    long long e1 = block_exclusive_scan<long long, 8>(v, s_scan, &t);
+    long long s1 = c1 + e1 + v;
+    c1 += t;
+    long long e2 = block_exclusive_scan<long long, 8>(s1, s_scan, &t);
+    long long s2 = c2 + e2 + s1;
+    c2 += t;
+    if (x < TW) tmp[(int64_t)y * TW + x] = s2;
+  }
+}
+
+// Double inclusive prefix along y of each column, written with a one-cell
+// zero border: sat[(y + 1) (TW + 1) + x + 1].
+__global__ void __launch_bounds__(256)
+k_sat_cols(const int64_t* __restrict__ tmp, int64_t* __restrict__ sat, int TW, int TH) {
+  const int x = blockIdx.x * blockDim.x + threadIdx.x;
+  if (x > TW) return;
+  const int64_t s = TW + 1;
+  if (x == TW) {  // the zero column
+    for (int y = 0; y <= TH; ++y) sat[(int64_t)y * s] = 0;
+    return;
+  }
+  sat[x + 1] = 0;
+  long long c1 = 0, c2 = 0;
+  for (int y = 0; y < TH; ++y) {
+    c1 += tmp[(int64_t)y * TW + x];
+    c2 += c1;
+    sat[(int64_t)(y + 1) * s + x + 1] = c2;
+  }
+}
+
+struct ProjWs {
+  int32_t* diff;
+  int64_t* tmp;
+  unsigned long long* lb;
+  unsigned int* ticket;
+  size_t bytes;
+};
+
+ProjWs carve_proj(void* ws, size_t cap, int64_t n, int32_t W, int32_t H) {
+  Carver cv(ws, cap);
+  const int64_t TW = tiles_x(W), TH = tiles_y(H);
+  const int64_t nb = (n + kProjThreads - 1) / kProjThreads;
+  ProjWs p;
+  p.ticket = cv.take<unsigned int>(64);
+  p.lb = cv.take<unsigned long long>(nb > 0 ? nb : 1);
+  p.diff = cv.take<int32_t>((TW + 1) * (TH + 1));
+  p.tmp = cv.take<int64_t>(TW * TH);
+  p.bytes = cv.off;
+  return p;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" size_t gs_project_workspace_size(int64_t n, int32_t width, int32_t height) {
+  if (n < 0 || width <= 0 || height <= 0) return 0;
+  return carve_proj(nullptr, 0, n, width, height).bytes;
+}
+
+extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uint32_t flags,
+                                const gs_proj* out, int64_t* tile_sat, void* ws, size_t ws_bytes,
+                                int32_t* dev_status, gs_stream stream) {
+  if (!model || !cam || !out || !tile_sat) return GS_ERR_ARG;
+  if (flags != 0) return GS_ERR_UNSUPPORTED;
+  if (model->n < 0 || model->n_pad < model->n || (model->n_pad & 3) || model->sh_degree < 0 ||
+      model->sh_degree > 3)
+    return GS_ERR_ARG;
+  if (cam->width <= 0 || cam->height <= 0 || !(cam->fx > 0) || !(cam->fy > 0)) return GS_ERR_ARG;
+  const int64_t TW = tiles_x(cam->width), TH = tiles_y(cam->height);
+  if (TW > 32767 || TH > 32767) return GS_ERR_UNSUPPORTED;
+  if (out->capacity < model->n || !out->n_cand) return GS_ERR_ARG;
+  if (model->n > 0 && (!model->params || !out->cand_idx || !out->slot || !out->rec || !out->rect ||
+                       !out->depth_key))
+    return GS_ERR_ARG;
+  if (!aligned(out->rec, 16) || !aligned(out->rect, 8) || !aligned(ws, 256)) return GS_ERR_ARG;
+  ProjWs w = carve_proj(ws, ws_bytes, model->n, cam->width, cam->height);
+  if (w.bytes > ws_bytes || !ws) return GS_ERR_CAPACITY;
+  cudaStream_t s = to_stream(stream);
+
+  ProjCam pc;
+  for (int k = 0; k < 9; ++k) pc.R[k] = (double)cam->R[k];
+  for (int k = 0; k < 3; ++k) pc.t[k] = (double)cam->t[k];
+  pc.fx = cam->fx; pc.fy = cam->fy; pc.cx = cam->cx; pc.cy = cam->cy;
+  pc.limx = (1.3 * (0.5 * (double)cam->width)) / pc.fx;
+  pc.limy = (1.3 * (0.5 * (double)cam->height)) / pc.fy;
+  for (int c = 0; c < 3; ++c)
+    pc.campos[c] = -(pc.R[c] * pc.t[0] + pc.R[3 + c] * pc.t[1] + pc.R[6 + c] * pc.t[2]);
+  pc.W = cam->width; pc.H = cam->height; pc.TW = (int32_t)TW; pc.TH = (int32_t)TH;
+
+  const int64_t nb = (model->n + kProjThreads - 1) / kProjThreads;
+  // ticket, look-back words and the difference grid start at zero
+  const size_t zero_bytes = (size_t)((char*)(w.diff + (TW + 1) * (TH + 1)) - (char*)ws);
+  GS_TRY(cudaMemsetAsync(ws, 0, zero_bytes, s));
+  if (nb > 0) {
+    k_project<<<(unsigned)nb, kProjThreads, 0, s>>>(
+        model->params, model->n, model->n_pad, model->sh_degree, pc, out->cand_idx, out->slot,
+        reinterpret_cast<float4*>(out->rec), reinterpret_cast<short4*>(out->rect), out->depth_key,
+        w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, dev_status);
+    GS_LAUNCH_CHECK();
+  } else {
+    GS_TRY(cudaMemsetAsync(out->n_cand, 0, sizeof(int32_t), s));
+  }
+  k_sat_rows<<<(unsigned)TH, 256, 0, s>>>(w.diff, w.tmp, (int)TW, (int)TH);
+  GS_LAUNCH_CHECK();
+  k_sat_cols<<<(unsigned)((TW + 1 + 255) / 256), 256, 0, s>>>(w.tmp, tile_sat, (int)TW, (int)TH);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}

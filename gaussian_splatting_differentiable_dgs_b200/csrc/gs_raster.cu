@@ -1,0 +1,545 @@
+// Tile rasteriser: front-to-back compositing (+ fused L1 loss) and the
+// reverse blend with per-tile reduction of the per-Gaussian gradients.
+//
+// SkipGS paper notes, "loss function / training strategy": the image is the
+// transmittance-weighted blend of the sorted Gaussians and the gradients
+// flow back through the transmittance accumulation; "key design 2": the
+// backward accumulates per-Gaussian gradients atomically.  BoundedGS project
+// page, section 01: a Leaf's gradient contribution is merged into the view's
+// gradient before its buffers are released (here: atomics into the compact
+// per-candidate g2d that lives for the whole view).
+//
+// One CTA per 16x16 tile of the Leaf; each thread owns PPT pixels of one
+// column.  The tile's list is staged through shared memory in batches of
+// one record per thread; within a batch every thread reads each record by
+// broadcast.  fp32 arithmetic with explicitly rounded operations in the
+// alpha path, so the backward retakes exactly the forward's skip decisions.
+#include <algorithm>
+
+#include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kAlphaMin = 1.0f / 255.0f;
+constexpr float kAlphaMax = 0.99f;
+constexpr float kTMin = 1e-4f;
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Staged record: position relative to the tile origin and the exponent
+// coefficients pre-scaled by -log2(e).
+struct Staged {
+  float gx, gy, beta, ns1;   // float4
+  float ns2, opac, r, g;     // float4
+  float b, s1, s2;           // natural-log coefficients (backward)
+  int32_t slot;
+};
+
+__device__ __forceinline__ Staged stage_record(const float4* __restrict__ rec, int32_t slot,
+                                               int tx, int ty) {
+  const float4 r0 = rec[3 * (int64_t)slot];
+  const float4 r1 = rec[3 * (int64_t)slot + 1];
+  const float4 r2 = rec[3 * (int64_t)slot + 2];
+  Staged s;
+  s.gx = __fadd_rn(__fsub_rn(r0.x, (float)(tx * kTile)), r0.z);
+  s.gy = __fadd_rn(__fsub_rn(r0.y, (float)(ty * kTile)), r0.w);
+  s.beta = r1.y;
+  s.ns1 = __fmul_rn(r1.x, -kLog2e);
+  s.ns2 = __fmul_rn(r1.z, -kLog2e);
+  s.opac = r1.w;
+  s.r = r2.x;
+  s.g = r2.y;
+  s.b = r2.z;
+  s.s1 = r1.x;
+  s.s2 = r1.z;
+  s.slot = slot;
+  return s;
+}
+
+struct Eval {
+  float dx, dy, t1, G, araw, alpha;
+};
+
+// alpha = min(0.99, o 2^(-q log2 e)),  q = s1 (dx + beta dy)^2 + s2 dy^2
+__device__ __forceinline__ Eval eval_alpha(float gx, float gy, float beta, float ns1, float ns2,
+                                           float opac, float px, float py) {
+  Eval e;
+  e.dx = __fsub_rn(gx, px);
+  e.dy = __fsub_rn(gy, py);
+  e.t1 = __fmaf_rn(beta, e.dy, e.dx);
+  const float qa = __fmul_rn(ns1, e.t1);
+  const float qb = __fmul_rn(ns2, e.dy);
+  const float ql = __fmaf_rn(qa, e.t1, __fmul_rn(qb, e.dy));
+  e.G = ex2_approx(ql);
+  e.araw = __fmul_rn(opac, e.G);
+  e.alpha = fminf(e.araw, kAlphaMax);
+  return e;
+}
+
+struct PixArgs {
+  int32_t x0, y0, w, h;
+  int64_t pitch, plane;
+  float* img;
+  float* T_final;
+  int32_t* last;
+  float* dL;
+  const float* target;
+  int32_t tx0, ty0;
+  int64_t tpitch, tplane;
+  float* loss_tiles;
+  float norm;
+};
+
+template <int PPT>
+struct TileGeom {
+  static constexpr int NT = 256 / PPT;
+  static constexpr int ROWS = 16 / PPT;
+};
+
+// ---------------------------------------------------------------------------
+// forward
+// ---------------------------------------------------------------------------
+template <int PPT>
+__global__ void __launch_bounds__(256 / PPT)
+k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
+             const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
+             int32_t* dev_status) {
+  constexpr int NT = TileGeom<PPT>::NT, ROWS = TileGeom<PPT>::ROWS;
+  __shared__ float4 sA[NT], sB[NT];
+  __shared__ float sC[NT];
+  __shared__ float s_red[NT / 32];
+  const int lw = leaf.x1 - leaf.x0;
+  const int ltile = blockIdx.x;
+  const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
+  const int64_t begin = ranges[2 * ltile], end = ranges[2 * ltile + 1];
+  const int t = threadIdx.x;
+  const int lx = t & 15, ly0 = t >> 4;
+  const float fpx = (float)lx + 0.5f;
+  float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
+  int lastp[PPT];
+  bool done[PPT], inside[PPT];
+#pragma unroll
+  for (int k = 0; k < PPT; ++k) {
+    const int ly = ly0 + k * ROWS;
+    fpy[k] = (float)ly + 0.5f;
+    inside[k] = (tx * kTile + lx < W) && (ty * kTile + ly < H);
+    done[k] = !inside[k];
+    T[k] = 1.0f;
+    Cr[k] = Cg[k] = Cb[k] = 0.0f;
+    lastp[k] = 0;
+  }
+  for (int64_t base = begin; base < end; base += NT) {
+    bool mine_done = true;
+#pragma unroll
+    for (int k = 0; k < PPT; ++k) mine_done = mine_done && done[k];
+    if (__syncthreads_count(mine_done) == NT) break;
+    const int64_t e = base + t;
+    if (e < end) {
+      const Staged s = stage_record(rec, vals[e], tx, ty);
+      sA[t] = make_float4(s.gx, s.gy, s.beta, s.ns1);
+      sB[t] = make_float4(s.ns2, s.opac, s.r, s.g);
+      sC[t] = s.b;
+    }
+    __syncthreads();
+    const int cnt = (int)min((int64_t)NT, end - base);
+    const int pos0 = (int)(base - begin);
+    for (int j = 0; j < cnt; ++j) {
+      const float4 A = sA[j];
+      const float4 B = sB[j];
+      const float Bb = sC[j];
+#pragma unroll
+      for (int k = 0; k < PPT; ++k) {
+        if (done[k]) continue;
+        const Eval ev = eval_alpha(A.x, A.y, A.z, A.w, B.x, B.y, fpx, fpy[k]);
+        if (ev.alpha < kAlphaMin) continue;
+        const float Tn = __fmul_rn(T[k], __fsub_rn(1.0f, ev.alpha));
+        if (Tn < kTMin) {
+          done[k] = true;
+          continue;
+        }
+        const float wgt = ev.alpha * T[k];
+        Cr[k] = fmaf(B.z, wgt, Cr[k]);
+        Cg[k] = fmaf(B.w, wgt, Cg[k]);
+        Cb[k] = fmaf(Bb, wgt, Cb[k]);
+        T[k] = Tn;
+        lastp[k] = pos0 + j + 1;
+      }
+    }
+  }
+  // epilogue: outputs and the fused L1 terms
+  float lsum = 0.0f;
+#pragma unroll
+  for (int k = 0; k < PPT; ++k) {
+    if (!inside[k]) continue;
+    const int x = tx * kTile + lx, y = ty * kTile + ly0 + k * ROWS;
+    const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
+    if (px.img) {
+      px.img[o] = Cr[k];
+      px.img[o + px.plane] = Cg[k];
+      px.img[o + 2 * px.plane] = Cb[k];
+    }
+    px.T_final[o] = T[k];
+    px.last[o] = lastp[k];
+    if (px.target) {
+      const float c[3] = {Cr[k], Cg[k], Cb[k]};
+      const int64_t ot = (int64_t)(y - px.ty0) * px.tpitch + (x - px.tx0);
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) {
+        const float d = c[ch] - px.target[ot + ch * px.tplane];
+        px.dL[o + ch * px.plane] = d > 0.0f ? px.norm : (d < 0.0f ? -px.norm : 0.0f);
+        lsum += fabsf(d);
+      }
+    }
+  }
+  if (px.target && px.loss_tiles) {
+    lsum = warp_sum(lsum);
+    if ((t & 31) == 0) s_red[t >> 5] = lsum;
+    __syncthreads();
+    if (t == 0) {
+      float tot = 0.0f;
+      for (int w = 0; w < NT / 32; ++w) tot += s_red[w];
+      px.loss_tiles[(int64_t)ty * TW + tx] = tot * px.norm;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// standalone L1 over a Leaf
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_loss_l1(gs_rect leaf, int W, int H, int TW, PixArgs px) {
+  __shared__ float s_red[8];
+  const int lw = leaf.x1 - leaf.x0;
+  const int tx = leaf.x0 + blockIdx.x % lw, ty = leaf.y0 + blockIdx.x / lw;
+  const int t = threadIdx.x;
+  const int x = tx * kTile + (t & 15), y = ty * kTile + (t >> 4);
+  float lsum = 0.0f;
+  if (x < W && y < H) {
+    const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
+    const int64_t ot = (int64_t)(y - px.ty0) * px.tpitch + (x - px.tx0);
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) {
+      const float d = px.img[o + ch * px.plane] - px.target[ot + ch * px.tplane];
+      px.dL[o + ch * px.plane] = d > 0.0f ? px.norm : (d < 0.0f ? -px.norm : 0.0f);
+      lsum += fabsf(d);
+    }
+  }
+  lsum = warp_sum(lsum);
+  if ((t & 31) == 0) s_red[t >> 5] = lsum;
+  __syncthreads();
+  if (t == 0 && px.loss_tiles) {
+    float tot = 0.0f;
+    for (int w = 0; w < 8; ++w) tot += s_red[w];
+    px.loss_tiles[(int64_t)ty * TW + tx] = tot * px.norm;
+  }
+}
+
+__global__ void __launch_bounds__(1024)
+k_loss_total(const float* __restrict__ tiles, int64_t n, double* __restrict__ out) {
+  __shared__ double s[32];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += 1024) acc += (double)tiles[i];
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) s[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < 32; ++w) tot += s[w];
+    *out = tot;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// backward
+// ---------------------------------------------------------------------------
+
+// Sum of 9 values over the warp, scattered: afterwards lane L with L even
+// and idx = (L >> 1) & 15 < 9 holds the warp total of value idx.  16
+// shuffles instead of 45 for nine independent butterflies.
+__device__ __forceinline__ float warp_reduce_scatter9(const float (&v)[9], int lane) {
+  float a[8];
+  {
+    const bool up = lane & 16;
+    // level 1: keep values 0..7 (low half) or 8..15 (high half; only 8 real)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float mine_keep = up ? (i == 0 ? v[8] : 0.0f) : v[i];
+      const float send = up ? v[i] : (i == 0 ? v[8] : 0.0f);
+      a[i] = mine_keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+  }
+  float b[4];
+  {
+    const bool up = lane & 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float keep = up ? a[4 + i] : a[i];
+      const float send = up ? a[i] : a[4 + i];
+      b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+  }
+  float c[2];
+  {
+    const bool up = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float keep = up ? b[2 + i] : b[i];
+      const float send = up ? b[i] : b[2 + i];
+      c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+  }
+  float d;
+  {
+    const bool up = lane & 2;
+    const float keep = up ? c[1] : c[0];
+    const float send = up ? c[0] : c[1];
+    d = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  d += __shfl_xor_sync(0xffffffffu, d, 1);
+  return d;
+}
+
+template <int PPT>
+__global__ void __launch_bounds__(256 / PPT)
+k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
+             const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, PixArgs px,
+             float* __restrict__ g2d, int32_t* dev_status) {
+  constexpr int NT = TileGeom<PPT>::NT, ROWS = TileGeom<PPT>::ROWS;
+  __shared__ float4 sA[NT], sB[NT];
+  __shared__ float4 sC[NT];       // {b, s1, s2, slot bits}
+  __shared__ float sg[NT][12];
+  __shared__ int s_touched[NT];
+  __shared__ int s_maxlast;
+  const int lw = leaf.x1 - leaf.x0;
+  const int ltile = blockIdx.x;
+  const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
+  const int64_t begin = ranges[2 * ltile];
+  const int t = threadIdx.x, lane = t & 31;
+  const int lx = t & 15, ly0 = t >> 4;
+  const float fpx = (float)lx + 0.5f;
+  float fpy[PPT], T[PPT], Ar[PPT], Ag[PPT], Ab[PPT], gr[PPT], gg[PPT], gb[PPT];
+  int lastp[PPT];
+  if (t == 0) s_maxlast = 0;
+  for (int e = t; e < NT * 12; e += NT) (&sg[0][0])[e] = 0.0f;
+  s_touched[t] = 0;
+  __syncthreads();
+  int mylast = 0;
+#pragma unroll
+  for (int k = 0; k < PPT; ++k) {
+    const int ly = ly0 + k * ROWS;
+    fpy[k] = (float)ly + 0.5f;
+    const int x = tx * kTile + lx, y = ty * kTile + ly;
+    Ar[k] = Ag[k] = Ab[k] = 0.0f;
+    if (x < W && y < H) {
+      const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
+      T[k] = px.T_final[o];
+      lastp[k] = px.last[o];
+      gr[k] = px.dL[o];
+      gg[k] = px.dL[o + px.plane];
+      gb[k] = px.dL[o + 2 * px.plane];
+    } else {
+      T[k] = 1.0f;
+      lastp[k] = 0;
+      gr[k] = gg[k] = gb[k] = 0.0f;
+    }
+    mylast = max(mylast, lastp[k]);
+  }
+  atomicMax(&s_maxlast, mylast);
+  __syncthreads();
+  const int tile_last = s_maxlast;
+
+  for (int bend = tile_last; bend > 0; bend -= NT) {
+    const int bstart = max(0, bend - NT);
+    const int cnt = bend - bstart;
+    if (t < cnt) {
+      const int pos = bend - 1 - t;
+      const Staged s = stage_record(rec, vals[begin + pos], tx, ty);
+      sA[t] = make_float4(s.gx, s.gy, s.beta, s.ns1);
+      sB[t] = make_float4(s.ns2, s.opac, s.r, s.g);
+      sC[t] = make_float4(s.b, s.s1, s.s2, __int_as_float(s.slot));
+    }
+    __syncthreads();
+    for (int j = 0; j < cnt; ++j) {
+      const int pos = bend - 1 - j;
+      const float4 A = sA[j];
+      const float4 B = sB[j];
+      const float4 Cc = sC[j];
+      float acc[9];
+#pragma unroll
+      for (int q = 0; q < 9; ++q) acc[q] = 0.0f;
+      bool any = false;
+#pragma unroll
+      for (int k = 0; k < PPT; ++k) {
+        if (pos >= lastp[k]) continue;
+        const Eval ev = eval_alpha(A.x, A.y, A.z, A.w, B.x, B.y, fpx, fpy[k]);
+        if (ev.alpha < kAlphaMin) continue;
+        any = true;
+        const float inv = __frcp_rn(1.0f - ev.alpha);
+        const float Tb = T[k] * inv;          // transmittance before this entry
+        const float wgt = ev.alpha * Tb;
+        acc[6] = fmaf(wgt, gr[k], acc[6]);
+        acc[7] = fmaf(wgt, gg[k], acc[7]);
+        acc[8] = fmaf(wgt, gb[k], acc[8]);
+        // dL/dalpha = sum_c g_c (rgb_c T_i - A_c / (1 - alpha))
+        float da = gr[k] * (B.z * Tb - Ar[k] * inv);
+        da = fmaf(gg[k], B.w * Tb - Ag[k] * inv, da);
+        da = fmaf(gb[k], Cc.x * Tb - Ab[k] * inv, da);
+        Ar[k] = fmaf(B.z, wgt, Ar[k]);
+        Ag[k] = fmaf(B.w, wgt, Ag[k]);
+        Ab[k] = fmaf(Cc.x, wgt, Ab[k]);
+        T[k] = Tb;
+        if (ev.araw <= kAlphaMax) {
+          const float dq = -ev.alpha * da;         // dL/dq (natural units)
+          acc[5] = fmaf(ev.G, da, acc[5]);          // dL/dopacity
+          const float s1t = 2.0f * Cc.y * ev.t1;    // dq/du = a dx + b dy
+          acc[0] = fmaf(dq, s1t, acc[0]);
+          acc[1] = fmaf(dq, fmaf(s1t, A.z, 2.0f * Cc.z * ev.dy), acc[1]);  // dq/dv
+          const float hdx = 0.5f * ev.dx;
+          acc[2] = fmaf(dq * hdx, ev.dx, acc[2]);
+          acc[3] = fmaf(dq * ev.dx, ev.dy, acc[3]);
+          acc[4] = fmaf(dq * 0.5f * ev.dy, ev.dy, acc[4]);
+        }
+      }
+      if (__any_sync(0xffffffffu, any)) {
+        const float tot = warp_reduce_scatter9(acc, lane);
+        const int idx = (lane >> 1) & 15;
+        if (!(lane & 1) && idx < 9) atomicAdd(&sg[j][idx], tot);
+        if (lane == 0) s_touched[j] = 1;
+      }
+    }
+    __syncthreads();
+    if (t < cnt && s_touched[t]) {
+      const int32_t slot = __float_as_int(sC[t].w);
+      float4* dst = reinterpret_cast<float4*>(g2d + (int64_t)slot * 12);
+      atomicAdd(dst, make_float4(sg[t][0], sg[t][1], sg[t][2], sg[t][3]));
+      atomicAdd(dst + 1, make_float4(sg[t][4], sg[t][5], sg[t][6], sg[t][7]));
+      atomicAdd(dst + 2, make_float4(sg[t][8], 0.0f, 0.0f, 0.0f));
+#pragma unroll
+      for (int q = 0; q < 9; ++q) sg[t][q] = 0.0f;
+      s_touched[t] = 0;
+    }
+    __syncthreads();
+  }
+}
+
+PixArgs to_args(const gs_pixels* p) {
+  PixArgs a;
+  a.x0 = p->x0; a.y0 = p->y0; a.w = p->w; a.h = p->h;
+  a.pitch = p->pitch; a.plane = p->plane;
+  a.img = p->img; a.T_final = p->T_final; a.last = p->last; a.dL = p->dL_dimg;
+  a.target = p->target; a.tx0 = p->tx0; a.ty0 = p->ty0; a.tpitch = p->tpitch;
+  a.tplane = p->tplane; a.loss_tiles = p->loss_tiles;
+  a.norm = (float)p->norm;
+  return a;
+}
+
+// The Leaf's pixels (clipped to the image) must lie inside the buffers.
+bool check_pixels(const gs_pixels* p, gs_rect leaf, const gs_camera* cam) {
+  if (!p) return false;
+  const int64_t X0 = (int64_t)leaf.x0 * kTile, Y0 = (int64_t)leaf.y0 * kTile;
+  const int64_t X1 = std::min<int64_t>((int64_t)leaf.x1 * kTile, cam->width);
+  const int64_t Y1 = std::min<int64_t>((int64_t)leaf.y1 * kTile, cam->height);
+  if (X0 < p->x0 || Y0 < p->y0 || X1 > (int64_t)p->x0 + p->w || Y1 > (int64_t)p->y0 + p->h)
+    return false;
+  if (p->pitch < p->w || p->plane < p->pitch * (int64_t)p->h) return false;
+  if (p->target) {
+    if (X0 < p->tx0 || Y0 < p->ty0 || p->tpitch < X1 - p->tx0) return false;
+    if (p->tplane < p->tpitch * (Y1 - p->ty0)) return false;
+  }
+  return true;
+}
+
+bool check_leaf(gs_rect leaf, const gs_camera* cam) {
+  const int64_t TW = tiles_x(cam->width), TH = tiles_y(cam->height);
+  return leaf.x0 >= 0 && leaf.y0 >= 0 && leaf.x1 > leaf.x0 && leaf.y1 > leaf.y0 &&
+         leaf.x1 <= TW && leaf.y1 <= TH;
+}
+
+int pick_ppt(uint32_t flags, int dflt) {
+  const int p = (int)(flags & 7u);
+  return (p == 1 || p == 2 || p == 4) ? p : dflt;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals, const int64_t* ranges,
+                                   gs_rect leaf, const gs_camera* cam, const gs_pixels* px,
+                                   uint32_t flags, int32_t* dev_status, gs_stream stream) {
+  if (!proj || !ranges || !cam || !check_leaf(leaf, cam) || !check_pixels(px, leaf, cam))
+    return GS_ERR_ARG;
+  if (!px->T_final || !px->last || (px->target && !px->dL_dimg)) return GS_ERR_ARG;
+  if (!aligned(proj->rec, 16)) return GS_ERR_ARG;
+  const int64_t ntiles = (int64_t)(leaf.x1 - leaf.x0) * (leaf.y1 - leaf.y0);
+  const PixArgs a = to_args(px);
+  const int TW = (int)tiles_x(cam->width);
+  cudaStream_t s = to_stream(stream);
+  const float4* rec = reinterpret_cast<const float4*>(proj->rec);
+  switch (pick_ppt(flags, 2)) {
+    case 1:
+      k_raster_fwd<1><<<(unsigned)ntiles, 256, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, TW, a, dev_status);
+      break;
+    case 2:
+      k_raster_fwd<2><<<(unsigned)ntiles, 128, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, TW, a, dev_status);
+      break;
+    default:
+      k_raster_fwd<4><<<(unsigned)ntiles, 64, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, TW, a, dev_status);
+      break;
+  }
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" gs_status gs_loss_l1(const gs_pixels* px, gs_rect leaf, const gs_camera* cam,
+                                gs_stream stream) {
+  if (!cam || !check_leaf(leaf, cam) || !check_pixels(px, leaf, cam)) return GS_ERR_ARG;
+  if (!px->img || !px->target || !px->dL_dimg) return GS_ERR_ARG;
+  const int64_t ntiles = (int64_t)(leaf.x1 - leaf.x0) * (leaf.y1 - leaf.y0);
+  k_loss_l1<<<(unsigned)ntiles, 256, 0, to_stream(stream)>>>(leaf, cam->width, cam->height,
+                                                             (int)tiles_x(cam->width), to_args(px));
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" gs_status gs_loss_total(const float* loss_tiles, int64_t n, double* loss,
+                                   gs_stream stream) {
+  if (n < 0 || !loss || (n > 0 && !loss_tiles)) return GS_ERR_ARG;
+  k_loss_total<<<1, 1024, 0, to_stream(stream)>>>(loss_tiles, n, loss);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals, const int64_t* ranges,
+                                   gs_rect leaf, const gs_camera* cam, const gs_pixels* px,
+                                   float* g2d, uint32_t flags, int32_t* dev_status,
+                                   gs_stream stream) {
+  if (!proj || !ranges || !cam || !g2d || !check_leaf(leaf, cam) || !check_pixels(px, leaf, cam))
+    return GS_ERR_ARG;
+  if (!px->T_final || !px->last || !px->dL_dimg) return GS_ERR_ARG;
+  if (!aligned(proj->rec, 16) || !aligned(g2d, 16)) return GS_ERR_ARG;
+  const int64_t ntiles = (int64_t)(leaf.x1 - leaf.x0) * (leaf.y1 - leaf.y0);
+  const PixArgs a = to_args(px);
+  cudaStream_t s = to_stream(stream);
+  const float4* rec = reinterpret_cast<const float4*>(proj->rec);
+  switch (pick_ppt(flags, 2)) {
+    case 1:
+      k_raster_bwd<1><<<(unsigned)ntiles, 256, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, a, g2d, dev_status);
+      break;
+    case 2:
+      k_raster_bwd<2><<<(unsigned)ntiles, 128, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, a, g2d, dev_status);
+      break;
+    default:
+      k_raster_bwd<4><<<(unsigned)ntiles, 64, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, a, g2d, dev_status);
+      break;
+  }
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}

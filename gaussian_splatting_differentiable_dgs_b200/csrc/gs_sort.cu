@@ -1,0 +1,320 @@
+// Stable LSD radix sort of (key, int32 value) pairs: one histogram pass over
+// all digits, then one "onesweep" pass per digit (Adinets & Merrill,
+// "Onesweep: a faster least significant digit radix sort for GPUs", 2022):
+// each block ranks its tile of 4096 items in shared memory, obtains the
+// global offset of each digit by decoupled look-back across tiles, and
+// scatters through a shared-memory staging buffer so runs of equal digits
+// leave as coalesced stores.
+//
+// Used twice per view: the depth presort of the candidates (32-bit keys),
+// and per Leaf a sort of the duplicated (tile << 32 | depth) keys on the
+// tile bits only.  Because the keys are emitted in depth order, the stable
+// tile-bit sort yields the same order as a full 64-bit sort.
+#include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kSortThreads = 512;
+constexpr int kIPT = 8;
+constexpr int kSortTile = kSortThreads * kIPT;  // 4096 items
+constexpr int kWarps = kSortThreads / 32;
+constexpr int kRadix = 256;
+
+struct SortPlan {
+  int passes;
+  int shift[8];
+  int bits[8];
+};
+
+SortPlan plan_sort(int begin_bit, int end_bit) {
+  SortPlan p{};
+  const int nb = end_bit - begin_bit;
+  if (nb <= 0) return p;
+  // an even number of passes keeps the result in the caller's buffers
+  p.passes = 2 * ((nb + 15) / 16);
+  const int per = (nb + p.passes - 1) / p.passes;
+  int b = begin_bit;
+  for (int k = 0; k < p.passes; ++k) {
+    p.shift[k] = b;
+    p.bits[k] = b + per <= end_bit ? per : end_bit - b;
+    if (p.bits[k] < 0) p.bits[k] = 0;
+    b += p.bits[k];
+  }
+  return p;
+}
+
+template <class K>
+__device__ __forceinline__ unsigned digit_of(K key, int shift, unsigned mask) {
+  return (unsigned)(key >> shift) & mask;
+}
+
+template <class K>
+__global__ void __launch_bounds__(kSortThreads)
+k_hist(const K* __restrict__ keys, int64_t n, SortPlan plan, unsigned long long* __restrict__ hist) {
+  __shared__ unsigned int sh[8][kRadix];
+  for (int e = threadIdx.x; e < 8 * kRadix; e += kSortThreads) (&sh[0][0])[e] = 0;
+  __syncthreads();
+  const int64_t stride = (int64_t)gridDim.x * kSortThreads;
+  for (int64_t i = (int64_t)blockIdx.x * kSortThreads + threadIdx.x; i < n; i += stride) {
+    const K k = keys[i];
+    for (int p = 0; p < plan.passes; ++p)
+      atomicAdd(&sh[p][digit_of(k, plan.shift[p], (1u << plan.bits[p]) - 1)], 1u);
+  }
+  __syncthreads();
+  for (int p = 0; p < plan.passes; ++p)
+    for (int d = threadIdx.x; d < kRadix; d += kSortThreads)
+      if (sh[p][d]) atomicAdd(&hist[p * kRadix + d], (unsigned long long)sh[p][d]);
+}
+
+template <class K>
+struct SortSmem {
+  K keys[kSortTile];
+  int32_t vals[kSortTile];
+  unsigned int wh[kWarps][kRadix];   // per-warp digit counts -> exclusive offsets
+  long long gbase[kRadix];           // global position of the tile's first item of digit d
+  unsigned int tex[kRadix];          // tile-local exclusive offset of digit d
+  unsigned int scan[kWarps + 1];
+  unsigned long long hscan[kWarps + 1];
+  unsigned int tile;
+};
+
+template <class K>
+__global__ void __launch_bounds__(kSortThreads)
+k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool iota,
+           K* __restrict__ dst_k, int32_t* __restrict__ dst_v, int64_t n, int shift, int bits,
+           const unsigned long long* __restrict__ hist, unsigned long long* __restrict__ status,
+           unsigned int* __restrict__ ticket, bool stall, int32_t* dev_status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SortSmem<K>& S = *reinterpret_cast<SortSmem<K>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const unsigned mask = (1u << bits) - 1u;
+  if (tid == 0) S.tile = atomicAdd(ticket, 1u);
+  for (int e = tid; e < kWarps * kRadix; e += kSortThreads) (&S.wh[0][0])[e] = 0;
+  __syncthreads();
+  const int64_t tile = S.tile;
+  const int64_t base = tile * kSortTile;
+
+  // load in warp-striped order: warp w owns items [w*256, w*256+256) of the tile
+  K key[kIPT];
+  int32_t val[kIPT];
+  unsigned dig[kIPT];
+  unsigned rank[kIPT];
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const int64_t idx = base + w * (32 * kIPT) + k * 32 + lane;
+    if (idx < n) {
+      key[k] = src_k[idx];
+      val[k] = iota ? (int32_t)idx : src_v[idx];
+      dig[k] = digit_of(key[k], shift, mask);
+    } else {
+      key[k] = 0;
+      val[k] = 0;
+      dig[k] = kRadix;  // sentinel: not ranked, not written
+    }
+  }
+  // stable rank within the warp: items in (k, lane) order
+  const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const unsigned peers = __match_any_sync(0xffffffffu, dig[k]);
+    unsigned cnt = 0;
+    if (dig[k] < kRadix) cnt = S.wh[w][dig[k]];
+    __syncwarp();
+    if (dig[k] < kRadix && lane == __ffs(peers) - 1) S.wh[w][dig[k]] = cnt + __popc(peers);
+    rank[k] = cnt + __popc(peers & lt_mask);
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // per digit: tile count, exclusive offsets across warps
+  unsigned tcount = 0;
+  if (tid < kRadix) {
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) {
+      const unsigned c = S.wh[ww][tid];
+      S.wh[ww][tid] = tcount;
+      tcount += c;
+    }
+    // publish this tile's aggregate as early as possible
+    unsigned long long* st = status + tile * kRadix + tid;
+    if (tile == 0) {
+      if (!stall) st_relaxed(st, kFlagInc | tcount);
+    } else {
+      st_relaxed(st, kFlagAgg | tcount);
+    }
+  }
+  // global start of each digit (exclusive scan of the histogram)
+  unsigned long long hcount = tid < kRadix ? hist[tid] : 0ull;
+  unsigned long long htot;
+  unsigned long long hstart = 0;
+  unsigned tstart = 0, ttot;
+  {
+    // both scans over the first 256 threads; the rest contribute zeros
+    unsigned long long hx = block_exclusive_scan<unsigned long long, kWarps>(
+        tid < kRadix ? hcount : 0ull, S.hscan, &htot);
+    hstart = hx;
+  }
+  tstart = block_exclusive_scan<unsigned, kWarps>(tid < kRadix ? tcount : 0u, S.scan, &ttot);
+  if (tid < kRadix) {
+    S.tex[tid] = tstart;
+    // look back over earlier tiles for this digit
+    long long excl = 0;
+    if (tile > 0) {
+      int64_t j = tile - 1;
+      int spins = 0;
+      while (j >= 0) {
+        const unsigned long long wv = ld_relaxed(status + j * kRadix + tid);
+        const unsigned flag = (unsigned)(wv >> 62);
+        if (flag == 0) {
+          if (++spins > kSpinCap) {
+            dev_flag(dev_status, GS_DEV_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+          continue;
+        }
+        excl += (long long)(wv & kValMask);
+        if (flag == 2) break;
+        --j;
+      }
+      st_relaxed(status + tile * kRadix + tid, kFlagInc | (unsigned long long)(excl + tcount));
+    }
+    S.gbase[tid] = (long long)hstart + excl;
+  }
+  __syncthreads();
+
+  // stage in shared memory in digit order (stable)
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    if (dig[k] < kRadix) {
+      const unsigned pos = S.tex[dig[k]] + S.wh[w][dig[k]] + rank[k];
+      S.keys[pos] = key[k];
+      S.vals[pos] = val[k];
+    }
+  }
+  __syncthreads();
+  const int64_t rem = n - base;
+  const int count = rem < kSortTile ? (int)rem : kSortTile;
+  for (int e = tid; e < count; e += kSortThreads) {
+    const K kk = S.keys[e];
+    const unsigned d = digit_of(kk, shift, mask);
+    const int64_t gpos = S.gbase[d] + (e - (int64_t)S.tex[d]);
+    if (gpos < 0 || gpos >= n) {
+      dev_flag(dev_status, GS_DEV_BOUNDS);
+      continue;
+    }
+    dst_k[gpos] = kk;
+    dst_v[gpos] = S.vals[e];
+  }
+}
+
+template <class K>
+__global__ void k_copy_pairs(const K* __restrict__ sk, K* __restrict__ dk, int32_t* __restrict__ dv,
+                             const int32_t* __restrict__ sv, bool iota, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  dk[i] = sk[i];
+  dv[i] = iota ? (int32_t)i : sv[i];
+}
+
+template <class K>
+struct SortWs {
+  K* alt_k;
+  int32_t* alt_v;
+  unsigned long long* hist;
+  unsigned int* tickets;
+  unsigned long long* status;
+  size_t zero_begin, zero_bytes, bytes;
+};
+
+template <class K>
+SortWs<K> carve_sort(void* ws, size_t cap, int64_t n, const SortPlan& p) {
+  Carver cv(ws, cap);
+  SortWs<K> s;
+  s.alt_k = cv.take<K>(n > 0 ? n : 1);
+  s.alt_v = cv.take<int32_t>(n > 0 ? n : 1);
+  const int64_t tiles = (n + kSortTile - 1) / kSortTile;
+  s.hist = cv.take<unsigned long long>((size_t)8 * kRadix);
+  s.zero_begin = (size_t)((char*)s.hist - (char*)ws);
+  s.tickets = cv.take<unsigned int>(64);
+  s.status = cv.take<unsigned long long>((size_t)(p.passes > 0 ? p.passes : 1) * (tiles > 0 ? tiles : 1) * kRadix);
+  s.bytes = cv.off;
+  s.zero_bytes = s.bytes - s.zero_begin;
+  return s;
+}
+
+template <class K>
+gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool stall, int64_t n,
+                    int begin_bit, int end_bit, void* ws, size_t ws_bytes, int32_t* dev_status,
+                    cudaStream_t s) {
+  const int kbits = (int)(8 * sizeof(K));
+  if (n < 0 || begin_bit < 0 || end_bit > kbits || begin_bit > end_bit) return GS_ERR_ARG;
+  if (n == 0) return GS_OK;
+  if (!keys || !vals || (!keys_in && !keys)) return GS_ERR_ARG;
+  if (n > (int64_t)INT32_MAX) return GS_ERR_UNSUPPORTED;  // values are int32 positions
+  const SortPlan plan = plan_sort(begin_bit, end_bit);
+  SortWs<K> w = carve_sort<K>(ws, ws_bytes, n, plan);
+  if (!ws || w.bytes > ws_bytes) return GS_ERR_CAPACITY;
+  if (!aligned(ws, 256)) return GS_ERR_ARG;
+  const K* first_k = keys_in ? keys_in : keys;
+  if (plan.passes == 0) {
+    if (keys_in || iota)
+      k_copy_pairs<K><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(first_k, keys, vals, vals, iota, n);
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+  }
+  GS_TRY(cudaMemsetAsync((char*)ws + w.zero_begin, 0, w.zero_bytes, s));
+  const int64_t tiles = (n + kSortTile - 1) / kSortTile;
+  const int hist_blocks = (int)(tiles < 1184 ? tiles : 1184);
+  k_hist<K><<<hist_blocks, kSortThreads, 0, s>>>(first_k, n, plan, w.hist);
+  GS_LAUNCH_CHECK();
+  const size_t smem = sizeof(SortSmem<K>);
+  GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const K* sk = first_k;
+  const int32_t* sv = vals;
+  bool siota = iota;
+  for (int p = 0; p < plan.passes; ++p) {
+    K* dk = (p & 1) ? keys : w.alt_k;
+    int32_t* dv = (p & 1) ? vals : w.alt_v;
+    k_onesweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
+        sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.hist + (size_t)p * kRadix,
+        w.status + (size_t)p * tiles * kRadix, w.tickets + p, stall && p == 0, dev_status);
+    GS_LAUNCH_CHECK();
+    sk = dk;
+    sv = dv;
+    siota = false;
+  }
+  return GS_OK;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" size_t gs_sort_workspace_size(int64_t n, int32_t key_bytes, int32_t begin_bit,
+                                         int32_t end_bit) {
+  if (n < 0 || begin_bit < 0 || end_bit < begin_bit) return 0;
+  const SortPlan p = plan_sort(begin_bit, end_bit);
+  if (key_bytes == 8) return carve_sort<uint64_t>(nullptr, 0, n, p).bytes;
+  if (key_bytes == 4) return carve_sort<uint32_t>(nullptr, 0, n, p).bytes;
+  return 0;
+}
+
+extern "C" gs_status gs_sort_keys(uint64_t* keys, int32_t* vals, int64_t n, int32_t begin_bit,
+                                  int32_t end_bit, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                  gs_stream stream) {
+  return sort_impl<uint64_t>(nullptr, keys, vals, false, false, n, begin_bit, end_bit, ws,
+                             ws_bytes, dev_status, to_stream(stream));
+}
+
+extern "C" gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys, int32_t* vals,
+                                    int64_t n, int32_t begin_bit, int32_t end_bit, uint32_t flags,
+                                    void* ws, size_t ws_bytes, int32_t* dev_status,
+                                    gs_stream stream) {
+  if (flags & ~(GS_SORT_IOTA | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
+  return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0,
+                             (flags & GS_SORT_TEST_STALL) != 0, n, begin_bit, end_bit, ws,
+                             ws_bytes, dev_status, to_stream(stream));
+}

@@ -1,0 +1,271 @@
+"""Per-view training step over the libgs C ABI (the BoundedGS schedule).
+
+BoundedGS project page, section 01: for one view the parameters stay fixed,
+each Leaf runs forward, loss and backward, its gradient is merged and its
+buffers are released before the next Leaf; after the whole view one update
+is applied.  Section 02: A -> B (raster backward collects the projected
+gradients, the raster buffers are released, then projection backward runs),
+B -> C (load-budgeted Leaves, re-planned from the current view's counts),
+C -> D -> E (candidate-only projected state and compact gradients).
+
+This module only sequences library calls and carves device buffers out of
+torch allocations; every stage runs in libgs kernels.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+DEFAULT_BUDGET = 384 << 20
+
+
+def _carve(arena: torch.Tensor, sizes):
+    """Split a uint8 arena into 256-byte aligned byte views."""
+    out, off = [], 0
+    for s in sizes:
+        off = (off + 255) // 256 * 256
+        out.append(arena[off:off + s])
+        off += s
+    return out, off
+
+
+def _carved_bytes(sizes):
+    off = 0
+    for s in sizes:
+        off = (off + 255) // 256 * 256 + s
+    return off
+
+
+@dataclasses.dataclass
+class ViewStats:
+    loss: float
+    n_cand: int
+    n_isect: int
+    n_leaves: int
+    leaves: np.ndarray
+    leaf_isect: np.ndarray
+    leaf_bytes: np.ndarray
+    over_budget: np.ndarray
+    peak_ws_bytes: int
+    arena_bytes: int
+
+
+class GaussianModel:
+    """Parameters and Adam moments, planar [P][n_pad] fp32 on the device."""
+
+    def __init__(self, params: np.ndarray | torch.Tensor, n: int, sh_degree: int,
+                 device="cuda"):
+        p = torch.as_tensor(params, dtype=torch.float32)
+        self.params = p.to(device).contiguous()
+        self.m = torch.zeros_like(self.params)
+        self.v = torch.zeros_like(self.params)
+        self.n = int(n)
+        self.sh_degree = int(sh_degree)
+        self.step = 0
+
+    @property
+    def P(self):
+        return self.params.shape[0]
+
+    @property
+    def n_pad(self):
+        return self.params.shape[1]
+
+    def struct(self) -> B.gs_model:
+        return B.gs_model(self.n, self.n_pad, self.sh_degree, 0, self.params.data_ptr())
+
+
+class Stepper:
+    """Runs the per-view step.  `hooks` (optional) is an object whose methods
+    `on_project(ctx)`, `on_leaf(ctx)`, `on_bwd(ctx)` see intermediate
+    buffers (used by the parity tests)."""
+
+    def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
+                 betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
+                 device="cuda"):
+        self.model = model
+        self.budget = int(budget)
+        self.lr, self.betas, self.eps = lr, betas, eps
+        self.raster_flags = raster_flags
+        self.fuse_adam = fuse_adam
+        self.device = torch.device(device)
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.launches = 0
+
+    # ------------------------------------------------------------------
+    def check(self):
+        st = B.gs_check(self.dev_status)
+        if st < 0:
+            raise B.GsError("device status", st)
+
+    def adam_args(self, step):
+        return B.gs_adam_args(self.lr, self.betas[0], self.betas[1], self.eps, step, 0)
+
+    # ------------------------------------------------------------------
+    def run_view(self, cam, target, leaves=None, hooks=None, update=True) -> ViewStats:
+        """cam: synth.Camera; target: [3][H][W] fp32, either a device tensor
+        (the whole view resident) or a pinned host tensor (each Leaf's crop
+        is uploaded before its forward).  `leaves` overrides the planner
+        (list of tile rects)."""
+        dev = self.device
+        m = self.model
+        W, H = cam.width, cam.height
+        TW, TH = (W + 15) // 16, (H + 15) // 16
+        T = TW * TH
+        tile_bits = max(1, math.ceil(math.log2(T))) if T > 1 else 1
+        camS = B.camera_struct(cam)
+        mod = m.struct()
+        st = self.dev_status
+        base_alloc = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        launches = 0
+
+        # ---- projection (+ counts, SAT) ---------------------------------
+        n = m.n
+        cap = max(n, 1)
+        n_cand_d = torch.zeros(1, dtype=torch.int32, device=dev)
+        cand_idx = torch.empty(cap, dtype=torch.int32, device=dev)
+        slot = torch.empty(cap, dtype=torch.int32, device=dev)
+        rec = torch.empty(cap * 12, dtype=torch.float32, device=dev)
+        rect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
+        dkey = torch.empty(cap, dtype=torch.int32, device=dev)
+        proj = B.gs_proj(cap, n_cand_d.data_ptr(), cand_idx.data_ptr(), slot.data_ptr(),
+                         rec.data_ptr(), rect.data_ptr(), dkey.data_ptr())
+        sat = torch.empty((TH + 1) * (TW + 1), dtype=torch.int64, device=dev)
+        ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
+        B.gs_project(mod, camS, proj, sat, ws, st)
+        launches += 4
+        del ws
+        sat_h = torch.empty(sat.shape, dtype=torch.int64, pin_memory=True)
+        nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+        sat_h.copy_(sat, non_blocking=True)
+        nc_h.copy_(n_cand_d, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()   # the one sync per view
+        C = int(nc_h[0])
+        sat_np = sat_h.numpy().reshape(TH + 1, TW + 1)
+        ctx = dict(proj=proj, cand_idx=cand_idx, slot=slot, rec=rec, rect=rect, depth_key=dkey,
+                   sat=sat, sat_host=sat_np, n_cand=C, TW=TW, TH=TH, cam=cam)
+        if hooks is not None and hasattr(hooks, "on_project"):
+            hooks.on_project(ctx)
+
+        # ---- depth presort --------------------------------------------------
+        order = torch.empty(max(C, 1), dtype=torch.int32, device=dev)
+        if C > 0:
+            k32 = torch.empty(C, dtype=torch.int32, device=dev)
+            ws = torch.empty(B.gs_sort_workspace_size(C, 4, 0, 32), dtype=torch.uint8, device=dev)
+            B.gs_sort_keys32(dkey, k32, order, C, 0, 32, B.GS_SORT_IOTA, ws, st)
+            launches += 1 + 4
+            del ws, k32
+        ctx["depth_order"] = order
+
+        # ---- Leaf plan ------------------------------------------------------
+        lm = B.gs_leaf_load_model(tile_bits)
+        if leaves is None:
+            _, lv, li, lb, ov = B.gs_leaf_partition(sat_np, TW, TH, W, H, lm, self.budget)
+        else:
+            lv = np.asarray(leaves, np.int32).reshape(-1, 4)
+            li = np.array([sat_np[y1, x1] - sat_np[y0, x1] - sat_np[y1, x0] + sat_np[y0, x0]
+                           for x0, y0, x1, y1 in lv], np.int64)
+            lb = np.zeros(len(lv), np.int64)
+            ov = np.zeros(len(lv), bool)
+
+        # ---- per-Leaf raster: forward + L1 + backward into compact g2d ----------
+        g2d = torch.zeros(max(C, 1) * 12, dtype=torch.float32, device=dev)
+        loss_tiles = torch.zeros(T, dtype=torch.float32, device=dev)
+        bin_ws = torch.empty(max(B.gs_bin_workspace_size(C), 256), dtype=torch.uint8, device=dev)
+        resident_target = target is not None and target.is_cuda
+        tgt = target if resident_target else None
+
+        def leaf_sizes(L, I):
+            x0, y0, x1, y1 = (int(v) for v in L)
+            pw = min(16 * x1, W) - 16 * x0
+            ph = min(16 * y1, H) - 16 * y0
+            npx = pw * ph
+            nt = (x1 - x0) * (y1 - y0)
+            sizes = [8 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 8, 32, 32 + tile_bits),
+                     12 * npx, 4 * npx, 4 * npx, 12 * npx]
+            if not resident_target:
+                sizes.append(12 * npx)
+            return sizes, (16 * x0, 16 * y0, pw, ph)
+
+        arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
+                          default=0)
+        arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
+        norm = 1.0 / (3.0 * W * H)
+        for k, (L, I) in enumerate(zip(lv, li)):
+            I = int(I)
+            sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
+            bufs, _ = _carve(arena, sizes)
+            keys = bufs[0].view(torch.int64)
+            vals = bufs[1].view(torch.int32)
+            ranges = bufs[2].view(torch.int64)
+            sort_ws = bufs[3]
+            img = bufs[4].view(torch.float32)
+            Tf = bufs[5].view(torch.float32)
+            last = bufs[6].view(torch.int32)
+            dL = bufs[7].view(torch.float32)
+            if resident_target:
+                # the whole view's target is read in place with its own pitch
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=tgt,
+                              target_origin=(0, 0), target_pitch=W, target_plane=W * H,
+                              loss_tiles=loss_tiles, norm=norm)
+            else:
+                # bounded supply: the Leaf's crop of a host target is uploaded
+                crop = bufs[8].view(torch.float32).view(3, ph, pw)
+                crop.copy_(target[:, py0:py0 + ph, px0:px0 + pw], non_blocking=True)
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
+                              target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm)
+            B.gs_bin_tiles(proj, C, order, L, TW, TH, sat, I, keys, vals, max(I, 1), ranges,
+                           bin_ws, st)
+            launches += 2
+            if I > 0:
+                B.gs_sort_keys(keys, vals, I, 32, 32 + tile_bits, sort_ws, st)
+                launches += 1 + 2 * ((tile_bits + 15) // 16)
+            B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
+            launches += 1
+            if hooks is not None and hasattr(hooks, "on_leaf"):
+                hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
+                                        ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
+                                        n_isect=I, px_rect=(px0, py0, pw, ph)))
+            B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
+            launches += 1
+        del arena, bin_ws  # raster buffers released before projection backward
+
+        loss_d = torch.zeros(1, dtype=torch.float64, device=dev)
+        B.gs_loss_total(loss_tiles, T, loss_d)
+        launches += 1
+        ctx["g2d"] = g2d
+        if hooks is not None and hasattr(hooks, "on_bwd"):
+            hooks.on_bwd(ctx)
+
+        # ---- projection backward fused with ONE Adam update -----------------
+        if update:
+            m.step += 1
+            if self.fuse_adam:
+                B.gs_project_bwd(mod, camS, proj, C, g2d, adam_m=m.m, adam_v=m.v,
+                                 fused=self.adam_args(m.step), dev_status=st)
+                launches += 1
+            else:
+                g3d = torch.empty(m.P * max(C, 1), dtype=torch.float32, device=dev)
+                B.gs_project_bwd(mod, camS, proj, C, g2d, g3d=g3d, g3d_stride=max(C, 1),
+                                 dev_status=st)
+                B.gs_adam(m.params, m.m, m.v, g3d, max(C, 1), slot, m.n, m.n_pad, m.P,
+                          self.adam_args(m.step))
+                launches += 2
+                del g3d
+        self.launches = launches
+        peak = torch.cuda.max_memory_allocated(dev) - base_alloc
+        if resident_target:
+            peak += target.numel() * target.element_size()
+        self._last_loss = loss_d
+        return ViewStats(loss=float("nan"), n_cand=C, n_isect=int(li.sum()),
+                         n_leaves=len(lv), leaves=lv, leaf_isect=li, leaf_bytes=lb,
+                         over_budget=ov, peak_ws_bytes=int(peak), arena_bytes=int(arena_bytes))
+
+    def last_loss(self) -> float:
+        return float(self._last_loss.item())

@@ -1,0 +1,311 @@
+/*
+ * gs.h -- C ABI of libgs: one 3D Gaussian Splatting training step on an
+ * NVIDIA B200 (sm_100a), with the BoundedGS memory scheme.
+ *
+ * The step for one view is
+ *
+ *   gs_project       cull + EWA projection of the candidate Gaussians,
+ *                    per-tile intersection counts and their summed-area table
+ *   gs_sort_keys32   depth presort of the candidates (once per view)
+ *   gs_leaf_partition  (host) split the tile grid into Leaves whose
+ *                    estimated load fits a byte budget
+ *   for each Leaf:
+ *     gs_bin_tiles   duplicated 64-bit keys (tile << 32 | depth) in depth order
+ *     gs_sort_keys   stable radix sort on the tile bits -> per-tile lists
+ *     gs_raster_fwd  front-to-back compositing (+ fused L1 loss)
+ *     gs_raster_bwd  reverse blend, accumulated into the view's compact
+ *                    per-candidate 2D gradients
+ *   gs_project_bwd   projection backward, fused with ONE Adam update per view
+ *
+ * Sources (page title, section):
+ *  - "BoundedGS: memory-efficient training for high-resolution 3D Gaussian
+ *    Splatting" (project page), section 01: gradients of a local region are
+ *    merged before its buffers are released; Leaves are sized by a load
+ *    estimate from overlaps, pixels and buffer layout; the whole view's
+ *    gradient is summed before one parameter update.  Section 02: A -> B
+ *    two-stage backward (raster backward first, then projection backward);
+ *    B -> C load-budgeted Leaves, over-budget regions split again, load
+ *    re-checked before each execution; C -> D -> E candidate-index
+ *    projection and compact gradients.
+ *  - "SkipGS: Post-Densification Backward Skipping for Efficient 3DGS
+ *    Training" (paper notes), sections "research background" (differentiable
+ *    rasterisation of anisotropic 3D Gaussians), "key design 2" (backward =
+ *    gradient back-propagation, atomic accumulation, coordinate and
+ *    covariance differentiation) and "loss function / training strategy"
+ *    (gradients through the projected 2D covariance and the transmittance
+ *    accumulation to means, quaternions, scales, opacities and SH
+ *    coefficients; Adam).
+ *
+ * Conventions
+ *  - Every call returns a gs_status.  Arguments are checked on the host;
+ *    errors found by a kernel are OR-ed into the caller's device word
+ *    `dev_status` (GS_DEV_* bits) and reported by gs_check().
+ *  - All device buffers are owned by the caller.  The library never
+ *    allocates or frees memory; scratch comes from a caller workspace whose
+ *    size the gs_*_workspace_size() queries return.  Workspaces need 256-byte
+ *    alignment.
+ *  - Every device call is asynchronous on the given stream (a cudaStream_t;
+ *    NULL = the legacy default stream) and never synchronises, except
+ *    gs_check().  There is no global state: calls on different streams with
+ *    different buffers may run concurrently.
+ *  - Layout of the model (planar SoA, fp32): params[P][n_pad],
+ *    P = 11 + 3 (D+1)^2:  0..2 mean, 3..5 log-scale, 6..9 quaternion
+ *    (w,x,y,z), 10 opacity logit, 11 + 3k + ch SH coefficient k, channel ch.
+ *    n_pad must be a multiple of 4 and params 16-byte aligned.
+ *  - Tiles are 16 x 16 pixels; TW = ceil(W/16), TH = ceil(H/16); tile id =
+ *    ty * TW + tx.  Pixel centres are at (x + 0.5, y + 0.5).
+ */
+#ifndef GS_H
+#define GS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t gs_status;
+#define GS_OK 0
+#define GS_WARN_BUDGET 1       /* a 1x1 Leaf is over budget (accepted) */
+#define GS_ERR_ARG (-1)        /* bad pointer, size, alignment or value */
+#define GS_ERR_CAPACITY (-2)   /* buffer or workspace too small; *needed set */
+#define GS_ERR_CUDA (-3)       /* a CUDA runtime call failed */
+#define GS_ERR_TIMEOUT (-4)    /* a bounded device wait gave up */
+#define GS_ERR_BOUNDS (-5)     /* a kernel saw an index out of range */
+#define GS_ERR_UNSUPPORTED (-6)
+
+/* bits a kernel ORs into *dev_status */
+#define GS_DEV_TIMEOUT 1u
+#define GS_DEV_BOUNDS 2u
+#define GS_DEV_NONFINITE 4u    /* non-finite parameter met; Gaussian culled */
+
+#define GS_TILE 16
+
+typedef void* gs_stream; /* cudaStream_t */
+
+/* Pinhole camera.  x_cam = R x_world + t (R row-major), OpenCV axes. */
+typedef struct gs_camera {
+  float R[9];
+  float t[3];
+  float fx, fy, cx, cy;
+  int32_t width, height;
+} gs_camera;
+
+typedef struct gs_model {
+  int64_t n;          /* Gaussians */
+  int64_t n_pad;      /* plane stride, multiple of 4, >= n */
+  int32_t sh_degree;  /* 0..3 */
+  int32_t reserved;
+  float* params;      /* device [P][n_pad] */
+} gs_model;
+
+/* Per-view projected state of the candidates (Gaussians that can touch the
+ * view), in ascending Gaussian index.  Written by gs_project.
+ * rec: 12 floats per candidate = three float4
+ *   {u_hi, v_hi, u_lo, v_lo}  screen position as an unevaluated fp32 pair
+ *   {s1, beta, s2, opacity}   q = s1 (dx + beta dy)^2 + s2 dy^2 with
+ *                             s1 = a/2, beta = b/a, s2 = 1/(2 Sigma'_11),
+ *                             (a, b, c) the conic Sigma'^-1
+ *   {R, G, B, depth}
+ * rect: tiles [x0, x1) x [y0, y1) covered by the 3-sigma square. */
+typedef struct gs_proj {
+  int64_t capacity;     /* candidate capacity of the arrays below (>= n) */
+  int32_t* n_cand;      /* device scalar */
+  int32_t* cand_idx;    /* device [capacity] Gaussian index of each slot */
+  int32_t* slot;        /* device [n] slot of Gaussian i, or -1 */
+  float* rec;           /* device [capacity][12], 16-byte aligned */
+  int16_t* rect;        /* device [capacity][4] */
+  uint32_t* depth_key;  /* device [capacity] bits of fp32 camera depth */
+} gs_proj;
+
+/* A rectangle of tiles, half-open. */
+typedef struct gs_rect {
+  int32_t x0, y0, x1, y1;
+} gs_rect;
+
+/* Per-pixel buffers of one Leaf.  Pixel (x, y) of the image, for x in
+ * [x0, x0 + w), y in [y0, y0 + h), lives at offset (y - y0) * pitch +
+ * (x - x0) of img, T_final, last and each colour plane of dL_dimg; colour
+ * planes are `plane` elements apart.  The target has its own layout: pixel
+ * (x, y), channel c at target[(y - ty0) * tpitch + (x - tx0) + c * tplane]
+ * (e.g. the whole view resident with tx0 = ty0 = 0, tpitch = W). */
+typedef struct gs_pixels {
+  int32_t x0, y0, w, h;
+  int64_t pitch;
+  int64_t plane;
+  float* img;             /* [3] planes: rendered colour (written by fwd) */
+  float* T_final;         /* transmittance after the last composited entry */
+  int32_t* last;          /* 1 + list position of the last composited entry */
+  float* dL_dimg;         /* [3] planes: dL/dcolour */
+  const float* target;    /* or NULL (the forward then skips the loss) */
+  int32_t tx0, ty0;
+  int64_t tpitch;
+  int64_t tplane;
+  float* loss_tiles;      /* per global tile: norm * sum |r - t|, or NULL */
+  double norm;            /* 1 / (3 W H): whole-view normaliser */
+} gs_pixels;
+
+/* Byte cost model of a Leaf (the buffers this library needs per unit). */
+typedef struct gs_load_model {
+  int64_t bytes_per_isect;
+  int64_t bytes_per_pixel;
+  int64_t bytes_per_tile;
+  int64_t fixed_bytes;
+  int64_t align;
+} gs_load_model;
+
+typedef struct gs_adam_args {
+  float lr, beta1, beta2, eps;
+  int32_t step;  /* 1 on the first update */
+  int32_t reserved;
+} gs_adam_args;
+
+int32_t gs_version(void);
+const char* gs_status_string(gs_status s);
+
+/* Synchronises `stream`, then reads and clears *dev_status.  Returns the
+ * most severe condition (GS_ERR_TIMEOUT > GS_ERR_BOUNDS > GS_OK). */
+gs_status gs_check(int32_t* dev_status, gs_stream stream);
+
+/* ---- 1. projection -------------------------------------------------------
+ * Cull + EWA projection.  For every Gaussian: t = R mu + t_cam; cull if
+ * t_z <= 0.2, |t_x/t_z| > 1.3 (W/2)/f_x or |t_y/t_z| > 1.3 (H/2)/f_y, the
+ * 2D covariance is not positive definite, or the tile rect is empty.  For
+ * candidates: Sigma = R S S^T R^T (normalised quaternion, S = exp(log-scale)),
+ * Sigma' = J W Sigma W^T J^T + 0.3 I, conic = Sigma'^-1, radius =
+ * ceil(3 sqrt(lambda_max)), colour = max(0, sum_k sh_k Y_k(d) + 0.5),
+ * opacity = sigmoid(logit), depth = t_z.  Candidates are compacted in
+ * ascending index order (slot map in proj->slot).  Also writes the
+ * (TH+1) x (TW+1) int64 summed-area table of per-tile intersection counts
+ * (row 0 and column 0 zero) to `tile_sat`.
+ * The projection arithmetic is fp64; records are rounded to fp32.
+ * flags: 0 (reserved). */
+size_t gs_project_workspace_size(int64_t n, int32_t width, int32_t height);
+gs_status gs_project(const gs_model* model, const gs_camera* cam,
+                     uint32_t flags, const gs_proj* out, int64_t* tile_sat,
+                     void* ws, size_t ws_bytes, int32_t* dev_status,
+                     gs_stream stream);
+
+/* ---- 2. radix sorts ------------------------------------------------------
+ * Stable LSD radix sort (onesweep: one histogram pass, then one pass per
+ * digit with decoupled look-back) of (key, value) pairs on key bits
+ * [begin_bit, end_bit).  The result is in keys[], vals[] (in place).  For
+ * the 32-bit variant, keys_in (if not NULL) is read instead of keys on the
+ * first pass, and flag GS_SORT_IOTA makes the input values 0..n-1.
+ * Bounded look-back waits: on expiry GS_DEV_TIMEOUT is set and the call
+ * returns without hanging. */
+#define GS_SORT_IOTA 1u
+/* Test hook of the bounded wait: the first tile of the first pass does not
+ * publish its counts, so every later tile's look-back runs out and reports
+ * GS_DEV_TIMEOUT (the result is then unspecified).  Never set otherwise. */
+#define GS_SORT_TEST_STALL 0x80000000u
+size_t gs_sort_workspace_size(int64_t n, int32_t key_bytes, int32_t begin_bit,
+                              int32_t end_bit);
+gs_status gs_sort_keys(uint64_t* keys, int32_t* vals, int64_t n,
+                       int32_t begin_bit, int32_t end_bit, void* ws,
+                       size_t ws_bytes, int32_t* dev_status, gs_stream stream);
+gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys,
+                         int32_t* vals, int64_t n, int32_t begin_bit,
+                         int32_t end_bit, uint32_t flags, void* ws,
+                         size_t ws_bytes, int32_t* dev_status,
+                         gs_stream stream);
+
+/* ---- 3. Leaf partition (host) --------------------------------------------
+ * Recursive split of the tile grid: a rect whose estimated load
+ *   align(I * b_isect) + align(pixels * b_px) + align(tiles * b_tile) + fixed
+ * (I from the host copy of the SAT, pixels clipped to the image) exceeds
+ * `budget` is cut at the midpoint of its longer side (x on ties) and both
+ * halves are processed, first half first; a 1x1 rect is always accepted and
+ * flagged over_budget if it does not fit.  Leaves come out in that
+ * depth-first order.  Returns GS_WARN_BUDGET if any Leaf is over budget,
+ * GS_ERR_CAPACITY if more than max_leaves would be needed (*n_leaves is
+ * then the number required). */
+gs_status gs_leaf_load_model(int32_t tile_bits, gs_load_model* out);
+gs_status gs_leaf_partition(const int64_t* sat_host, int32_t TW, int32_t TH,
+                            int32_t width, int32_t height,
+                            const gs_load_model* lm, int64_t budget,
+                            gs_rect* leaves, int64_t* leaf_isect,
+                            int64_t* leaf_bytes, uint8_t* over_budget,
+                            int32_t max_leaves, int32_t* n_leaves);
+
+/* ---- 4. binning ----------------------------------------------------------
+ * For the candidates in depth order (depth_order[0..n_cand)), emit one
+ * entry per tile of rect ∩ leaf: key = (tile id << 32) | depth_key, value =
+ * candidate slot, in depth order; and the Leaf's per-tile ranges
+ * (ranges[2 * (ly * lw + lx)] = begin, [+1] = end, offsets into keys/vals,
+ * tile rows of the Leaf in row-major order) from the device SAT.
+ * n_isect: the Leaf's intersection count (from the host SAT); must be <=
+ * capacity, else GS_ERR_CAPACITY with *needed = n_isect. */
+size_t gs_bin_workspace_size(int64_t n_cand);
+gs_status gs_bin_tiles(const gs_proj* proj, int64_t n_cand,
+                       const int32_t* depth_order, gs_rect leaf, int32_t TW,
+                       int32_t TH, const int64_t* tile_sat, int64_t n_isect,
+                       uint64_t* keys, int32_t* vals, int64_t capacity,
+                       int64_t* ranges, int64_t* needed, void* ws,
+                       size_t ws_bytes, int32_t* dev_status, gs_stream stream);
+
+/* ---- 5. raster forward ---------------------------------------------------
+ * Per pixel p of the Leaf, over its tile's list in order: d = (u, v) - p;
+ * q = (a d_x^2 + c d_y^2)/2 + b d_x d_y; alpha = min(0.99, o exp(-q)); skip
+ * if alpha < 1/255; T' = T (1 - alpha); stop (without compositing) if
+ * T' < 1e-4; else C += rgb alpha T, T = T'.  Background 0.  Writes img,
+ * T_final, last; if px->target is set, also the L1 loss terms (as
+ * gs_loss_l1).  fp32 arithmetic.
+ * flags & 7 selects the pixels per thread (1, 2 or 4; 0 = default); the
+ * result does not depend on it.  The same flag applies to gs_raster_bwd. */
+gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals,
+                        const int64_t* ranges, gs_rect leaf,
+                        const gs_camera* cam, const gs_pixels* px,
+                        uint32_t flags, int32_t* dev_status, gs_stream stream);
+
+/* ---- 6. L1 loss ----------------------------------------------------------
+ * For the Leaf's pixels: dL/dimg = sign(img - target) * norm (sign(0) = 0)
+ * and, per global tile, loss_tiles[tile] = norm * sum |img - target| in a
+ * fixed order.  gs_loss_total sums loss_tiles[0..n) in a fixed order in
+ * fp64 into *loss (device), so the loss is independent of the Leaves. */
+gs_status gs_loss_l1(const gs_pixels* px, gs_rect leaf, const gs_camera* cam,
+                     gs_stream stream);
+gs_status gs_loss_total(const float* loss_tiles, int64_t n, double* loss,
+                        gs_stream stream);
+
+/* ---- 7. raster backward --------------------------------------------------
+ * Reverse blend over list positions last-1 .. 0 with the forward's skip
+ * tests, transmittance recovered as T_i = T_{i+1} / (1 - alpha_i).
+ * Accumulates (adds) per candidate slot into g2d[slot][12] the gradients
+ * {du, dv, da, db, dc, dopacity, dR, dG, dB, 0, 0, 0} ((a, b, c) = conic)
+ * with per-tile reduction before the global atomics. */
+gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals,
+                        const int64_t* ranges, gs_rect leaf,
+                        const gs_camera* cam, const gs_pixels* px, float* g2d,
+                        uint32_t flags, int32_t* dev_status, gs_stream stream);
+
+/* ---- 8. projection backward ----------------------------------------------
+ * Stage 2 of the two-stage backward: the exact derivative of gs_project's
+ * candidate formulas, from g2d[slot][12] to every parameter (mean including
+ * the SH view-direction term, log-scale, quaternion through the
+ * normalisation, opacity logit, SH).  If `fused` is NULL, writes compact
+ * gradients g3d[P][g3d_stride] (column = candidate slot).  Otherwise applies
+ * one Adam update (as gs_adam with a zero gradient for non-candidates) to
+ * model->params, adam_m and adam_v over all n Gaussians; g3d is unused. */
+gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
+                         const gs_proj* proj, int64_t n_cand,
+                         const float* g2d, float* g3d, int64_t g3d_stride,
+                         float* adam_m, float* adam_v,
+                         const gs_adam_args* fused, int32_t* dev_status,
+                         gs_stream stream);
+
+/* ---- 9. Adam -------------------------------------------------------------
+ * m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+ * p -= lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps), for i < n, all P
+ * planes.  If slot is NULL, g is dense [P][n_pad]; else g is compact
+ * [P][g_stride] and Gaussian i reads column slot[i] (zero if -1). */
+gs_status gs_adam(float* params, float* m, float* v, const float* g,
+                  int64_t g_stride, const int32_t* slot, int64_t n,
+                  int64_t n_pad, int32_t P, const gs_adam_args* args,
+                  gs_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GS_H */
