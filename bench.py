@@ -1,0 +1,439 @@
+"""Benchmark of one 3DGS training step (fwd + L1 + bwd + one Adam update per
+view, BoundedGS Leaf schedule) on the outdoor-like synthetic scene:
+6,000,000 Gaussians, SH degree 3, 5000x3300, 8 views on a circle, 384 MiB
+Leaf budget.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank trains an
+independent replica of the workload on its own GPU (no data-path
+collective); value is the total over ranks divided by the max-over-ranks
+device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("fwd+bwd+Adam step ms & Gaussian-tile intersections/s per B200; "
+          "peak working set GiB")
+UNIT = "intersections/s"
+SM_COUNT, LANES_PER_SM = 148, 128
+# algorithmic lane-ops per pixel-Gaussian pair (measurement)
+OPS_FWD_VISIT, OPS_FWD_KEPT = 11, 8
+OPS_BWD_VISIT, OPS_BWD_KEPT = 11, 32
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=16)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--gaussians", type=int, default=6_000_000)
+    ap.add_argument("--width", type=int, default=5000)
+    ap.add_argument("--height", type=int, default=3300)
+    ap.add_argument("--views", type=int, default=8)
+    ap.add_argument("--budget-mib", type=float, default=384)
+    ap.add_argument("--raster-ppt", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-tiles", type=int, default=64)
+    return ap.parse_args()
+
+
+def workload_name(a):
+    return (f"outdoor_{a.gaussians / 1e6:g}m_{a.width}x{a.height}: {a.gaussians:,} Gaussians "
+            f"SH3, {a.views} views on a radius-4 circle, {a.budget_mib:g} MiB Leaf budget")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """Times the oracle's stages on samples of one view and scales each to
+    the full step: projection of a 1/8 subset of the Gaussians (x8), tile
+    lists (scatter + stable sort) of a 1/16 subset of the candidates (x16),
+    raster forward + L1 + raster backward on `n_tiles` uniformly random tiles
+    (x tiles / n_tiles), projection backward on a 1/16 subset of the
+    candidates (x16) and Adam on a 1/64 subset of the Gaussians (x64)."""
+
+    def __init__(self, scene, cams, target_fn, n_tiles=64, seed=0):
+        from oracle import oracle as O
+        self.O = O
+        O.build()
+        self.scene = scene
+        self.cams = cams
+        self.n_tiles = n_tiles
+        self.rng = np.random.default_rng(seed)
+        self.target_fn = target_fn
+        self.cache = {}
+
+    def _setup(self, v):
+        if v in self.cache:
+            return self.cache[v]
+        O, sc, cam = self.O, self.scene, self.cams[v]
+        p64 = sc.params.astype(np.float64)
+        pr = O.project(p64, sc.n, sc.sh_degree, cam)
+        TW, TH = O.grid(cam)
+        counts = O.tile_counts_fast(pr["rect"], TW, TH).reshape(-1)
+        self.cache[v] = (p64, pr, counts, TW, TH)
+        return self.cache[v]
+
+    def step(self, v):
+        O, sc, cam = self.O, self.scene, self.cams[v]
+        p64, pr, counts, TW, TH = self._setup(v)
+        n = sc.n
+        W, H = cam.width, cam.height
+        I_total = int(counts.sum())
+        # projection of 1/8 of the Gaussians
+        sub = np.sort(self.rng.choice(n, n // 8, replace=False))
+        ps = np.ascontiguousarray(p64[:, sub])
+        t0 = time.perf_counter()
+        O.project(ps, len(sub), sc.sh_degree, cam)
+        t_proj = (time.perf_counter() - t0) * n / len(sub)
+        # tile lists: scatter + per-tile stable sort for 1/16 of the candidates
+        C = len(pr["cand_idx"])
+        cs = np.sort(self.rng.choice(C, max(C // 16, 1), replace=False))
+        t0 = time.perf_counter()
+        O.tile_lists_all(pr["rect"][cs], pr["key"][cs], TW, TH)
+        t_lists = (time.perf_counter() - t0) * C / len(cs)
+        # raster forward + L1 + raster backward on uniformly random tiles
+        tiles = np.sort(self.rng.choice(TW * TH, self.n_tiles, replace=False)).astype(np.int32)
+        off, vals = O.tile_lists(pr["rect"], pr["key"], TW, tiles)
+        target = self.target_fn(v)
+        tg = O.gather_tiles(np.pad(target, ((0, 0), (0, TH * 16 - H), (0, TW * 16 - W))),
+                            tiles, TW, 3)
+        t0 = time.perf_counter()
+        fw = O.raster_fwd(pr["rec"], TW, W, H, tiles, off, vals)
+        valid = (fw["flags"] & 0x80) == 0
+        d = np.where(valid[:, None, :], fw["img"] - tg, 0.0)
+        dL = np.sign(d) / (3.0 * W * H)
+        O.raster_bwd(pr["rec"], TW, W, H, tiles, off, vals, dL)
+        t_raster = (time.perf_counter() - t0) * (TW * TH) / self.n_tiles
+        I_s = int(off[-1])
+        # projection backward on 1/16 of the candidates
+        g2d = self.rng.normal(size=(len(cs), 9)) * 1e-3
+        t0 = time.perf_counter()
+        O.project_bwd(p64, sc.sh_degree, cam, pr["cand_idx"][cs], g2d)
+        t_pbwd = (time.perf_counter() - t0) * C / len(cs)
+        # Adam on 1/64 of the Gaussians (all planes)
+        k = max(n // 64, 1)
+        pa = p64[:, :k]
+        g = self.rng.normal(size=pa.shape)
+        t0 = time.perf_counter()
+        O.adam(pa, np.zeros_like(pa), np.zeros_like(pa), g, step=1)
+        t_adam = (time.perf_counter() - t0) * n / k
+        est = t_proj + t_lists + t_raster + t_pbwd + t_adam
+        return dict(est_step_s=est, I_total=I_total, sample_isect=I_s,
+                    parts=dict(project=t_proj, lists=t_lists, raster=t_raster,
+                               project_bwd=t_pbwd, adam=t_adam))
+
+    def describe(self):
+        return (f"per step: oracle projection of 1/8 of the Gaussians (x8), tile lists of 1/16 "
+                f"of the candidates (x16), raster fwd + L1 + raster bwd on {self.n_tiles} "
+                f"uniformly random tiles (x tiles/{self.n_tiles}), projection bwd on 1/16 of the "
+                f"candidates (x16), Adam on 1/64 of the Gaussians (x64); value = the view's "
+                f"intersections / estimated step time")
+
+
+# ---------------------------------------------------------------------------
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from gaussian_splatting_differentiable_dgs_b200 import synth
+
+    if a.impl == "reference":
+        return run_reference(a, rank, world)
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper, STAGES
+
+    scene, cams = synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
+                                      n_views=a.views)
+    W, H = a.width, a.height
+    budget = int(a.budget_mib * (1 << 20))
+    # targets: renders of the jittered copy (means N(0, 0.02), colour N(0, 0.05))
+    jit = synth.jittered(scene, seed=1)
+    jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
+    js = Stepper(jm, budget=budget, raster_flags=a.raster_ppt)
+    targets = [js.render(c) for c in cams]
+    torch.cuda.synchronize()
+    del jm, js
+    model = GaussianModel(scene.params, scene.n, scene.sh_degree)
+    stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt)
+    nv = len(cams)
+    view_of = lambda k: (k + rank) % nv
+
+    for k in range(a.warmup):
+        stp.run_view(cams[view_of(k)], targets[view_of(k)])
+    stp.check()
+
+    # ---- timed region (device time, CUDA events on the launching stream) -----
+    timing = {}
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    stats = []
+    for k in range(a.steps):
+        v = view_of(a.warmup + k)
+        stats.append(stp.run_view(cams[v], targets[v], timing=timing))
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    stp.check()
+    ms = e0.elapsed_time(e1)
+    isect = sum(s.n_isect for s in stats)
+    launches = sum(s.launches for s in stats)
+    peak_ws = max(s.peak_ws_bytes for s in stats)
+    stage_ms = {name: sum(x.elapsed_time(y) for x, y in timing.get(name, [])) for name in STAGES}
+    stage_n = {name: len(timing.get(name, [])) for name in STAGES}
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+        t = torch.tensor([isect], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t)
+        isect_all = float(t.item())
+    else:
+        ms_max, isect_all = ms, float(isect)
+    value = isect_all / (ms_max / 1e3)
+
+    # ---- accounting step (untimed): work counters per launch -----------------
+    counters = torch.zeros(4, dtype=torch.int64, device="cuda")
+    acc_timing = {}
+    v = view_of(a.warmup + a.steps)
+    acc = stp.run_view(cams[v], targets[v], counters=counters, timing=acc_timing)
+    torch.cuda.synchronize()
+    cnt = [int(x) for x in counters.cpu()]
+    ops_fwd = cnt[0] * OPS_FWD_VISIT + cnt[1] * OPS_FWD_KEPT
+    ops_bwd = cnt[2] * OPS_BWD_VISIT + cnt[3] * OPS_BWD_KEPT
+
+    peaks, peak_src = load_peaks()
+    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    alu_peak = SM_COUNT * LANES_PER_SM * sm_mhz * 1e6  # lane-ops/s
+    # dominant kernel over the timed region
+    dom = max(STAGES, key=lambda s: stage_ms[s])
+    n_steps = a.steps
+    per_step = {s: stage_ms[s] / n_steps for s in STAGES}
+    if dom in ("raster_bwd", "raster_fwd"):
+        ops = ops_bwd if dom == "raster_bwd" else ops_fwd
+        ach = ops / (per_step[dom] / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": f"k_{dom}", "achieved": round(ach, 3),
+                "peak": round(alu_peak / 1e12, 3), "unit": "Tlane-op/s",
+                "frac": round(ach / (alu_peak / 1e12), 4), "traffic": None,
+                "peak_source": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {sm_mhz:g} MHz "
+                               f"(sm_max_mhz of {peak_src})"}
+    else:
+        P = model.P
+        C = acc.n_cand
+        byt = scene.n * P * 24 + C * (48 + 16) + scene.n * 4
+        ach = byt / (per_step[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": round(ach, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                "traffic": None}
+
+    # ---- end to end through host buffers --------------------------------------
+    e2e = None
+    if not a.no_e2e:
+        host_t = [t.cpu().pin_memory() for t in targets]
+        dev_t = torch.empty_like(targets[0])
+        loss_h = torch.empty(1, dtype=torch.float64, pin_memory=True)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record()
+        e2e_isect = 0
+        for k in range(a.steps):
+            v = view_of(k)
+            dev_t.copy_(host_t[v], non_blocking=True)
+            s = stp.run_view(cams[v], dev_t)
+            loss_h.copy_(stp._last_loss, non_blocking=True)
+            e2e_isect += s.n_isect
+        f1.record()
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        if dist:
+            t = torch.tensor([ems], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+            t = torch.tensor([e2e_isect], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t)
+            e2e_isect = float(t.item())
+        TW, TH = (W + 15) // 16, (H + 15) // 16
+        e2e = {"value": e2e_isect / (ems / 1e3), "unit": UNIT, "ms_per_step": ems / a.steps,
+               "h2d_bytes_per_step": 3 * W * H * 4,
+               "d2h_bytes_per_step": (TW + 1) * (TH + 1) * 8 + 4 + 8}
+
+    # ---- CPU baseline (rank 0, one GPU) ---------------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu:
+        tg_host = {}
+
+        def target_fn(v):
+            if v not in tg_host:
+                tg_host[v] = targets[v].cpu().numpy().astype(np.float64)
+            return tg_host[v]
+
+        osm = OracleSample(scene, cams, target_fn, n_tiles=a.cpu_tiles)
+        r = osm.step(0)
+        from oracle import oracle as O
+        cpu = {"value": r["I_total"] / r["est_step_s"], "unit": UNIT,
+               "cores": O.num_threads(), "kind": "oracle", "sample": osm.describe(),
+               "est_step_s": round(r["est_step_s"], 2),
+               "parts_s": {k: round(x, 2) for k, x in r["parts"].items()}}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded generator; targets = renders of a jittered copy)",
+            "config": {"workload": workload_name(a), "gaussians": a.gaussians, "sh_degree": 3,
+                       "width": W, "height": H, "views": nv, "leaf_budget_mib": a.budget_mib,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (4.25 GB of params + Adam moments "
+                             "stream every step)"},
+            "peak_ws_gib": peak_ws / 2 ** 30,
+            "isect_per_view": isect / a.steps,
+            "candidates_per_view": statistics.mean(s.n_cand for s in stats),
+            "leaves_per_view": statistics.mean(s.n_leaves for s in stats),
+            "stage_ms_per_step": {s: round(per_step[s], 3) for s in STAGES},
+            "stage_launches_per_step": {s: stage_n[s] / n_steps for s in STAGES},
+            "work": {"fwd_pairs_evaluated": cnt[0], "fwd_pairs_composited": cnt[1],
+                     "bwd_pairs_evaluated": cnt[2], "bwd_pairs_differentiated": cnt[3]},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clk,
+        }
+        print(json.dumps(out))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(a, rank, world):
+    """The oracle, as it stands, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from gaussian_splatting_differentiable_dgs_b200 import synth
+    scene, cams = synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
+                                      n_views=a.views)
+    jit = synth.jittered(scene, seed=1)
+    cache = {}
+
+    def target_fn(v):
+        # the oracle's own render of the jittered copy, on the sampled tiles
+        # only matters for the L1 sign; a seeded image stands in for it
+        if v not in cache:
+            cache[v] = synth.random_image(a.width, a.height, 100 + v).astype(np.float64)
+        return cache[v]
+
+    del jit
+    osm = OracleSample(scene, cams, target_fn, n_tiles=a.cpu_tiles)
+    for k in range(a.warmup):
+        osm.step(k % len(cams))
+    t0 = time.perf_counter()
+    ests, isects = [], []
+    for k in range(a.steps):
+        r = osm.step(k % len(cams))
+        ests.append(r["est_step_s"])
+        isects.append(r["I_total"])
+    wall = time.perf_counter() - t0
+    from oracle import oracle as O
+    value = sum(isects) / sum(ests)
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(ests) / a.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": workload_name(a)},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.num_threads(),
+                            "kind": "oracle", "sample": osm.describe()},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0},
+           "wall_s": wall}
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

@@ -61,12 +61,12 @@ class gs_pixels(C.Structure):
                 ("T_final", C.c_void_p), ("last", C.c_void_p), ("dL_dimg", C.c_void_p),
                 ("target", C.c_void_p), ("tx0", C.c_int32), ("ty0", C.c_int32),
                 ("tpitch", C.c_int64), ("tplane", C.c_int64), ("loss_tiles", C.c_void_p),
-                ("norm", C.c_double)]
+                ("norm", C.c_double), ("counters", C.c_void_p)]
 
 
 def pixels(x0, y0, w, h, img, T_final, last, dL, target=None, target_origin=(0, 0),
            target_pitch=None, target_plane=None, loss_tiles=None, norm=0.0, pitch=None,
-           plane=None) -> gs_pixels:
+           plane=None, counters=None) -> gs_pixels:
     """Descriptor of Leaf-local pixel buffers (pitch w, plane w*h by default)."""
     pitch = w if pitch is None else pitch
     plane = pitch * h if plane is None else plane
@@ -79,6 +79,7 @@ def pixels(x0, y0, w, h, img, T_final, last, dL, target=None, target_origin=(0, 
     p.tplane = target_plane if target_plane is not None else plane
     p.loss_tiles = ptr(loss_tiles)
     p.norm = norm
+    p.counters = ptr(counters)
     return p
 
 
@@ -88,8 +89,8 @@ class gs_load_model(C.Structure):
 
 
 class gs_adam_args(C.Structure):
-    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float),
-                ("eps", C.c_float), ("step", C.c_int32), ("reserved", C.c_int32)]
+    _fields_ = [("lr", C.c_double), ("beta1", C.c_double), ("beta2", C.c_double),
+                ("eps", C.c_double), ("step", C.c_int32), ("reserved", C.c_int32)]
 
 
 SYMBOLS = [

@@ -26,14 +26,14 @@ struct BwdCam {
 };
 
 struct AdamK {
-  float lr, b1, b2, eps, bc1, bc2;
+  float lr, b1, b2, omb1, omb2, eps, bc1, bc2;
 };
 
 __device__ __forceinline__ void adam_update(float* __restrict__ p, float* __restrict__ m,
                                             float* __restrict__ v, int64_t idx, float g,
                                             const AdamK& a) {
-  const float mm = fmaf(a.b1, m[idx], (1.0f - a.b1) * g);
-  const float vv = fmaf(a.b2, v[idx], (1.0f - a.b2) * g * g);
+  const float mm = fmaf(a.b1, m[idx], a.omb1 * g);
+  const float vv = fmaf(a.b2, v[idx], a.omb2 * g * g);
   m[idx] = mm;
   v[idx] = vv;
   const float mh = mm / a.bc1;
@@ -290,12 +290,14 @@ bool make_adam(const gs_adam_args* args, AdamK* a) {
   if (!args || args->step < 1 || !(args->lr >= 0) || !(args->beta1 >= 0 && args->beta1 < 1) ||
       !(args->beta2 >= 0 && args->beta2 < 1) || !(args->eps > 0))
     return false;
-  a->lr = args->lr;
-  a->b1 = args->beta1;
-  a->b2 = args->beta2;
-  a->eps = args->eps;
-  a->bc1 = (float)(1.0 - pow((double)args->beta1, (double)args->step));
-  a->bc2 = (float)(1.0 - pow((double)args->beta2, (double)args->step));
+  a->lr = (float)args->lr;
+  a->b1 = (float)args->beta1;
+  a->b2 = (float)args->beta2;
+  a->omb1 = (float)(1.0 - args->beta1);
+  a->omb2 = (float)(1.0 - args->beta2);
+  a->eps = (float)args->eps;
+  a->bc1 = (float)(1.0 - pow(args->beta1, (double)args->step));
+  a->bc2 = (float)(1.0 - pow(args->beta2, (double)args->step));
   return true;
 }
 

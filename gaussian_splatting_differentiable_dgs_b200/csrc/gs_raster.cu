@@ -94,6 +94,7 @@ struct PixArgs {
   int64_t tpitch, tplane;
   float* loss_tiles;
   float norm;
+  unsigned long long* counters;
 };
 
 template <int PPT>
@@ -105,7 +106,7 @@ struct TileGeom {
 // ---------------------------------------------------------------------------
 // forward
 // ---------------------------------------------------------------------------
-template <int PPT>
+template <int PPT, bool COUNT>
 __global__ void __launch_bounds__(256 / PPT)
 k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
@@ -124,6 +125,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
   int lastp[PPT];
   bool done[PPT], inside[PPT];
+  unsigned n_vis = 0, n_kept = 0;
 #pragma unroll
   for (int k = 0; k < PPT; ++k) {
     const int ly = ly0 + k * ROWS;
@@ -157,12 +159,14 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       for (int k = 0; k < PPT; ++k) {
         if (done[k]) continue;
         const Eval ev = eval_alpha(A.x, A.y, A.z, A.w, B.x, B.y, fpx, fpy[k]);
+        if (COUNT) ++n_vis;
         if (ev.alpha < kAlphaMin) continue;
         const float Tn = __fmul_rn(T[k], __fsub_rn(1.0f, ev.alpha));
         if (Tn < kTMin) {
           done[k] = true;
           continue;
         }
+        if (COUNT) ++n_kept;
         const float wgt = ev.alpha * T[k];
         Cr[k] = fmaf(B.z, wgt, Cr[k]);
         Cg[k] = fmaf(B.w, wgt, Cg[k]);
@@ -171,6 +175,10 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         lastp[k] = pos0 + j + 1;
       }
     }
+  }
+  if (COUNT) {
+    atomicAdd(&px.counters[0], (unsigned long long)n_vis);
+    atomicAdd(&px.counters[1], (unsigned long long)n_kept);
   }
   // epilogue: outputs and the fused L1 terms
   float lsum = 0.0f;
@@ -305,7 +313,7 @@ __device__ __forceinline__ float warp_reduce_scatter9(const float (&v)[9], int l
   return d;
 }
 
-template <int PPT>
+template <int PPT, bool COUNT>
 __global__ void __launch_bounds__(256 / PPT)
 k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, PixArgs px,
@@ -353,6 +361,7 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   atomicMax(&s_maxlast, mylast);
   __syncthreads();
   const int tile_last = s_maxlast;
+  unsigned n_vis = 0, n_kept = 0;
 
   for (int bend = tile_last; bend > 0; bend -= NT) {
     const int bstart = max(0, bend - NT);
@@ -378,7 +387,9 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       for (int k = 0; k < PPT; ++k) {
         if (pos >= lastp[k]) continue;
         const Eval ev = eval_alpha(A.x, A.y, A.z, A.w, B.x, B.y, fpx, fpy[k]);
+        if (COUNT) ++n_vis;
         if (ev.alpha < kAlphaMin) continue;
+        if (COUNT) ++n_kept;
         any = true;
         const float inv = __frcp_rn(1.0f - ev.alpha);
         const float Tb = T[k] * inv;          // transmittance before this entry
@@ -426,6 +437,10 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     }
     __syncthreads();
   }
+  if (COUNT) {
+    atomicAdd(&px.counters[0], (unsigned long long)n_vis);
+    atomicAdd(&px.counters[1], (unsigned long long)n_kept);
+  }
 }
 
 PixArgs to_args(const gs_pixels* p) {
@@ -436,6 +451,7 @@ PixArgs to_args(const gs_pixels* p) {
   a.target = p->target; a.tx0 = p->tx0; a.ty0 = p->ty0; a.tpitch = p->tpitch;
   a.tplane = p->tplane; a.loss_tiles = p->loss_tiles;
   a.norm = (float)p->norm;
+  a.counters = p->counters;
   return a;
 }
 
@@ -483,17 +499,16 @@ extern "C" gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals, con
   const int TW = (int)tiles_x(cam->width);
   cudaStream_t s = to_stream(stream);
   const float4* rec = reinterpret_cast<const float4*>(proj->rec);
+  const unsigned nb = (unsigned)ntiles;
+  const int W = cam->width, H = cam->height;
+  const bool cnt = px->counters != nullptr;
+#define GS_FWD(P, C) k_raster_fwd<P, C><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, TW, a, dev_status)
   switch (pick_ppt(flags, 2)) {
-    case 1:
-      k_raster_fwd<1><<<(unsigned)ntiles, 256, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, TW, a, dev_status);
-      break;
-    case 2:
-      k_raster_fwd<2><<<(unsigned)ntiles, 128, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, TW, a, dev_status);
-      break;
-    default:
-      k_raster_fwd<4><<<(unsigned)ntiles, 64, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, TW, a, dev_status);
-      break;
+    case 1: if (cnt) GS_FWD(1, true); else GS_FWD(1, false); break;
+    case 2: if (cnt) GS_FWD(2, true); else GS_FWD(2, false); break;
+    default: if (cnt) GS_FWD(4, true); else GS_FWD(4, false); break;
   }
+#undef GS_FWD
   GS_LAUNCH_CHECK();
   return GS_OK;
 }
@@ -529,17 +544,16 @@ extern "C" gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals, con
   const PixArgs a = to_args(px);
   cudaStream_t s = to_stream(stream);
   const float4* rec = reinterpret_cast<const float4*>(proj->rec);
+  const unsigned nb = (unsigned)ntiles;
+  const int W = cam->width, H = cam->height;
+  const bool cnt = px->counters != nullptr;
+#define GS_BWD(P, C) k_raster_bwd<P, C><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, a, g2d, dev_status)
   switch (pick_ppt(flags, 2)) {
-    case 1:
-      k_raster_bwd<1><<<(unsigned)ntiles, 256, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, a, g2d, dev_status);
-      break;
-    case 2:
-      k_raster_bwd<2><<<(unsigned)ntiles, 128, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, a, g2d, dev_status);
-      break;
-    default:
-      k_raster_bwd<4><<<(unsigned)ntiles, 64, 0, s>>>(rec, vals, ranges, leaf, cam->width, cam->height, a, g2d, dev_status);
-      break;
+    case 1: if (cnt) GS_BWD(1, true); else GS_BWD(1, false); break;
+    case 2: if (cnt) GS_BWD(2, true); else GS_BWD(2, false); break;
+    default: if (cnt) GS_BWD(4, true); else GS_BWD(4, false); break;
   }
+#undef GS_BWD
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

@@ -23,6 +23,9 @@ from . import binding as B
 
 DEFAULT_BUDGET = 384 << 20
 
+STAGES = ("project", "sort_depth", "bin", "sort_tiles", "raster_fwd", "raster_bwd",
+          "project_bwd")
+
 
 def _carve(arena: torch.Tensor, sizes):
     """Split a uint8 arena into 256-byte aligned byte views."""
@@ -43,7 +46,6 @@ def _carved_bytes(sizes):
 
 @dataclasses.dataclass
 class ViewStats:
-    loss: float
     n_cand: int
     n_isect: int
     n_leaves: int
@@ -53,13 +55,13 @@ class ViewStats:
     over_budget: np.ndarray
     peak_ws_bytes: int
     arena_bytes: int
+    launches: int
 
 
 class GaussianModel:
     """Parameters and Adam moments, planar [P][n_pad] fp32 on the device."""
 
-    def __init__(self, params: np.ndarray | torch.Tensor, n: int, sh_degree: int,
-                 device="cuda"):
+    def __init__(self, params, n: int, sh_degree: int, device="cuda"):
         p = torch.as_tensor(params, dtype=torch.float32)
         self.params = p.to(device).contiguous()
         self.m = torch.zeros_like(self.params)
@@ -80,10 +82,29 @@ class GaussianModel:
         return B.gs_model(self.n, self.n_pad, self.sh_degree, 0, self.params.data_ptr())
 
 
+class _Timer:
+    def __init__(self, timing):
+        self.timing = timing
+
+    def tic(self, name):
+        if self.timing is None:
+            return None
+        e0 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        return name, e0
+
+    def toc(self, tk):
+        if tk is None:
+            return
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record()
+        self.timing.setdefault(tk[0], []).append((tk[1], e1))
+
+
 class Stepper:
     """Runs the per-view step.  `hooks` (optional) is an object whose methods
-    `on_project(ctx)`, `on_leaf(ctx)`, `on_bwd(ctx)` see intermediate
-    buffers (used by the parity tests)."""
+    `on_project(ctx)`, `on_leaf(ctx, leaf_ctx)`, `on_bwd(ctx)` see
+    intermediate buffers (used by the parity tests)."""
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
@@ -95,9 +116,8 @@ class Stepper:
         self.fuse_adam = fuse_adam
         self.device = torch.device(device)
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
-        self.launches = 0
+        self._last_loss = None
 
-    # ------------------------------------------------------------------
     def check(self):
         st = B.gs_check(self.dev_status)
         if st < 0:
@@ -106,13 +126,25 @@ class Stepper:
     def adam_args(self, step):
         return B.gs_adam_args(self.lr, self.betas[0], self.betas[1], self.eps, step, 0)
 
+    def last_loss(self) -> float:
+        return float(self._last_loss.item())
+
     # ------------------------------------------------------------------
-    def run_view(self, cam, target, leaves=None, hooks=None, update=True) -> ViewStats:
-        """cam: synth.Camera; target: [3][H][W] fp32, either a device tensor
-        (the whole view resident) or a pinned host tensor (each Leaf's crop
-        is uploaded before its forward).  `leaves` overrides the planner
-        (list of tile rects)."""
+    def run_view(self, cam, target, leaves=None, hooks=None, update=True, backward=True,
+                 timing=None, counters=None) -> ViewStats:
+        """One view.  target: [3][H][W] fp32, a device tensor (the whole view
+        resident, read in place) or a pinned host tensor (each Leaf's crop is
+        uploaded before its forward); None renders only (no loss, backward or
+        update).  leaves: tile rects overriding the planner.  timing: dict
+        that receives (start, end) CUDA event pairs per stage (STAGES).
+        counters: device int64[4] work counters ([0:2] forward, [2:4]
+        backward)."""
         dev = self.device
+        if target is None:
+            backward = update = False
+        clk = _Timer(timing)
+        cnt_f = counters[0:2] if counters is not None else None
+        cnt_b = counters[2:4] if counters is not None else None
         m = self.model
         W, H = cam.width, cam.height
         TW, TH = (W + 15) // 16, (H + 15) // 16
@@ -138,8 +170,10 @@ class Stepper:
                          rec.data_ptr(), rect.data_ptr(), dkey.data_ptr())
         sat = torch.empty((TH + 1) * (TW + 1), dtype=torch.int64, device=dev)
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
+        tk = clk.tic("project")
         B.gs_project(mod, camS, proj, sat, ws, st)
-        launches += 4
+        clk.toc(tk)
+        launches += 3 if n > 0 else 2
         del ws
         sat_h = torch.empty(sat.shape, dtype=torch.int64, pin_memory=True)
         nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
@@ -158,7 +192,9 @@ class Stepper:
         if C > 0:
             k32 = torch.empty(C, dtype=torch.int32, device=dev)
             ws = torch.empty(B.gs_sort_workspace_size(C, 4, 0, 32), dtype=torch.uint8, device=dev)
+            tk = clk.tic("sort_depth")
             B.gs_sort_keys32(dkey, k32, order, C, 0, 32, B.GS_SORT_IOTA, ws, st)
+            clk.toc(tk)
             launches += 1 + 4
             del ws, k32
         ctx["depth_order"] = order
@@ -174,12 +210,11 @@ class Stepper:
             lb = np.zeros(len(lv), np.int64)
             ov = np.zeros(len(lv), bool)
 
-        # ---- per-Leaf raster: forward + L1 + backward into compact g2d ----------
+        # ---- per-Leaf raster: forward + L1 + backward into compact g2d ------
         g2d = torch.zeros(max(C, 1) * 12, dtype=torch.float32, device=dev)
         loss_tiles = torch.zeros(T, dtype=torch.float32, device=dev)
         bin_ws = torch.empty(max(B.gs_bin_workspace_size(C), 256), dtype=torch.uint8, device=dev)
         resident_target = target is not None and target.is_cuda
-        tgt = target if resident_target else None
 
         def leaf_sizes(L, I):
             x0, y0, x1, y1 = (int(v) for v in L)
@@ -189,7 +224,7 @@ class Stepper:
             nt = (x1 - x0) * (y1 - y0)
             sizes = [8 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 8, 32, 32 + tile_bits),
                      12 * npx, 4 * npx, 4 * npx, 12 * npx]
-            if not resident_target:
+            if target is not None and not resident_target:
                 sizes.append(12 * npx)
             return sizes, (16 * x0, 16 * y0, pw, ph)
 
@@ -197,7 +232,7 @@ class Stepper:
                           default=0)
         arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
         norm = 1.0 / (3.0 * W * H)
-        for k, (L, I) in enumerate(zip(lv, li)):
+        for L, I in zip(lv, li):
             I = int(I)
             sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
             bufs, _ = _carve(arena, sizes)
@@ -211,34 +246,50 @@ class Stepper:
             dL = bufs[7].view(torch.float32)
             if resident_target:
                 # the whole view's target is read in place with its own pitch
-                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=tgt,
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
                               target_origin=(0, 0), target_pitch=W, target_plane=W * H,
-                              loss_tiles=loss_tiles, norm=norm)
-            else:
+                              loss_tiles=loss_tiles, norm=norm, counters=cnt_f)
+            elif target is not None:
                 # bounded supply: the Leaf's crop of a host target is uploaded
                 crop = bufs[8].view(torch.float32).view(3, ph, pw)
                 crop.copy_(target[:, py0:py0 + ph, px0:px0 + pw], non_blocking=True)
                 px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
-                              target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm)
+                              target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm,
+                              counters=cnt_f)
+            else:
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
+            tk = clk.tic("bin")
             B.gs_bin_tiles(proj, C, order, L, TW, TH, sat, I, keys, vals, max(I, 1), ranges,
                            bin_ws, st)
-            launches += 2
+            clk.toc(tk)
+            launches += 2 if (C > 0 and I > 0) else 1
             if I > 0:
+                tk = clk.tic("sort_tiles")
                 B.gs_sort_keys(keys, vals, I, 32, 32 + tile_bits, sort_ws, st)
+                clk.toc(tk)
                 launches += 1 + 2 * ((tile_bits + 15) // 16)
+            tk = clk.tic("raster_fwd")
             B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
+            clk.toc(tk)
             launches += 1
             if hooks is not None and hasattr(hooks, "on_leaf"):
                 hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
                                         ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
                                         n_isect=I, px_rect=(px0, py0, pw, ph)))
-            B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
-            launches += 1
+            if backward:
+                if cnt_b is not None:
+                    px.counters = cnt_b.data_ptr()
+                tk = clk.tic("raster_bwd")
+                B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
+                clk.toc(tk)
+                launches += 1
         del arena, bin_ws  # raster buffers released before projection backward
 
         loss_d = torch.zeros(1, dtype=torch.float64, device=dev)
-        B.gs_loss_total(loss_tiles, T, loss_d)
-        launches += 1
+        if target is not None:
+            B.gs_loss_total(loss_tiles, T, loss_d)
+            launches += 1
+        self._last_loss = loss_d
         ctx["g2d"] = g2d
         if hooks is not None and hasattr(hooks, "on_bwd"):
             hooks.on_bwd(ctx)
@@ -247,8 +298,10 @@ class Stepper:
         if update:
             m.step += 1
             if self.fuse_adam:
+                tk = clk.tic("project_bwd")
                 B.gs_project_bwd(mod, camS, proj, C, g2d, adam_m=m.m, adam_v=m.v,
                                  fused=self.adam_args(m.step), dev_status=st)
+                clk.toc(tk)
                 launches += 1
             else:
                 g3d = torch.empty(m.P * max(C, 1), dtype=torch.float32, device=dev)
@@ -258,14 +311,21 @@ class Stepper:
                           self.adam_args(m.step))
                 launches += 2
                 del g3d
-        self.launches = launches
         peak = torch.cuda.max_memory_allocated(dev) - base_alloc
         if resident_target:
             peak += target.numel() * target.element_size()
-        self._last_loss = loss_d
-        return ViewStats(loss=float("nan"), n_cand=C, n_isect=int(li.sum()),
-                         n_leaves=len(lv), leaves=lv, leaf_isect=li, leaf_bytes=lb,
-                         over_budget=ov, peak_ws_bytes=int(peak), arena_bytes=int(arena_bytes))
+        return ViewStats(n_cand=C, n_isect=int(li.sum()), n_leaves=len(lv), leaves=lv,
+                         leaf_isect=li, leaf_bytes=lb, over_budget=ov, peak_ws_bytes=int(peak),
+                         arena_bytes=int(arena_bytes), launches=launches)
 
-    def last_loss(self) -> float:
-        return float(self._last_loss.item())
+    def render(self, cam) -> torch.Tensor:
+        """Forward-only render of the whole view: [3][H][W] fp32 on the device."""
+        img = torch.zeros((3, cam.height, cam.width), dtype=torch.float32, device=self.device)
+
+        class _Copy:
+            def on_leaf(self, ctx, lc):
+                x0, y0, w, h = lc["px_rect"]
+                img[:, y0:y0 + h, x0:x0 + w] = lc["img"][:3 * w * h].view(3, h, w)
+
+        self.run_view(cam, None, hooks=_Copy())
+        return img

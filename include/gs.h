@@ -144,6 +144,10 @@ typedef struct gs_pixels {
   int64_t tplane;
   float* loss_tiles;      /* per global tile: norm * sum |r - t|, or NULL */
   double norm;            /* 1 / (3 W H): whole-view normaliser */
+  /* optional work counters (NULL = off): [0] += pixel-Gaussian pairs
+   * evaluated, [1] += pairs composited (forward) / differentiated
+   * (backward).  Used to account the work of a launch. */
+  unsigned long long* counters;
 } gs_pixels;
 
 /* Byte cost model of a Leaf (the buffers this library needs per unit). */
@@ -155,8 +159,11 @@ typedef struct gs_load_model {
   int64_t align;
 } gs_load_model;
 
+/* Hyper-parameters in fp64; the kernels apply the fp32 roundings of lr,
+ * beta1, beta2, (1 - beta1), (1 - beta2), eps and the bias corrections
+ * 1 - beta^t, each computed in fp64 on the host. */
 typedef struct gs_adam_args {
-  float lr, beta1, beta2, eps;
+  double lr, beta1, beta2, eps;
   int32_t step;  /* 1 on the first update */
   int32_t reserved;
 } gs_adam_args;
