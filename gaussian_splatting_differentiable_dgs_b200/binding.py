@@ -96,7 +96,7 @@ class gs_adam_args(C.Structure):
 SYMBOLS = [
     "gs_version", "gs_status_string", "gs_check",
     "gs_project_workspace_size", "gs_project",
-    "gs_sort_workspace_size", "gs_sort_keys", "gs_sort_keys32",
+    "gs_sort_workspace_size", "gs_sort_keys", "gs_sort_keys32", "gs_sort_keys32_noalloc",
     "gs_leaf_load_model", "gs_leaf_partition",
     "gs_bin_workspace_size", "gs_bin_tiles",
     "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
@@ -119,6 +119,7 @@ def _load():
         "gs_sort_workspace_size": (sz, [i64, i32, i32, i32]),
         "gs_sort_keys": (i32, [p, p, i64, i32, i32, p, sz, p, p]),
         "gs_sort_keys32": (i32, [p, p, p, i64, i32, i32, u32, p, sz, p, p]),
+        "gs_sort_keys32_noalloc": (i32, [p, p, p, i64, i32, i32, u32, p, p]),
         "gs_leaf_load_model": (i32, [i32, P(gs_load_model)]),
         "gs_leaf_partition": (i32, [p, i32, i32, i32, i32, P(gs_load_model), i64, p, p, p, p,
                                     i32, P(i32)]),
@@ -225,6 +226,18 @@ def gs_sort_keys32(keys_in, keys, vals, n, begin_bit, end_bit, flags, ws, dev_st
                                                    begin_bit, end_bit, flags, ptr(ws),
                                                    ws.numel() * ws.element_size(),
                                                    ptr(dev_status), _stream(stream)))
+
+
+SORT_NOALLOC_MAX_N = 1 << 18
+
+
+def gs_sort_keys32_noalloc(keys_in, keys, vals, n, begin_bit, end_bit, flags, dev_status,
+                           stream=None):
+    """gs_sort_keys32 without a workspace (library-held scratch, n <= 2**18).
+    Calls must not overlap on the GPU: they share that scratch."""
+    return _ok("gs_sort_keys32_noalloc", _L.gs_sort_keys32_noalloc(
+        ptr(keys_in), ptr(keys), ptr(vals), n, begin_bit, end_bit, flags, ptr(dev_status),
+        _stream(stream)))
 
 
 def gs_leaf_load_model(tile_bits) -> gs_load_model:

@@ -10,6 +10,8 @@
 // and per Leaf a sort of the duplicated (tile << 32 | depth) keys on the
 // tile bits only.  Because the keys are emitted in depth order, the stable
 // tile-bit sort yields the same order as a full 64-bit sort.
+#include <mutex>
+
 #include "gs_internal.cuh"
 
 namespace gs {
@@ -317,4 +319,62 @@ extern "C" gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys, int
   return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0,
                              (flags & GS_SORT_TEST_STALL) != 0, n, begin_bit, end_bit, ws,
                              ws_bytes, dev_status, to_stream(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of gs_sort_keys32.
+//
+// Some callers cannot allocate device memory at the moment they need a sort:
+// for example a plugin inside a host application whose allocator has already
+// reserved the whole device, or a latency-critical loop where an allocation
+// (which may synchronise the device) is not acceptable.  For them the scratch
+// of the sort lives in this file-scope device array instead of a caller
+// workspace.  Every GPU that loads the library holds the array until exit.
+// ---------------------------------------------------------------------------
+namespace gs {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)3 << 20;  // 3 MiB
+static __device__ __align__(256) unsigned char g_sort_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_sort_scratch for the current device, looked up once
+// per device (the host-side name of the array is not a device address).
+gs_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GS_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_sort_scratch) != cudaSuccess || !p) return GS_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return GS_OK;
+}
+
+}  // namespace
+}  // namespace gs
+
+extern "C" gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* keys,
+                                            int32_t* vals, int64_t n, int32_t begin_bit,
+                                            int32_t end_bit, uint32_t flags, int32_t* dev_status,
+                                            gs_stream stream) {
+  if (flags & ~(GS_SORT_IOTA | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
+  if (n < 0) return GS_ERR_ARG;
+  if (n > GS_SORT_NOALLOC_MAX_N) return GS_ERR_CAPACITY;
+  if (n == 0) return GS_OK;
+  void* scratch = nullptr;
+  const gs_status st = scratch_address(&scratch);
+  if (st != GS_OK) return st;
+  // the whole plan must fit the array (it does for every n <= the maximum)
+  if (gs_sort_workspace_size(n, 4, begin_bit, end_bit) > kNoAllocScratchBytes)
+    return GS_ERR_CAPACITY;
+  return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0,
+                             (flags & GS_SORT_TEST_STALL) != 0, n, begin_bit, end_bit, scratch,
+                             kNoAllocScratchBytes, dev_status, to_stream(stream));
 }

@@ -218,6 +218,26 @@ gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys,
                          size_t ws_bytes, int32_t* dev_status,
                          gs_stream stream);
 
+/* Allocation-free variant of gs_sort_keys32 (no counterpart on the pages;
+ * an addition of this library).  For callers that cannot allocate device
+ * memory when they need the sort, e.g. code inside a host application whose
+ * allocator owns the whole device, or a latency-critical loop that must not
+ * risk an allocation's implicit device synchronisation.  Same arguments and
+ * result as gs_sort_keys32 without the workspace: the scratch is a 3 MiB
+ * array inside the library that every GPU loading the library holds until
+ * the process exits.  n > GS_SORT_NOALLOC_MAX_N returns GS_ERR_CAPACITY and
+ * launches nothing.  The first call on a device looks up the array's device
+ * address (make that first call before any stream capture).  It never
+ * calls cudaMalloc or cudaFree.  All calls share the one array: calls that
+ * overlap on the GPU (e.g. on two streams) race and give wrong results;
+ * serialise them.  The parts of the array that must start at zero are
+ * cleared by every call, so a call does not depend on the previous one. */
+#define GS_SORT_NOALLOC_MAX_N (1 << 18)
+gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* keys,
+                                 int32_t* vals, int64_t n, int32_t begin_bit,
+                                 int32_t end_bit, uint32_t flags,
+                                 int32_t* dev_status, gs_stream stream);
+
 /* ---- 3. Leaf partition (host) --------------------------------------------
  * Recursive split of the tile grid: a rect whose estimated load
  *   align(I * b_isect) + align(pixels * b_px) + align(tiles * b_tile) + fixed
