@@ -98,6 +98,7 @@ SYMBOLS = [
     "gs_project_workspace_size", "gs_project",
     "gs_sort_workspace_size", "gs_sort_keys", "gs_sort_keys32", "gs_sort_keys32_noalloc",
     "gs_leaf_load_model", "gs_leaf_partition",
+    "gs_depth_order_workspace_size", "gs_depth_order",
     "gs_bin_workspace_size", "gs_bin_tiles",
     "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
     "gs_project_bwd", "gs_adam",
@@ -124,7 +125,9 @@ def _load():
         "gs_leaf_partition": (i32, [p, i32, i32, i32, i32, P(gs_load_model), i64, p, p, p, p,
                                     i32, P(i32)]),
         "gs_bin_workspace_size": (sz, [i64]),
-        "gs_bin_tiles": (i32, [P(gs_proj), i64, p, gs_rect, i32, i32, p, i64, p, p, i64, p,
+        "gs_depth_order_workspace_size": (sz, [i64]),
+        "gs_depth_order": (i32, [P(gs_proj), i64, p, p, p, sz, p, p]),
+        "gs_bin_tiles": (i32, [P(gs_proj), i64, p, p, gs_rect, i32, i32, p, i64, p, p, p, i64, p,
                                P(i64), p, sz, p, p]),
         "gs_raster_fwd": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), u32, p, p]),
         "gs_loss_l1": (i32, [P(gs_pixels), gs_rect, P(gs_camera), p]),
@@ -269,18 +272,37 @@ def gs_leaf_partition(sat_host, TW, TH, width, height, lm: gs_load_model, budget
         return st, leaves[:k].copy(), li[:k].copy(), lb[:k].copy(), ov[:k].astype(bool)
 
 
+def gs_depth_order_workspace_size(n_cand) -> int:
+    return _L.gs_depth_order_workspace_size(n_cand)
+
+
+def gs_depth_order(proj: gs_proj, n_cand, depth_order, depth_rect, ws, dev_status, stream=None):
+    return _ok("gs_depth_order", _L.gs_depth_order(C.byref(proj), n_cand, ptr(depth_order),
+                                                   ptr(depth_rect), ptr(ws),
+                                                   ws.numel() * ws.element_size(),
+                                                   ptr(dev_status), _stream(stream)))
+
+
 def gs_bin_workspace_size(n_cand) -> int:
     return _L.gs_bin_workspace_size(n_cand)
 
 
-def gs_bin_tiles(proj: gs_proj, n_cand, depth_order, leaf, TW, TH, tile_sat, n_isect, keys,
-                 vals, capacity, ranges, ws, dev_status, stream=None):
+def gs_bin_tiles(proj: gs_proj, n_cand, depth_order, depth_rect, leaf, TW, TH, tile_sat, n_isect,
+                 tile_keys, vals, capacity, ranges, ws, dev_status, keys64=None, stream=None):
     needed = C.c_int64(0)
-    st = _L.gs_bin_tiles(C.byref(proj), n_cand, ptr(depth_order), gs_rect(*[int(v) for v in leaf]),
-                         TW, TH, ptr(tile_sat), n_isect, ptr(keys), ptr(vals), capacity,
-                         ptr(ranges), C.byref(needed), ptr(ws), ws.numel() * ws.element_size(),
+    st = _L.gs_bin_tiles(C.byref(proj), n_cand, ptr(depth_order), ptr(depth_rect),
+                         gs_rect(*[int(v) for v in leaf]), TW, TH, ptr(tile_sat), n_isect,
+                         ptr(tile_keys), ptr(vals), ptr(keys64), capacity, ptr(ranges),
+                         C.byref(needed), ptr(ws), ws.numel() * ws.element_size(),
                          ptr(dev_status), _stream(stream))
     return _ok("gs_bin_tiles", st, needed.value if st == GS_ERR_CAPACITY else None)
+
+
+def local_tile_bits(leaf) -> int:
+    """Bits of a Leaf's local tile index (the sort range for its entries)."""
+    x0, y0, x1, y1 = (int(v) for v in leaf)
+    nt = (x1 - x0) * (y1 - y0)
+    return (nt - 1).bit_length() if nt > 1 else 0
 
 
 def gs_raster_fwd(proj: gs_proj, vals, ranges, leaf, cam: gs_camera, px: gs_pixels, dev_status,

@@ -43,7 +43,7 @@ __device__ __forceinline__ void adam_update(float* __restrict__ p, float* __rest
 
 // Gradients of one candidate.  `emit(plane, g)` receives every parameter's
 // gradient exactly once, SH planes first, then planes 10 .. 0.
-template <class Emit>
+template <bool WITH_SH, class Emit>
 __device__ __forceinline__ void candidate_grad(const float* __restrict__ P, int64_t n_pad, int64_t i,
                                                int D, const BwdCam& c, const float* __restrict__ g2,
                                                const float4 rgb_rec, Emit&& emit) {
@@ -161,6 +161,7 @@ __device__ __forceinline__ void candidate_grad(const float* __restrict__ P, int6
   const double o = 1.0 / (1.0 + exp(-(double)P[10 * n_pad + i]));
   const double dlogit = dO * o * (1.0 - o);
 
+  if constexpr (WITH_SH) {
   // SH coefficients and the view direction
   double ex = mx - c.campos[0], ey = my - c.campos[1], ez = mz - c.campos[2];
   const double en = sqrt(ex * ex + ey * ey + ez * ez);
@@ -210,20 +211,21 @@ __device__ __forceinline__ void candidate_grad(const float* __restrict__ P, int6
         dd[1] += coef * dY[k][1];
         dd[2] += coef * dY[k][2];
       }
-      emit(plane, (float)g);
+      emit(plane, g);
     }
   }
   const double ddot = dd[0] * ex + dd[1] * ey + dd[2] * ez;
   dmean[0] += (dd[0] - ex * ddot) / en;
   dmean[1] += (dd[1] - ey * ddot) / en;
   dmean[2] += (dd[2] - ez * ddot) / en;
-  emit(10, (float)dlogit);
+  }
+  emit(10, dlogit);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) emit(6 + k, (float)dq[k]);
+  for (int k = 0; k < 4; ++k) emit(6 + k, dq[k]);
 #pragma unroll
-  for (int k = 0; k < 3; ++k) emit(3 + k, (float)dls[k]);
+  for (int k = 0; k < 3; ++k) emit(3 + k, dls[k]);
 #pragma unroll
-  for (int k = 0; k < 3; ++k) emit(k, (float)dmean[k]);
+  for (int k = 0; k < 3; ++k) emit(k, dmean[k]);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -233,27 +235,8 @@ k_project_bwd(const float* __restrict__ P, int64_t n_pad, int D, BwdCam cam, int
   const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (j >= n_cand) return;
   const int64_t i = cand_idx[j];
-  candidate_grad(P, n_pad, i, D, cam, g2d + 12 * j, rec[3 * j + 2],
-                 [&](int plane, float g) { g3d[(int64_t)plane * stride + j] = g; });
-}
-
-__global__ void __launch_bounds__(kThreads)
-k_project_bwd_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
-                   int64_t n, int64_t n_pad, int D, int nP, BwdCam cam,
-                   const int32_t* __restrict__ slot_map, const float4* __restrict__ rec,
-                   const float* __restrict__ g2d, AdamK a) {
-  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (i >= n) return;
-  const int32_t s = slot_map[i];
-  if (s >= 0) {
-    // gradients of the candidate; each plane is updated as soon as its
-    // gradient is known (the SH planes before the mean, which needs the
-    // view-direction term)
-    candidate_grad(P, n_pad, i, D, cam, g2d + 12 * (int64_t)s, rec[3 * (int64_t)s + 2],
-                   [&](int plane, float g) { adam_update(P, m, v, (int64_t)plane * n_pad + i, g, a); });
-  } else {
-    for (int plane = 0; plane < nP; ++plane) adam_update(P, m, v, (int64_t)plane * n_pad + i, 0.0f, a);
-  }
+  candidate_grad<true>(P, n_pad, i, D, cam, g2d + 12 * j, rec[3 * j + 2],
+                 [&](int plane, double g) { g3d[(int64_t)plane * stride + j] = (float)g; });
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -272,6 +255,122 @@ k_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
   for (int plane = 0; plane < nP; ++plane) {
     const float gg = has ? g[(int64_t)plane * g_stride + col] : 0.0f;
     adam_update(P, m, v, (int64_t)plane * n_pad + i, gg, a);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused path, stage 1: geometric gradients of each candidate (fp64), i.e.
+// everything except the SH coefficients and the view-direction term of the
+// mean, which stage 2 forms while it streams the SH planes.  Scratch layout
+// (14 floats per candidate): double mean[3][C] (kept in fp64: stage 2 adds
+// the view-direction term and the sum may cancel), then float rest[8][C]
+// for planes 3..10 (log-scale, quaternion, logit).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+k_project_bwd_geo(const float* __restrict__ P, int64_t n_pad, BwdCam cam, int64_t n_cand,
+                  const int32_t* __restrict__ cand_idx, const float* __restrict__ g2d,
+                  double* __restrict__ g_mean, float* __restrict__ g_rest) {
+  const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (j >= n_cand) return;
+  const int64_t i = cand_idx[j];
+  candidate_grad<false>(P, n_pad, i, 0, cam, g2d + 12 * j, make_float4(0.f, 0.f, 0.f, 0.f),
+                 [&](int plane, double gv) {
+                   if (plane < 3) g_mean[(int64_t)plane * n_cand + j] = gv;
+                   else if (plane < 11) g_rest[(int64_t)(plane - 3) * n_cand + j] = (float)gv;
+                 });
+}
+
+// fp64 real SH basis (same ordering and normalisation as candidate_grad's)
+// and its gradient, unrolled over the coefficients of degree D.
+template <int D, class F>
+__device__ __forceinline__ void sh_terms(double x, double y, double z, F&& f) {
+  const double kPi = 3.141592653589793;
+  f(0, 0.5 / sqrt(kPi), 0.0, 0.0, 0.0);
+  if (D < 1) return;
+  const double k1 = sqrt(3.0 / (4.0 * kPi));
+  f(1, -k1 * y, 0.0, -k1, 0.0);
+  f(2, k1 * z, 0.0, 0.0, k1);
+  f(3, -k1 * x, -k1, 0.0, 0.0);
+  if (D < 2) return;
+  const double xx = x * x, yy = y * y, zz = z * z;
+  const double k2a = 0.5 * sqrt(15.0 / kPi), k2b = 0.25 * sqrt(5.0 / kPi),
+               k2c = 0.25 * sqrt(15.0 / kPi);
+  f(4, k2a * x * y, k2a * y, k2a * x, 0.0);
+  f(5, -k2a * y * z, 0.0, -k2a * z, -k2a * y);
+  f(6, k2b * (2.0 * zz - xx - yy), -2.0 * k2b * x, -2.0 * k2b * y, 4.0 * k2b * z);
+  f(7, -k2a * x * z, -k2a * z, 0.0, -k2a * x);
+  f(8, k2c * (xx - yy), 2.0 * k2c * x, -2.0 * k2c * y, 0.0);
+  if (D < 3) return;
+  const double k3a = 0.25 * sqrt(35.0 / (2.0 * kPi)), k3b = 0.5 * sqrt(105.0 / kPi),
+               k3c = 0.25 * sqrt(21.0 / (2.0 * kPi)), k3d = 0.25 * sqrt(7.0 / kPi),
+               k3e = 0.25 * sqrt(105.0 / kPi);
+  f(9, -k3a * y * (3.0 * xx - yy), -6.0 * k3a * x * y, -3.0 * k3a * (xx - yy), 0.0);
+  f(10, k3b * x * y * z, k3b * y * z, k3b * x * z, k3b * x * y);
+  f(11, -k3c * y * (4.0 * zz - xx - yy), 2.0 * k3c * x * y, -k3c * (4.0 * zz - xx - 3.0 * yy),
+    -8.0 * k3c * y * z);
+  f(12, k3d * z * (2.0 * zz - 3.0 * xx - 3.0 * yy), -6.0 * k3d * x * z, -6.0 * k3d * y * z,
+    k3d * (6.0 * zz - 3.0 * xx - 3.0 * yy));
+  f(13, -k3c * x * (4.0 * zz - xx - yy), -k3c * (4.0 * zz - 3.0 * xx - yy), 2.0 * k3c * x * y,
+    -8.0 * k3c * x * z);
+  f(14, k3e * z * (xx - yy), 2.0 * k3e * x * z, -2.0 * k3e * y * z, k3e * (xx - yy));
+  f(15, -k3a * x * (xx - 3.0 * yy), -3.0 * k3a * (xx - yy), 6.0 * k3a * x * y, 0.0);
+}
+
+// Fused path, stage 2: one thread per Gaussian streams its planes once:
+// SH planes (gradient = dL/dcolour * Y_k(d), plus the view-direction term
+// accumulated for the mean), then logit, quaternion, log-scale (compact
+// geometric gradients) and the mean.  Non-candidates get g = 0.
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+k_adam_fused(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v, int64_t n,
+             int64_t n_pad, BwdCam cam, const int32_t* __restrict__ slot_map,
+             const float4* __restrict__ rec, const float* __restrict__ g2d,
+             const double* __restrict__ g_mean, const float* __restrict__ g_rest, int64_t n_cand,
+             AdamK a) {
+  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (i >= n) return;
+  const int32_t s = slot_map[i];
+  const bool cand = s >= 0;
+  const float mx = P[i], my = P[n_pad + i], mz = P[2 * n_pad + i];
+  double gr = 0.0, gg = 0.0, gb = 0.0;
+  double dx = 0.0, dy = 0.0, dz = 0.0, dn = 1.0;
+  if (cand) {
+    const float4 rgb = rec[3 * (int64_t)s + 2];
+    const float* g2 = g2d + 12 * (int64_t)s;
+    gr = rgb.x > 0.f ? (double)g2[6] : 0.0;
+    gg = rgb.y > 0.f ? (double)g2[7] : 0.0;
+    gb = rgb.z > 0.f ? (double)g2[8] : 0.0;
+    dx = (double)mx - cam.campos[0];
+    dy = (double)my - cam.campos[1];
+    dz = (double)mz - cam.campos[2];
+    dn = sqrt(dx * dx + dy * dy + dz * dz);
+    dx /= dn; dy /= dn; dz /= dn;
+  }
+  // SH planes: gradient dL/dcolour * Y_k(d); the view-direction term of the
+  // mean (fp64: the tangential projection below cancels)
+  double ddx = 0.0, ddy = 0.0, ddz = 0.0;
+  sh_terms<D>(dx, dy, dz, [&](int k, double Y, double Yx, double Yy, double Yz) {
+    const int64_t base = (int64_t)(11 + 3 * k) * n_pad + i;
+    const double w = gr * P[base] + gg * P[base + n_pad] + gb * P[base + 2 * n_pad];
+    ddx = fma(w, Yx, ddx);
+    ddy = fma(w, Yy, ddy);
+    ddz = fma(w, Yz, ddz);
+    adam_update(P, m, v, base, (float)(gr * Y), a);
+    adam_update(P, m, v, base + n_pad, (float)(gg * Y), a);
+    adam_update(P, m, v, base + 2 * n_pad, (float)(gb * Y), a);
+  });
+  const double ddot = ddx * dx + ddy * dy + ddz * dz;
+#pragma unroll
+  for (int k = 10; k >= 3; --k) {
+    const float gk = cand ? g_rest[(int64_t)(k - 3) * n_cand + s] : 0.f;
+    adam_update(P, m, v, (int64_t)k * n_pad + i, gk, a);
+  }
+  const double d[3] = {dx, dy, dz}, ddv[3] = {ddx, ddy, ddz};
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    float gk = 0.f;
+    if (cand) gk = (float)(g_mean[(int64_t)k * n_cand + s] + (ddv[k] - d[k] * ddot) / dn);
+    adam_update(P, m, v, (int64_t)k * n_pad + i, gk, a);
   }
 }
 
@@ -317,7 +416,6 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
   if (n_cand > 0 && (!g2d || !proj->rec || !aligned(g2d, 16))) return GS_ERR_ARG;
   const BwdCam c = make_cam(cam);
   const int D = model->sh_degree;
-  const int nP = 11 + 3 * (D + 1) * (D + 1);
   cudaStream_t s = to_stream(stream);
   const float4* rec = reinterpret_cast<const float4*>(proj->rec);
   if (!fused) {
@@ -332,8 +430,28 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
   if (!make_adam(fused, &a)) return GS_ERR_ARG;
   if (!adam_m || !adam_v || !proj->slot) return GS_ERR_ARG;
   if (model->n == 0) return GS_OK;
-  k_project_bwd_adam<<<(unsigned)((model->n + kThreads - 1) / kThreads), kThreads, 0, s>>>(
-      model->params, adam_m, adam_v, model->n, model->n_pad, D, nP, c, proj->slot, rec, g2d, a);
+  // stage 1 needs 14 floats per candidate of scratch (8-byte aligned), in g3d
+  if (n_cand > 0 && (!g3d || g3d_stride < 14 * n_cand || !proj->cand_idx || !aligned(g3d, 8)))
+    return GS_ERR_ARG;
+  double* g_mean = reinterpret_cast<double*>(g3d);
+  float* g_rest = g3d + 6 * n_cand;
+  if (n_cand > 0) {
+    k_project_bwd_geo<<<(unsigned)((n_cand + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        model->params, model->n_pad, c, n_cand, proj->cand_idx, g2d, g_mean, g_rest);
+    GS_LAUNCH_CHECK();
+  }
+  const unsigned nb = (unsigned)((model->n + kThreads - 1) / kThreads);
+#define GS_ADAM_FUSED(DD)                                                                     \
+  k_adam_fused<DD><<<nb, kThreads, 0, s>>>(model->params, adam_m, adam_v, model->n,            \
+                                           model->n_pad, c, proj->slot, rec, g2d, g_mean, g_rest, \
+                                           n_cand, a)
+  switch (D) {
+    case 0: GS_ADAM_FUSED(0); break;
+    case 1: GS_ADAM_FUSED(1); break;
+    case 2: GS_ADAM_FUSED(2); break;
+    default: GS_ADAM_FUSED(3); break;
+  }
+#undef GS_ADAM_FUSED
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

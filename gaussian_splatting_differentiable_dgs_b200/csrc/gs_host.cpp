@@ -110,14 +110,16 @@ extern "C" gs_status gs_check(int32_t* dev_status, gs_stream stream) {
 }
 
 // Per-unit bytes of the buffers one Leaf needs (see gs.h).  Intersections:
-// keys + values + their sort double buffers (24 B) plus the look-back words
-// of the tile-bit sort (256 x 8 B per 4096 items per pass).  Pixels: colour
-// (12), T_final (4), last (4), target crop (12), dL/dcolour (12).  Tiles:
-// the int64 range pair.  Fixed: sort histograms, tickets and alignment.
+// 32-bit tile keys + 32-bit values + their sort double buffers (16 B) plus
+// the look-back words of the tile sort (256 x 8 B per 4096 items per pass).
+// tile_bits: bits of the whole grid's tile count, an upper bound of any
+// Leaf's local bits.  Pixels: colour (12), T_final (4), last (4), target
+// crop (12), dL/dcolour (12).  Tiles: the int64 range pair.  Fixed: sort
+// histograms, tickets and alignment.
 extern "C" gs_status gs_leaf_load_model(int32_t tile_bits, gs_load_model* out) {
   if (!out || tile_bits < 0 || tile_bits > 32) return GS_ERR_ARG;
   const int passes = tile_bits == 0 ? 0 : 2 * ((tile_bits + 15) / 16);
-  out->bytes_per_isect = 24 + (passes + 1) / 2;
+  out->bytes_per_isect = 16 + (passes + 1) / 2;
   out->bytes_per_pixel = 44;
   out->bytes_per_tile = 16;
   out->fixed_bytes = 8 * 256 * 8 + 64 * 4 + (int64_t)passes * 256 * 8 + 16 * 256;

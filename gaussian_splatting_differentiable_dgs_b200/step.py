@@ -187,17 +187,18 @@ class Stepper:
         if hooks is not None and hasattr(hooks, "on_project"):
             hooks.on_project(ctx)
 
-        # ---- depth presort --------------------------------------------------
+        # ---- depth presort (+ rects gathered in depth order) ------------------
         order = torch.empty(max(C, 1), dtype=torch.int32, device=dev)
+        drect = torch.empty(max(C, 1) * 4, dtype=torch.int16, device=dev)
         if C > 0:
-            k32 = torch.empty(C, dtype=torch.int32, device=dev)
-            ws = torch.empty(B.gs_sort_workspace_size(C, 4, 0, 32), dtype=torch.uint8, device=dev)
+            ws = torch.empty(B.gs_depth_order_workspace_size(C), dtype=torch.uint8, device=dev)
             tk = clk.tic("sort_depth")
-            B.gs_sort_keys32(dkey, k32, order, C, 0, 32, B.GS_SORT_IOTA, ws, st)
+            B.gs_depth_order(proj, C, order, drect, ws, st)
             clk.toc(tk)
-            launches += 1 + 4
-            del ws, k32
+            launches += 1 + 4 + 1
+            del ws
         ctx["depth_order"] = order
+        ctx["depth_rect"] = drect
 
         # ---- Leaf plan ------------------------------------------------------
         lm = B.gs_leaf_load_model(tile_bits)
@@ -222,7 +223,8 @@ class Stepper:
             ph = min(16 * y1, H) - 16 * y0
             npx = pw * ph
             nt = (x1 - x0) * (y1 - y0)
-            sizes = [8 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 8, 32, 32 + tile_bits),
+            lb_bits = B.local_tile_bits(L)
+            sizes = [4 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 4, 0, lb_bits),
                      12 * npx, 4 * npx, 4 * npx, 12 * npx]
             if target is not None and not resident_target:
                 sizes.append(12 * npx)
@@ -236,7 +238,7 @@ class Stepper:
             I = int(I)
             sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
             bufs, _ = _carve(arena, sizes)
-            keys = bufs[0].view(torch.int64)
+            keys = bufs[0].view(torch.int32)
             vals = bufs[1].view(torch.int32)
             ranges = bufs[2].view(torch.int64)
             sort_ws = bufs[3]
@@ -259,15 +261,16 @@ class Stepper:
             else:
                 px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
             tk = clk.tic("bin")
-            B.gs_bin_tiles(proj, C, order, L, TW, TH, sat, I, keys, vals, max(I, 1), ranges,
+            B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1), ranges,
                            bin_ws, st)
             clk.toc(tk)
             launches += 2 if (C > 0 and I > 0) else 1
-            if I > 0:
+            lb_bits = B.local_tile_bits(L)
+            if I > 0 and lb_bits > 0:
                 tk = clk.tic("sort_tiles")
-                B.gs_sort_keys(keys, vals, I, 32, 32 + tile_bits, sort_ws, st)
+                B.gs_sort_keys32(None, keys, vals, I, 0, lb_bits, 0, sort_ws, st)
                 clk.toc(tk)
-                launches += 1 + 2 * ((tile_bits + 15) // 16)
+                launches += 1 + 2 * ((lb_bits + 15) // 16)
             tk = clk.tic("raster_fwd")
             B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
             clk.toc(tk)
@@ -298,11 +301,14 @@ class Stepper:
         if update:
             m.step += 1
             if self.fuse_adam:
+                geo = torch.empty(14 * max(C, 1), dtype=torch.float32, device=dev)
                 tk = clk.tic("project_bwd")
-                B.gs_project_bwd(mod, camS, proj, C, g2d, adam_m=m.m, adam_v=m.v,
-                                 fused=self.adam_args(m.step), dev_status=st)
+                B.gs_project_bwd(mod, camS, proj, C, g2d, g3d=geo, g3d_stride=geo.numel(),
+                                 adam_m=m.m, adam_v=m.v, fused=self.adam_args(m.step),
+                                 dev_status=st)
                 clk.toc(tk)
-                launches += 1
+                launches += 2 if C > 0 else 1
+                del geo
             else:
                 g3d = torch.empty(m.P * max(C, 1), dtype=torch.float32, device=dev)
                 B.gs_project_bwd(mod, camS, proj, C, g2d, g3d=g3d, g3d_stride=max(C, 1),

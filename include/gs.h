@@ -6,12 +6,14 @@
  *
  *   gs_project       cull + EWA projection of the candidate Gaussians,
  *                    per-tile intersection counts and their summed-area table
- *   gs_sort_keys32   depth presort of the candidates (once per view)
+ *   gs_depth_order   depth presort of the candidates (once per view)
  *   gs_leaf_partition  (host) split the tile grid into Leaves whose
  *                    estimated load fits a byte budget
  *   for each Leaf:
- *     gs_bin_tiles   duplicated 64-bit keys (tile << 32 | depth) in depth order
- *     gs_sort_keys   stable radix sort on the tile bits -> per-tile lists
+ *     gs_bin_tiles   one entry per (candidate, tile) in depth order
+ *     gs_sort_keys32 stable radix sort on the Leaf-local tile index
+ *                    -> per-tile lists (the order of the 64-bit keys
+ *                    tile << 32 | depth)
  *     gs_raster_fwd  front-to-back compositing (+ fused L1 loss)
  *     gs_raster_bwd  reverse blend, accumulated into the view's compact
  *                    per-candidate 2D gradients
@@ -256,21 +258,35 @@ gs_status gs_leaf_partition(const int64_t* sat_host, int32_t TW, int32_t TH,
                             int64_t* leaf_bytes, uint8_t* over_budget,
                             int32_t max_leaves, int32_t* n_leaves);
 
-/* ---- 4. binning ----------------------------------------------------------
- * For the candidates in depth order (depth_order[0..n_cand)), emit one
- * entry per tile of rect ∩ leaf: key = (tile id << 32) | depth_key, value =
- * candidate slot, in depth order; and the Leaf's per-tile ranges
- * (ranges[2 * (ly * lw + lx)] = begin, [+1] = end, offsets into keys/vals,
- * tile rows of the Leaf in row-major order) from the device SAT.
- * n_isect: the Leaf's intersection count (from the host SAT); must be <=
- * capacity, else GS_ERR_CAPACITY with *needed = n_isect. */
+/* ---- 4. depth order and binning -----------------------------------------
+ * gs_depth_order (once per view): depth_order[0..n_cand) = candidate slots
+ * sorted by the fp32 bits of their depth (stable: equal depths keep the
+ * ascending Gaussian index), and depth_rect[j] = rect[depth_order[j]].
+ *
+ * gs_bin_tiles (per Leaf): for the candidates in depth order, one entry per
+ * tile of rect ∩ leaf, written in depth order: vals = candidate slot,
+ * tile_keys = Leaf-local tile index (ly * leaf width + lx), and, if keys64
+ * is not NULL, the duplicated 64-bit key (tile id << 32) | depth_key.  A
+ * stable sort of (tile_keys, vals) on the low ceil(log2(Leaf tiles)) bits
+ * (gs_sort_keys32) then gives the order of the 64-bit keys, i.e. each tile's
+ * list front to back with ties by Gaussian index.  Also writes the Leaf's
+ * per-tile ranges (ranges[2 t] = begin, [2 t + 1] = end, t = local tile
+ * index) from the device SAT.  n_isect: the Leaf's intersection count (from
+ * the host SAT); must be <= capacity, else GS_ERR_CAPACITY with *needed. */
+size_t gs_depth_order_workspace_size(int64_t n_cand);
+gs_status gs_depth_order(const gs_proj* proj, int64_t n_cand,
+                         int32_t* depth_order, int16_t* depth_rect, void* ws,
+                         size_t ws_bytes, int32_t* dev_status,
+                         gs_stream stream);
 size_t gs_bin_workspace_size(int64_t n_cand);
 gs_status gs_bin_tiles(const gs_proj* proj, int64_t n_cand,
-                       const int32_t* depth_order, gs_rect leaf, int32_t TW,
-                       int32_t TH, const int64_t* tile_sat, int64_t n_isect,
-                       uint64_t* keys, int32_t* vals, int64_t capacity,
-                       int64_t* ranges, int64_t* needed, void* ws,
-                       size_t ws_bytes, int32_t* dev_status, gs_stream stream);
+                       const int32_t* depth_order, const int16_t* depth_rect,
+                       gs_rect leaf, int32_t TW, int32_t TH,
+                       const int64_t* tile_sat, int64_t n_isect,
+                       uint32_t* tile_keys, int32_t* vals, uint64_t* keys64,
+                       int64_t capacity, int64_t* ranges, int64_t* needed,
+                       void* ws, size_t ws_bytes, int32_t* dev_status,
+                       gs_stream stream);
 
 /* ---- 5. raster forward ---------------------------------------------------
  * Per pixel p of the Leaf, over its tile's list in order: d = (u, v) - p;
@@ -314,7 +330,11 @@ gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals,
  * normalisation, opacity logit, SH).  If `fused` is NULL, writes compact
  * gradients g3d[P][g3d_stride] (column = candidate slot).  Otherwise applies
  * one Adam update (as gs_adam with a zero gradient for non-candidates) to
- * model->params, adam_m and adam_v over all n Gaussians; g3d is unused. */
+ * model->params, adam_m and adam_v over all n Gaussians, in two passes: the
+ * candidates' geometric gradients (fp64) into g3d used as scratch (>= 14 *
+ * n_cand floats, 8-byte aligned, g3d_stride = its size in floats), then one
+ * streaming pass
+ * over every Gaussian's planes that forms the SH gradients on the fly. */
 gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
                          const gs_proj* proj, int64_t n_cand,
                          const float* g2d, float* g3d, int64_t g3d_stride,

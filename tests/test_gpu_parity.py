@@ -211,20 +211,48 @@ def _leaf_tiles(L, TW):
     return np.array([ty * TW + tx for ty in range(y0, y1) for tx in range(x0, x1)], np.int32)
 
 
-def _bin_leaf(pb, C, order_d, L, TW, TH, sat_d, I, tile_bits):
+def _bin_leaf(pb, C, order_d, drect_d, L, TW, TH, sat_d, I, tile_bits):
+    """Bin one Leaf (with the 64-bit keys), then sort it two ways: the
+    product path (32-bit local tile keys) and the 64-bit keys on their tile
+    bits.  Returns the emitted keys64 and both sorted results."""
     b = B()
-    keys = torch.zeros(max(I, 1), dtype=torch.int64, device="cuda")
-    vals = torch.zeros(max(I, 1), dtype=torch.int32, device="cuda")
+    n = max(I, 1)
+    tkeys = torch.zeros(n, dtype=torch.int32, device="cuda")
+    vals = torch.zeros(n, dtype=torch.int32, device="cuda")
+    keys64 = torch.zeros(n, dtype=torch.int64, device="cuda")
     nt = (L[2] - L[0]) * (L[3] - L[1])
     ranges = torch.zeros(2 * nt, dtype=torch.int64, device="cuda")
     ws = torch.empty(max(b.gs_bin_workspace_size(C), 256), dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    b.gs_bin_tiles(pb.struct, C, order_d, L, TW, TH, sat_d, I, keys, vals, max(I, 1), ranges, ws,
-                   st)
-    if I:
-        b.gs_sort_keys(keys, vals, I, 32, 32 + tile_bits, _sort_ws(I, 8, 32, 32 + tile_bits), st)
+    b.gs_bin_tiles(pb.struct, C, order_d, drect_d, L, TW, TH, sat_d, I, tkeys, vals, n, ranges, ws,
+                   st, keys64=keys64)
     assert b.gs_check(st) == 0
-    return keys, vals, ranges
+    emitted = (keys64.cpu().numpy().view(np.uint64)[:I].copy(), tkeys.cpu().numpy()[:I].copy(),
+               vals.cpu().numpy()[:I].copy())
+    k64, v64 = keys64.clone(), vals.clone()
+    lb = b.local_tile_bits(L)
+    if I and lb:
+        b.gs_sort_keys32(None, tkeys, vals, I, 0, lb, 0, _sort_ws(I, 4, 0, lb), st)
+        b.gs_sort_keys(k64, v64, I, 32, 32 + tile_bits, _sort_ws(I, 8, 32, 32 + tile_bits), st)
+    assert b.gs_check(st) == 0
+    return emitted, tkeys, vals, k64, v64, ranges
+
+
+def test_depth_order(oracle_mod):
+    sc, cam = scene("hd")
+    pr = oracle_mod.project(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam)
+    C = len(pr["cand_idx"])
+    pb = ProjBuffers.from_oracle(pr, sc.n)
+    b = B()
+    order = torch.zeros(C, dtype=torch.int32, device="cuda")
+    drect = torch.zeros(4 * C, dtype=torch.int16, device="cuda")
+    ws = torch.empty(b.gs_depth_order_workspace_size(C), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b.gs_depth_order(pb.struct, C, order, drect, ws, st)
+    assert b.gs_check(st) == 0
+    exp = np.argsort(pr["key"], kind="stable")
+    assert (order.cpu().numpy() == exp).all()
+    assert (drect.cpu().numpy().reshape(-1, 4) == pr["rect"][exp]).all()
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "hd"])
@@ -238,8 +266,9 @@ def test_bin_sort_ranges_bitexact(oracle_mod, name):
     sat_d = torch.as_tensor(sat.reshape(-1)).cuda()
     order = np.argsort(pr["key"], kind="stable").astype(np.int32)
     order_d = torch.as_tensor(order).cuda()
+    drect_d = torch.as_tensor(pr["rect"][order].astype(np.int16).reshape(-1)).cuda()
     tile_bits = max(1, math.ceil(math.log2(TW * TH)))
-    lm = [25, 44, 16, 30000, 512]
+    lm = [17, 44, 16, 30000, 512]
     budget = {"tiny": 150_000, "ragged": 40_000, "hd": 8_000_000}[name]
     leaves = oracle_mod.leaf_partition(sat, TW, TH, cam.width, cam.height, lm, budget)[0]
     assert len(leaves) > 1
@@ -249,15 +278,26 @@ def test_bin_sort_ranges_bitexact(oracle_mod, name):
         tiles = _leaf_tiles(L, TW)
         off, vals_o = oracle_mod.tile_lists(pr["rect"], pr["key"], TW, tiles)
         I = int(off[-1])
-        keys, vals, ranges = _bin_leaf(pb, C, order_d, L, TW, TH, sat_d, I, tile_bits)
+        emitted, tkeys, vals, k64, v64, ranges = _bin_leaf(pb, C, order_d, drect_d, L, TW, TH,
+                                                           sat_d, I, tile_bits)
         rg = ranges.cpu().numpy().reshape(-1, 2)
         assert (rg[:, 0] == off[:-1]).all() and (rg[:, 1] == off[1:]).all()
-        v = vals.cpu().numpy()[:I]
-        assert (v == vals_o).all()
-        k = keys.cpu().numpy().view(np.uint64)[:I]
         tile_of = np.repeat(tiles.astype(np.uint64), np.diff(off))
         exp_k = (tile_of << np.uint64(32)) | pr["key"][vals_o].astype(np.uint64)
-        assert (k == exp_k).all()
+        # emitted 64-bit keys: the oracle's multiset, in depth order of the candidates
+        k_emit, t_emit, v_emit = emitted
+        assert (np.sort(k_emit) == np.sort(exp_k)).all()
+        depth_rank = np.empty(C, np.int64)
+        depth_rank[order] = np.arange(C)
+        assert (np.diff(depth_rank[v_emit]) >= 0).all()
+        x0, y0, x1, y1 = L
+        g_tile = (k_emit >> np.uint64(32)).astype(np.int64)
+        loc = (g_tile // TW - y0) * (x1 - x0) + (g_tile % TW - x0)
+        assert (t_emit == loc).all()
+        # both sorts give the oracle's per-tile lists, bit-exactly
+        assert (vals.cpu().numpy()[:I] == vals_o).all()
+        assert (v64.cpu().numpy()[:I] == vals_o).all()
+        assert (k64.cpu().numpy().view(np.uint64)[:I] == exp_k).all()
 
 
 # ---------------------------------------------------------------------------
@@ -518,8 +558,10 @@ def test_fused_project_bwd_adam(oracle_mod, name):
     model = b.gs_model(sc.n, sc.n_pad, sc.sh_degree, 0, params.data_ptr())
     g2 = np.zeros((C, 12), np.float32)
     g2[:, :9] = g2d
+    geo = torch.zeros(14 * C, device="cuda")
     b.gs_project_bwd(model, b.camera_struct(cam), pb.struct, C, torch.as_tensor(g2.reshape(-1)).cuda(),
-                     adam_m=md, adam_v=vd, fused=b.gs_adam_args(1e-3, 0.9, 0.999, 1e-8, 2, 0))
+                     g3d=geo, g3d_stride=geo.numel(), adam_m=md, adam_v=vd,
+                     fused=b.gs_adam_args(1e-3, 0.9, 0.999, 1e-8, 2, 0))
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     assert b.gs_check(st) == 0
     n = sc.n

@@ -49,8 +49,8 @@ def test_host_argument_checks(gsb):
     # capacity errors report the needed size
     proj = b.gs_proj(10, 1, 1, 1, 16, 8, 1)
     needed = ctypes.c_int64(0)
-    st = L.gs_bin_tiles(ctypes.byref(proj), 10, 1, b.gs_rect(0, 0, 2, 2), 4, 4, 8, 1000, 8, 8,
-                        999, 8, ctypes.byref(needed), 256, 1 << 20, None, None)
+    st = L.gs_bin_tiles(ctypes.byref(proj), 10, 8, 8, b.gs_rect(0, 0, 2, 2), 4, 4, 8, 1000, 8, 8,
+                        None, 999, 8, ctypes.byref(needed), 256, 1 << 20, None, None)
     assert st == b.GS_ERR_CAPACITY and needed.value == 1000
 
 
@@ -60,7 +60,8 @@ def test_workspace_sizes(gsb):
     s1 = b.gs_sort_workspace_size(1 << 20, 8, 32, 48)
     s2 = b.gs_sort_workspace_size(1 << 20, 8, 32, 64)
     assert s2 > s1 > 12 << 20
-    assert b.gs_bin_workspace_size(1 << 20) >= 8 * (1 << 20) // 256
+    assert b.gs_bin_workspace_size(1 << 20) >= 8 * (1 << 20) // 1024
+    assert b.gs_depth_order_workspace_size(1 << 20) > 12 << 20
 
 
 def test_load_model_matches_buffers(gsb):
@@ -69,11 +70,11 @@ def test_load_model_matches_buffers(gsb):
         lm = b.gs_leaf_load_model(bits)
         passes = 2 * ((bits + 15) // 16)
         n = 5_000_000
-        need = 12 * n + b.gs_sort_workspace_size(n, 8, 32, 32 + bits)
+        need = 8 * n + b.gs_sort_workspace_size(n, 4, 0, bits)
         est = lm.bytes_per_isect * n + lm.fixed_bytes
         assert need <= est
         assert lm.bytes_per_pixel == 44 and lm.bytes_per_tile == 16 and lm.align == 512
-        assert lm.bytes_per_isect == 24 + (passes + 1) // 2
+        assert lm.bytes_per_isect == 16 + (passes + 1) // 2
 
 
 def _lm_list(lm):
