@@ -150,7 +150,7 @@ class OracleSample:
         p64, pr, counts, TW, TH = self._setup(v)
         n = sc.n
         W, H = cam.width, cam.height
-        I_total = int(counts.sum())
+        I_total = int(pr["rec"][:, 14].sum())   # tiles of the 3-sigma squares
         # projection of 1/8 of the Gaussians
         sub = np.sort(self.rng.choice(n, n // 8, replace=False))
         ps = np.ascontiguousarray(p64[:, sub])
@@ -263,7 +263,8 @@ def main():
     clk = clocks.stop()
     stp.check()
     ms = e0.elapsed_time(e1)
-    isect = sum(s.n_isect for s in stats)
+    isect = sum(s.n_isect_square for s in stats)   # conventional 3-sigma-square count
+    entries = sum(s.n_isect for s in stats)         # entries of the tight tile lists
     launches = sum(s.launches for s in stats)
     peak_ws = max(s.peak_ws_bytes for s in stats)
     stage_ms = {name: sum(x.elapsed_time(y) for x, y in timing.get(name, [])) for name in STAGES}
@@ -331,7 +332,7 @@ def main():
             dev_t.copy_(host_t[v], non_blocking=True)
             s = stp.run_view(cams[v], dev_t)
             loss_h.copy_(stp._last_loss, non_blocking=True)
-            e2e_isect += s.n_isect
+            e2e_isect += s.n_isect_square
         f1.record()
         torch.cuda.synchronize()
         ems = f0.elapsed_time(f1)
@@ -378,6 +379,7 @@ def main():
                              "stream every step)"},
             "peak_ws_gib": peak_ws / 2 ** 30,
             "isect_per_view": isect / a.steps,
+            "list_entries_per_view": entries / a.steps,
             "candidates_per_view": statistics.mean(s.n_cand for s in stats),
             "leaves_per_view": statistics.mean(s.n_leaves for s in stats),
             "stage_ms_per_step": {s: round(per_step[s], 3) for s in STAGES},

@@ -48,7 +48,7 @@ class gs_model(C.Structure):
 class gs_proj(C.Structure):
     _fields_ = [("capacity", C.c_int64), ("n_cand", C.c_void_p), ("cand_idx", C.c_void_p),
                 ("slot", C.c_void_p), ("rec", C.c_void_p), ("rect", C.c_void_p),
-                ("depth_key", C.c_void_p)]
+                ("depth_key", C.c_void_p), ("square_isect", C.c_void_p)]
 
 
 class gs_rect(C.Structure):
@@ -96,7 +96,8 @@ class gs_adam_args(C.Structure):
 SYMBOLS = [
     "gs_version", "gs_status_string", "gs_check",
     "gs_project_workspace_size", "gs_project",
-    "gs_sort_workspace_size", "gs_sort_keys", "gs_sort_keys32", "gs_sort_keys32_noalloc",
+    "gs_sort_workspace_size", "gs_sort_keys", "gs_sort_keys32", "gs_sort_tiles",
+    "gs_sort_keys32_noalloc",
     "gs_leaf_load_model", "gs_leaf_partition",
     "gs_depth_order_workspace_size", "gs_depth_order",
     "gs_bin_workspace_size", "gs_bin_tiles",
@@ -121,6 +122,7 @@ def _load():
         "gs_sort_keys": (i32, [p, p, i64, i32, i32, p, sz, p, p]),
         "gs_sort_keys32": (i32, [p, p, p, i64, i32, i32, u32, p, sz, p, p]),
         "gs_sort_keys32_noalloc": (i32, [p, p, p, i64, i32, i32, u32, p, p]),
+        "gs_sort_tiles": (i32, [p, p, i64, p, i64, p, sz, p, p]),
         "gs_leaf_load_model": (i32, [i32, P(gs_load_model)]),
         "gs_leaf_partition": (i32, [p, i32, i32, i32, i32, P(gs_load_model), i64, p, p, p, p,
                                     i32, P(i32)]),
@@ -229,6 +231,12 @@ def gs_sort_keys32(keys_in, keys, vals, n, begin_bit, end_bit, flags, ws, dev_st
                                                    begin_bit, end_bit, flags, ptr(ws),
                                                    ws.numel() * ws.element_size(),
                                                    ptr(dev_status), _stream(stream)))
+
+
+def gs_sort_tiles(tile_keys, vals, n, ranges, n_tiles, ws, dev_status, stream=None):
+    return _ok("gs_sort_tiles", _L.gs_sort_tiles(ptr(tile_keys), ptr(vals), n, ptr(ranges), n_tiles,
+                                                 ptr(ws), ws.numel() * ws.element_size(),
+                                                 ptr(dev_status), _stream(stream)))
 
 
 SORT_NOALLOC_MAX_N = 1 << 18

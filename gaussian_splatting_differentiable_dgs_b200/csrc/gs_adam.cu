@@ -280,66 +280,79 @@ k_project_bwd_geo(const float* __restrict__ P, int64_t n_pad, BwdCam cam, int64_
                  });
 }
 
-// fp64 real SH basis (same ordering and normalisation as candidate_grad's)
-// and its gradient, unrolled over the coefficients of degree D.
-template <int D, class F>
-__device__ __forceinline__ void sh_terms(double x, double y, double z, F&& f) {
+// fp64 real SH basis function k (same ordering and normalisation as
+// candidate_grad's) and its gradient; k is a compile-time constant after
+// unrolling, so the switch folds away.
+__device__ __forceinline__ void sh_term(int k, double x, double y, double z, double& Y,
+                                        double& Yx, double& Yy, double& Yz) {
   const double kPi = 3.141592653589793;
-  f(0, 0.5 / sqrt(kPi), 0.0, 0.0, 0.0);
-  if (D < 1) return;
-  const double k1 = sqrt(3.0 / (4.0 * kPi));
-  f(1, -k1 * y, 0.0, -k1, 0.0);
-  f(2, k1 * z, 0.0, 0.0, k1);
-  f(3, -k1 * x, -k1, 0.0, 0.0);
-  if (D < 2) return;
   const double xx = x * x, yy = y * y, zz = z * z;
+  const double k1 = sqrt(3.0 / (4.0 * kPi));
   const double k2a = 0.5 * sqrt(15.0 / kPi), k2b = 0.25 * sqrt(5.0 / kPi),
                k2c = 0.25 * sqrt(15.0 / kPi);
-  f(4, k2a * x * y, k2a * y, k2a * x, 0.0);
-  f(5, -k2a * y * z, 0.0, -k2a * z, -k2a * y);
-  f(6, k2b * (2.0 * zz - xx - yy), -2.0 * k2b * x, -2.0 * k2b * y, 4.0 * k2b * z);
-  f(7, -k2a * x * z, -k2a * z, 0.0, -k2a * x);
-  f(8, k2c * (xx - yy), 2.0 * k2c * x, -2.0 * k2c * y, 0.0);
-  if (D < 3) return;
   const double k3a = 0.25 * sqrt(35.0 / (2.0 * kPi)), k3b = 0.5 * sqrt(105.0 / kPi),
                k3c = 0.25 * sqrt(21.0 / (2.0 * kPi)), k3d = 0.25 * sqrt(7.0 / kPi),
                k3e = 0.25 * sqrt(105.0 / kPi);
-  f(9, -k3a * y * (3.0 * xx - yy), -6.0 * k3a * x * y, -3.0 * k3a * (xx - yy), 0.0);
-  f(10, k3b * x * y * z, k3b * y * z, k3b * x * z, k3b * x * y);
-  f(11, -k3c * y * (4.0 * zz - xx - yy), 2.0 * k3c * x * y, -k3c * (4.0 * zz - xx - 3.0 * yy),
-    -8.0 * k3c * y * z);
-  f(12, k3d * z * (2.0 * zz - 3.0 * xx - 3.0 * yy), -6.0 * k3d * x * z, -6.0 * k3d * y * z,
-    k3d * (6.0 * zz - 3.0 * xx - 3.0 * yy));
-  f(13, -k3c * x * (4.0 * zz - xx - yy), -k3c * (4.0 * zz - 3.0 * xx - yy), 2.0 * k3c * x * y,
-    -8.0 * k3c * x * z);
-  f(14, k3e * z * (xx - yy), 2.0 * k3e * x * z, -2.0 * k3e * y * z, k3e * (xx - yy));
-  f(15, -k3a * x * (xx - 3.0 * yy), -3.0 * k3a * (xx - yy), 6.0 * k3a * x * y, 0.0);
+  switch (k) {
+    case 0: Y = 0.5 / sqrt(kPi); Yx = Yy = Yz = 0.0; break;
+    case 1: Y = -k1 * y; Yx = 0.0; Yy = -k1; Yz = 0.0; break;
+    case 2: Y = k1 * z; Yx = 0.0; Yy = 0.0; Yz = k1; break;
+    case 3: Y = -k1 * x; Yx = -k1; Yy = 0.0; Yz = 0.0; break;
+    case 4: Y = k2a * x * y; Yx = k2a * y; Yy = k2a * x; Yz = 0.0; break;
+    case 5: Y = -k2a * y * z; Yx = 0.0; Yy = -k2a * z; Yz = -k2a * y; break;
+    case 6: Y = k2b * (2.0 * zz - xx - yy); Yx = -2.0 * k2b * x; Yy = -2.0 * k2b * y;
+            Yz = 4.0 * k2b * z; break;
+    case 7: Y = -k2a * x * z; Yx = -k2a * z; Yy = 0.0; Yz = -k2a * x; break;
+    case 8: Y = k2c * (xx - yy); Yx = 2.0 * k2c * x; Yy = -2.0 * k2c * y; Yz = 0.0; break;
+    case 9: Y = -k3a * y * (3.0 * xx - yy); Yx = -6.0 * k3a * x * y; Yy = -3.0 * k3a * (xx - yy);
+            Yz = 0.0; break;
+    case 10: Y = k3b * x * y * z; Yx = k3b * y * z; Yy = k3b * x * z; Yz = k3b * x * y; break;
+    case 11: Y = -k3c * y * (4.0 * zz - xx - yy); Yx = 2.0 * k3c * x * y;
+             Yy = -k3c * (4.0 * zz - xx - 3.0 * yy); Yz = -8.0 * k3c * y * z; break;
+    case 12: Y = k3d * z * (2.0 * zz - 3.0 * xx - 3.0 * yy); Yx = -6.0 * k3d * x * z;
+             Yy = -6.0 * k3d * y * z; Yz = k3d * (6.0 * zz - 3.0 * xx - 3.0 * yy); break;
+    case 13: Y = -k3c * x * (4.0 * zz - xx - yy); Yx = -k3c * (4.0 * zz - 3.0 * xx - yy);
+             Yy = 2.0 * k3c * x * y; Yz = -8.0 * k3c * x * z; break;
+    case 14: Y = k3e * z * (xx - yy); Yx = 2.0 * k3e * x * z; Yy = -2.0 * k3e * y * z;
+             Yz = k3e * (xx - yy); break;
+    default: Y = -k3a * x * (xx - 3.0 * yy); Yx = -3.0 * k3a * (xx - yy); Yy = 6.0 * k3a * x * y;
+             Yz = 0.0; break;
+  }
+}
+
+__device__ __forceinline__ void adam_vals(float& p, float& m, float& v, float g, const AdamK& a) {
+  m = fmaf(a.b1, m, a.omb1 * g);
+  v = fmaf(a.b2, v, a.omb2 * g * g);
+  p = p - a.lr * (m / a.bc1) / (sqrtf(v / a.bc2) + a.eps);
 }
 
 // Fused path, stage 2: one thread per Gaussian streams its planes once:
 // SH planes (gradient = dL/dcolour * Y_k(d), plus the view-direction term
-// accumulated for the mean), then logit, quaternion, log-scale (compact
-// geometric gradients) and the mean.  Non-candidates get g = 0.
+// accumulated for the mean), then log-scale, quaternion, logit (compact
+// geometric gradients) and the mean.  Non-candidates get g = 0.  Loads of a
+// group of planes are issued before any of its stores.
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 k_adam_fused(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v, int64_t n,
              int64_t n_pad, BwdCam cam, const int32_t* __restrict__ slot_map,
              const float4* __restrict__ rec, const float* __restrict__ g2d,
              const double* __restrict__ g_mean, const float* __restrict__ g_rest, int64_t n_cand,
              AdamK a) {
+  constexpr int KS = (D + 1) * (D + 1);
+  constexpr int GK = 2;  // SH coefficients per load group (6 planes)
   const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (i >= n) return;
   const int32_t s = slot_map[i];
   const bool cand = s >= 0;
   const float mx = P[i], my = P[n_pad + i], mz = P[2 * n_pad + i];
-  double gr = 0.0, gg = 0.0, gb = 0.0;
+  double gc[3] = {0.0, 0.0, 0.0};
   double dx = 0.0, dy = 0.0, dz = 0.0, dn = 1.0;
   if (cand) {
     const float4 rgb = rec[3 * (int64_t)s + 2];
     const float* g2 = g2d + 12 * (int64_t)s;
-    gr = rgb.x > 0.f ? (double)g2[6] : 0.0;
-    gg = rgb.y > 0.f ? (double)g2[7] : 0.0;
-    gb = rgb.z > 0.f ? (double)g2[8] : 0.0;
+    gc[0] = rgb.x > 0.f ? (double)g2[6] : 0.0;
+    gc[1] = rgb.y > 0.f ? (double)g2[7] : 0.0;
+    gc[2] = rgb.z > 0.f ? (double)g2[8] : 0.0;
     dx = (double)mx - cam.campos[0];
     dy = (double)my - cam.campos[1];
     dz = (double)mz - cam.campos[2];
@@ -347,30 +360,88 @@ k_adam_fused(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v
     dx /= dn; dy /= dn; dz /= dn;
   }
   // SH planes: gradient dL/dcolour * Y_k(d); the view-direction term of the
-  // mean (fp64: the tangential projection below cancels)
+  // mean in fp64 (the tangential projection below cancels)
   double ddx = 0.0, ddy = 0.0, ddz = 0.0;
-  sh_terms<D>(dx, dy, dz, [&](int k, double Y, double Yx, double Yy, double Yz) {
-    const int64_t base = (int64_t)(11 + 3 * k) * n_pad + i;
-    const double w = gr * P[base] + gg * P[base + n_pad] + gb * P[base + 2 * n_pad];
-    ddx = fma(w, Yx, ddx);
-    ddy = fma(w, Yy, ddy);
-    ddz = fma(w, Yz, ddz);
-    adam_update(P, m, v, base, (float)(gr * Y), a);
-    adam_update(P, m, v, base + n_pad, (float)(gg * Y), a);
-    adam_update(P, m, v, base + 2 * n_pad, (float)(gb * Y), a);
-  });
-  const double ddot = ddx * dx + ddy * dy + ddz * dz;
+#pragma unroll 1
+  for (int k0 = 0; k0 < KS; k0 += GK) {
+    float pv[GK][3], mv[GK][3], vv[GK][3];
 #pragma unroll
-  for (int k = 10; k >= 3; --k) {
-    const float gk = cand ? g_rest[(int64_t)(k - 3) * n_cand + s] : 0.f;
-    adam_update(P, m, v, (int64_t)k * n_pad + i, gk, a);
+    for (int kk = 0; kk < GK; ++kk)
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) {
+        if (k0 + kk >= KS) continue;
+        const int64_t idx = (int64_t)(11 + 3 * (k0 + kk) + ch) * n_pad + i;
+        pv[kk][ch] = P[idx];
+        mv[kk][ch] = m[idx];
+        vv[kk][ch] = v[idx];
+      }
+#pragma unroll
+    for (int kk = 0; kk < GK; ++kk) {
+      if (k0 + kk >= KS) continue;
+      double Y, Yx, Yy, Yz;
+      sh_term(k0 + kk, dx, dy, dz, Y, Yx, Yy, Yz);
+      const double w = gc[0] * pv[kk][0] + gc[1] * pv[kk][1] + gc[2] * pv[kk][2];
+      ddx = fma(w, Yx, ddx);
+      ddy = fma(w, Yy, ddy);
+      ddz = fma(w, Yz, ddz);
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) adam_vals(pv[kk][ch], mv[kk][ch], vv[kk][ch], (float)(gc[ch] * Y), a);
+    }
+#pragma unroll
+    for (int kk = 0; kk < GK; ++kk)
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) {
+        if (k0 + kk >= KS) continue;
+        const int64_t idx = (int64_t)(11 + 3 * (k0 + kk) + ch) * n_pad + i;
+        P[idx] = pv[kk][ch];
+        m[idx] = mv[kk][ch];
+        v[idx] = vv[kk][ch];
+      }
+  }
+  const double ddot = ddx * dx + ddy * dy + ddz * dz;
+  // geometric planes 3..10 in two groups of four, then the mean 0..2
+#pragma unroll 1
+  for (int k0 = 3; k0 < 11; k0 += 4) {
+    float pg[4], mg[4], vg[4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int64_t idx = (int64_t)(k0 + kk) * n_pad + i;
+      pg[kk] = P[idx];
+      mg[kk] = m[idx];
+      vg[kk] = v[idx];
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const float gk = cand ? g_rest[(int64_t)(k0 + kk - 3) * n_cand + s] : 0.f;
+      adam_vals(pg[kk], mg[kk], vg[kk], gk, a);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int64_t idx = (int64_t)(k0 + kk) * n_pad + i;
+      P[idx] = pg[kk];
+      m[idx] = mg[kk];
+      v[idx] = vg[kk];
+    }
+  }
+  float pg[3] = {mx, my, mz}, mg[3], vg[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    mg[k] = m[(int64_t)k * n_pad + i];
+    vg[k] = v[(int64_t)k * n_pad + i];
   }
   const double d[3] = {dx, dy, dz}, ddv[3] = {ddx, ddy, ddz};
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     float gk = 0.f;
     if (cand) gk = (float)(g_mean[(int64_t)k * n_cand + s] + (ddv[k] - d[k] * ddot) / dn);
-    adam_update(P, m, v, (int64_t)k * n_pad + i, gk, a);
+    adam_vals(pg[k], mg[k], vg[k], gk, a);
+  }
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int64_t idx = (int64_t)k * n_pad + i;
+    P[idx] = pg[k];
+    m[idx] = mg[k];
+    v[idx] = vg[k];
   }
 }
 

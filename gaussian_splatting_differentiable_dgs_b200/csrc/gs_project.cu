@@ -12,6 +12,7 @@
 // nothing here, and it makes every integer decision (cull, tile rect, depth
 // key) independent of fp32 rounding.  The camera-space position, screen
 // position and cull tests use explicitly rounded operations in a fixed order.
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "gs_internal.cuh"
@@ -65,6 +66,7 @@ struct ProjOut {
   float4 r0, r1, r2;
   short4 rect;
   uint32_t key;
+  int64_t square_tiles;
 };
 
 // Returns true if Gaussian i is a candidate and fills `o`.
@@ -150,11 +152,31 @@ __device__ __forceinline__ bool project_gaussian(const float* __restrict__ P, in
   const double rad = ceil(3.0 * sqrt(lam));
   const int64_t rx0 = (int64_t)floor((u - rad) / kTile), rx1 = (int64_t)floor((u + rad) / kTile) + 1;
   const int64_t ry0 = (int64_t)floor((v - rad) / kTile), ry1 = (int64_t)floor((v + rad) / kTile) + 1;
-  const int64_t x0 = rx0 < 0 ? 0 : (rx0 > c.TW ? c.TW : rx0);
-  const int64_t x1 = rx1 < 0 ? 0 : (rx1 > c.TW ? c.TW : rx1);
-  const int64_t y0 = ry0 < 0 ? 0 : (ry0 > c.TH ? c.TH : ry0);
-  const int64_t y1 = ry1 < 0 ? 0 : (ry1 > c.TH ? c.TH : ry1);
+  const double opac = 1.0 / (1.0 + exp(-(double)pv[7]));
+  // tiles whose pixel-centre box can see alpha >= 1/255: o exp(-q) >= 1/255
+  // holds only inside the ellipse q <= ln(255 o); its bounding box, inflated
+  // well beyond the fp32 error of the rasteriser's alpha, bounds the rect
+  const double lq = log(255.0 * opac);
+  if (!(lq > -1e-4)) return false;  // never reaches 1/255 anywhere
+  const double qb = fmax(lq, 0.0) * 1.0001 + 1e-4;
+  const double hx = sqrt(2.0 * qb * c00) + 0.01, hy = sqrt(2.0 * qb * c11) + 0.01;
+  const int64_t bx0 = (int64_t)ceil((u - hx - 15.5) / kTile), bx1 = (int64_t)floor((u + hx - 0.5) / kTile) + 1;
+  const int64_t by0 = (int64_t)ceil((v - hy - 15.5) / kTile), by1 = (int64_t)floor((v + hy - 0.5) / kTile) + 1;
+  const int64_t cx0 = rx0 > bx0 ? rx0 : bx0, cx1 = rx1 < bx1 ? rx1 : bx1;
+  const int64_t cy0 = ry0 > by0 ? ry0 : by0, cy1 = ry1 < by1 ? ry1 : by1;
+  const int64_t x0 = cx0 < 0 ? 0 : (cx0 > c.TW ? c.TW : cx0);
+  const int64_t x1 = cx1 < 0 ? 0 : (cx1 > c.TW ? c.TW : cx1);
+  const int64_t y0 = cy0 < 0 ? 0 : (cy0 > c.TH ? c.TH : cy0);
+  const int64_t y1 = cy1 < 0 ? 0 : (cy1 > c.TH ? c.TH : cy1);
   if (x0 >= x1 || y0 >= y1) return false;
+  {
+    // tiles of the plain 3-sigma square (clamped), counted for the metric
+    const int64_t sx0 = rx0 < 0 ? 0 : (rx0 > c.TW ? c.TW : rx0);
+    const int64_t sx1 = rx1 < 0 ? 0 : (rx1 > c.TW ? c.TW : rx1);
+    const int64_t sy0 = ry0 < 0 ? 0 : (ry0 > c.TH ? c.TH : ry0);
+    const int64_t sy1 = ry1 < 0 ? 0 : (ry1 > c.TH ? c.TH : ry1);
+    o.square_tiles = (sx1 > sx0 && sy1 > sy0) ? (sx1 - sx0) * (sy1 - sy0) : 0;
+  }
 
   // colour from SH at the direction camera centre -> mean
   double dx = x - c.campos[0], dy = y - c.campos[1], dz = z - c.campos[2];
@@ -171,10 +193,13 @@ __device__ __forceinline__ bool project_gaussian(const float* __restrict__ P, in
       rgb[ch] += (double)s * Y[k];
     }
   }
-  const double opac = 1.0 / (1.0 + exp(-(double)pv[7]));
-
   const float uh = (float)u, vh = (float)v;
-  o.r0 = make_float4(uh, vh, (float)(u - (double)uh), (float)(v - (double)vh));
+  // u, v as fp32 + fp16 corrections (|lo| <= ulp(u)/2, so the pair is exact
+  // to ~2e-7 px); the alpha box half extents as fp16 rounded up
+  const __half2 lo = __floats2half2_rn((float)(u - (double)uh), (float)(v - (double)vh));
+  const __half2 box = __halves2half2(__float2half_ru((float)hx), __float2half_ru((float)hy));
+  o.r0 = make_float4(uh, vh, __uint_as_float(*reinterpret_cast<const unsigned*>(&lo)),
+                     __uint_as_float(*reinterpret_cast<const unsigned*>(&box)));
   const double a = c11 / det, b = -c01 / det;
   o.r1 = make_float4((float)(0.5 * a), (float)(b / a), (float)(0.5 / c11), (float)opac);
   const float depth = (float)tz;
@@ -189,7 +214,8 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, int D, Pro
           int32_t* __restrict__ cand_idx, int32_t* __restrict__ slot_map, float4* __restrict__ rec,
           short4* __restrict__ rect, uint32_t* __restrict__ depth_key, int32_t* __restrict__ diff,
           unsigned long long* __restrict__ lb, unsigned int* __restrict__ ticket,
-          int32_t* __restrict__ n_cand, int64_t n_blocks, int64_t capacity, int32_t* dev_status) {
+          int32_t* __restrict__ n_cand, int64_t n_blocks, int64_t capacity,
+          unsigned long long* __restrict__ square_isect, int32_t* dev_status) {
   __shared__ unsigned int s_b;
   __shared__ int s_scan[kProjThreads / 32 + 1];
   __shared__ long long s_prefix;
@@ -226,6 +252,11 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, int D, Pro
     atomicAdd(&diff[o.rect.w * s + o.rect.z], 1);
   }
   if (b == n_blocks - 1 && threadIdx.x == 0) *n_cand = (int32_t)(s_prefix + total);
+  if (square_isect) {
+    unsigned long long sq = (cand && fits) ? (unsigned long long)o.square_tiles : 0ull;
+    sq = warp_sum(sq);
+    if ((threadIdx.x & 31) == 0 && sq) atomicAdd(square_isect, sq);
+  }
 }
 
 // Double inclusive prefix along x of each row (y < TH, x < TW).
@@ -333,11 +364,12 @@ extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uin
   // ticket, look-back words and the difference grid start at zero
   const size_t zero_bytes = (size_t)((char*)(w.diff + (TW + 1) * (TH + 1)) - (char*)ws);
   GS_TRY(cudaMemsetAsync(ws, 0, zero_bytes, s));
+  if (out->square_isect) GS_TRY(cudaMemsetAsync(out->square_isect, 0, sizeof(unsigned long long), s));
   if (nb > 0) {
     k_project<<<(unsigned)nb, kProjThreads, 0, s>>>(
         model->params, model->n, model->n_pad, model->sh_degree, pc, out->cand_idx, out->slot,
         reinterpret_cast<float4*>(out->rec), reinterpret_cast<short4*>(out->rect), out->depth_key,
-        w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, dev_status);
+        w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, out->square_isect, dev_status);
     GS_LAUNCH_CHECK();
   } else {
     GS_TRY(cudaMemsetAsync(out->n_cand, 0, sizeof(int32_t), s));

@@ -14,6 +14,8 @@
 // one record per thread; within a batch every thread reads each record by
 // broadcast.  fp32 arithmetic with explicitly rounded operations in the
 // alpha path, so the backward retakes exactly the forward's skip decisions.
+#include <cuda_fp16.h>
+
 #include <algorithm>
 
 #include "gs_internal.cuh"
@@ -38,6 +40,7 @@ struct Staged {
   float gx, gy, beta, ns1;   // float4
   float ns2, opac, r, g;     // float4
   float b, s1, s2;           // natural-log coefficients (backward)
+  float hx, hy;              // alpha box half extents
   int32_t slot;
 };
 
@@ -47,8 +50,13 @@ __device__ __forceinline__ Staged stage_record(const float4* __restrict__ rec, i
   const float4 r1 = rec[3 * (int64_t)slot + 1];
   const float4 r2 = rec[3 * (int64_t)slot + 2];
   Staged s;
-  s.gx = __fadd_rn(__fsub_rn(r0.x, (float)(tx * kTile)), r0.z);
-  s.gy = __fadd_rn(__fsub_rn(r0.y, (float)(ty * kTile)), r0.w);
+  const unsigned lo_bits = __float_as_uint(r0.z), box_bits = __float_as_uint(r0.w);
+  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&lo_bits));
+  const float2 box = __half22float2(*reinterpret_cast<const __half2*>(&box_bits));
+  s.gx = __fadd_rn(__fsub_rn(r0.x, (float)(tx * kTile)), lo.x);
+  s.gy = __fadd_rn(__fsub_rn(r0.y, (float)(ty * kTile)), lo.y);
+  s.hx = box.x;
+  s.hy = box.y;
   s.beta = r1.y;
   s.ns1 = __fmul_rn(r1.x, -kLog2e);
   s.ns2 = __fmul_rn(r1.z, -kLog2e);
@@ -97,11 +105,52 @@ struct PixArgs {
   unsigned long long* counters;
 };
 
+// Pixel layout: each warp owns a compact BW x BH block of the tile (8x4,
+// 8x8 or 16x8 pixels for PPT = 1, 2, 4); lane l of warp w holds pixels
+// (bx0 + l % BW, by0 + l / BW + k * LROWS), k < PPT.
 template <int PPT>
 struct TileGeom {
   static constexpr int NT = 256 / PPT;
-  static constexpr int ROWS = 16 / PPT;
+  static constexpr int NW = NT / 32;
+  static constexpr int BW = PPT == 4 ? 16 : 8;
+  static constexpr int BH = 32 * PPT / BW;
+  static constexpr int LROWS = 32 / BW;
+  static constexpr int BX = 16 / BW;
 };
+
+struct WarpPix {
+  int lx, ly0;            // first pixel of the lane (tile-relative)
+  float x0, x1, y0, y1;   // the warp's pixel-centre box (tile-relative)
+};
+
+template <int PPT>
+__device__ __forceinline__ WarpPix warp_pixels(int t) {
+  using G = TileGeom<PPT>;
+  const int w = t >> 5, l = t & 31;
+  const int bx0 = (w % G::BX) * G::BW, by0 = (w / G::BX) * G::BH;
+  WarpPix p;
+  p.lx = bx0 + l % G::BW;
+  p.ly0 = by0 + l / G::BW;
+  p.x0 = (float)bx0 + 0.5f;
+  p.x1 = (float)(bx0 + G::BW) - 0.5f;
+  p.y0 = (float)by0 + 0.5f;
+  p.y1 = (float)(by0 + G::BH) - 0.5f;
+  return p;
+}
+
+// Tile-relative bounding box of the region where alpha >= 1/255 can hold
+// (o exp(-q) >= 1/255 <=> q <= ln(255 o)), from the half extents the
+// projection stores (inflated far beyond the fp32 error of the per-pixel
+// alpha and rounded up): a warp whose pixel box misses it would have
+// skipped the Gaussian at every pixel anyway, so culling by it leaves every
+// result bit-identical.
+__device__ __forceinline__ float4 alpha_box(const Staged& st) {
+  return make_float4(st.gx - st.hx, st.gx + st.hx, st.gy - st.hy, st.gy + st.hy);
+}
+
+__device__ __forceinline__ bool box_misses(const float4& b, const WarpPix& p) {
+  return (b.x > p.x1) | (b.y < p.x0) | (b.z > p.y1) | (b.w < p.y0);
+}
 
 // ---------------------------------------------------------------------------
 // forward
@@ -111,26 +160,27 @@ __global__ void __launch_bounds__(256 / PPT)
 k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
              int32_t* dev_status) {
-  constexpr int NT = TileGeom<PPT>::NT, ROWS = TileGeom<PPT>::ROWS;
-  __shared__ float4 sA[NT], sB[NT];
+  using G = TileGeom<PPT>;
+  constexpr int NT = G::NT;
+  __shared__ float4 sBox[NT], sA[NT], sB[NT];
   __shared__ float sC[NT];
-  __shared__ float s_red[NT / 32];
+  __shared__ float s_red[G::NW];
   const int lw = leaf.x1 - leaf.x0;
   const int ltile = blockIdx.x;
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile], end = ranges[2 * ltile + 1];
   const int t = threadIdx.x;
-  const int lx = t & 15, ly0 = t >> 4;
-  const float fpx = (float)lx + 0.5f;
+  const WarpPix wp = warp_pixels<PPT>(t);
+  const float fpx = (float)wp.lx + 0.5f;
   float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
   int lastp[PPT];
   bool done[PPT], inside[PPT];
   unsigned n_vis = 0, n_kept = 0;
 #pragma unroll
   for (int k = 0; k < PPT; ++k) {
-    const int ly = ly0 + k * ROWS;
+    const int ly = wp.ly0 + k * G::LROWS;
     fpy[k] = (float)ly + 0.5f;
-    inside[k] = (tx * kTile + lx < W) && (ty * kTile + ly < H);
+    inside[k] = (tx * kTile + wp.lx < W) && (ty * kTile + ly < H);
     done[k] = !inside[k];
     T[k] = 1.0f;
     Cr[k] = Cg[k] = Cb[k] = 0.0f;
@@ -143,15 +193,24 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     if (__syncthreads_count(mine_done) == NT) break;
     const int64_t e = base + t;
     if (e < end) {
-      const Staged s = stage_record(rec, vals[e], tx, ty);
-      sA[t] = make_float4(s.gx, s.gy, s.beta, s.ns1);
-      sB[t] = make_float4(s.ns2, s.opac, s.r, s.g);
-      sC[t] = s.b;
+      const Staged st = stage_record(rec, vals[e], tx, ty);
+      sBox[t] = alpha_box(st);
+      sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
+      sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+      sC[t] = st.b;
     }
     __syncthreads();
+    if (__all_sync(0xffffffffu, mine_done)) continue;  // nothing left for this warp
     const int cnt = (int)min((int64_t)NT, end - base);
     const int pos0 = (int)(base - begin);
     for (int j = 0; j < cnt; ++j) {
+      if ((j & 31) == 31) {
+        bool d_all = true;
+#pragma unroll
+        for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
+        if (__all_sync(0xffffffffu, d_all)) break;
+      }
+      if (box_misses(sBox[j], wp)) continue;  // warp-uniform
       const float4 A = sA[j];
       const float4 B = sB[j];
       const float Bb = sC[j];
@@ -185,7 +244,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
 #pragma unroll
   for (int k = 0; k < PPT; ++k) {
     if (!inside[k]) continue;
-    const int x = tx * kTile + lx, y = ty * kTile + ly0 + k * ROWS;
+    const int x = tx * kTile + wp.lx, y = ty * kTile + wp.ly0 + k * G::LROWS;
     const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
     if (px.img) {
       px.img[o] = Cr[k];
@@ -211,7 +270,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     __syncthreads();
     if (t == 0) {
       float tot = 0.0f;
-      for (int w = 0; w < NT / 32; ++w) tot += s_red[w];
+      for (int w = 0; w < G::NW; ++w) tot += s_red[w];
       px.loss_tiles[(int64_t)ty * TW + tx] = tot * px.norm;
     }
   }
@@ -318,8 +377,9 @@ __global__ void __launch_bounds__(256 / PPT)
 k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, PixArgs px,
              float* __restrict__ g2d, int32_t* dev_status) {
-  constexpr int NT = TileGeom<PPT>::NT, ROWS = TileGeom<PPT>::ROWS;
-  __shared__ float4 sA[NT], sB[NT];
+  using G = TileGeom<PPT>;
+  constexpr int NT = G::NT;
+  __shared__ float4 sBox[NT], sA[NT], sB[NT];
   __shared__ float4 sC[NT];       // {b, s1, s2, slot bits}
   __shared__ float sg[NT][12];
   __shared__ int s_touched[NT];
@@ -329,8 +389,8 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile];
   const int t = threadIdx.x, lane = t & 31;
-  const int lx = t & 15, ly0 = t >> 4;
-  const float fpx = (float)lx + 0.5f;
+  const WarpPix wp = warp_pixels<PPT>(t);
+  const float fpx = (float)wp.lx + 0.5f;
   float fpy[PPT], T[PPT], Ar[PPT], Ag[PPT], Ab[PPT], gr[PPT], gg[PPT], gb[PPT];
   int lastp[PPT];
   if (t == 0) s_maxlast = 0;
@@ -340,9 +400,9 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   int mylast = 0;
 #pragma unroll
   for (int k = 0; k < PPT; ++k) {
-    const int ly = ly0 + k * ROWS;
+    const int ly = wp.ly0 + k * G::LROWS;
     fpy[k] = (float)ly + 0.5f;
-    const int x = tx * kTile + lx, y = ty * kTile + ly;
+    const int x = tx * kTile + wp.lx, y = ty * kTile + ly;
     Ar[k] = Ag[k] = Ab[k] = 0.0f;
     if (x < W && y < H) {
       const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
@@ -358,7 +418,8 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     }
     mylast = max(mylast, lastp[k]);
   }
-  atomicMax(&s_maxlast, mylast);
+  const int warp_last = __reduce_max_sync(0xffffffffu, mylast);
+  if (lane == 0) atomicMax(&s_maxlast, warp_last);
   __syncthreads();
   const int tile_last = s_maxlast;
   unsigned n_vis = 0, n_kept = 0;
@@ -368,13 +429,17 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     const int cnt = bend - bstart;
     if (t < cnt) {
       const int pos = bend - 1 - t;
-      const Staged s = stage_record(rec, vals[begin + pos], tx, ty);
-      sA[t] = make_float4(s.gx, s.gy, s.beta, s.ns1);
-      sB[t] = make_float4(s.ns2, s.opac, s.r, s.g);
-      sC[t] = make_float4(s.b, s.s1, s.s2, __int_as_float(s.slot));
+      const Staged st = stage_record(rec, vals[begin + pos], tx, ty);
+      sBox[t] = alpha_box(st);
+      sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
+      sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+      sC[t] = make_float4(st.b, st.s1, st.s2, __int_as_float(st.slot));
     }
     __syncthreads();
-    for (int j = 0; j < cnt; ++j) {
+    // positions at or beyond every lane's `last` need no work in this warp
+    const int jstart = max(0, bend - warp_last);
+    for (int j = jstart; j < cnt; ++j) {
+      if (box_misses(sBox[j], wp)) continue;  // warp-uniform
       const int pos = bend - 1 - j;
       const float4 A = sA[j];
       const float4 B = sB[j];

@@ -22,6 +22,7 @@ constexpr int kIPT = 8;
 constexpr int kSortTile = kSortThreads * kIPT;  // 4096 items
 constexpr int kWarps = kSortThreads / 32;
 constexpr int kRadix = 256;
+constexpr int kLookWin = 16;  // predecessors read per look-back round trip
 
 struct SortPlan {
   int passes;
@@ -67,6 +68,26 @@ k_hist(const K* __restrict__ keys, int64_t n, SortPlan plan, unsigned long long*
   for (int p = 0; p < plan.passes; ++p)
     for (int d = threadIdx.x; d < kRadix; d += kSortThreads)
       if (sh[p][d]) atomicAdd(&hist[p * kRadix + d], (unsigned long long)sh[p][d]);
+}
+
+// Digit histograms of keys 0..n_tiles-1 whose multiplicities are the range
+// lengths (ranges[2t+1] - ranges[2t]): the keys need not be read.
+__global__ void __launch_bounds__(256)
+k_hist_from_ranges(const int64_t* __restrict__ ranges, int64_t n_tiles, SortPlan plan,
+                   unsigned long long* __restrict__ hist) {
+  __shared__ unsigned long long sh[8][kRadix];
+  for (int e = threadIdx.x; e < 8 * kRadix; e += 256) (&sh[0][0])[e] = 0;
+  __syncthreads();
+  for (int64_t t = (int64_t)blockIdx.x * 256 + threadIdx.x; t < n_tiles; t += (int64_t)gridDim.x * 256) {
+    const unsigned long long c = (unsigned long long)(ranges[2 * t + 1] - ranges[2 * t]);
+    if (!c) continue;
+    for (int p = 0; p < plan.passes; ++p)
+      atomicAdd(&sh[p][((uint64_t)t >> plan.shift[p]) & ((1u << plan.bits[p]) - 1)], c);
+  }
+  __syncthreads();
+  for (int p = 0; p < plan.passes; ++p)
+    for (int d = threadIdx.x; d < kRadix; d += 256)
+      if (sh[p][d]) atomicAdd(&hist[p * kRadix + d], sh[p][d]);
 }
 
 template <class K>
@@ -160,25 +181,36 @@ k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool 
   tstart = block_exclusive_scan<unsigned, kWarps>(tid < kRadix ? tcount : 0u, S.scan, &ttot);
   if (tid < kRadix) {
     S.tex[tid] = tstart;
-    // look back over earlier tiles for this digit
+    // look back over earlier tiles for this digit, kLookWin predecessors per
+    // round trip (their status words are loaded together)
     long long excl = 0;
     if (tile > 0) {
       int64_t j = tile - 1;
       int spins = 0;
-      while (j >= 0) {
-        const unsigned long long wv = ld_relaxed(status + j * kRadix + tid);
-        const unsigned flag = (unsigned)(wv >> 62);
-        if (flag == 0) {
-          if (++spins > kSpinCap) {
-            dev_flag(dev_status, GS_DEV_TIMEOUT);
-            break;
+      bool found = false, timed_out = false;
+      while (j >= 0 && !found && !timed_out) {
+        unsigned long long wv[kLookWin];
+#pragma unroll
+        for (int i = 0; i < kLookWin; ++i)
+          wv[i] = (j - i >= 0) ? ld_relaxed(status + (j - i) * kRadix + tid) : kFlagInc;
+#pragma unroll
+        for (int i = 0; i < kLookWin; ++i) {
+          if (found || timed_out) break;
+          unsigned long long w = wv[i];
+          while ((w >> 62) == 0) {  // not yet published: wait for this one
+            if (++spins > kSpinCap) {
+              dev_flag(dev_status, GS_DEV_TIMEOUT);
+              timed_out = true;
+              break;
+            }
+            __nanosleep(64);
+            w = ld_relaxed(status + (j - i) * kRadix + tid);
           }
-          __nanosleep(64);
-          continue;
+          if (timed_out) break;
+          excl += (long long)(w & kValMask);
+          if ((w >> 62) == 2) found = true;
         }
-        excl += (long long)(wv & kValMask);
-        if (flag == 2) break;
-        --j;
+        j -= kLookWin;
       }
       st_relaxed(status + tile * kRadix + tid, kFlagInc | (unsigned long long)(excl + tcount));
     }
@@ -249,7 +281,7 @@ SortWs<K> carve_sort(void* ws, size_t cap, int64_t n, const SortPlan& p) {
 template <class K>
 gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool stall, int64_t n,
                     int begin_bit, int end_bit, void* ws, size_t ws_bytes, int32_t* dev_status,
-                    cudaStream_t s) {
+                    cudaStream_t s, const int64_t* ranges = nullptr, int64_t n_tiles = 0) {
   const int kbits = (int)(8 * sizeof(K));
   if (n < 0 || begin_bit < 0 || end_bit > kbits || begin_bit > end_bit) return GS_ERR_ARG;
   if (n == 0) return GS_OK;
@@ -268,8 +300,14 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
   }
   GS_TRY(cudaMemsetAsync((char*)ws + w.zero_begin, 0, w.zero_bytes, s));
   const int64_t tiles = (n + kSortTile - 1) / kSortTile;
-  const int hist_blocks = (int)(tiles < 1184 ? tiles : 1184);
-  k_hist<K><<<hist_blocks, kSortThreads, 0, s>>>(first_k, n, plan, w.hist);
+  if (ranges) {
+    const int64_t hb = (n_tiles + 255) / 256;
+    k_hist_from_ranges<<<(unsigned)(hb < 296 ? (hb > 0 ? hb : 1) : 296), 256, 0, s>>>(
+        ranges, n_tiles, plan, w.hist);
+  } else {
+    const int hist_blocks = (int)(tiles < 1184 ? tiles : 1184);
+    k_hist<K><<<hist_blocks, kSortThreads, 0, s>>>(first_k, n, plan, w.hist);
+  }
   GS_LAUNCH_CHECK();
   const size_t smem = sizeof(SortSmem<K>);
   GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -309,6 +347,16 @@ extern "C" gs_status gs_sort_keys(uint64_t* keys, int32_t* vals, int64_t n, int3
                                   gs_stream stream) {
   return sort_impl<uint64_t>(nullptr, keys, vals, false, false, n, begin_bit, end_bit, ws,
                              ws_bytes, dev_status, to_stream(stream));
+}
+
+extern "C" gs_status gs_sort_tiles(uint32_t* tile_keys, int32_t* vals, int64_t n,
+                                   const int64_t* ranges, int64_t n_tiles, void* ws,
+                                   size_t ws_bytes, int32_t* dev_status, gs_stream stream) {
+  if (n < 0 || n_tiles < 0 || (n_tiles > 0 && !ranges)) return GS_ERR_ARG;
+  if (n_tiles > ((int64_t)1 << 32)) return GS_ERR_UNSUPPORTED;
+  const int bits = n_tiles > 1 ? 64 - __builtin_clzll((unsigned long long)(n_tiles - 1)) : 0;
+  return sort_impl<uint32_t>(nullptr, tile_keys, vals, false, false, n, 0, bits, ws, ws_bytes,
+                             dev_status, to_stream(stream), ranges, n_tiles);
 }
 
 extern "C" gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys, int32_t* vals,

@@ -47,7 +47,8 @@ def _carved_bytes(sizes):
 @dataclasses.dataclass
 class ViewStats:
     n_cand: int
-    n_isect: int
+    n_isect: int          # entries of the (tight) tile lists
+    n_isect_square: int   # tiles of the candidates' plain 3-sigma squares
     n_leaves: int
     leaves: np.ndarray
     leaf_isect: np.ndarray
@@ -166,8 +167,9 @@ class Stepper:
         rec = torch.empty(cap * 12, dtype=torch.float32, device=dev)
         rect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
         dkey = torch.empty(cap, dtype=torch.int32, device=dev)
+        sq_d = torch.zeros(1, dtype=torch.int64, device=dev)
         proj = B.gs_proj(cap, n_cand_d.data_ptr(), cand_idx.data_ptr(), slot.data_ptr(),
-                         rec.data_ptr(), rect.data_ptr(), dkey.data_ptr())
+                         rec.data_ptr(), rect.data_ptr(), dkey.data_ptr(), sq_d.data_ptr())
         sat = torch.empty((TH + 1) * (TW + 1), dtype=torch.int64, device=dev)
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
         tk = clk.tic("project")
@@ -177,10 +179,13 @@ class Stepper:
         del ws
         sat_h = torch.empty(sat.shape, dtype=torch.int64, pin_memory=True)
         nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+        sq_h = torch.empty(1, dtype=torch.int64, pin_memory=True)
         sat_h.copy_(sat, non_blocking=True)
         nc_h.copy_(n_cand_d, non_blocking=True)
+        sq_h.copy_(sq_d, non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()   # the one sync per view
         C = int(nc_h[0])
+        n_square = int(sq_h[0])
         sat_np = sat_h.numpy().reshape(TH + 1, TW + 1)
         ctx = dict(proj=proj, cand_idx=cand_idx, slot=slot, rec=rec, rect=rect, depth_key=dkey,
                    sat=sat, sat_host=sat_np, n_cand=C, TW=TW, TH=TH, cam=cam)
@@ -268,7 +273,7 @@ class Stepper:
             lb_bits = B.local_tile_bits(L)
             if I > 0 and lb_bits > 0:
                 tk = clk.tic("sort_tiles")
-                B.gs_sort_keys32(None, keys, vals, I, 0, lb_bits, 0, sort_ws, st)
+                B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
                 clk.toc(tk)
                 launches += 1 + 2 * ((lb_bits + 15) // 16)
             tk = clk.tic("raster_fwd")
@@ -320,7 +325,8 @@ class Stepper:
         peak = torch.cuda.max_memory_allocated(dev) - base_alloc
         if resident_target:
             peak += target.numel() * target.element_size()
-        return ViewStats(n_cand=C, n_isect=int(li.sum()), n_leaves=len(lv), leaves=lv,
+        return ViewStats(n_cand=C, n_isect=int(li.sum()), n_isect_square=n_square,
+                         n_leaves=len(lv), leaves=lv,
                          leaf_isect=li, leaf_bytes=lb, over_budget=ov, peak_ws_bytes=int(peak),
                          arena_bytes=int(arena_bytes), launches=launches)
 

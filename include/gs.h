@@ -11,7 +11,7 @@
  *                    estimated load fits a byte budget
  *   for each Leaf:
  *     gs_bin_tiles   one entry per (candidate, tile) in depth order
- *     gs_sort_keys32 stable radix sort on the Leaf-local tile index
+ *     gs_sort_tiles  stable radix sort on the Leaf-local tile index
  *                    -> per-tile lists (the order of the 64-bit keys
  *                    tile << 32 | depth)
  *     gs_raster_fwd  front-to-back compositing (+ fused L1 loss)
@@ -105,12 +105,21 @@ typedef struct gs_model {
 /* Per-view projected state of the candidates (Gaussians that can touch the
  * view), in ascending Gaussian index.  Written by gs_project.
  * rec: 12 floats per candidate = three float4
- *   {u_hi, v_hi, u_lo, v_lo}  screen position as an unevaluated fp32 pair
+ *   {u_hi, v_hi, lo, box}     u = u_hi + lo.x, v = v_hi + lo.y with lo a
+ *                             half2 of fp16 corrections (bits in a float);
+ *                             box a half2 of the alpha box half extents
+ *                             (hx, hy) rounded up
  *   {s1, beta, s2, opacity}   q = s1 (dx + beta dy)^2 + s2 dy^2 with
  *                             s1 = a/2, beta = b/a, s2 = 1/(2 Sigma'_11),
  *                             (a, b, c) the conic Sigma'^-1
  *   {R, G, B, depth}
- * rect: tiles [x0, x1) x [y0, y1) covered by the 3-sigma square. */
+ * rect: tiles [x0, x1) x [y0, y1): those of the 3-sigma square whose
+ * pixel-centre box [16 tx + 0.5, 16 tx + 15.5] x [16 ty + 0.5, 16 ty + 15.5]
+ * meets the bounding box of the region where alpha can reach 1/255 (the
+ * ellipse q <= ln(255 o), inflated by 1e-4 relative + 1e-4 in q and 0.01
+ * px).  Every tile left out would skip the Gaussian at every pixel, so the
+ * image and gradients equal those of the plain 3-sigma square.  A Gaussian
+ * with 255 o < exp(-1e-4) is never a candidate. */
 typedef struct gs_proj {
   int64_t capacity;     /* candidate capacity of the arrays below (>= n) */
   int32_t* n_cand;      /* device scalar */
@@ -119,6 +128,10 @@ typedef struct gs_proj {
   float* rec;           /* device [capacity][12], 16-byte aligned */
   int16_t* rect;        /* device [capacity][4] */
   uint32_t* depth_key;  /* device [capacity] bits of fp32 camera depth */
+  /* optional device scalar (NULL = off): total tiles of the candidates'
+   * plain 3-sigma squares (clamped to the grid), the conventional count of
+   * Gaussian-tile intersections */
+  unsigned long long* square_isect;
 } gs_proj;
 
 /* A rectangle of tiles, half-open. */
@@ -219,6 +232,17 @@ gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys,
                          int32_t end_bit, uint32_t flags, void* ws,
                          size_t ws_bytes, int32_t* dev_status,
                          gs_stream stream);
+
+/* Sort of binned entries by tile: (tile_keys, vals) with tile_keys in
+ * [0, n_tiles) stably by key (bits [0, ceil(log2 n_tiles))), the digit
+ * histograms taken from ranges (key t occurs ranges[2t+1] - ranges[2t]
+ * times, as gs_bin_tiles writes them) instead of a pass over the keys.
+ * Workspace: gs_sort_workspace_size(n, 4, 0, ceil(log2 n_tiles)).  Keys
+ * that disagree with the ranges give an unspecified order (a scatter out of
+ * range sets GS_DEV_BOUNDS and is skipped). */
+gs_status gs_sort_tiles(uint32_t* tile_keys, int32_t* vals, int64_t n,
+                        const int64_t* ranges, int64_t n_tiles, void* ws,
+                        size_t ws_bytes, int32_t* dev_status, gs_stream stream);
 
 /* Allocation-free variant of gs_sort_keys32 (no counterpart on the pages;
  * an addition of this library).  For callers that cannot allocate device

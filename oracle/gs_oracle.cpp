@@ -146,6 +146,7 @@ struct Forward3D {
   double J[6], T[6], S2[3], S2p[3], det, conic[3];
   double radius;
   int64_t rect[4];
+  int64_t square_tiles;
   double dir[3], dnorm, rgb_raw[3], rgb[3], opac;
   bool cand;
   uint8_t flags;
@@ -225,11 +226,34 @@ void project_one(const double* params, int64_t n_pad, int32_t D, const Cam& k,
   double r3 = 3.0 * std::sqrt(lam);
   f.radius = std::ceil(r3);
   if (std::fabs(r3 - std::nearbyint(r3)) <= 1e-9 * r3) f.flags |= OR_F_RADIUS_NEAR;
-  // tiles covered by the closed square [u-r, u+r] x [v-r, v+r]
-  f.rect[0] = clampi(floor_div_tile(f.u - f.radius), 0, TW);
-  f.rect[1] = clampi(floor_div_tile(f.v - f.radius), 0, TH);
-  f.rect[2] = clampi(floor_div_tile(f.u + f.radius) + 1, 0, TW);
-  f.rect[3] = clampi(floor_div_tile(f.v + f.radius) + 1, 0, TH);
+  // tiles covered by the closed square [u-r, u+r] x [v-r, v+r] ...
+  int64_t sq[4] = {floor_div_tile(f.u - f.radius), floor_div_tile(f.v - f.radius),
+                   floor_div_tile(f.u + f.radius) + 1, floor_div_tile(f.v + f.radius) + 1};
+  f.square_tiles = (clampi(sq[2], 0, TW) - clampi(sq[0], 0, TW)) *
+                   (clampi(sq[3], 0, TH) - clampi(sq[1], 0, TH));
+  // ... restricted to the tiles whose pixel-centre box (16 t + 0.5 .. 16 t
+  // + 15.5) meets the bounding box of {alpha >= 1/255} = {q <= ln(255 o)},
+  // inflated (1e-4 relative + 1e-4 in q, 0.01 px) beyond fp32 rounding.
+  // Reading: a tile outside it would skip the Gaussian at every pixel, so
+  // the image and gradients are those of the plain square.
+  f.opac = 1.0 / (1.0 + std::exp(-P(10)));
+  double lq = std::log(255.0 * f.opac);
+  if (std::fabs(lq + 1e-4) <= 1e-9) f.flags |= OR_F_RADIUS_NEAR;
+  if (!(lq > -1e-4)) return;  // alpha never reaches 1/255
+  double qb = std::max(lq, 0.0) * 1.0001 + 1e-4;
+  double hx = std::sqrt(2.0 * qb * f.S2p[0]) + 0.01;
+  double hy = std::sqrt(2.0 * qb * f.S2p[2]) + 0.01;
+  double e[4] = {(f.u - hx - 15.5) / kTile, (f.v - hy - 15.5) / kTile,
+                 (f.u + hx - 0.5) / kTile, (f.v + hy - 0.5) / kTile};
+  for (double x : e)
+    if (std::fabs(x - std::nearbyint(x)) <= 1e-9 * std::max(1.0, std::fabs(x)))
+      f.flags |= OR_F_RADIUS_NEAR;
+  int64_t bb[4] = {(int64_t)std::ceil(e[0]), (int64_t)std::ceil(e[1]),
+                   (int64_t)std::floor(e[2]) + 1, (int64_t)std::floor(e[3]) + 1};
+  f.rect[0] = clampi(std::max(sq[0], bb[0]), 0, TW);
+  f.rect[1] = clampi(std::max(sq[1], bb[1]), 0, TH);
+  f.rect[2] = clampi(std::min(sq[2], bb[2]), 0, TW);
+  f.rect[3] = clampi(std::min(sq[3], bb[3]), 0, TH);
   if (f.rect[0] >= f.rect[2] || f.rect[1] >= f.rect[3]) return;
   // view-dependent colour from SH at the direction camera centre -> mean
   double cc[3];
@@ -248,7 +272,6 @@ void project_one(const double* params, int64_t n_pad, int32_t D, const Cam& k,
     f.rgb[ch] = f.rgb_raw[ch] < 0 ? 0.0 : f.rgb_raw[ch];
     if (std::fabs(f.rgb_raw[ch]) <= 1e-9) f.flags |= OR_F_CLAMP_NEAR;
   }
-  f.opac = 1.0 / (1.0 + std::exp(-P(10)));
   f.cand = true;
 }
 
@@ -363,6 +386,7 @@ int64_t or_project(const double* params, int64_t n, int64_t n_pad, int32_t D,
     r[OR_OPAC] = f.opac;
     r[OR_R] = f.rgb[0]; r[OR_G] = f.rgb[1]; r[OR_BL] = f.rgb[2];
     r[OR_S00] = f.S2p[0]; r[OR_S01] = f.S2p[1]; r[OR_S11] = f.S2p[2];
+    r[OR_SQUARE] = (double)f.square_tiles;
     for (int j = 0; j < 4; ++j) rect[4 * i + j] = (int32_t)f.rect[j];
     float dz = (float)f.tcam[2];
     uint32_t bits;

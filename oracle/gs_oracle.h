@@ -28,6 +28,7 @@ enum {
   OR_A = 4, OR_B = 5, OR_C = 6, OR_OPAC = 7,
   OR_R = 8, OR_G = 9, OR_BL = 10,
   OR_S00 = 11, OR_S01 = 12, OR_S11 = 13,
+  OR_SQUARE = 14,  /* tiles of the plain 3-sigma square (clamped) */
   OR_REC = 16
 };
 

@@ -25,8 +25,15 @@ def encode_records(rec_c):
     u, v = rec_c[:, 0], rec_c[:, 1]
     uh, vh = u.astype(np.float32), v.astype(np.float32)
     out[:, 0], out[:, 1] = uh, vh
-    out[:, 2] = (u - uh.astype(np.float64)).astype(np.float32)
-    out[:, 3] = (v - vh.astype(np.float64)).astype(np.float32)
+    lo = np.stack([u - uh.astype(np.float64), v - vh.astype(np.float64)], 1).astype(np.float16)
+    out[:, 2] = lo.view(np.float32).reshape(-1)
+    # alpha box half extents (the library's bound), fp16 rounded up
+    lq = np.log(255.0 * rec_c[:, 7])
+    qb = np.maximum(lq, 0.0) * 1.0001 + 1e-4
+    hx = (np.sqrt(2 * qb * rec_c[:, 11]) + 0.01).astype(np.float32)
+    hy = (np.sqrt(2 * qb * rec_c[:, 13]) + 0.01).astype(np.float32)
+    box = np.stack([_half_up(hx), _half_up(hy)], 1)
+    out[:, 3] = box.view(np.float32).reshape(-1)
     a, b = rec_c[:, 4], rec_c[:, 5]
     S11 = rec_c[:, 13]
     out[:, 4] = (0.5 * a).astype(np.float32)
@@ -38,15 +45,26 @@ def encode_records(rec_c):
     return out
 
 
+def _half_up(x):
+    """fp32 -> fp16 rounded towards +inf."""
+    h = np.asarray(x, np.float32).astype(np.float16)
+    low = h.astype(np.float32) < x
+    h[low] = np.nextafter(h[low], np.float16(np.inf))
+    return h
+
+
 def decode_records(rec12):
     """Library records [C][12] -> dict of fp64 fields (conic reconstructed)."""
-    r = np.asarray(rec12, np.float32).reshape(-1, 12).astype(np.float64)
+    raw = np.asarray(rec12, np.float32).reshape(-1, 12)
+    r = raw.astype(np.float64)
+    lo = np.ascontiguousarray(raw[:, 2]).view(np.float16).reshape(-1, 2).astype(np.float64)
+    box = np.ascontiguousarray(raw[:, 3]).view(np.float16).reshape(-1, 2).astype(np.float64)
     s1, beta, s2 = r[:, 4], r[:, 5], r[:, 6]
     a = 2 * s1
     b = beta * a
     c = 2 * s2 + beta * beta * a
-    return dict(u=r[:, 0] + r[:, 2], v=r[:, 1] + r[:, 3], a=a, b=b, c=c, s1=s1, beta=beta,
-                s2=s2, opac=r[:, 7], rgb=r[:, 8:11], depth=r[:, 11])
+    return dict(u=r[:, 0] + lo[:, 0], v=r[:, 1] + lo[:, 1], a=a, b=b, c=c, s1=s1, beta=beta,
+                s2=s2, opac=r[:, 7], rgb=r[:, 8:11], depth=r[:, 11], hx=box[:, 0], hy=box[:, 1])
 
 
 class ProjBuffers:
@@ -61,10 +79,11 @@ class ProjBuffers:
         self.rec = torch.zeros(cap * 12, dtype=torch.float32, device=dev)
         self.rect = torch.zeros(cap * 4, dtype=torch.int16, device=dev)
         self.depth_key = torch.zeros(cap, dtype=torch.int32, device=dev)
+        self.square = torch.zeros(1, dtype=torch.int64, device=dev)
         b = B()
         self.struct = b.gs_proj(cap, self.n_cand.data_ptr(), self.cand_idx.data_ptr(),
                                 self.slot.data_ptr(), self.rec.data_ptr(), self.rect.data_ptr(),
-                                self.depth_key.data_ptr())
+                                self.depth_key.data_ptr(), self.square.data_ptr())
 
     @classmethod
     def from_oracle(cls, pr, n):

@@ -199,25 +199,67 @@ def test_cull_rules(oracle_mod):
         assert oracle_mod.project(p, 1, 0, cam)["is_cand"][0] == expect, mean
 
 
+def _alpha_box(rec):
+    """Half extents of the inflated alpha >= 1/255 box (the reading's bound)."""
+    lq = np.log(255.0 * rec[:, 7])
+    q = np.maximum(lq, 0.0) * 1.0001 + 1e-4
+    return np.sqrt(2 * q * rec[:, 11]) + 0.01, np.sqrt(2 * q * rec[:, 13]) + 0.01
+
+
 def test_rect_and_depth_key_bruteforce(oracle_mod):
     sc, cams = synth.tiny_oracle_scene(0)
     cam = cams[0]
     pr = oracle_mod.project(sc.params, sc.n, 0, cam)
     TW, TH = oracle_mod.grid(cam)
     rec, rect = pr["rec"], pr["rect"]
+    hx, hy = _alpha_box(rec)
     for j in range(0, len(rec), 7):
         u, v, r = rec[j, 0], rec[j, 1], rec[j, 3]
+        # tiles meeting the closed 3-sigma square AND whose pixel-centre box
+        # meets the alpha box
         tiles = [(tx, ty) for ty in range(TH) for tx in range(TW)
                  if tx * 16 <= u + r and (tx + 1) * 16 > u - r
-                 and ty * 16 <= v + r and (ty + 1) * 16 > v - r]
+                 and ty * 16 <= v + r and (ty + 1) * 16 > v - r
+                 and tx * 16 + 0.5 <= u + hx[j] and tx * 16 + 15.5 >= u - hx[j]
+                 and ty * 16 + 0.5 <= v + hy[j] and ty * 16 + 15.5 >= v - hy[j]]
         xs = [a for a, _ in tiles]
         ys = [b for _, b in tiles]
         assert (rect[j] == [min(xs), min(ys), max(xs) + 1, max(ys) + 1]).all()
         assert len(tiles) == (rect[j, 2] - rect[j, 0]) * (rect[j, 3] - rect[j, 1])
+        square = [(tx, ty) for ty in range(TH) for tx in range(TW)
+                  if tx * 16 <= u + r and (tx + 1) * 16 > u - r
+                  and ty * 16 <= v + r and (ty + 1) * 16 > v - r]
+        assert rec[j, 14] == len(square)
     keys = np.float32(rec[:, 2]).view(np.uint32)
     assert (keys == pr["key"]).all()
     # candidates = the Gaussians that pass; ascending index
     assert (np.diff(pr["cand_idx"]) > 0).all()
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_tight_rect_leaves_image_unchanged(oracle_mod, seed):
+    """Reading: dropping the tiles of the 3-sigma square that the alpha box
+    misses changes neither image nor transmittance (those tiles skip the
+    Gaussian at every pixel); only the list positions (`last`) move."""
+    sc, cams = synth.tiny_scene(n=60, width=96, height=80, sh_degree=3, seed=seed,
+                                scale_px=(1.0, 9.0), opacity=(0.01, 0.99))
+    cam = cams[0]
+    TW, TH = oracle_mod.grid(cam)
+    pr = oracle_mod.project(sc.params.astype(np.float64), sc.n, 3, cam)
+    rec = pr["rec"]
+    u, v, r = rec[:, 0], rec[:, 1], rec[:, 3]
+    square = np.stack([np.floor((u - r) / 16), np.floor((v - r) / 16),
+                       np.floor((u + r) / 16) + 1, np.floor((v + r) / 16) + 1], 1)
+    square = np.clip(square, 0, [TW, TH, TW, TH]).astype(np.int32)
+    assert ((pr["rect"][:, :2] >= square[:, :2]) & (pr["rect"][:, 2:] <= square[:, 2:])).all()
+    tiles = np.arange(TW * TH, dtype=np.int32)
+    outs = []
+    for rc in (pr["rect"], square):
+        off, vals = oracle_mod.tile_lists(rc, pr["key"], TW, tiles)
+        outs.append((len(vals), oracle_mod.raster_fwd(rec, TW, cam.width, cam.height, tiles, off, vals)))
+    (n_tight, a), (n_sq, b) = outs
+    assert n_tight < n_sq
+    assert (a["img"] == b["img"]).all() and (a["T"] == b["T"]).all()
 
 
 # ---------------------------------------------------------------------------
