@@ -22,6 +22,7 @@ GS_ERR_TIMEOUT = -4
 GS_ERR_BOUNDS = -5
 GS_ERR_UNSUPPORTED = -6
 GS_SORT_IOTA = 1
+GS_SORT_ONESWEEP = 2
 GS_SORT_TEST_STALL = 0x80000000
 TILE = 16
 

@@ -27,6 +27,8 @@ struct BwdCam {
 
 struct AdamK {
   float lr, b1, b2, omb1, omb2, eps, bc1, bc2;
+  float step;     // lr / (1 - b1^t)
+  float rsbc2;    // 1 / sqrt(1 - b2^t)
 };
 
 __device__ __forceinline__ void adam_update(float* __restrict__ p, float* __restrict__ m,
@@ -36,9 +38,7 @@ __device__ __forceinline__ void adam_update(float* __restrict__ p, float* __rest
   const float vv = fmaf(a.b2, v[idx], a.omb2 * g * g);
   m[idx] = mm;
   v[idx] = vv;
-  const float mh = mm / a.bc1;
-  const float vh = vv / a.bc2;
-  p[idx] = p[idx] - a.lr * mh / (sqrtf(vh) + a.eps);
+  p[idx] = fmaf(-a.step, __fdividef(mm, fmaf(sqrtf(vv), a.rsbc2, a.eps)), p[idx]);
 }
 
 // Gradients of one candidate.  `emit(plane, g)` receives every parameter's
@@ -320,10 +320,12 @@ __device__ __forceinline__ void sh_term(int k, double x, double y, double z, dou
   }
 }
 
+// p -= lr (m / bc1) / (sqrt(v / bc2) + eps), with the bias corrections
+// folded into two host-computed factors and one fast division (2 ulp).
 __device__ __forceinline__ void adam_vals(float& p, float& m, float& v, float g, const AdamK& a) {
   m = fmaf(a.b1, m, a.omb1 * g);
   v = fmaf(a.b2, v, a.omb2 * g * g);
-  p = p - a.lr * (m / a.bc1) / (sqrtf(v / a.bc2) + a.eps);
+  p = fmaf(-a.step, __fdividef(m, fmaf(sqrtf(v), a.rsbc2, a.eps)), p);
 }
 
 // Fused path, stage 2: one thread per Gaussian streams its planes once:
@@ -378,14 +380,19 @@ k_adam_fused(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v
 #pragma unroll
     for (int kk = 0; kk < GK; ++kk) {
       if (k0 + kk >= KS) continue;
-      double Y, Yx, Yy, Yz;
-      sh_term(k0 + kk, dx, dy, dz, Y, Yx, Yy, Yz);
-      const double w = gc[0] * pv[kk][0] + gc[1] * pv[kk][1] + gc[2] * pv[kk][2];
-      ddx = fma(w, Yx, ddx);
-      ddy = fma(w, Yy, ddy);
-      ddz = fma(w, Yz, ddz);
+      float gy[3] = {0.f, 0.f, 0.f};
+      if (cand) {
+        double Y, Yx, Yy, Yz;
+        sh_term(k0 + kk, dx, dy, dz, Y, Yx, Yy, Yz);
+        const double w = gc[0] * pv[kk][0] + gc[1] * pv[kk][1] + gc[2] * pv[kk][2];
+        ddx = fma(w, Yx, ddx);
+        ddy = fma(w, Yy, ddy);
+        ddz = fma(w, Yz, ddz);
 #pragma unroll
-      for (int ch = 0; ch < 3; ++ch) adam_vals(pv[kk][ch], mv[kk][ch], vv[kk][ch], (float)(gc[ch] * Y), a);
+        for (int ch = 0; ch < 3; ++ch) gy[ch] = (float)(gc[ch] * Y);
+      }
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) adam_vals(pv[kk][ch], mv[kk][ch], vv[kk][ch], gy[ch], a);
     }
 #pragma unroll
     for (int kk = 0; kk < GK; ++kk)
@@ -466,8 +473,12 @@ bool make_adam(const gs_adam_args* args, AdamK* a) {
   a->omb1 = (float)(1.0 - args->beta1);
   a->omb2 = (float)(1.0 - args->beta2);
   a->eps = (float)args->eps;
-  a->bc1 = (float)(1.0 - pow(args->beta1, (double)args->step));
-  a->bc2 = (float)(1.0 - pow(args->beta2, (double)args->step));
+  const double bc1 = 1.0 - pow(args->beta1, (double)args->step);
+  const double bc2 = 1.0 - pow(args->beta2, (double)args->step);
+  a->bc1 = (float)bc1;
+  a->bc2 = (float)bc2;
+  a->step = (float)(args->lr / bc1);
+  a->rsbc2 = (float)(1.0 / sqrt(bc2));
   return true;
 }
 

@@ -122,7 +122,7 @@ extern "C" gs_status gs_leaf_load_model(int32_t tile_bits, gs_load_model* out) {
   out->bytes_per_isect = 16 + (passes + 1) / 2;
   out->bytes_per_pixel = 44;
   out->bytes_per_tile = 16;
-  out->fixed_bytes = 8 * 256 * 8 + 64 * 4 + (int64_t)passes * 256 * 8 + 16 * 256;
+  out->fixed_bytes = 2 * 8 * 256 * 8 + 64 * 4 + (int64_t)passes * 256 * 8 + 16 * 256;
   out->align = 512;
   return GS_OK;
 }

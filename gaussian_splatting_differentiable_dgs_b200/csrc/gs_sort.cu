@@ -17,12 +17,27 @@
 namespace gs {
 namespace {
 
-constexpr int kSortThreads = 512;
-constexpr int kIPT = 8;
-constexpr int kSortTile = kSortThreads * kIPT;  // 4096 items
+// Launch shape (overridable at build time for tuning sweeps).
+#ifndef GS_SORT_THREADS
+#define GS_SORT_THREADS 512
+#endif
+#ifndef GS_SORT_IPT
+#define GS_SORT_IPT 8
+#endif
+#ifndef GS_SORT_WIN
+#define GS_SORT_WIN 4
+#endif
+#ifndef GS_SORT_MINB
+#define GS_SORT_MINB 2
+#endif
+
+constexpr int kSortThreads = GS_SORT_THREADS;
+constexpr int kIPT = GS_SORT_IPT;
+constexpr int kSortTile = kSortThreads * kIPT;
 constexpr int kWarps = kSortThreads / 32;
 constexpr int kRadix = 256;
-constexpr int kLookWin = 16;  // predecessors read per look-back round trip
+constexpr int kLookWin = GS_SORT_WIN;  // predecessors read per look-back round trip
+static_assert(kSortThreads >= kRadix, "one thread per digit");
 
 struct SortPlan {
   int passes;
@@ -90,6 +105,17 @@ k_hist_from_ranges(const int64_t* __restrict__ ranges, int64_t n_tiles, SortPlan
       if (sh[p][d]) atomicAdd(&hist[p * kRadix + d], sh[p][d]);
 }
 
+// Exclusive scan of each pass's digit histogram (one block per pass):
+// start[p][d] = number of keys with a smaller digit in pass p.
+__global__ void __launch_bounds__(kRadix)
+k_hist_scan(const unsigned long long* __restrict__ hist, unsigned long long* __restrict__ start) {
+  __shared__ unsigned long long s_scan[kRadix / 32 + 1];
+  const int p = blockIdx.x, d = threadIdx.x;
+  unsigned long long tot;
+  start[p * kRadix + d] =
+      block_exclusive_scan<unsigned long long, kRadix / 32>(hist[p * kRadix + d], s_scan, &tot);
+}
+
 template <class K>
 struct SortSmem {
   K keys[kSortTile];
@@ -98,12 +124,11 @@ struct SortSmem {
   long long gbase[kRadix];           // global position of the tile's first item of digit d
   unsigned int tex[kRadix];          // tile-local exclusive offset of digit d
   unsigned int scan[kWarps + 1];
-  unsigned long long hscan[kWarps + 1];
   unsigned int tile;
 };
 
 template <class K>
-__global__ void __launch_bounds__(kSortThreads)
+__global__ void __launch_bounds__(kSortThreads, GS_SORT_MINB)
 k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool iota,
            K* __restrict__ dst_k, int32_t* __restrict__ dst_v, int64_t n, int shift, int bits,
            const unsigned long long* __restrict__ hist, unsigned long long* __restrict__ status,
@@ -167,17 +192,9 @@ k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool 
       st_relaxed(st, kFlagAgg | tcount);
     }
   }
-  // global start of each digit (exclusive scan of the histogram)
-  unsigned long long hcount = tid < kRadix ? hist[tid] : 0ull;
-  unsigned long long htot;
-  unsigned long long hstart = 0;
+  // global start of each digit (precomputed per pass)
+  const unsigned long long hstart = tid < kRadix ? hist[tid] : 0ull;
   unsigned tstart = 0, ttot;
-  {
-    // both scans over the first 256 threads; the rest contribute zeros
-    unsigned long long hx = block_exclusive_scan<unsigned long long, kWarps>(
-        tid < kRadix ? hcount : 0ull, S.hscan, &htot);
-    hstart = hx;
-  }
   tstart = block_exclusive_scan<unsigned, kWarps>(tid < kRadix ? tcount : 0u, S.scan, &ttot);
   if (tid < kRadix) {
     S.tex[tid] = tstart;
@@ -188,6 +205,24 @@ k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool 
       int64_t j = tile - 1;
       int spins = 0;
       bool found = false, timed_out = false;
+      {
+        // the nearest predecessor alone first: usually it is already final
+        unsigned long long w = ld_relaxed(status + j * kRadix + tid);
+        while ((w >> 62) == 0) {
+          if (++spins > kSpinCap) {
+            dev_flag(dev_status, GS_DEV_TIMEOUT);
+            timed_out = true;
+            break;
+          }
+          __nanosleep(32);
+          w = ld_relaxed(status + j * kRadix + tid);
+        }
+        if (!timed_out) {
+          excl += (long long)(w & kValMask);
+          found = (w >> 62) == 2;
+        }
+        --j;
+      }
       while (j >= 0 && !found && !timed_out) {
         unsigned long long wv[kLookWin];
 #pragma unroll
@@ -243,6 +278,129 @@ k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Chain-free digit pass (upsweep / scan / downsweep): per-tile digit counts
+// are stored digit-major, scanned per digit across tiles, and each tile then
+// scatters to its precomputed offsets.  No tile waits on another.
+// ---------------------------------------------------------------------------
+template <class K>
+__global__ void __launch_bounds__(kSortThreads)
+k_upsweep(const K* __restrict__ keys, int64_t n, int shift, int bits, int64_t tiles,
+          unsigned int* __restrict__ counts) {
+  __shared__ unsigned int sh[kRadix];
+  const unsigned mask = (1u << bits) - 1u;
+  for (int d = threadIdx.x; d < kRadix; d += kSortThreads) sh[d] = 0;
+  __syncthreads();
+  const int64_t base = (int64_t)blockIdx.x * kSortTile;
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const int64_t idx = base + (int64_t)k * kSortThreads + threadIdx.x;
+    if (idx < n) atomicAdd(&sh[digit_of(keys[idx], shift, mask)], 1u);
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < kRadix; d += kSortThreads)
+    counts[(int64_t)d * tiles + blockIdx.x] = sh[d];
+}
+
+// Block d: counts[d][0..tiles) -> exclusive prefix + global start of digit d.
+__global__ void __launch_bounds__(1024)
+k_scan_tiles(unsigned int* __restrict__ counts, int64_t tiles,
+             const unsigned long long* __restrict__ start) {
+  __shared__ unsigned long long s_scan[1024 / 32 + 1];
+  const int d = blockIdx.x;
+  unsigned int* row = counts + (int64_t)d * tiles;
+  unsigned long long carry = start[d];
+  for (int64_t t0 = 0; t0 < tiles; t0 += 1024) {
+    const int64_t t = t0 + threadIdx.x;
+    const unsigned long long c = t < tiles ? row[t] : 0ull;
+    unsigned long long tot;
+    const unsigned long long ex = block_exclusive_scan<unsigned long long, 32>(c, s_scan, &tot);
+    if (t < tiles) row[t] = (unsigned int)(carry + ex);
+    carry += tot;
+  }
+}
+
+template <class K>
+__global__ void __launch_bounds__(kSortThreads, GS_SORT_MINB)
+k_downsweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool iota,
+            K* __restrict__ dst_k, int32_t* __restrict__ dst_v, int64_t n, int shift, int bits,
+            const unsigned int* __restrict__ offsets, int64_t tiles, int32_t* dev_status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SortSmem<K>& S = *reinterpret_cast<SortSmem<K>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const unsigned mask = (1u << bits) - 1u;
+  const int64_t tile = blockIdx.x;
+  for (int e = tid; e < kWarps * kRadix; e += kSortThreads) (&S.wh[0][0])[e] = 0;
+  // global base of each digit for this tile (stored 32-bit: n < 2^32)
+  if (tid < kRadix) S.gbase[tid] = offsets[(int64_t)tid * tiles + tile];
+  __syncthreads();
+  const int64_t base = tile * kSortTile;
+  K key[kIPT];
+  int32_t val[kIPT];
+  unsigned dig[kIPT];
+  unsigned rank[kIPT];
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const int64_t idx = base + w * (32 * kIPT) + k * 32 + lane;
+    if (idx < n) {
+      key[k] = src_k[idx];
+      val[k] = iota ? (int32_t)idx : src_v[idx];
+      dig[k] = digit_of(key[k], shift, mask);
+    } else {
+      key[k] = 0;
+      val[k] = 0;
+      dig[k] = kRadix;
+    }
+  }
+  const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const unsigned peers = __match_any_sync(0xffffffffu, dig[k]);
+    unsigned cnt = 0;
+    if (dig[k] < kRadix) cnt = S.wh[w][dig[k]];
+    __syncwarp();
+    if (dig[k] < kRadix && lane == __ffs(peers) - 1) S.wh[w][dig[k]] = cnt + __popc(peers);
+    rank[k] = cnt + __popc(peers & lt_mask);
+    __syncwarp();
+  }
+  __syncthreads();
+  unsigned tcount = 0;
+  if (tid < kRadix) {
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) {
+      const unsigned c = S.wh[ww][tid];
+      S.wh[ww][tid] = tcount;
+      tcount += c;
+    }
+  }
+  unsigned ttot;
+  const unsigned tstart = block_exclusive_scan<unsigned, kWarps>(tid < kRadix ? tcount : 0u, S.scan, &ttot);
+  if (tid < kRadix) S.tex[tid] = tstart;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    if (dig[k] < kRadix) {
+      const unsigned pos = S.tex[dig[k]] + S.wh[w][dig[k]] + rank[k];
+      S.keys[pos] = key[k];
+      S.vals[pos] = val[k];
+    }
+  }
+  __syncthreads();
+  const int64_t rem = n - base;
+  const int count = rem < kSortTile ? (int)rem : kSortTile;
+  for (int e = tid; e < count; e += kSortThreads) {
+    const K kk = S.keys[e];
+    const unsigned d = digit_of(kk, shift, mask);
+    const int64_t gpos = S.gbase[d] + (e - (int64_t)S.tex[d]);
+    if (gpos < 0 || gpos >= n) {
+      dev_flag(dev_status, GS_DEV_BOUNDS);
+      continue;
+    }
+    dst_k[gpos] = kk;
+    dst_v[gpos] = S.vals[e];
+  }
+}
+
 template <class K>
 __global__ void k_copy_pairs(const K* __restrict__ sk, K* __restrict__ dk, int32_t* __restrict__ dv,
                              const int32_t* __restrict__ sv, bool iota, int64_t n) {
@@ -257,9 +415,11 @@ struct SortWs {
   K* alt_k;
   int32_t* alt_v;
   unsigned long long* hist;
+  unsigned long long* hstart;
   unsigned int* tickets;
   unsigned long long* status;
-  size_t zero_begin, zero_bytes, bytes;
+  unsigned int* counts;
+  size_t zero_begin, zero_small, zero_bytes, bytes;
 };
 
 template <class K>
@@ -269,10 +429,15 @@ SortWs<K> carve_sort(void* ws, size_t cap, int64_t n, const SortPlan& p) {
   s.alt_k = cv.take<K>(n > 0 ? n : 1);
   s.alt_v = cv.take<int32_t>(n > 0 ? n : 1);
   const int64_t tiles = (n + kSortTile - 1) / kSortTile;
+  s.hstart = cv.take<unsigned long long>((size_t)8 * kRadix);
   s.hist = cv.take<unsigned long long>((size_t)8 * kRadix);
   s.zero_begin = (size_t)((char*)s.hist - (char*)ws);
   s.tickets = cv.take<unsigned int>(64);
+  // the onesweep look-back words, or (same region) the per-tile digit
+  // counts of the upsweep/downsweep passes
+  s.zero_small = cv.off - s.zero_begin;   // histograms and tickets
   s.status = cv.take<unsigned long long>((size_t)(p.passes > 0 ? p.passes : 1) * (tiles > 0 ? tiles : 1) * kRadix);
+  s.counts = reinterpret_cast<unsigned int*>(s.status);
   s.bytes = cv.off;
   s.zero_bytes = s.bytes - s.zero_begin;
   return s;
@@ -281,7 +446,9 @@ SortWs<K> carve_sort(void* ws, size_t cap, int64_t n, const SortPlan& p) {
 template <class K>
 gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool stall, int64_t n,
                     int begin_bit, int end_bit, void* ws, size_t ws_bytes, int32_t* dev_status,
-                    cudaStream_t s, const int64_t* ranges = nullptr, int64_t n_tiles = 0) {
+                    cudaStream_t s, const int64_t* ranges = nullptr, int64_t n_tiles = 0,
+                    bool chained = false) {
+  chained = chained || stall;
   const int kbits = (int)(8 * sizeof(K));
   if (n < 0 || begin_bit < 0 || end_bit > kbits || begin_bit > end_bit) return GS_ERR_ARG;
   if (n == 0) return GS_OK;
@@ -298,7 +465,7 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
     GS_LAUNCH_CHECK();
     return GS_OK;
   }
-  GS_TRY(cudaMemsetAsync((char*)ws + w.zero_begin, 0, w.zero_bytes, s));
+  GS_TRY(cudaMemsetAsync((char*)ws + w.zero_begin, 0, chained ? w.zero_bytes : w.zero_small, s));
   const int64_t tiles = (n + kSortTile - 1) / kSortTile;
   if (ranges) {
     const int64_t hb = (n_tiles + 255) / 256;
@@ -309,17 +476,42 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
     k_hist<K><<<hist_blocks, kSortThreads, 0, s>>>(first_k, n, plan, w.hist);
   }
   GS_LAUNCH_CHECK();
+  k_hist_scan<<<plan.passes, kRadix, 0, s>>>(w.hist, w.hstart);
+  GS_LAUNCH_CHECK();
   const size_t smem = sizeof(SortSmem<K>);
-  GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  // a shared-memory carveout large enough for several blocks per SM
+  if (chained) {
+    GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared));
+  } else {
+    GS_TRY(cudaFuncSetAttribute(k_downsweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    GS_TRY(cudaFuncSetAttribute(k_downsweep<K>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared));
+  }
   const K* sk = first_k;
   const int32_t* sv = vals;
   bool siota = iota;
   for (int p = 0; p < plan.passes; ++p) {
     K* dk = (p & 1) ? keys : w.alt_k;
     int32_t* dv = (p & 1) ? vals : w.alt_v;
-    k_onesweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
-        sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.hist + (size_t)p * kRadix,
-        w.status + (size_t)p * tiles * kRadix, w.tickets + p, stall && p == 0, dev_status);
+    if (chained) {
+      k_onesweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
+          sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.hstart + (size_t)p * kRadix,
+          w.status + (size_t)p * tiles * kRadix, w.tickets + p, stall && p == 0, dev_status);
+      GS_LAUNCH_CHECK();
+      sk = dk;
+      sv = dv;
+      siota = false;
+      continue;
+    }
+    k_upsweep<K><<<(unsigned)tiles, kSortThreads, 0, s>>>(sk, n, plan.shift[p], plan.bits[p], tiles,
+                                                            w.counts);
+    GS_LAUNCH_CHECK();
+    k_scan_tiles<<<kRadix, 1024, 0, s>>>(w.counts, tiles, w.hstart + (size_t)p * kRadix);
+    GS_LAUNCH_CHECK();
+    k_downsweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
+        sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.counts, tiles, dev_status);
     GS_LAUNCH_CHECK();
     sk = dk;
     sv = dv;
@@ -363,10 +555,11 @@ extern "C" gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys, int
                                     int64_t n, int32_t begin_bit, int32_t end_bit, uint32_t flags,
                                     void* ws, size_t ws_bytes, int32_t* dev_status,
                                     gs_stream stream) {
-  if (flags & ~(GS_SORT_IOTA | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
+  if (flags & ~(GS_SORT_IOTA | GS_SORT_ONESWEEP | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
   return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0,
                              (flags & GS_SORT_TEST_STALL) != 0, n, begin_bit, end_bit, ws,
-                             ws_bytes, dev_status, to_stream(stream));
+                             ws_bytes, dev_status, to_stream(stream), nullptr, 0,
+                             (flags & GS_SORT_ONESWEEP) != 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -412,7 +605,7 @@ extern "C" gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* k
                                             int32_t* vals, int64_t n, int32_t begin_bit,
                                             int32_t end_bit, uint32_t flags, int32_t* dev_status,
                                             gs_stream stream) {
-  if (flags & ~(GS_SORT_IOTA | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
+  if (flags & ~(GS_SORT_IOTA | GS_SORT_ONESWEEP | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
   if (n < 0) return GS_ERR_ARG;
   if (n > GS_SORT_NOALLOC_MAX_N) return GS_ERR_CAPACITY;
   if (n == 0) return GS_OK;
@@ -424,5 +617,6 @@ extern "C" gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* k
     return GS_ERR_CAPACITY;
   return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0,
                              (flags & GS_SORT_TEST_STALL) != 0, n, begin_bit, end_bit, scratch,
-                             kNoAllocScratchBytes, dev_status, to_stream(stream));
+                             kNoAllocScratchBytes, dev_status, to_stream(stream), nullptr, 0,
+                             (flags & GS_SORT_ONESWEEP) != 0);
 }

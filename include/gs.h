@@ -210,14 +210,19 @@ gs_status gs_project(const gs_model* model, const gs_camera* cam,
                      gs_stream stream);
 
 /* ---- 2. radix sorts ------------------------------------------------------
- * Stable LSD radix sort (onesweep: one histogram pass, then one pass per
- * digit with decoupled look-back) of (key, value) pairs on key bits
- * [begin_bit, end_bit).  The result is in keys[], vals[] (in place).  For
- * the 32-bit variant, keys_in (if not NULL) is read instead of keys on the
- * first pass, and flag GS_SORT_IOTA makes the input values 0..n-1.
- * Bounded look-back waits: on expiry GS_DEV_TIMEOUT is set and the call
- * returns without hanging. */
+ * Stable LSD radix sort of (key, value) pairs on key bits [begin_bit,
+ * end_bit), 8-bit digits, an even number of passes: a histogram of every
+ * digit in one pass over the keys, then per digit either three kernels
+ * (per-tile digit counts, a scan of the counts per digit, a stable scatter
+ * per tile; the default) or, with GS_SORT_ONESWEEP, one kernel with
+ * decoupled look-back across tiles (Adinets & Merrill's "onesweep").  The
+ * result is in keys[], vals[] (in place).  For the 32-bit variant, keys_in
+ * (if not NULL) is read instead of keys on the first pass, and flag
+ * GS_SORT_IOTA makes the input values 0..n-1.  The onesweep look-back waits
+ * are bounded: on expiry GS_DEV_TIMEOUT is set and the call returns
+ * without hanging. */
 #define GS_SORT_IOTA 1u
+#define GS_SORT_ONESWEEP 2u
 /* Test hook of the bounded wait: the first tile of the first pass does not
  * publish its counts, so every later tile's look-back runs out and reports
  * GS_DEV_TIMEOUT (the result is then unspecified).  Never set otherwise. */

@@ -294,6 +294,7 @@ struct PixelOut {
   int32_t last, n_eval;
   uint8_t flags;
   uint64_t sig;
+  double T_err;  // relative error bound of an fp32 evaluation of T
 };
 
 void composite_pixel(const double* rec, const int32_t* list, int64_t len,
@@ -304,6 +305,7 @@ void composite_pixel(const double* rec, const int32_t* list, int64_t len,
   o.n_eval = 0;
   o.flags = 0;
   o.sig = 0x12345;
+  o.T_err = 0.0;
   int32_t n_kept = 0;
   for (int64_t p = 0; p < len; ++p) {
     const double* r = rec + (int64_t)list[p] * OR_REC;
@@ -338,6 +340,10 @@ void composite_pixel(const double* rec, const int32_t* list, int64_t len,
     }
     if (kept) kept->push_back({(int32_t)p, alpha, o.T, G, dx, dy, clamped});
     for (int ch = 0; ch < 3; ++ch) o.C[ch] += r[OR_R + ch] * alpha * o.T;
+    // fp32 T = prod (1 - alpha): each factor carries the relative error of
+    // its alpha (exp and q rounding, unless clamped) scaled by
+    // alpha / (1 - alpha), plus one rounding of the product
+    o.T_err += (clamped ? 0.0 : alpha / (1.0 - alpha) * (3e-7 + 5e-7 * q)) + 1.2e-7;
     o.T = Tn;
     o.last = (int32_t)p + 1;
     n_kept++;
@@ -458,7 +464,7 @@ int32_t or_raster_fwd(int64_t C, const double* rec, int32_t TW, int32_t W,
                       int32_t H, const int32_t* tiles, int64_t n_tiles,
                       const int64_t* offsets, const int32_t* vals, double* img,
                       double* T_final, int32_t* last, uint8_t* pflags,
-                      int32_t* n_eval, uint64_t* sig) {
+                      int32_t* n_eval, uint64_t* sig, double* T_err) {
   (void)C;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t k = 0; k < n_tiles; ++k) {
@@ -470,7 +476,7 @@ int32_t or_raster_fwd(int64_t C, const double* rec, int32_t TW, int32_t W,
       int64_t o = k * 256 + j;
       PixelOut po;
       if (x >= W || y >= H) {
-        po = PixelOut{{0, 0, 0}, 1.0, 0, 0, OR_P_INVALID, 0};
+        po = PixelOut{{0, 0, 0}, 1.0, 0, 0, OR_P_INVALID, 0, 0.0};
       } else {
         composite_pixel(rec, list, len, x + 0.5, y + 0.5, po, nullptr);
       }
@@ -480,6 +486,7 @@ int32_t or_raster_fwd(int64_t C, const double* rec, int32_t TW, int32_t W,
       pflags[o] = po.flags;
       n_eval[o] = po.n_eval;
       sig[o] = po.sig;
+      if (T_err) T_err[o] = po.T_err;
     }
   }
   return 0;

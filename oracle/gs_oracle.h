@@ -70,12 +70,13 @@ int64_t or_tile_lists_scatter(int64_t C, const int32_t* rect,
 /* Front-to-back compositing of requested tiles.  Per tile k outputs are
  * compact: img[k][3][256], T_final[k][256], last[k][256], pflags[k][256],
  * n_eval[k][256] (list entries visited), sig[k][256] (hash of every
- * discrete decision taken for the pixel). */
+ * discrete decision taken for the pixel), T_err[k][256] (optional: bound of
+ * the relative error of an fp32 evaluation of T_final). */
 int32_t or_raster_fwd(int64_t C, const double* rec, int32_t TW, int32_t W,
                       int32_t H, const int32_t* tiles, int64_t n_tiles,
                       const int64_t* offsets, const int32_t* vals, double* img,
                       double* T_final, int32_t* last, uint8_t* pflags,
-                      int32_t* n_eval, uint64_t* sig);
+                      int32_t* n_eval, uint64_t* sig, double* T_err);
 
 /* Reverse blend: accumulates dL/d{u,v,a,b,c,o,R,G,B} per candidate into
  * g2d[C][9] given dL/dpixel[k][3][256] for the requested tiles. */

@@ -72,7 +72,7 @@ def lib():
         L.or_tile_lists_scatter.restype = i64
         L.or_tile_lists_scatter.argtypes = [i64, p, p, i32, i32, p, p]
         L.or_raster_fwd.argtypes = [i64, p, i32, i32, i32, p, i64, p, p,
-                                    p, p, p, p, p, p]
+                                    p, p, p, p, p, p, p]
         L.or_raster_bwd.argtypes = [i64, p, i32, i32, i32, p, i64, p, p, p, p]
         L.or_project_bwd.argtypes = [p, i64, i32, p, i64, p, p, p]
         L.or_leaf_partition.restype = i32
@@ -171,13 +171,14 @@ def raster_fwd(rec_c, TW, W, H, tiles, off, vals):
     fl = np.zeros((k, 256), np.uint8)
     ne = np.zeros((k, 256), np.int32)
     sig = np.zeros((k, 256), np.uint64)
+    terr = np.zeros((k, 256))
     vals = np.ascontiguousarray(vals, np.int32)
     if len(vals) == 0:
         vals = np.zeros(1, np.int32)
     lib().or_raster_fwd(len(rec_c), _p(rec_c), TW, W, H, _p(tiles), k,
                         _p(np.ascontiguousarray(off, np.int64)), _p(vals),
-                        _p(img), _p(T), _p(last), _p(fl), _p(ne), _p(sig))
-    return dict(img=img, T=T, last=last, flags=fl, n_eval=ne, sig=sig)
+                        _p(img), _p(T), _p(last), _p(fl), _p(ne), _p(sig), _p(terr))
+    return dict(img=img, T=T, last=last, flags=fl, n_eval=ne, sig=sig, T_err=terr)
 
 
 def raster_bwd(rec_c, TW, W, H, tiles, off, vals, dL_dpix, g2d=None):
