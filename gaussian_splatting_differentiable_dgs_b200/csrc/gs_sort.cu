@@ -292,10 +292,27 @@ k_upsweep(const K* __restrict__ keys, int64_t n, int shift, int bits, int64_t ti
   for (int d = threadIdx.x; d < kRadix; d += kSortThreads) sh[d] = 0;
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kSortTile;
+  if constexpr (sizeof(K) == 4 && kIPT % 4 == 0) {
+    // four keys per 128-bit load where the whole quad is in range
 #pragma unroll
-  for (int k = 0; k < kIPT; ++k) {
-    const int64_t idx = base + (int64_t)k * kSortThreads + threadIdx.x;
-    if (idx < n) atomicAdd(&sh[digit_of(keys[idx], shift, mask)], 1u);
+    for (int k = 0; k < kIPT / 4; ++k) {
+      const int64_t q = base + 4 * ((int64_t)k * kSortThreads + threadIdx.x);
+      if (q + 3 < n) {
+        const uint4 v4 = *reinterpret_cast<const uint4*>(keys + q);
+        atomicAdd(&sh[(v4.x >> shift) & mask], 1u);
+        atomicAdd(&sh[(v4.y >> shift) & mask], 1u);
+        atomicAdd(&sh[(v4.z >> shift) & mask], 1u);
+        atomicAdd(&sh[(v4.w >> shift) & mask], 1u);
+      } else {
+        for (int64_t i = q; i < n && i < q + 4; ++i) atomicAdd(&sh[digit_of(keys[i], shift, mask)], 1u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kIPT; ++k) {
+      const int64_t idx = base + (int64_t)k * kSortThreads + threadIdx.x;
+      if (idx < n) atomicAdd(&sh[digit_of(keys[idx], shift, mask)], 1u);
+    }
   }
   __syncthreads();
   for (int d = threadIdx.x; d < kRadix; d += kSortThreads)
@@ -401,6 +418,109 @@ k_downsweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool
   }
 }
 
+// Leaner downsweep for 32-bit keys: (key, value) staged as one 64-bit word,
+// one per-digit delta (global start - tile-local start), loops sized to the
+// pass's active digits.
+struct DownSmem32 {
+  unsigned long long kv[kSortTile];
+  unsigned int wh[kWarps][kRadix];
+  int gdelta[kRadix];
+  unsigned int scan[kWarps + 1];
+};
+
+__global__ void __launch_bounds__(kSortThreads, GS_SORT_MINB)
+k_downsweep32(const uint32_t* __restrict__ src_k, const int32_t* __restrict__ src_v, bool iota,
+              uint32_t* __restrict__ dst_k, int32_t* __restrict__ dst_v, int n, int shift,
+              int bits, const unsigned int* __restrict__ offsets, int tiles, int32_t* dev_status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  DownSmem32& S = *reinterpret_cast<DownSmem32*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const unsigned mask = (1u << bits) - 1u;
+  const int nd = 1 << bits;  // active digits
+  const int tile = blockIdx.x;
+  if (nd >= 4) {
+    const int q = nd / 4;  // uint4 words per warp row
+    for (int e = tid; e < kWarps * q; e += kSortThreads)
+      reinterpret_cast<uint4*>(&S.wh[e / q][0])[e % q] = make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    for (int e = tid; e < kWarps * nd; e += kSortThreads) S.wh[e / nd][e % nd] = 0u;
+  }
+  int gb = 0;
+  if (tid < nd) gb = (int)offsets[(int64_t)tid * tiles + tile];
+  __syncthreads();
+  const int base = tile * kSortTile;
+  const bool full = base + kSortTile <= n;
+  uint32_t key[kIPT];
+  int32_t val[kIPT];
+  unsigned dig[kIPT];
+  unsigned rank[kIPT];
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const int idx = base + w * (32 * kIPT) + k * 32 + lane;
+    if (full || idx < n) {
+      key[k] = src_k[idx];
+      val[k] = iota ? idx : src_v[idx];
+      dig[k] = (key[k] >> shift) & mask;
+    } else {
+      key[k] = 0u;
+      val[k] = 0;
+      dig[k] = kRadix;
+    }
+  }
+  const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const unsigned peers = __match_any_sync(0xffffffffu, dig[k]);
+    const bool ok = dig[k] < kRadix;
+    const unsigned cnt = ok ? S.wh[w][dig[k]] : 0u;
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) S.wh[w][dig[k]] = cnt + __popc(peers);
+    rank[k] = cnt + __popc(peers & lt_mask);
+    __syncwarp();
+  }
+  __syncthreads();
+  unsigned tcount = 0;
+  if (tid < nd) {
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) {
+      const unsigned c = S.wh[ww][tid];
+      S.wh[ww][tid] = tcount;
+      tcount += c;
+    }
+  }
+  unsigned ttot;
+  const unsigned tstart = block_exclusive_scan<unsigned, kWarps>(tid < nd ? tcount : 0u, S.scan, &ttot);
+  if (tid < nd) {
+    S.gdelta[tid] = gb - (int)tstart;
+    // fold the tile-local digit start into the per-warp offsets
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) S.wh[ww][tid] += tstart;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k)
+    if (dig[k] < kRadix)
+      S.kv[S.wh[w][dig[k]] + rank[k]] =
+          (unsigned long long)key[k] | ((unsigned long long)(uint32_t)val[k] << 32);
+  __syncthreads();
+  const int count = full ? kSortTile : n - base;
+#pragma unroll
+  for (int k = 0; k < kIPT; ++k) {
+    const int e = k * kSortThreads + tid;
+    if (full || e < count) {
+      const unsigned long long kv = S.kv[e];
+      const uint32_t kk = (uint32_t)kv;
+      const int gpos = S.gdelta[(kk >> shift) & mask] + e;
+      if ((unsigned)gpos >= (unsigned)n) {
+        dev_flag(dev_status, GS_DEV_BOUNDS);
+        continue;
+      }
+      dst_k[gpos] = kk;
+      dst_v[gpos] = (int32_t)(kv >> 32);
+    }
+  }
+}
+
 template <class K>
 __global__ void k_copy_pairs(const K* __restrict__ sk, K* __restrict__ dk, int32_t* __restrict__ dv,
                              const int32_t* __restrict__ sv, bool iota, int64_t n) {
@@ -479,10 +599,17 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
   k_hist_scan<<<plan.passes, kRadix, 0, s>>>(w.hist, w.hstart);
   GS_LAUNCH_CHECK();
   const size_t smem = sizeof(SortSmem<K>);
+  // the lean 32-bit downsweep indexes with int
+  const bool use32 = sizeof(K) == 4 && n <= (int64_t)INT32_MAX - kSortTile;
   // a shared-memory carveout large enough for several blocks per SM
   if (chained) {
     GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared));
+  } else if (use32) {
+    GS_TRY(cudaFuncSetAttribute(k_downsweep32, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(DownSmem32)));
+    GS_TRY(cudaFuncSetAttribute(k_downsweep32, cudaFuncAttributePreferredSharedMemoryCarveout,
                                 cudaSharedmemCarveoutMaxShared));
   } else {
     GS_TRY(cudaFuncSetAttribute(k_downsweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -510,8 +637,14 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
     GS_LAUNCH_CHECK();
     k_scan_tiles<<<kRadix, 1024, 0, s>>>(w.counts, tiles, w.hstart + (size_t)p * kRadix);
     GS_LAUNCH_CHECK();
-    k_downsweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
-        sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.counts, tiles, dev_status);
+    if (use32) {
+      k_downsweep32<<<(unsigned)tiles, kSortThreads, sizeof(DownSmem32), s>>>(
+          reinterpret_cast<const uint32_t*>(sk), sv, siota, reinterpret_cast<uint32_t*>(dk), dv,
+          (int)n, plan.shift[p], plan.bits[p], w.counts, (int)tiles, dev_status);
+    } else {
+      k_downsweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
+          sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.counts, tiles, dev_status);
+    }
     GS_LAUNCH_CHECK();
     sk = dk;
     sv = dv;
