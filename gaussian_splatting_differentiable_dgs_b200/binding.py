@@ -95,7 +95,7 @@ class gs_adam_args(C.Structure):
 
 
 SYMBOLS = [
-    "gs_version", "gs_status_string", "gs_check",
+    "gs_version", "gs_status_string", "gs_check", "gs_launch_counter",
     "gs_project_workspace_size", "gs_project",
     "gs_sort_workspace_size", "gs_sort_keys", "gs_sort_keys32", "gs_sort_tiles",
     "gs_sort_keys32_noalloc",
@@ -115,6 +115,7 @@ def _load():
     P = C.POINTER
     sig = {
         "gs_version": (i32, []),
+        "gs_launch_counter": (i64, []),
         "gs_status_string": (C.c_char_p, [i32]),
         "gs_check": (i32, [p, p]),
         "gs_project_workspace_size": (sz, [i64, i32, i32]),
@@ -161,6 +162,11 @@ def status_string(s: int) -> str:
 
 def version() -> int:
     return _L.gs_version()
+
+
+def gs_launch_counter() -> int:
+    """Kernel launches the library has issued in this process."""
+    return int(_L.gs_launch_counter())
 
 
 def ptr(x) -> int | None:

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <vector>
 
 #include "gs.h"
@@ -79,9 +80,17 @@ void plan_leaves(Plan& p, gs_rect root) {
   }
 }
 
+std::atomic<int64_t> g_launches{0};
+
 }  // namespace
 
+namespace gs {
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace gs
+
 extern "C" int32_t gs_version(void) { return 1; }
+
+extern "C" int64_t gs_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
 
 extern "C" const char* gs_status_string(gs_status s) {
   switch (s) {

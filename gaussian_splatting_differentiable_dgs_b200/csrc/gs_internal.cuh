@@ -12,7 +12,17 @@
     if (e_ != cudaSuccess) return GS_ERR_CUDA;         \
   } while (0)
 
-#define GS_LAUNCH_CHECK() GS_TRY(cudaGetLastError())
+namespace gs {
+// process-wide count of kernel launches issued by this library (gs_host.cpp)
+void note_launch();
+}  // namespace gs
+
+// every kernel launch of the library is followed by exactly one of these
+#define GS_LAUNCH_CHECK()          \
+  do {                             \
+    gs::note_launch();             \
+    GS_TRY(cudaGetLastError());    \
+  } while (0)
 
 namespace gs {
 

@@ -156,7 +156,7 @@ class Stepper:
         st = self.dev_status
         base_alloc = torch.cuda.memory_allocated(dev)
         torch.cuda.reset_peak_memory_stats(dev)
-        launches = 0
+        launch0 = B.gs_launch_counter()
 
         # ---- projection (+ counts, SAT) ---------------------------------
         n = m.n
@@ -175,7 +175,6 @@ class Stepper:
         tk = clk.tic("project")
         B.gs_project(mod, camS, proj, sat, ws, st)
         clk.toc(tk)
-        launches += 3 if n > 0 else 2
         del ws
         sat_h = torch.empty(sat.shape, dtype=torch.int64, pin_memory=True)
         nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
@@ -200,7 +199,6 @@ class Stepper:
             tk = clk.tic("sort_depth")
             B.gs_depth_order(proj, C, order, drect, ws, st)
             clk.toc(tk)
-            launches += 1 + 4 + 1
             del ws
         ctx["depth_order"] = order
         ctx["depth_rect"] = drect
@@ -269,17 +267,14 @@ class Stepper:
             B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1), ranges,
                            bin_ws, st)
             clk.toc(tk)
-            launches += 2 if (C > 0 and I > 0) else 1
             lb_bits = B.local_tile_bits(L)
             if I > 0 and lb_bits > 0:
                 tk = clk.tic("sort_tiles")
                 B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
                 clk.toc(tk)
-                launches += 1 + 2 * ((lb_bits + 15) // 16)
             tk = clk.tic("raster_fwd")
             B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
             clk.toc(tk)
-            launches += 1
             if hooks is not None and hasattr(hooks, "on_leaf"):
                 hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
                                         ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
@@ -290,13 +285,11 @@ class Stepper:
                 tk = clk.tic("raster_bwd")
                 B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
                 clk.toc(tk)
-                launches += 1
         del arena, bin_ws  # raster buffers released before projection backward
 
         loss_d = torch.zeros(1, dtype=torch.float64, device=dev)
         if target is not None:
             B.gs_loss_total(loss_tiles, T, loss_d)
-            launches += 1
         self._last_loss = loss_d
         ctx["g2d"] = g2d
         if hooks is not None and hasattr(hooks, "on_bwd"):
@@ -312,7 +305,6 @@ class Stepper:
                                  adam_m=m.m, adam_v=m.v, fused=self.adam_args(m.step),
                                  dev_status=st)
                 clk.toc(tk)
-                launches += 2 if C > 0 else 1
                 del geo
             else:
                 g3d = torch.empty(m.P * max(C, 1), dtype=torch.float32, device=dev)
@@ -320,7 +312,6 @@ class Stepper:
                                  dev_status=st)
                 B.gs_adam(m.params, m.m, m.v, g3d, max(C, 1), slot, m.n, m.n_pad, m.P,
                           self.adam_args(m.step))
-                launches += 2
                 del g3d
         peak = torch.cuda.max_memory_allocated(dev) - base_alloc
         if resident_target:
@@ -328,7 +319,8 @@ class Stepper:
         return ViewStats(n_cand=C, n_isect=int(li.sum()), n_isect_square=n_square,
                          n_leaves=len(lv), leaves=lv,
                          leaf_isect=li, leaf_bytes=lb, over_budget=ov, peak_ws_bytes=int(peak),
-                         arena_bytes=int(arena_bytes), launches=launches)
+                         arena_bytes=int(arena_bytes),
+                         launches=B.gs_launch_counter() - launch0)
 
     def render(self, cam) -> torch.Tensor:
         """Forward-only render of the whole view: [3][H][W] fp32 on the device."""

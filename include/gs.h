@@ -186,6 +186,12 @@ typedef struct gs_adam_args {
 int32_t gs_version(void);
 const char* gs_status_string(gs_status s);
 
+/* Number of kernel launches this library has issued in the calling process
+ * since it was loaded (all devices and streams; launches that failed to
+ * start included).  Host-only, thread-safe; no counterpart in the method,
+ * it serves launch accounting of the callers. */
+int64_t gs_launch_counter(void);
+
 /* Synchronises `stream`, then reads and clears *dev_status.  Returns the
  * most severe condition (GS_ERR_TIMEOUT > GS_ERR_BOUNDS > GS_OK). */
 gs_status gs_check(int32_t* dev_status, gs_stream stream);

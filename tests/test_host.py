@@ -39,6 +39,7 @@ def test_exports_every_declared_symbol(gsb):
 def test_host_argument_checks(gsb):
     b = gsb
     L = b.lib()
+    launches0 = b.gs_launch_counter()
     # null structs / sizes are rejected before any device work
     assert L.gs_project(None, None, 0, None, None, None, 0, None, None) == b.GS_ERR_ARG
     assert L.gs_sort_keys(None, None, 5, 0, 70, None, 0, None, None) == b.GS_ERR_ARG
@@ -52,6 +53,8 @@ def test_host_argument_checks(gsb):
     st = L.gs_bin_tiles(ctypes.byref(proj), 10, 8, 8, b.gs_rect(0, 0, 2, 2), 4, 4, 8, 1000, 8, 8,
                         None, 999, 8, ctypes.byref(needed), 256, 1 << 20, None, None)
     assert st == b.GS_ERR_CAPACITY and needed.value == 1000
+    # ... and none of the rejected calls launched a kernel
+    assert b.gs_launch_counter() == launches0
 
 
 def test_workspace_sizes(gsb):
