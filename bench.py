@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--views", type=int, default=8)
     ap.add_argument("--budget-mib", type=float, default=384)
     ap.add_argument("--raster-ppt", type=int, default=0)
+    ap.add_argument("--binning", default="expand", choices=["expand", "sort"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
@@ -230,12 +231,12 @@ def main():
     # targets: renders of the jittered copy (means N(0, 0.02), colour N(0, 0.05))
     jit = synth.jittered(scene, seed=1)
     jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
-    js = Stepper(jm, budget=budget, raster_flags=a.raster_ppt)
+    js = Stepper(jm, budget=budget, raster_flags=a.raster_ppt, binning=a.binning)
     targets = [js.render(c) for c in cams]
     torch.cuda.synchronize()
     del jm, js
     model = GaussianModel(scene.params, scene.n, scene.sh_degree)
-    stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt)
+    stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt, binning=a.binning)
     nv = len(cams)
     view_of = lambda k: (k + rank) % nv
 
@@ -374,12 +375,14 @@ def main():
             "data": "synthetic (seeded generator; targets = renders of a jittered copy)",
             "config": {"workload": workload_name(a), "gaussians": a.gaussians, "sh_degree": 3,
                        "width": W, "height": H, "views": nv, "leaf_budget_mib": a.budget_mib,
+                       "binning": a.binning,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (4.25 GB of params + Adam moments "
                              "stream every step)"},
             "peak_ws_gib": peak_ws / 2 ** 30,
             "isect_per_view": isect / a.steps,
             "list_entries_per_view": entries / a.steps,
+            "block_entries_per_view": sum(s.n_block_entries for s in stats) / a.steps,
             "candidates_per_view": statistics.mean(s.n_cand for s in stats),
             "leaves_per_view": statistics.mean(s.n_leaves for s in stats),
             "stage_ms_per_step": {s: round(per_step[s], 3) for s in STAGES},

@@ -102,6 +102,8 @@ SYMBOLS = [
     "gs_leaf_load_model", "gs_leaf_partition",
     "gs_depth_order_workspace_size", "gs_depth_order",
     "gs_bin_workspace_size", "gs_bin_tiles",
+    "gs_block_sat_workspace_size", "gs_block_sat", "gs_bin_blocks_workspace_size",
+    "gs_bin_blocks", "gs_expand_workspace_size", "gs_expand_tiles",
     "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
     "gs_project_bwd", "gs_adam",
 ]
@@ -125,7 +127,7 @@ def _load():
         "gs_sort_keys32": (i32, [p, p, p, i64, i32, i32, u32, p, sz, p, p]),
         "gs_sort_keys32_noalloc": (i32, [p, p, p, i64, i32, i32, u32, p, p]),
         "gs_sort_tiles": (i32, [p, p, i64, p, i64, p, sz, p, p]),
-        "gs_leaf_load_model": (i32, [i32, P(gs_load_model)]),
+        "gs_leaf_load_model": (i32, [i32, i32, P(gs_load_model)]),
         "gs_leaf_partition": (i32, [p, i32, i32, i32, i32, P(gs_load_model), i64, p, p, p, p,
                                     i32, P(i32)]),
         "gs_bin_workspace_size": (sz, [i64]),
@@ -133,6 +135,14 @@ def _load():
         "gs_depth_order": (i32, [P(gs_proj), i64, p, p, p, sz, p, p]),
         "gs_bin_tiles": (i32, [P(gs_proj), i64, p, p, gs_rect, i32, i32, p, i64, p, p, p, i64, p,
                                P(i64), p, sz, p, p]),
+        "gs_block_sat_workspace_size": (sz, [i32, i32]),
+        "gs_block_sat": (i32, [P(gs_proj), i32, i32, p, p, sz, p, p]),
+        "gs_bin_blocks_workspace_size": (sz, [i64, i64, i32, i32]),
+        "gs_bin_blocks": (i32, [P(gs_proj), i64, p, p, i32, i32, p, i64, p, i64, p, P(i64), p, sz,
+                                p, p]),
+        "gs_expand_workspace_size": (sz, [gs_rect, i64]),
+        "gs_expand_tiles": (i32, [P(gs_proj), p, p, i64, gs_rect, i32, i32, p, i64, p, i64, p,
+                                  P(i64), p, sz, p, p]),
         "gs_raster_fwd": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), u32, p, p]),
         "gs_loss_l1": (i32, [P(gs_pixels), gs_rect, P(gs_camera), p]),
         "gs_loss_total": (i32, [p, i64, p, p]),
@@ -258,9 +268,14 @@ def gs_sort_keys32_noalloc(keys_in, keys, vals, n, begin_bit, end_bit, flags, de
         _stream(stream)))
 
 
-def gs_leaf_load_model(tile_bits) -> gs_load_model:
+GS_BIN_SORT = 0
+GS_BIN_EXPAND = 1
+TILE_BLOCK = 8
+
+
+def gs_leaf_load_model(tile_bits, binning=GS_BIN_EXPAND) -> gs_load_model:
     lm = gs_load_model()
-    _ok("gs_leaf_load_model", _L.gs_leaf_load_model(tile_bits, C.byref(lm)))
+    _ok("gs_leaf_load_model", _L.gs_leaf_load_model(binning, tile_bits, C.byref(lm)))
     return lm
 
 
@@ -311,6 +326,53 @@ def gs_bin_tiles(proj: gs_proj, n_cand, depth_order, depth_rect, leaf, TW, TH, t
                          C.byref(needed), ptr(ws), ws.numel() * ws.element_size(),
                          ptr(dev_status), _stream(stream))
     return _ok("gs_bin_tiles", st, needed.value if st == GS_ERR_CAPACITY else None)
+
+
+def gs_block_sat_workspace_size(TW, TH) -> int:
+    return _L.gs_block_sat_workspace_size(TW, TH)
+
+
+def gs_block_sat(proj: gs_proj, TW, TH, block_sat, ws, dev_status, stream=None):
+    return _ok("gs_block_sat", _L.gs_block_sat(C.byref(proj), TW, TH, ptr(block_sat), ptr(ws),
+                                               ws.numel() * ws.element_size(), ptr(dev_status),
+                                               _stream(stream)))
+
+
+def gs_bin_blocks_workspace_size(n_cand, n_entries, TW, TH) -> int:
+    return _L.gs_bin_blocks_workspace_size(n_cand, n_entries, TW, TH)
+
+
+def gs_bin_blocks(proj: gs_proj, n_cand, depth_order, depth_rect, TW, TH, block_sat, n_entries,
+                  block_vals, capacity, block_ranges, ws, dev_status, stream=None):
+    needed = C.c_int64(0)
+    st = _L.gs_bin_blocks(C.byref(proj), n_cand, ptr(depth_order), ptr(depth_rect), TW, TH,
+                          ptr(block_sat), n_entries, ptr(block_vals), capacity, ptr(block_ranges),
+                          C.byref(needed), ptr(ws), ws.numel() * ws.element_size(),
+                          ptr(dev_status), _stream(stream))
+    return _ok("gs_bin_blocks", st, needed.value if st == GS_ERR_CAPACITY else None)
+
+
+def gs_expand_workspace_size(leaf, block_entries) -> int:
+    return _L.gs_expand_workspace_size(gs_rect(*[int(v) for v in leaf]), int(block_entries))
+
+
+def gs_expand_tiles(proj: gs_proj, block_vals, block_ranges, block_entries, leaf, TW, TH,
+                    tile_sat, n_isect, vals, capacity, ranges, ws, dev_status, stream=None):
+    needed = C.c_int64(0)
+    st = _L.gs_expand_tiles(C.byref(proj), ptr(block_vals), ptr(block_ranges), int(block_entries),
+                            gs_rect(*[int(v) for v in leaf]), TW, TH, ptr(tile_sat), n_isect,
+                            ptr(vals), capacity, ptr(ranges), C.byref(needed), ptr(ws),
+                            ws.numel() * ws.element_size(), ptr(dev_status), _stream(stream))
+    return _ok("gs_expand_tiles", st, needed.value if st == GS_ERR_CAPACITY else None)
+
+
+def block_entries(block_sat_host, leaf) -> int:
+    """Summed block-list lengths of the blocks meeting a Leaf (host SAT)."""
+    x0, y0, x1, y1 = (int(v) for v in leaf)
+    bx0, by0 = x0 // TILE_BLOCK, y0 // TILE_BLOCK
+    bx1, by1 = (x1 - 1) // TILE_BLOCK + 1, (y1 - 1) // TILE_BLOCK + 1
+    S = block_sat_host
+    return int(S[by1, bx1] - S[by0, bx1] - S[by1, bx0] + S[by0, bx0])
 
 
 def local_tile_bits(leaf) -> int:

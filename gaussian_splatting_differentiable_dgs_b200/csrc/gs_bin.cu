@@ -32,6 +32,9 @@ k_gather_rects(const short4* __restrict__ rect, const int32_t* __restrict__ orde
   if (j < n) out[j] = rect[order[j]];
 }
 
+// BLK = 1: entries per tile; BLK = GS_TILE_BLOCK: entries per block of
+// BLK x BLK tiles (the candidate's tile rect widened to whole blocks).
+template <int BLK>
 __global__ void __launch_bounds__(kBinThreads)
 k_bin(const short4* __restrict__ drect, const int32_t* __restrict__ order,
       const uint32_t* __restrict__ depth_key, int64_t n_cand, gs_rect leaf, int TW,
@@ -57,10 +60,17 @@ k_bin(const short4* __restrict__ drect, const int32_t* __restrict__ order,
     int x0 = 0, y0 = 0, w = 1;
     if (j < n_cand) {
       const short4 r = drect[j];
-      x0 = max((int)r.x, leaf.x0);
-      const int x1 = min((int)r.z, leaf.x1);
-      y0 = max((int)r.y, leaf.y0);
-      const int y1 = min((int)r.w, leaf.y1);
+      int rx0 = r.x, ry0 = r.y, rx1 = r.z, ry1 = r.w;
+      if (BLK > 1) {  // rects are non-empty, so r.z, r.w >= 1
+        rx0 /= BLK;
+        ry0 /= BLK;
+        rx1 = (rx1 - 1) / BLK + 1;
+        ry1 = (ry1 - 1) / BLK + 1;
+      }
+      x0 = max(rx0, leaf.x0);
+      const int x1 = min(rx1, leaf.x1);
+      y0 = max(ry0, leaf.y0);
+      const int y1 = min(ry1, leaf.y1);
       if (x1 > x0 && y1 > y0) {
         w = x1 - x0;
         cnt[k] = (long long)w * (y1 - y0);
@@ -132,6 +142,318 @@ __global__ void k_ranges(const int64_t* __restrict__ sat, gs_rect leaf, int TW,
   const long long cnt = sat_rect(sat, s, tx, ty, tx + 1, ty + 1);
   ranges[2 * t] = begin;
   ranges[2 * t + 1] = begin + cnt;
+}
+
+// ---------------------------------------------------------------------------
+// Two-level binning.  Per view, every candidate is listed once per block of
+// GS_TILE_BLOCK x GS_TILE_BLOCK tiles that its rect meets, in depth order
+// (k_bin<GS_TILE_BLOCK> + a stable sort on the block id).  Per Leaf, each
+// block list is cut into chunks of kExpChunk entries; a chunk turns each
+// candidate's rect into a 64-bit mask over the block's tiles (clipped to the
+// Leaf) and ranks the candidates per tile with warp ballots, so the entry of
+// (candidate, tile) goes straight to its place in the tile's segment, whose
+// begin the tile SAT gives.  Two passes: per-(chunk, tile) counts, an
+// exclusive scan over the chunks of each block, then the writes.  The order
+// within a tile is the block list's order, i.e. the depth order.
+// ---------------------------------------------------------------------------
+constexpr int kBlk = GS_TILE_BLOCK;
+static_assert(kBlk == 8, "tile masks are 64-bit");
+constexpr int kExpThreads = 256;
+constexpr int kExpRounds = 4;
+constexpr int kExpChunk = kExpThreads * kExpRounds;
+constexpr int kExpWarps = kExpThreads / 32;
+
+struct LeafBlocks {
+  int bx0, by0, bw, bh;  // the blocks that meet the Leaf
+};
+
+__host__ __device__ inline LeafBlocks leaf_blocks(gs_rect leaf) {
+  LeafBlocks b;
+  b.bx0 = leaf.x0 / kBlk;
+  b.by0 = leaf.y0 / kBlk;
+  b.bw = (leaf.x1 - 1) / kBlk + 1 - b.bx0;
+  b.bh = (leaf.y1 - 1) / kBlk + 1 - b.by0;
+  return b;
+}
+
+// rect ∩ leaf ∩ block (bx, by) in block-local tile coordinates; empty when
+// x1 <= x0 (then x0 = x1 = y0 = y1 = 0).
+struct LocalRect {
+  int x0, x1, y0, y1;
+};
+
+__device__ __forceinline__ LocalRect local_rect(short4 r, gs_rect leaf, int bx, int by) {
+  const int ox = bx * kBlk, oy = by * kBlk;
+  LocalRect q;
+  q.x0 = max(max((int)r.x, leaf.x0), ox) - ox;
+  q.x1 = min(min((int)r.z, leaf.x1), ox + kBlk) - ox;
+  q.y0 = max(max((int)r.y, leaf.y0), oy) - oy;
+  q.y1 = min(min((int)r.w, leaf.y1), oy + kBlk) - oy;
+  if (q.x1 <= q.x0 || q.y1 <= q.y0) q.x0 = q.x1 = q.y0 = q.y1 = 0;
+  return q;
+}
+
+// byte x set to 1 for x in [x0, x1) (0 <= x0 <= x1 <= 8)
+__device__ __forceinline__ uint64_t row_bytes(int x0, int x1) {
+  const uint64_t hi = x1 >= kBlk ? ~0ull : ((1ull << (8 * x1)) - 1ull);
+  const uint64_t lo = x0 >= kBlk ? ~0ull : ((1ull << (8 * x0)) - 1ull);
+  return (hi & ~lo) & 0x0101010101010101ull;
+}
+
+// bit (ly * 8 + lx) set for the tiles of the local rect
+__device__ __forceinline__ uint64_t tile_mask(const LocalRect& q) {
+  const uint64_t row = (uint64_t)(((1u << q.x1) - 1u) & ~((1u << q.x0) - 1u));
+  return row_bytes(q.y0, q.y1) * row;
+}
+
+// This warp's count of tile (lane & 7, row) for rows lane >> 3 (lo) and
+// 4 + (lane >> 3) (hi), i.e. tiles lane and 32 + lane: per row, the lanes'
+// byte-packed rows are summed with one reduction per 4 tiles (counts <= 32
+// fit a byte).
+__device__ __forceinline__ void warp_tile_counts(const LocalRect& q, int lane, unsigned& c_lo,
+                                                 unsigned& c_hi) {
+  const uint64_t rb = row_bytes(q.x0, q.x1);
+  const int ymin = __reduce_min_sync(0xffffffffu, q.x1 > q.x0 ? q.y0 : kBlk);
+  const int ymax = __reduce_max_sync(0xffffffffu, q.y1);
+  const int my_row = lane >> 3, my_x = lane & 7;
+  c_lo = c_hi = 0;
+  for (int y = ymin; y < ymax; ++y) {
+    const bool in = q.y0 <= y && y < q.y1;
+    const unsigned wl = __reduce_add_sync(0xffffffffu, in ? (unsigned)rb : 0u);
+    const unsigned wh = __reduce_add_sync(0xffffffffu, in ? (unsigned)(rb >> 32) : 0u);
+    const unsigned v = ((my_x < 4 ? wl : wh) >> (8 * (my_x & 3))) & 0xffu;
+    if (my_row == y) c_lo = v;
+    if (my_row + 4 == y) c_hi = v;
+  }
+}
+
+// chunk_start[i] = first chunk of the i-th block of the Leaf (row-major over
+// LeafBlocks), chunk_start[nbl] = total; one block of 1024 threads.
+__global__ void __launch_bounds__(1024)
+k_expand_plan(const int64_t* __restrict__ block_ranges, int BW, LeafBlocks lb,
+              int64_t* __restrict__ chunk_start, int64_t max_chunks, int32_t* dev_status) {
+  __shared__ long long s_scan[33];
+  const int nbl = lb.bw * lb.bh;
+  long long carry = 0;
+  for (int base = 0; base < nbl; base += 1024) {
+    const int i = base + threadIdx.x;
+    long long c = 0;
+    if (i < nbl) {
+      const int64_t b = (int64_t)(lb.by0 + i / lb.bw) * BW + lb.bx0 + i % lb.bw;
+      const long long len = block_ranges[2 * b + 1] - block_ranges[2 * b];
+      c = (len + kExpChunk - 1) / kExpChunk;
+    }
+    long long tot;
+    const long long ex = block_exclusive_scan<long long, 32>(c, s_scan, &tot);
+    if (i < nbl) chunk_start[i] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) {
+    chunk_start[nbl] = carry;
+    if (carry > max_chunks) dev_flag(dev_status, GS_DEV_BOUNDS);
+  }
+}
+
+struct ChunkPos {
+  int i, bx, by;
+  int64_t begin, end;
+};
+
+// the block and entry range of chunk g (g < total)
+__device__ __forceinline__ ChunkPos chunk_pos(int64_t g, const int64_t* __restrict__ chunk_start,
+                                              int nbl, LeafBlocks lb, int BW,
+                                              const int64_t* __restrict__ block_ranges) {
+  int lo = 0, hi = nbl - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (chunk_start[mid] <= g) lo = mid;
+    else hi = mid - 1;
+  }
+  ChunkPos c;
+  c.i = lo;
+  c.bx = lb.bx0 + lo % lb.bw;
+  c.by = lb.by0 + lo / lb.bw;
+  const int64_t b = (int64_t)c.by * BW + c.bx;
+  c.begin = block_ranges[2 * b] + (g - chunk_start[lo]) * kExpChunk;
+  const int64_t e = block_ranges[2 * b + 1];
+  c.end = c.begin + kExpChunk < e ? c.begin + kExpChunk : e;
+  return c;
+}
+
+__global__ void __launch_bounds__(kExpThreads)
+k_expand_count(const short4* __restrict__ rect, const int32_t* __restrict__ block_vals,
+               const int64_t* __restrict__ block_ranges, int BW, LeafBlocks lb, gs_rect leaf,
+               const int64_t* __restrict__ chunk_start, int32_t* __restrict__ cnt) {
+  __shared__ unsigned int s_wc[kExpWarps][64];
+  const int nbl = lb.bw * lb.bh;
+  const int64_t g = blockIdx.x;
+  if (g >= chunk_start[nbl]) return;
+  const ChunkPos c = chunk_pos(g, chunk_start, nbl, lb, BW, block_ranges);
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  unsigned acc_lo = 0, acc_hi = 0;  // lane j: tiles j and 32 + j
+#pragma unroll 1
+  for (int k = 0; k < kExpRounds; ++k) {
+    const int64_t p = c.begin + k * kExpThreads + t;
+    LocalRect q{0, 0, 0, 0};
+    if (p < c.end) q = local_rect(rect[block_vals[p]], leaf, c.bx, c.by);
+    unsigned n_lo, n_hi;
+    warp_tile_counts(q, lane, n_lo, n_hi);
+    acc_lo += n_lo;
+    acc_hi += n_hi;
+  }
+  s_wc[w][lane] = acc_lo;
+  s_wc[w][32 + lane] = acc_hi;
+  __syncthreads();
+  if (t < 64) {
+    unsigned sum = 0;
+#pragma unroll
+    for (int ww = 0; ww < kExpWarps; ++ww) sum += s_wc[ww][t];
+    cnt[g * 64 + t] = (int32_t)sum;
+  }
+}
+
+// one thread per (block of the Leaf, tile of the block): the exclusive scan
+// of the tile's chunk counts, started at the tile's begin in the Leaf list;
+// the counts must add up to the tile's SAT count.
+__global__ void __launch_bounds__(256)
+k_expand_scan(const int32_t* __restrict__ cnt, const int64_t* __restrict__ chunk_start,
+              LeafBlocks lb, gs_rect leaf, const int64_t* __restrict__ ranges,
+              int64_t* __restrict__ base, int64_t max_chunks, int32_t* dev_status) {
+  const int nbl = lb.bw * lb.bh;
+  const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (idx >= (int64_t)nbl * 64) return;
+  const int i = (int)(idx >> 6), j = (int)(idx & 63);
+  const int tx = (lb.bx0 + i % lb.bw) * kBlk + (j & 7);
+  const int ty = (lb.by0 + i / lb.bw) * kBlk + (j >> 3);
+  // (a plan over max_chunks has already been flagged by k_expand_plan)
+  const int64_t g0 = min(chunk_start[i], max_chunks), g1 = min(chunk_start[i + 1], max_chunks);
+  if (tx < leaf.x0 || tx >= leaf.x1 || ty < leaf.y0 || ty >= leaf.y1) {
+    for (int64_t g = g0; g < g1; ++g) base[g * 64 + j] = 0;
+    return;
+  }
+  const int64_t lt = (int64_t)(ty - leaf.y0) * (leaf.x1 - leaf.x0) + (tx - leaf.x0);
+  long long run = ranges[2 * lt];
+  for (int64_t g = g0; g < g1; ++g) {
+    base[g * 64 + j] = run;
+    run += cnt[g * 64 + j];
+  }
+  if (run != ranges[2 * lt + 1]) dev_flag(dev_status, GS_DEV_BOUNDS);
+}
+
+__global__ void __launch_bounds__(kExpThreads)
+k_expand_write(const short4* __restrict__ rect, const int32_t* __restrict__ block_vals,
+               const int64_t* __restrict__ block_ranges, int BW, LeafBlocks lb, gs_rect leaf,
+               const int64_t* __restrict__ chunk_start, const int64_t* __restrict__ base,
+               int32_t* __restrict__ vals, int32_t capacity, int32_t* dev_status) {
+  __shared__ int s_cur[64];
+  __shared__ int s_off[kExpWarps][64];
+  __shared__ unsigned int s_wc[kExpWarps][64];
+  const int nbl = lb.bw * lb.bh;
+  const int64_t g = blockIdx.x;
+  if (g >= chunk_start[nbl]) return;
+  const ChunkPos c = chunk_pos(g, chunk_start, nbl, lb, BW, block_ranges);
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  // positions fit 32 bits: the host limits a Leaf list to INT32_MAX entries
+  if (t < 64) s_cur[t] = (int)base[g * 64 + t];
+  bool bad = false;
+#pragma unroll 1
+  for (int k = 0; k < kExpRounds; ++k) {
+    const int64_t p = c.begin + k * kExpThreads + t;
+    LocalRect q{0, 0, 0, 0};
+    int32_t slot = 0;
+    if (p < c.end) {
+      slot = block_vals[p];
+      q = local_rect(rect[slot], leaf, c.bx, c.by);
+    }
+    unsigned n_lo, n_hi;
+    warp_tile_counts(q, lane, n_lo, n_hi);
+    s_wc[w][lane] = n_lo;
+    s_wc[w][32 + lane] = n_hi;
+    const uint64_t m = tile_mask(q);
+    const unsigned mlo = (unsigned)m, mhi = (unsigned)(m >> 32);
+    const unsigned olo = __reduce_or_sync(0xffffffffu, mlo);
+    const unsigned ohi = __reduce_or_sync(0xffffffffu, mhi);
+    __syncthreads();
+    if (t < 64) {
+      int run = s_cur[t];
+#pragma unroll
+      for (int ww = 0; ww < kExpWarps; ++ww) {
+        s_off[ww][t] = run;
+        run += (int)s_wc[ww][t];
+      }
+      s_cur[t] = run;
+    }
+    __syncthreads();
+    // one coalesced store per tile: the warp's entries of tile j are
+    // consecutive in the tile's segment, in lane (= list) order
+    for (unsigned r = olo; r; r &= r - 1) {
+      const int j = __ffs(r) - 1;
+      const bool mine = (mlo >> j) & 1u;
+      const unsigned bal = __ballot_sync(0xffffffffu, mine);
+      if (mine) {
+        const int pos = s_off[w][j] + __popc(bal & lt_mask);
+        if ((unsigned)pos < (unsigned)capacity) vals[pos] = slot;
+        else bad = true;
+      }
+    }
+    for (unsigned r = ohi; r; r &= r - 1) {
+      const int j = __ffs(r) - 1;
+      const bool mine = (mhi >> j) & 1u;
+      const unsigned bal = __ballot_sync(0xffffffffu, mine);
+      if (mine) {
+        const int pos = s_off[w][32 + j] + __popc(bal & lt_mask);
+        if ((unsigned)pos < (unsigned)capacity) vals[pos] = slot;
+        else bad = true;
+      }
+    }
+    __syncthreads();  // s_wc / s_off are rewritten by the next round
+  }
+  if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
+}
+
+struct BlockBinWs {
+  unsigned int* ticket;
+  unsigned long long* lb;
+  uint32_t* keys;
+  void* sort_ws;
+  size_t sort_bytes;
+  size_t bytes;
+};
+
+BlockBinWs carve_block_bin(void* ws, size_t cap, int64_t n_cand, int64_t n_entries, int64_t nblocks) {
+  Carver cv(ws, cap);
+  BlockBinWs w;
+  w.ticket = cv.take<unsigned int>(64);
+  const int64_t nb = (n_cand + kBinChunk - 1) / kBinChunk;
+  w.lb = cv.take<unsigned long long>(nb > 0 ? nb : 1);
+  w.keys = cv.take<uint32_t>(n_entries > 0 ? n_entries : 1);
+  const int bits = nblocks > 1 ? 64 - __builtin_clzll((unsigned long long)(nblocks - 1)) : 0;
+  w.sort_bytes = gs_sort_workspace_size(n_entries, 4, 0, bits);
+  w.sort_ws = cv.take<unsigned char>(w.sort_bytes);
+  w.bytes = cv.off;
+  return w;
+}
+
+struct ExpandWs {
+  int64_t* chunk_start;
+  int32_t* cnt;
+  int64_t* base;
+  int64_t max_chunks;
+  size_t bytes;
+};
+
+ExpandWs carve_expand(void* ws, size_t cap, gs_rect leaf, int64_t block_entries) {
+  Carver cv(ws, cap);
+  ExpandWs w;
+  const LeafBlocks lb = leaf_blocks(leaf);
+  const int64_t nbl = (int64_t)lb.bw * lb.bh;
+  w.max_chunks = (block_entries + kExpChunk - 1) / kExpChunk + nbl;
+  w.chunk_start = cv.take<int64_t>(nbl + 1);
+  w.cnt = cv.take<int32_t>(w.max_chunks * 64);
+  w.base = cv.take<int64_t>(w.max_chunks * 64);
+  w.bytes = cv.off;
+  return w;
 }
 
 struct BinWs {
@@ -234,9 +556,108 @@ extern "C" gs_status gs_bin_tiles(const gs_proj* proj, int64_t n_cand, const int
   if (n_cand == 0 || n_isect == 0) return GS_OK;
   GS_TRY(cudaMemsetAsync(ws, 0, w.bytes, s));
   const int64_t nb = (n_cand + kBinChunk - 1) / kBinChunk;
-  k_bin<<<(unsigned)nb, kBinThreads, 0, s>>>(
+  k_bin<1><<<(unsigned)nb, kBinThreads, 0, s>>>(
       reinterpret_cast<const short4*>(depth_rect), depth_order, proj->depth_key, n_cand, leaf, TW,
       tile_keys, vals, keys64, capacity, w.lb, w.ticket, dev_status);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" size_t gs_bin_blocks_workspace_size(int64_t n_cand, int64_t n_entries, int32_t TW,
+                                               int32_t TH) {
+  if (n_cand < 0 || n_entries < 0 || TW <= 0 || TH <= 0) return 0;
+  const int64_t nblocks = (int64_t)((TW + kBlk - 1) / kBlk) * ((TH + kBlk - 1) / kBlk);
+  return carve_block_bin(nullptr, 0, n_cand, n_entries, nblocks).bytes;
+}
+
+extern "C" gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand, const int32_t* depth_order,
+                                   const int16_t* depth_rect, int32_t TW, int32_t TH,
+                                   const int64_t* block_sat, int64_t n_entries,
+                                   int32_t* block_vals, int64_t capacity, int64_t* block_ranges,
+                                   int64_t* needed, void* ws, size_t ws_bytes,
+                                   int32_t* dev_status, gs_stream stream) {
+  if (!proj || n_cand < 0 || n_cand > proj->capacity || TW <= 0 || TH <= 0 || TW > 32767 ||
+      TH > 32767 || !block_sat || !block_ranges || n_entries < 0)
+    return GS_ERR_ARG;
+  if (n_entries > capacity) {
+    if (needed) *needed = n_entries;
+    return GS_ERR_CAPACITY;
+  }
+  if (n_cand > 0 && (!depth_order || !depth_rect)) return GS_ERR_ARG;
+  if (n_entries > 0 && !block_vals) return GS_ERR_ARG;
+  const int32_t BW = (TW + kBlk - 1) / kBlk, BH = (TH + kBlk - 1) / kBlk;
+  const int64_t nblocks = (int64_t)BW * BH;
+  BlockBinWs w = carve_block_bin(ws, ws_bytes, n_cand, n_entries, nblocks);
+  if (!ws || w.bytes > ws_bytes) {
+    if (needed) *needed = (int64_t)w.bytes;
+    return GS_ERR_CAPACITY;
+  }
+  if (!aligned(ws, 256) || !aligned(depth_rect, 8)) return GS_ERR_ARG;
+  cudaStream_t s = to_stream(stream);
+  const gs_rect grid{0, 0, BW, BH};
+  k_ranges<<<(unsigned)((nblocks + 255) / 256), 256, 0, s>>>(block_sat, grid, BW, block_ranges);
+  GS_LAUNCH_CHECK();
+  if (n_cand == 0 || n_entries == 0) return GS_OK;
+  GS_TRY(cudaMemsetAsync(ws, 0, (size_t)((char*)w.keys - (char*)ws), s));
+  const int64_t nb = (n_cand + kBinChunk - 1) / kBinChunk;
+  k_bin<kBlk><<<(unsigned)nb, kBinThreads, 0, s>>>(
+      reinterpret_cast<const short4*>(depth_rect), depth_order, nullptr, n_cand, grid, BW, w.keys,
+      block_vals, nullptr, capacity, w.lb, w.ticket, dev_status);
+  GS_LAUNCH_CHECK();
+  return gs_sort_tiles(w.keys, block_vals, n_entries, block_ranges, nblocks, w.sort_ws,
+                       w.sort_bytes, dev_status, stream);
+}
+
+extern "C" size_t gs_expand_workspace_size(gs_rect leaf, int64_t block_entries) {
+  if (leaf.x0 < 0 || leaf.y0 < 0 || leaf.x1 <= leaf.x0 || leaf.y1 <= leaf.y0 || block_entries < 0)
+    return 0;
+  return carve_expand(nullptr, 0, leaf, block_entries).bytes;
+}
+
+extern "C" gs_status gs_expand_tiles(const gs_proj* proj, const int32_t* block_vals,
+                                     const int64_t* block_ranges, int64_t block_entries,
+                                     gs_rect leaf, int32_t TW, int32_t TH,
+                                     const int64_t* tile_sat, int64_t n_isect, int32_t* vals,
+                                     int64_t capacity, int64_t* ranges, int64_t* needed, void* ws,
+                                     size_t ws_bytes, int32_t* dev_status, gs_stream stream) {
+  if (!proj || TW <= 0 || TH <= 0 || TW > 32767 || TH > 32767 || !tile_sat || !ranges ||
+      !block_ranges || block_entries < 0 || n_isect < 0)
+    return GS_ERR_ARG;
+  if (leaf.x0 < 0 || leaf.y0 < 0 || leaf.x1 <= leaf.x0 || leaf.y1 <= leaf.y0 || leaf.x1 > TW ||
+      leaf.y1 > TH)
+    return GS_ERR_ARG;
+  if (n_isect > capacity) {
+    if (needed) *needed = n_isect;
+    return GS_ERR_CAPACITY;
+  }
+  if (capacity > (int64_t)INT32_MAX) return GS_ERR_UNSUPPORTED;  // 32-bit list positions
+  if (n_isect > 0 && (!vals || !block_vals || !proj->rect)) return GS_ERR_ARG;
+  ExpandWs w = carve_expand(ws, ws_bytes, leaf, block_entries);
+  if (!ws || w.bytes > ws_bytes) {
+    if (needed) *needed = (int64_t)w.bytes;
+    return GS_ERR_CAPACITY;
+  }
+  if (!aligned(ws, 256) || !aligned(proj->rect, 8)) return GS_ERR_ARG;
+  cudaStream_t s = to_stream(stream);
+  const int64_t ntiles = (int64_t)(leaf.x1 - leaf.x0) * (leaf.y1 - leaf.y0);
+  k_ranges<<<(unsigned)((ntiles + 255) / 256), 256, 0, s>>>(tile_sat, leaf, TW, ranges);
+  GS_LAUNCH_CHECK();
+  if (n_isect == 0 || block_entries == 0) return GS_OK;
+  const int32_t BW = (TW + kBlk - 1) / kBlk;
+  const LeafBlocks lb = leaf_blocks(leaf);
+  const int64_t nbl = (int64_t)lb.bw * lb.bh;
+  const short4* r4 = reinterpret_cast<const short4*>(proj->rect);
+  k_expand_plan<<<1, 1024, 0, s>>>(block_ranges, BW, lb, w.chunk_start, w.max_chunks, dev_status);
+  GS_LAUNCH_CHECK();
+  k_expand_count<<<(unsigned)w.max_chunks, kExpThreads, 0, s>>>(r4, block_vals, block_ranges, BW,
+                                                                lb, leaf, w.chunk_start, w.cnt);
+  GS_LAUNCH_CHECK();
+  k_expand_scan<<<(unsigned)((nbl * 64 + 255) / 256), 256, 0, s>>>(
+      w.cnt, w.chunk_start, lb, leaf, ranges, w.base, w.max_chunks, dev_status);
+  GS_LAUNCH_CHECK();
+  k_expand_write<<<(unsigned)w.max_chunks, kExpThreads, 0, s>>>(
+      r4, block_vals, block_ranges, BW, lb, leaf, w.chunk_start, w.base, vals, (int32_t)capacity,
+      dev_status);
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

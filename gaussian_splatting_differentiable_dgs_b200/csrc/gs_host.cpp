@@ -118,21 +118,30 @@ extern "C" gs_status gs_check(int32_t* dev_status, gs_stream stream) {
   return GS_OK;
 }
 
-// Per-unit bytes of the buffers one Leaf needs (see gs.h).  Intersections:
-// 32-bit tile keys + 32-bit values + their sort double buffers (16 B) plus
-// the look-back words of the tile sort (256 x 8 B per 4096 items per pass).
-// tile_bits: bits of the whole grid's tile count, an upper bound of any
-// Leaf's local bits.  Pixels: colour (12), T_final (4), last (4), target
-// crop (12), dL/dcolour (12).  Tiles: the int64 range pair.  Fixed: sort
+// Per-unit bytes of the buffers one Leaf needs.
+// GS_BIN_SORT (gs_bin_tiles + gs_sort_tiles): intersections take 32-bit tile
+// keys + 32-bit values + their sort double buffers (16 B) plus the counts of
+// the tile sort (256 x 4 B per 4096 items per pass); tile_bits, the bits of
+// the whole grid's tile count, bounds any Leaf's local bits.  Fixed: sort
 // histograms, tickets and alignment.
-extern "C" gs_status gs_leaf_load_model(int32_t tile_bits, gs_load_model* out) {
+// GS_BIN_EXPAND (gs_expand_tiles): intersections take their 32-bit value
+// only; fixed: the alignment of the Leaf's buffers.
+// Both: pixels take colour (12), T_final (4), last (4), target crop (12) and
+// dL/dcolour (12); tiles the int64 range pair.
+extern "C" gs_status gs_leaf_load_model(int32_t binning, int32_t tile_bits, gs_load_model* out) {
   if (!out || tile_bits < 0 || tile_bits > 32) return GS_ERR_ARG;
-  const int passes = tile_bits == 0 ? 0 : 2 * ((tile_bits + 15) / 16);
-  out->bytes_per_isect = 16 + (passes + 1) / 2;
   out->bytes_per_pixel = 44;
   out->bytes_per_tile = 16;
-  out->fixed_bytes = 2 * 8 * 256 * 8 + 64 * 4 + (int64_t)passes * 256 * 8 + 16 * 256;
   out->align = 512;
+  if (binning == GS_BIN_EXPAND) {
+    out->bytes_per_isect = 4;
+    out->fixed_bytes = 8 * 256;
+    return GS_OK;
+  }
+  if (binning != GS_BIN_SORT) return GS_ERR_ARG;
+  const int passes = tile_bits == 0 ? 0 : 2 * ((tile_bits + 15) / 16);
+  out->bytes_per_isect = 16 + (passes + 1) / 2;
+  out->fixed_bytes = 2 * 8 * 256 * 8 + 64 * 4 + (int64_t)passes * 256 * 8 + 16 * 256;
   return GS_OK;
 }
 

@@ -299,6 +299,54 @@ k_sat_cols(const int64_t* __restrict__ tmp, int64_t* __restrict__ sat, int TW, i
   }
 }
 
+// Corners of each candidate's block rect (blocks of GS_TILE_BLOCK x
+// GS_TILE_BLOCK tiles) into a difference grid; the count comes from the
+// device (candidates written by the projection).  The grid is small and hot,
+// so each CTA accumulates into a shared copy (SHARED) and adds its non-zero
+// cells once.
+template <bool SHARED>
+__global__ void __launch_bounds__(256)
+k_block_diff(const short4* __restrict__ rect, const int32_t* __restrict__ n_cand, int64_t cap,
+             int BW, int cells, int32_t* __restrict__ diff) {
+  extern __shared__ int32_t s_diff[];
+  int32_t* d = SHARED ? s_diff : diff;
+  if (SHARED) {
+    for (int c = threadIdx.x; c < cells; c += 256) s_diff[c] = 0;
+    __syncthreads();
+  }
+  const int64_t n = min((int64_t)*n_cand, cap);
+  const int s = BW + 1;
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256) {
+    const short4 r = rect[i];
+    const int bx0 = r.x / GS_TILE_BLOCK, by0 = r.y / GS_TILE_BLOCK;
+    const int bx1 = (r.z - 1) / GS_TILE_BLOCK + 1, by1 = (r.w - 1) / GS_TILE_BLOCK + 1;
+    atomicAdd(&d[by0 * s + bx0], 1);
+    atomicAdd(&d[by0 * s + bx1], -1);
+    atomicAdd(&d[by1 * s + bx0], -1);
+    atomicAdd(&d[by1 * s + bx1], 1);
+  }
+  if (SHARED) {
+    __syncthreads();
+    for (int c = threadIdx.x; c < cells; c += 256)
+      if (s_diff[c] != 0) atomicAdd(&diff[c], s_diff[c]);
+  }
+}
+
+struct BlockWs {
+  int32_t* diff;
+  int64_t* tmp;
+  size_t bytes;
+};
+
+BlockWs carve_block(void* ws, size_t cap, int64_t BW, int64_t BH) {
+  Carver cv(ws, cap);
+  BlockWs w;
+  w.diff = cv.take<int32_t>((BW + 1) * (BH + 1));
+  w.tmp = cv.take<int64_t>(BW * BH);
+  w.bytes = cv.off;
+  return w;
+}
+
 struct ProjWs {
   int32_t* diff;
   int64_t* tmp;
@@ -377,6 +425,50 @@ extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uin
   k_sat_rows<<<(unsigned)TH, 256, 0, s>>>(w.diff, w.tmp, (int)TW, (int)TH);
   GS_LAUNCH_CHECK();
   k_sat_cols<<<(unsigned)((TW + 1 + 255) / 256), 256, 0, s>>>(w.tmp, tile_sat, (int)TW, (int)TH);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" size_t gs_block_sat_workspace_size(int32_t TW, int32_t TH) {
+  if (TW <= 0 || TH <= 0) return 0;
+  return carve_block(nullptr, 0, (TW + GS_TILE_BLOCK - 1) / GS_TILE_BLOCK,
+                     (TH + GS_TILE_BLOCK - 1) / GS_TILE_BLOCK)
+      .bytes;
+}
+
+extern "C" gs_status gs_block_sat(const gs_proj* proj, int32_t TW, int32_t TH, int64_t* block_sat,
+                                  void* ws, size_t ws_bytes, int32_t* dev_status,
+                                  gs_stream stream) {
+  (void)dev_status;
+  if (!proj || !proj->n_cand || !block_sat || TW <= 0 || TH <= 0 || TW > 32767 || TH > 32767)
+    return GS_ERR_ARG;
+  if (proj->capacity > 0 && !proj->rect) return GS_ERR_ARG;
+  if (!aligned(proj->rect, 8) || !aligned(ws, 256)) return GS_ERR_ARG;
+  const int64_t BW = (TW + GS_TILE_BLOCK - 1) / GS_TILE_BLOCK;
+  const int64_t BH = (TH + GS_TILE_BLOCK - 1) / GS_TILE_BLOCK;
+  BlockWs w = carve_block(ws, ws_bytes, BW, BH);
+  if (!ws || w.bytes > ws_bytes) return GS_ERR_CAPACITY;
+  cudaStream_t s = to_stream(stream);
+  GS_TRY(cudaMemsetAsync(w.diff, 0, sizeof(int32_t) * (BW + 1) * (BH + 1), s));
+  if (proj->capacity > 0) {
+    const int64_t want = (proj->capacity + 255) / 256;
+    const int cells = (int)((BW + 1) * (BH + 1));
+    const short4* r4 = reinterpret_cast<const short4*>(proj->rect);
+    if (cells <= 12 * 1024) {  // 48 KB of shared counters
+      // one wave of CTAs, each taking a long strided share of the candidates
+      const unsigned nb = (unsigned)(want < 148 * 2 ? want : 148 * 2);
+      k_block_diff<true><<<nb, 256, cells * sizeof(int32_t), s>>>(r4, proj->n_cand,
+                                                                 proj->capacity, (int)BW, cells,
+                                                                 w.diff);
+    } else {
+      k_block_diff<false><<<(unsigned)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
+          r4, proj->n_cand, proj->capacity, (int)BW, cells, w.diff);
+    }
+    GS_LAUNCH_CHECK();
+  }
+  k_sat_rows<<<(unsigned)BH, 256, 0, s>>>(w.diff, w.tmp, (int)BW, (int)BH);
+  GS_LAUNCH_CHECK();
+  k_sat_cols<<<(unsigned)((BW + 1 + 255) / 256), 256, 0, s>>>(w.tmp, block_sat, (int)BW, (int)BH);
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

@@ -23,7 +23,7 @@ from . import binding as B
 
 DEFAULT_BUDGET = 384 << 20
 
-STAGES = ("project", "sort_depth", "bin", "sort_tiles", "raster_fwd", "raster_bwd",
+STAGES = ("project", "sort_depth", "bin", "sort_tiles", "expand", "raster_fwd", "raster_bwd",
           "project_bwd")
 
 
@@ -49,6 +49,7 @@ class ViewStats:
     n_cand: int
     n_isect: int          # entries of the (tight) tile lists
     n_isect_square: int   # tiles of the candidates' plain 3-sigma squares
+    n_block_entries: int  # entries of the per-block lists (two-level binning)
     n_leaves: int
     leaves: np.ndarray
     leaf_isect: np.ndarray
@@ -109,8 +110,11 @@ class Stepper:
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
-                 device="cuda"):
+                 binning="expand", device="cuda"):
+        if binning not in ("expand", "sort"):
+            raise ValueError(f"binning must be 'expand' or 'sort', not {binning!r}")
         self.model = model
+        self.binning = binning
         self.budget = int(budget)
         self.lr, self.betas, self.eps = lr, betas, eps
         self.raster_flags = raster_flags
@@ -174,8 +178,18 @@ class Stepper:
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
         tk = clk.tic("project")
         B.gs_project(mod, camS, proj, sat, ws, st)
+        expand = self.binning == "expand"
+        if expand:
+            BW, BH = (TW + B.TILE_BLOCK - 1) // B.TILE_BLOCK, (TH + B.TILE_BLOCK - 1) // B.TILE_BLOCK
+            bsat = torch.empty((BH + 1) * (BW + 1), dtype=torch.int64, device=dev)
+            bws = torch.empty(B.gs_block_sat_workspace_size(TW, TH), dtype=torch.uint8, device=dev)
+            B.gs_block_sat(proj, TW, TH, bsat, bws, st)
+            del bws
         clk.toc(tk)
         del ws
+        if expand:
+            bsat_h = torch.empty(bsat.shape, dtype=torch.int64, pin_memory=True)
+            bsat_h.copy_(bsat, non_blocking=True)
         sat_h = torch.empty(sat.shape, dtype=torch.int64, pin_memory=True)
         nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
         sq_h = torch.empty(1, dtype=torch.int64, pin_memory=True)
@@ -203,8 +217,24 @@ class Stepper:
         ctx["depth_order"] = order
         ctx["depth_rect"] = drect
 
+        # ---- per-block candidate lists (two-level binning) ------------------
+        if expand:
+            bsat_np = bsat_h.numpy().reshape(BH + 1, BW + 1)
+            n_blk = int(bsat_np[BH, BW])
+            bvals = torch.empty(max(n_blk, 1), dtype=torch.int32, device=dev)
+            branges = torch.empty(2 * BW * BH, dtype=torch.int64, device=dev)
+            ws = torch.empty(max(B.gs_bin_blocks_workspace_size(C, n_blk, TW, TH), 256),
+                             dtype=torch.uint8, device=dev)
+            tk = clk.tic("bin")
+            B.gs_bin_blocks(proj, C, order, drect, TW, TH, bsat, n_blk, bvals, max(n_blk, 1),
+                            branges, ws, st)
+            clk.toc(tk)
+            del ws
+            ctx.update(block_sat=bsat, block_sat_host=bsat_np, block_vals=bvals,
+                       block_ranges=branges, n_block_entries=n_blk)
+
         # ---- Leaf plan ------------------------------------------------------
-        lm = B.gs_leaf_load_model(tile_bits)
+        lm = B.gs_leaf_load_model(tile_bits, B.GS_BIN_EXPAND if expand else B.GS_BIN_SORT)
         if leaves is None:
             _, lv, li, lb, ov = B.gs_leaf_partition(sat_np, TW, TH, W, H, lm, self.budget)
         else:
@@ -217,7 +247,13 @@ class Stepper:
         # ---- per-Leaf raster: forward + L1 + backward into compact g2d ------
         g2d = torch.zeros(max(C, 1) * 12, dtype=torch.float32, device=dev)
         loss_tiles = torch.zeros(T, dtype=torch.float32, device=dev)
-        bin_ws = torch.empty(max(B.gs_bin_workspace_size(C), 256), dtype=torch.uint8, device=dev)
+        if expand:
+            bin_ws = torch.empty(max(max((B.gs_expand_workspace_size(L, B.block_entries(bsat_np, L))
+                                          for L in lv), default=0), 256),
+                                 dtype=torch.uint8, device=dev)
+        else:
+            bin_ws = torch.empty(max(B.gs_bin_workspace_size(C), 256), dtype=torch.uint8,
+                                 device=dev)
         resident_target = target is not None and target.is_cuda
 
         def leaf_sizes(L, I):
@@ -226,9 +262,12 @@ class Stepper:
             ph = min(16 * y1, H) - 16 * y0
             npx = pw * ph
             nt = (x1 - x0) * (y1 - y0)
-            lb_bits = B.local_tile_bits(L)
-            sizes = [4 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 4, 0, lb_bits),
-                     12 * npx, 4 * npx, 4 * npx, 12 * npx]
+            if expand:
+                sizes = [0, 4 * I, 16 * nt, 0, 12 * npx, 4 * npx, 4 * npx, 12 * npx]
+            else:
+                lb_bits = B.local_tile_bits(L)
+                sizes = [4 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 4, 0, lb_bits),
+                         12 * npx, 4 * npx, 4 * npx, 12 * npx]
             if target is not None and not resident_target:
                 sizes.append(12 * npx)
             return sizes, (16 * x0, 16 * y0, pw, ph)
@@ -263,12 +302,18 @@ class Stepper:
                               counters=cnt_f)
             else:
                 px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
-            tk = clk.tic("bin")
-            B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1), ranges,
-                           bin_ws, st)
-            clk.toc(tk)
+            if expand:
+                tk = clk.tic("expand")
+                B.gs_expand_tiles(proj, bvals, branges, B.block_entries(bsat_np, L), L, TW, TH,
+                                  sat, I, vals, max(I, 1), ranges, bin_ws, st)
+                clk.toc(tk)
+            else:
+                tk = clk.tic("bin")
+                B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1),
+                               ranges, bin_ws, st)
+                clk.toc(tk)
             lb_bits = B.local_tile_bits(L)
-            if I > 0 and lb_bits > 0:
+            if not expand and I > 0 and lb_bits > 0:
                 tk = clk.tic("sort_tiles")
                 B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
                 clk.toc(tk)
@@ -317,6 +362,7 @@ class Stepper:
         if resident_target:
             peak += target.numel() * target.element_size()
         return ViewStats(n_cand=C, n_isect=int(li.sum()), n_isect_square=n_square,
+                         n_block_entries=n_blk if expand else 0,
                          n_leaves=len(lv), leaves=lv,
                          leaf_isect=li, leaf_bytes=lb, over_budget=ov, peak_ws_bytes=int(peak),
                          arena_bytes=int(arena_bytes),

@@ -83,6 +83,8 @@ typedef int32_t gs_status;
 #define GS_DEV_NONFINITE 4u    /* non-finite parameter met; Gaussian culled */
 
 #define GS_TILE 16
+/* tiles per side of a block of the two-level binning (section 4) */
+#define GS_TILE_BLOCK 8
 
 typedef void* gs_stream; /* cudaStream_t */
 
@@ -285,7 +287,15 @@ gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* keys,
  * depth-first order.  Returns GS_WARN_BUDGET if any Leaf is over budget,
  * GS_ERR_CAPACITY if more than max_leaves would be needed (*n_leaves is
  * then the number required). */
-gs_status gs_leaf_load_model(int32_t tile_bits, gs_load_model* out);
+/* gs_leaf_load_model: the per-unit bytes of one Leaf's buffers for the
+ * binning path used (GS_BIN_SORT: gs_bin_tiles + gs_sort_tiles with
+ * tile_bits = bits of the grid's tile count; GS_BIN_EXPAND:
+ * gs_expand_tiles, whose per-view block lists and chunk tables are not part
+ * of a Leaf's load). */
+#define GS_BIN_SORT 0
+#define GS_BIN_EXPAND 1
+gs_status gs_leaf_load_model(int32_t binning, int32_t tile_bits,
+                             gs_load_model* out);
 gs_status gs_leaf_partition(const int64_t* sat_host, int32_t TW, int32_t TH,
                             int32_t width, int32_t height,
                             const gs_load_model* lm, int64_t budget,
@@ -322,6 +332,53 @@ gs_status gs_bin_tiles(const gs_proj* proj, int64_t n_cand,
                        int64_t capacity, int64_t* ranges, int64_t* needed,
                        void* ws, size_t ws_bytes, int32_t* dev_status,
                        gs_stream stream);
+
+/* Two-level binning: the same per-Leaf lists as gs_bin_tiles followed by the
+ * tile sort (bit-identical vals and ranges), without per-entry keys or a
+ * sort of the Leaf's entries.  An implementation choice of this library for
+ * the binning step of the 3D Gaussian Splatting paper (section 6: per-tile
+ * lists ordered by depth); the pages do not describe it.
+ *
+ * gs_block_sat (once per view, may run before the host learns n_cand):
+ * block_sat = (BH + 1) x (BW + 1) summed-area table (zero first row and
+ * column), BW = ceil(TW / GS_TILE_BLOCK), BH likewise, of the number of
+ * candidates whose tile rect meets each block of GS_TILE_BLOCK^2 tiles.
+ * Reads the candidate count *proj->n_cand on the device.
+ *
+ * gs_bin_blocks (once per view): per block, in row-major block order, the
+ * slots of the candidates meeting it in depth order (block_vals), with
+ * block_ranges[2 b], [2 b + 1] = begin, end of block b.  n_entries = the
+ * total (block_sat[BH][BW] from a host copy); must be <= capacity, else
+ * GS_ERR_CAPACITY with *needed.  The workspace also holds the block keys and
+ * their sort.
+ *
+ * gs_expand_tiles (per Leaf): vals/ranges exactly as gs_bin_tiles +
+ * gs_sort_tiles give them (ranges from the tile SAT, n_isect the Leaf's
+ * count from the host SAT).  block_entries: the summed lengths of the block
+ * lists of the blocks meeting the Leaf (from a host copy of block_sat); it
+ * sizes the workspace.  A plan or a per-tile count that does not match the
+ * SAT sets GS_DEV_BOUNDS in *dev_status. */
+size_t gs_block_sat_workspace_size(int32_t TW, int32_t TH);
+gs_status gs_block_sat(const gs_proj* proj, int32_t TW, int32_t TH,
+                       int64_t* block_sat, void* ws, size_t ws_bytes,
+                       int32_t* dev_status, gs_stream stream);
+size_t gs_bin_blocks_workspace_size(int64_t n_cand, int64_t n_entries,
+                                    int32_t TW, int32_t TH);
+gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand,
+                        const int32_t* depth_order, const int16_t* depth_rect,
+                        int32_t TW, int32_t TH, const int64_t* block_sat,
+                        int64_t n_entries, int32_t* block_vals,
+                        int64_t capacity, int64_t* block_ranges,
+                        int64_t* needed, void* ws, size_t ws_bytes,
+                        int32_t* dev_status, gs_stream stream);
+size_t gs_expand_workspace_size(gs_rect leaf, int64_t block_entries);
+gs_status gs_expand_tiles(const gs_proj* proj, const int32_t* block_vals,
+                          const int64_t* block_ranges, int64_t block_entries,
+                          gs_rect leaf, int32_t TW, int32_t TH,
+                          const int64_t* tile_sat, int64_t n_isect,
+                          int32_t* vals, int64_t capacity, int64_t* ranges,
+                          int64_t* needed, void* ws, size_t ws_bytes,
+                          int32_t* dev_status, gs_stream stream);
 
 /* ---- 5. raster forward ---------------------------------------------------
  * Per pixel p of the Leaf, over its tile's list in order: d = (u, v) - p;

@@ -630,17 +630,18 @@ class Capture:
         self.cand_idx = ctx["cand_idx"][:ctx["n_cand"]].cpu().numpy()
 
 
-@pytest.mark.parametrize("name,budget", [("tiny", 384 << 20), ("tiny", 120_000),
-                                         ("ragged", 30_000), ("small3", 200_000),
-                                         ("hd", 384 << 20), ("hd", 20 << 20)])
-def test_end_to_end_step(oracle_mod, name, budget):
+@pytest.mark.parametrize("name,budget,binning", [
+    ("tiny", 384 << 20, "expand"), ("tiny", 120_000, "expand"), ("tiny", 120_000, "sort"),
+    ("ragged", 30_000, "expand"), ("small3", 200_000, "expand"), ("small3", 200_000, "sort"),
+    ("hd", 384 << 20, "expand"), ("hd", 20 << 20, "expand"), ("hd", 20 << 20, "sort")])
+def test_end_to_end_step(oracle_mod, name, budget, binning):
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, cam = scene(name)
     target = synth.random_image(cam.width, cam.height, 12) * 0.6
     ref = oracle_mod.step(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam,
                           target.astype(np.float64))
     model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=budget, fuse_adam=False)
+    stp = Stepper(model, budget=budget, fuse_adam=False, binning=binning)
     cap = Capture(cam.width, cam.height)
     stats = stp.run_view(cam, torch.as_tensor(target).cuda(), hooks=cap)
     stp.check()

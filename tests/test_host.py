@@ -70,7 +70,7 @@ def test_workspace_sizes(gsb):
 def test_load_model_matches_buffers(gsb):
     b = gsb
     for bits in (8, 13, 16, 20):
-        lm = b.gs_leaf_load_model(bits)
+        lm = b.gs_leaf_load_model(bits, b.GS_BIN_SORT)
         passes = 2 * ((bits + 15) // 16)
         n = 5_000_000
         need = 8 * n + b.gs_sort_workspace_size(n, 4, 0, bits)
@@ -78,6 +78,12 @@ def test_load_model_matches_buffers(gsb):
         assert need <= est
         assert lm.bytes_per_pixel == 44 and lm.bytes_per_tile == 16 and lm.align == 512
         assert lm.bytes_per_isect == 16 + (passes + 1) // 2
+    # two-level binning: a Leaf holds its 32-bit values, ranges and pixels
+    lm = b.gs_leaf_load_model(20, b.GS_BIN_EXPAND)
+    assert lm.bytes_per_isect == 4 and lm.bytes_per_pixel == 44 and lm.bytes_per_tile == 16
+    assert lm.fixed_bytes >= 8 * 255  # the 256-byte alignment of up to 8 buffers
+    with pytest.raises(b.GsError):
+        b.gs_leaf_load_model(20, 7)
 
 
 def _lm_list(lm):
@@ -92,7 +98,7 @@ def test_leaf_partition_matches_oracle(gsb, oracle_mod, seed):
     cnt = rng.poisson(rng.uniform(1, 4000), size=(TH, TW)).astype(np.int64)
     cnt[: TH // 3, : TW // 4] *= 40
     sat = oracle_mod.sat(cnt)
-    lm = gsb.gs_leaf_load_model(16)
+    lm = gsb.gs_leaf_load_model(16, gsb.GS_BIN_SORT)
     for budget in (1, 200_000, 5_000_000, 60_000_000, 10 ** 12):
         st, lv, li, lb, ov = gsb.gs_leaf_partition(sat, TW, TH, W, H, lm, budget)
         ol, oi, ob, oo = oracle_mod.leaf_partition(sat, TW, TH, W, H, _lm_list(lm), budget)
@@ -103,6 +109,6 @@ def test_leaf_partition_matches_oracle(gsb, oracle_mod, seed):
 def test_leaf_partition_capacity_retry(gsb, oracle_mod):
     cnt = np.full((40, 50), 3000, np.int64)
     sat = oracle_mod.sat(cnt)
-    lm = gsb.gs_leaf_load_model(12)
+    lm = gsb.gs_leaf_load_model(12, gsb.GS_BIN_SORT)
     st, lv, *_ = gsb.gs_leaf_partition(sat, 50, 40, 800, 640, lm, 300_000, max_leaves=2)
     assert len(lv) > 2  # the wrapper grew the output after GS_ERR_CAPACITY
