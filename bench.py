@@ -59,6 +59,63 @@ def workload_name(a):
             f"SH3, {a.views} views on a radius-4 circle, {a.budget_mib:g} MiB Leaf budget")
 
 
+def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_peak, W, H):
+    """Roofline time of the step: for each stage the larger of its compulsory
+    HBM bytes / measured copy bandwidth and its lane-ops / ALU issue peak,
+    summed; frac = that sum / the measured step time.  Bytes per view:
+      project      N*12 (means for the cull) + N*4 (slot map)
+                   + C*((P-3)*4 + 48 + 8 + 4 + 4) (rest of a candidate's
+                   parameters; record, rect, depth key, candidate index)
+      sort_depth   4 passes x C x 16 (keys + values in and out) + C*4
+                   (histogram read) + C*20 (rect gather)
+      bin          C*8 (block counts) + C*12 (order + rects) + E_blk*8
+                   (keys + values) + 2 passes x E_blk x 20 (block sort)
+      sort_tiles   2 passes x I x 20 (the bin + sort path only)
+      expand       2 passes x R_blk x 12 (block entries + rect gathers) +
+                   I*4 (the Leaf lists)
+      raster_fwd   I*4 + C*48 + pixels*(20 + 12 + 12) (colour, T, last;
+                   target; dL/dcolour)
+      raster_bwd   I*4 + C*48 + pixels*(20 + 12) + C*48 (gradient atomics)
+      project_bwd  N*P*24 (p, m, v read and written) + C*(48 + 48 + 56*2)
+                   (g2d, record, fp64 geometric scratch) + N*4 (slot map)
+    (E_blk = block-list entries, R_blk = their reads over the Leaves, I =
+    tile-list entries, C = candidates, N = Gaussians.)  The raster stages'
+    lane-ops are the accounting view's counters scaled to each view's I."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    n, P = model.n, model.P
+    k = len(stats)
+    C = sum(s.n_cand for s in stats) / k
+    I = sum(s.n_isect for s in stats) / k
+    E = sum(s.n_block_entries for s in stats) / k
+    R = sum(s.n_block_reads for s in stats) / k
+    px = W * H
+    expand = a.binning == "expand"
+    byt = {
+        "project": n * 12 + n * 4 + C * ((P - 3) * 4 + 64),
+        "sort_depth": C * (4 * 16 + 4 + 20),
+        "bin": (C * 8 + C * 12 + E * 8 + E * 40) if expand else C * 12 * max(1, stats[0].n_leaves) + I * 8,
+        "sort_tiles": 0.0 if expand else I * 40,
+        "expand": (R * 24 + I * 4) if expand else 0.0,
+        "raster_fwd": I * 4 + C * 48 + px * 44,
+        "raster_bwd": I * 4 + C * 96 + px * 32,
+        "project_bwd": n * P * 24 + C * 208 + n * 4,
+    }
+    scale = I / max(acc.n_isect, 1)
+    ops = {"raster_fwd": ops_fwd * scale, "raster_bwd": ops_bwd * scale}
+    stages, total = {}, 0.0
+    for s, b in byt.items():
+        t_hbm = b / hbm * 1e3
+        t_alu = ops.get(s, 0.0) / alu_peak * 1e3
+        t = max(t_hbm, t_alu)
+        total += t
+        stages[s] = {"bound": "alu" if t_alu > t_hbm else "hbm", "roofline_ms": round(t, 4),
+                     "measured_ms": round(per_step.get(s, 0.0), 4), "bytes": round(b),
+                     "lane_ops": round(ops.get(s, 0.0))}
+    measured = sum(per_step.values())
+    return {"roofline_ms": round(total, 4), "stages_ms": round(measured, 4),
+            "frac": round(total / measured, 4) if measured > 0 else None, "stages": stages}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -315,6 +372,10 @@ def main():
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
                 "traffic": None}
 
+    # ---- step roofline: per stage max(algorithmic bytes / HBM, lane-ops / ALU)
+    step_roof = step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks,
+                              alu_peak, W, H)
+
     # ---- end to end through host buffers --------------------------------------
     e2e = None
     if not a.no_e2e:
@@ -345,9 +406,14 @@ def main():
             dist.all_reduce(t)
             e2e_isect = float(t.item())
         TW, TH = (W + 15) // 16, (H + 15) // 16
+        BW, BH = (TW + 7) // 8, (TH + 7) // 8
+        # per step: the tile SAT, candidate count, 3-sigma count, block SAT
+        # (two-level binning) and the loss
+        d2h = (TW + 1) * (TH + 1) * 8 + 4 + 8 + 8
+        if a.binning == "expand":
+            d2h += (BW + 1) * (BH + 1) * 8
         e2e = {"value": e2e_isect / (ems / 1e3), "unit": UNIT, "ms_per_step": ems / a.steps,
-               "h2d_bytes_per_step": 3 * W * H * 4,
-               "d2h_bytes_per_step": (TW + 1) * (TH + 1) * 8 + 4 + 8}
+               "h2d_bytes_per_step": 3 * W * H * 4, "d2h_bytes_per_step": d2h}
 
     # ---- CPU baseline (rank 0, one GPU) ---------------------------------------
     cpu = None
@@ -389,7 +455,7 @@ def main():
             "stage_launches_per_step": {s: stage_n[s] / n_steps for s in STAGES},
             "work": {"fwd_pairs_evaluated": cnt[0], "fwd_pairs_composited": cnt[1],
                      "bwd_pairs_evaluated": cnt[2], "bwd_pairs_differentiated": cnt[3]},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk,
         }
         print(json.dumps(out))

@@ -50,6 +50,7 @@ class ViewStats:
     n_isect: int          # entries of the (tight) tile lists
     n_isect_square: int   # tiles of the candidates' plain 3-sigma squares
     n_block_entries: int  # entries of the per-block lists (two-level binning)
+    n_block_reads: int    # block-list entries the Leaves' expansions read (summed)
     n_leaves: int
     leaves: np.ndarray
     leaf_isect: np.ndarray
@@ -363,6 +364,7 @@ class Stepper:
             peak += target.numel() * target.element_size()
         return ViewStats(n_cand=C, n_isect=int(li.sum()), n_isect_square=n_square,
                          n_block_entries=n_blk if expand else 0,
+                         n_block_reads=sum(B.block_entries(bsat_np, L) for L in lv) if expand else 0,
                          n_leaves=len(lv), leaves=lv,
                          leaf_isect=li, leaf_bytes=lb, over_budget=ov, peak_ws_bytes=int(peak),
                          arena_bytes=int(arena_bytes),
