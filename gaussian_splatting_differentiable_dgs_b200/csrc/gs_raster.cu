@@ -119,8 +119,7 @@ struct TileGeom {
 };
 
 struct WarpPix {
-  int lx, ly0;            // first pixel of the lane (tile-relative)
-  float x0, x1, y0, y1;   // the warp's pixel-centre box (tile-relative)
+  int lx, ly0;  // first pixel of the lane (tile-relative)
 };
 
 template <int PPT>
@@ -131,10 +130,6 @@ __device__ __forceinline__ WarpPix warp_pixels(int t) {
   WarpPix p;
   p.lx = bx0 + l % G::BW;
   p.ly0 = by0 + l / G::BW;
-  p.x0 = (float)bx0 + 0.5f;
-  p.x1 = (float)(bx0 + G::BW) - 0.5f;
-  p.y0 = (float)by0 + 0.5f;
-  p.y1 = (float)(by0 + G::BH) - 0.5f;
   return p;
 }
 
@@ -143,13 +138,42 @@ __device__ __forceinline__ WarpPix warp_pixels(int t) {
 // projection stores (inflated far beyond the fp32 error of the per-pixel
 // alpha and rounded up): a warp whose pixel box misses it would have
 // skipped the Gaussian at every pixel anyway, so culling by it leaves every
-// result bit-identical.
+// result bit-identical.  The staging thread turns the box into one bit per
+// warp; each warp then walks only its own compacted list of records.
 __device__ __forceinline__ float4 alpha_box(const Staged& st) {
   return make_float4(st.gx - st.hx, st.gx + st.hx, st.gy - st.hy, st.gy + st.hy);
 }
 
-__device__ __forceinline__ bool box_misses(const float4& b, const WarpPix& p) {
-  return (b.x > p.x1) | (b.y < p.x0) | (b.z > p.y1) | (b.w < p.y0);
+// Bit w set if the alpha box meets the pixel-centre box of warp w.
+template <int PPT>
+__device__ __forceinline__ unsigned warp_mask(const float4& b) {
+  using G = TileGeom<PPT>;
+  unsigned m = 0;
+#pragma unroll
+  for (int w = 0; w < G::NW; ++w) {
+    const float x0 = (float)((w % G::BX) * G::BW) + 0.5f, x1 = x0 + (float)(G::BW - 1);
+    const float y0 = (float)((w / G::BX) * G::BH) + 0.5f, y1 = y0 + (float)(G::BH - 1);
+    const bool miss = (b.x > x1) | (b.y < x0) | (b.z > y1) | (b.w < y0);
+    m |= miss ? 0u : (1u << w);
+  }
+  return m;
+}
+
+// The batch positions j in [j0, cnt) whose record meets warp w's pixels, in
+// ascending order, into list[0..n); returns n (warp-uniform).
+__device__ __forceinline__ int warp_list(const uint8_t* __restrict__ s_mask, int j0, int cnt, int w,
+                                         int lane, uint8_t* __restrict__ list) {
+  int n = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c = j0; c < cnt; c += 32) {
+    const int j = c + lane;
+    const bool m = j < cnt && ((s_mask[j] >> w) & 1u);
+    const unsigned b = __ballot_sync(0xffffffffu, m);
+    if (m) list[n + __popc(b & lt)] = (uint8_t)j;
+    n += __popc(b);
+  }
+  __syncwarp();
+  return n;
 }
 
 // ---------------------------------------------------------------------------
@@ -162,14 +186,16 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              int32_t* dev_status) {
   using G = TileGeom<PPT>;
   constexpr int NT = G::NT;
-  __shared__ float4 sBox[NT], sA[NT], sB[NT];
+  __shared__ float4 sA[NT], sB[NT];
   __shared__ float sC[NT];
+  __shared__ uint8_t s_mask[NT];
+  __shared__ uint8_t s_list[G::NW][NT];
   __shared__ float s_red[G::NW];
   const int lw = leaf.x1 - leaf.x0;
   const int ltile = blockIdx.x;
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile], end = ranges[2 * ltile + 1];
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const WarpPix wp = warp_pixels<PPT>(t);
   const float fpx = (float)wp.lx + 0.5f;
   float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
@@ -194,7 +220,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     const int64_t e = base + t;
     if (e < end) {
       const Staged st = stage_record(rec, vals[e], tx, ty);
-      sBox[t] = alpha_box(st);
+      s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
       sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
       sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
       sC[t] = st.b;
@@ -202,18 +228,22 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     __syncthreads();
     if (__all_sync(0xffffffffu, mine_done)) continue;  // nothing left for this warp
     const int cnt = (int)min((int64_t)NT, end - base);
-    const int pos0 = (int)(base - begin);
-    for (int j = 0; j < cnt; ++j) {
-      if ((j & 31) == 31) {
+    const int pos1 = (int)(base - begin) + 1;
+    const int nl = warp_list(s_mask, 0, cnt, w, lane, s_list[w]);
+    for (int i0 = 0; i0 < nl; i0 += 32) {
+      if (i0 > 0) {
         bool d_all = true;
 #pragma unroll
         for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
         if (__all_sync(0xffffffffu, d_all)) break;
       }
-      if (box_misses(sBox[j], wp)) continue;  // warp-uniform
+      const int i1 = min(nl, i0 + 32);
+      for (int i = i0; i < i1; ++i) {
+      const int j = s_list[w][i];
       const float4 A = sA[j];
       const float4 B = sB[j];
       const float Bb = sC[j];
+      const int posn = pos1 + j;
 #pragma unroll
       for (int k = 0; k < PPT; ++k) {
         if (done[k]) continue;
@@ -231,7 +261,8 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         Cg[k] = fmaf(B.w, wgt, Cg[k]);
         Cb[k] = fmaf(Bb, wgt, Cb[k]);
         T[k] = Tn;
-        lastp[k] = pos0 + j + 1;
+        lastp[k] = posn;
+      }
       }
     }
   }
@@ -379,8 +410,10 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              float* __restrict__ g2d, int32_t* dev_status) {
   using G = TileGeom<PPT>;
   constexpr int NT = G::NT;
-  __shared__ float4 sBox[NT], sA[NT], sB[NT];
-  __shared__ float4 sC[NT];       // {b, s1, s2, slot bits}
+  __shared__ float4 sA[NT], sB[NT];
+  __shared__ float4 sC[NT];       // {b, 2 s1, 2 s2, slot bits}
+  __shared__ uint8_t s_mask[NT];
+  __shared__ uint8_t s_list[G::NW][NT];
   __shared__ float sg[NT][12];
   __shared__ int s_touched[NT];
   __shared__ int s_maxlast;
@@ -388,10 +421,11 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   const int ltile = blockIdx.x;
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile];
-  const int t = threadIdx.x, lane = t & 31;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const WarpPix wp = warp_pixels<PPT>(t);
   const float fpx = (float)wp.lx + 0.5f;
-  float fpy[PPT], T[PPT], Ar[PPT], Ag[PPT], Ab[PPT], gr[PPT], gg[PPT], gb[PPT];
+  // S = sum_c g_c A_c, A_c = colour composited behind the current entry
+  float fpy[PPT], T[PPT], S[PPT], gr[PPT], gg[PPT], gb[PPT];
   int lastp[PPT];
   if (t == 0) s_maxlast = 0;
   for (int e = t; e < NT * 12; e += NT) (&sg[0][0])[e] = 0.0f;
@@ -403,7 +437,7 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     const int ly = wp.ly0 + k * G::LROWS;
     fpy[k] = (float)ly + 0.5f;
     const int x = tx * kTile + wp.lx, y = ty * kTile + ly;
-    Ar[k] = Ag[k] = Ab[k] = 0.0f;
+    S[k] = 0.0f;
     if (x < W && y < H) {
       const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
       T[k] = px.T_final[o];
@@ -430,16 +464,17 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     if (t < cnt) {
       const int pos = bend - 1 - t;
       const Staged st = stage_record(rec, vals[begin + pos], tx, ty);
-      sBox[t] = alpha_box(st);
+      s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
       sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
       sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
-      sC[t] = make_float4(st.b, st.s1, st.s2, __int_as_float(st.slot));
+      sC[t] = make_float4(st.b, 2.0f * st.s1, 2.0f * st.s2, __int_as_float(st.slot));
     }
     __syncthreads();
     // positions at or beyond every lane's `last` need no work in this warp
     const int jstart = max(0, bend - warp_last);
-    for (int j = jstart; j < cnt; ++j) {
-      if (box_misses(sBox[j], wp)) continue;  // warp-uniform
+    const int nl = warp_list(s_mask, jstart, cnt, w, lane, s_list[w]);
+    for (int i = 0; i < nl; ++i) {
+      const int j = s_list[w][i];
       const int pos = bend - 1 - j;
       const float4 A = sA[j];
       const float4 B = sB[j];
@@ -463,25 +498,25 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         acc[7] = fmaf(wgt, gg[k], acc[7]);
         acc[8] = fmaf(wgt, gb[k], acc[8]);
         // dL/dalpha = sum_c g_c (rgb_c T_i - A_c / (1 - alpha))
-        float da = gr[k] * (B.z * Tb - Ar[k] * inv);
-        da = fmaf(gg[k], B.w * Tb - Ag[k] * inv, da);
-        da = fmaf(gb[k], Cc.x * Tb - Ab[k] * inv, da);
-        Ar[k] = fmaf(B.z, wgt, Ar[k]);
-        Ag[k] = fmaf(B.w, wgt, Ag[k]);
-        Ab[k] = fmaf(Cc.x, wgt, Ab[k]);
+        //           = T_i (g . rgb) - S / (1 - alpha)
+        const float grgb = fmaf(gb[k], Cc.x, fmaf(gg[k], B.w, gr[k] * B.z));
+        const float da = fmaf(Tb, grgb, -S[k] * inv);
+        S[k] = fmaf(wgt, grgb, S[k]);
         T[k] = Tb;
         if (ev.araw <= kAlphaMax) {
           const float dq = -ev.alpha * da;         // dL/dq (natural units)
           acc[5] = fmaf(ev.G, da, acc[5]);          // dL/dopacity
-          const float s1t = 2.0f * Cc.y * ev.t1;    // dq/du = a dx + b dy
+          const float s1t = Cc.y * ev.t1;           // dq/du = a dx + b dy
           acc[0] = fmaf(dq, s1t, acc[0]);
-          acc[1] = fmaf(dq, fmaf(s1t, A.z, 2.0f * Cc.z * ev.dy), acc[1]);  // dq/dv
-          const float hdx = 0.5f * ev.dx;
-          acc[2] = fmaf(dq * hdx, ev.dx, acc[2]);
+          acc[1] = fmaf(dq, fmaf(s1t, A.z, Cc.z * ev.dy), acc[1]);  // dq/dv
+          const float hq = 0.5f * dq;
+          acc[2] = fmaf(hq * ev.dx, ev.dx, acc[2]);
           acc[3] = fmaf(dq * ev.dx, ev.dy, acc[3]);
-          acc[4] = fmaf(dq * 0.5f * ev.dy, ev.dy, acc[4]);
+          acc[4] = fmaf(hq * ev.dy, ev.dy, acc[4]);
         }
       }
+      // reduce first: per-lane shared atomics on the same 9 words cost more
+      // than the reduction, even with only 2 lanes kept
       if (__any_sync(0xffffffffu, any)) {
         const float tot = warp_reduce_scatter9(acc, lane);
         const int idx = (lane >> 1) & 15;
@@ -613,7 +648,7 @@ extern "C" gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals, con
   const int W = cam->width, H = cam->height;
   const bool cnt = px->counters != nullptr;
 #define GS_BWD(P, C) k_raster_bwd<P, C><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, a, g2d, dev_status)
-  switch (pick_ppt(flags, 2)) {
+  switch (pick_ppt(flags, 4)) {
     case 1: if (cnt) GS_BWD(1, true); else GS_BWD(1, false); break;
     case 2: if (cnt) GS_BWD(2, true); else GS_BWD(2, false); break;
     default: if (cnt) GS_BWD(4, true); else GS_BWD(4, false); break;

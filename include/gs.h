@@ -387,8 +387,9 @@ gs_status gs_expand_tiles(const gs_proj* proj, const int32_t* block_vals,
  * T' < 1e-4; else C += rgb alpha T, T = T'.  Background 0.  Writes img,
  * T_final, last; if px->target is set, also the L1 loss terms (as
  * gs_loss_l1).  fp32 arithmetic.
- * flags & 7 selects the pixels per thread (1, 2 or 4; 0 = default); the
- * result does not depend on it.  The same flag applies to gs_raster_bwd. */
+ * flags & 7 selects the pixels per thread (1, 2 or 4; 0 = the default, 2
+ * here and 4 in gs_raster_bwd, the faster shapes on B200); the result does
+ * not depend on it.  The same flag applies to gs_raster_bwd. */
 gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals,
                         const int64_t* ranges, gs_rect leaf,
                         const gs_camera* cam, const gs_pixels* px,
