@@ -70,6 +70,12 @@ __device__ __forceinline__ Staged stage_record(const float4* __restrict__ rec, i
   return s;
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct Eval {
   float dx, dy, t1, G, araw, alpha;
 };
@@ -491,7 +497,9 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         if (ev.alpha < kAlphaMin) continue;
         if (COUNT) ++n_kept;
         any = true;
-        const float inv = __frcp_rn(1.0f - ev.alpha);
+        // T only scales gradient values here (no decision depends on it), so
+        // the hardware reciprocal (about 1 ulp) is enough
+        const float inv = rcp_approx(1.0f - ev.alpha);
         const float Tb = T[k] * inv;          // transmittance before this entry
         const float wgt = ev.alpha * Tb;
         acc[6] = fmaf(wgt, gr[k], acc[6]);

@@ -407,7 +407,8 @@ gs_status gs_loss_total(const float* loss_tiles, int64_t n, double* loss,
 
 /* ---- 7. raster backward --------------------------------------------------
  * Reverse blend over list positions last-1 .. 0 with the forward's skip
- * tests, transmittance recovered as T_i = T_{i+1} / (1 - alpha_i).
+ * tests, transmittance recovered as T_i = T_{i+1} / (1 - alpha_i) (with the
+ * hardware reciprocal: T only scales gradient values, no decision).
  * Accumulates (adds) per candidate slot into g2d[slot][12] the gradients
  * {du, dv, da, db, dc, dopacity, dR, dG, dB, 0, 0, 0} ((a, b, c) = conic)
  * with per-tile reduction before the global atomics. */
