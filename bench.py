@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--views", type=int, default=8)
     ap.add_argument("--budget-mib", type=float, default=384)
     ap.add_argument("--raster-ppt", type=int, default=0)
-    ap.add_argument("--binning", default="expand", choices=["expand", "sort"])
+    ap.add_argument("--binning", default="fused", choices=["fused", "expand", "sort"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
@@ -73,9 +73,10 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
       sort_tiles   2 passes x I x 20 (the bin + sort path only)
       expand       2 passes x R_blk x 12 (block entries + rect gathers) +
                    I*4 (the Leaf lists)
-      raster_fwd   I*4 + C*48 + pixels*(20 + 12 + 12) (colour, T, last;
-                   target; dL/dcolour)
-      raster_bwd   I*4 + C*48 + pixels*(20 + 12) + C*48 (gradient atomics)
+      raster_fwd   C*48 + pixels*(20 + 12 + 12) (records; colour, T, last;
+                   target; dL/dcolour; the list entries a tile reads stop where
+                   its pixels saturate, so none are counted)
+      raster_bwd   C*48 + pixels*(20 + 12) + C*48 (gradient atomics)
       project_bwd  N*P*24 (p, m, v read and written) + C*(48 + 48 + 56*2)
                    (g2d, record, fp64 geometric scratch) + N*4 (slot map)
     (E_blk = block-list entries, R_blk = their reads over the Leaves, I =
@@ -89,15 +90,15 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
     E = sum(s.n_block_entries for s in stats) / k
     R = sum(s.n_block_reads for s in stats) / k
     px = W * H
-    expand = a.binning == "expand"
+    expand = a.binning in ("expand", "fused")
     byt = {
         "project": n * 12 + n * 4 + C * ((P - 3) * 4 + 64),
         "sort_depth": C * (4 * 16 + 4 + 20),
         "bin": (C * 8 + C * 12 + E * 8 + E * 40) if expand else C * 12 * max(1, stats[0].n_leaves) + I * 8,
         "sort_tiles": 0.0 if expand else I * 40,
-        "expand": (R * 24 + I * 4) if expand else 0.0,
-        "raster_fwd": I * 4 + C * 48 + px * 44,
-        "raster_bwd": I * 4 + C * 96 + px * 32,
+        "expand": (R * 24 + I * 4) if a.binning == "expand" else 0.0,
+        "raster_fwd": C * 48 + px * 44,
+        "raster_bwd": C * 96 + px * 32,
         "project_bwd": n * P * 24 + C * 208 + n * 4,
     }
     scale = I / max(acc.n_isect, 1)
@@ -410,7 +411,7 @@ def main():
         # per step: the tile SAT, candidate count, 3-sigma count, block SAT
         # (two-level binning) and the loss
         d2h = (TW + 1) * (TH + 1) * 8 + 4 + 8 + 8
-        if a.binning == "expand":
+        if a.binning in ("expand", "fused"):
             d2h += (BW + 1) * (BH + 1) * 8
         e2e = {"value": e2e_isect / (ems / 1e3), "unit": UNIT, "ms_per_step": ems / a.steps,
                "h2d_bytes_per_step": 3 * W * H * 4, "d2h_bytes_per_step": d2h}

@@ -104,6 +104,7 @@ SYMBOLS = [
     "gs_bin_workspace_size", "gs_bin_tiles",
     "gs_block_sat_workspace_size", "gs_block_sat", "gs_bin_blocks_workspace_size",
     "gs_bin_blocks", "gs_expand_workspace_size", "gs_expand_tiles",
+    "gs_tile_ranges", "gs_raster_fwd_blocks",
     "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
     "gs_project_bwd", "gs_adam",
 ]
@@ -144,6 +145,9 @@ def _load():
         "gs_expand_tiles": (i32, [P(gs_proj), p, p, i64, gs_rect, i32, i32, p, i64, p, i64, p,
                                   P(i64), p, sz, p, p]),
         "gs_raster_fwd": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), u32, p, p]),
+        "gs_tile_ranges": (i32, [p, i32, i32, gs_rect, p, p]),
+        "gs_raster_fwd_blocks": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), p,
+                                       i64, i64, p, P(i64), u32, p, p]),
         "gs_loss_l1": (i32, [P(gs_pixels), gs_rect, P(gs_camera), p]),
         "gs_loss_total": (i32, [p, i64, p, p]),
         "gs_raster_bwd": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), p, u32, p,
@@ -388,6 +392,23 @@ def gs_raster_fwd(proj: gs_proj, vals, ranges, leaf, cam: gs_camera, px: gs_pixe
                                                  gs_rect(*[int(v) for v in leaf]), C.byref(cam),
                                                  C.byref(px), flags, ptr(dev_status),
                                                  _stream(stream)))
+
+
+def gs_tile_ranges(tile_sat, TW, TH, leaf, ranges, stream=None):
+    return _ok("gs_tile_ranges", _L.gs_tile_ranges(ptr(tile_sat), TW, TH,
+                                                   gs_rect(*[int(v) for v in leaf]), ptr(ranges),
+                                                   _stream(stream)))
+
+
+def gs_raster_fwd_blocks(proj: gs_proj, block_vals, block_ranges, leaf, cam: gs_camera,
+                         px: gs_pixels, vals, capacity, n_isect, ranges, dev_status, flags=0,
+                         stream=None):
+    needed = C.c_int64(0)
+    st = _L.gs_raster_fwd_blocks(C.byref(proj), ptr(block_vals), ptr(block_ranges),
+                                 gs_rect(*[int(v) for v in leaf]), C.byref(cam), C.byref(px),
+                                 ptr(vals), capacity, n_isect, ptr(ranges), C.byref(needed), flags,
+                                 ptr(dev_status), _stream(stream))
+    return _ok("gs_raster_fwd_blocks", st, needed.value if st == GS_ERR_CAPACITY else None)
 
 
 def gs_loss_l1(px: gs_pixels, leaf, cam: gs_camera, stream=None):

@@ -661,3 +661,16 @@ extern "C" gs_status gs_expand_tiles(const gs_proj* proj, const int32_t* block_v
   GS_LAUNCH_CHECK();
   return GS_OK;
 }
+
+extern "C" gs_status gs_tile_ranges(const int64_t* tile_sat, int32_t TW, int32_t TH, gs_rect leaf,
+                                    int64_t* ranges, gs_stream stream) {
+  if (!tile_sat || !ranges || TW <= 0 || TH <= 0) return GS_ERR_ARG;
+  if (leaf.x0 < 0 || leaf.y0 < 0 || leaf.x1 <= leaf.x0 || leaf.y1 <= leaf.y0 || leaf.x1 > TW ||
+      leaf.y1 > TH)
+    return GS_ERR_ARG;
+  const int64_t ntiles = (int64_t)(leaf.x1 - leaf.x0) * (leaf.y1 - leaf.y0);
+  k_ranges<<<(unsigned)((ntiles + 255) / 256), 256, 0, to_stream(stream)>>>(tile_sat, leaf, TW,
+                                                                             ranges);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}

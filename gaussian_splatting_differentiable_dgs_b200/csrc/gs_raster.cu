@@ -17,6 +17,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "gs_internal.cuh"
 
@@ -167,40 +168,66 @@ __device__ __forceinline__ unsigned warp_mask(const float4& b) {
 
 // The batch positions j in [j0, cnt) whose record meets warp w's pixels, in
 // ascending order, into list[0..n); returns n (warp-uniform).
+template <class LT>
 __device__ __forceinline__ int warp_list(const uint8_t* __restrict__ s_mask, int j0, int cnt, int w,
-                                         int lane, uint8_t* __restrict__ list) {
+                                         int lane, LT* __restrict__ list) {
   int n = 0;
   const unsigned lt = (1u << lane) - 1u;
   for (int c = j0; c < cnt; c += 32) {
     const int j = c + lane;
     const bool m = j < cnt && ((s_mask[j] >> w) & 1u);
     const unsigned b = __ballot_sync(0xffffffffu, m);
-    if (m) list[n + __popc(b & lt)] = (uint8_t)j;
+    if (m) list[n + __popc(b & lt)] = (LT)j;
     n += __popc(b);
   }
   __syncwarp();
   return n;
 }
 
+// Source of a tile's list for the forward when it is built on the fly: the
+// depth-ordered candidate list of the tile's block of GS_TILE_BLOCK^2 tiles,
+// filtered by "tile inside the candidate's rect" (which keeps the order, so
+// the result is the tile's list), written to vals_out as it is consumed.
+struct BlockSrc {
+  const short4* rect;
+  const int32_t* block_vals;
+  const int64_t* block_ranges;
+  int BW;
+  int32_t* vals_out;
+  int64_t* ranges_io;  // in: the tile's segment [begin, end); out: end = begin + written
+};
+
 // ---------------------------------------------------------------------------
 // forward
 // ---------------------------------------------------------------------------
-template <int PPT, bool COUNT>
+// BLK = false: the tile's list is vals[ranges]; BLK = true: it is built
+// from the block list (BlockSrc), in fills of at least NT entries (so a fill
+// holds fewer than 2 NT), and only as far as the tile's pixels need it.
+template <int PPT, bool COUNT, bool BLK>
 __global__ void __launch_bounds__(256 / PPT)
 k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
-             const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
-             int32_t* dev_status) {
+             const int64_t* ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
+             BlockSrc bsrc, int32_t* dev_status) {
   using G = TileGeom<PPT>;
   constexpr int NT = G::NT;
-  __shared__ float4 sA[NT], sB[NT];
-  __shared__ float sC[NT];
-  __shared__ uint8_t s_mask[NT];
-  __shared__ uint8_t s_list[G::NW][NT];
+  constexpr int CAP = BLK ? 2 * NT : NT;
+  using LT = std::conditional_t<(CAP <= 256), uint8_t, uint16_t>;
+  __shared__ float4 sA[CAP], sB[CAP];
+  __shared__ float sC[CAP];
+  __shared__ uint8_t s_mask[CAP];
+  __shared__ LT s_list[G::NW][CAP];
   __shared__ float s_red[G::NW];
+  __shared__ int s_wcnt[G::NW];
   const int lw = leaf.x1 - leaf.x0;
   const int ltile = blockIdx.x;
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile], end = ranges[2 * ltile + 1];
+  int64_t bp = 0, be = 0, n_done = 0;  // block-list cursor / end, entries consumed
+  if (BLK) {
+    const int64_t b = (int64_t)(ty / GS_TILE_BLOCK) * bsrc.BW + tx / GS_TILE_BLOCK;
+    bp = bsrc.block_ranges[2 * b];
+    be = bsrc.block_ranges[2 * b + 1];
+  }
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const WarpPix wp = warp_pixels<PPT>(t);
   const float fpx = (float)wp.lx + 0.5f;
@@ -218,24 +245,70 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     Cr[k] = Cg[k] = Cb[k] = 0.0f;
     lastp[k] = 0;
   }
-  for (int64_t base = begin; base < end; base += NT) {
+  bool bad = false;
+  for (int64_t base = begin;; base += NT) {
+    if (!BLK && base >= end) break;
     bool mine_done = true;
 #pragma unroll
     for (int k = 0; k < PPT; ++k) mine_done = mine_done && done[k];
     if (__syncthreads_count(mine_done) == NT) break;
-    const int64_t e = base + t;
-    if (e < end) {
-      const Staged st = stage_record(rec, vals[e], tx, ty);
-      s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
-      sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-      sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
-      sC[t] = st.b;
+    int cnt, pos1;
+    if (BLK) {
+      if (bp >= be) break;
+      // fill: filter block-list batches of NT until at least NT entries
+      const unsigned ltm = (1u << lane) - 1u;
+      cnt = 0;
+      while (cnt < NT && bp < be) {
+        const int64_t q = bp + t;
+        bool hit = false;
+        int32_t slot = 0;
+        if (q < be) {
+          slot = bsrc.block_vals[q];
+          const short4 r = bsrc.rect[slot];
+          hit = (r.x <= tx) & (tx < r.z) & (r.y <= ty) & (ty < r.w);
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, hit);
+        if (lane == 0) s_wcnt[w] = __popc(bal);
+        __syncthreads();
+        int wb = 0, tot = 0;
+#pragma unroll
+        for (int ww = 0; ww < G::NW; ++ww) {
+          const int c = s_wcnt[ww];
+          wb += ww < w ? c : 0;
+          tot += c;
+        }
+        if (hit) {
+          const int k = cnt + wb + __popc(bal & ltm);
+          const Staged st = stage_record(rec, slot, tx, ty);
+          s_mask[k] = (uint8_t)warp_mask<PPT>(alpha_box(st));
+          sA[k] = make_float4(st.gx, st.gy, st.beta, st.ns1);
+          sB[k] = make_float4(st.ns2, st.opac, st.r, st.g);
+          sC[k] = st.b;
+          const int64_t o = begin + n_done + k;
+          if (o < end) bsrc.vals_out[o] = slot;
+          else bad = true;
+        }
+        cnt += tot;
+        bp += NT;
+        __syncthreads();  // s_wcnt is rewritten by the next batch
+      }
+      pos1 = (int)n_done + 1;
+      n_done += cnt;
+    } else {
+      const int64_t e = base + t;
+      if (e < end) {
+        const Staged st = stage_record(rec, vals[e], tx, ty);
+        s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
+        sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
+        sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+        sC[t] = st.b;
+      }
+      __syncthreads();
+      cnt = (int)min((int64_t)NT, end - base);
+      pos1 = (int)(base - begin) + 1;
     }
-    __syncthreads();
     if (__all_sync(0xffffffffu, mine_done)) continue;  // nothing left for this warp
-    const int cnt = (int)min((int64_t)NT, end - base);
-    const int pos1 = (int)(base - begin) + 1;
-    const int nl = warp_list(s_mask, 0, cnt, w, lane, s_list[w]);
+    const int nl = warp_list<LT>(s_mask, 0, cnt, w, lane, s_list[w]);
     for (int i0 = 0; i0 < nl; i0 += 32) {
       if (i0 > 0) {
         bool d_all = true;
@@ -275,6 +348,10 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   if (COUNT) {
     atomicAdd(&px.counters[0], (unsigned long long)n_vis);
     atomicAdd(&px.counters[1], (unsigned long long)n_kept);
+  }
+  if (BLK) {
+    if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
+    if (t == 0) bsrc.ranges_io[2 * ltile + 1] = begin + (n_done < end - begin ? n_done : end - begin);
   }
   // epilogue: outputs and the fused L1 terms
   float lsum = 0.0f;
@@ -478,7 +555,7 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     __syncthreads();
     // positions at or beyond every lane's `last` need no work in this warp
     const int jstart = max(0, bend - warp_last);
-    const int nl = warp_list(s_mask, jstart, cnt, w, lane, s_list[w]);
+    const int nl = warp_list<uint8_t>(s_mask, jstart, cnt, w, lane, s_list[w]);
     for (int i = 0; i < nl; ++i) {
       const int j = s_list[w][i];
       const int pos = bend - 1 - j;
@@ -610,7 +687,47 @@ extern "C" gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals, con
   const unsigned nb = (unsigned)ntiles;
   const int W = cam->width, H = cam->height;
   const bool cnt = px->counters != nullptr;
-#define GS_FWD(P, C) k_raster_fwd<P, C><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, TW, a, dev_status)
+  const BlockSrc none{nullptr, nullptr, nullptr, 0, nullptr, nullptr};
+#define GS_FWD(P, C) \
+  k_raster_fwd<P, C, false><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, TW, a, none, dev_status)
+  switch (pick_ppt(flags, 2)) {
+    case 1: if (cnt) GS_FWD(1, true); else GS_FWD(1, false); break;
+    case 2: if (cnt) GS_FWD(2, true); else GS_FWD(2, false); break;
+    default: if (cnt) GS_FWD(4, true); else GS_FWD(4, false); break;
+  }
+#undef GS_FWD
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" gs_status gs_raster_fwd_blocks(const gs_proj* proj, const int32_t* block_vals,
+                                          const int64_t* block_ranges, gs_rect leaf,
+                                          const gs_camera* cam, const gs_pixels* px,
+                                          int32_t* vals, int64_t capacity, int64_t n_isect,
+                                          int64_t* ranges, int64_t* needed, uint32_t flags,
+                                          int32_t* dev_status, gs_stream stream) {
+  if (!proj || !ranges || !cam || !block_ranges || !check_leaf(leaf, cam) ||
+      !check_pixels(px, leaf, cam) || n_isect < 0)
+    return GS_ERR_ARG;
+  if (n_isect > capacity) {
+    if (needed) *needed = n_isect;
+    return GS_ERR_CAPACITY;
+  }
+  if (!px->T_final || !px->last || (px->target && !px->dL_dimg)) return GS_ERR_ARG;
+  if (n_isect > 0 && (!vals || !block_vals || !proj->rect)) return GS_ERR_ARG;
+  if (!aligned(proj->rec, 16) || !aligned(proj->rect, 8)) return GS_ERR_ARG;
+  const int64_t ntiles = (int64_t)(leaf.x1 - leaf.x0) * (leaf.y1 - leaf.y0);
+  const PixArgs a = to_args(px);
+  const int TW = (int)tiles_x(cam->width);
+  cudaStream_t s = to_stream(stream);
+  const float4* rec = reinterpret_cast<const float4*>(proj->rec);
+  const unsigned nb = (unsigned)ntiles;
+  const int W = cam->width, H = cam->height;
+  const bool cnt = px->counters != nullptr;
+  const BlockSrc src{reinterpret_cast<const short4*>(proj->rect), block_vals, block_ranges,
+                     (TW + GS_TILE_BLOCK - 1) / GS_TILE_BLOCK, vals, ranges};
+#define GS_FWD(P, C) \
+  k_raster_fwd<P, C, true><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, TW, a, src, dev_status)
   switch (pick_ppt(flags, 2)) {
     case 1: if (cnt) GS_FWD(1, true); else GS_FWD(1, false); break;
     case 2: if (cnt) GS_FWD(2, true); else GS_FWD(2, false); break;

@@ -111,9 +111,9 @@ class Stepper:
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
-                 binning="expand", device="cuda"):
-        if binning not in ("expand", "sort"):
-            raise ValueError(f"binning must be 'expand' or 'sort', not {binning!r}")
+                 binning="fused", device="cuda"):
+        if binning not in ("fused", "expand", "sort"):
+            raise ValueError(f"binning must be 'fused', 'expand' or 'sort', not {binning!r}")
         self.model = model
         self.binning = binning
         self.budget = int(budget)
@@ -179,7 +179,11 @@ class Stepper:
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
         tk = clk.tic("project")
         B.gs_project(mod, camS, proj, sat, ws, st)
-        expand = self.binning == "expand"
+        # fused: per-block lists, each tile's list built inside the forward;
+        # expand: per-block lists expanded into full tile lists per Leaf;
+        # sort: per-Leaf (tile, candidate) entries sorted by tile
+        fused = self.binning == "fused"
+        expand = self.binning in ("expand", "fused")
         if expand:
             BW, BH = (TW + B.TILE_BLOCK - 1) // B.TILE_BLOCK, (TH + B.TILE_BLOCK - 1) // B.TILE_BLOCK
             bsat = torch.empty((BH + 1) * (BW + 1), dtype=torch.int64, device=dev)
@@ -248,7 +252,9 @@ class Stepper:
         # ---- per-Leaf raster: forward + L1 + backward into compact g2d ------
         g2d = torch.zeros(max(C, 1) * 12, dtype=torch.float32, device=dev)
         loss_tiles = torch.zeros(T, dtype=torch.float32, device=dev)
-        if expand:
+        if fused:
+            bin_ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        elif expand:
             bin_ws = torch.empty(max(max((B.gs_expand_workspace_size(L, B.block_entries(bsat_np, L))
                                           for L in lv), default=0), 256),
                                  dtype=torch.uint8, device=dev)
@@ -303,7 +309,9 @@ class Stepper:
                               counters=cnt_f)
             else:
                 px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
-            if expand:
+            if fused:
+                B.gs_tile_ranges(sat, TW, TH, L, ranges)
+            elif expand:
                 tk = clk.tic("expand")
                 B.gs_expand_tiles(proj, bvals, branges, B.block_entries(bsat_np, L), L, TW, TH,
                                   sat, I, vals, max(I, 1), ranges, bin_ws, st)
@@ -319,7 +327,11 @@ class Stepper:
                 B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
                 clk.toc(tk)
             tk = clk.tic("raster_fwd")
-            B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
+            if fused:
+                B.gs_raster_fwd_blocks(proj, bvals, branges, L, camS, px, vals, max(I, 1), I,
+                                       ranges, st, self.raster_flags)
+            else:
+                B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
             clk.toc(tk)
             if hooks is not None and hasattr(hooks, "on_leaf"):
                 hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,

@@ -395,6 +395,30 @@ gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals,
                         const gs_camera* cam, const gs_pixels* px,
                         uint32_t flags, int32_t* dev_status, gs_stream stream);
 
+/* gs_tile_ranges: the Leaf's per-tile list segments from the tile SAT
+ * (ranges[2 t] = begin, [2 t + 1] = end, t = local tile index), as
+ * gs_bin_tiles writes them.
+ *
+ * gs_raster_fwd_blocks: gs_raster_fwd with the tile lists built on the fly
+ * from the per-block lists of gs_bin_blocks (an implementation choice of
+ * this library, not on the pages): each tile filters its block's
+ * depth-ordered list by "tile inside the candidate's rect", which is the
+ * tile's list, and composites it; it stops reading once its pixels are
+ * done.  ranges: in, the segments of gs_tile_ranges; out, end = begin + the
+ * number of list entries consumed, and vals[begin .. end) = that prefix of
+ * the tile's list (everything gs_raster_bwd reads: positions < last).
+ * Image, T_final, last and loss are identical to gs_raster_fwd on the full
+ * lists.  n_isect: the Leaf's count (host SAT), must be <= capacity. */
+gs_status gs_tile_ranges(const int64_t* tile_sat, int32_t TW, int32_t TH,
+                         gs_rect leaf, int64_t* ranges, gs_stream stream);
+gs_status gs_raster_fwd_blocks(const gs_proj* proj, const int32_t* block_vals,
+                               const int64_t* block_ranges, gs_rect leaf,
+                               const gs_camera* cam, const gs_pixels* px,
+                               int32_t* vals, int64_t capacity,
+                               int64_t n_isect, int64_t* ranges,
+                               int64_t* needed, uint32_t flags,
+                               int32_t* dev_status, gs_stream stream);
+
 /* ---- 6. L1 loss ----------------------------------------------------------
  * For the Leaf's pixels: dL/dimg = sign(img - target) * norm (sign(0) = 0)
  * and, per global tile, loss_tiles[tile] = norm * sum |img - target| in a

@@ -186,6 +186,76 @@ def test_two_level_binning_leaf_without_entries(oracle_mod):
     case.check_leaf((0, 0, 20, 10))
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged", "hd"])
+def test_fused_forward_matches_oracle(oracle_mod, name):
+    """gs_raster_fwd_blocks: image, T, last and loss as the oracle's
+    compositing of the full lists; vals holds an exact prefix of each tile's
+    list that covers every position the backward reads (< last)."""
+    sc, cams = {"tiny": synth.tiny_oracle_scene, "hd": synth.hd_cluster_scene}.get(
+        name, lambda s: synth.tiny_scene(n=80, width=83, height=61, sh_degree=3, seed=4))(0)
+    cam = cams[0]
+    b = B()
+    pr = oracle_mod.project(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam)
+    TW, TH = oracle_mod.grid(cam)
+    W, H = cam.width, cam.height
+    case = Case(oracle_mod, pr["rect"], pr["key"], TW, TH)
+    case.pb = ProjBuffers.from_oracle(pr, sc.n)  # the real records
+    case.block_sat()
+    case.bin_blocks()
+    target = synth.random_image(W, H, 3) * 0.6
+    tgt = torch.as_tensor(target.astype(np.float32)).cuda()
+    leaves = [(0, 0, TW, TH), (1, 0, max(2, TW // 2 + 1), max(1, TH - 1))]
+    for L in leaves:
+        x0, y0, x1, y1 = L
+        tiles = _leaf_tiles(L, TW)
+        off, vals_o = oracle_mod.tile_lists(pr["rect"], pr["key"], TW, tiles)
+        I = int(off[-1])
+        px0, py0 = 16 * x0, 16 * y0
+        pw, ph = min(16 * x1, W) - px0, min(16 * y1, H) - py0
+        npx = pw * ph
+        img = torch.zeros(3 * npx, device="cuda")
+        Tf = torch.zeros(npx, device="cuda")
+        last = torch.zeros(npx, dtype=torch.int32, device="cuda")
+        dL = torch.zeros(3 * npx, device="cuda")
+        loss_tiles = torch.zeros(TW * TH, device="cuda")
+        px = b.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=tgt, target_origin=(0, 0),
+                      target_pitch=W, target_plane=W * H, loss_tiles=loss_tiles,
+                      norm=1.0 / (3.0 * W * H))
+        vals = torch.full((max(I, 1),), -1, dtype=torch.int32, device="cuda")
+        ranges = torch.zeros(2 * len(tiles), dtype=torch.int64, device="cuda")
+        b.gs_tile_ranges(case.sat_d, TW, TH, L, ranges)
+        b.gs_raster_fwd_blocks(case.pb.struct, case.bvals, case.branges, L, b.camera_struct(cam),
+                               px, vals, max(I, 1), I, ranges, case.st)
+        assert b.gs_check(case.st) == 0
+        # the same outputs as the full-list forward on the oracle's lists
+        ref_img = torch.zeros_like(img)
+        ref_T = torch.zeros_like(Tf)
+        ref_last = torch.zeros_like(last)
+        ref_dL = torch.zeros_like(dL)
+        ref_lt = torch.zeros_like(loss_tiles)
+        pxr = b.pixels(px0, py0, pw, ph, ref_img, ref_T, ref_last, ref_dL, target=tgt,
+                       target_origin=(0, 0), target_pitch=W, target_plane=W * H,
+                       loss_tiles=ref_lt, norm=1.0 / (3.0 * W * H))
+        vals_full = torch.as_tensor(vals_o if I else np.zeros(1, np.int32)).cuda()
+        rg_full = torch.as_tensor(np.stack([off[:-1], off[1:]], 1).astype(np.int64).reshape(-1)).cuda()
+        b.gs_raster_fwd(case.pb.struct, vals_full, rg_full, L, b.camera_struct(cam), pxr, case.st)
+        assert b.gs_check(case.st) == 0
+        assert torch.equal(img, ref_img) and torch.equal(Tf, ref_T) and torch.equal(last, ref_last)
+        assert torch.equal(dL, ref_dL) and torch.equal(loss_tiles, ref_lt)
+        # vals: the exact prefix of each oracle list that the backward reads
+        rg = ranges.cpu().numpy().reshape(-1, 2)
+        v = vals.cpu().numpy()
+        lst = last.cpu().numpy().reshape(ph, pw)
+        for k, tile in enumerate(tiles):
+            tx, ty = tile % TW, tile // TW
+            a, e = int(rg[k, 0]), int(rg[k, 1])
+            assert a == off[k] and off[k] <= e <= off[k + 1]
+            assert (v[a:e] == vals_o[off[k]:off[k] + (e - a)]).all()
+            ys, xs = 16 * ty - py0, 16 * tx - px0
+            need = lst[max(ys, 0):ys + 16, max(xs, 0):xs + 16]
+            assert need.size == 0 or need.max() <= e - a
+
+
 def test_step_paths_agree(oracle_mod):
     """The step with the two-level binning and with bin + tile sort: the same
     image, loss and Leaf plan inputs; gradients equal up to atomic order."""
@@ -194,7 +264,7 @@ def test_step_paths_agree(oracle_mod):
     cam = cams[0]
     target = torch.as_tensor(synth.random_image(cam.width, cam.height, 2) * 0.5).cuda()
     outs = []
-    for binning in ("expand", "sort"):
+    for binning in ("fused", "expand", "sort"):
         model = GaussianModel(sc.params, sc.n, sc.sh_degree)
         stp = Stepper(model, budget=6 << 20, binning=binning)
         seen = {}
@@ -206,11 +276,12 @@ def test_step_paths_agree(oracle_mod):
         stats = stp.run_view(cam, target, hooks=Hooks(), update=False)
         stp.check()
         outs.append((stats, seen, stp.last_loss()))
-    (s0, h0, l0), (s1, h1, l1) = outs
-    assert s0.n_isect == s1.n_isect and s0.n_leaves <= s1.n_leaves
-    assert l0 == l1
+    (s0, h0, l0) = outs[-1]
     g0 = h0["g2d"].cpu().numpy().reshape(-1, 12)
-    g1 = h1["g2d"].cpu().numpy().reshape(-1, 12)
-    for f in range(9):
-        d = np.linalg.norm(g0[:, f] - g1[:, f])
-        assert d <= 1e-5 * max(np.linalg.norm(g1[:, f]), 1e-30), f
+    for s1, h1, l1 in outs[:-1]:
+        assert s0.n_isect == s1.n_isect and s1.n_leaves <= s0.n_leaves
+        assert l0 == l1
+        g1 = h1["g2d"].cpu().numpy().reshape(-1, 12)
+        for f in range(9):
+            d = np.linalg.norm(g0[:, f] - g1[:, f])
+            assert d <= 1e-5 * max(np.linalg.norm(g0[:, f]), 1e-30), f

@@ -631,9 +631,10 @@ class Capture:
 
 
 @pytest.mark.parametrize("name,budget,binning", [
-    ("tiny", 384 << 20, "expand"), ("tiny", 120_000, "expand"), ("tiny", 120_000, "sort"),
-    ("ragged", 30_000, "expand"), ("small3", 200_000, "expand"), ("small3", 200_000, "sort"),
-    ("hd", 384 << 20, "expand"), ("hd", 20 << 20, "expand"), ("hd", 20 << 20, "sort")])
+    ("tiny", 384 << 20, "fused"), ("tiny", 120_000, "fused"), ("tiny", 120_000, "expand"),
+    ("tiny", 120_000, "sort"), ("ragged", 30_000, "fused"), ("small3", 200_000, "fused"),
+    ("small3", 200_000, "sort"), ("hd", 384 << 20, "fused"), ("hd", 20 << 20, "fused"),
+    ("hd", 20 << 20, "expand"), ("hd", 20 << 20, "sort")])
 def test_end_to_end_step(oracle_mod, name, budget, binning):
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, cam = scene(name)
