@@ -30,15 +30,22 @@ METRIC = ("fwd+bwd+Adam step ms & Gaussian-tile intersections/s per B200; "
           "peak working set GiB")
 UNIT = "intersections/s"
 SM_COUNT, LANES_PER_SM = 148, 128
-# algorithmic lane-ops per pixel-Gaussian pair (measurement)
+# Algorithmic lane-ops per pixel-Gaussian pair.  Every evaluation (forward
+# and backward): dx, dy, t1 = dx + beta dy, two products, q (mul + fma),
+# exp2, o * G, the 0.99 clamp and the 1/255 test = 11.  A composited pair
+# (forward): 1 - alpha, T (1 - alpha), the T test, alpha T, three colour
+# fmas, the T update = 8.  A differentiated pair (backward): 1 - alpha and
+# its reciprocal, T_i, alpha T_i, three colour gradients, g . rgb (3),
+# dL/dalpha (2), the running sum S, the clamp test, dL/dq, dL/do, and the
+# geometric terms du (2), dv (3), da, db, dc (2 each) with 0.5 dq = 28.
 OPS_FWD_VISIT, OPS_FWD_KEPT = 11, 8
-OPS_BWD_VISIT, OPS_BWD_KEPT = 11, 32
+OPS_BWD_VISIT, OPS_BWD_KEPT = 11, 28
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=48)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--gaussians", type=int, default=6_000_000)
@@ -76,7 +83,8 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
       raster_fwd   C*48 + pixels*(20 + 12 + 12) (records; colour, T, last;
                    target; dL/dcolour; the list entries a tile reads stop where
                    its pixels saturate, so none are counted)
-      raster_bwd   C*48 + pixels*(20 + 12) + C*48 (gradient atomics)
+      raster_bwd   C*48 + pixels*20 (T, last, dL/dcolour) + C*48 (gradient
+                   atomics)
       project_bwd  N*P*24 (p, m, v read and written) + C*(48 + 48 + 56*2)
                    (g2d, record, fp64 geometric scratch) + N*4 (slot map)
     (E_blk = block-list entries, R_blk = their reads over the Leaves, I =
@@ -98,7 +106,7 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
         "sort_tiles": 0.0 if expand else I * 40,
         "expand": (R * 24 + I * 4) if a.binning == "expand" else 0.0,
         "raster_fwd": C * 48 + px * 44,
-        "raster_bwd": C * 96 + px * 32,
+        "raster_bwd": C * 96 + px * 20,
         "project_bwd": n * P * 24 + C * 208 + n * 4,
     }
     scale = I / max(acc.n_isect, 1)
@@ -117,6 +125,26 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
             "frac": round(total / measured, 4) if measured > 0 else None, "stages": stages}
 
 
+def profile_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/<kernel>_*_dram.json), or None when there is none or the
+    kernel's source file has changed since it was taken."""
+    import glob
+    import hashlib
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*_dram.json"))):
+        try:
+            with open(path) as f:
+                rec = json.load(f)
+            src = os.path.join(ROOT, rec["source"])
+            with open(src, "rb") as f:
+                digest = hashlib.sha256(f.read()).hexdigest()
+        except (OSError, KeyError, ValueError):
+            continue
+        if digest == rec.get("source_sha256"):
+            return rec["dram_bytes_per_launch"], os.path.relpath(path, ROOT)
+    return None, None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -129,25 +157,30 @@ def load_peaks():
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling every 100 ms from before the warm-up to the end of
+    the timed region; stop(t0, t1) keeps the samples stamped inside [t0, t1]
+    (host wall clock), all samples if none is."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            import tempfile
+            self.f = tempfile.NamedTemporaryFile("w", suffix=f"_clocks_gpu{gpu_index}.csv",
+                                                 delete=False)
+            self.path = self.f.name
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "100", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
         if self.proc is None:
             return None
+        import datetime
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -157,15 +190,24 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+            if len(parts) >= 10:
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    ts = None
+                rows.append([ts] + parts[1:])
+        os.unlink(self.path)
+        if t0 is not None and t1 is not None:
+            inside = [r for r in rows if r[0] is not None and t0 <= r[0] <= t1]
+            rows = inside or rows
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        num = lambda x: x.replace(".", "", 1).isdigit()
+        sm = [float(r[2]) for r in rows if num(r[2])]
+        mx = [float(r[3]) for r in rows if num(r[3])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
-        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[6 + k].lower() == "active"})
+        loaded = [x for x in sm if x > 0.5 * max(sm)] if sm else []
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
@@ -262,6 +304,27 @@ class OracleSample:
 
 
 # ---------------------------------------------------------------------------
+# replicas: rank r takes views r, r + 1, ... (mod the view count); the job's
+# time is the slowest rank's, its work the sum over ranks
+# ---------------------------------------------------------------------------
+def rank_view(k, rank, n_views):
+    return (k + rank) % n_views
+
+
+def combine_ranks(ms, units, dist, device):
+    """(max over ranks of ms, sum over ranks of units); dist = None for one
+    process.  Every rank must call it, in the same order."""
+    if dist is None:
+        return float(ms), float(units)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([float(units)], dtype=torch.float64, device=device)
+    dist.all_reduce(u)
+    return float(t.item()), float(u.item())
+
+
+# ---------------------------------------------------------------------------
 def main():
     a = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -296,18 +359,19 @@ def main():
     model = GaussianModel(scene.params, scene.n, scene.sh_degree)
     stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt, binning=a.binning)
     nv = len(cams)
-    view_of = lambda k: (k + rank) % nv
+    view_of = lambda k: rank_view(k, rank, nv)
 
+    clocks = ClockSampler(local)
     for k in range(a.warmup):
         stp.run_view(cams[view_of(k)], targets[view_of(k)])
     stp.check()
 
     # ---- timed region (device time, CUDA events on the launching stream) -----
     timing = {}
-    clocks = ClockSampler(local)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    wall0 = time.time()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -319,7 +383,7 @@ def main():
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(wall0, time.time())
     stp.check()
     ms = e0.elapsed_time(e1)
     isect = sum(s.n_isect_square for s in stats)   # conventional 3-sigma-square count
@@ -328,15 +392,7 @@ def main():
     peak_ws = max(s.peak_ws_bytes for s in stats)
     stage_ms = {name: sum(x.elapsed_time(y) for x, y in timing.get(name, [])) for name in STAGES}
     stage_n = {name: len(timing.get(name, [])) for name in STAGES}
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-        t = torch.tensor([isect], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t)
-        isect_all = float(t.item())
-    else:
-        ms_max, isect_all = ms, float(isect)
+    ms_max, isect_all = combine_ranks(ms, isect, dist, "cuda")
     value = isect_all / (ms_max / 1e3)
 
     # ---- accounting step (untimed): work counters per launch -----------------
@@ -359,9 +415,11 @@ def main():
     if dom in ("raster_bwd", "raster_fwd"):
         ops = ops_bwd if dom == "raster_bwd" else ops_fwd
         ach = ops / (per_step[dom] / 1e3) / 1e12
+        traffic, traffic_src = profile_traffic(f"k_{dom}")
         roof = {"bound": "alu", "kernel": f"k_{dom}", "achieved": round(ach, 3),
                 "peak": round(alu_peak / 1e12, 3), "unit": "Tlane-op/s",
-                "frac": round(ach / (alu_peak / 1e12), 4), "traffic": None,
+                "frac": round(ach / (alu_peak / 1e12), 4), "traffic": traffic,
+                "traffic_source": traffic_src,
                 "peak_source": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {sm_mhz:g} MHz "
                                f"(sm_max_mhz of {peak_src})"}
     else:
@@ -398,14 +456,7 @@ def main():
             e2e_isect += s.n_isect_square
         f1.record()
         torch.cuda.synchronize()
-        ems = f0.elapsed_time(f1)
-        if dist:
-            t = torch.tensor([ems], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-            t = torch.tensor([e2e_isect], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t)
-            e2e_isect = float(t.item())
+        ems, e2e_isect = combine_ranks(f0.elapsed_time(f1), e2e_isect, dist, "cuda")
         TW, TH = (W + 15) // 16, (H + 15) // 16
         BW, BH = (TW + 7) // 8, (TH + 7) // 8
         # per step: the tile SAT, candidate count, 3-sigma count, block SAT

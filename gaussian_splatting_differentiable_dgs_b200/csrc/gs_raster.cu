@@ -201,8 +201,12 @@ struct BlockSrc {
 // forward
 // ---------------------------------------------------------------------------
 // BLK = false: the tile's list is vals[ranges]; BLK = true: it is built
-// from the block list (BlockSrc), in fills of at least NT entries (so a fill
-// holds fewer than 2 NT), and only as far as the tile's pixels need it.
+// from the block list (BlockSrc) and only as far as the tile's pixels need
+// it.  A fill reads kFillU x NT block-list entries at once (kFillU loads in
+// flight per thread), keeps the hits in list order in s_hits and in the
+// Leaf's vals; the hits are then staged and composited NT at a time.
+constexpr int kFillU = 2;
+
 template <int PPT, bool COUNT, bool BLK>
 __global__ void __launch_bounds__(256 / PPT)
 k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
@@ -210,19 +214,23 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              BlockSrc bsrc, int32_t* dev_status) {
   using G = TileGeom<PPT>;
   constexpr int NT = G::NT;
-  constexpr int CAP = BLK ? 2 * NT : NT;
+  constexpr int CAP = NT;
   using LT = std::conditional_t<(CAP <= 256), uint8_t, uint16_t>;
+  constexpr int HCAP = BLK ? kFillU * NT : 1;
   __shared__ float4 sA[CAP], sB[CAP];
   __shared__ float sC[CAP];
   __shared__ uint8_t s_mask[CAP];
   __shared__ LT s_list[G::NW][CAP];
   __shared__ float s_red[G::NW];
-  __shared__ int s_wcnt[G::NW];
+  __shared__ int s_wcnt[kFillU][G::NW];
+  __shared__ int32_t s_hits[HCAP];
   const int lw = leaf.x1 - leaf.x0;
   const int ltile = blockIdx.x;
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile], end = ranges[2 * ltile + 1];
-  int64_t bp = 0, be = 0, n_done = 0;  // block-list cursor / end, entries consumed
+  // block-list cursor / end, list entries written, staged; hit-list cursor / length
+  int64_t bp = 0, be = 0, n_filled = 0, n_staged = 0;
+  int hp = 0, nh = 0;
   if (BLK) {
     const int64_t b = (int64_t)(ty / GS_TILE_BLOCK) * bsrc.BW + tx / GS_TILE_BLOCK;
     bp = bsrc.block_ranges[2 * b];
@@ -254,46 +262,65 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     if (__syncthreads_count(mine_done) == NT) break;
     int cnt, pos1;
     if (BLK) {
-      if (bp >= be) break;
-      // fill: filter block-list batches of NT until at least NT entries
-      const unsigned ltm = (1u << lane) - 1u;
-      cnt = 0;
-      while (cnt < NT && bp < be) {
-        const int64_t q = bp + t;
-        bool hit = false;
-        int32_t slot = 0;
-        if (q < be) {
-          slot = bsrc.block_vals[q];
-          const short4 r = bsrc.rect[slot];
-          hit = (r.x <= tx) & (tx < r.z) & (r.y <= ty) & (ty < r.w);
-        }
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        if (lane == 0) s_wcnt[w] = __popc(bal);
-        __syncthreads();
-        int wb = 0, tot = 0;
+      if (hp >= nh) {
+        // fill: kFillU x NT block-list entries, hits kept in list order
+        if (bp >= be) break;
+        int32_t sl[kFillU];
+        short4 rc[kFillU];
 #pragma unroll
-        for (int ww = 0; ww < G::NW; ++ww) {
-          const int c = s_wcnt[ww];
-          wb += ww < w ? c : 0;
-          tot += c;
+        for (int u = 0; u < kFillU; ++u) {
+          const int64_t q = bp + (int64_t)u * NT + t;
+          sl[u] = q < be ? bsrc.block_vals[q] : -1;
         }
-        if (hit) {
-          const int k = cnt + wb + __popc(bal & ltm);
-          const Staged st = stage_record(rec, slot, tx, ty);
-          s_mask[k] = (uint8_t)warp_mask<PPT>(alpha_box(st));
-          sA[k] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-          sB[k] = make_float4(st.ns2, st.opac, st.r, st.g);
-          sC[k] = st.b;
-          const int64_t o = begin + n_done + k;
-          if (o < end) bsrc.vals_out[o] = slot;
-          else bad = true;
+#pragma unroll
+        for (int u = 0; u < kFillU; ++u)
+          if (sl[u] >= 0) rc[u] = bsrc.rect[sl[u]];
+        const unsigned ltm = (1u << lane) - 1u;
+        unsigned bal[kFillU];
+#pragma unroll
+        for (int u = 0; u < kFillU; ++u) {
+          const bool hit = sl[u] >= 0 && (rc[u].x <= tx) & (tx < rc[u].z) & (rc[u].y <= ty) &
+                                             (ty < rc[u].w);
+          bal[u] = __ballot_sync(0xffffffffu, hit);
+          if (lane == 0) s_wcnt[u][w] = __popc(bal[u]);
         }
-        cnt += tot;
-        bp += NT;
-        __syncthreads();  // s_wcnt is rewritten by the next batch
+        __syncthreads();
+        int run = 0, off[kFillU];
+#pragma unroll
+        for (int u = 0; u < kFillU; ++u)
+#pragma unroll
+          for (int ww = 0; ww < G::NW; ++ww) {
+            if (ww == w) off[u] = run;
+            run += s_wcnt[u][ww];
+          }
+#pragma unroll
+        for (int u = 0; u < kFillU; ++u)
+          if ((bal[u] >> lane) & 1u) {
+            const int k = off[u] + __popc(bal[u] & ltm);
+            s_hits[k] = sl[u];
+            const int64_t o = begin + n_filled + k;
+            if (o < end) bsrc.vals_out[o] = sl[u];
+            else bad = true;
+          }
+        nh = run;
+        hp = 0;
+        n_filled += run;
+        bp += (int64_t)kFillU * NT;
+        __syncthreads();  // s_hits visible; s_wcnt free again
+        if (nh == 0) continue;
       }
-      pos1 = (int)n_done + 1;
-      n_done += cnt;
+      cnt = min(NT, nh - hp);
+      if (t < cnt) {
+        const Staged st = stage_record(rec, s_hits[hp + t], tx, ty);
+        s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
+        sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
+        sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+        sC[t] = st.b;
+      }
+      __syncthreads();
+      pos1 = (int)n_staged + 1;
+      n_staged += cnt;
+      hp += cnt;
     } else {
       const int64_t e = base + t;
       if (e < end) {
@@ -351,7 +378,8 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   }
   if (BLK) {
     if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
-    if (t == 0) bsrc.ranges_io[2 * ltile + 1] = begin + (n_done < end - begin ? n_done : end - begin);
+    if (t == 0)
+      bsrc.ranges_io[2 * ltile + 1] = begin + (n_filled < end - begin ? n_filled : end - begin);
   }
   // epilogue: outputs and the fused L1 terms
   float lsum = 0.0f;

@@ -336,8 +336,9 @@ gs_status gs_bin_tiles(const gs_proj* proj, int64_t n_cand,
 /* Two-level binning: the same per-Leaf lists as gs_bin_tiles followed by the
  * tile sort (bit-identical vals and ranges), without per-entry keys or a
  * sort of the Leaf's entries.  An implementation choice of this library for
- * the binning step of the 3D Gaussian Splatting paper (section 6: per-tile
- * lists ordered by depth); the pages do not describe it.
+ * the binning step (per-tile lists in depth order) of the tile rasteriser
+ * that the SkipGS paper notes ("loss function / training strategy") leave
+ * unchanged; the pages do not describe it.
  *
  * gs_block_sat (once per view, may run before the host learns n_cand):
  * block_sat = (BH + 1) x (BW + 1) summed-area table (zero first row and

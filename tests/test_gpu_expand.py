@@ -1,8 +1,10 @@
 """Two-level binning (per-block candidate lists, then per-Leaf expansion into
 per-tile segments) against the oracle's per-tile lists: vals and ranges must
 be bit-identical to the lists sorted by (depth bits, candidate position),
-the order of the 3D Gaussian Splatting paper, section 6.  The block-level
-intermediates are checked against their plain definitions."""
+the front-to-back order the tile rasteriser composites in (SkipGS paper
+notes, "loss function / training strategy": the rasterisation pipeline is
+the standard one).  The block-level intermediates are checked against their
+plain definitions."""
 import numpy as np
 import pytest
 import torch
