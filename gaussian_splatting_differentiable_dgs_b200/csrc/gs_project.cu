@@ -62,17 +62,20 @@ __device__ __forceinline__ void sh_basis(double x, double y, double z, int D, do
   Y[15] = -k3a * x * (xx - 3.0 * yy);
 }
 
-struct ProjOut {
-  float4 r0, r1, r2;
+// The geometric part of a candidate's projection (everything but colour).
+struct ProjGeo {
+  double x, y, z;        // mean
+  double u, v, hx, hy;   // pixel position, alpha-box half extents
+  double c00, c01, c11, det, opac, tz;
   short4 rect;
-  uint32_t key;
   int64_t square_tiles;
 };
 
-// Returns true if Gaussian i is a candidate and fills `o`.
-__device__ __forceinline__ bool project_gaussian(const float* __restrict__ P, int64_t n_pad,
-                                                 int64_t i, int D, const ProjCam& c,
-                                                 ProjOut& o, bool& nonfinite) {
+// Cull + geometry of Gaussian i from its 11 geometric planes; true if it is
+// a candidate.  The SH planes are read only for candidates (sh_colour).
+__device__ __forceinline__ bool project_geometry(const float* __restrict__ P, int64_t n_pad,
+                                                 int64_t i, const ProjCam& c, ProjGeo& o,
+                                                 bool& nonfinite) {
   const double x = P[i], y = P[n_pad + i], z = P[2 * n_pad + i];
   double tc[3];
 #pragma unroll
@@ -169,6 +172,10 @@ __device__ __forceinline__ bool project_gaussian(const float* __restrict__ P, in
   const int64_t y0 = cy0 < 0 ? 0 : (cy0 > c.TH ? c.TH : cy0);
   const int64_t y1 = cy1 < 0 ? 0 : (cy1 > c.TH ? c.TH : cy1);
   if (x0 >= x1 || y0 >= y1) return false;
+  o.x = x; o.y = y; o.z = z;
+  o.u = u; o.v = v; o.hx = hx; o.hy = hy;
+  o.c00 = c00; o.c01 = c01; o.c11 = c11; o.det = det; o.opac = opac; o.tz = tz;
+  o.rect = make_short4((short)x0, (short)y0, (short)x1, (short)y1);
   {
     // tiles of the plain 3-sigma square (clamped), counted for the metric
     const int64_t sx0 = rx0 < 0 ? 0 : (rx0 > c.TW ? c.TW : rx0);
@@ -178,39 +185,49 @@ __device__ __forceinline__ bool project_gaussian(const float* __restrict__ P, in
     o.square_tiles = (sx1 > sx0 && sy1 > sy0) ? (sx1 - sx0) * (sy1 - sy0) : 0;
   }
 
-  // colour from SH at the direction camera centre -> mean
-  double dx = x - c.campos[0], dy = y - c.campos[1], dz = z - c.campos[2];
-  const double dn = sqrt(dx * dx + dy * dy + dz * dz);
-  dx /= dn; dy /= dn; dz /= dn;
-  double Y[16];
-  sh_basis(dx, dy, dz, D, Y);
-  const int ksh = (D + 1) * (D + 1);
-  double rgb[3] = {0.5, 0.5, 0.5};
-  for (int k = 0; k < ksh; ++k) {
-#pragma unroll
-    for (int ch = 0; ch < 3; ++ch) {
-      float s = P[(11 + 3 * k + ch) * n_pad + i];
-      rgb[ch] += (double)s * Y[k];
-    }
-  }
-  const float uh = (float)u, vh = (float)v;
-  // u, v as fp32 + fp16 corrections (|lo| <= ulp(u)/2, so the pair is exact
-  // to ~2e-7 px); the alpha box half extents as fp16 rounded up
-  const __half2 lo = __floats2half2_rn((float)(u - (double)uh), (float)(v - (double)vh));
-  const __half2 box = __halves2half2(__float2half_ru((float)hx), __float2half_ru((float)hy));
-  o.r0 = make_float4(uh, vh, __uint_as_float(*reinterpret_cast<const unsigned*>(&lo)),
-                     __uint_as_float(*reinterpret_cast<const unsigned*>(&box)));
-  const double a = c11 / det, b = -c01 / det;
-  o.r1 = make_float4((float)(0.5 * a), (float)(b / a), (float)(0.5 / c11), (float)opac);
-  const float depth = (float)tz;
-  o.r2 = make_float4((float)fmax(rgb[0], 0.0), (float)fmax(rgb[1], 0.0), (float)fmax(rgb[2], 0.0), depth);
-  o.rect = make_short4((short)x0, (short)y0, (short)x1, (short)y1);
-  o.key = __float_as_uint(depth);
   return true;
 }
 
-__global__ void __launch_bounds__(kProjThreads)
-k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, int D, ProjCam cam,
+// Colour from SH at the direction camera centre -> mean, then the record.
+template <int D>
+__device__ __forceinline__ void sh_record(const float* __restrict__ P, int64_t n_pad, int64_t i,
+                                          const ProjCam& c, const ProjGeo& g, float4& r0,
+                                          float4& r1, float4& r2) {
+  double dx = g.x - c.campos[0], dy = g.y - c.campos[1], dz = g.z - c.campos[2];
+  const double dn = sqrt(dx * dx + dy * dy + dz * dz);
+  dx /= dn; dy /= dn; dz /= dn;
+  constexpr int ksh = (D + 1) * (D + 1);
+  float sh[ksh][3];
+#pragma unroll
+  for (int k = 0; k < ksh; ++k)
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) sh[k][ch] = P[(11 + 3 * k + ch) * n_pad + i];
+  double Y[16];
+  sh_basis(dx, dy, dz, D, Y);
+  double rgb[3] = {0.5, 0.5, 0.5};
+#pragma unroll
+  for (int k = 0; k < ksh; ++k)
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) rgb[ch] += (double)sh[k][ch] * Y[k];
+  const float uh = (float)g.u, vh = (float)g.v;
+  // u, v as fp32 + fp16 corrections (|lo| <= ulp(u)/2, so the pair is exact
+  // to ~2e-7 px); the alpha box half extents as fp16 rounded up
+  const __half2 lo = __floats2half2_rn((float)(g.u - (double)uh), (float)(g.v - (double)vh));
+  const __half2 box = __halves2half2(__float2half_ru((float)g.hx), __float2half_ru((float)g.hy));
+  r0 = make_float4(uh, vh, __uint_as_float(*reinterpret_cast<const unsigned*>(&lo)),
+                   __uint_as_float(*reinterpret_cast<const unsigned*>(&box)));
+  const double a = g.c11 / g.det, b = -g.c01 / g.det;
+  r1 = make_float4((float)(0.5 * a), (float)(b / a), (float)(0.5 / g.c11), (float)g.opac);
+  const float depth = (float)g.tz;
+  r2 = make_float4((float)fmax(rgb[0], 0.0), (float)fmax(rgb[1], 0.0), (float)fmax(rgb[2], 0.0),
+                   depth);
+}
+
+// 3 CTAs per SM: the degree-3 instance fits in 85 registers with a few bytes
+// of spill, faster than 2 CTAs at 92
+template <int D>
+__global__ void __launch_bounds__(kProjThreads, 3)
+k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam cam,
           int32_t* __restrict__ cand_idx, int32_t* __restrict__ slot_map, float4* __restrict__ rec,
           short4* __restrict__ rect, uint32_t* __restrict__ depth_key, int32_t* __restrict__ diff,
           unsigned long long* __restrict__ lb, unsigned int* __restrict__ ticket,
@@ -223,9 +240,11 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, int D, Pro
   __syncthreads();
   const int64_t b = s_b;
   const int64_t i = b * kProjThreads + threadIdx.x;
-  ProjOut o;
+  ProjGeo o;
   bool nonfinite = false;
-  const bool cand = i < n && project_gaussian(params, n_pad, i, D, cam, o, nonfinite);
+  // cull and geometry first, so the CTA's scan below waits only on the 11
+  // geometric planes; the 48 SH planes are read after it, by candidates
+  const bool cand = i < n && project_geometry(params, n_pad, i, cam, o, nonfinite);
   if (nonfinite) dev_flag(dev_status, GS_DEV_NONFINITE);
   int total;
   const int rank = block_exclusive_scan<int, kProjThreads / 32>(cand ? 1 : 0, s_scan, &total);
@@ -239,12 +258,14 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, int D, Pro
   if (cand && !fits) dev_flag(dev_status, GS_DEV_BOUNDS);
   if (i < n) slot_map[i] = (cand && fits) ? (int32_t)slot : -1;
   if (cand && fits) {
+    float4 r0, r1, r2;
+    sh_record<D>(params, n_pad, i, cam, o, r0, r1, r2);
     cand_idx[slot] = (int32_t)i;
-    rec[3 * slot] = o.r0;
-    rec[3 * slot + 1] = o.r1;
-    rec[3 * slot + 2] = o.r2;
+    rec[3 * slot] = r0;
+    rec[3 * slot + 1] = r1;
+    rec[3 * slot + 2] = r2;
     rect[slot] = o.rect;
-    depth_key[slot] = o.key;
+    depth_key[slot] = __float_as_uint(r2.w);
     const int64_t s = cam.TW + 1;
     atomicAdd(&diff[o.rect.y * s + o.rect.x], 1);
     atomicAdd(&diff[o.rect.y * s + o.rect.z], -1);
@@ -414,10 +435,18 @@ extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uin
   GS_TRY(cudaMemsetAsync(ws, 0, zero_bytes, s));
   if (out->square_isect) GS_TRY(cudaMemsetAsync(out->square_isect, 0, sizeof(unsigned long long), s));
   if (nb > 0) {
-    k_project<<<(unsigned)nb, kProjThreads, 0, s>>>(
-        model->params, model->n, model->n_pad, model->sh_degree, pc, out->cand_idx, out->slot,
-        reinterpret_cast<float4*>(out->rec), reinterpret_cast<short4*>(out->rect), out->depth_key,
-        w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, out->square_isect, dev_status);
+#define GS_PROJ(DD)                                                                          \
+  k_project<DD><<<(unsigned)nb, kProjThreads, 0, s>>>(                                       \
+      model->params, model->n, model->n_pad, pc, out->cand_idx, out->slot,                   \
+      reinterpret_cast<float4*>(out->rec), reinterpret_cast<short4*>(out->rect), out->depth_key, \
+      w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, out->square_isect, dev_status)
+    switch (model->sh_degree) {
+      case 0: GS_PROJ(0); break;
+      case 1: GS_PROJ(1); break;
+      case 2: GS_PROJ(2); break;
+      default: GS_PROJ(3); break;
+    }
+#undef GS_PROJ
     GS_LAUNCH_CHECK();
   } else {
     GS_TRY(cudaMemsetAsync(out->n_cand, 0, sizeof(int32_t), s));
