@@ -438,8 +438,9 @@ def main():
     # ---- end to end through host buffers --------------------------------------
     e2e = None
     if not a.no_e2e:
+        # the step's public call with the view's target in pinned host memory:
+        # each Leaf's crop is uploaded on a copy stream, overlapped with compute
         host_t = [t.cpu().pin_memory() for t in targets]
-        dev_t = torch.empty_like(targets[0])
         loss_h = torch.empty(1, dtype=torch.float64, pin_memory=True)
         if dist:
             dist.barrier()
@@ -450,8 +451,7 @@ def main():
         e2e_isect = 0
         for k in range(a.steps):
             v = view_of(k)
-            dev_t.copy_(host_t[v], non_blocking=True)
-            s = stp.run_view(cams[v], dev_t)
+            s = stp.run_view(cams[v], host_t[v])
             loss_h.copy_(stp._last_loss, non_blocking=True)
             e2e_isect += s.n_isect_square
         f1.record()

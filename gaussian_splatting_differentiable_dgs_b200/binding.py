@@ -104,7 +104,7 @@ SYMBOLS = [
     "gs_bin_workspace_size", "gs_bin_tiles",
     "gs_block_sat_workspace_size", "gs_block_sat", "gs_bin_blocks_workspace_size",
     "gs_bin_blocks", "gs_expand_workspace_size", "gs_expand_tiles",
-    "gs_tile_ranges", "gs_raster_fwd_blocks",
+    "gs_tile_ranges", "gs_raster_fwd_blocks", "gs_upload_crop",
     "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
     "gs_project_bwd", "gs_adam",
 ]
@@ -146,6 +146,7 @@ def _load():
                                   P(i64), p, sz, p, p]),
         "gs_raster_fwd": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), u32, p, p]),
         "gs_tile_ranges": (i32, [p, i32, i32, gs_rect, p, p]),
+        "gs_upload_crop": (i32, [p, i64, i64, i32, i32, i32, i32, i32, p, i64, i64, p]),
         "gs_raster_fwd_blocks": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), p,
                                        i64, i64, p, P(i64), u32, p, p]),
         "gs_loss_l1": (i32, [P(gs_pixels), gs_rect, P(gs_camera), p]),
@@ -409,6 +410,14 @@ def gs_raster_fwd_blocks(proj: gs_proj, block_vals, block_ranges, leaf, cam: gs_
                                  ptr(vals), capacity, n_isect, ptr(ranges), C.byref(needed), flags,
                                  ptr(dev_status), _stream(stream))
     return _ok("gs_raster_fwd_blocks", st, needed.value if st == GS_ERR_CAPACITY else None)
+
+
+def gs_upload_crop(host, x0, y0, w, h, dev, stream=None):
+    """Crop of a planar host image [C][H][W] (pinned for an async copy) into a
+    contiguous device buffer [C][h][w]."""
+    C_, H_, W_ = host.shape
+    return _ok("gs_upload_crop", _L.gs_upload_crop(host.data_ptr(), W_, H_ * W_, x0, y0, w, h, C_,
+                                                   ptr(dev), w, w * h, _stream(stream)))
 
 
 def gs_loss_l1(px: gs_pixels, leaf, cam: gs_camera, stream=None):

@@ -165,3 +165,27 @@ extern "C" gs_status gs_leaf_partition(const int64_t* sat_host, int32_t TW, int3
   if (p.count > max_leaves) return GS_ERR_CAPACITY;
   return p.any_over ? GS_WARN_BUDGET : GS_OK;
 }
+
+// Leaf crop of a planar host image ([channels][height][host_pitch] floats,
+// plane stride host_plane) into a device buffer, one 2D copy per channel.
+// Asynchronous when the host memory is pinned.
+extern "C" gs_status gs_upload_crop(const float* host, int64_t host_pitch, int64_t host_plane,
+                                    int32_t x0, int32_t y0, int32_t w, int32_t h,
+                                    int32_t channels, float* dev, int64_t dev_pitch,
+                                    int64_t dev_plane, gs_stream stream) {
+  if (!host || !dev || x0 < 0 || y0 < 0 || w < 0 || h < 0 || channels < 1) return GS_ERR_ARG;
+  if (w == 0 || h == 0) return GS_OK;
+  if (host_pitch < (int64_t)x0 + w || host_plane < host_pitch * ((int64_t)y0 + h) ||
+      dev_pitch < w || dev_plane < dev_pitch * (int64_t)h)
+    return GS_ERR_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int32_t c = 0; c < channels; ++c) {
+    const float* src = host + c * host_plane + (int64_t)y0 * host_pitch + x0;
+    float* dst = dev + c * dev_plane;
+    if (cudaMemcpy2DAsync(dst, (size_t)dev_pitch * sizeof(float), src,
+                          (size_t)host_pitch * sizeof(float), (size_t)w * sizeof(float),
+                          (size_t)h, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return GS_ERR_CUDA;
+  }
+  return GS_OK;
+}

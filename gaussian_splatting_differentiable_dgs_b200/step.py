@@ -123,6 +123,7 @@ class Stepper:
         self.device = torch.device(device)
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
         self._last_loss = None
+        self._copy_stream = None
 
     def check(self):
         st = B.gs_check(self.dev_status)
@@ -275,15 +276,39 @@ class Stepper:
                 lb_bits = B.local_tile_bits(L)
                 sizes = [4 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 4, 0, lb_bits),
                          12 * npx, 4 * npx, 4 * npx, 12 * npx]
-            if target is not None and not resident_target:
-                sizes.append(12 * npx)
             return sizes, (16 * x0, 16 * y0, pw, ph)
 
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
         arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
         norm = 1.0 / (3.0 * W * H)
-        for L, I in zip(lv, li):
+        # bounded supply of a host target: each Leaf's crop is uploaded on a
+        # copy stream into one of two buffers, Leaf k + 2's upload waiting
+        # until Leaf k's forward (the only reader) is done
+        host_target = target is not None and not resident_target
+        if host_target:
+            rects = [leaf_sizes(L, 0)[1] for L in lv]
+            crop_n = max((3 * w * h for _, _, w, h in rects), default=1)
+            crops = [torch.empty(max(crop_n, 1), dtype=torch.float32, device=dev) for _ in range(2)]
+            if self._copy_stream is None:
+                self._copy_stream = torch.cuda.Stream(device=dev)
+            cs = self._copy_stream
+            up = [torch.cuda.Event() for _ in lv]
+            freed = [None, None]
+            main = torch.cuda.current_stream(dev)
+
+            def upload(k):
+                x_, y_, w_, h_ = rects[k]
+                if freed[k % 2] is not None:
+                    cs.wait_event(freed[k % 2])
+                else:
+                    cs.wait_stream(main)  # the buffers were allocated on the main stream
+                B.gs_upload_crop(target, x_, y_, w_, h_, crops[k % 2], stream=cs)
+                up[k].record(cs)
+
+            for k in range(min(2, len(lv))):
+                upload(k)
+        for li_k, (L, I) in enumerate(zip(lv, li)):
             I = int(I)
             sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
             bufs, _ = _carve(arena, sizes)
@@ -300,10 +325,9 @@ class Stepper:
                 px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
                               target_origin=(0, 0), target_pitch=W, target_plane=W * H,
                               loss_tiles=loss_tiles, norm=norm, counters=cnt_f)
-            elif target is not None:
-                # bounded supply: the Leaf's crop of a host target is uploaded
-                crop = bufs[8].view(torch.float32).view(3, ph, pw)
-                crop.copy_(target[:, py0:py0 + ph, px0:px0 + pw], non_blocking=True)
+            elif host_target:
+                crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
+                main.wait_event(up[li_k])
                 px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
                               target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm,
                               counters=cnt_f)
@@ -333,6 +357,12 @@ class Stepper:
             else:
                 B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
             clk.toc(tk)
+            if host_target:
+                ev = torch.cuda.Event()
+                ev.record(main)
+                freed[li_k % 2] = ev
+                if li_k + 2 < len(lv):
+                    upload(li_k + 2)
             if hooks is not None and hasattr(hooks, "on_leaf"):
                 hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
                                         ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
@@ -344,6 +374,8 @@ class Stepper:
                 B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
                 clk.toc(tk)
         del arena, bin_ws  # raster buffers released before projection backward
+        if host_target:
+            del crops
 
         loss_d = torch.zeros(1, dtype=torch.float64, device=dev)
         if target is not None:

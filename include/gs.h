@@ -420,6 +420,18 @@ gs_status gs_raster_fwd_blocks(const gs_proj* proj, const int32_t* block_vals,
                                int64_t* needed, uint32_t flags,
                                int32_t* dev_status, gs_stream stream);
 
+/* gs_upload_crop: the Leaf's crop [x0, x0 + w) x [y0, y0 + h) of a planar
+ * host image (channels planes of host_plane floats, rows of host_pitch) into
+ * a device buffer (rows of dev_pitch, planes of dev_plane), one 2D copy per
+ * channel on `stream` (asynchronous when the host memory is pinned).  The
+ * bounded supply of the supervision image, one Leaf at a time (BoundedGS
+ * page, section 02 B -> C: the Leaf's forward, loss and backward). */
+gs_status gs_upload_crop(const float* host, int64_t host_pitch,
+                         int64_t host_plane, int32_t x0, int32_t y0, int32_t w,
+                         int32_t h, int32_t channels, float* dev,
+                         int64_t dev_pitch, int64_t dev_plane,
+                         gs_stream stream);
+
 /* ---- 6. L1 loss ----------------------------------------------------------
  * For the Leaf's pixels: dL/dimg = sign(img - target) * norm (sign(0) = 0)
  * and, per global tile, loss_tiles[tile] = norm * sum |img - target| in a

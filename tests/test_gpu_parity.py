@@ -671,6 +671,32 @@ def test_end_to_end_step(oracle_mod, name, budget, binning):
         assert d.max() <= 2.1e-3, gname  # at most one sign flip of a ~zero gradient
 
 
+def test_host_target_matches_resident_target():
+    """The bounded supply of a pinned host target (per-Leaf crops uploaded on a
+    copy stream, double-buffered) gives the same loss and last as the
+    resident target, and the same gradients up to atomic order."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    tgt = synth.random_image(cam.width, cam.height, 8) * 0.5
+    outs = []
+    for host in (False, True):
+        model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+        stp = Stepper(model, budget=6 << 20)
+        t = torch.as_tensor(tgt).pin_memory() if host else torch.as_tensor(tgt).cuda()
+        cap = Capture(cam.width, cam.height)
+        stats = stp.run_view(cam, t, hooks=cap)
+        stp.check()
+        assert stats.n_leaves >= 3
+        outs.append((stp.last_loss(), cap.last.copy(), cap.g2d.copy(), model.params.cpu().numpy()))
+    (l0, last0, g0, p0), (l1, last1, g1, p1) = outs
+    assert l0 == l1 and (last0 == last1).all()
+    for f in range(9):
+        assert rel_l2(g1[:, f], g0[:, f]) <= 1e-5
+    # Adam moves a parameter by about lr whatever the gradient's size, so an
+    # atomic-order sign flip of a ~zero gradient moves it by up to 2 lr
+    assert np.abs(p1 - p0).max() <= 2.1e-3
+
+
 def test_leaf_invariance_gpu(oracle_mod):
     """Any Leaf partition: bit-identical image and loss, the same summed
     gradients (atomics reorder only)."""
