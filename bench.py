@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--budget-mib", type=float, default=384)
     ap.add_argument("--raster-ppt", type=int, default=0)
     ap.add_argument("--binning", default="fused", choices=["fused", "expand", "sort"])
+    ap.add_argument("--sweep", default=None,
+                    help="comma-separated widths: resolution sweep, whole image vs bounded")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
@@ -334,6 +336,8 @@ def main():
 
     if a.impl == "reference":
         return run_reference(a, rank, world)
+    if a.sweep:
+        return run_sweep(a)
 
     import torch
     torch.cuda.set_device(local)
@@ -514,6 +518,75 @@ def main():
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_sweep(a):
+    """Resolution sweep on the outdoor scene at a fixed camera pose and field
+    of view (3:2 images): per width, (a) the whole-image configuration with
+    a single-stage backward ("original") and (b) the bounded one (two-stage
+    backward, Leaves under the budget, candidate-index projection, compact
+    gradients).  Both start from the same parameters; the first step's L1
+    loss is compared, then `steps` steps are timed.  One JSON line per run
+    and a summary line."""
+    import torch
+    from gaussian_splatting_differentiable_dgs_b200 import synth
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    torch.cuda.set_device(0)
+    scene, _ = synth.outdoor_scene(a.gaussians, seed=0, width=1000, height=667, n_views=1)
+    jit = synth.jittered(scene, seed=1)
+    budget = int(a.budget_mib * (1 << 20))
+    rows = []
+    for width in [int(w) for w in a.sweep.split(",")]:
+        cam = synth.sweep_camera(width)
+        jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
+        target_dev = Stepper(jm, budget=budget).render(cam)
+        del jm
+        # whole image: the view's target resident; bounded: the supervision
+        # supplied one Leaf crop at a time from pinned host memory
+        target_host = target_dev.cpu().pin_memory()
+        losses = {}
+        for mode in ("original", "bounded"):
+            target = target_dev if mode == "original" else target_host
+            model = GaussianModel(scene.params, scene.n, scene.sh_degree)
+            stp = Stepper(model, budget=budget, mode=mode, binning=a.binning)
+            torch.cuda.synchronize()
+            torch.cuda.reset_peak_memory_stats()
+            base = torch.cuda.memory_allocated()
+            st0 = stp.run_view(cam, target)
+            losses[mode] = stp.last_loss()
+            for _ in range(max(a.warmup - 1, 0)):
+                stp.run_view(cam, target)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(a.steps):
+                st = stp.run_view(cam, target)
+            e1.record()
+            torch.cuda.synchronize()
+            stp.check()
+            ms = e0.elapsed_time(e1) / a.steps
+            peak = (torch.cuda.max_memory_allocated() - base) / 2 ** 30
+            row = {"sweep": "resolution", "width": width, "height": cam.height, "mode": mode,
+                   "target": "resident" if mode == "original" else "pinned host, per-Leaf crops",
+                   "ms_per_step": round(ms, 3),
+                   "working_set_gib": round(st0.peak_ws_bytes / 2 ** 30, 4),
+                   "device_peak_above_model_gib": round(peak, 4),
+                   "loss_first_step": losses[mode], "leaves": st.n_leaves,
+                   "candidates": st.n_cand, "isect": st.n_isect_square,
+                   "list_entries": st.n_isect}
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+            del stp, model
+            torch.cuda.empty_cache()
+        rel = abs(losses["original"] - losses["bounded"]) / max(abs(losses["original"]), 1e-30)
+        rows.append({"sweep": "resolution", "width": width, "l1_rel_diff": rel})
+        print(json.dumps(rows[-1]), flush=True)
+        del target, target_dev, target_host
+        torch.cuda.empty_cache()
+    diffs = [r["l1_rel_diff"] for r in rows if "l1_rel_diff" in r]
+    print(json.dumps({"sweep": "resolution", "summary": True, "max_l1_rel_diff": max(diffs),
+                      "workload": workload_name(a) + ", camera 0 pose, fixed field of view"}))
 
 
 def run_reference(a, rank, world):

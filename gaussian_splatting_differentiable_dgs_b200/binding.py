@@ -273,6 +273,7 @@ def gs_sort_keys32_noalloc(keys_in, keys, vals, n, begin_bit, end_bit, flags, de
         _stream(stream)))
 
 
+GS_PROJ_DENSE = 1
 GS_BIN_SORT = 0
 GS_BIN_EXPAND = 1
 TILE_BLOCK = 8

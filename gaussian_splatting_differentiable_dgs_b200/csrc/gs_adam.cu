@@ -235,6 +235,11 @@ k_project_bwd(const float* __restrict__ P, int64_t n_pad, int D, BwdCam cam, int
   const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (j >= n_cand) return;
   const int64_t i = cand_idx[j];
+  if (rec[3 * j + 2].w < 0.f) {  // culled Gaussian of the dense layout: no gradient
+    for (int plane = 0; plane < 11 + 3 * (D + 1) * (D + 1); ++plane)
+      g3d[(int64_t)plane * stride + j] = 0.f;
+    return;
+  }
   candidate_grad<true>(P, n_pad, i, D, cam, g2d + 12 * j, rec[3 * j + 2],
                  [&](int plane, double g) { g3d[(int64_t)plane * stride + j] = (float)g; });
 }
@@ -268,11 +273,17 @@ k_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads)
 k_project_bwd_geo(const float* __restrict__ P, int64_t n_pad, BwdCam cam, int64_t n_cand,
-                  const int32_t* __restrict__ cand_idx, const float* __restrict__ g2d,
-                  double* __restrict__ g_mean, float* __restrict__ g_rest) {
+                  const int32_t* __restrict__ cand_idx, const float4* __restrict__ rec,
+                  const float* __restrict__ g2d, double* __restrict__ g_mean,
+                  float* __restrict__ g_rest) {
   const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (j >= n_cand) return;
   const int64_t i = cand_idx[j];
+  if (rec[3 * j + 2].w < 0.f) {  // culled Gaussian of the dense layout
+    for (int plane = 0; plane < 3; ++plane) g_mean[(int64_t)plane * n_cand + j] = 0.0;
+    for (int plane = 0; plane < 8; ++plane) g_rest[(int64_t)plane * n_cand + j] = 0.f;
+    return;
+  }
   candidate_grad<false>(P, n_pad, i, 0, cam, g2d + 12 * j, make_float4(0.f, 0.f, 0.f, 0.f),
                  [&](int plane, double gv) {
                    if (plane < 3) g_mean[(int64_t)plane * n_cand + j] = gv;
@@ -519,7 +530,7 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
   float* g_rest = g3d + 6 * n_cand;
   if (n_cand > 0) {
     k_project_bwd_geo<<<(unsigned)((n_cand + kThreads - 1) / kThreads), kThreads, 0, s>>>(
-        model->params, model->n_pad, c, n_cand, proj->cand_idx, g2d, g_mean, g_rest);
+        model->params, model->n_pad, c, n_cand, proj->cand_idx, rec, g2d, g_mean, g_rest);
     GS_LAUNCH_CHECK();
   }
   const unsigned nb = (unsigned)((model->n + kThreads - 1) / kThreads);

@@ -61,7 +61,8 @@ k_bin(const short4* __restrict__ drect, const int32_t* __restrict__ order,
     if (j < n_cand) {
       const short4 r = drect[j];
       int rx0 = r.x, ry0 = r.y, rx1 = r.z, ry1 = r.w;
-      if (BLK > 1) {  // rects are non-empty, so r.z, r.w >= 1
+      if (rx1 <= rx0 || ry1 <= ry0) rx1 = rx0 = ry1 = ry0 = 0;  // culled (dense layout)
+      if (BLK > 1 && rx1 > rx0) {  // a non-empty rect has r.z, r.w >= 1
         rx0 /= BLK;
         ry0 /= BLK;
         rx1 = (rx1 - 1) / BLK + 1;

@@ -232,7 +232,7 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
           short4* __restrict__ rect, uint32_t* __restrict__ depth_key, int32_t* __restrict__ diff,
           unsigned long long* __restrict__ lb, unsigned int* __restrict__ ticket,
           int32_t* __restrict__ n_cand, int64_t n_blocks, int64_t capacity,
-          unsigned long long* __restrict__ square_isect, int32_t* dev_status) {
+          unsigned long long* __restrict__ square_isect, bool dense, int32_t* dev_status) {
   __shared__ unsigned int s_b;
   __shared__ int s_scan[kProjThreads / 32 + 1];
   __shared__ long long s_prefix;
@@ -246,6 +246,41 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
   // geometric planes; the 48 SH planes are read after it, by candidates
   const bool cand = i < n && project_geometry(params, n_pad, i, cam, o, nonfinite);
   if (nonfinite) dev_flag(dev_status, GS_DEV_NONFINITE);
+  if (dense) {
+    // every Gaussian keeps slot i; a culled one gets an empty rect, depth -1
+    // and the largest depth key (it is never binned)
+    if (i < n) {
+      slot_map[i] = (int32_t)i;
+      cand_idx[i] = (int32_t)i;
+      if (cand) {
+        float4 r0, r1, r2;
+        sh_record<D>(params, n_pad, i, cam, o, r0, r1, r2);
+        rec[3 * i] = r0;
+        rec[3 * i + 1] = r1;
+        rec[3 * i + 2] = r2;
+        rect[i] = o.rect;
+        depth_key[i] = __float_as_uint(r2.w);
+        const int64_t s = cam.TW + 1;
+        atomicAdd(&diff[o.rect.y * s + o.rect.x], 1);
+        atomicAdd(&diff[o.rect.y * s + o.rect.z], -1);
+        atomicAdd(&diff[o.rect.w * s + o.rect.x], -1);
+        atomicAdd(&diff[o.rect.w * s + o.rect.z], 1);
+      } else {
+        rec[3 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        rec[3 * i + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        rec[3 * i + 2] = make_float4(0.f, 0.f, 0.f, -1.f);
+        rect[i] = make_short4(0, 0, 0, 0);
+        depth_key[i] = 0xffffffffu;
+      }
+      if (i == n - 1) *n_cand = (int32_t)n;
+    }
+    if (square_isect) {  // every lane of the warp takes part
+      unsigned long long sq = cand ? (unsigned long long)o.square_tiles : 0ull;
+      sq = warp_sum(sq);
+      if ((threadIdx.x & 31) == 0 && sq) atomicAdd(square_isect, sq);
+    }
+    return;
+  }
   int total;
   const int rank = block_exclusive_scan<int, kProjThreads / 32>(cand ? 1 : 0, s_scan, &total);
   if (threadIdx.x < 32) {
@@ -339,6 +374,7 @@ k_block_diff(const short4* __restrict__ rect, const int32_t* __restrict__ n_cand
   const int s = BW + 1;
   for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256) {
     const short4 r = rect[i];
+    if (r.z <= r.x || r.w <= r.y) continue;  // a culled Gaussian of the dense layout
     const int bx0 = r.x / GS_TILE_BLOCK, by0 = r.y / GS_TILE_BLOCK;
     const int bx1 = (r.z - 1) / GS_TILE_BLOCK + 1, by1 = (r.w - 1) / GS_TILE_BLOCK + 1;
     atomicAdd(&d[by0 * s + bx0], 1);
@@ -403,7 +439,8 @@ extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uin
                                 const gs_proj* out, int64_t* tile_sat, void* ws, size_t ws_bytes,
                                 int32_t* dev_status, gs_stream stream) {
   if (!model || !cam || !out || !tile_sat) return GS_ERR_ARG;
-  if (flags != 0) return GS_ERR_UNSUPPORTED;
+  if (flags & ~GS_PROJ_DENSE) return GS_ERR_UNSUPPORTED;
+  const bool dense = (flags & GS_PROJ_DENSE) != 0;
   if (model->n < 0 || model->n_pad < model->n || (model->n_pad & 3) || model->sh_degree < 0 ||
       model->sh_degree > 3)
     return GS_ERR_ARG;
@@ -439,7 +476,8 @@ extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uin
   k_project<DD><<<(unsigned)nb, kProjThreads, 0, s>>>(                                       \
       model->params, model->n, model->n_pad, pc, out->cand_idx, out->slot,                   \
       reinterpret_cast<float4*>(out->rec), reinterpret_cast<short4*>(out->rect), out->depth_key, \
-      w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, out->square_isect, dev_status)
+      w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, out->square_isect, dense,     \
+      dev_status)
     switch (model->sh_degree) {
       case 0: GS_PROJ(0); break;
       case 1: GS_PROJ(1); break;

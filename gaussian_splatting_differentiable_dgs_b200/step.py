@@ -111,9 +111,17 @@ class Stepper:
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
-                 binning="fused", device="cuda"):
+                 binning="fused", mode="bounded", device="cuda"):
         if binning not in ("fused", "expand", "sort"):
             raise ValueError(f"binning must be 'fused', 'expand' or 'sort', not {binning!r}")
+        if mode not in ("bounded", "original"):
+            raise ValueError(f"mode must be 'bounded' or 'original', not {mode!r}")
+        # bounded: two-stage backward, Leaves under the budget, candidate-index
+        # projection and compact gradients (BoundedGS page, section 02, A -> E);
+        # original: the whole-image configuration A of the same page (dense
+        # projection state, one whole-image Leaf whose raster buffers stay
+        # alive through the projection backward, dense gradients)
+        self.mode = mode
         self.model = model
         self.binning = binning
         self.budget = int(budget)
@@ -179,7 +187,8 @@ class Stepper:
         sat = torch.empty((TH + 1) * (TW + 1), dtype=torch.int64, device=dev)
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
         tk = clk.tic("project")
-        B.gs_project(mod, camS, proj, sat, ws, st)
+        original = self.mode == "original"
+        B.gs_project(mod, camS, proj, sat, ws, st, flags=B.GS_PROJ_DENSE if original else 0)
         # fused: per-block lists, each tile's list built inside the forward;
         # expand: per-block lists expanded into full tile lists per Leaf;
         # sort: per-Leaf (tile, candidate) entries sorted by tile
@@ -241,6 +250,8 @@ class Stepper:
 
         # ---- Leaf plan ------------------------------------------------------
         lm = B.gs_leaf_load_model(tile_bits, B.GS_BIN_EXPAND if expand else B.GS_BIN_SORT)
+        if leaves is None and original:
+            leaves = [(0, 0, TW, TH)]
         if leaves is None:
             _, lv, li, lb, ov = B.gs_leaf_partition(sat_np, TW, TH, W, H, lm, self.budget)
         else:
@@ -373,9 +384,10 @@ class Stepper:
                 tk = clk.tic("raster_bwd")
                 B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
                 clk.toc(tk)
-        del arena, bin_ws  # raster buffers released before projection backward
-        if host_target:
-            del crops
+        if not original:
+            del arena, bin_ws  # raster buffers released before projection backward
+            if host_target:
+                del crops
 
         loss_d = torch.zeros(1, dtype=torch.float64, device=dev)
         if target is not None:
@@ -388,7 +400,7 @@ class Stepper:
         # ---- projection backward fused with ONE Adam update -----------------
         if update:
             m.step += 1
-            if self.fuse_adam:
+            if self.fuse_adam and not original:
                 geo = torch.empty(14 * max(C, 1), dtype=torch.float32, device=dev)
                 tk = clk.tic("project_bwd")
                 B.gs_project_bwd(mod, camS, proj, C, g2d, g3d=geo, g3d_stride=geo.numel(),
@@ -398,10 +410,12 @@ class Stepper:
                 del geo
             else:
                 g3d = torch.empty(m.P * max(C, 1), dtype=torch.float32, device=dev)
+                tk = clk.tic("project_bwd")
                 B.gs_project_bwd(mod, camS, proj, C, g2d, g3d=g3d, g3d_stride=max(C, 1),
                                  dev_status=st)
                 B.gs_adam(m.params, m.m, m.v, g3d, max(C, 1), slot, m.n, m.n_pad, m.P,
                           self.adam_args(m.step))
+                clk.toc(tk)
                 del g3d
         peak = torch.cuda.max_memory_allocated(dev) - base_alloc
         if resident_target:

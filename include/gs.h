@@ -210,7 +210,12 @@ gs_status gs_check(int32_t* dev_status, gs_stream stream);
  * (TH+1) x (TW+1) int64 summed-area table of per-tile intersection counts
  * (row 0 and column 0 zero) to `tile_sat`.
  * The projection arithmetic is fp64; records are rounded to fp32.
- * flags: 0 (reserved). */
+ * flags: 0, or GS_PROJ_DENSE: the whole-image ("Original") layout of the
+ * BoundedGS page, Fig. A and the ablation's configuration A: every Gaussian
+ * keeps slot i (n_cand = n, cand_idx = identity), a culled one gets an
+ * empty rect, depth -1 in its record and depth key 0xffffffff; the SAT and
+ * all later stages skip it. */
+#define GS_PROJ_DENSE 1u
 size_t gs_project_workspace_size(int64_t n, int32_t width, int32_t height);
 gs_status gs_project(const gs_model* model, const gs_camera* cam,
                      uint32_t flags, const gs_proj* out, int64_t* tile_sat,

@@ -150,6 +150,39 @@ def _sort_ws(n, kb, lo, hi):
                        device="cuda")
 
 
+def test_project_dense_layout(oracle_mod):
+    """GS_PROJ_DENSE: slot i for every Gaussian; candidates' records, rects and
+    keys equal the compact projection's, culled ones are marked; same SAT."""
+    sc, cam = scene("hd")
+    b = B()
+    pb, sat, params = run_project(sc, cam)
+    C = int(pb.n_cand.item())
+    n = sc.n
+    pd = ProjBuffers(n)
+    model = b.gs_model(n, sc.n_pad, sc.sh_degree, 0, params.data_ptr())
+    TW, TH = (cam.width + 15) // 16, (cam.height + 15) // 16
+    sat_d = torch.zeros((TH + 1) * (TW + 1), dtype=torch.int64, device="cuda")
+    ws = torch.empty(b.gs_project_workspace_size(n, cam.width, cam.height), dtype=torch.uint8,
+                     device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b.gs_project(model, b.camera_struct(cam), pd.struct, sat_d, ws, st, flags=b.GS_PROJ_DENSE)
+    assert b.gs_check(st) == 0
+    assert int(pd.n_cand.item()) == n and C < n
+    assert (sat_d.cpu().numpy().reshape(TH + 1, TW + 1) == sat).all()
+    assert (pd.cand_idx.cpu().numpy() == np.arange(n)).all()
+    ci = pb.cand_idx[:C].cpu().numpy()
+    live = np.zeros(n, bool)
+    live[ci] = True
+    rec_d = pd.rec.cpu().numpy().reshape(n, 12)
+    rec_c = pb.rec[:12 * C].cpu().numpy().reshape(C, 12)
+    assert (rec_d[ci].view(np.uint32) == rec_c.view(np.uint32)).all()
+    assert (pd.rect.cpu().numpy().reshape(n, 4)[ci] == pb.rect[:4 * C].cpu().numpy().reshape(C, 4)).all()
+    assert (pd.depth_key.cpu().numpy()[ci] == pb.depth_key[:C].cpu().numpy()).all()
+    assert (rec_d[~live, 11] == -1).all()
+    assert (pd.rect.cpu().numpy().reshape(n, 4)[~live] == 0).all()
+    assert (pd.depth_key.cpu().numpy()[~live].view(np.uint32) == 0xffffffff).all()
+
+
 @pytest.mark.parametrize("n", [1, 100, 4095, 4096, 4097, 50_000, 1_000_003])
 @pytest.mark.parametrize("bits", [(0, 32), (0, 13), (7, 23), (3, 3)])
 @pytest.mark.parametrize("onesweep", [False, True])
@@ -630,23 +663,31 @@ class Capture:
         self.cand_idx = ctx["cand_idx"][:ctx["n_cand"]].cpu().numpy()
 
 
-@pytest.mark.parametrize("name,budget,binning", [
-    ("tiny", 384 << 20, "fused"), ("tiny", 120_000, "fused"), ("tiny", 120_000, "expand"),
-    ("tiny", 120_000, "sort"), ("ragged", 30_000, "fused"), ("small3", 200_000, "fused"),
-    ("small3", 200_000, "sort"), ("hd", 384 << 20, "fused"), ("hd", 20 << 20, "fused"),
-    ("hd", 20 << 20, "expand"), ("hd", 20 << 20, "sort")])
-def test_end_to_end_step(oracle_mod, name, budget, binning):
+@pytest.mark.parametrize("name,budget,binning,mode", [
+    ("tiny", 384 << 20, "fused", "bounded"), ("tiny", 120_000, "fused", "bounded"),
+    ("tiny", 120_000, "expand", "bounded"), ("tiny", 120_000, "sort", "bounded"),
+    ("ragged", 30_000, "fused", "bounded"), ("small3", 200_000, "fused", "bounded"),
+    ("small3", 200_000, "sort", "bounded"), ("hd", 384 << 20, "fused", "bounded"),
+    ("hd", 20 << 20, "fused", "bounded"), ("hd", 20 << 20, "expand", "bounded"),
+    ("hd", 20 << 20, "sort", "bounded"), ("tiny", 120_000, "fused", "original"),
+    ("ragged", 30_000, "sort", "original"), ("hd", 20 << 20, "fused", "original")])
+def test_end_to_end_step(oracle_mod, name, budget, binning, mode):
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, cam = scene(name)
     target = synth.random_image(cam.width, cam.height, 12) * 0.6
     ref = oracle_mod.step(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam,
                           target.astype(np.float64))
     model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=budget, fuse_adam=False, binning=binning)
+    stp = Stepper(model, budget=budget, fuse_adam=False, binning=binning, mode=mode)
     cap = Capture(cam.width, cam.height)
     stats = stp.run_view(cam, torch.as_tensor(target).cuda(), hooks=cap)
     stp.check()
-    if budget < (384 << 20):
+    if mode == "original":
+        assert stats.n_leaves == 1 and stats.n_cand == sc.n
+        live = np.isin(np.arange(sc.n), ref["proj"]["cand_idx"])
+        cap.cand_idx = np.arange(sc.n)[live]
+        cap.g2d = cap.g2d[:sc.n][live]
+    elif budget < (384 << 20):
         assert stats.n_leaves > 1
     assert stats.n_isect == ref["n_isect"]
     ok = (ref["pflags"] & 0x81) == 0
