@@ -81,11 +81,12 @@ struct Eval {
   float dx, dy, t1, G, araw, alpha;
 };
 
-// alpha = min(0.99, o 2^(-q log2 e)),  q = s1 (dx + beta dy)^2 + s2 dy^2
-__device__ __forceinline__ Eval eval_alpha(float gx, float gy, float beta, float ns1, float ns2,
-                                           float opac, float px, float py) {
+// alpha = min(0.99, o 2^(-q log2 e)),  q = s1 (dx + beta dy)^2 + s2 dy^2,
+// with dx = gx - px given (a lane's pixels share their column)
+__device__ __forceinline__ Eval eval_alpha(float dx, float gy, float beta, float ns1, float ns2,
+                                           float opac, float py) {
   Eval e;
-  e.dx = __fsub_rn(gx, px);
+  e.dx = dx;
   e.dy = __fsub_rn(gy, py);
   e.t1 = __fmaf_rn(beta, e.dy, e.dx);
   const float qa = __fmul_rn(ns1, e.t1);
@@ -350,10 +351,11 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       const float4 B = sB[j];
       const float Bb = sC[j];
       const int posn = pos1 + j;
+      const float dx = __fsub_rn(A.x, fpx);
 #pragma unroll
       for (int k = 0; k < PPT; ++k) {
         if (done[k]) continue;
-        const Eval ev = eval_alpha(A.x, A.y, A.z, A.w, B.x, B.y, fpx, fpy[k]);
+        const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
         if (COUNT) ++n_vis;
         if (ev.alpha < kAlphaMin) continue;
         const float Tn = __fmul_rn(T[k], __fsub_rn(1.0f, ev.alpha));
@@ -593,11 +595,15 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       float acc[9];
 #pragma unroll
       for (int q = 0; q < 9; ++q) acc[q] = 0.0f;
+      // the lane's pixels share dx, so the geometric terms need only
+      // sum dq, sum dq dy and sum dq dy^2 over them
+      float sq = 0.0f, sqy = 0.0f, sqyy = 0.0f;
       bool any = false;
+      const float dx = __fsub_rn(A.x, fpx);
 #pragma unroll
       for (int k = 0; k < PPT; ++k) {
         if (pos >= lastp[k]) continue;
-        const Eval ev = eval_alpha(A.x, A.y, A.z, A.w, B.x, B.y, fpx, fpy[k]);
+        const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
         if (COUNT) ++n_vis;
         if (ev.alpha < kAlphaMin) continue;
         if (COUNT) ++n_kept;
@@ -619,15 +625,20 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         if (ev.araw <= kAlphaMax) {
           const float dq = -ev.alpha * da;         // dL/dq (natural units)
           acc[5] = fmaf(ev.G, da, acc[5]);          // dL/dopacity
-          const float s1t = Cc.y * ev.t1;           // dq/du = a dx + b dy
-          acc[0] = fmaf(dq, s1t, acc[0]);
-          acc[1] = fmaf(dq, fmaf(s1t, A.z, Cc.z * ev.dy), acc[1]);  // dq/dv
-          const float hq = 0.5f * dq;
-          acc[2] = fmaf(hq * ev.dx, ev.dx, acc[2]);
-          acc[3] = fmaf(dq * ev.dx, ev.dy, acc[3]);
-          acc[4] = fmaf(hq * ev.dy, ev.dy, acc[4]);
+          sq += dq;
+          const float dqy = dq * ev.dy;
+          sqy += dqy;
+          sqyy = fmaf(dqy, ev.dy, sqyy);
         }
       }
+      // q = (a dx^2 + c dy^2) / 2 + b dx dy with a = 2 s1, b = beta a,
+      // c = 2 s2 + beta b: dq/du = a dx + b dy, dq/dv = b dx + c dy
+      // = beta dq/du + 2 s2 dy, dq/da = dx^2 / 2, dq/db = dx dy, dq/dc = dy^2 / 2
+      acc[0] = Cc.y * fmaf(A.z, sqy, dx * sq);
+      acc[1] = fmaf(A.z, acc[0], Cc.z * sqy);
+      acc[2] = 0.5f * dx * dx * sq;
+      acc[3] = dx * sqy;
+      acc[4] = 0.5f * sqyy;
       // reduce first: per-lane shared atomics on the same 9 words cost more
       // than the reduction, even with only 2 lanes kept
       if (__any_sync(0xffffffffu, any)) {
