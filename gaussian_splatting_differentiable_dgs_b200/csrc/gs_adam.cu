@@ -42,124 +42,125 @@ __device__ __forceinline__ void adam_update(float* __restrict__ p, float* __rest
 }
 
 // Gradients of one candidate.  `emit(plane, g)` receives every parameter's
-// gradient exactly once, SH planes first, then planes 10 .. 0.
-template <bool WITH_SH, class Emit>
+// gradient exactly once, SH planes first, then planes 10 .. 0.  Real: the
+// type of the geometric chain (the SH part is fp64).
+template <bool WITH_SH, class Real, class Emit>
 __device__ __forceinline__ void candidate_grad(const float* __restrict__ P, int64_t n_pad, int64_t i,
                                                int D, const BwdCam& c, const float* __restrict__ g2,
                                                const float4 rgb_rec, Emit&& emit) {
-  const double mx = P[i], my = P[n_pad + i], mz = P[2 * n_pad + i];
-  double tc[3];
+  const Real mx = P[i], my = P[n_pad + i], mz = P[2 * n_pad + i];
+  Real tc[3];
 #pragma unroll
-  for (int r = 0; r < 3; ++r) tc[r] = c.R[3 * r] * mx + c.R[3 * r + 1] * my + c.R[3 * r + 2] * mz + c.t[r];
-  const double tx = tc[0], ty = tc[1], tz = tc[2];
-  double qw = P[6 * n_pad + i], qx = P[7 * n_pad + i], qy = P[8 * n_pad + i], qz = P[9 * n_pad + i];
-  const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+  for (int r = 0; r < 3; ++r) tc[r] = Real(c.R[3 * r]) * mx + Real(c.R[3 * r + 1]) * my + Real(c.R[3 * r + 2]) * mz + Real(c.t[r]);
+  const Real tx = tc[0], ty = tc[1], tz = tc[2];
+  Real qw = P[6 * n_pad + i], qx = P[7 * n_pad + i], qy = P[8 * n_pad + i], qz = P[9 * n_pad + i];
+  const Real qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
   qw /= qn; qx /= qn; qy /= qn; qz /= qn;
-  double Rg[9];
-  Rg[0] = 1.0 - 2.0 * (qy * qy + qz * qz); Rg[1] = 2.0 * (qx * qy - qw * qz); Rg[2] = 2.0 * (qx * qz + qw * qy);
-  Rg[3] = 2.0 * (qx * qy + qw * qz); Rg[4] = 1.0 - 2.0 * (qx * qx + qz * qz); Rg[5] = 2.0 * (qy * qz - qw * qx);
-  Rg[6] = 2.0 * (qx * qz - qw * qy); Rg[7] = 2.0 * (qy * qz + qw * qx); Rg[8] = 1.0 - 2.0 * (qx * qx + qy * qy);
-  double sc[3];
+  Real Rg[9];
+  Rg[0] = Real(1.0) - Real(2.0) * (qy * qy + qz * qz); Rg[1] = Real(2.0) * (qx * qy - qw * qz); Rg[2] = Real(2.0) * (qx * qz + qw * qy);
+  Rg[3] = Real(2.0) * (qx * qy + qw * qz); Rg[4] = Real(1.0) - Real(2.0) * (qx * qx + qz * qz); Rg[5] = Real(2.0) * (qy * qz - qw * qx);
+  Rg[6] = Real(2.0) * (qx * qz - qw * qy); Rg[7] = Real(2.0) * (qy * qz + qw * qx); Rg[8] = Real(1.0) - Real(2.0) * (qx * qx + qy * qy);
+  Real sc[3];
 #pragma unroll
-  for (int k = 0; k < 3; ++k) sc[k] = exp((double)P[(3 + k) * n_pad + i]);
-  double M[9];
+  for (int k = 0; k < 3; ++k) sc[k] = exp((Real)P[(3 + k) * n_pad + i]);
+  Real M[9];
 #pragma unroll
   for (int r = 0; r < 3; ++r)
 #pragma unroll
     for (int k = 0; k < 3; ++k) M[3 * r + k] = Rg[3 * r + k] * sc[k];
-  double Sg[9];
+  Real Sg[9];
 #pragma unroll
   for (int r = 0; r < 3; ++r)
 #pragma unroll
     for (int k = 0; k < 3; ++k)
       Sg[3 * r + k] = M[3 * r] * M[3 * k] + M[3 * r + 1] * M[3 * k + 1] + M[3 * r + 2] * M[3 * k + 2];
-  const double tz2 = tz * tz;
-  const double j00 = c.fx / tz, j02 = -c.fx * tx / tz2, j11 = c.fy / tz, j12 = -c.fy * ty / tz2;
-  double T0[3], T1[3];
+  const Real tz2 = tz * tz;
+  const Real j00 = Real(c.fx) / tz, j02 = -Real(c.fx) * tx / tz2, j11 = Real(c.fy) / tz, j12 = -Real(c.fy) * ty / tz2;
+  Real T0[3], T1[3];
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
-    T0[k] = j00 * c.R[k] + j02 * c.R[6 + k];
-    T1[k] = j11 * c.R[3 + k] + j12 * c.R[6 + k];
+    T0[k] = j00 * Real(c.R[k]) + j02 * Real(c.R[6 + k]);
+    T1[k] = j11 * Real(c.R[3 + k]) + j12 * Real(c.R[6 + k]);
   }
-  double A0[3], A1[3];  // rows of T Sigma
+  Real A0[3], A1[3];  // rows of T Sigma
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     A0[k] = T0[0] * Sg[k] + T0[1] * Sg[3 + k] + T0[2] * Sg[6 + k];
     A1[k] = T1[0] * Sg[k] + T1[1] * Sg[3 + k] + T1[2] * Sg[6 + k];
   }
-  const double c00 = A0[0] * T0[0] + A0[1] * T0[1] + A0[2] * T0[2] + 0.3;
-  const double c01 = 0.5 * ((A0[0] * T1[0] + A0[1] * T1[1] + A0[2] * T1[2]) +
+  const Real c00 = A0[0] * T0[0] + A0[1] * T0[1] + A0[2] * T0[2] + Real(0.3);
+  const Real c01 = Real(0.5) * ((A0[0] * T1[0] + A0[1] * T1[1] + A0[2] * T1[2]) +
                             (A1[0] * T0[0] + A1[1] * T0[1] + A1[2] * T0[2]));
-  const double c11 = A1[0] * T1[0] + A1[1] * T1[1] + A1[2] * T1[2] + 0.3;
-  const double det = c00 * c11 - c01 * c01;
-  const double qa = c11 / det, qb = -c01 / det, qc = c00 / det;  // conic
+  const Real c11 = A1[0] * T1[0] + A1[1] * T1[1] + A1[2] * T1[2] + Real(0.3);
+  const Real det = c00 * c11 - c01 * c01;
+  const Real qa = c11 / det, qb = -c01 / det, qc = c00 / det;  // conic
 
-  const double du = g2[0], dv = g2[1], dA = g2[2], dB = g2[3], dC = g2[4], dO = g2[5];
-  const double dcol[3] = {g2[6], g2[7], g2[8]};
+  const Real du = g2[0], dv = g2[1], dA = g2[2], dB = g2[3], dC = g2[4], dO = g2[5];
+  const Real dcol[3] = {g2[6], g2[7], g2[8]};
 
   // conic -> Sigma': dS = -Q Gbar Q,  Gbar = [[dA, dB/2], [dB/2, dC]]
-  const double hB = 0.5 * dB;
-  const double m00 = qa * dA + qb * hB, m01 = qa * hB + qb * dC;
-  const double m10 = qb * dA + qc * hB, m11 = qb * hB + qc * dC;
-  const double G00 = -(m00 * qa + m01 * qb);
-  const double G01 = -(m00 * qb + m01 * qc);
-  const double G11 = -(m10 * qb + m11 * qc);
-  // Sigma' = T Sigma T^T + 0.3 I  ->  dSigma = T^T G T,  dT = 2 G T Sigma
-  double dS[9];
+  const Real hB = Real(0.5) * dB;
+  const Real m00 = qa * dA + qb * hB, m01 = qa * hB + qb * dC;
+  const Real m10 = qb * dA + qc * hB, m11 = qb * hB + qc * dC;
+  const Real G00 = -(m00 * qa + m01 * qb);
+  const Real G01 = -(m00 * qb + m01 * qc);
+  const Real G11 = -(m10 * qb + m11 * qc);
+  // Sigma' = T Sigma T^T + Real(0.3) I  ->  dSigma = T^T G T,  dT = 2 G T Sigma
+  Real dS[9];
 #pragma unroll
   for (int r = 0; r < 3; ++r)
 #pragma unroll
     for (int k = 0; k < 3; ++k)
       dS[3 * r + k] = T0[r] * (G00 * T0[k] + G01 * T1[k]) + T1[r] * (G01 * T0[k] + G11 * T1[k]);
-  double dT0[3], dT1[3];
+  Real dT0[3], dT1[3];
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
-    dT0[k] = 2.0 * (G00 * A0[k] + G01 * A1[k]);
-    dT1[k] = 2.0 * (G01 * A0[k] + G11 * A1[k]);
+    dT0[k] = Real(2.0) * (G00 * A0[k] + G01 * A1[k]);
+    dT1[k] = Real(2.0) * (G01 * A0[k] + G11 * A1[k]);
   }
   // T = J W
-  const double dJ00 = dT0[0] * c.R[0] + dT0[1] * c.R[1] + dT0[2] * c.R[2];
-  const double dJ02 = dT0[0] * c.R[6] + dT0[1] * c.R[7] + dT0[2] * c.R[8];
-  const double dJ11 = dT1[0] * c.R[3] + dT1[1] * c.R[4] + dT1[2] * c.R[5];
-  const double dJ12 = dT1[0] * c.R[6] + dT1[1] * c.R[7] + dT1[2] * c.R[8];
-  const double tz3 = tz2 * tz;
-  const double dtx = -dJ02 * c.fx / tz2 + du * c.fx / tz;
-  const double dty = -dJ12 * c.fy / tz2 + dv * c.fy / tz;
-  const double dtz = -dJ00 * c.fx / tz2 + dJ02 * 2.0 * c.fx * tx / tz3 - dJ11 * c.fy / tz2 +
-                     dJ12 * 2.0 * c.fy * ty / tz3 - du * c.fx * tx / tz2 - dv * c.fy * ty / tz2;
-  double dmean[3];
+  const Real dJ00 = dT0[0] * Real(c.R[0]) + dT0[1] * Real(c.R[1]) + dT0[2] * Real(c.R[2]);
+  const Real dJ02 = dT0[0] * Real(c.R[6]) + dT0[1] * Real(c.R[7]) + dT0[2] * Real(c.R[8]);
+  const Real dJ11 = dT1[0] * Real(c.R[3]) + dT1[1] * Real(c.R[4]) + dT1[2] * Real(c.R[5]);
+  const Real dJ12 = dT1[0] * Real(c.R[6]) + dT1[1] * Real(c.R[7]) + dT1[2] * Real(c.R[8]);
+  const Real tz3 = tz2 * tz;
+  const Real dtx = -dJ02 * Real(c.fx) / tz2 + du * Real(c.fx) / tz;
+  const Real dty = -dJ12 * Real(c.fy) / tz2 + dv * Real(c.fy) / tz;
+  const Real dtz = -dJ00 * Real(c.fx) / tz2 + dJ02 * Real(2.0) * Real(c.fx) * tx / tz3 - dJ11 * Real(c.fy) / tz2 +
+                     dJ12 * Real(2.0) * Real(c.fy) * ty / tz3 - du * Real(c.fx) * tx / tz2 - dv * Real(c.fy) * ty / tz2;
+  Real dmean[3];
 #pragma unroll
-  for (int k = 0; k < 3; ++k) dmean[k] = c.R[k] * dtx + c.R[3 + k] * dty + c.R[6 + k] * dtz;
+  for (int k = 0; k < 3; ++k) dmean[k] = Real(c.R[k]) * dtx + Real(c.R[3 + k]) * dty + Real(c.R[6 + k]) * dtz;
   // Sigma = M M^T,  M = R S
-  double dM[9];
+  Real dM[9];
 #pragma unroll
   for (int r = 0; r < 3; ++r)
 #pragma unroll
     for (int k = 0; k < 3; ++k)
-      dM[3 * r + k] = 2.0 * (dS[3 * r] * M[k] + dS[3 * r + 1] * M[3 + k] + dS[3 * r + 2] * M[6 + k]);
-  double dls[3];
+      dM[3 * r + k] = Real(2.0) * (dS[3 * r] * M[k] + dS[3 * r + 1] * M[3 + k] + dS[3 * r + 2] * M[6 + k]);
+  Real dls[3];
 #pragma unroll
   for (int k = 0; k < 3; ++k)
     dls[k] = (dM[k] * Rg[k] + dM[3 + k] * Rg[3 + k] + dM[6 + k] * Rg[6 + k]) * sc[k];
-  double gR[9];
+  Real gR[9];
 #pragma unroll
   for (int r = 0; r < 3; ++r)
 #pragma unroll
     for (int k = 0; k < 3; ++k) gR[3 * r + k] = dM[3 * r + k] * sc[k];
   // rotation of the unit quaternion -> (w, x, y, z)
-  const double gw = 2.0 * (-qz * gR[1] + qy * gR[2] + qz * gR[3] - qx * gR[5] - qy * gR[6] + qx * gR[7]);
-  const double gx = 2.0 * (qy * gR[1] + qz * gR[2] + qy * gR[3] - 2.0 * qx * gR[4] - qw * gR[5] +
-                           qz * gR[6] + qw * gR[7] - 2.0 * qx * gR[8]);
-  const double gy = 2.0 * (-2.0 * qy * gR[0] + qx * gR[1] + qw * gR[2] + qx * gR[3] + qz * gR[5] -
-                           qw * gR[6] + qz * gR[7] - 2.0 * qy * gR[8]);
-  const double gz = 2.0 * (-2.0 * qz * gR[0] - qw * gR[1] + qx * gR[2] + qw * gR[3] - 2.0 * qz * gR[4] +
+  const Real gw = Real(2.0) * (-qz * gR[1] + qy * gR[2] + qz * gR[3] - qx * gR[5] - qy * gR[6] + qx * gR[7]);
+  const Real gx = Real(2.0) * (qy * gR[1] + qz * gR[2] + qy * gR[3] - Real(2.0) * qx * gR[4] - qw * gR[5] +
+                           qz * gR[6] + qw * gR[7] - Real(2.0) * qx * gR[8]);
+  const Real gy = Real(2.0) * (-Real(2.0) * qy * gR[0] + qx * gR[1] + qw * gR[2] + qx * gR[3] + qz * gR[5] -
+                           qw * gR[6] + qz * gR[7] - Real(2.0) * qy * gR[8]);
+  const Real gz = Real(2.0) * (-Real(2.0) * qz * gR[0] - qw * gR[1] + qx * gR[2] + qw * gR[3] - Real(2.0) * qz * gR[4] +
                            qy * gR[5] + qx * gR[6] + qy * gR[7]);
-  const double qdot = gw * qw + gx * qx + gy * qy + gz * qz;
-  const double dq[4] = {(gw - qw * qdot) / qn, (gx - qx * qdot) / qn, (gy - qy * qdot) / qn,
+  const Real qdot = gw * qw + gx * qx + gy * qy + gz * qz;
+  const Real dq[4] = {(gw - qw * qdot) / qn, (gx - qx * qdot) / qn, (gy - qy * qdot) / qn,
                         (gz - qz * qdot) / qn};
   // opacity logit
-  const double o = 1.0 / (1.0 + exp(-(double)P[10 * n_pad + i]));
-  const double dlogit = dO * o * (1.0 - o);
+  const Real o = Real(1.0) / (Real(1.0) + exp(-(Real)P[10 * n_pad + i]));
+  const Real dlogit = dO * o * (Real(1.0) - o);
 
   if constexpr (WITH_SH) {
   // SH coefficients and the view direction
@@ -240,7 +241,7 @@ k_project_bwd(const float* __restrict__ P, int64_t n_pad, int D, BwdCam cam, int
       g3d[(int64_t)plane * stride + j] = 0.f;
     return;
   }
-  candidate_grad<true>(P, n_pad, i, D, cam, g2d + 12 * j, rec[3 * j + 2],
+  candidate_grad<true, double>(P, n_pad, i, D, cam, g2d + 12 * j, rec[3 * j + 2],
                  [&](int plane, double g) { g3d[(int64_t)plane * stride + j] = (float)g; });
 }
 
@@ -264,12 +265,14 @@ k_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
 }
 
 // ---------------------------------------------------------------------------
-// Fused path, stage 1: geometric gradients of each candidate (fp64), i.e.
+// Fused path, stage 1: geometric gradients of each candidate, i.e.
 // everything except the SH coefficients and the view-direction term of the
-// mean, which stage 2 forms while it streams the SH planes.  Scratch layout
-// (14 floats per candidate): double mean[3][C] (kept in fp64: stage 2 adds
-// the view-direction term and the sum may cancel), then float rest[8][C]
-// for planes 3..10 (log-scale, quaternion, logit).
+// mean, which stage 2 forms (fp64) while it streams the SH planes.  The
+// chain runs in fp32 (per-tensor relative L2 error about 3e-6 against the
+// fp64 oracle; the parity bound is 1e-4).  Scratch layout (14 floats per
+// candidate): double mean[3][C] (stage 2 adds the view-direction term, and
+// the sum may cancel), then float rest[8][C] for planes 3..10 (log-scale,
+// quaternion, logit).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads)
 k_project_bwd_geo(const float* __restrict__ P, int64_t n_pad, BwdCam cam, int64_t n_cand,
@@ -284,7 +287,7 @@ k_project_bwd_geo(const float* __restrict__ P, int64_t n_pad, BwdCam cam, int64_
     for (int plane = 0; plane < 8; ++plane) g_rest[(int64_t)plane * n_cand + j] = 0.f;
     return;
   }
-  candidate_grad<false>(P, n_pad, i, 0, cam, g2d + 12 * j, make_float4(0.f, 0.f, 0.f, 0.f),
+  candidate_grad<false, float>(P, n_pad, i, 0, cam, g2d + 12 * j, make_float4(0.f, 0.f, 0.f, 0.f),
                  [&](int plane, double gv) {
                    if (plane < 3) g_mean[(int64_t)plane * n_cand + j] = gv;
                    else if (plane < 11) g_rest[(int64_t)(plane - 3) * n_cand + j] = (float)gv;

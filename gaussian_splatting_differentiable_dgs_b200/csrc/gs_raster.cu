@@ -374,9 +374,13 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       }
     }
   }
-  if (COUNT) {
-    atomicAdd(&px.counters[0], (unsigned long long)n_vis);
-    atomicAdd(&px.counters[1], (unsigned long long)n_kept);
+  if (COUNT) {  // one atomic per warp: per-thread ones on one word serialise
+    const unsigned long long a = warp_sum((unsigned long long)n_vis);
+    const unsigned long long b = warp_sum((unsigned long long)n_kept);
+    if ((t & 31) == 0) {
+      atomicAdd(&px.counters[0], a);
+      atomicAdd(&px.counters[1], b);
+    }
   }
   if (BLK) {
     if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
@@ -661,9 +665,13 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     }
     __syncthreads();
   }
-  if (COUNT) {
-    atomicAdd(&px.counters[0], (unsigned long long)n_vis);
-    atomicAdd(&px.counters[1], (unsigned long long)n_kept);
+  if (COUNT) {  // one atomic per warp: per-thread ones on one word serialise
+    const unsigned long long a = warp_sum((unsigned long long)n_vis);
+    const unsigned long long b = warp_sum((unsigned long long)n_kept);
+    if ((t & 31) == 0) {
+      atomicAdd(&px.counters[0], a);
+      atomicAdd(&px.counters[1], b);
+    }
   }
 }
 

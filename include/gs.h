@@ -467,7 +467,7 @@ gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals,
  * gradients g3d[P][g3d_stride] (column = candidate slot).  Otherwise applies
  * one Adam update (as gs_adam with a zero gradient for non-candidates) to
  * model->params, adam_m and adam_v over all n Gaussians, in two passes: the
- * candidates' geometric gradients (fp64) into g3d used as scratch (>= 14 *
+ * candidates' geometric gradients (fp32 chain) into g3d used as scratch (>= 14 *
  * n_cand floats, 8-byte aligned, g3d_stride = its size in floats), then one
  * streaming pass
  * over every Gaussian's planes that forms the SH gradients on the fly. */

@@ -632,14 +632,34 @@ def test_fused_project_bwd_adam(oracle_mod, name):
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     assert b.gs_check(st) == 0
     n = sc.n
-    # m and v are sums of two terms that can cancel: bound the error by the
-    # magnitude of the terms (fp32 rounding of the terms and of g)
-    gm = np.abs(grad[:, :n])
+    ci = pr["cand_idx"]
+    md_h, vd_h, pd_h = md.cpu().numpy(), vd.cpu().numpy(), params.cpu().numpy()
+    # 1. the candidates' geometric gradients (scratch planes 3..10, fp32
+    #    chain) against the oracle: relative L2 per tensor
+    raw = geo.cpu().numpy()
+    g_rest = raw[6 * C:14 * C].reshape(8, C).astype(np.float64)
+    for k in range(8):
+        assert rel_l2(g_rest[k], g3d_o[3 + k]) <= GRAD_TOL, 3 + k
+    # 2. Adam on those planes: element-wise against the update of the
+    #    kernel's own gradients.  m and v are sums of two terms that can
+    #    cancel: the bound follows the magnitude of the terms
+    own = grad.copy()
+    own[3:11, ci] = g_rest
+    pe2, me2, ve2 = oracle_mod.adam(sc.params, m0, v0, own, step=2)
+    gm = np.abs(own[:, :n])
     m_scale = 0.9 * np.abs(m0[:, :n]) + 0.1 * gm
     v_scale = 0.999 * v0[:, :n] + 0.001 * gm * gm
-    assert (np.abs(md.cpu().numpy()[:, :n] - me[:, :n]) <= 1e-6 * m_scale + 1e-30).all()
-    assert (np.abs(vd.cpu().numpy()[:, :n] - ve[:, :n]) <= 1e-6 * v_scale + 1e-30).all()
-    np.testing.assert_allclose(params.cpu().numpy()[:, :n], pe[:, :n], rtol=1e-6, atol=2e-8)
+    rows = np.r_[3:11, 11:sc.P]   # geometric planes (own g) and SH planes (fp64 g)
+    assert (np.abs(md_h[rows, :n] - me2[rows, :n]) <= 1e-6 * m_scale[rows] + 1e-30).all()
+    assert (np.abs(vd_h[rows, :n] - ve2[rows, :n]) <= 1e-6 * v_scale[rows] + 1e-30).all()
+    np.testing.assert_allclose(pd_h[rows, :n], pe2[rows, :n], rtol=1e-6, atol=2e-8)
+    # 3. the SH planes' gradients equal the oracle's (the same m as above)
+    assert (np.abs(me2[11:, :n] - me[11:, :n]) <= 1e-6 * m_scale[11:] + 1e-30).all()
+    # 4. the mean planes (geometric + view-direction terms): the gradient
+    #    implied by m against the oracle, relative L2 per tensor
+    g_mean = (md_h[0:3, :n].astype(np.float64) - 0.9 * m0[0:3, :n]) / 0.1
+    for k in range(3):
+        assert rel_l2(g_mean[k, ci], grad[k, ci]) <= GRAD_TOL, k
 
 
 # ---------------------------------------------------------------------------
