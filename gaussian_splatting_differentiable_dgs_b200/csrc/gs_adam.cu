@@ -342,127 +342,213 @@ __device__ __forceinline__ void adam_vals(float& p, float& m, float& v, float g,
   p = fmaf(-a.step, __fdividef(m, fmaf(sqrtf(v), a.rsbc2, a.eps)), p);
 }
 
-// Fused path, stage 2: one thread per Gaussian streams its planes once:
-// SH planes (gradient = dL/dcolour * Y_k(d), plus the view-direction term
-// accumulated for the mean), then log-scale, quaternion, logit (compact
-// geometric gradients) and the mean.  Non-candidates get g = 0.  Loads of a
-// group of planes are issued before any of its stores.
+// Fused path, stage 2, staged through shared memory: a CTA owns kThreads
+// consecutive Gaussians (one per compute thread).  Each (plane, array)
+// segment of p, m, v is a contiguous run of kThreads floats, moved by bulk
+// asynchronous copies into a ring of kStages stages (one group of up to 4
+// planes x 3 arrays each).  A producer warp fills a stage (its loads
+// complete on the stage's "full" mbarrier); the 8 compute warps update it in
+// place and arrive on its "empty" mbarrier; the producer then writes the
+// group back with bulk stores and refills the stage once they have read it.
+// Groups: the SH planes by coefficient (3 planes), then log-scale,
+// quaternion, logit, and the mean last (it needs the view-direction term
+// summed over the SH planes).  Every wait is bounded; on expiry the CTA
+// flags GS_DEV_TIMEOUT, lets its own copies finish and exits.
+#ifndef GS_ADAM_STAGES
+#define GS_ADAM_STAGES 6
+#endif
+#ifndef GS_ADAM_CTA
+#define GS_ADAM_CTA 256
+#endif
+constexpr int kStages = GS_ADAM_STAGES;
+constexpr int kGroupPlanes = 4;
+constexpr int kAT = GS_ADAM_CTA;  // Gaussians (compute threads) per CTA
+constexpr int kComputeWarps = kAT / 32;
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 3)
-k_adam_fused(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v, int64_t n,
-             int64_t n_pad, BwdCam cam, const int32_t* __restrict__ slot_map,
-             const float4* __restrict__ rec, const float* __restrict__ g2d,
-             const double* __restrict__ g_mean, const float* __restrict__ g_rest, int64_t n_cand,
-             AdamK a) {
-  constexpr int KS = (D + 1) * (D + 1);
-  constexpr int GK = 2;  // SH coefficients per load group (6 planes)
-  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (i >= n) return;
-  const int32_t s = slot_map[i];
-  const bool cand = s >= 0;
-  const float mx = P[i], my = P[n_pad + i], mz = P[2 * n_pad + i];
+struct AdamGroups {
+  static constexpr int KS = (D + 1) * (D + 1);
+  static constexpr int N = KS + 4;
+  __device__ static int first(int g) {
+    return g < KS ? 11 + 3 * g : (g == KS ? 3 : g == KS + 1 ? 6 : g == KS + 2 ? 10 : 0);
+  }
+  __device__ static int count(int g) {
+    return g < KS ? 3 : (g == KS ? 3 : g == KS + 1 ? 4 : g == KS + 2 ? 1 : 3);
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAT + 32, 3)
+k_adam_stream(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v, int64_t n,
+              int64_t n_pad, BwdCam cam, const int32_t* __restrict__ slot_map,
+              const float4* __restrict__ rec, const float* __restrict__ g2d,
+              const double* __restrict__ g_mean, const float* __restrict__ g_rest,
+              int64_t n_cand, AdamK a, int32_t* dev_status) {
+  using G = AdamGroups<D>;
+  extern __shared__ __align__(128) float s_ring[];  // [kStages][3][kGroupPlanes][kAT]
+  __shared__ unsigned long long s_full[kStages], s_empty[kStages];
+  __shared__ int s_abort;
+  const int t = threadIdx.x;
+  const int64_t i0 = (int64_t)blockIdx.x * kAT;
+  const int cnt = (int)min((int64_t)kAT, n - i0);
+  const unsigned seg = (unsigned)(((cnt + 3) & ~3) * sizeof(float));  // <= n_pad - i0
+  auto slot_ptr = [&](int st, int aj, int pl) {
+    return s_ring + ((st * 3 + aj) * kGroupPlanes + pl) * kAT;
+  };
+  if (t == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&s_full[st], 1);
+      mbar_init(&s_empty[st], kComputeWarps);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (t >= kAT) {  // ---- producer warp (one lane) ----
+    if (t == kAT) {
+      float* arr[3] = {P, m, v};
+      auto issue = [&](int g) {
+        const int st = g % kStages, f = G::first(g), c = G::count(g);
+        mbar_arrive_expect_tx(&s_full[st], 3u * c * seg);
+        for (int aj = 0; aj < 3; ++aj)
+          for (int pl = 0; pl < c; ++pl)
+            bulk_load(slot_ptr(st, aj, pl), arr[aj] + (int64_t)(f + pl) * n_pad + i0, seg,
+                      &s_full[st]);
+      };
+      auto writeback = [&](int g) {
+        const int st = g % kStages, f = G::first(g), c = G::count(g);
+        for (int aj = 0; aj < 3; ++aj)
+          for (int pl = 0; pl < c; ++pl)
+            bulk_store(arr[aj] + (int64_t)(f + pl) * n_pad + i0, slot_ptr(st, aj, pl), seg);
+        bulk_commit();
+      };
+      int issued = 0;
+      for (; issued < kStages && issued < G::N; ++issued) issue(issued);
+      bool ok = true;
+      for (int g = 0; g < G::N && ok; ++g) {
+        const int st = g % kStages;
+        if (!mbar_wait(&s_empty[st], (unsigned)((g / kStages) & 1)) ||
+            *(volatile int*)&s_abort) {
+          ok = false;
+          break;
+        }
+        writeback(g);
+        if (issued < G::N) {
+          bulk_wait_read_all();  // the stage's data have left for global memory
+          issue(issued++);
+        }
+      }
+      if (!ok) {
+        *(volatile int*)&s_abort = 1;
+        dev_flag(dev_status, GS_DEV_TIMEOUT);
+      }
+      bulk_wait_all();
+      if (!ok)  // loads still in flight (the latest of each stage) must land
+                // before the CTA's memory goes
+        for (int h = issued > kStages ? issued - kStages : 0; h < issued; ++h)
+          mbar_wait(&s_full[h % kStages], (unsigned)((h / kStages) & 1));
+    }
+    return;
+  }
+
+  // ---- compute warps: per-Gaussian state, read while the groups stream in
+  const int64_t i = i0 + t;
+  const int lane = t & 31;
+  const bool in = i < n;
+  const int32_t sl = in ? slot_map[i] : -1;
+  const bool cand = sl >= 0;
   double gc[3] = {0.0, 0.0, 0.0};
   double dx = 0.0, dy = 0.0, dz = 0.0, dn = 1.0;
+  double gm[3] = {0.0, 0.0, 0.0};
+  float gr[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) gr[k] = 0.f;
   if (cand) {
-    const float4 rgb = rec[3 * (int64_t)s + 2];
-    const float* g2 = g2d + 12 * (int64_t)s;
+    const float4 rgb = rec[3 * (int64_t)sl + 2];
+    const float* g2 = g2d + 12 * (int64_t)sl;
     gc[0] = rgb.x > 0.f ? (double)g2[6] : 0.0;
     gc[1] = rgb.y > 0.f ? (double)g2[7] : 0.0;
     gc[2] = rgb.z > 0.f ? (double)g2[8] : 0.0;
-    dx = (double)mx - cam.campos[0];
-    dy = (double)my - cam.campos[1];
-    dz = (double)mz - cam.campos[2];
+    dx = (double)P[i] - cam.campos[0];
+    dy = (double)P[n_pad + i] - cam.campos[1];
+    dz = (double)P[2 * n_pad + i] - cam.campos[2];
     dn = sqrt(dx * dx + dy * dy + dz * dz);
     dx /= dn; dy /= dn; dz /= dn;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) gm[k] = g_mean[(int64_t)k * n_cand + sl];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) gr[k] = g_rest[(int64_t)k * n_cand + sl];
   }
-  // SH planes: gradient dL/dcolour * Y_k(d); the view-direction term of the
-  // mean in fp64 (the tangential projection below cancels)
   double ddx = 0.0, ddy = 0.0, ddz = 0.0;
 #pragma unroll 1
-  for (int k0 = 0; k0 < KS; k0 += GK) {
-    float pv[GK][3], mv[GK][3], vv[GK][3];
+  for (int g = 0; g < G::N; ++g) {
+    const int st = g % kStages;
+    const bool got = mbar_wait(&s_full[st], (unsigned)((g / kStages) & 1));
+    if (!got || *(volatile int*)&s_abort) {
+      *(volatile int*)&s_abort = 1;
+      break;
+    }
+    if (in) {
+      float* pp = slot_ptr(st, 0, 0) + t;
+      float* mp = slot_ptr(st, 1, 0) + t;
+      float* vp = slot_ptr(st, 2, 0) + t;
+      if (g < G::KS) {
+        float pv[3], mv[3], vv[3];
 #pragma unroll
-    for (int kk = 0; kk < GK; ++kk)
+        for (int ch = 0; ch < 3; ++ch) {
+          pv[ch] = pp[ch * kAT];
+          mv[ch] = mp[ch * kAT];
+          vv[ch] = vp[ch * kAT];
+        }
+        float gy[3] = {0.f, 0.f, 0.f};
+        if (cand) {
+          double Y, Yx, Yy, Yz;
+          sh_term(g, dx, dy, dz, Y, Yx, Yy, Yz);
+          const double w = gc[0] * pv[0] + gc[1] * pv[1] + gc[2] * pv[2];
+          ddx = fma(w, Yx, ddx);
+          ddy = fma(w, Yy, ddy);
+          ddz = fma(w, Yz, ddz);
 #pragma unroll
-      for (int ch = 0; ch < 3; ++ch) {
-        if (k0 + kk >= KS) continue;
-        const int64_t idx = (int64_t)(11 + 3 * (k0 + kk) + ch) * n_pad + i;
-        pv[kk][ch] = P[idx];
-        mv[kk][ch] = m[idx];
-        vv[kk][ch] = v[idx];
+          for (int ch = 0; ch < 3; ++ch) gy[ch] = (float)(gc[ch] * Y);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) {
+          adam_vals(pv[ch], mv[ch], vv[ch], gy[ch], a);
+          pp[ch * kAT] = pv[ch];
+          mp[ch * kAT] = mv[ch];
+          vp[ch * kAT] = vv[ch];
+        }
+      } else {
+        const int f = G::first(g), c = G::count(g);
+        float gv[4];
+        if (f == 0) {  // the mean: geometric + view-direction terms
+          const double ddot = ddx * dx + ddy * dy + ddz * dz;
+          gv[0] = cand ? (float)(gm[0] + (ddx - dx * ddot) / dn) : 0.f;
+          gv[1] = cand ? (float)(gm[1] + (ddy - dy * ddot) / dn) : 0.f;
+          gv[2] = cand ? (float)(gm[2] + (ddz - dz * ddot) / dn) : 0.f;
+          gv[3] = 0.f;
+        } else if (f == 3) {  // log-scale
+          gv[0] = gr[0]; gv[1] = gr[1]; gv[2] = gr[2]; gv[3] = 0.f;
+        } else if (f == 6) {  // quaternion
+          gv[0] = gr[3]; gv[1] = gr[4]; gv[2] = gr[5]; gv[3] = gr[6];
+        } else {  // opacity logit
+          gv[0] = gr[7]; gv[1] = gv[2] = gv[3] = 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (k >= c) break;
+          float pk = pp[k * kAT], mk = mp[k * kAT], vk = vp[k * kAT];
+          adam_vals(pk, mk, vk, gv[k], a);
+          pp[k * kAT] = pk;
+          mp[k * kAT] = mk;
+          vp[k * kAT] = vk;
+        }
       }
-#pragma unroll
-    for (int kk = 0; kk < GK; ++kk) {
-      if (k0 + kk >= KS) continue;
-      float gy[3] = {0.f, 0.f, 0.f};
-      if (cand) {
-        double Y, Yx, Yy, Yz;
-        sh_term(k0 + kk, dx, dy, dz, Y, Yx, Yy, Yz);
-        const double w = gc[0] * pv[kk][0] + gc[1] * pv[kk][1] + gc[2] * pv[kk][2];
-        ddx = fma(w, Yx, ddx);
-        ddy = fma(w, Yy, ddy);
-        ddz = fma(w, Yz, ddz);
-#pragma unroll
-        for (int ch = 0; ch < 3; ++ch) gy[ch] = (float)(gc[ch] * Y);
-      }
-#pragma unroll
-      for (int ch = 0; ch < 3; ++ch) adam_vals(pv[kk][ch], mv[kk][ch], vv[kk][ch], gy[ch], a);
     }
-#pragma unroll
-    for (int kk = 0; kk < GK; ++kk)
-#pragma unroll
-      for (int ch = 0; ch < 3; ++ch) {
-        if (k0 + kk >= KS) continue;
-        const int64_t idx = (int64_t)(11 + 3 * (k0 + kk) + ch) * n_pad + i;
-        P[idx] = pv[kk][ch];
-        m[idx] = mv[kk][ch];
-        v[idx] = vv[kk][ch];
-      }
-  }
-  const double ddot = ddx * dx + ddy * dy + ddz * dz;
-  // geometric planes 3..10 in two groups of four, then the mean 0..2
-#pragma unroll 1
-  for (int k0 = 3; k0 < 11; k0 += 4) {
-    float pg[4], mg[4], vg[4];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int64_t idx = (int64_t)(k0 + kk) * n_pad + i;
-      pg[kk] = P[idx];
-      mg[kk] = m[idx];
-      vg[kk] = v[idx];
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const float gk = cand ? g_rest[(int64_t)(k0 + kk - 3) * n_cand + s] : 0.f;
-      adam_vals(pg[kk], mg[kk], vg[kk], gk, a);
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int64_t idx = (int64_t)(k0 + kk) * n_pad + i;
-      P[idx] = pg[kk];
-      m[idx] = mg[kk];
-      v[idx] = vg[kk];
-    }
-  }
-  float pg[3] = {mx, my, mz}, mg[3], vg[3];
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    mg[k] = m[(int64_t)k * n_pad + i];
-    vg[k] = v[(int64_t)k * n_pad + i];
-  }
-  const double d[3] = {dx, dy, dz}, ddv[3] = {ddx, ddy, ddz};
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    float gk = 0.f;
-    if (cand) gk = (float)(g_mean[(int64_t)k * n_cand + s] + (ddv[k] - d[k] * ddot) / dn);
-    adam_vals(pg[k], mg[k], vg[k], gk, a);
-  }
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    const int64_t idx = (int64_t)k * n_pad + i;
-    P[idx] = pg[k];
-    m[idx] = mg[k];
-    v[idx] = vg[k];
+    fence_proxy_async_smem();  // this thread's updates before the bulk stores
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s_empty[st]);
   }
 }
 
@@ -536,11 +622,24 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
         model->params, model->n_pad, c, n_cand, proj->cand_idx, rec, g2d, g_mean, g_rest);
     GS_LAUNCH_CHECK();
   }
-  const unsigned nb = (unsigned)((model->n + kThreads - 1) / kThreads);
-#define GS_ADAM_FUSED(DD)                                                                     \
-  k_adam_fused<DD><<<nb, kThreads, 0, s>>>(model->params, adam_m, adam_v, model->n,            \
-                                           model->n_pad, c, proj->slot, rec, g2d, g_mean, g_rest, \
-                                           n_cand, a)
+  // bulk copies want 16-byte aligned segments: planes of n_pad (a multiple
+  // of 4) floats, arrays 16-byte aligned
+  if ((model->n_pad & 3) || !aligned(model->params, 16) || !aligned(adam_m, 16) ||
+      !aligned(adam_v, 16))
+    return GS_ERR_ARG;
+  const size_t ring = sizeof(float) * kStages * 3 * kGroupPlanes * kAT;
+  const unsigned nbs = (unsigned)((model->n + kAT - 1) / kAT);
+#define GS_ADAM_FUSED(DD)                                                                       \
+  do {                                                                                          \
+    GS_TRY(cudaFuncSetAttribute(k_adam_stream<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                (int)ring));                                                    \
+    GS_TRY(cudaFuncSetAttribute(k_adam_stream<DD>,                                              \
+                                cudaFuncAttributePreferredSharedMemoryCarveout,                 \
+                                cudaSharedmemCarveoutMaxShared));                               \
+    k_adam_stream<DD><<<nbs, kAT + 32, ring, s>>>(model->params, adam_m, adam_v, model->n,      \
+                                                 model->n_pad, c, proj->slot, rec, g2d, g_mean, \
+                                                 g_rest, n_cand, a, dev_status);                \
+  } while (0)
   switch (D) {
     case 0: GS_ADAM_FUSED(0); break;
     case 1: GS_ADAM_FUSED(1); break;
