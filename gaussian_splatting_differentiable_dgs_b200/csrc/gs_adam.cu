@@ -631,11 +631,8 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
   const unsigned nbs = (unsigned)((model->n + kAT - 1) / kAT);
 #define GS_ADAM_FUSED(DD)                                                                       \
   do {                                                                                          \
-    GS_TRY(cudaFuncSetAttribute(k_adam_stream<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                (int)ring));                                                    \
-    GS_TRY(cudaFuncSetAttribute(k_adam_stream<DD>,                                              \
-                                cudaFuncAttributePreferredSharedMemoryCarveout,                 \
-                                cudaSharedmemCarveoutMaxShared));                               \
+    static std::atomic<unsigned long long> done{0};                                             \
+    GS_TRY(smem_attrs_once((const void*)k_adam_stream<DD>, (int)ring, &done));                  \
     k_adam_stream<DD><<<nbs, kAT + 32, ring, s>>>(model->params, adam_m, adam_v, model->n,      \
                                                  model->n_pad, c, proj->slot, rec, g2d, g_mean, \
                                                  g_rest, n_cand, a, dev_status);                \

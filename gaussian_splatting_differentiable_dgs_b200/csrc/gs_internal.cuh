@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stdint.h>
 
 #include "gs.h"
@@ -41,6 +43,24 @@ inline int64_t tiles_x(int32_t w) { return (w + kTile - 1) / kTile; }
 inline int64_t tiles_y(int32_t h) { return (h + kTile - 1) / kTile; }
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Sets a kernel's dynamic shared-memory limit and a maximal shared carveout
+// once per device (the attributes persist in the context): a call per launch
+// would cost host time on every step.  `done` is the call site's device
+// mask; `bytes` must not change between calls for the same kernel.
+inline cudaError_t smem_attrs_once(const void* fn, int bytes, std::atomic<unsigned long long>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done->load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done->fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Carves typed sub-buffers out of a caller workspace (256-byte aligned).
 struct Carver {

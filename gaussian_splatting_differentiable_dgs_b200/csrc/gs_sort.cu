@@ -603,18 +603,14 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
   const bool use32 = sizeof(K) == 4 && n <= (int64_t)INT32_MAX - kSortTile;
   // a shared-memory carveout large enough for several blocks per SM
   if (chained) {
-    GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    GS_TRY(cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                cudaSharedmemCarveoutMaxShared));
+    static std::atomic<unsigned long long> done{0};
+    GS_TRY(smem_attrs_once((const void*)k_onesweep<K>, (int)smem, &done));
   } else if (use32) {
-    GS_TRY(cudaFuncSetAttribute(k_downsweep32, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sizeof(DownSmem32)));
-    GS_TRY(cudaFuncSetAttribute(k_downsweep32, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                cudaSharedmemCarveoutMaxShared));
+    static std::atomic<unsigned long long> done{0};
+    GS_TRY(smem_attrs_once((const void*)k_downsweep32, (int)sizeof(DownSmem32), &done));
   } else {
-    GS_TRY(cudaFuncSetAttribute(k_downsweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    GS_TRY(cudaFuncSetAttribute(k_downsweep<K>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                cudaSharedmemCarveoutMaxShared));
+    static std::atomic<unsigned long long> done{0};
+    GS_TRY(smem_attrs_once((const void*)k_downsweep<K>, (int)smem, &done));
   }
   const K* sk = first_k;
   const int32_t* sv = vals;
