@@ -152,17 +152,47 @@ __device__ __forceinline__ float4 alpha_box(const Staged& st) {
   return make_float4(st.gx - st.hx, st.gx + st.hx, st.gy - st.hy, st.gy + st.hy);
 }
 
-// Bit w set if the alpha box meets the pixel-centre box of warp w.
+// q(e) = s1 (ex + beta ey)^2 + s2 ey^2 at an offset e from the mean.
+__device__ __forceinline__ float q_at(float ex, float ey, float s1, float beta, float s2) {
+  const float t = fmaf(beta, ey, ex);
+  return fmaf(s1 * t, t, s2 * ey * ey);
+}
+
+// Bit w set if the record can reach alpha >= 1/255 at a pixel centre of warp
+// w: its alpha box meets the warp's pixel-centre rectangle, and the smallest
+// q over that rectangle stays below ln(255 o) plus a margin (1e-3 + 1e-4
+// |ln(255 o)|, about a thousand times the fp32 error of the per-pixel q).
+// q is convex, so its minimum over the rectangle is 0 when the mean lies
+// inside, else on an edge, where it has a closed form.  A cleared bit means
+// every pixel of the warp would skip the record, so culling by it changes
+// no result.
 template <int PPT>
-__device__ __forceinline__ unsigned warp_mask(const float4& b) {
+__device__ __forceinline__ unsigned warp_mask(const Staged& st) {
   using G = TileGeom<PPT>;
+  const float4 b = alpha_box(st);
+  const float lq = __logf(255.0f * st.opac);
+  const float qthr = lq + 1e-3f + 1e-4f * fabsf(lq);
+  const float s1 = st.s1, beta = st.beta, s2 = st.s2;
+  // on an edge ex = const, the best ey is k ex
+  const float k = -s1 * beta / fmaf(s1 * beta, beta, s2);
   unsigned m = 0;
 #pragma unroll
   for (int w = 0; w < G::NW; ++w) {
     const float x0 = (float)((w % G::BX) * G::BW) + 0.5f, x1 = x0 + (float)(G::BW - 1);
     const float y0 = (float)((w / G::BX) * G::BH) + 0.5f, y1 = y0 + (float)(G::BH - 1);
     const bool miss = (b.x > x1) | (b.y < x0) | (b.z > y1) | (b.w < y0);
-    m |= miss ? 0u : (1u << w);
+    // the rectangle relative to the mean (pixel - mean; q is even)
+    const float ex0 = x0 - st.gx, ex1 = x1 - st.gx, ey0 = y0 - st.gy, ey1 = y1 - st.gy;
+    const bool inside = (ex0 <= 0.f) & (ex1 >= 0.f) & (ey0 <= 0.f) & (ey1 >= 0.f);
+    float qmin = 0.f;
+    if (!inside) {
+      const float qa = q_at(ex0, fminf(fmaxf(k * ex0, ey0), ey1), s1, beta, s2);
+      const float qb = q_at(ex1, fminf(fmaxf(k * ex1, ey0), ey1), s1, beta, s2);
+      const float qc = q_at(fminf(fmaxf(-beta * ey0, ex0), ex1), ey0, s1, beta, s2);
+      const float qd = q_at(fminf(fmaxf(-beta * ey1, ex0), ex1), ey1, s1, beta, s2);
+      qmin = fminf(fminf(qa, qb), fminf(qc, qd));
+    }
+    m |= (miss || qmin > qthr) ? 0u : (1u << w);
   }
   return m;
 }
@@ -313,7 +343,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       cnt = min(NT, nh - hp);
       if (t < cnt) {
         const Staged st = stage_record(rec, s_hits[hp + t], tx, ty);
-        s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
+        s_mask[t] = (uint8_t)warp_mask<PPT>(st);
         sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
         sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
         sC[t] = st.b;
@@ -326,7 +356,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       const int64_t e = base + t;
       if (e < end) {
         const Staged st = stage_record(rec, vals[e], tx, ty);
-        s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
+        s_mask[t] = (uint8_t)warp_mask<PPT>(st);
         sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
         sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
         sC[t] = st.b;
@@ -581,7 +611,7 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     if (t < cnt) {
       const int pos = bend - 1 - t;
       const Staged st = stage_record(rec, vals[begin + pos], tx, ty);
-      s_mask[t] = (uint8_t)warp_mask<PPT>(alpha_box(st));
+      s_mask[t] = (uint8_t)warp_mask<PPT>(st);
       sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
       sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
       sC[t] = make_float4(st.b, 2.0f * st.s1, 2.0f * st.s2, __int_as_float(st.slot));
