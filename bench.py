@@ -30,16 +30,16 @@ METRIC = ("fwd+bwd+Adam step ms & Gaussian-tile intersections/s per B200; "
           "peak working set GiB")
 UNIT = "intersections/s"
 SM_COUNT, LANES_PER_SM = 148, 128
-# Algorithmic lane-ops per pixel-Gaussian pair.  Every evaluation (forward
-# and backward): dx, dy, t1 = dx + beta dy, two products, q (mul + fma),
-# exp2, o * G, the 0.99 clamp and the 1/255 test = 11.  A composited pair
-# (forward): 1 - alpha, T (1 - alpha), the T test, alpha T, three colour
-# fmas, the T update = 8.  A differentiated pair (backward): 1 - alpha and
-# its reciprocal, T_i, alpha T_i, three colour gradients, g . rgb (3),
-# dL/dalpha (2), the running sum S, the clamp test, dL/dq, dL/do, and the
-# geometric terms du (2), dv (3), da, db, dc (2 each) with 0.5 dq = 28.
-OPS_FWD_VISIT, OPS_FWD_KEPT = 11, 8
-OPS_BWD_VISIT, OPS_BWD_KEPT = 11, 28
+# Algorithmic issue work of the raster stages: E evaluations times k
+# lane-ops each.  E is the method's pixel-Gaussian evaluations: in the
+# forward, each pixel's tile list up to its stop (the whole list if it never
+# stops); in the backward, its entries before last.  The kernels evaluate
+# fewer (their exact warp culling skips pairs that cannot reach 1/255); the
+# forward's accounting variant counts E itself.  k per evaluation: forward
+# 16 (2 sub, 5 fma/mul for q, ex2 and its scale, the clamp, the test, a
+# 4-op blend), backward 40 (the forward's evaluation plus the reverse blend
+# and the 9 gradient terms).
+K_FWD, K_BWD = 16, 40
 
 
 def parse():
@@ -91,7 +91,8 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
                    (g2d, record, fp64 geometric scratch) + N*4 (slot map)
     (E_blk = block-list entries, R_blk = their reads over the Leaves, I =
     tile-list entries, C = candidates, N = Gaussians.)  The raster stages'
-    lane-ops are the accounting view's counters scaled to each view's I."""
+    lane-ops are E k (K_FWD, K_BWD) from the accounting view, scaled to each
+    view's I."""
     hbm = peaks["hbm_gbs"] * 1e9
     n, P = model.n, model.P
     k = len(stats)
@@ -400,14 +401,14 @@ def main():
     value = isect_all / (ms_max / 1e3)
 
     # ---- accounting step (untimed): work counters per launch -----------------
-    counters = torch.zeros(4, dtype=torch.int64, device="cuda")
+    counters = torch.zeros(6, dtype=torch.int64, device="cuda")
     acc_timing = {}
     v = view_of(a.warmup + a.steps)
     acc = stp.run_view(cams[v], targets[v], counters=counters, timing=acc_timing)
     torch.cuda.synchronize()
     cnt = [int(x) for x in counters.cpu()]
-    ops_fwd = cnt[0] * OPS_FWD_VISIT + cnt[1] * OPS_FWD_KEPT
-    ops_bwd = cnt[2] * OPS_BWD_VISIT + cnt[3] * OPS_BWD_KEPT
+    ops_fwd = cnt[2] * K_FWD
+    ops_bwd = cnt[3] * K_BWD
 
     peaks, peak_src = load_peaks()
     sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
@@ -509,8 +510,9 @@ def main():
             "leaves_per_view": statistics.mean(s.n_leaves for s in stats),
             "stage_ms_per_step": {s: round(per_step[s], 3) for s in STAGES},
             "stage_launches_per_step": {s: stage_n[s] / n_steps for s in STAGES},
-            "work": {"fwd_pairs_evaluated": cnt[0], "fwd_pairs_composited": cnt[1],
-                     "bwd_pairs_evaluated": cnt[2], "bwd_pairs_differentiated": cnt[3]},
+            "work": {"method_fwd_evaluations": cnt[2], "method_bwd_evaluations": cnt[3],
+                     "fwd_pairs_evaluated": cnt[0], "fwd_pairs_composited": cnt[1],
+                     "bwd_pairs_evaluated": cnt[4], "bwd_pairs_differentiated": cnt[5]},
             "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk,
         }

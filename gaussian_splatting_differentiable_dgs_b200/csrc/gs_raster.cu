@@ -272,6 +272,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   const float fpx = (float)wp.lx + 0.5f;
   float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
   int lastp[PPT];
+  int stopn[PPT];  // COUNT: 1-based list position of the stopping entry, 0 = none
   bool done[PPT], inside[PPT];
   unsigned n_vis = 0, n_kept = 0;
 #pragma unroll
@@ -283,6 +284,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     T[k] = 1.0f;
     Cr[k] = Cg[k] = Cb[k] = 0.0f;
     lastp[k] = 0;
+    stopn[k] = 0;
   }
   bool bad = false;
   for (int64_t base = begin;; base += NT) {
@@ -391,6 +393,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         const float Tn = __fmul_rn(T[k], __fsub_rn(1.0f, ev.alpha));
         if (Tn < kTMin) {
           done[k] = true;
+          if (COUNT) stopn[k] = posn;
           continue;
         }
         if (COUNT) ++n_kept;
@@ -405,11 +408,24 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     }
   }
   if (COUNT) {  // one atomic per warp: per-thread ones on one word serialise
+    // the method's evaluations: each pixel visits its tile's list up to its
+    // stop (or the whole list), and the backward revisits it up to last
+    unsigned long long e_f = 0, e_b = 0;
+#pragma unroll
+    for (int k = 0; k < PPT; ++k)
+      if (inside[k]) {
+        e_f += stopn[k] ? (unsigned long long)stopn[k] : (unsigned long long)(end - begin);
+        e_b += (unsigned long long)lastp[k];
+      }
     const unsigned long long a = warp_sum((unsigned long long)n_vis);
     const unsigned long long b = warp_sum((unsigned long long)n_kept);
+    const unsigned long long c = warp_sum(e_f);
+    const unsigned long long d = warp_sum(e_b);
     if ((t & 31) == 0) {
       atomicAdd(&px.counters[0], a);
       atomicAdd(&px.counters[1], b);
+      atomicAdd(&px.counters[2], c);
+      atomicAdd(&px.counters[3], d);
     }
   }
   if (BLK) {

@@ -152,14 +152,14 @@ class Stepper:
         uploaded before its forward); None renders only (no loss, backward or
         update).  leaves: tile rects overriding the planner.  timing: dict
         that receives (start, end) CUDA event pairs per stage (STAGES).
-        counters: device int64[4] work counters ([0:2] forward, [2:4]
+        counters: device int64[6] work counters ([0:4] forward, [4:6]
         backward)."""
         dev = self.device
         if target is None:
             backward = update = False
         clk = _Timer(timing)
-        cnt_f = counters[0:2] if counters is not None else None
-        cnt_b = counters[2:4] if counters is not None else None
+        cnt_f = counters[0:4] if counters is not None else None
+        cnt_b = counters[4:6] if counters is not None else None
         m = self.model
         W, H = cam.width, cam.height
         TW, TH = (W + 15) // 16, (H + 15) // 16

@@ -163,7 +163,11 @@ typedef struct gs_pixels {
   double norm;            /* 1 / (3 W H): whole-view normaliser */
   /* optional work counters (NULL = off): [0] += pixel-Gaussian pairs
    * evaluated, [1] += pairs composited (forward) / differentiated
-   * (backward).  Used to account the work of a launch. */
+   * (backward); the forward also adds [2] += the method's evaluations
+   * (each pixel's list entries up to its stop, or the whole list) and
+   * [3] += the sum of last (the backward's evaluations), so a forward
+   * needs 4 counters, a backward 2.  Used to account the work of a
+   * launch. */
   unsigned long long* counters;
 } gs_pixels;
 
