@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--binning", default="fused", choices=["fused", "expand", "sort"])
     ap.add_argument("--sweep", default=None,
                     help="comma-separated widths: resolution sweep, whole image vs bounded")
+    ap.add_argument("--schedules", action="store_true",
+                    help="schedule comparison: Leaves, 3x3 groups at 128 MiB, fixed 8x8 blocks")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
@@ -339,6 +341,8 @@ def main():
         return run_reference(a, rank, world)
     if a.sweep:
         return run_sweep(a)
+    if a.schedules:
+        return run_schedules(a)
 
     import torch
     torch.cuda.set_device(local)
@@ -589,6 +593,62 @@ def run_sweep(a):
     diffs = [r["l1_rel_diff"] for r in rows if "l1_rel_diff" in r]
     print(json.dumps({"sweep": "resolution", "summary": True, "max_l1_rel_diff": max(diffs),
                       "workload": workload_name(a) + ", camera 0 pose, fixed field of view"}))
+
+
+def run_schedules(a):
+    """Schedules of one pass over the views of the outdoor scene (defaults:
+    the scene at --gaussians, --width x --height, --views views):
+    (1) Leaves under --budget-mib, one Adam update per view; (2) 3x3 groups,
+    each with its own candidate projection, Leaves under 128 MiB, one update
+    per view; (3) a fixed 8x8 grid of blocks, one Leaf and one Adam update
+    per block (64 per view).  Each starts from the same parameters; the
+    targets (renders of the jittered copy) are made per view outside the
+    timed events.  One JSON line per schedule."""
+    import torch
+    from gaussian_splatting_differentiable_dgs_b200 import synth
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    torch.cuda.set_device(0)
+    scene, cams = synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
+                                      n_views=a.views)
+    jit = synth.jittered(scene, seed=1)
+    budget = int(a.budget_mib * (1 << 20))
+    plans = [("leaves", dict(budget=budget), None),
+             ("groups3x3_128MiB", dict(budget=128 << 20), (3, 3)),
+             ("blocks8x8", dict(budget=1 << 40), (8, 8))]
+    for name, kw, split in plans:
+        model = GaussianModel(scene.params, scene.n, scene.sh_degree)
+        stp = Stepper(model, **kw)
+        jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
+        renderer = Stepper(jm, budget=budget)
+        total_ms, losses, peak, leaves, updates0 = 0.0, [], 0, 0, model.step
+        for cam in cams:
+            target = renderer.render(cam)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            if split is None:
+                st = stp.run_view(cam, target)
+            elif name.startswith("groups"):
+                st = stp.run_view_grouped(cam, target, groups=split)
+            else:
+                st = stp.run_view_blocks(cam, target, blocks=split)
+            e1.record()
+            torch.cuda.synchronize()
+            stp.check()
+            total_ms += e0.elapsed_time(e1)
+            losses.append(stp.last_loss())
+            peak = max(peak, st.peak_ws_bytes)
+            leaves += st.n_leaves
+            del target
+        print(json.dumps({"schedule": name, "views": len(cams), "ms_per_view": total_ms / len(cams),
+                          "pass_s": total_ms / 1e3, "working_set_gib": peak / 2 ** 30,
+                          "mean_loss": float(np.mean(losses)),
+                          "adam_updates": model.step - updates0,
+                          "leaves_per_view": leaves / len(cams),
+                          "workload": workload_name(a)}), flush=True)
+        del stp, model, renderer, jm
+        torch.cuda.empty_cache()
 
 
 def run_reference(a, rank, world):

@@ -104,7 +104,8 @@ SYMBOLS = [
     "gs_bin_workspace_size", "gs_bin_tiles",
     "gs_block_sat_workspace_size", "gs_block_sat", "gs_bin_blocks_workspace_size",
     "gs_bin_blocks", "gs_expand_workspace_size", "gs_expand_tiles",
-    "gs_tile_ranges", "gs_raster_fwd_blocks", "gs_upload_crop",
+    "gs_tile_ranges", "gs_raster_fwd_blocks", "gs_upload_crop", "gs_project_region",
+    "gs_grad_accumulate",
     "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
     "gs_project_bwd", "gs_adam",
 ]
@@ -123,6 +124,9 @@ def _load():
         "gs_check": (i32, [p, p]),
         "gs_project_workspace_size": (sz, [i64, i32, i32]),
         "gs_project": (i32, [P(gs_model), P(gs_camera), u32, P(gs_proj), p, p, sz, p, p]),
+        "gs_project_region": (i32, [P(gs_model), P(gs_camera), u32, gs_rect, P(gs_proj), p, p, sz,
+                                    p, p]),
+        "gs_grad_accumulate": (i32, [p, i64, p, i64, i32, p, i64, p]),
         "gs_sort_workspace_size": (sz, [i64, i32, i32, i32]),
         "gs_sort_keys": (i32, [p, p, i64, i32, i32, p, sz, p, p]),
         "gs_sort_keys32": (i32, [p, p, p, i64, i32, i32, u32, p, sz, p, p]),
@@ -235,6 +239,19 @@ def gs_project(model: gs_model, cam: gs_camera, proj: gs_proj, tile_sat, ws, dev
     return _ok("gs_project", _L.gs_project(C.byref(model), C.byref(cam), flags, C.byref(proj),
                                            ptr(tile_sat), ptr(ws), ws.numel() * ws.element_size(),
                                            ptr(dev_status), _stream(stream)))
+
+
+def gs_project_region(model: gs_model, cam: gs_camera, region, proj: gs_proj, tile_sat, ws,
+                      dev_status, flags=0, stream=None):
+    return _ok("gs_project_region", _L.gs_project_region(
+        C.byref(model), C.byref(cam), flags, gs_rect(*[int(v) for v in region]), C.byref(proj),
+        ptr(tile_sat), ptr(ws), ws.numel() * ws.element_size(), ptr(dev_status), _stream(stream)))
+
+
+def gs_grad_accumulate(g3d, g3d_stride, cand_idx, n_cand, P, G, n_pad, stream=None):
+    return _ok("gs_grad_accumulate", _L.gs_grad_accumulate(ptr(g3d), g3d_stride, ptr(cand_idx),
+                                                           n_cand, P, ptr(G), n_pad,
+                                                           _stream(stream)))
 
 
 def gs_sort_workspace_size(n, key_bytes, begin_bit, end_bit) -> int:

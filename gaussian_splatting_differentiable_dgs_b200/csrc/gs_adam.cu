@@ -552,6 +552,20 @@ k_adam_stream(float* __restrict__ P, float* __restrict__ m, float* __restrict__ 
   }
 }
 
+// Dense gradient accumulation: G[plane][cand_idx[j]] += g3d[plane][j].  A
+// Gaussian is at most one candidate of a projection, so no two threads add
+// to one element.
+__global__ void __launch_bounds__(kThreads)
+k_grad_accumulate(const float* __restrict__ g3d, int64_t stride,
+                  const int32_t* __restrict__ cand_idx, int64_t n_cand, int nP,
+                  float* __restrict__ G, int64_t n_pad) {
+  const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (j >= n_cand) return;
+  const int64_t i = cand_idx[j];
+  for (int plane = 0; plane < nP; ++plane)
+    G[(int64_t)plane * n_pad + i] += g3d[(int64_t)plane * stride + j];
+}
+
 BwdCam make_cam(const gs_camera* cam) {
   BwdCam c;
   for (int k = 0; k < 9; ++k) c.R[k] = cam->R[k];
@@ -658,6 +672,18 @@ extern "C" gs_status gs_adam(float* params, float* m, float* v, const float* g, 
   if (!slot && g_stride < n) return GS_ERR_ARG;
   k_adam<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, to_stream(stream)>>>(
       params, m, v, g, g_stride, slot, n, n_pad, P, a);
+  GS_LAUNCH_CHECK();
+  return GS_OK;
+}
+
+extern "C" gs_status gs_grad_accumulate(const float* g3d, int64_t g3d_stride,
+                                        const int32_t* cand_idx, int64_t n_cand, int32_t P,
+                                        float* G, int64_t n_pad, gs_stream stream) {
+  if (n_cand < 0 || P <= 0 || n_pad < 0 || g3d_stride < n_cand) return GS_ERR_ARG;
+  if (n_cand == 0) return GS_OK;
+  if (!g3d || !cand_idx || !G) return GS_ERR_ARG;
+  k_grad_accumulate<<<(unsigned)((n_cand + kThreads - 1) / kThreads), kThreads, 0,
+                      to_stream(stream)>>>(g3d, g3d_stride, cand_idx, n_cand, P, G, n_pad);
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

@@ -27,6 +27,7 @@ struct ProjCam {
   double fx, fy, cx, cy, limx, limy;
   double campos[3];
   int32_t W, H, TW, TH;
+  int32_t RX0, RY0, RX1, RY1;  // tile region the rects are clipped to
 };
 
 // Real SH basis, degree <= 3: Y_0 = 1/(2 sqrt(pi)), band l = 1 ordered
@@ -73,9 +74,12 @@ struct ProjGeo {
 
 // Cull + geometry of Gaussian i from its 11 geometric planes; true if it is
 // a candidate.  The SH planes are read only for candidates (sh_colour).
+// `counted` is set once the Gaussian is a candidate of the full view (its
+// square tiles in the region then count towards the 3-sigma total, even if
+// its tight rect misses the region).
 __device__ __forceinline__ bool project_geometry(const float* __restrict__ P, int64_t n_pad,
                                                  int64_t i, const ProjCam& c, ProjGeo& o,
-                                                 bool& nonfinite) {
+                                                 bool& nonfinite, bool& counted) {
   const double x = P[i], y = P[n_pad + i], z = P[2 * n_pad + i];
   double tc[3];
 #pragma unroll
@@ -167,23 +171,29 @@ __device__ __forceinline__ bool project_geometry(const float* __restrict__ P, in
   const int64_t by0 = (int64_t)ceil((v - hy - 15.5) / kTile), by1 = (int64_t)floor((v + hy - 0.5) / kTile) + 1;
   const int64_t cx0 = rx0 > bx0 ? rx0 : bx0, cx1 = rx1 < bx1 ? rx1 : bx1;
   const int64_t cy0 = ry0 > by0 ? ry0 : by0, cy1 = ry1 < by1 ? ry1 : by1;
-  const int64_t x0 = cx0 < 0 ? 0 : (cx0 > c.TW ? c.TW : cx0);
-  const int64_t x1 = cx1 < 0 ? 0 : (cx1 > c.TW ? c.TW : cx1);
-  const int64_t y0 = cy0 < 0 ? 0 : (cy0 > c.TH ? c.TH : cy0);
-  const int64_t y1 = cy1 < 0 ? 0 : (cy1 > c.TH ? c.TH : cy1);
+  {  // a candidate of the full view: its tight rect meets the grid
+    const int64_t gx0 = cx0 < 0 ? 0 : cx0, gx1 = cx1 > c.TW ? c.TW : cx1;
+    const int64_t gy0 = cy0 < 0 ? 0 : cy0, gy1 = cy1 > c.TH ? c.TH : cy1;
+    if (gx0 >= gx1 || gy0 >= gy1) return false;
+  }
+  counted = true;
+  {
+    // tiles of the plain 3-sigma square within the region, for the metric
+    const int64_t sx0 = rx0 < c.RX0 ? c.RX0 : (rx0 > c.RX1 ? c.RX1 : rx0);
+    const int64_t sx1 = rx1 < c.RX0 ? c.RX0 : (rx1 > c.RX1 ? c.RX1 : rx1);
+    const int64_t sy0 = ry0 < c.RY0 ? c.RY0 : (ry0 > c.RY1 ? c.RY1 : ry0);
+    const int64_t sy1 = ry1 < c.RY0 ? c.RY0 : (ry1 > c.RY1 ? c.RY1 : ry1);
+    o.square_tiles = (sx1 > sx0 && sy1 > sy0) ? (sx1 - sx0) * (sy1 - sy0) : 0;
+  }
+  const int64_t x0 = cx0 < c.RX0 ? c.RX0 : (cx0 > c.RX1 ? c.RX1 : cx0);
+  const int64_t x1 = cx1 < c.RX0 ? c.RX0 : (cx1 > c.RX1 ? c.RX1 : cx1);
+  const int64_t y0 = cy0 < c.RY0 ? c.RY0 : (cy0 > c.RY1 ? c.RY1 : cy0);
+  const int64_t y1 = cy1 < c.RY0 ? c.RY0 : (cy1 > c.RY1 ? c.RY1 : cy1);
   if (x0 >= x1 || y0 >= y1) return false;
   o.x = x; o.y = y; o.z = z;
   o.u = u; o.v = v; o.hx = hx; o.hy = hy;
   o.c00 = c00; o.c01 = c01; o.c11 = c11; o.det = det; o.opac = opac; o.tz = tz;
   o.rect = make_short4((short)x0, (short)y0, (short)x1, (short)y1);
-  {
-    // tiles of the plain 3-sigma square (clamped), counted for the metric
-    const int64_t sx0 = rx0 < 0 ? 0 : (rx0 > c.TW ? c.TW : rx0);
-    const int64_t sx1 = rx1 < 0 ? 0 : (rx1 > c.TW ? c.TW : rx1);
-    const int64_t sy0 = ry0 < 0 ? 0 : (ry0 > c.TH ? c.TH : ry0);
-    const int64_t sy1 = ry1 < 0 ? 0 : (ry1 > c.TH ? c.TH : ry1);
-    o.square_tiles = (sx1 > sx0 && sy1 > sy0) ? (sx1 - sx0) * (sy1 - sy0) : 0;
-  }
 
   return true;
 }
@@ -241,10 +251,11 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
   const int64_t b = s_b;
   const int64_t i = b * kProjThreads + threadIdx.x;
   ProjGeo o;
-  bool nonfinite = false;
+  o.square_tiles = 0;
+  bool nonfinite = false, counted = false;
   // cull and geometry first, so the CTA's scan below waits only on the 11
   // geometric planes; the 48 SH planes are read after it, by candidates
-  const bool cand = i < n && project_geometry(params, n_pad, i, cam, o, nonfinite);
+  const bool cand = i < n && project_geometry(params, n_pad, i, cam, o, nonfinite, counted);
   if (nonfinite) dev_flag(dev_status, GS_DEV_NONFINITE);
   if (dense) {
     // every Gaussian keeps slot i; a culled one gets an empty rect, depth -1
@@ -275,7 +286,7 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
       if (i == n - 1) *n_cand = (int32_t)n;
     }
     if (square_isect) {  // every lane of the warp takes part
-      unsigned long long sq = cand ? (unsigned long long)o.square_tiles : 0ull;
+      unsigned long long sq = counted ? (unsigned long long)o.square_tiles : 0ull;
       sq = warp_sum(sq);
       if ((threadIdx.x & 31) == 0 && sq) atomicAdd(square_isect, sq);
     }
@@ -309,7 +320,7 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
   }
   if (b == n_blocks - 1 && threadIdx.x == 0) *n_cand = (int32_t)(s_prefix + total);
   if (square_isect) {
-    unsigned long long sq = (cand && fits) ? (unsigned long long)o.square_tiles : 0ull;
+    unsigned long long sq = counted ? (unsigned long long)o.square_tiles : 0ull;
     sq = warp_sum(sq);
     if ((threadIdx.x & 31) == 0 && sq) atomicAdd(square_isect, sq);
   }
@@ -438,6 +449,16 @@ extern "C" size_t gs_project_workspace_size(int64_t n, int32_t width, int32_t he
 extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uint32_t flags,
                                 const gs_proj* out, int64_t* tile_sat, void* ws, size_t ws_bytes,
                                 int32_t* dev_status, gs_stream stream) {
+  if (!cam || cam->width <= 0 || cam->height <= 0) return GS_ERR_ARG;
+  const gs_rect all{0, 0, (int32_t)tiles_x(cam->width), (int32_t)tiles_y(cam->height)};
+  return gs_project_region(model, cam, flags, all, out, tile_sat, ws, ws_bytes, dev_status,
+                           stream);
+}
+
+extern "C" gs_status gs_project_region(const gs_model* model, const gs_camera* cam,
+                                       uint32_t flags, gs_rect region, const gs_proj* out,
+                                       int64_t* tile_sat, void* ws, size_t ws_bytes,
+                                       int32_t* dev_status, gs_stream stream) {
   if (!model || !cam || !out || !tile_sat) return GS_ERR_ARG;
   if (flags & ~GS_PROJ_DENSE) return GS_ERR_UNSUPPORTED;
   const bool dense = (flags & GS_PROJ_DENSE) != 0;
@@ -465,6 +486,10 @@ extern "C" gs_status gs_project(const gs_model* model, const gs_camera* cam, uin
   for (int c = 0; c < 3; ++c)
     pc.campos[c] = -(pc.R[c] * pc.t[0] + pc.R[3 + c] * pc.t[1] + pc.R[6 + c] * pc.t[2]);
   pc.W = cam->width; pc.H = cam->height; pc.TW = (int32_t)TW; pc.TH = (int32_t)TH;
+  if (region.x0 < 0 || region.y0 < 0 || region.x1 <= region.x0 || region.y1 <= region.y0 ||
+      region.x1 > TW || region.y1 > TH)
+    return GS_ERR_ARG;
+  pc.RX0 = region.x0; pc.RY0 = region.y0; pc.RX1 = region.x1; pc.RY1 = region.y1;
 
   const int64_t nb = (model->n + kProjThreads - 1) / kProjThreads;
   // ticket, look-back words and the difference grid start at zero

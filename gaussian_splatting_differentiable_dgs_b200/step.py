@@ -61,6 +61,23 @@ class ViewStats:
     launches: int
 
 
+def _merge_stats(stats):
+    """Statistics of a view run as several regions."""
+    return ViewStats(
+        n_cand=sum(x.n_cand for x in stats), n_isect=sum(x.n_isect for x in stats),
+        n_isect_square=sum(x.n_isect_square for x in stats),
+        n_block_entries=sum(x.n_block_entries for x in stats),
+        n_block_reads=sum(x.n_block_reads for x in stats),
+        n_leaves=sum(x.n_leaves for x in stats),
+        leaves=np.concatenate([x.leaves for x in stats]),
+        leaf_isect=np.concatenate([x.leaf_isect for x in stats]),
+        leaf_bytes=np.concatenate([x.leaf_bytes for x in stats]),
+        over_budget=np.concatenate([x.over_budget for x in stats]),
+        peak_ws_bytes=max(x.peak_ws_bytes for x in stats),
+        arena_bytes=max(x.arena_bytes for x in stats),
+        launches=sum(x.launches for x in stats))
+
+
 class GaussianModel:
     """Parameters and Adam moments, planar [P][n_pad] fp32 on the device."""
 
@@ -146,14 +163,17 @@ class Stepper:
 
     # ------------------------------------------------------------------
     def run_view(self, cam, target, leaves=None, hooks=None, update=True, backward=True,
-                 timing=None, counters=None) -> ViewStats:
+                 timing=None, counters=None, region=None, grad_out=None) -> ViewStats:
         """One view.  target: [3][H][W] fp32, a device tensor (the whole view
         resident, read in place) or a pinned host tensor (each Leaf's crop is
         uploaded before its forward); None renders only (no loss, backward or
         update).  leaves: tile rects overriding the planner.  timing: dict
         that receives (start, end) CUDA event pairs per stage (STAGES).
         counters: device int64[6] work counters ([0:4] forward, [4:6]
-        backward)."""
+        backward).  region: tile rect (x0, y0, x1, y1) the step is restricted
+        to (its Gaussians projected, its Leaves planned; default the whole
+        grid).  grad_out: dense [P][n_pad] gradient the view's gradient is
+        added to instead of taking the Adam step."""
         dev = self.device
         if target is None:
             backward = update = False
@@ -188,7 +208,11 @@ class Stepper:
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
         tk = clk.tic("project")
         original = self.mode == "original"
-        B.gs_project(mod, camS, proj, sat, ws, st, flags=B.GS_PROJ_DENSE if original else 0)
+        pflags = B.GS_PROJ_DENSE if original else 0
+        if region is None:
+            B.gs_project(mod, camS, proj, sat, ws, st, flags=pflags)
+        else:
+            B.gs_project_region(mod, camS, region, proj, sat, ws, st, flags=pflags)
         # fused: per-block lists, each tile's list built inside the forward;
         # expand: per-block lists expanded into full tile lists per Leaf;
         # sort: per-Leaf (tile, candidate) entries sorted by tile
@@ -251,8 +275,18 @@ class Stepper:
         # ---- Leaf plan ------------------------------------------------------
         lm = B.gs_leaf_load_model(tile_bits, B.GS_BIN_EXPAND if expand else B.GS_BIN_SORT)
         if leaves is None and original:
-            leaves = [(0, 0, TW, TH)]
-        if leaves is None:
+            leaves = [tuple(region) if region is not None else (0, 0, TW, TH)]
+        if leaves is None and region is not None:
+            # plan inside the region: its own SAT (zero first row and column)
+            rx0, ry0, rx1, ry1 = (int(v) for v in region)
+            sub = (sat_np[ry0:ry1 + 1, rx0:rx1 + 1] - sat_np[ry0:ry1 + 1, rx0:rx0 + 1]
+                   - sat_np[ry0:ry0 + 1, rx0:rx1 + 1] + sat_np[ry0, rx0])
+            rw = min(16 * rx1, W) - 16 * rx0
+            rh = min(16 * ry1, H) - 16 * ry0
+            _, lv, li, lb, ov = B.gs_leaf_partition(sub, rx1 - rx0, ry1 - ry0, rw, rh, lm,
+                                                    self.budget)
+            lv = lv + np.array([rx0, ry0, rx0, ry0], np.int32)
+        elif leaves is None:
             _, lv, li, lb, ov = B.gs_leaf_partition(sat_np, TW, TH, W, H, lm, self.budget)
         else:
             lv = np.asarray(leaves, np.int32).reshape(-1, 4)
@@ -398,7 +432,16 @@ class Stepper:
             hooks.on_bwd(ctx)
 
         # ---- projection backward fused with ONE Adam update -----------------
-        if update:
+        if update and grad_out is not None:
+            # the view's gradient goes to the caller's dense sum
+            g3d = torch.empty(m.P * max(C, 1), dtype=torch.float32, device=dev)
+            tk = clk.tic("project_bwd")
+            B.gs_project_bwd(mod, camS, proj, C, g2d, g3d=g3d, g3d_stride=max(C, 1),
+                             dev_status=st)
+            B.gs_grad_accumulate(g3d, max(C, 1), cand_idx, C, m.P, grad_out, m.n_pad)
+            clk.toc(tk)
+            del g3d
+        elif update:
             m.step += 1
             if self.fuse_adam and not original:
                 geo = torch.empty(14 * max(C, 1), dtype=torch.float32, device=dev)
@@ -427,6 +470,55 @@ class Stepper:
                          leaf_isect=li, leaf_bytes=lb, over_budget=ov, peak_ws_bytes=int(peak),
                          arena_bytes=int(arena_bytes),
                          launches=B.gs_launch_counter() - launch0)
+
+    @staticmethod
+    def split_regions(TW, TH, gx, gy):
+        """gx x gy tile-aligned regions covering the grid, row by row."""
+        xs = [round(k * TW / gx) for k in range(gx + 1)]
+        ys = [round(k * TH / gy) for k in range(gy + 1)]
+        return [(xs[i], ys[j], xs[i + 1], ys[j + 1]) for j in range(gy) for i in range(gx)
+                if xs[i + 1] > xs[i] and ys[j + 1] > ys[j]]
+
+    def run_view_grouped(self, cam, target, groups=(3, 3), timing=None, hooks=None):
+        """One view in gx x gy groups (BoundedGS page, section 02, "finer
+        grouping", ablation F): each group projects only the Gaussians that
+        can touch it and plans its own Leaves; their gradients are summed into
+        one dense gradient (kept, like the Adam moments, for the model's
+        lifetime), then ONE Adam update.  Same image, loss and update as
+        run_view (the sums reorder)."""
+        m = self.model
+        TW, TH = (cam.width + 15) // 16, (cam.height + 15) // 16
+        if getattr(self, "_G", None) is None or self._G.shape != m.params.shape:
+            self._G = torch.zeros_like(m.params)
+        else:
+            self._G.zero_()
+        stats, loss = [], None
+        for r in self.split_regions(TW, TH, *groups):
+            st = self.run_view(cam, target, region=r, grad_out=self._G, timing=timing,
+                               hooks=hooks)
+            stats.append(st)
+            loss = self._last_loss if loss is None else loss + self._last_loss
+        m.step += 1
+        tk = _Timer(timing).tic("project_bwd")
+        B.gs_adam(m.params, m.m, m.v, self._G, m.n_pad, None, m.n, m.n_pad, m.P,
+                  self.adam_args(m.step))
+        _Timer(timing).toc(tk)
+        self._last_loss = loss
+        return _merge_stats(stats)
+
+    def run_view_blocks(self, cam, target, blocks=(8, 8), timing=None, hooks=None):
+        """The fixed-block schedule of the BoundedGS page (Figs. 5-6): the
+        view cut into a fixed bx x by grid, each block a step of its own with
+        its own Adam update.  Returns the merged statistics; the loss is the
+        sum of the blocks' losses."""
+        TW, TH = (cam.width + 15) // 16, (cam.height + 15) // 16
+        stats, loss = [], None
+        for r in self.split_regions(TW, TH, *blocks):
+            st = self.run_view(cam, target, region=r, timing=timing, hooks=hooks)
+            stats.append(st)
+            loss = self._last_loss if loss is None else loss + self._last_loss
+        self._last_loss = loss
+        return _merge_stats(stats)
 
     def render(self, cam) -> torch.Tensor:
         """Forward-only render of the whole view: [3][H][W] fp32 on the device."""

@@ -220,11 +220,22 @@ gs_status gs_check(int32_t* dev_status, gs_stream stream);
  * empty rect, depth -1 in its record and depth key 0xffffffff; the SAT and
  * all later stages skip it. */
 #define GS_PROJ_DENSE 1u
+/* gs_project_region: gs_project with every tile rect clipped to `region`
+ * (tile units, half-open, inside the grid); a Gaussian whose rect misses it
+ * is culled, the SAT and the 3-sigma count cover the region only.  The cull
+ * tests, positions and records are the full view's, so a pixel of the
+ * region gets the same list as with gs_project.  It serves the grouped and
+ * fixed-block schedules (BoundedGS page, section 02 "from rendering to full
+ * training" (F: finer grouping) and Figs. 5-6 (fixed blocks)). */
 size_t gs_project_workspace_size(int64_t n, int32_t width, int32_t height);
 gs_status gs_project(const gs_model* model, const gs_camera* cam,
                      uint32_t flags, const gs_proj* out, int64_t* tile_sat,
                      void* ws, size_t ws_bytes, int32_t* dev_status,
                      gs_stream stream);
+gs_status gs_project_region(const gs_model* model, const gs_camera* cam,
+                            uint32_t flags, gs_rect region, const gs_proj* out,
+                            int64_t* tile_sat, void* ws, size_t ws_bytes,
+                            int32_t* dev_status, gs_stream stream);
 
 /* ---- 2. radix sorts ------------------------------------------------------
  * Stable LSD radix sort of (key, value) pairs on key bits [begin_bit,
@@ -481,6 +492,16 @@ gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
                          float* adam_m, float* adam_v,
                          const gs_adam_args* fused, int32_t* dev_status,
                          gs_stream stream);
+
+/* gs_grad_accumulate: adds compact gradients g3d[P][g3d_stride] (column j =
+ * candidate j) into a dense gradient G[P][n_pad] at column cand_idx[j].  A
+ * Gaussian is at most one candidate of a projection, so this is a plain
+ * add.  It sums the groups of a grouped schedule into the view's gradient
+ * before its one Adam update (BoundedGS page, section 01: the whole view's
+ * gradient is summed, then one update). */
+gs_status gs_grad_accumulate(const float* g3d, int64_t g3d_stride,
+                             const int32_t* cand_idx, int64_t n_cand, int32_t P,
+                             float* G, int64_t n_pad, gs_stream stream);
 
 /* ---- 9. Adam -------------------------------------------------------------
  * m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;

@@ -782,3 +782,95 @@ def test_leaf_invariance_gpu(oracle_mod):
         assert loss == loss0
         for f in range(9):
             assert rel_l2(g[:, f], g0[:, f]) <= 1e-5
+
+
+# ---------------------------------------------------------------------------
+# region projection and the grouped / fixed-block schedules
+# ---------------------------------------------------------------------------
+
+def test_project_region_matches_full_projection():
+    """gs_project_region: the full view's candidates whose rect meets the
+    region, with the rect clipped to it and the same records."""
+    sc, cam = scene("hd")
+    b = B()
+    pb, sat_full, params = run_project(sc, cam)
+    C = int(pb.n_cand.item())
+    ci = pb.cand_idx[:C].cpu().numpy()
+    rect = pb.rect[:4 * C].cpu().numpy().reshape(-1, 4).astype(np.int64)
+    rec = pb.rec[:12 * C].cpu().numpy().reshape(-1, 12)
+    TW, TH = (cam.width + 15) // 16, (cam.height + 15) // 16
+    model = b.gs_model(sc.n, sc.n_pad, sc.sh_degree, 0, params.data_ptr())
+    for region in [(0, 0, TW, TH), (3, 5, 41, 30), (TW - 7, TH - 3, TW, TH), (10, 10, 11, 11)]:
+        x0, y0, x1, y1 = region
+        cr = np.stack([np.maximum(rect[:, 0], x0), np.maximum(rect[:, 1], y0),
+                       np.minimum(rect[:, 2], x1), np.minimum(rect[:, 3], y1)], 1)
+        keep = (cr[:, 2] > cr[:, 0]) & (cr[:, 3] > cr[:, 1])
+        pr = ProjBuffers(sc.n)
+        sat = torch.zeros((TH + 1) * (TW + 1), dtype=torch.int64, device="cuda")
+        ws = torch.empty(b.gs_project_workspace_size(sc.n, cam.width, cam.height),
+                         dtype=torch.uint8, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        b.gs_project_region(model, b.camera_struct(cam), region, pr.struct, sat, ws, st)
+        assert b.gs_check(st) == 0
+        Cr = int(pr.n_cand.item())
+        assert Cr == keep.sum()
+        assert (pr.cand_idx[:Cr].cpu().numpy() == ci[keep]).all()
+        assert (pr.rect[:4 * Cr].cpu().numpy().reshape(-1, 4) == cr[keep]).all()
+        got = pr.rec[:12 * Cr].cpu().numpy().reshape(-1, 12)
+        assert (got.view(np.uint32) == rec[keep].view(np.uint32)).all()
+        cnt = np.zeros((TH, TW), np.int64)
+        for a0, b0, a1, b1 in cr[keep]:
+            cnt[b0:b1, a0:a1] += 1
+        s = np.zeros((TH + 1, TW + 1), np.int64)
+        s[1:, 1:] = cnt.cumsum(0).cumsum(1)
+        assert (sat.cpu().numpy().reshape(TH + 1, TW + 1) == s).all()
+
+
+def test_grouped_step_matches_view():
+    """3x3 groups, each with its own projection and Leaves, one summed
+    gradient and one Adam update: the same image, last and loss as the view,
+    the same update up to summation order."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    tgt = torch.as_tensor(synth.random_image(cam.width, cam.height, 9) * 0.5).cuda()
+    outs = []
+    for grouped in (False, True):
+        model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+        stp = Stepper(model, budget=2 << 20)
+        cap = Capture(cam.width, cam.height)
+        if grouped:
+            stats = stp.run_view_grouped(cam, tgt, groups=(3, 3), hooks=cap)
+        else:
+            stats = stp.run_view(cam, tgt, hooks=cap)
+        stp.check()
+        assert model.step == 1
+        outs.append((stats, cap.img.copy(), cap.last.copy(), stp.last_loss(),
+                     model.params.cpu().numpy()))
+    (s0, i0, l0, loss0, p0), (s1, i1, l1, loss1, p1) = outs
+    assert (i0 == i1).all() and (l0 == l1).all()
+    assert abs(loss1 - loss0) <= 1e-12 * loss0
+    assert s1.n_isect == s0.n_isect and s1.n_isect_square == s0.n_isect_square
+    assert s1.n_cand >= s0.n_cand  # Gaussians across groups are candidates of each
+    # Adam moves a parameter by about lr; an atomic-order sign flip of a ~zero
+    # gradient by up to 2 lr
+    assert np.abs(p1 - p0).max() <= 2.1e-3
+    assert np.median(np.abs(p1 - p0)) <= 1e-7
+
+
+def test_fixed_block_schedule():
+    """Fixed 2x2 blocks, one Adam update each: with lr = 0 the blocks' losses
+    sum to the view's loss and the optimizer takes one step per block."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    tgt = torch.as_tensor(synth.random_image(cam.width, cam.height, 4) * 0.5).cuda()
+    model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+    stp = Stepper(model, budget=4 << 20, lr=0.0)
+    stp.run_view(cam, tgt)
+    loss_view = stp.last_loss()
+    model2 = GaussianModel(sc.params, sc.n, sc.sh_degree)
+    stp2 = Stepper(model2, budget=4 << 20, lr=0.0)
+    stats = stp2.run_view_blocks(cam, tgt, blocks=(2, 2))
+    stp2.check()
+    assert model2.step == 4
+    assert abs(stp2.last_loss() - loss_view) <= 1e-12 * loss_view
+    assert (model2.params.cpu().numpy() == sc.params).all()
