@@ -300,7 +300,7 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
   }
   __syncthreads();
   const int64_t slot = s_prefix + rank;
-  const bool fits = slot < capacity;  // false only after a timed-out look-back
+  const bool fits = slot < capacity;  // false beyond the caller's capacity (it retries)
   if (cand && !fits) dev_flag(dev_status, GS_DEV_BOUNDS);
   if (i < n) slot_map[i] = (cand && fits) ? (int32_t)slot : -1;
   if (cand && fits) {
@@ -468,7 +468,8 @@ extern "C" gs_status gs_project_region(const gs_model* model, const gs_camera* c
   if (cam->width <= 0 || cam->height <= 0 || !(cam->fx > 0) || !(cam->fy > 0)) return GS_ERR_ARG;
   const int64_t TW = tiles_x(cam->width), TH = tiles_y(cam->height);
   if (TW > 32767 || TH > 32767) return GS_ERR_UNSUPPORTED;
-  if (out->capacity < model->n || !out->n_cand) return GS_ERR_ARG;
+  if (out->capacity < 0 || !out->n_cand) return GS_ERR_ARG;
+  if ((flags & GS_PROJ_DENSE) && out->capacity < model->n) return GS_ERR_ARG;
   if (model->n > 0 && (!model->params || !out->cand_idx || !out->slot || !out->rec || !out->rect ||
                        !out->depth_key))
     return GS_ERR_ARG;

@@ -149,6 +149,7 @@ class Stepper:
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
         self._last_loss = None
         self._copy_stream = None
+        self._cap_hint = {}  # region -> candidate capacity for the next view
 
     def check(self):
         st = B.gs_check(self.dev_status)
@@ -193,26 +194,19 @@ class Stepper:
         launch0 = B.gs_launch_counter()
 
         # ---- projection (+ counts, SAT) ---------------------------------
+        # Candidate state is sized for the candidates, not the model: from
+        # the last count of this region plus 5 %; a view with more candidates
+        # than that is projected again with the exact count.
         n = m.n
-        cap = max(n, 1)
-        n_cand_d = torch.zeros(1, dtype=torch.int32, device=dev)
-        cand_idx = torch.empty(cap, dtype=torch.int32, device=dev)
-        slot = torch.empty(cap, dtype=torch.int32, device=dev)
-        rec = torch.empty(cap * 12, dtype=torch.float32, device=dev)
-        rect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
-        dkey = torch.empty(cap, dtype=torch.int32, device=dev)
-        sq_d = torch.zeros(1, dtype=torch.int64, device=dev)
-        proj = B.gs_proj(cap, n_cand_d.data_ptr(), cand_idx.data_ptr(), slot.data_ptr(),
-                         rec.data_ptr(), rect.data_ptr(), dkey.data_ptr(), sq_d.data_ptr())
+        original = self.mode == "original"
+        pflags = B.GS_PROJ_DENSE if original else 0
+        hint_key = tuple(region) if region is not None else None
+        hint = self._cap_hint.get(hint_key)
+        cap = max(n, 1) if (original or hint is None) else max(min(n, hint), 1)
+        slot = torch.empty(max(n, 1), dtype=torch.int32, device=dev)
         sat = torch.empty((TH + 1) * (TW + 1), dtype=torch.int64, device=dev)
         ws = torch.empty(B.gs_project_workspace_size(n, W, H), dtype=torch.uint8, device=dev)
         tk = clk.tic("project")
-        original = self.mode == "original"
-        pflags = B.GS_PROJ_DENSE if original else 0
-        if region is None:
-            B.gs_project(mod, camS, proj, sat, ws, st, flags=pflags)
-        else:
-            B.gs_project_region(mod, camS, region, proj, sat, ws, st, flags=pflags)
         # fused: per-block lists, each tile's list built inside the forward;
         # expand: per-block lists expanded into full tile lists per Leaf;
         # sort: per-Leaf (tile, candidate) entries sorted by tile
@@ -222,21 +216,43 @@ class Stepper:
             BW, BH = (TW + B.TILE_BLOCK - 1) // B.TILE_BLOCK, (TH + B.TILE_BLOCK - 1) // B.TILE_BLOCK
             bsat = torch.empty((BH + 1) * (BW + 1), dtype=torch.int64, device=dev)
             bws = torch.empty(B.gs_block_sat_workspace_size(TW, TH), dtype=torch.uint8, device=dev)
-            B.gs_block_sat(proj, TW, TH, bsat, bws, st)
-            del bws
-        clk.toc(tk)
-        del ws
-        if expand:
             bsat_h = torch.empty(bsat.shape, dtype=torch.int64, pin_memory=True)
-            bsat_h.copy_(bsat, non_blocking=True)
         sat_h = torch.empty(sat.shape, dtype=torch.int64, pin_memory=True)
         nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
         sq_h = torch.empty(1, dtype=torch.int64, pin_memory=True)
-        sat_h.copy_(sat, non_blocking=True)
-        nc_h.copy_(n_cand_d, non_blocking=True)
-        sq_h.copy_(sq_d, non_blocking=True)
-        torch.cuda.current_stream(dev).synchronize()   # the one sync per view
+        while True:
+            n_cand_d = torch.zeros(1, dtype=torch.int32, device=dev)
+            cand_idx = torch.empty(cap, dtype=torch.int32, device=dev)
+            rec = torch.empty(cap * 12, dtype=torch.float32, device=dev)
+            rect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
+            dkey = torch.empty(cap, dtype=torch.int32, device=dev)
+            sq_d = torch.zeros(1, dtype=torch.int64, device=dev)
+            proj = B.gs_proj(cap, n_cand_d.data_ptr(), cand_idx.data_ptr(), slot.data_ptr(),
+                             rec.data_ptr(), rect.data_ptr(), dkey.data_ptr(), sq_d.data_ptr())
+            if region is None:
+                B.gs_project(mod, camS, proj, sat, ws, st, flags=pflags)
+            else:
+                B.gs_project_region(mod, camS, region, proj, sat, ws, st, flags=pflags)
+            if expand:
+                B.gs_block_sat(proj, TW, TH, bsat, bws, st)
+                bsat_h.copy_(bsat, non_blocking=True)
+            sat_h.copy_(sat, non_blocking=True)
+            nc_h.copy_(n_cand_d, non_blocking=True)
+            sq_h.copy_(sq_d, non_blocking=True)
+            torch.cuda.current_stream(dev).synchronize()   # the one sync per view
+            if int(nc_h[0]) <= cap:
+                break
+            # more candidates than the capacity hint: the kernel skipped (and
+            # flagged) those beyond it; clear the flag and project again
+            B.gs_check(st)
+            cap = int(nc_h[0])
+        clk.toc(tk)
+        del ws
+        if expand:
+            del bws
         C = int(nc_h[0])
+        if not original:
+            self._cap_hint[hint_key] = C + C // 20 + 1024
         n_square = int(sq_h[0])
         sat_np = sat_h.numpy().reshape(TH + 1, TW + 1)
         ctx = dict(proj=proj, cand_idx=cand_idx, slot=slot, rec=rec, rect=rect, depth_key=dkey,

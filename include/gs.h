@@ -213,6 +213,9 @@ gs_status gs_check(int32_t* dev_status, gs_stream stream);
  * ascending index order (slot map in proj->slot).  Also writes the
  * (TH+1) x (TW+1) int64 summed-area table of per-tile intersection counts
  * (row 0 and column 0 zero) to `tile_sat`.
+ * proj->capacity may be below n: candidates beyond it are not written,
+ * GS_DEV_BOUNDS is set and *n_cand still receives the full count, so the
+ * caller can retry with that capacity (the dense layout needs n).
  * The projection arithmetic is fp64; records are rounded to fp32.
  * flags: 0, or GS_PROJ_DENSE: the whole-image ("Original") layout of the
  * BoundedGS page, Fig. A and the ablation's configuration A: every Gaussian

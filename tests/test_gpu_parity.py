@@ -874,3 +874,26 @@ def test_fixed_block_schedule():
     assert model2.step == 4
     assert abs(stp2.last_loss() - loss_view) <= 1e-12 * loss_view
     assert (model2.params.cpu().numpy() == sc.params).all()
+
+
+def test_candidate_capacity_retry():
+    """Candidate buffers sized from a hint below the view's count: the step
+    projects again with the exact count and gives the same result."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    tgt = torch.as_tensor(synth.random_image(cam.width, cam.height, 6) * 0.5).cuda()
+    outs = []
+    for hint in (None, 1000):
+        model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+        stp = Stepper(model, budget=4 << 20)
+        if hint is not None:
+            stp._cap_hint[None] = hint
+        cap = Capture(cam.width, cam.height)
+        stats = stp.run_view(cam, tgt, hooks=cap)
+        stp.check()
+        outs.append((stats.n_cand, cap.img.copy(), cap.last.copy(), stp.last_loss()))
+        # the next view of this region is sized from this count
+        assert stp._cap_hint[None] >= stats.n_cand
+    (c0, i0, l0, s0), (c1, i1, l1, s1) = outs
+    assert c0 == c1 > 1000
+    assert (i0 == i1).all() and (l0 == l1).all() and s0 == s1
