@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--binning", default="fused", choices=["fused", "expand", "sort"])
     ap.add_argument("--sweep", default=None,
                     help="comma-separated widths: resolution sweep, whole image vs bounded")
+    ap.add_argument("--skipgs", type=int, default=0,
+                    help="N training steps over the views with and without the SkipGS gate")
+    ap.add_argument("--skipgs-warmup", type=int, default=16)
     ap.add_argument("--schedules", action="store_true",
                     help="schedule comparison: Leaves, 3x3 groups at 128 MiB, fixed 8x8 blocks")
     ap.add_argument("--no-e2e", action="store_true")
@@ -343,6 +346,8 @@ def main():
         return run_sweep(a)
     if a.schedules:
         return run_schedules(a)
+    if a.skipgs:
+        return run_skipgs(a)
 
     import torch
     torch.cuda.set_device(local)
@@ -648,6 +653,50 @@ def run_schedules(a):
                           "leaves_per_view": leaves / len(cams),
                           "workload": workload_name(a)}), flush=True)
         del stp, model, renderer, jm
+        torch.cuda.empty_cache()
+
+
+def run_skipgs(a):
+    """`skipgs` training steps cycling over the views, once with every
+    backward and once behind the SkipGS gate (warm-up --skipgs-warmup
+    steps, beta 0.95, rho_lo 0.5), from the same parameters; the targets
+    are renders of the jittered copy.  One JSON line per run."""
+    import torch
+    from gaussian_splatting_differentiable_dgs_b200 import synth
+    from gaussian_splatting_differentiable_dgs_b200.skipgs import BackwardGate
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    torch.cuda.set_device(0)
+    scene, cams = synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
+                                      n_views=a.views)
+    jit = synth.jittered(scene, seed=1)
+    budget = int(a.budget_mib * (1 << 20))
+    jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
+    targets = [Stepper(jm, budget=budget).render(c) for c in cams]
+    del jm
+    for gated in (False, True):
+        model = GaussianModel(scene.params, scene.n, scene.sh_degree)
+        stp = Stepper(model, budget=budget)
+        gate = BackwardGate(warmup=a.skipgs_warmup) if gated else None
+        losses = []
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k in range(a.skipgs):
+            v = k % len(cams)
+            stp.run_view(cams[v], targets[v], gate=gate.decide_for(v) if gated else None)
+            losses.append(stp._last_loss)
+        e1.record()
+        torch.cuda.synchronize()
+        stp.check()
+        ms = e0.elapsed_time(e1) / a.skipgs
+        tail = [float(x.item()) for x in losses[-len(cams):]]
+        print(json.dumps({"schedule": "skipgs" if gated else "every_backward", "steps": a.skipgs,
+                          "ms_per_step": ms, "backward_steps": gate.b if gated else a.skipgs,
+                          "rho_min": gate.rho_min if gated else None,
+                          "mean_loss_last_pass": float(np.mean(tail)),
+                          "workload": workload_name(a)}), flush=True)
+        del stp, model
         torch.cuda.empty_cache()
 
 

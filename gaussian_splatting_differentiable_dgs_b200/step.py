@@ -164,7 +164,8 @@ class Stepper:
 
     # ------------------------------------------------------------------
     def run_view(self, cam, target, leaves=None, hooks=None, update=True, backward=True,
-                 timing=None, counters=None, region=None, grad_out=None) -> ViewStats:
+                 timing=None, counters=None, region=None, grad_out=None,
+                 gate=None) -> ViewStats:
         """One view.  target: [3][H][W] fp32, a device tensor (the whole view
         resident, read in place) or a pinned host tensor (each Leaf's crop is
         uploaded before its forward); None renders only (no loss, backward or
@@ -174,7 +175,9 @@ class Stepper:
         backward).  region: tile rect (x0, y0, x1, y1) the step is restricted
         to (its Gaussians projected, its Leaves planned; default the whole
         grid).  grad_out: dense [P][n_pad] gradient the view's gradient is
-        added to instead of taking the Adam step."""
+        added to instead of taking the Adam step.  gate: callable(loss) ->
+        bool asked with the view's forward loss (skipgs.BackwardGate); False
+        skips the backward and the update."""
         dev = self.device
         if target is None:
             backward = update = False
@@ -354,86 +357,105 @@ class Stepper:
             if self._copy_stream is None:
                 self._copy_stream = torch.cuda.Stream(device=dev)
             cs = self._copy_stream
-            up = [torch.cuda.Event() for _ in lv]
-            freed = [None, None]
-            main = torch.cuda.current_stream(dev)
 
-            def upload(k):
-                x_, y_, w_, h_ = rects[k]
-                if freed[k % 2] is not None:
-                    cs.wait_event(freed[k % 2])
-                else:
-                    cs.wait_stream(main)  # the buffers were allocated on the main stream
-                B.gs_upload_crop(target, x_, y_, w_, h_, crops[k % 2], stream=cs)
-                up[k].record(cs)
-
-            for k in range(min(2, len(lv))):
-                upload(k)
-        for li_k, (L, I) in enumerate(zip(lv, li)):
-            I = int(I)
-            sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
-            bufs, _ = _carve(arena, sizes)
-            keys = bufs[0].view(torch.int32)
-            vals = bufs[1].view(torch.int32)
-            ranges = bufs[2].view(torch.int64)
-            sort_ws = bufs[3]
-            img = bufs[4].view(torch.float32)
-            Tf = bufs[5].view(torch.float32)
-            last = bufs[6].view(torch.int32)
-            dL = bufs[7].view(torch.float32)
-            if resident_target:
-                # the whole view's target is read in place with its own pitch
-                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
-                              target_origin=(0, 0), target_pitch=W, target_plane=W * H,
-                              loss_tiles=loss_tiles, norm=norm, counters=cnt_f)
-            elif host_target:
-                crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
-                main.wait_event(up[li_k])
-                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
-                              target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm,
-                              counters=cnt_f)
-            else:
-                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
-            if fused:
-                B.gs_tile_ranges(sat, TW, TH, L, ranges)
-            elif expand:
-                tk = clk.tic("expand")
-                B.gs_expand_tiles(proj, bvals, branges, B.block_entries(bsat_np, L), L, TW, TH,
-                                  sat, I, vals, max(I, 1), ranges, bin_ws, st)
-                clk.toc(tk)
-            else:
-                tk = clk.tic("bin")
-                B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1),
-                               ranges, bin_ws, st)
-                clk.toc(tk)
-            lb_bits = B.local_tile_bits(L)
-            if not expand and I > 0 and lb_bits > 0:
-                tk = clk.tic("sort_tiles")
-                B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
-                clk.toc(tk)
-            tk = clk.tic("raster_fwd")
-            if fused:
-                B.gs_raster_fwd_blocks(proj, bvals, branges, L, camS, px, vals, max(I, 1), I,
-                                       ranges, st, self.raster_flags)
-            else:
-                B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
-            clk.toc(tk)
+        def leaf_pass(with_bwd):
+            """Every Leaf: lists, forward (+ L1) and, if with_bwd, backward."""
             if host_target:
-                ev = torch.cuda.Event()
-                ev.record(main)
-                freed[li_k % 2] = ev
-                if li_k + 2 < len(lv):
-                    upload(li_k + 2)
-            if hooks is not None and hasattr(hooks, "on_leaf"):
-                hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
-                                        ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
-                                        n_isect=I, px_rect=(px0, py0, pw, ph)))
-            if backward:
-                if cnt_b is not None:
-                    px.counters = cnt_b.data_ptr()
-                tk = clk.tic("raster_bwd")
-                B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
+                up = [torch.cuda.Event() for _ in lv]
+                freed = [None, None]
+                main = torch.cuda.current_stream(dev)
+
+                def upload(k):
+                    x_, y_, w_, h_ = rects[k]
+                    if freed[k % 2] is not None:
+                        cs.wait_event(freed[k % 2])
+                    else:
+                        cs.wait_stream(main)  # the buffers were allocated on the main stream
+                    B.gs_upload_crop(target, x_, y_, w_, h_, crops[k % 2], stream=cs)
+                    up[k].record(cs)
+
+                for k in range(min(2, len(lv))):
+                    upload(k)
+            for li_k, (L, I) in enumerate(zip(lv, li)):
+                I = int(I)
+                sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
+                bufs, _ = _carve(arena, sizes)
+                keys = bufs[0].view(torch.int32)
+                vals = bufs[1].view(torch.int32)
+                ranges = bufs[2].view(torch.int64)
+                sort_ws = bufs[3]
+                img = bufs[4].view(torch.float32)
+                Tf = bufs[5].view(torch.float32)
+                last = bufs[6].view(torch.int32)
+                dL = bufs[7].view(torch.float32)
+                if resident_target:
+                    # the whole view's target is read in place with its own pitch
+                    px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
+                                  target_origin=(0, 0), target_pitch=W, target_plane=W * H,
+                                  loss_tiles=loss_tiles, norm=norm, counters=cnt_f)
+                elif host_target:
+                    crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
+                    main.wait_event(up[li_k])
+                    px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
+                                  target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm,
+                                  counters=cnt_f)
+                else:
+                    px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
+                if fused:
+                    B.gs_tile_ranges(sat, TW, TH, L, ranges)
+                elif expand:
+                    tk = clk.tic("expand")
+                    B.gs_expand_tiles(proj, bvals, branges, B.block_entries(bsat_np, L), L, TW, TH,
+                                      sat, I, vals, max(I, 1), ranges, bin_ws, st)
+                    clk.toc(tk)
+                else:
+                    tk = clk.tic("bin")
+                    B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1),
+                                   ranges, bin_ws, st)
+                    clk.toc(tk)
+                lb_bits = B.local_tile_bits(L)
+                if not expand and I > 0 and lb_bits > 0:
+                    tk = clk.tic("sort_tiles")
+                    B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
+                    clk.toc(tk)
+                tk = clk.tic("raster_fwd")
+                if fused:
+                    B.gs_raster_fwd_blocks(proj, bvals, branges, L, camS, px, vals, max(I, 1), I,
+                                           ranges, st, self.raster_flags)
+                else:
+                    B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
                 clk.toc(tk)
+                if host_target:
+                    ev = torch.cuda.Event()
+                    ev.record(main)
+                    freed[li_k % 2] = ev
+                    if li_k + 2 < len(lv):
+                        upload(li_k + 2)
+                if hooks is not None and hasattr(hooks, "on_leaf"):
+                    hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
+                                            ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
+                                            n_isect=I, px_rect=(px0, py0, pw, ph)))
+                if with_bwd:
+                    if cnt_b is not None:
+                        px.counters = cnt_b.data_ptr()
+                    tk = clk.tic("raster_bwd")
+                    B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
+                    clk.toc(tk)
+
+        # SkipGS gate: the view's loss from a forward pass decides whether the
+        # backward and the update run (then the Leaves are rendered again
+        # with their backward; the projection and lists are reused)
+        if gate is not None and backward:
+            leaf_pass(False)
+            pre = torch.zeros(1, dtype=torch.float64, device=dev)
+            B.gs_loss_total(loss_tiles, T, pre)
+            if gate(float(pre.item())):
+                loss_tiles.zero_()
+                leaf_pass(True)
+            else:
+                backward = update = False
+        else:
+            leaf_pass(backward)
         if not original:
             del arena, bin_ws  # raster buffers released before projection backward
             if host_target:

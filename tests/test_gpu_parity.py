@@ -897,3 +897,41 @@ def test_candidate_capacity_retry():
     (c0, i0, l0, s0), (c1, i1, l1, s1) = outs
     assert c0 == c1 > 1000
     assert (i0 == i1).all() and (l0 == l1).all() and s0 == s1
+
+
+def test_gated_step():
+    """run_view with a backward gate: a skipped step leaves the parameters
+    and the optimizer untouched and reports the forward loss; an accepted
+    step equals the ungated one (the Leaves are rendered twice)."""
+    from gaussian_splatting_differentiable_dgs_b200.skipgs import BackwardGate
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    tgt = torch.as_tensor(synth.random_image(cam.width, cam.height, 3) * 0.5).cuda()
+    runs = {}
+    for mode in ("plain", "skip", "take"):
+        model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+        stp = Stepper(model, budget=3 << 20)
+        gate = None if mode == "plain" else (lambda loss, m=mode: m == "take")
+        stats = stp.run_view(cam, tgt, gate=gate)
+        stp.check()
+        runs[mode] = (stp.last_loss(), model.params.cpu().numpy(), model.step, stats.n_leaves)
+    lp, pp, sp, nl = runs["plain"]
+    ls, ps, ss, _ = runs["skip"]
+    lt, pt, st_, _ = runs["take"]
+    assert nl > 1
+    assert ls == lp and lt == lp
+    assert ss == 0 and (ps == sc.params).all()
+    assert st_ == sp == 1 and np.abs(pt - pp).max() <= 2.1e-3
+    assert np.median(np.abs(pt - pp)) <= 1e-7
+    # the SkipGS gate over a few steps: warm-up steps update, the rest follow the rule
+    model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+    stp = Stepper(model, budget=3 << 20)
+    g = BackwardGate(warmup=2)
+    took = []
+    for k in range(5):
+        before = model.params.clone()
+        stp.run_view(cam, tgt, gate=g.decide_for(0))
+        stp.check()
+        took.append(g.last[3])
+        assert bool((model.params != before).any()) == g.last[3]
+    assert took[:2] == [True, True] and g.b == sum(took) and model.step == g.b
