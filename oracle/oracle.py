@@ -20,6 +20,15 @@ Stages and their sources (page title, section):
   gradient back-propagation, atomic accumulation).
 * L1 loss over the whole view                -- BoundedGS, section 01: every
   Leaf keeps full-view supervision; the normaliser is the full image.
+* composite loss (1 - lambda) L1 + lambda (1 - SSIM), lambda = 0.2
+                                             -- SkipGS notes, "loss function
+  / training strategy".  SSIM is the structural similarity index of Wang,
+  Bovik, Sheikh and Simoncelli (IEEE TIP 2004) with its Gaussian window
+  (11 x 11, sigma 1.5) and constants C1 = (0.01)^2, C2 = (0.03)^2 for a
+  data range of 1 (readings: the pages name SSIM only).  Windows are
+  local to each Leaf's pixel rectangle, zero outside it (BoundedGS,
+  section 02: local SSIM windows differ from full-image ones at the
+  boundary); one Leaf covering the view is the full-image SSIM.
 * Leaf partition                             -- BoundedGS, section 01 (load
   from overlaps, pixels and buffer layout) and section 02, B -> C (split
   over-budget regions again).
@@ -254,6 +263,97 @@ def loss_l1(img, target, norm_count):
     return float(np.abs(d).sum() / norm_count), np.sign(d) / norm_count
 
 
+SSIM_RADIUS = 5
+SSIM_SIGMA = 1.5
+SSIM_C1 = 0.01 ** 2
+SSIM_C2 = 0.03 ** 2
+SSIM_LAMBDA = 0.2
+
+
+def ssim_window():
+    """The 1D factor g of the 11 x 11 Gaussian window w(i, j) = g(i) g(j):
+    g(k) proportional to exp(-k^2 / (2 sigma^2)), k = -5..5, sum 1."""
+    k = np.arange(-SSIM_RADIUS, SSIM_RADIUS + 1, dtype=np.float64)
+    g = np.exp(-k * k / (2.0 * SSIM_SIGMA ** 2))
+    return g / g.sum()
+
+
+def window_sum(img):
+    """Gaussian-weighted local sum of a [h][w] plane with zero outside it:
+    out[y, x] = sum_{i, j} w(i, j) img[y + i, x + j], i, j = -5..5, written
+    out as the 121 shifted, weighted copies of the plane."""
+    g = ssim_window()
+    R = SSIM_RADIUS
+    h, w = img.shape
+    pad = np.zeros((h + 2 * R, w + 2 * R))
+    pad[R:R + h, R:R + w] = img
+    out = np.zeros((h, w))
+    for i in range(2 * R + 1):
+        for j in range(2 * R + 1):
+            out += g[i] * g[j] * pad[i:i + h, j:j + w]
+    return out
+
+
+def ssim_moments(x, y):
+    """Local statistics of one channel pair: mu_x, mu_y, sigma_x^2,
+    sigma_y^2, sigma_xy (Wang et al. 2004, eq. 14-16 with the Gaussian
+    window)."""
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    mx, my = window_sum(x), window_sum(y)
+    sxx = window_sum(x * x) - mx * mx
+    syy = window_sum(y * y) - my * my
+    sxy = window_sum(x * y) - mx * my
+    return mx, my, sxx, syy, sxy
+
+
+def ssim_map(x, y):
+    """Per-pixel SSIM of [C][h][w] images (eq. 13 of Wang et al. with
+    C3 = C2 / 2): luminance (2 mu_x mu_y + C1) / (mu_x^2 + mu_y^2 + C1)
+    times contrast-structure (2 sigma_xy + C2) / (sigma_x^2 + sigma_y^2 + C2)."""
+    out = np.zeros(np.shape(x))
+    for c in range(out.shape[0]):
+        mx, my, sxx, syy, sxy = ssim_moments(x[c], y[c])
+        out[c] = ((2 * mx * my + SSIM_C1) * (2 * sxy + SSIM_C2)) / \
+                 ((mx * mx + my * my + SSIM_C1) * (sxx + syy + SSIM_C2))
+    return out
+
+
+def ssim_map_grad(x, y):
+    """d (sum of ssim_map(x, y)) / d x for [C][h][w] images.  S at pixel q
+    depends on x through the window sums m = W[x], e = W[x^2], f = W[x y];
+    with the partials of S in those (sigma_x^2 = e - m^2, sigma_xy =
+    f - m mu_y), the chain rule gives
+      dS_sum/dx_p = W[dS/dm](p) + 2 x_p W[dS/de](p) + y_p W[dS/df](p)
+    (the window is symmetric and zero outside the image, so the transposed
+    window sum is the window sum)."""
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    out = np.zeros(x.shape)
+    for c in range(x.shape[0]):
+        mx, my, sxx, syy, sxy = ssim_moments(x[c], y[c])
+        a = 2 * mx * my + SSIM_C1
+        b = 2 * sxy + SSIM_C2
+        cc = mx * mx + my * my + SSIM_C1
+        d = sxx + syy + SSIM_C2
+        S = a * b / (cc * d)
+        # total partials of S = a b / (cc d) in (m, e, f)
+        dS_dm = S * (2 * my / a - 2 * my / b - 2 * mx / cc + 2 * mx / d)
+        dS_de = -S / d
+        dS_df = 2 * S / b
+        out[c] = window_sum(dS_dm) + 2 * x[c] * window_sum(dS_de) + y[c] * window_sum(dS_df)
+    return out
+
+
+def loss_ssim(img, target, norm_count):
+    """SSIM term of one pixel rectangle (windows local to it):
+    L = sum (1 - S) / norm_count, and dL/dimg."""
+    img = np.asarray(img, np.float64)
+    target = np.asarray(target, np.float64)
+    S = ssim_map(img, target)
+    return float((1.0 - S).sum() / norm_count), -ssim_map_grad(img, target) / norm_count
+
+
 def adam(p, m, v, g, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, step=1):
     """One Adam step (bias-corrected), fp64; returns new (p, m, v)."""
     p = np.asarray(p, np.float64)
@@ -316,10 +416,13 @@ def render(params, n, sh_degree, cam):
 
 
 def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
-         lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, t=1):
+         lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, t=1, ssim_lambda=None):
     """One training step for one view: project, per-Leaf raster forward +
-    L1 + raster backward (summed over Leaves), projection backward, one
-    Adam update.  `leaves` is a list of tile rects; None = whole image."""
+    loss + raster backward (summed over Leaves), projection backward, one
+    Adam update.  `leaves` is a list of tile rects; None = whole image.
+    The loss is L1, or with `ssim_lambda` the composite
+    (1 - lambda) L1 + lambda (1 - SSIM), SSIM over each Leaf's pixel
+    rectangle (loss_ssim), both normalised by 3 W H."""
     W, H = cam.width, cam.height
     TW, TH = grid(cam)
     pr = project(params, n, sh_degree, cam)
@@ -345,8 +448,24 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
         valid = (fw["flags"] & P_INVALID) == 0
         tg = gather_tiles(tpad, tiles, TW, 3)
         d = np.where(valid[:, None, :], fw["img"] - tg, 0.0)
-        loss += float(np.abs(d).sum() / norm)
-        dL = np.sign(d) / norm
+        if ssim_lambda is None:
+            loss += float(np.abs(d).sum() / norm)
+            dL = np.sign(d) / norm
+        else:
+            lam = float(ssim_lambda)
+            loss += (1.0 - lam) * float(np.abs(d).sum() / norm)
+            dL = (1.0 - lam) * np.sign(d) / norm
+            # the Leaf's pixel rectangle, clipped to the image
+            px0, py0 = x0 * 16, y0 * 16
+            px1, py1 = min(x1 * 16, W), min(y1 * 16, H)
+            fimg = scatter_tiles(fw["img"], tiles, TW, TH, TW * 16, TH * 16, 3)
+            r_img = fimg[:, py0:py1, px0:px1]
+            r_tg = tpad[:, py0:py1, px0:px1]
+            ls, gs = loss_ssim(r_img, r_tg, norm)
+            loss += lam * ls
+            gpad = np.zeros((3, TH * 16, TW * 16))
+            gpad[:, py0:py1, px0:px1] = lam * gs
+            dL = dL + gather_tiles(gpad, tiles, TW, 3)
         raster_bwd(pr["rec"], TW, W, H, tiles, off, vals, dL, g2d)
         n_eval += int(fw["n_eval"][valid].sum())
         for j, tt in enumerate(tiles):
@@ -386,6 +505,20 @@ def decision_signature(params, n, sh_degree, cam, target):
     return h
 
 
-def loss_only(params, n, sh_degree, cam, target):
+def loss_only(params, n, sh_degree, cam, target, ssim_lambda=None, leaves=None):
+    """The view's loss from a full-image render: L1, or the composite loss
+    with SSIM windows local to each Leaf's pixel rectangle (as step)."""
     r = render(params, n, sh_degree, cam)
-    return float(np.abs(r["img"] - target).sum() / (3.0 * cam.width * cam.height))
+    norm = 3.0 * cam.width * cam.height
+    l1 = float(np.abs(r["img"] - target).sum() / norm)
+    if ssim_lambda is None:
+        return l1
+    TW, TH = grid(cam)
+    if leaves is None:
+        leaves = [(0, 0, TW, TH)]
+    ls = 0.0
+    for (x0, y0, x1, y1) in leaves:
+        sl = (slice(None), slice(y0 * 16, min(y1 * 16, cam.height)),
+              slice(x0 * 16, min(x1 * 16, cam.width)))
+        ls += loss_ssim(r["img"][sl], np.asarray(target)[sl], norm)[0]
+    return (1.0 - ssim_lambda) * l1 + ssim_lambda * ls

@@ -613,3 +613,156 @@ def test_leaf_invariance_oracle(oracle_mod):
         for a, b in [(0, 3), (3, 6), (6, 10), (10, 11), (11, st["grad"].shape[0])]:
             ga, gb = st["grad"][a:b], whole["grad"][a:b]
             assert np.linalg.norm(ga - gb) <= 1e-12 * np.linalg.norm(gb) + 1e-300
+
+
+# ---------------------------------------------------------------------------
+# SSIM term of the composite loss (structural similarity of Wang et al. 2004,
+# Gaussian window 11 x 11, sigma 1.5, zero outside the pixel rectangle)
+# ---------------------------------------------------------------------------
+def _interior(a, r=5):
+    return a[..., r:-r, r:-r]
+
+
+def test_ssim_window_sums_match_scipy(oracle_mod):
+    """The windowed sums are a zero-padded correlation with the 2D Gaussian
+    of sigma 1.5 truncated at radius 5, as scipy.ndimage computes it."""
+    from scipy import ndimage
+    O = oracle_mod
+    rng = np.random.default_rng(3)
+    x = rng.random((19, 27))
+    out = O.window_sum(x)
+    # scipy's own Gaussian filter (truncate = 5 / 1.5 gives radius 5), zero padding
+    ref = ndimage.gaussian_filter(x, 1.5, mode="constant", cval=0.0, truncate=5.0 / 1.5)
+    assert np.abs(out - ref).max() <= 1e-14
+    g = O.ssim_window()
+    assert len(g) == 11 and abs(g.sum() - 1.0) <= 1e-15 and np.allclose(g, g[::-1])
+
+
+def test_ssim_identical_images(oracle_mod):
+    O = oracle_mod
+    x = np.random.default_rng(4).random((3, 12, 17))
+    assert np.abs(O.ssim_map(x, x) - 1.0).max() <= 1e-12
+    assert np.abs(O.ssim_map_grad(x, x)).max() <= 1e-10
+    L, g = O.loss_ssim(x, x, 3 * 12 * 17)
+    assert abs(L) <= 1e-12
+
+
+def test_ssim_constant_images_closed_form(oracle_mod):
+    """Constant planes a, b: wherever the window lies inside the image the
+    variances vanish and S is the luminance term alone."""
+    O = oracle_mod
+    a, b = 0.3, 0.7
+    x = np.full((1, 15, 16), a)
+    y = np.full((1, 15, 16), b)
+    S = _interior(O.ssim_map(x, y))
+    assert np.abs(S - (2 * a * b + O.SSIM_C1) / (a * a + b * b + O.SSIM_C1)).max() <= 1e-12
+
+
+def test_ssim_special_structures(oracle_mod):
+    """With library window sums m = W[x], s = W[x^2] - m^2 (scipy), in the
+    interior: y = x + delta keeps the structure term at 1; y = 1 - x makes
+    sigma_xy = -sigma^2; y = k x scales the variances by k^2."""
+    from scipy import ndimage
+    O = oracle_mod
+    filt = lambda z: ndimage.gaussian_filter(z, 1.5, mode="constant", cval=0.0, truncate=5.0 / 1.5)
+    x = np.random.default_rng(5).uniform(0.2, 0.8, (1, 24, 25))
+    mu = _interior(filt(x[0]))
+    var = _interior(filt(x[0] ** 2)) - mu ** 2
+    C1, C2 = O.SSIM_C1, O.SSIM_C2
+    lum = lambda m1, m2: (2 * m1 * m2 + C1) / (m1 ** 2 + m2 ** 2 + C1)
+    d = 0.05
+    S = _interior(O.ssim_map(x, x + d))[0]
+    assert np.abs(S - lum(mu, mu + d)).max() <= 1e-10
+    S = _interior(O.ssim_map(x, 1.0 - x))[0]
+    assert np.abs(S - lum(mu, 1 - mu) * (C2 - 2 * var) / (2 * var + C2)).max() <= 1e-10
+    k = 0.6
+    S = _interior(O.ssim_map(x, k * x))[0]
+    cs = (2 * k * var + C2) / ((1 + k * k) * var + C2)
+    assert np.abs(S - lum(mu, k * mu) * cs).max() <= 1e-10
+
+
+def test_ssim_crop_interior_matches_full_image(oracle_mod):
+    """Local windows: SSIM over a crop agrees with the full image's at pixels
+    whose window lies inside the crop, and differs at the crop's edge."""
+    O = oracle_mod
+    rng = np.random.default_rng(6)
+    x, y = rng.random((2, 3, 40, 44))
+    full = O.ssim_map(x, y)
+    crop = O.ssim_map(x[:, 7:30, 9:37], y[:, 7:30, 9:37])
+    assert np.abs(_interior(crop) - _interior(full[:, 7:30, 9:37])).max() <= 1e-12
+    assert np.abs(crop[:, 0, :] - full[:, 7, 9:37]).max() > 1e-3
+
+
+def test_ssim_gradient_finite_differences(oracle_mod):
+    """The analytic gradient of sum(S) against central differences at every
+    pixel (borders included) of a small random pair."""
+    O = oracle_mod
+    rng = np.random.default_rng(7)
+    x, y = rng.uniform(0.1, 0.9, (2, 2, 9, 13))
+    g = O.ssim_map_grad(x, y)
+    h = 1e-6
+    fd = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        fd[idx] = (O.ssim_map(xp, y).sum() - O.ssim_map(xm, y).sum()) / (2 * h)
+    assert np.abs(g - fd).max() <= 1e-7 * max(1.0, np.abs(fd).max())
+
+
+def test_composite_loss_step_weights(oracle_mod):
+    """step(ssim_lambda=0) is the L1 step; for lambda in (0, 1) the loss is
+    the weighted sum of the L1 step's loss and the SSIM term computed by
+    loss_ssim on the rendered image (one Leaf = the whole image)."""
+    O = oracle_mod
+    sc, cams = synth.tiny_scene(n=60, width=45, height=37, sh_degree=1, seed=2)
+    cam = cams[0]
+    p64 = sc.params.astype(np.float64)
+    tgt = synth.random_image(cam.width, cam.height, 3).astype(np.float64)
+    r1 = O.step(p64, sc.n, sc.sh_degree, cam, tgt)
+    r0 = O.step(p64, sc.n, sc.sh_degree, cam, tgt, ssim_lambda=0.0)
+    # the oracle's threaded gradient sums vary in their last bits between runs
+    assert r0["loss"] == r1["loss"]
+    assert np.abs(r0["grad"] - r1["grad"]).max() <= 1e-14 * np.abs(r1["grad"]).max()
+    lam = 0.2
+    rs = O.step(p64, sc.n, sc.sh_degree, cam, tgt, ssim_lambda=lam)
+    ls, _ = O.loss_ssim(r1["img"], tgt, 3.0 * cam.width * cam.height)
+    assert abs(rs["loss"] - ((1 - lam) * r1["loss"] + lam * ls)) <= 1e-12
+    assert np.abs(rs["grad"] - r1["grad"]).max() > 1e-3 * np.abs(r1["grad"]).max()
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_composite_loss_gradient_finite_differences(oracle_mod, seed):
+    """The whole step's gradient of the composite loss, over two Leaves
+    (SSIM windows local to each), against central differences of the
+    rendered loss."""
+    O = oracle_mod
+    sc, cams = synth.tiny_scene(n=6, width=40, height=36, sh_degree=1, seed=seed)
+    cam = cams[0]
+    TW, TH = O.grid(cam)
+    leaves = [(0, 0, 1, TH), (1, 0, TW, TH)]
+    tgt = synth.random_image(cam.width, cam.height, seed + 9).astype(np.float64) * 0.6
+    st = O.step(sc.params, sc.n, 1, cam, tgt, leaves=leaves, ssim_lambda=O.SSIM_LAMBDA)
+    assert abs(st["loss"] - O.loss_only(sc.params.astype(np.float64), sc.n, 1, cam, tgt,
+                                        O.SSIM_LAMBDA, leaves)) <= 1e-12
+    grad = st["grad"]
+    base = sc.params.astype(np.float64)
+    sig0 = O.decision_signature(base, sc.n, 1, cam, tgt)
+    checked = skipped = 0
+    scale = np.abs(grad[:, :sc.n]).max()
+    for plane in range(base.shape[0]):
+        for i in range(sc.n):
+            h = 1e-6 * max(abs(base[plane, i]), 1e-1)
+            pp, pm = base.copy(), base.copy()
+            pp[plane, i] += h
+            pm[plane, i] -= h
+            if (O.decision_signature(pp, sc.n, 1, cam, tgt) != sig0 or
+                    O.decision_signature(pm, sc.n, 1, cam, tgt) != sig0):
+                skipped += 1
+                continue
+            fd = (O.loss_only(pp, sc.n, 1, cam, tgt, O.SSIM_LAMBDA, leaves) -
+                  O.loss_only(pm, sc.n, 1, cam, tgt, O.SSIM_LAMBDA, leaves)) / (2 * h)
+            an = grad[plane, i]
+            assert abs(fd - an) <= 1e-3 * abs(an) + 1e-7 * scale + 1e-13, (plane, i, fd, an)
+            checked += 1
+    assert checked > 0.8 * (checked + skipped), (checked, skipped)
