@@ -40,6 +40,12 @@ SM_COUNT, LANES_PER_SM = 148, 128
 # 4-op blend), backward 40 (the forward's evaluation plus the reverse blend
 # and the 9 gradient terms).
 K_FWD, K_BWD = 16, 40
+# SSIM term, lane-ops per pixel and channel with its gradient: the window
+# sums of x, y, x^2, y^2, x y (5 maps x 2 separable passes x 11 taps), the
+# three products, S and its three partials (about 30 operations, a division
+# counted as one), the window sums of the partials (3 x 2 x 11) and their
+# combination (4).
+K_SSIM = 110 + 3 + 30 + 66 + 4
 
 
 def parse():
@@ -55,6 +61,9 @@ def parse():
     ap.add_argument("--budget-mib", type=float, default=384)
     ap.add_argument("--raster-ppt", type=int, default=0)
     ap.add_argument("--binning", default="fused", choices=["fused", "expand", "sort"])
+    ap.add_argument("--loss", default="l1", choices=["l1", "l1_ssim"],
+                    help="l1: the L1 photometric loss; l1_ssim: (1 - 0.2) L1 + 0.2 (1 - SSIM) "
+                         "with SSIM windows local to each Leaf")
     ap.add_argument("--sweep", default=None,
                     help="comma-separated widths: resolution sweep, whole image vs bounded")
     ap.add_argument("--skipgs", type=int, default=0,
@@ -92,6 +101,8 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
                    its pixels saturate, so none are counted)
       raster_bwd   C*48 + pixels*20 (T, last, dL/dcolour) + C*48 (gradient
                    atomics)
+      ssim         pixels*48 (render and target read, dL/dcolour read and
+                   written; with --loss l1_ssim), lane-ops pixels*3*K_SSIM
       project_bwd  N*P*24 (p, m, v read and written) + C*(48 + 48 + 56*2)
                    (g2d, record, fp64 geometric scratch) + N*4 (slot map)
     (E_blk = block-list entries, R_blk = their reads over the Leaves, I =
@@ -119,6 +130,9 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
     }
     scale = I / max(acc.n_isect, 1)
     ops = {"raster_fwd": ops_fwd * scale, "raster_bwd": ops_bwd * scale}
+    if a.loss == "l1_ssim":
+        byt["ssim"] = px * 48
+        ops["ssim"] = px * 3 * K_SSIM
     stages, total = {}, 0.0
     for s, b in byt.items():
         t_hbm = b / hbm * 1e3
@@ -371,7 +385,8 @@ def main():
     torch.cuda.synchronize()
     del jm, js
     model = GaussianModel(scene.params, scene.n, scene.sh_degree)
-    stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt, binning=a.binning)
+    stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt, binning=a.binning,
+                  loss=a.loss)
     nv = len(cams)
     view_of = lambda k: rank_view(k, rank, nv)
 
@@ -483,7 +498,7 @@ def main():
 
     # ---- CPU baseline (rank 0, one GPU) ---------------------------------------
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu:
+    if rank == 0 and world == 1 and not a.no_cpu and a.loss == "l1":
         tg_host = {}
 
         def target_fn(v):
@@ -507,7 +522,7 @@ def main():
             "data": "synthetic (seeded generator; targets = renders of a jittered copy)",
             "config": {"workload": workload_name(a), "gaussians": a.gaussians, "sh_degree": 3,
                        "width": W, "height": H, "views": nv, "leaf_budget_mib": a.budget_mib,
-                       "binning": a.binning,
+                       "binning": a.binning, "loss": a.loss,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (4.25 GB of params + Adam moments "
                              "stream every step)"},

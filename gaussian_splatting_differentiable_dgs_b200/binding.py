@@ -106,7 +106,8 @@ SYMBOLS = [
     "gs_bin_blocks", "gs_expand_workspace_size", "gs_expand_tiles",
     "gs_tile_ranges", "gs_raster_fwd_blocks", "gs_upload_crop", "gs_project_region",
     "gs_grad_accumulate",
-    "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_raster_bwd",
+    "gs_raster_fwd", "gs_loss_l1", "gs_loss_total", "gs_ssim_workspace_size", "gs_loss_ssim",
+    "gs_raster_bwd",
     "gs_project_bwd", "gs_adam",
 ]
 
@@ -155,6 +156,8 @@ def _load():
                                        i64, i64, p, P(i64), u32, p, p]),
         "gs_loss_l1": (i32, [P(gs_pixels), gs_rect, P(gs_camera), p]),
         "gs_loss_total": (i32, [p, i64, p, p]),
+        "gs_ssim_workspace_size": (sz, [gs_rect, P(gs_camera)]),
+        "gs_loss_ssim": (i32, [P(gs_pixels), gs_rect, P(gs_camera), C.c_double, p, sz, p]),
         "gs_raster_bwd": (i32, [P(gs_proj), p, p, gs_rect, P(gs_camera), P(gs_pixels), p, u32, p,
                                 p]),
         "gs_project_bwd": (i32, [P(gs_model), P(gs_camera), P(gs_proj), i64, p, p, i64, p, p,
@@ -293,7 +296,9 @@ def gs_sort_keys32_noalloc(keys_in, keys, vals, n, begin_bit, end_bit, flags, de
 GS_PROJ_DENSE = 1
 GS_BIN_SORT = 0
 GS_BIN_EXPAND = 1
+GS_LOAD_SSIM = 0x100
 TILE_BLOCK = 8
+SSIM_LAMBDA = 0.2
 
 
 def gs_leaf_load_model(tile_bits, binning=GS_BIN_EXPAND) -> gs_load_model:
@@ -445,6 +450,19 @@ def gs_loss_l1(px: gs_pixels, leaf, cam: gs_camera, stream=None):
 
 def gs_loss_total(loss_tiles, n, loss, stream=None):
     return _ok("gs_loss_total", _L.gs_loss_total(ptr(loss_tiles), n, ptr(loss), _stream(stream)))
+
+
+def gs_ssim_workspace_size(leaf, cam: gs_camera) -> int:
+    return int(_L.gs_ssim_workspace_size(gs_rect(*[int(v) for v in leaf]), C.byref(cam)))
+
+
+def gs_loss_ssim(px: gs_pixels, leaf, cam: gs_camera, weight, ws=None, stream=None):
+    """ws: a device byte buffer of gs_ssim_workspace_size bytes, or None for
+    the loss only (no gradient)."""
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    return _ok("gs_loss_ssim", _L.gs_loss_ssim(C.byref(px), gs_rect(*[int(v) for v in leaf]),
+                                               C.byref(cam), float(weight), ptr(ws), nbytes,
+                                               _stream(stream)))
 
 
 def gs_raster_bwd(proj: gs_proj, vals, ranges, leaf, cam: gs_camera, px: gs_pixels, g2d,

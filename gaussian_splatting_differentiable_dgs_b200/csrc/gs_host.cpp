@@ -127,10 +127,13 @@ extern "C" gs_status gs_check(int32_t* dev_status, gs_stream stream) {
 // GS_BIN_EXPAND (gs_expand_tiles): intersections take their 32-bit value
 // only; fixed: the alignment of the Leaf's buffers.
 // Both: pixels take colour (12), T_final (4), last (4), target crop (12) and
-// dL/dcolour (12); tiles the int64 range pair.
+// dL/dcolour (12), with the SSIM term 36 more; tiles the int64 range pair.
 extern "C" gs_status gs_leaf_load_model(int32_t binning, int32_t tile_bits, gs_load_model* out) {
   if (!out || tile_bits < 0 || tile_bits > 32) return GS_ERR_ARG;
-  out->bytes_per_pixel = 44;
+  const bool ssim = (binning & GS_LOAD_SSIM) != 0;
+  binning &= ~GS_LOAD_SSIM;
+  // the SSIM term's workspace: three partials per pixel and channel
+  out->bytes_per_pixel = 44 + (ssim ? 36 : 0);
   out->bytes_per_tile = 16;
   out->align = 512;
   if (binning == GS_BIN_EXPAND) {

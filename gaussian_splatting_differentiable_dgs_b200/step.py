@@ -23,8 +23,8 @@ from . import binding as B
 
 DEFAULT_BUDGET = 384 << 20
 
-STAGES = ("project", "sort_depth", "bin", "sort_tiles", "expand", "raster_fwd", "raster_bwd",
-          "project_bwd")
+STAGES = ("project", "sort_depth", "bin", "sort_tiles", "expand", "raster_fwd", "ssim",
+          "raster_bwd", "project_bwd")
 
 
 def _carve(arena: torch.Tensor, sizes):
@@ -128,7 +128,8 @@ class Stepper:
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
-                 binning="fused", mode="bounded", device="cuda"):
+                 binning="fused", mode="bounded", loss="l1", ssim_lambda=B.SSIM_LAMBDA,
+                 device="cuda"):
         if binning not in ("fused", "expand", "sort"):
             raise ValueError(f"binning must be 'fused', 'expand' or 'sort', not {binning!r}")
         if mode not in ("bounded", "original"):
@@ -138,6 +139,13 @@ class Stepper:
         # original: the whole-image configuration A of the same page (dense
         # projection state, one whole-image Leaf whose raster buffers stay
         # alive through the projection backward, dense gradients)
+        if loss not in ("l1", "l1_ssim"):
+            raise ValueError(f"loss must be 'l1' or 'l1_ssim', not {loss!r}")
+        # l1: the L1 photometric loss; l1_ssim: the composite
+        # (1 - lambda) L1 + lambda (1 - SSIM) of 3DGS training (SkipGS notes,
+        # "loss function / training strategy"), SSIM windows local to each Leaf
+        self.loss = loss
+        self.ssim_lambda = float(ssim_lambda)
         self.mode = mode
         self.model = model
         self.binning = binning
@@ -292,7 +300,9 @@ class Stepper:
                        block_ranges=branges, n_block_entries=n_blk)
 
         # ---- Leaf plan ------------------------------------------------------
-        lm = B.gs_leaf_load_model(tile_bits, B.GS_BIN_EXPAND if expand else B.GS_BIN_SORT)
+        ssim = self.loss == "l1_ssim" and target is not None
+        lm = B.gs_leaf_load_model(tile_bits, (B.GS_BIN_EXPAND if expand else B.GS_BIN_SORT) |
+                                  (B.GS_LOAD_SSIM if ssim else 0))
         if leaves is None and original:
             leaves = [tuple(region) if region is not None else (0, 0, TW, TH)]
         if leaves is None and region is not None:
@@ -340,12 +350,15 @@ class Stepper:
                 lb_bits = B.local_tile_bits(L)
                 sizes = [4 * I, 4 * I, 16 * nt, B.gs_sort_workspace_size(I, 4, 0, lb_bits),
                          12 * npx, 4 * npx, 4 * npx, 12 * npx]
+            sizes.append(36 * npx if ssim else 0)  # the SSIM term's partials
             return sizes, (16 * x0, 16 * y0, pw, ph)
 
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
         arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
         norm = 1.0 / (3.0 * W * H)
+        # with the SSIM term the forward's L1 part carries (1 - lambda)
+        norm_l1 = (1.0 - self.ssim_lambda) * norm if ssim else norm
         # bounded supply of a host target: each Leaf's crop is uploaded on a
         # copy stream into one of two buffers, Leaf k + 2's upload waiting
         # until Leaf k's forward (the only reader) is done
@@ -392,13 +405,13 @@ class Stepper:
                     # the whole view's target is read in place with its own pitch
                     px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
                                   target_origin=(0, 0), target_pitch=W, target_plane=W * H,
-                                  loss_tiles=loss_tiles, norm=norm, counters=cnt_f)
+                                  loss_tiles=loss_tiles, norm=norm_l1, counters=cnt_f)
                 elif host_target:
                     crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
                     main.wait_event(up[li_k])
                     px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
-                                  target_origin=(px0, py0), loss_tiles=loss_tiles, norm=norm,
-                                  counters=cnt_f)
+                                  target_origin=(px0, py0), loss_tiles=loss_tiles,
+                                  norm=norm_l1, counters=cnt_f)
                 else:
                     px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
                 if fused:
@@ -425,6 +438,13 @@ class Stepper:
                 else:
                     B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
                 clk.toc(tk)
+                if ssim:
+                    # the Leaf's SSIM term: loss, and with the backward its
+                    # gradient added to the L1 part of dL
+                    tk = clk.tic("ssim")
+                    B.gs_loss_ssim(px, L, camS, self.ssim_lambda * norm,
+                                   bufs[8] if with_bwd else None)
+                    clk.toc(tk)
                 if host_target:
                     ev = torch.cuda.Event()
                     ev.record(main)

@@ -317,6 +317,8 @@ gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* keys,
  * of a Leaf's load). */
 #define GS_BIN_SORT 0
 #define GS_BIN_EXPAND 1
+/* or-ed into `binning`: the Leaf also holds gs_loss_ssim's workspace */
+#define GS_LOAD_SSIM 0x100
 gs_status gs_leaf_load_model(int32_t binning, int32_t tile_bits,
                              gs_load_model* out);
 gs_status gs_leaf_partition(const int64_t* sat_host, int32_t TW, int32_t TH,
@@ -464,6 +466,36 @@ gs_status gs_loss_l1(const gs_pixels* px, gs_rect leaf, const gs_camera* cam,
                      gs_stream stream);
 gs_status gs_loss_total(const float* loss_tiles, int64_t n, double* loss,
                         gs_stream stream);
+
+/* ---- 6b. SSIM term of the composite loss ---------------------------------
+ * The composite photometric loss (1 - lambda) L1 + lambda (1 - SSIM),
+ * lambda = 0.2 (SkipGS paper notes, "loss function / training strategy"),
+ * with SSIM windows local to the Leaf (BoundedGS page, section 02: local
+ * SSIM windows differ from full-image SSIM at their boundary).  SSIM is the
+ * structural similarity of Wang et al. (IEEE TIP 2004): over the Leaf's
+ * pixel rectangle R (its tiles clipped to the image), per channel, window
+ * sums W[.] with the 11 x 11 Gaussian window (sigma 1.5, normalised; zero
+ * outside R) of the render x = px->img and the target y = px->target give
+ * mu_x = W[x], mu_y = W[y], sigma_x^2 = W[x^2] - mu_x^2, sigma_y^2,
+ * sigma_xy = W[x y] - mu_x mu_y, and
+ *   S = (2 mu_x mu_y + C1)(2 sigma_xy + C2) /
+ *       ((mu_x^2 + mu_y^2 + C1)(sigma_x^2 + sigma_y^2 + C2)),
+ * C1 = 0.01^2, C2 = 0.03^2 (data range 1).
+ *
+ * gs_loss_ssim adds weight * sum over each tile's pixels and channels of
+ * (1 - S) to px->loss_tiles[tile] (global tile index, fixed summation
+ * order) and, when ws is not NULL, weight * d sum(1 - S) / dx to
+ * px->dL_dimg.  The L1 part comes first: gs_raster_fwd (or gs_loss_l1) with
+ * px->norm = (1 - lambda) / (3 W H) writes dL_dimg and loss_tiles; then
+ * weight = lambda / (3 W H).  ws (device, 16-byte aligned, at least
+ * gs_ssim_workspace_size(leaf, cam) bytes) holds the partials of S in
+ * (W[x], W[x^2], W[x y]) per pixel and channel between the two launches;
+ * ws = NULL computes the loss only (one launch).  px->img and px->target
+ * must cover R; px->loss_tiles must not be NULL.  fp32 arithmetic. */
+size_t gs_ssim_workspace_size(gs_rect leaf, const gs_camera* cam);
+gs_status gs_loss_ssim(const gs_pixels* px, gs_rect leaf, const gs_camera* cam,
+                       double weight, void* ws, size_t ws_bytes,
+                       gs_stream stream);
 
 /* ---- 7. raster backward --------------------------------------------------
  * Reverse blend over list positions last-1 .. 0 with the forward's skip
