@@ -10,8 +10,9 @@
 //    the Leaf's rectangle R); separable window sums (rows, then columns) of x, y,
 //    x^2, y^2, x y; per pixel S, the tile's sum of (1 - S), and the partials of S
 //    in the three window sums that depend on x (W[x], W[x^2], W[x y]).
-//  k_ssim_grad: the window sums of those partials (the window is symmetric and
-//    zero outside R, so the transposed sum is the window sum) combine into
+//  k_ssim_grad: the window sums of those partials (columns, then rows; the
+//    window is symmetric and zero outside R, so the transposed sum is the
+//    window sum) combine into
 //    d S_sum / dx_p = W[dS/dm](p) + 2 x_p W[dS/de](p) + y_p W[dS/df](p).
 // Both stages keep their inputs in registers along a row or a column (each
 // thread produces 8 or 16 outputs from 18 or 26 staged values), so shared
@@ -54,7 +55,7 @@ __device__ __forceinline__ bool in_rect(const SsimArgs& a, int x, int y) {
   return x >= a.X0 && x < a.X1 && y >= a.Y0 && y < a.Y1;
 }
 
-__global__ void __launch_bounds__(256) k_ssim_stats(SsimArgs a) {
+__global__ void __launch_bounds__(256, 4) k_ssim_stats(SsimArgs a) {
   __shared__ float s_in[2][3][kE][kXP];     // x, y of the tile and its halo
   __shared__ float s_h[3][5][kE][kHP];      // row sums of x, y, x^2, y^2, xy
   __shared__ float s_red[8];
@@ -66,16 +67,30 @@ __global__ void __launch_bounds__(256) k_ssim_stats(SsimArgs a) {
   const int tx = a.lx0 + blockIdx.x % a.lw, ty = a.ly0 + blockIdx.x / a.lw;
   const int ox = tx * kTile - kR, oy = ty * kTile - kR;
 
-  for (int i = t; i < 3 * kE * kE; i += 256) {
-    const int c = i / (kE * kE), r = (i / kE) % kE, col = i % kE;
-    const int gx = ox + col, gy = oy + r;
-    float xv = 0.0f, yv = 0.0f;
-    if (in_rect(a, gx, gy)) {
-      xv = a.img[(int64_t)(gy - a.iy0) * a.ipitch + (gx - a.ix0) + c * a.iplane];
-      yv = a.target[(int64_t)(gy - a.ty0) * a.tpitch + (gx - a.tx0) + c * a.tplane];
+  // staging: warp w takes rows w, w + 8, ...; lane = column of the halo tile
+  {
+    const int lane = t & 31, gx = ox + lane;
+    const bool colok = lane < kE && gx >= a.X0 && gx < a.X1;
+    for (int r = t >> 5; r < kE; r += 8) {
+      const int gy = oy + r;
+      float xv[3] = {0.0f, 0.0f, 0.0f}, yv[3] = {0.0f, 0.0f, 0.0f};
+      if (colok && gy >= a.Y0 && gy < a.Y1) {
+        const float* xp = a.img + (int64_t)(gy - a.iy0) * a.ipitch + (gx - a.ix0);
+        const float* yp = a.target + (int64_t)(gy - a.ty0) * a.tpitch + (gx - a.tx0);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          xv[c] = xp[c * a.iplane];
+          yv[c] = yp[c * a.tplane];
+        }
+      }
+      if (lane < kE) {
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          s_in[0][c][r][lane] = xv[c];
+          s_in[1][c][r][lane] = yv[c];
+        }
+      }
     }
-    s_in[0][c][r][col] = xv;
-    s_in[1][c][r][col] = yv;
   }
   __syncthreads();
 
@@ -158,9 +173,9 @@ __global__ void __launch_bounds__(256) k_ssim_stats(SsimArgs a) {
       lsum += 1.0f - S;
       if (a.ws) {
         // partials of S = A B / (C D) in W[x], W[x^2], W[x y] (sigma terms
-        // expanded), written without dividing by A or B
+        // expanded), written with the one reciprocal 1 / (C D)
         const float dm = (2.0f * m2 * (Bc - A) + 2.0f * m1 * S * (Cc - D)) * inv;
-        const float de = -S / D;
+        const float de = -S * Cc * inv;
         const float df = 2.0f * A * inv;
         a.ws[(3 * c + 0) * a.wplane + o] = dm;
         a.ws[(3 * c + 1) * a.wplane + o] = de;
@@ -178,34 +193,66 @@ __global__ void __launch_bounds__(256) k_ssim_stats(SsimArgs a) {
   }
 }
 
-constexpr int kGradIn = 9 * kE * kXP;     // staged partials with halo
-constexpr int kGradRow = 9 * kE * kHP;    // their row sums
-constexpr int kGradSmem = (kGradIn + kGradRow) * 4;
+constexpr int kGradIn = 9 * kE * kXP;       // staged partials with halo
+constexpr int kGradCol = 9 * kTile * kXP;    // their column sums (16 rows x 26)
+constexpr int kGradSmem = (kGradIn + kGradCol) * 4;
 
 __global__ void __launch_bounds__(256) k_ssim_grad(SsimArgs a) {
   extern __shared__ float smem[];
   float(*s_p)[kE][kXP] = reinterpret_cast<float(*)[kE][kXP]>(smem);
-  float(*s_h)[kE][kHP] = reinterpret_cast<float(*)[kE][kHP]>(smem + kGradIn);
+  float(*s_c)[kTile][kXP] = reinterpret_cast<float(*)[kTile][kXP]>(smem + kGradIn);
   float(*s_v)[kTile][kHP] = reinterpret_cast<float(*)[kTile][kHP]>(smem);
-  static_assert(9 * kTile * kHP <= kGradIn, "column sums must fit the staging area");
+  static_assert(9 * kTile * kHP <= kGradIn, "window sums must fit the staging area");
 
   const int t = threadIdx.x;
   const int tx = a.lx0 + blockIdx.x % a.lw, ty = a.ly0 + blockIdx.x / a.lw;
   const int ox = tx * kTile - kR, oy = ty * kTile - kR;
 
-  for (int i = t; i < 9 * kE * kE; i += 256) {
-    const int p = i / (kE * kE), r = (i / kE) % kE, col = i % kE;
-    const int gx = ox + col, gy = oy + r;
-    s_p[p][r][col] = in_rect(a, gx, gy)
-                         ? a.ws[p * a.wplane + (int64_t)(gy - a.Y0) * a.wpitch + (gx - a.X0)]
-                         : 0.0f;
+  {
+    const int lane = t & 31, gx = ox + lane;
+    const bool colok = lane < kE && gx >= a.X0 && gx < a.X1;
+    for (int r = t >> 5; r < kE; r += 8) {
+      const int gy = oy + r;
+      float v[9];
+#pragma unroll
+      for (int p = 0; p < 9; ++p) v[p] = 0.0f;
+      if (colok && gy >= a.Y0 && gy < a.Y1) {
+        const float* wp = a.ws + (int64_t)(gy - a.Y0) * a.wpitch + (gx - a.X0);
+#pragma unroll
+        for (int p = 0; p < 9; ++p) v[p] = wp[p * a.wplane];
+      }
+      if (lane < kE) {
+#pragma unroll
+        for (int p = 0; p < 9; ++p) s_p[p][r][lane] = v[p];
+      }
+    }
   }
   __syncthreads();
 
-  // rows: thread (plane, r) -> 16 outputs from 26 inputs
+  // columns first: thread (plane, col of 26) -> 16 outputs from 26 inputs
   if (t < 9 * kE) {
-    const int p = t / kE, r = t % kE;
-    const float* row = &s_p[p][r][0];
+    const int p = t / kE, col = t % kE;
+    float acc[kTile];
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kE; ++k) {
+      const float v = s_p[p][k][col];
+#pragma unroll
+      for (int i = 0; i < kTile; ++i) {
+        const int tap = k - i;
+        if (tap >= 0 && tap < kN) acc[i] = fmaf(a.g[tap], v, acc[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) s_c[p][i][col] = acc[i];
+  }
+  __syncthreads();
+
+  // rows: thread (plane, row) -> 16 outputs from 26 column sums
+  if (t < 9 * kTile) {
+    const int p = t >> 4, r = t & 15;
+    const float* row = &s_c[p][r][0];
     float acc[kTile];
 #pragma unroll
     for (int j = 0; j < kTile; ++j) acc[j] = 0.0f;
@@ -219,27 +266,7 @@ __global__ void __launch_bounds__(256) k_ssim_grad(SsimArgs a) {
       }
     }
 #pragma unroll
-    for (int j = 0; j < kTile; ++j) s_h[p][r][j] = acc[j];
-  }
-  __syncthreads();
-
-  // columns: thread (plane, col) -> 16 outputs from 26 row sums
-  if (t < 9 * kTile) {
-    const int p = t >> 4, col = t & 15;
-    float acc[kTile];
-#pragma unroll
-    for (int i = 0; i < kTile; ++i) acc[i] = 0.0f;
-#pragma unroll
-    for (int k = 0; k < kE; ++k) {
-      const float v = s_h[p][k][col];
-#pragma unroll
-      for (int i = 0; i < kTile; ++i) {
-        const int tap = k - i;
-        if (tap >= 0 && tap < kN) acc[i] = fmaf(a.g[tap], v, acc[i]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kTile; ++i) s_v[p][i][col] = acc[i];
+    for (int j = 0; j < kTile; ++j) s_v[p][r][j] = acc[j];
   }
   __syncthreads();
 
