@@ -258,6 +258,12 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 }
 
 // the bulk stores committed so far are complete
+// hint: bring [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple of
+// 16); completes asynchronously, nothing waits on it
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }

@@ -21,6 +21,9 @@ namespace gs {
 namespace {
 
 constexpr int kProjThreads = 256;
+// blocks between a block and the one whose geometric planes it prefetches:
+// about one wave of resident blocks (148 SMs x 3)
+constexpr int kProjAhead = 444;
 
 struct ProjCam {
   double R[9], t[3];
@@ -242,7 +245,8 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
           short4* __restrict__ rect, uint32_t* __restrict__ depth_key, int32_t* __restrict__ diff,
           unsigned long long* __restrict__ lb, unsigned int* __restrict__ ticket,
           int32_t* __restrict__ n_cand, int64_t n_blocks, int64_t capacity,
-          unsigned long long* __restrict__ square_isect, bool dense, int32_t* dev_status) {
+          unsigned long long* __restrict__ square_isect, bool dense, bool prefetch,
+          int32_t* dev_status) {
   __shared__ unsigned int s_b;
   __shared__ int s_scan[kProjThreads / 32 + 1];
   __shared__ long long s_prefix;
@@ -250,6 +254,19 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
   __syncthreads();
   const int64_t b = s_b;
   const int64_t i = b * kProjThreads + threadIdx.x;
+  // the block's SH segments (1 KB per plane) head for L2 while the geometry,
+  // the scan and the look-back run; the geometric planes of the block one
+  // wave ahead likewise
+  constexpr int kSH = 3 * (D + 1) * (D + 1);
+  if (prefetch && threadIdx.x < kSH + 11) {
+    const int64_t blk = threadIdx.x < kSH ? b : b + kProjAhead;
+    const int plane = threadIdx.x < kSH ? 11 + threadIdx.x : threadIdx.x - kSH;
+    const int64_t first = blk * kProjThreads;
+    if (first < n) {
+      const int64_t cnt = n_pad - first < kProjThreads ? n_pad - first : kProjThreads;
+      bulk_prefetch_l2(params + (int64_t)plane * n_pad + first, (unsigned)(cnt * 4));
+    }
+  }
   ProjGeo o;
   o.square_tiles = 0;
   bool nonfinite = false, counted = false;
@@ -503,7 +520,7 @@ extern "C" gs_status gs_project_region(const gs_model* model, const gs_camera* c
       model->params, model->n, model->n_pad, pc, out->cand_idx, out->slot,                   \
       reinterpret_cast<float4*>(out->rec), reinterpret_cast<short4*>(out->rect), out->depth_key, \
       w.diff, w.lb, w.ticket, out->n_cand, nb, out->capacity, out->square_isect, dense,     \
-      dev_status)
+      aligned(model->params, 16), dev_status)
     switch (model->sh_degree) {
       case 0: GS_PROJ(0); break;
       case 1: GS_PROJ(1); break;
