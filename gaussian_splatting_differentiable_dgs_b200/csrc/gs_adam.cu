@@ -274,7 +274,8 @@ k_adam(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v,
 // the sum may cancel), then float rest[8][C] for planes 3..10 (log-scale,
 // quaternion, logit).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads)
+// 4 CTAs per SM (64 registers): the chain is latency-bound on its gathers
+__global__ void __launch_bounds__(kThreads, 4)
 k_project_bwd_geo(const float* __restrict__ P, int64_t n_pad, BwdCam cam, int64_t n_cand,
                   const int32_t* __restrict__ cand_idx, const float4* __restrict__ rec,
                   const float* __restrict__ g2d, double* __restrict__ g_mean,
@@ -377,7 +378,11 @@ struct AdamGroups {
   }
 };
 
-template <int D>
+// GEO: the candidate's fp32 geometric chain runs in the compute warps'
+// prologue (its inputs are the candidate's own parameters, g2d row and
+// record), overlapping the first groups' loads; otherwise its results come
+// from k_project_bwd_geo through g_mean / g_rest.
+template <int D, bool GEO>
 __global__ void __launch_bounds__(kAT + 32, 3)
 k_adam_stream(float* __restrict__ P, float* __restrict__ m, float* __restrict__ v, int64_t n,
               int64_t n_pad, BwdCam cam, const int32_t* __restrict__ slot_map,
@@ -475,10 +480,19 @@ k_adam_stream(float* __restrict__ P, float* __restrict__ m, float* __restrict__ 
     dz = (double)P[2 * n_pad + i] - cam.campos[2];
     dn = sqrt(dx * dx + dy * dy + dz * dz);
     dx /= dn; dy /= dn; dz /= dn;
+    if (GEO) {
+      if (rgb.w >= 0.f)  // not a culled Gaussian of the dense layout
+        candidate_grad<false, float>(P, n_pad, i, 0, cam, g2, make_float4(0.f, 0.f, 0.f, 0.f),
+                                     [&](int plane, double gv) {
+                                       if (plane < 3) gm[plane] = gv;
+                                       else if (plane < 11) gr[plane - 3] = (float)gv;
+                                     });
+    } else {
 #pragma unroll
-    for (int k = 0; k < 3; ++k) gm[k] = g_mean[(int64_t)k * n_cand + sl];
+      for (int k = 0; k < 3; ++k) gm[k] = g_mean[(int64_t)k * n_cand + sl];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) gr[k] = g_rest[(int64_t)k * n_cand + sl];
+      for (int k = 0; k < 8; ++k) gr[k] = g_rest[(int64_t)k * n_cand + sl];
+    }
   }
   double ddx = 0.0, ddy = 0.0, ddz = 0.0;
 #pragma unroll 1
@@ -626,12 +640,14 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
   if (!make_adam(fused, &a)) return GS_ERR_ARG;
   if (!adam_m || !adam_v || !proj->slot) return GS_ERR_ARG;
   if (model->n == 0) return GS_OK;
-  // stage 1 needs 14 floats per candidate of scratch (8-byte aligned), in g3d
-  if (n_cand > 0 && (!g3d || g3d_stride < 14 * n_cand || !proj->cand_idx || !aligned(g3d, 8)))
+  // two-pass form: 14 floats per candidate of scratch (8-byte aligned) in g3d;
+  // g3d = NULL runs the geometric chain inside the stream
+  const bool two_pass = g3d != nullptr;
+  if (two_pass && n_cand > 0 && (g3d_stride < 14 * n_cand || !proj->cand_idx || !aligned(g3d, 8)))
     return GS_ERR_ARG;
   double* g_mean = reinterpret_cast<double*>(g3d);
-  float* g_rest = g3d + 6 * n_cand;
-  if (n_cand > 0) {
+  float* g_rest = two_pass ? g3d + 6 * n_cand : nullptr;
+  if (two_pass && n_cand > 0) {
     k_project_bwd_geo<<<(unsigned)((n_cand + kThreads - 1) / kThreads), kThreads, 0, s>>>(
         model->params, model->n_pad, c, n_cand, proj->cand_idx, rec, g2d, g_mean, g_rest);
     GS_LAUNCH_CHECK();
@@ -643,13 +659,18 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
     return GS_ERR_ARG;
   const size_t ring = sizeof(float) * kStages * 3 * kGroupPlanes * kAT;
   const unsigned nbs = (unsigned)((model->n + kAT - 1) / kAT);
-#define GS_ADAM_FUSED(DD)                                                                       \
+#define GS_ADAM_FUSED2(DD, GG)                                                                \
   do {                                                                                          \
     static std::atomic<unsigned long long> done{0};                                             \
-    GS_TRY(smem_attrs_once((const void*)k_adam_stream<DD>, (int)ring, &done));                  \
-    k_adam_stream<DD><<<nbs, kAT + 32, ring, s>>>(model->params, adam_m, adam_v, model->n,      \
-                                                 model->n_pad, c, proj->slot, rec, g2d, g_mean, \
-                                                 g_rest, n_cand, a, dev_status);                \
+    GS_TRY(smem_attrs_once((const void*)k_adam_stream<DD, GG>, (int)ring, &done));              \
+    k_adam_stream<DD, GG><<<nbs, kAT + 32, ring, s>>>(model->params, adam_m, adam_v, model->n,  \
+                                                     model->n_pad, c, proj->slot, rec, g2d,     \
+                                                     g_mean, g_rest, n_cand, a, dev_status);    \
+  } while (0)
+#define GS_ADAM_FUSED(DD)                       \
+  do {                                          \
+    if (two_pass) GS_ADAM_FUSED2(DD, false);    \
+    else GS_ADAM_FUSED2(DD, true);              \
   } while (0)
   switch (D) {
     case 0: GS_ADAM_FUSED(0); break;
@@ -658,6 +679,7 @@ extern "C" gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
     default: GS_ADAM_FUSED(3); break;
   }
 #undef GS_ADAM_FUSED
+#undef GS_ADAM_FUSED2
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

@@ -516,11 +516,12 @@ gs_status gs_raster_bwd(const gs_proj* proj, const int32_t* vals,
  * normalisation, opacity logit, SH).  If `fused` is NULL, writes compact
  * gradients g3d[P][g3d_stride] (column = candidate slot).  Otherwise applies
  * one Adam update (as gs_adam with a zero gradient for non-candidates) to
- * model->params, adam_m and adam_v over all n Gaussians, in two passes: the
- * candidates' geometric gradients (fp32 chain) into g3d used as scratch (>= 14 *
- * n_cand floats, 8-byte aligned, g3d_stride = its size in floats), then one
- * streaming pass
- * over every Gaussian's planes that forms the SH gradients on the fly. */
+ * model->params, adam_m and adam_v over all n Gaussians in one streaming pass
+ * over every Gaussian's planes that forms the SH gradients on the fly.  The
+ * candidates' geometric gradients (fp32 chain) are computed inside that pass
+ * when g3d is NULL; with g3d given they come from a first pass into g3d used
+ * as scratch (>= 14 * n_cand floats, 8-byte aligned, g3d_stride = its size in
+ * floats).  Both forms give the same update up to fp32 rounding. */
 gs_status gs_project_bwd(const gs_model* model, const gs_camera* cam,
                          const gs_proj* proj, int64_t n_cand,
                          const float* g2d, float* g3d, int64_t g3d_stride,

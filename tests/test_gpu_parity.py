@@ -662,6 +662,49 @@ def test_fused_project_bwd_adam(oracle_mod, name):
         assert rel_l2(g_mean[k, ci], grad[k, ci]) <= GRAD_TOL, k
 
 
+@pytest.mark.parametrize("name", ["small3", "hd"])
+def test_fused_project_bwd_adam_in_stream(oracle_mod, name):
+    """g3d = NULL: the geometric chain runs inside the Adam stream.  The
+    gradients implied by the updated m (g = (m - 0.9 m0) / 0.1) match the
+    oracle's per tensor, and the SH planes match the two-pass form."""
+    sc, cam = scene(name)
+    pr = oracle_mod.project(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam)
+    C = len(pr["cand_idx"])
+    rng = np.random.default_rng(4)
+    g2d = (rng.normal(size=(C, 9)) * 1e-3).astype(np.float32)
+    g3d_o = oracle_mod.project_bwd(sc.params.astype(np.float64), sc.sh_degree, cam,
+                                   pr["cand_idx"], g2d.astype(np.float64))
+    m0 = (rng.normal(size=sc.params.shape) * 1e-4).astype(np.float32)
+    v0 = rng.uniform(0, 1e-7, size=sc.params.shape).astype(np.float32)
+    b = B()
+    pb = ProjBuffers.from_oracle(pr, sc.n)
+    g2 = np.zeros((C, 12), np.float32)
+    g2[:, :9] = g2d
+    g2_d = torch.as_tensor(g2.reshape(-1)).cuda()
+    out = []
+    for two_pass in (False, True):
+        params = torch.as_tensor(sc.params).cuda()
+        md, vd = torch.as_tensor(m0).cuda(), torch.as_tensor(v0).cuda()
+        model = b.gs_model(sc.n, sc.n_pad, sc.sh_degree, 0, params.data_ptr())
+        geo = torch.zeros(14 * C, device="cuda") if two_pass else None
+        b.gs_project_bwd(model, b.camera_struct(cam), pb.struct, C, g2_d, g3d=geo,
+                         g3d_stride=geo.numel() if two_pass else 0, adam_m=md, adam_v=vd,
+                         fused=b.gs_adam_args(1e-3, 0.9, 0.999, 1e-8, 2, 0))
+        torch.cuda.synchronize()
+        out.append((params.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy()))
+    (p1, m1, v1), (p2, m2, v2) = out
+    n = sc.n
+    ci = pr["cand_idx"]
+    g_impl = (m1[:, :n].astype(np.float64) - 0.9 * m0[:, :n]) / 0.1
+    for k in range(11):
+        assert rel_l2(g_impl[k, ci], g3d_o[k]) <= GRAD_TOL, k
+    np.testing.assert_allclose(m1[11:, :n], m2[11:, :n], rtol=1e-6, atol=1e-30)
+    np.testing.assert_allclose(p1[11:, :n], p2[11:, :n], rtol=1e-6, atol=2e-8)
+    # non-candidates: m, v decay and p moves by the same dense rule in both
+    nc = np.setdiff1d(np.arange(n), ci)
+    assert np.array_equal(m1[:, nc], m2[:, nc]) and np.array_equal(v1[:, nc], v2[:, nc])
+
+
 # ---------------------------------------------------------------------------
 # end to end through the Step driver
 # ---------------------------------------------------------------------------
@@ -935,3 +978,26 @@ def test_gated_step():
         took.append(g.last[3])
         assert bool((model.params != before).any()) == g.last[3]
     assert took[:2] == [True, True] and g.b == sum(took) and model.step == g.b
+
+
+def test_in_stream_chain_step_matches_two_pass():
+    """Stepper(fuse_adam="in_stream") (geometric chain inside the Adam
+    stream, no scratch) takes the same step as the default two-pass form up
+    to fp32 rounding of the chain, and needs no more working set (less where
+    the projection backward sets the peak)."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("small3")
+    target = torch.as_tensor(synth.random_image(cam.width, cam.height, 6) * 0.5).cuda()
+    outs = []
+    for fa in (True, "in_stream"):
+        model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+        stp = Stepper(model, budget=100_000, fuse_adam=fa)
+        stats = stp.run_view(cam, target)
+        stp.check()
+        outs.append((stp.last_loss(), model.params.cpu().numpy(), model.m.cpu().numpy(),
+                     stats.peak_ws_bytes))
+    (l0, p0, m0, w0), (l1, p1, m1, w1) = outs
+    assert l0 == l1
+    assert np.abs(p1 - p0).max() <= 2.1e-3
+    assert rel_l2(m1, m0) <= 1e-5
+    assert w1 <= w0
