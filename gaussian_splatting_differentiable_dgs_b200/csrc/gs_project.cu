@@ -114,7 +114,8 @@ __device__ __forceinline__ bool project_geometry(const float* __restrict__ P, in
     nonfinite = true;
     return false;
   }
-  qw /= qn; qx /= qn; qy /= qn; qz /= qn;
+  const double iqn = 1.0 / qn;
+  qw *= iqn; qx *= iqn; qy *= iqn; qz *= iqn;
   double Rg[9];
   Rg[0] = 1.0 - 2.0 * (qy * qy + qz * qz); Rg[1] = 2.0 * (qx * qy - qw * qz); Rg[2] = 2.0 * (qx * qz + qw * qy);
   Rg[3] = 2.0 * (qx * qy + qw * qz); Rg[4] = 1.0 - 2.0 * (qx * qx + qz * qz); Rg[5] = 2.0 * (qy * qz - qw * qx);
@@ -135,8 +136,9 @@ __device__ __forceinline__ bool project_geometry(const float* __restrict__ P, in
   Sg[4] = M[3] * M[6] + M[4] * M[7] + M[5] * M[8];
   Sg[5] = M[6] * M[6] + M[7] * M[7] + M[8] * M[8];
   // T = J W, J the perspective Jacobian at t
-  const double j00 = c.fx / tz, j02 = -c.fx * xn / tz;
-  const double j11 = c.fy / tz, j12 = -c.fy * yn / tz;
+  const double itz = 1.0 / tz;
+  const double j00 = c.fx * itz, j02 = -j00 * xn;
+  const double j11 = c.fy * itz, j12 = -j11 * yn;
   double T0[3], T1[3];
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
@@ -207,8 +209,8 @@ __device__ __forceinline__ void sh_record(const float* __restrict__ P, int64_t n
                                           const ProjCam& c, const ProjGeo& g, float4& r0,
                                           float4& r1, float4& r2) {
   double dx = g.x - c.campos[0], dy = g.y - c.campos[1], dz = g.z - c.campos[2];
-  const double dn = sqrt(dx * dx + dy * dy + dz * dz);
-  dx /= dn; dy /= dn; dz /= dn;
+  const double idn = 1.0 / sqrt(dx * dx + dy * dy + dz * dz);
+  dx *= idn; dy *= idn; dz *= idn;
   constexpr int ksh = (D + 1) * (D + 1);
   float sh[ksh][3];
 #pragma unroll
@@ -229,8 +231,12 @@ __device__ __forceinline__ void sh_record(const float* __restrict__ P, int64_t n
   const __half2 box = __halves2half2(__float2half_ru((float)g.hx), __float2half_ru((float)g.hy));
   r0 = make_float4(uh, vh, __uint_as_float(*reinterpret_cast<const unsigned*>(&lo)),
                    __uint_as_float(*reinterpret_cast<const unsigned*>(&box)));
-  const double a = g.c11 / g.det, b = -g.c01 / g.det;
-  r1 = make_float4((float)(0.5 * a), (float)(b / a), (float)(0.5 / g.c11), (float)g.opac);
+  // conic (a, b, c) = (c11, -c01, c00) / det; the record keeps s1 = a / 2,
+  // beta = b / a = -c01 / c11 and s2 = (c - b^2 / a) / 2 = 1 / (2 c11), so
+  // that q = s1 (dx + beta dy)^2 + s2 dy^2
+  const double ic11 = 1.0 / g.c11;
+  r1 = make_float4((float)(0.5 * g.c11 / g.det), (float)(-g.c01 * ic11), (float)(0.5 * ic11),
+                   (float)g.opac);
   const float depth = (float)g.tz;
   r2 = make_float4((float)fmax(rgb[0], 0.0), (float)fmax(rgb[1], 0.0), (float)fmax(rgb[2], 0.0),
                    depth);

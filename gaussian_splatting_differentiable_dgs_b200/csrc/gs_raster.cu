@@ -35,11 +35,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Staged record: position relative to the tile origin and the exponent
-// coefficients pre-scaled by -log2(e).
+// Staged record: position relative to the tile origin, the exponent
+// coefficients pre-scaled by -log2(e) and the opacity as its log2, which
+// joins the exponent (o 2^x = 2^(x + log2 o)).
 struct Staged {
   float gx, gy, beta, ns1;   // float4
-  float ns2, opac, r, g;     // float4
+  float ns2, lo2, r, g;      // float4
+  float opac;
   float b, s1, s2;           // natural-log coefficients (backward)
   float hx, hy;              // alpha box half extents
   int32_t slot;
@@ -62,6 +64,7 @@ __device__ __forceinline__ Staged stage_record(const float4* __restrict__ rec, i
   s.ns1 = __fmul_rn(r1.x, -kLog2e);
   s.ns2 = __fmul_rn(r1.z, -kLog2e);
   s.opac = r1.w;
+  s.lo2 = log2f(r1.w);
   s.r = r2.x;
   s.g = r2.y;
   s.b = r2.z;
@@ -78,22 +81,21 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 struct Eval {
-  float dx, dy, t1, G, araw, alpha;
+  float dx, dy, t1, araw, alpha;
 };
 
-// alpha = min(0.99, o 2^(-q log2 e)),  q = s1 (dx + beta dy)^2 + s2 dy^2,
-// with dx = gx - px given (a lane's pixels share their column)
+// alpha = min(0.99, o e^-q) = min(0.99, 2^(log2 o - q log2 e)),
+// q = s1 (dx + beta dy)^2 + s2 dy^2, with dx = gx - px given (a lane's
+// pixels share their column); araw = o e^-q is the unclamped value
 __device__ __forceinline__ Eval eval_alpha(float dx, float gy, float beta, float ns1, float ns2,
-                                           float opac, float py) {
+                                           float lo2, float py) {
   Eval e;
   e.dx = dx;
   e.dy = __fsub_rn(gy, py);
   e.t1 = __fmaf_rn(beta, e.dy, e.dx);
   const float qa = __fmul_rn(ns1, e.t1);
-  const float qb = __fmul_rn(ns2, e.dy);
-  const float ql = __fmaf_rn(qa, e.t1, __fmul_rn(qb, e.dy));
-  e.G = ex2_approx(ql);
-  e.araw = __fmul_rn(opac, e.G);
+  const float qb = __fmaf_rn(__fmul_rn(ns2, e.dy), e.dy, lo2);
+  e.araw = ex2_approx(__fmaf_rn(qa, e.t1, qb));
   e.alpha = fminf(e.araw, kAlphaMax);
   return e;
 }
@@ -347,7 +349,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         const Staged st = stage_record(rec, s_hits[hp + t], tx, ty);
         s_mask[t] = (uint8_t)warp_mask<PPT>(st);
         sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-        sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+        sB[t] = make_float4(st.ns2, st.lo2, st.r, st.g);
         sC[t] = st.b;
       }
       __syncthreads();
@@ -360,7 +362,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         const Staged st = stage_record(rec, vals[e], tx, ty);
         s_mask[t] = (uint8_t)warp_mask<PPT>(st);
         sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-        sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+        sB[t] = make_float4(st.ns2, st.lo2, st.r, st.g);
         sC[t] = st.b;
       }
       __syncthreads();
@@ -390,7 +392,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
         if (COUNT) ++n_vis;
         if (ev.alpha < kAlphaMin) continue;
-        const float Tn = __fmul_rn(T[k], __fsub_rn(1.0f, ev.alpha));
+        const float Tn = __fmaf_rn(-ev.alpha, T[k], T[k]);  // T (1 - alpha), one rounding
         if (Tn < kTMin) {
           done[k] = true;
           if (COUNT) stopn[k] = posn;
@@ -520,54 +522,34 @@ k_loss_total(const float* __restrict__ tiles, int64_t n, double* __restrict__ ou
 // backward
 // ---------------------------------------------------------------------------
 
-// Sum of 9 values over the warp, scattered: afterwards lane L with L even
-// and idx = (L >> 1) & 15 < 9 holds the warp total of value idx.  16
-// shuffles instead of 45 for nine independent butterflies.
-__device__ __forceinline__ float warp_reduce_scatter9(const float (&v)[9], int lane) {
-  float a[8];
-  {
-    const bool up = lane & 16;
-    // level 1: keep values 0..7 (low half) or 8..15 (high half; only 8 real)
+// Sum of 9 values over the warp through a 32 x 9 shared staging area (one
+// per warp): every lane stores its 9 values, then lane 3 v + p (v < 9,
+// p < 3) adds value v of lanes p, p + 3, p + 6, ... (11 or 10 of them) and
+// the three partial sums of value v meet in lane 3 v.  Stride 9 keeps both
+// the stores and the loads free of bank conflicts (9 and 27 are odd, and
+// 9 p + v < 27 is distinct over the reading lanes).  About 35 instructions
+// instead of the ~70 of a nine-value shuffle butterfly.  Returns the total
+// of value lane / 3 in lanes 3 v; other lanes return garbage.
+__device__ __forceinline__ float warp_reduce9_smem(const float (&v)[9], float* __restrict__ red,
+                                                   int lane, int rv, int rp) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float mine_keep = up ? (i == 0 ? v[8] : 0.0f) : v[i];
-      const float send = up ? v[i] : (i == 0 ? v[8] : 0.0f);
-      a[i] = mine_keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-  }
-  float b[4];
-  {
-    const bool up = lane & 8;
+  for (int q = 0; q < 9; ++q) red[lane * 9 + q] = v[q];
+  __syncwarp();
+  float s = 0.0f;
+  if (lane < 27) {
+    const float* src = red + rp * 9 + rv;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float keep = up ? a[4 + i] : a[i];
-      const float send = up ? a[i] : a[4 + i];
-      b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
+    for (int k = 0; k < 11; ++k)
+      if (3 * k + rp < 32) s += src[27 * k];
   }
-  float c[2];
-  {
-    const bool up = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float keep = up ? b[2 + i] : b[i];
-      const float send = up ? b[i] : b[2 + i];
-      c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-  }
-  float d;
-  {
-    const bool up = lane & 2;
-    const float keep = up ? c[1] : c[0];
-    const float send = up ? c[0] : c[1];
-    d = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-  d += __shfl_xor_sync(0xffffffffu, d, 1);
-  return d;
+  const float s1 = __shfl_down_sync(0xffffffffu, s, 1);
+  const float s2 = __shfl_down_sync(0xffffffffu, s, 2);
+  __syncwarp();  // the staging area is free for the next record
+  return s + s1 + s2;
 }
 
 template <int PPT, bool COUNT>
-__global__ void __launch_bounds__(256 / PPT)
+__global__ void __launch_bounds__(256 / PPT, PPT == 4 ? 14 : 1)
 k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, PixArgs px,
              float* __restrict__ g2d, int32_t* dev_status) {
@@ -579,12 +561,14 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   __shared__ uint8_t s_list[G::NW][NT];
   __shared__ float sg[NT][12];
   __shared__ int s_touched[NT];
+  __shared__ float s_red[G::NW][32 * 9];
   __shared__ int s_maxlast;
   const int lw = leaf.x1 - leaf.x0;
   const int ltile = blockIdx.x;
   const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
   const int64_t begin = ranges[2 * ltile];
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int rv = lane / 3, rp = lane - 3 * (lane / 3);  // reduction role (warp_reduce9_smem)
   const WarpPix wp = warp_pixels<PPT>(t);
   const float fpx = (float)wp.lx + 0.5f;
   // S = sum_c g_c A_c, A_c = colour composited behind the current entry
@@ -629,7 +613,7 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       const Staged st = stage_record(rec, vals[begin + pos], tx, ty);
       s_mask[t] = (uint8_t)warp_mask<PPT>(st);
       sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-      sB[t] = make_float4(st.ns2, st.opac, st.r, st.g);
+      sB[t] = make_float4(st.ns2, st.lo2, st.r, st.g);
       sC[t] = make_float4(st.b, 2.0f * st.s1, 2.0f * st.s2, __int_as_float(st.slot));
     }
     __syncthreads();
@@ -674,36 +658,46 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         T[k] = Tb;
         if (ev.araw <= kAlphaMax) {
           const float dq = -ev.alpha * da;         // dL/dq (natural units)
-          acc[5] = fmaf(ev.G, da, acc[5]);          // dL/dopacity
+          acc[5] = fmaf(ev.araw, da, acc[5]);       // o dL/dopacity (1/o at the flush)
           sq += dq;
           const float dqy = dq * ev.dy;
           sqy += dqy;
           sqyy = fmaf(dqy, ev.dy, sqyy);
         }
       }
-      // q = (a dx^2 + c dy^2) / 2 + b dx dy with a = 2 s1, b = beta a,
-      // c = 2 s2 + beta b: dq/du = a dx + b dy, dq/dv = b dx + c dy
-      // = beta dq/du + 2 s2 dy, dq/da = dx^2 / 2, dq/db = dx dy, dq/dc = dy^2 / 2
-      acc[0] = Cc.y * fmaf(A.z, sqy, dx * sq);
-      acc[1] = fmaf(A.z, acc[0], Cc.z * sqy);
-      acc[2] = 0.5f * dx * dx * sq;
+      // the geometric gradients are linear in five moments of dq over the
+      // warp's pixels: sum dx dq, sum dx^2 dq, sum dq dy, sum dx dq dy and
+      // sum dq dy^2 (turned into du, dv, da, db, dc once per record at the
+      // flush below)
+      const float dxq = dx * sq;
+      acc[0] = dxq;
+      acc[1] = dx * dxq;
+      acc[2] = sqy;
       acc[3] = dx * sqy;
-      acc[4] = 0.5f * sqyy;
+      acc[4] = sqyy;
       // reduce first: per-lane shared atomics on the same 9 words cost more
       // than the reduction, even with only 2 lanes kept
       if (__any_sync(0xffffffffu, any)) {
-        const float tot = warp_reduce_scatter9(acc, lane);
-        const int idx = (lane >> 1) & 15;
-        if (!(lane & 1) && idx < 9) atomicAdd(&sg[j][idx], tot);
+        const float tot = warp_reduce9_smem(acc, s_red[w], lane, rv, rp);
+        if (lane < 27 && rp == 0) atomicAdd(&sg[j][rv], tot);
         if (lane == 0) s_touched[j] = 1;
       }
     }
     __syncthreads();
     if (t < cnt && s_touched[t]) {
-      const int32_t slot = __float_as_int(sC[t].w);
+      const float4 Cc = sC[t];
+      const int32_t slot = __float_as_int(Cc.w);
+      const float beta = sA[t].z;
+      // q = (a dx^2 + c dy^2) / 2 + b dx dy with a = 2 s1, b = beta a,
+      // c = 2 s2 + beta b: dq/du = a dx + b dy, dq/dv = b dx + c dy
+      // = beta dq/du + 2 s2 dy, dq/da = dx^2 / 2, dq/db = dx dy, dq/dc = dy^2 / 2
+      const float du = Cc.y * fmaf(beta, sg[t][2], sg[t][0]);
+      const float dv = fmaf(beta, du, Cc.z * sg[t][2]);
       float4* dst = reinterpret_cast<float4*>(g2d + (int64_t)slot * 12);
-      atomicAdd(dst, make_float4(sg[t][0], sg[t][1], sg[t][2], sg[t][3]));
-      atomicAdd(dst + 1, make_float4(sg[t][4], sg[t][5], sg[t][6], sg[t][7]));
+      atomicAdd(dst, make_float4(du, dv, 0.5f * sg[t][1], sg[t][3]));
+      // dL/do = sum e^-q dL/dalpha = (sum o e^-q dL/dalpha) / o, 1/o = 2^-log2 o
+      const float inv_o = ex2_approx(-sB[t].y);
+      atomicAdd(dst + 1, make_float4(0.5f * sg[t][4], sg[t][5] * inv_o, sg[t][6], sg[t][7]));
       atomicAdd(dst + 2, make_float4(sg[t][8], 0.0f, 0.0f, 0.0f));
 #pragma unroll
       for (int q = 0; q < 9; ++q) sg[t][q] = 0.0f;
