@@ -317,18 +317,21 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
   }
   int total;
   const int rank = block_exclusive_scan<int, kProjThreads / 32>(cand ? 1 : 0, s_scan, &total);
+  // warp 0 resolves the block's prefix while every warp forms its
+  // candidates' records (which do not depend on the slot), so the look-back
+  // latency hides behind the SH reads and arithmetic
   if (threadIdx.x < 32) {
     int64_t ex = lookback_warp(lb, b, total, dev_status);
     if (threadIdx.x == 0) s_prefix = ex;
   }
+  float4 r0, r1, r2;
+  if (cand) sh_record<D>(params, n_pad, i, cam, o, r0, r1, r2);
   __syncthreads();
   const int64_t slot = s_prefix + rank;
   const bool fits = slot < capacity;  // false beyond the caller's capacity (it retries)
   if (cand && !fits) dev_flag(dev_status, GS_DEV_BOUNDS);
   if (i < n) slot_map[i] = (cand && fits) ? (int32_t)slot : -1;
   if (cand && fits) {
-    float4 r0, r1, r2;
-    sh_record<D>(params, n_pad, i, cam, o, r0, r1, r2);
     cand_idx[slot] = (int32_t)i;
     rec[3 * slot] = r0;
     rec[3 * slot + 1] = r1;

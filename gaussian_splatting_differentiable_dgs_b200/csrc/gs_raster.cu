@@ -241,7 +241,7 @@ struct BlockSrc {
 constexpr int kFillU = 2;
 
 template <int PPT, bool COUNT, bool BLK>
-__global__ void __launch_bounds__(256 / PPT)
+__global__ void __launch_bounds__(256 / PPT, PPT == 2 ? 8 : 1)
 k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
              BlockSrc bsrc, int32_t* dev_status) {
@@ -386,25 +386,28 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       const float Bb = sC[j];
       const int posn = pos1 + j;
       const float dx = __fsub_rn(A.x, fpx);
+      // branch-free: every pixel evaluates, and selects keep the state of
+      // a pixel that is done, skips the entry or stops at it (a zero weight
+      // leaves the colour sums unchanged)
 #pragma unroll
       for (int k = 0; k < PPT; ++k) {
-        if (done[k]) continue;
         const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
-        if (COUNT) ++n_vis;
-        if (ev.alpha < kAlphaMin) continue;
+        if (COUNT) n_vis += done[k] ? 0u : 1u;
+        const bool use = !done[k] && ev.alpha >= kAlphaMin;
         const float Tn = __fmaf_rn(-ev.alpha, T[k], T[k]);  // T (1 - alpha), one rounding
-        if (Tn < kTMin) {
-          done[k] = true;
-          if (COUNT) stopn[k] = posn;
-          continue;
+        const bool stop = use && Tn < kTMin;
+        const bool comp = use && !stop;
+        if (COUNT) {
+          stopn[k] = stop ? posn : stopn[k];
+          n_kept += comp ? 1u : 0u;
         }
-        if (COUNT) ++n_kept;
-        const float wgt = ev.alpha * T[k];
+        done[k] = done[k] || stop;
+        const float wgt = comp ? ev.alpha * T[k] : 0.0f;
         Cr[k] = fmaf(B.z, wgt, Cr[k]);
         Cg[k] = fmaf(B.w, wgt, Cg[k]);
         Cb[k] = fmaf(Bb, wgt, Cb[k]);
-        T[k] = Tn;
-        lastp[k] = posn;
+        T[k] = comp ? Tn : T[k];
+        lastp[k] = comp ? posn : lastp[k];
       }
       }
     }
@@ -634,19 +637,24 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       float sq = 0.0f, sqy = 0.0f, sqyy = 0.0f;
       bool any = false;
       const float dx = __fsub_rn(A.x, fpx);
+      // branch-free: an entry at or beyond the pixel's last, or below 1/255,
+      // enters with alpha = 0, which leaves T, S and every sum unchanged
 #pragma unroll
       for (int k = 0; k < PPT; ++k) {
-        if (pos >= lastp[k]) continue;
+        const bool inl = pos < lastp[k];
         const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
-        if (COUNT) ++n_vis;
-        if (ev.alpha < kAlphaMin) continue;
-        if (COUNT) ++n_kept;
-        any = true;
+        const bool use = inl && ev.alpha >= kAlphaMin;
+        if (COUNT) {
+          n_vis += inl ? 1u : 0u;
+          n_kept += use ? 1u : 0u;
+        }
+        any = any || use;
+        const float au = use ? ev.alpha : 0.0f;
         // T only scales gradient values here (no decision depends on it), so
         // the hardware reciprocal (about 1 ulp) is enough
-        const float inv = rcp_approx(1.0f - ev.alpha);
+        const float inv = rcp_approx(1.0f - au);
         const float Tb = T[k] * inv;          // transmittance before this entry
-        const float wgt = ev.alpha * Tb;
+        const float wgt = au * Tb;
         acc[6] = fmaf(wgt, gr[k], acc[6]);
         acc[7] = fmaf(wgt, gg[k], acc[7]);
         acc[8] = fmaf(wgt, gb[k], acc[8]);
@@ -655,15 +663,15 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         const float grgb = fmaf(gb[k], Cc.x, fmaf(gg[k], B.w, gr[k] * B.z));
         const float da = fmaf(Tb, grgb, -S[k] * inv);
         S[k] = fmaf(wgt, grgb, S[k]);
-        T[k] = Tb;
-        if (ev.araw <= kAlphaMax) {
-          const float dq = -ev.alpha * da;         // dL/dq (natural units)
-          acc[5] = fmaf(ev.araw, da, acc[5]);       // o dL/dopacity (1/o at the flush)
-          sq += dq;
-          const float dqy = dq * ev.dy;
-          sqy += dqy;
-          sqyy = fmaf(dqy, ev.dy, sqyy);
-        }
+        T[k] = use ? Tb : T[k];
+        // unclamped entries: dL/dq (natural units) and o dL/dopacity
+        const bool unc = use && ev.araw <= kAlphaMax;
+        const float dq = unc ? -ev.alpha * da : 0.0f;
+        acc[5] = fmaf(unc ? ev.araw : 0.0f, da, acc[5]);  // 1/o at the flush
+        sq += dq;
+        const float dqy = dq * ev.dy;
+        sqy += dqy;
+        sqyy = fmaf(dqy, ev.dy, sqyy);
       }
       // the geometric gradients are linear in five moments of dq over the
       // warp's pixels: sum dx dq, sum dx^2 dq, sum dq dy, sum dx dq dy and
