@@ -19,7 +19,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
-# extra nvcc flags (e.g. -DGS_BWD_BATCH=1 to compare tuning constants); a
+# extra nvcc flags (e.g. -DGS_ADAM_STAGES=4 to compare tuning constants); a
 # change of them is not tracked, so rebuild with --force after setting them
 FLAGS += os.environ.get("GS_NVCC_FLAGS", "").split()
 
