@@ -664,10 +664,11 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
         const float da = fmaf(Tb, grgb, -S[k] * inv);
         S[k] = fmaf(wgt, grgb, S[k]);
         T[k] = use ? Tb : T[k];
-        // unclamped entries: dL/dq (natural units) and o dL/dopacity
-        const bool unc = use && ev.araw <= kAlphaMax;
-        const float dq = unc ? -ev.alpha * da : 0.0f;
-        acc[5] = fmaf(unc ? ev.araw : 0.0f, da, acc[5]);  // 1/o at the flush
+        // unclamped entries (where alpha = araw = o e^-q): dL/dq (natural
+        // units) = -alpha dL/dalpha, and o dL/dopacity = alpha dL/dalpha
+        const float ua = ev.araw <= kAlphaMax ? au : 0.0f;
+        const float dq = -ua * da;
+        acc[5] = fmaf(ua, da, acc[5]);  // 1/o at the flush
         sq += dq;
         const float dqy = dq * ev.dy;
         sqy += dqy;
