@@ -129,7 +129,7 @@ class Stepper:
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
                  binning="fused", mode="bounded", loss="l1", ssim_lambda=B.SSIM_LAMBDA,
-                 device="cuda"):
+                 leaf_streams=1, device="cuda"):
         if binning not in ("fused", "expand", "sort"):
             raise ValueError(f"binning must be 'fused', 'expand' or 'sort', not {binning!r}")
         if mode not in ("bounded", "original"):
@@ -141,6 +141,12 @@ class Stepper:
         # alive through the projection backward, dense gradients)
         if loss not in ("l1", "l1_ssim"):
             raise ValueError(f"loss must be 'l1' or 'l1_ssim', not {loss!r}")
+        # leaf_streams = 2: consecutive Leaves alternate between two streams
+        # and two raster arenas, so one Leaf's kernels fill the SMs that the
+        # other's last CTAs leave idle (two Leaves' raster buffers in flight,
+        # each within the budget)
+        if leaf_streams not in (1, 2):
+            raise ValueError(f"leaf_streams must be 1 or 2, not {leaf_streams!r}")
         # l1: the L1 photometric loss; l1_ssim: the composite
         # (1 - lambda) L1 + lambda (1 - SSIM) of 3DGS training (SkipGS notes,
         # "loss function / training strategy"), SSIM windows local to each Leaf
@@ -157,6 +163,8 @@ class Stepper:
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
         self._last_loss = None
         self._copy_stream = None
+        self.leaf_streams = leaf_streams
+        self._leaf_stream = None
         self._cap_hint = {}  # region -> candidate capacity for the next view
 
     def check(self):
@@ -356,6 +364,14 @@ class Stepper:
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
         arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
+        two = self.leaf_streams == 2 and len(lv) > 1 and not original
+        main = torch.cuda.current_stream(dev)
+        arenas, lstreams = [arena], [main]
+        if two:
+            arenas.append(torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev))
+            if self._leaf_stream is None:
+                self._leaf_stream = torch.cuda.Stream(device=dev)
+            lstreams.append(self._leaf_stream)
         norm = 1.0 / (3.0 * W * H)
         # with the SSIM term the forward's L1 part carries (1 - lambda)
         norm_l1 = (1.0 - self.ssim_lambda) * norm if ssim else norm
@@ -371,12 +387,15 @@ class Stepper:
                 self._copy_stream = torch.cuda.Stream(device=dev)
             cs = self._copy_stream
 
+        hstate = {}  # the host target's upload state, shared by leaf_pass and leaf_one
+
         def leaf_pass(with_bwd):
             """Every Leaf: lists, forward (+ L1) and, if with_bwd, backward."""
+            if two:
+                lstreams[1].wait_stream(main)  # g2d, lists and tables are ready
             if host_target:
                 up = [torch.cuda.Event() for _ in lv]
                 freed = [None, None]
-                main = torch.cuda.current_stream(dev)
 
                 def upload(k):
                     x_, y_, w_, h_ = rects[k]
@@ -389,10 +408,21 @@ class Stepper:
 
                 for k in range(min(2, len(lv))):
                     upload(k)
+                hstate.update(up=up, freed=freed, upload=upload)
             for li_k, (L, I) in enumerate(zip(lv, li)):
+                with torch.cuda.stream(lstreams[li_k % len(lstreams)]):
+                    leaf_one(li_k, L, I, with_bwd)
+            if two:
+                main.wait_stream(lstreams[1])
+
+        def leaf_one(li_k, L, I, with_bwd):
+            """One Leaf on the current stream, with its arena."""
+            if True:
+                ls = torch.cuda.current_stream(dev)
+                up, freed, upload = hstate.get("up"), hstate.get("freed"), hstate.get("upload")
                 I = int(I)
                 sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
-                bufs, _ = _carve(arena, sizes)
+                bufs, _ = _carve(arenas[li_k % len(arenas)], sizes)
                 keys = bufs[0].view(torch.int32)
                 vals = bufs[1].view(torch.int32)
                 ranges = bufs[2].view(torch.int64)
@@ -408,7 +438,7 @@ class Stepper:
                                   loss_tiles=loss_tiles, norm=norm_l1, counters=cnt_f)
                 elif host_target:
                     crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
-                    main.wait_event(up[li_k])
+                    ls.wait_event(up[li_k])
                     px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
                                   target_origin=(px0, py0), loss_tiles=loss_tiles,
                                   norm=norm_l1, counters=cnt_f)
@@ -447,7 +477,7 @@ class Stepper:
                     clk.toc(tk)
                 if host_target:
                     ev = torch.cuda.Event()
-                    ev.record(main)
+                    ev.record(ls)
                     freed[li_k % 2] = ev
                     if li_k + 2 < len(lv):
                         upload(li_k + 2)

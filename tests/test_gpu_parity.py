@@ -726,22 +726,27 @@ class Capture:
         self.cand_idx = ctx["cand_idx"][:ctx["n_cand"]].cpu().numpy()
 
 
-@pytest.mark.parametrize("name,budget,binning,mode", [
-    ("tiny", 384 << 20, "fused", "bounded"), ("tiny", 120_000, "fused", "bounded"),
-    ("tiny", 120_000, "expand", "bounded"), ("tiny", 120_000, "sort", "bounded"),
-    ("ragged", 30_000, "fused", "bounded"), ("small3", 200_000, "fused", "bounded"),
-    ("small3", 200_000, "sort", "bounded"), ("hd", 384 << 20, "fused", "bounded"),
-    ("hd", 20 << 20, "fused", "bounded"), ("hd", 20 << 20, "expand", "bounded"),
-    ("hd", 20 << 20, "sort", "bounded"), ("tiny", 120_000, "fused", "original"),
-    ("ragged", 30_000, "sort", "original"), ("hd", 20 << 20, "fused", "original")])
-def test_end_to_end_step(oracle_mod, name, budget, binning, mode):
+@pytest.mark.parametrize("name,budget,binning,mode,streams", [
+    ("tiny", 384 << 20, "fused", "bounded", 1), ("tiny", 120_000, "fused", "bounded", 1),
+    ("tiny", 120_000, "expand", "bounded", 1), ("tiny", 120_000, "sort", "bounded", 1),
+    ("ragged", 30_000, "fused", "bounded", 1), ("small3", 200_000, "fused", "bounded", 1),
+    ("small3", 200_000, "sort", "bounded", 1), ("hd", 384 << 20, "fused", "bounded", 1),
+    ("hd", 20 << 20, "fused", "bounded", 1), ("hd", 20 << 20, "expand", "bounded", 1),
+    ("hd", 20 << 20, "sort", "bounded", 1), ("tiny", 120_000, "fused", "original", 1),
+    ("ragged", 30_000, "sort", "original", 1), ("hd", 20 << 20, "fused", "original", 1),
+    # two Leaves in flight on two streams with two raster arenas
+    ("tiny", 120_000, "fused", "bounded", 2), ("ragged", 30_000, "fused", "bounded", 2),
+    ("small3", 200_000, "expand", "bounded", 2), ("hd", 20 << 20, "fused", "bounded", 2),
+    ("hd", 20 << 20, "sort", "bounded", 2)])
+def test_end_to_end_step(oracle_mod, name, budget, binning, mode, streams):
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, cam = scene(name)
     target = synth.random_image(cam.width, cam.height, 12) * 0.6
     ref = oracle_mod.step(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam,
                           target.astype(np.float64))
     model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=budget, fuse_adam=False, binning=binning, mode=mode)
+    stp = Stepper(model, budget=budget, fuse_adam=False, binning=binning, mode=mode,
+                  leaf_streams=streams)
     cap = Capture(cam.width, cam.height)
     stats = stp.run_view(cam, torch.as_tensor(target).cuda(), hooks=cap)
     stp.check()
@@ -775,17 +780,19 @@ def test_end_to_end_step(oracle_mod, name, budget, binning, mode):
         assert d.max() <= 2.1e-3, gname  # at most one sign flip of a ~zero gradient
 
 
-def test_host_target_matches_resident_target():
+@pytest.mark.parametrize("streams", [1, 2])
+def test_host_target_matches_resident_target(streams):
     """The bounded supply of a pinned host target (per-Leaf crops uploaded on a
     copy stream, double-buffered) gives the same loss and last as the
-    resident target, and the same gradients up to atomic order."""
+    resident target, and the same gradients up to atomic order; with one or
+    two Leaf streams."""
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, cam = scene("hd")
     tgt = synth.random_image(cam.width, cam.height, 8) * 0.5
     outs = []
     for host in (False, True):
         model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-        stp = Stepper(model, budget=6 << 20)
+        stp = Stepper(model, budget=6 << 20, leaf_streams=streams)
         t = torch.as_tensor(tgt).pin_memory() if host else torch.as_tensor(tgt).cuda()
         cap = Capture(cam.width, cam.height)
         stats = stp.run_view(cam, t, hooks=cap)
@@ -812,9 +819,10 @@ def test_leaf_invariance_gpu(oracle_mod):
              [(x, y, x + 1, y + 1) for y in range(TH) for x in range(TW)],
              [(0, 0, 3, TH), (3, 0, TW, 4), (3, 4, TW, TH)]]
     outs = []
-    for leaves in parts:
+    # the multi-Leaf partitions also with two Leaves in flight (two streams)
+    for leaves, streams in [(q, 1) for q in parts] + [(parts[2], 2), (parts[3], 2)]:
         model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-        stp = Stepper(model, budget=100_000)
+        stp = Stepper(model, budget=100_000, leaf_streams=streams)
         cap = Capture(cam.width, cam.height)
         stp.run_view(cam, target, leaves=leaves, hooks=cap, update=False)
         stp.check()

@@ -112,3 +112,17 @@ def test_leaf_partition_capacity_retry(gsb, oracle_mod):
     lm = gsb.gs_leaf_load_model(12, gsb.GS_BIN_SORT)
     st, lv, *_ = gsb.gs_leaf_partition(sat, 50, 40, 800, 640, lm, 300_000, max_leaves=2)
     assert len(lv) > 2  # the wrapper grew the output after GS_ERR_CAPACITY
+
+
+def test_stepper_rejects_unknown_options():
+    """Stepper's options are checked on the host before any device work."""
+    import numpy as np
+    import pytest
+    from gaussian_splatting_differentiable_dgs_b200 import synth
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, _ = synth.tiny_scene(n=4)
+    model = GaussianModel(np.asarray(sc.params), sc.n, sc.sh_degree, device="cpu")
+    for kw in ({"leaf_streams": 3}, {"leaf_streams": 0}, {"binning": "tiles"},
+               {"mode": "whole"}, {"loss": "l2"}):
+        with pytest.raises(ValueError):
+            Stepper(model, device="cpu", **kw)
