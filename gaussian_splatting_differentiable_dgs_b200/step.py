@@ -367,8 +367,10 @@ class Stepper:
         two = self.leaf_streams == 2 and len(lv) > 1 and not original
         main = torch.cuda.current_stream(dev)
         arenas, lstreams = [arena], [main]
+        bin_wss = [bin_ws]
         if two:
             arenas.append(torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev))
+            bin_wss.append(torch.empty_like(bin_ws))  # the list builders' scratch, per stream
             if self._leaf_stream is None:
                 self._leaf_stream = torch.cuda.Stream(device=dev)
             lstreams.append(self._leaf_stream)
@@ -417,80 +419,80 @@ class Stepper:
 
         def leaf_one(li_k, L, I, with_bwd):
             """One Leaf on the current stream, with its arena."""
-            if True:
-                ls = torch.cuda.current_stream(dev)
-                up, freed, upload = hstate.get("up"), hstate.get("freed"), hstate.get("upload")
-                I = int(I)
-                sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
-                bufs, _ = _carve(arenas[li_k % len(arenas)], sizes)
-                keys = bufs[0].view(torch.int32)
-                vals = bufs[1].view(torch.int32)
-                ranges = bufs[2].view(torch.int64)
-                sort_ws = bufs[3]
-                img = bufs[4].view(torch.float32)
-                Tf = bufs[5].view(torch.float32)
-                last = bufs[6].view(torch.int32)
-                dL = bufs[7].view(torch.float32)
-                if resident_target:
-                    # the whole view's target is read in place with its own pitch
-                    px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
-                                  target_origin=(0, 0), target_pitch=W, target_plane=W * H,
-                                  loss_tiles=loss_tiles, norm=norm_l1, counters=cnt_f)
-                elif host_target:
-                    crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
-                    ls.wait_event(up[li_k])
-                    px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
-                                  target_origin=(px0, py0), loss_tiles=loss_tiles,
-                                  norm=norm_l1, counters=cnt_f)
-                else:
-                    px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
-                if fused:
-                    B.gs_tile_ranges(sat, TW, TH, L, ranges)
-                elif expand:
-                    tk = clk.tic("expand")
-                    B.gs_expand_tiles(proj, bvals, branges, B.block_entries(bsat_np, L), L, TW, TH,
-                                      sat, I, vals, max(I, 1), ranges, bin_ws, st)
-                    clk.toc(tk)
-                else:
-                    tk = clk.tic("bin")
-                    B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1),
-                                   ranges, bin_ws, st)
-                    clk.toc(tk)
-                lb_bits = B.local_tile_bits(L)
-                if not expand and I > 0 and lb_bits > 0:
-                    tk = clk.tic("sort_tiles")
-                    B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
-                    clk.toc(tk)
-                tk = clk.tic("raster_fwd")
-                if fused:
-                    B.gs_raster_fwd_blocks(proj, bvals, branges, L, camS, px, vals, max(I, 1), I,
-                                           ranges, st, self.raster_flags)
-                else:
-                    B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
+            ls = torch.cuda.current_stream(dev)
+            up, freed, upload = hstate.get("up"), hstate.get("freed"), hstate.get("upload")
+            I = int(I)
+            sizes, (px0, py0, pw, ph) = leaf_sizes(L, I)
+            bufs, _ = _carve(arenas[li_k % len(arenas)], sizes)
+            lws = bin_wss[li_k % len(bin_wss)]
+            keys = bufs[0].view(torch.int32)
+            vals = bufs[1].view(torch.int32)
+            ranges = bufs[2].view(torch.int64)
+            sort_ws = bufs[3]
+            img = bufs[4].view(torch.float32)
+            Tf = bufs[5].view(torch.float32)
+            last = bufs[6].view(torch.int32)
+            dL = bufs[7].view(torch.float32)
+            if resident_target:
+                # the whole view's target is read in place with its own pitch
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=target,
+                              target_origin=(0, 0), target_pitch=W, target_plane=W * H,
+                              loss_tiles=loss_tiles, norm=norm_l1, counters=cnt_f)
+            elif host_target:
+                crop = crops[li_k % 2][:3 * pw * ph].view(3, ph, pw)
+                ls.wait_event(up[li_k])
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, target=crop,
+                              target_origin=(px0, py0), loss_tiles=loss_tiles,
+                              norm=norm_l1, counters=cnt_f)
+            else:
+                px = B.pixels(px0, py0, pw, ph, img, Tf, last, dL, counters=cnt_f)
+            if fused:
+                B.gs_tile_ranges(sat, TW, TH, L, ranges)
+            elif expand:
+                tk = clk.tic("expand")
+                B.gs_expand_tiles(proj, bvals, branges, B.block_entries(bsat_np, L), L, TW, TH,
+                                  sat, I, vals, max(I, 1), ranges, lws, st)
                 clk.toc(tk)
-                if ssim:
-                    # the Leaf's SSIM term: loss, and with the backward its
-                    # gradient added to the L1 part of dL
-                    tk = clk.tic("ssim")
-                    B.gs_loss_ssim(px, L, camS, self.ssim_lambda * norm,
-                                   bufs[8] if with_bwd else None)
-                    clk.toc(tk)
-                if host_target:
-                    ev = torch.cuda.Event()
-                    ev.record(ls)
-                    freed[li_k % 2] = ev
-                    if li_k + 2 < len(lv):
-                        upload(li_k + 2)
-                if hooks is not None and hasattr(hooks, "on_leaf"):
-                    hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
-                                            ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
-                                            n_isect=I, px_rect=(px0, py0, pw, ph)))
-                if with_bwd:
-                    if cnt_b is not None:
-                        px.counters = cnt_b.data_ptr()
-                    tk = clk.tic("raster_bwd")
-                    B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
-                    clk.toc(tk)
+            else:
+                tk = clk.tic("bin")
+                B.gs_bin_tiles(proj, C, order, drect, L, TW, TH, sat, I, keys, vals, max(I, 1),
+                               ranges, lws, st)
+                clk.toc(tk)
+            lb_bits = B.local_tile_bits(L)
+            if not expand and I > 0 and lb_bits > 0:
+                tk = clk.tic("sort_tiles")
+                B.gs_sort_tiles(keys, vals, I, ranges, (L[2] - L[0]) * (L[3] - L[1]), sort_ws, st)
+                clk.toc(tk)
+            tk = clk.tic("raster_fwd")
+            if fused:
+                B.gs_raster_fwd_blocks(proj, bvals, branges, L, camS, px, vals, max(I, 1), I,
+                                       ranges, st, self.raster_flags)
+            else:
+                B.gs_raster_fwd(proj, vals, ranges, L, camS, px, st, self.raster_flags)
+            clk.toc(tk)
+            if ssim:
+                # the Leaf's SSIM term: loss, and with the backward its
+                # gradient added to the L1 part of dL
+                tk = clk.tic("ssim")
+                B.gs_loss_ssim(px, L, camS, self.ssim_lambda * norm,
+                               bufs[8] if with_bwd else None)
+                clk.toc(tk)
+            if host_target:
+                ev = torch.cuda.Event()
+                ev.record(ls)
+                freed[li_k % 2] = ev
+                if li_k + 2 < len(lv):
+                    upload(li_k + 2)
+            if hooks is not None and hasattr(hooks, "on_leaf"):
+                hooks.on_leaf(ctx, dict(leaf=tuple(int(v) for v in L), keys=keys, vals=vals,
+                                        ranges=ranges, img=img, T_final=Tf, last=last, dL=dL,
+                                        n_isect=I, px_rect=(px0, py0, pw, ph)))
+            if with_bwd:
+                if cnt_b is not None:
+                    px.counters = cnt_b.data_ptr()
+                tk = clk.tic("raster_bwd")
+                B.gs_raster_bwd(proj, vals, ranges, L, camS, px, g2d, st, self.raster_flags)
+                clk.toc(tk)
 
         # SkipGS gate: the view's loss from a forward pass decides whether the
         # backward and the update run (then the Leaves are rendered again
@@ -507,7 +509,11 @@ class Stepper:
         else:
             leaf_pass(backward)
         if not original:
-            del arena, bin_ws  # raster buffers released before projection backward
+            # raster buffers released before projection backward (the main
+            # stream has waited for the Leaf stream, so the memory is free)
+            arenas.clear()
+            bin_wss.clear()
+            del arena, bin_ws
             if host_target:
                 del crops
 

@@ -808,6 +808,27 @@ def test_host_target_matches_resident_target(streams):
     assert np.abs(p1 - p0).max() <= 2.1e-3
 
 
+def test_two_leaf_streams_working_set():
+    """Two Leaves in flight hold at most one more Leaf arena than one Leaf at
+    a time, and both release the raster buffers before projection backward
+    (the same loss either way)."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    target = torch.as_tensor(synth.random_image(cam.width, cam.height, 6) * 0.5).cuda()
+    out = {}
+    for streams in (1, 2):
+        model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+        stp = Stepper(model, budget=6 << 20, leaf_streams=streams)
+        stats = stp.run_view(cam, target)
+        stp.check()
+        assert stats.n_leaves >= 3
+        out[streams] = (stats, stp.last_loss())
+    (s1, l1), (s2, l2) = out[1], out[2]
+    assert l1 == l2
+    arena = max(int(b) for b in s1.leaf_bytes)
+    assert s2.peak_ws_bytes <= s1.peak_ws_bytes + arena + (1 << 20)
+
+
 def test_leaf_invariance_gpu(oracle_mod):
     """Any Leaf partition: bit-identical image and loss, the same summed
     gradients (atomics reorder only)."""
