@@ -67,6 +67,9 @@ def parse():
     # CUDA-event times give the kernels' own durations when the timed region
     # overlaps Leaves
     ap.add_argument("--stage-steps", type=int, default=8)
+    # projection backward: the geometric chain as its own pass ("two_pass")
+    # or inside the Adam stream ("in_stream")
+    ap.add_argument("--fuse-adam", default="two_pass", choices=["two_pass", "in_stream"])
     ap.add_argument("--binning", default="fused", choices=["fused", "expand", "sort"])
     ap.add_argument("--loss", default="l1", choices=["l1", "l1_ssim"],
                     help="l1: the L1 photometric loss; l1_ssim: (1 - 0.2) L1 + 0.2 (1 - SSIM) "
@@ -397,7 +400,8 @@ def main():
     del jm, js
     model = GaussianModel(scene.params, scene.n, scene.sh_degree)
     stp = Stepper(model, budget=budget, raster_flags=a.raster_ppt, binning=a.binning,
-                  loss=a.loss, leaf_streams=a.leaf_streams)
+                  loss=a.loss, leaf_streams=a.leaf_streams,
+                  fuse_adam=True if a.fuse_adam == "two_pass" else "in_stream")
     nv = len(cams)
     view_of = lambda k: rank_view(k, rank, nv)
 
