@@ -1,7 +1,7 @@
 """Benchmark of one 3DGS training step (fwd + L1 + bwd + one Adam update per
 view, BoundedGS Leaf schedule) on the outdoor-like synthetic scene:
 6,000,000 Gaussians, SH degree 3, 5000x3300, 8 views on a circle, 384 MiB
-Leaf budget.
+Leaf budget, two Leaves in flight (--leaf-streams 1: one at a time).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
