@@ -971,10 +971,12 @@ def test_candidate_capacity_retry():
     assert (i0 == i1).all() and (l0 == l1).all() and s0 == s1
 
 
-def test_gated_step():
+@pytest.mark.parametrize("streams", [1, 2])
+def test_gated_step(streams):
     """run_view with a backward gate: a skipped step leaves the parameters
     and the optimizer untouched and reports the forward loss; an accepted
-    step equals the ungated one (the Leaves are rendered twice)."""
+    step equals the ungated one (the Leaves are rendered twice); with one or
+    two Leaf streams."""
     from gaussian_splatting_differentiable_dgs_b200.skipgs import BackwardGate
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, cam = scene("hd")
@@ -982,7 +984,7 @@ def test_gated_step():
     runs = {}
     for mode in ("plain", "skip", "take"):
         model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-        stp = Stepper(model, budget=3 << 20)
+        stp = Stepper(model, budget=3 << 20, leaf_streams=streams)
         gate = None if mode == "plain" else (lambda loss, m=mode: m == "take")
         stats = stp.run_view(cam, tgt, gate=gate)
         stp.check()

@@ -173,9 +173,10 @@ def test_ssim_identical_and_constant(oracle_mod):
     assert rel_l2(dL, grad) <= GRAD_L2
 
 
-@pytest.mark.parametrize("mode,budget", [("bounded", 60_000), ("bounded", 384 << 20),
-                                         ("original", 384 << 20)])
-def test_composite_loss_step(oracle_mod, mode, budget):
+@pytest.mark.parametrize("mode,budget,streams", [("bounded", 60_000, 1), ("bounded", 384 << 20, 1),
+                                                 ("original", 384 << 20, 1),
+                                                 ("bounded", 60_000, 2)])
+def test_composite_loss_step(oracle_mod, mode, budget, streams):
     """One training step with (1 - lambda) L1 + lambda (1 - SSIM) against the
     oracle's step with the same Leaves (SSIM windows local to each)."""
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
@@ -198,7 +199,8 @@ def test_composite_loss_step(oracle_mod, mode, budget):
             self.leaves = []
 
     model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=budget, fuse_adam=False, mode=mode, loss="l1_ssim")
+    stp = Stepper(model, budget=budget, fuse_adam=False, mode=mode, loss="l1_ssim",
+                  leaf_streams=streams)
     hk = Leaves()
     stats = stp.run_view(cam, torch.as_tensor(target).cuda(), hooks=hk)
     stp.check()
