@@ -126,3 +126,41 @@ def test_stepper_rejects_unknown_options():
                {"mode": "whole"}, {"loss": "l2"}):
         with pytest.raises(ValueError):
             Stepper(model, device="cpu", **kw)
+
+
+def test_step_roofline_properties():
+    """bench.step_roofline: each stage takes the larger of its HBM and ALU
+    times, the fraction is the roofline over the step time, and it responds
+    to the peaks and the step time as a roofline must."""
+    import types
+    import bench
+
+    a = types.SimpleNamespace(binning="fused", loss="l1")
+    model = types.SimpleNamespace(n=1_000_000, P=59)
+    st = types.SimpleNamespace(n_cand=800_000, n_isect=50_000_000, n_block_entries=3_000_000,
+                               n_block_reads=0, n_leaves=2)
+    acc = types.SimpleNamespace(n_isect=50_000_000)
+    per_step = {"project": 0.2, "raster_bwd": 0.5, "project_bwd": 0.4}
+    peaks = {"hbm_gbs": 6000.0}
+    alu = 37e12
+
+    def run(peaks, alu, step_ms, ops_bwd=4e10):
+        return bench.step_roofline(a, model, [st], acc, 1e10, ops_bwd, per_step, peaks, alu,
+                                   2000, 1000, step_ms)
+
+    r = run(peaks, alu, 2.0)
+    s = r["stages"]
+    for name, v in s.items():
+        t_hbm = v["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e3
+        t_alu = v["lane_ops"] / alu * 1e3
+        assert abs(v["roofline_ms"] - max(t_hbm, t_alu)) <= 1e-4
+        assert v["bound"] == ("alu" if t_alu > t_hbm else "hbm")
+    assert s["raster_bwd"]["bound"] == "alu" and s["project_bwd"]["bound"] == "hbm"
+    assert abs(r["roofline_ms"] - sum(v["roofline_ms"] for v in s.values())) <= 1e-3
+    assert abs(r["frac"] - r["roofline_ms"] / 2.0) <= 1e-4
+    assert abs(run(peaks, alu, 4.0)["frac"] - r["frac"] / 2) <= 1e-4
+    # twice the bandwidth halves every HBM-bound stage's roofline time
+    r2 = run({"hbm_gbs": 12000.0}, alu, 2.0)
+    assert abs(r2["stages"]["project_bwd"]["roofline_ms"] * 2
+               - s["project_bwd"]["roofline_ms"]) <= 1e-3
+    assert r2["stages"]["raster_bwd"]["roofline_ms"] == s["raster_bwd"]["roofline_ms"]
