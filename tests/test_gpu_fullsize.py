@@ -67,9 +67,9 @@ def test_full_size_step_sampled(oracle_mod):
     TW, TH = O.grid(cam)
     target = (synth.random_image(W, H, 11) * 0.6).astype(np.float32)
 
-    # ---- the GPU step, as bench.py runs it ----------------------------------
+    # ---- the GPU step, as bench.py runs it (two Leaves in flight) ------------
     model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=384 << 20)
+    stp = Stepper(model, budget=384 << 20, leaf_streams=2)
     grab = Grab(W, H)
     stats = stp.run_view(cam, torch.as_tensor(target).cuda(), hooks=grab)
     stp.check()
