@@ -124,7 +124,17 @@ class _Timer:
 class Stepper:
     """Runs the per-view step.  `hooks` (optional) is an object whose methods
     `on_project(ctx)`, `on_leaf(ctx, leaf_ctx)`, `on_bwd(ctx)` see
-    intermediate buffers (used by the parity tests)."""
+    intermediate buffers (used by the parity tests).
+
+    Options: budget (bytes per Leaf), Adam's lr / betas / eps, raster_flags
+    (pixels per thread of the raster kernels, 0 = their defaults), fuse_adam
+    (True: projection backward fused with Adam, geometric chain as its own
+    pass; "in_stream": the chain inside the Adam stream; False: compact 3D
+    gradients and a separate Adam), binning ("fused", "expand", "sort": the
+    three list builders), mode ("bounded" or the whole-image "original"),
+    loss ("l1" or "l1_ssim" with weight ssim_lambda), leaf_streams (1: one
+    Leaf at a time; 2: consecutive Leaves on two streams with two raster
+    arenas)."""
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
                  betas=(0.9, 0.999), eps=1e-8, raster_flags=0, fuse_adam=True,
