@@ -240,17 +240,8 @@ struct BlockSrc {
 // Leaf's vals; the hits are then staged and composited NT at a time.
 constexpr int kFillU = 2;
 
-// CTAs per SM the raster kernels' register budgets are sized for (forward
-// with 2 pixels per thread, backward with 4), overridable for tuning sweeps
-#ifndef GS_FWD_MINB
-#define GS_FWD_MINB 8
-#endif
-#ifndef GS_BWD_MINB
-#define GS_BWD_MINB 14
-#endif
-
 template <int PPT, bool COUNT, bool BLK>
-__global__ void __launch_bounds__(256 / PPT, PPT == 2 ? GS_FWD_MINB : 1)
+__global__ void __launch_bounds__(256 / PPT, PPT == 2 ? 8 : 1)
 k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* ranges, gs_rect leaf, int W, int H, int TW, PixArgs px,
              BlockSrc bsrc, int32_t* dev_status) {
@@ -561,7 +552,7 @@ __device__ __forceinline__ float warp_reduce9_smem(const float (&v)[9], float* _
 }
 
 template <int PPT, bool COUNT>
-__global__ void __launch_bounds__(256 / PPT, PPT == 4 ? GS_BWD_MINB : 1)
+__global__ void __launch_bounds__(256 / PPT, PPT == 4 ? 14 : 1)
 k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              const int64_t* __restrict__ ranges, gs_rect leaf, int W, int H, PixArgs px,
              float* __restrict__ g2d, int32_t* dev_status) {
