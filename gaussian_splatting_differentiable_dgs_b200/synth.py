@@ -249,6 +249,32 @@ def tiny_scene(n: int = 8, width: int = 48, height: int = 40, sh_degree: int = 0
     return Scene(params, n, sh_degree), [axis_camera(f, width, height)]
 
 
+def edge_needle_scene(n: int = 48, width: int = 96, height: int = 80,
+                      sh_degree: int = 3, seed: int = 0, opacity=(0.02, 0.999)):
+    """Needle-thin anisotropic Gaussians around the image border: one local
+    axis 8-40 px long, the other two 0.2-0.6 px, random orientations; means
+    within 6 px of a random border on either side of it, identity camera."""
+    rng = np.random.default_rng(seed)
+    f = 60.0
+    z = rng.uniform(2.0, 4.0, n)
+    side = rng.integers(0, 4, n)
+    along = rng.uniform(0.0, 1.0, n)
+    across = rng.uniform(-6.0, 6.0, n)
+    px = np.where(side == 0, across, np.where(side == 1, width + across, along * width))
+    py = np.where(side == 2, across, np.where(side == 3, height + across, along * height))
+    mean = np.stack([(px - width / 2) * z / f, (py - height / 2) * z / f, z], 1)
+    sig_px = np.stack([rng.uniform(8.0, 40.0, n), rng.uniform(0.2, 0.6, n),
+                       rng.uniform(0.2, 0.6, n)], 1)
+    log_scale = np.log(sig_px * z[:, None] / f)
+    quat = _unit_quats(rng, n)
+    o = rng.uniform(opacity[0], opacity[1], n)
+    logit = np.log(o / (1 - o))
+    colour = rng.uniform(0.05, 0.95, size=(n, 3))
+    params = _fill(_empty(n, sh_degree), n, sh_degree, mean, log_scale, quat,
+                   logit, colour, rng, sh_rest_sigma=0.1)
+    return Scene(params, n, sh_degree), [axis_camera(f, width, height)]
+
+
 def jittered(scene: Scene, seed: int, mean_sigma=0.02, colour_sigma=0.05) -> Scene:
     """Copy of `scene` with means + N(0, mean_sigma) and the degree-0 colour
     + N(0, colour_sigma) (higher SH bands untouched)."""

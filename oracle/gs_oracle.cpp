@@ -153,8 +153,10 @@ struct Forward3D {
 };
 
 // Cull + EWA projection of Gaussian i (cull rules and constants: readings).
+// `tight` selects the rect: the tiles of the 3-sigma square that meet the
+// alpha >= 1/255 box (the library's binning), or the plain square.
 void project_one(const double* params, int64_t n_pad, int32_t D, const Cam& k,
-                 int32_t W, int32_t H, int64_t i, Forward3D& f) {
+                 int32_t W, int32_t H, int64_t i, Forward3D& f, bool tight) {
   const int TW = (W + kTile - 1) / kTile, TH = (H + kTile - 1) / kTile;
   auto P = [&](int plane) { return params[(int64_t)plane * n_pad + i]; };
   f.cand = false;
@@ -237,23 +239,31 @@ void project_one(const double* params, int64_t n_pad, int32_t D, const Cam& k,
   // Reading: a tile outside it would skip the Gaussian at every pixel, so
   // the image and gradients are those of the plain square.
   f.opac = 1.0 / (1.0 + std::exp(-P(10)));
-  double lq = std::log(255.0 * f.opac);
-  if (std::fabs(lq + 1e-4) <= 1e-9) f.flags |= OR_F_RADIUS_NEAR;
-  if (!(lq > -1e-4)) return;  // alpha never reaches 1/255
-  double qb = std::max(lq, 0.0) * 1.0001 + 1e-4;
-  double hx = std::sqrt(2.0 * qb * f.S2p[0]) + 0.01;
-  double hy = std::sqrt(2.0 * qb * f.S2p[2]) + 0.01;
-  double e[4] = {(f.u - hx - 15.5) / kTile, (f.v - hy - 15.5) / kTile,
-                 (f.u + hx - 0.5) / kTile, (f.v + hy - 0.5) / kTile};
-  for (double x : e)
-    if (std::fabs(x - std::nearbyint(x)) <= 1e-9 * std::max(1.0, std::fabs(x)))
-      f.flags |= OR_F_RADIUS_NEAR;
-  int64_t bb[4] = {(int64_t)std::ceil(e[0]), (int64_t)std::ceil(e[1]),
-                   (int64_t)std::floor(e[2]) + 1, (int64_t)std::floor(e[3]) + 1};
-  f.rect[0] = clampi(std::max(sq[0], bb[0]), 0, TW);
-  f.rect[1] = clampi(std::max(sq[1], bb[1]), 0, TH);
-  f.rect[2] = clampi(std::min(sq[2], bb[2]), 0, TW);
-  f.rect[3] = clampi(std::min(sq[3], bb[3]), 0, TH);
+  if (tight) {
+    double lq = std::log(255.0 * f.opac);
+    if (std::fabs(lq + 1e-4) <= 1e-9) f.flags |= OR_F_RADIUS_NEAR;
+    if (!(lq > -1e-4)) return;  // alpha never reaches 1/255
+    double qb = std::max(lq, 0.0) * 1.0001 + 1e-4;
+    double hx = std::sqrt(2.0 * qb * f.S2p[0]) + 0.01;
+    double hy = std::sqrt(2.0 * qb * f.S2p[2]) + 0.01;
+    double e[4] = {(f.u - hx - 15.5) / kTile, (f.v - hy - 15.5) / kTile,
+                   (f.u + hx - 0.5) / kTile, (f.v + hy - 0.5) / kTile};
+    for (double x : e)
+      if (std::fabs(x - std::nearbyint(x)) <= 1e-9 * std::max(1.0, std::fabs(x)))
+        f.flags |= OR_F_RADIUS_NEAR;
+    int64_t bb[4] = {(int64_t)std::ceil(e[0]), (int64_t)std::ceil(e[1]),
+                     (int64_t)std::floor(e[2]) + 1, (int64_t)std::floor(e[3]) + 1};
+    f.rect[0] = clampi(std::max(sq[0], bb[0]), 0, TW);
+    f.rect[1] = clampi(std::max(sq[1], bb[1]), 0, TH);
+    f.rect[2] = clampi(std::min(sq[2], bb[2]), 0, TW);
+    f.rect[3] = clampi(std::min(sq[3], bb[3]), 0, TH);
+  } else {
+    // the plain closed 3-sigma square, clamped to the grid
+    f.rect[0] = clampi(sq[0], 0, TW);
+    f.rect[1] = clampi(sq[1], 0, TH);
+    f.rect[2] = clampi(sq[2], 0, TW);
+    f.rect[3] = clampi(sq[3], 0, TH);
+  }
   if (f.rect[0] >= f.rect[2] || f.rect[1] >= f.rect[3]) return;
   // view-dependent colour from SH at the direction camera centre -> mean
   double cc[3];
@@ -369,16 +379,16 @@ void or_sh_basis(const double* d, double* Y, double* dY) {
   sh_eval(d[0], d[1], d[2], Y, dY);
 }
 
-int64_t or_project(const double* params, int64_t n, int64_t n_pad, int32_t D,
-                   const double* cam, int32_t W, int32_t H, uint8_t* is_cand,
-                   double* rec, int32_t* rect, uint32_t* depth_key,
-                   uint8_t* flags) {
+int64_t or_project_rects(const double* params, int64_t n, int64_t n_pad,
+                         int32_t D, const double* cam, int32_t W, int32_t H,
+                         int32_t tight, uint8_t* is_cand, double* rec,
+                         int32_t* rect, uint32_t* depth_key, uint8_t* flags) {
   Cam k = load_cam(cam);
   int64_t count = 0;
 #pragma omp parallel for schedule(static) reduction(+ : count)
   for (int64_t i = 0; i < n; ++i) {
     Forward3D f;
-    project_one(params, n_pad, D, k, W, H, i, f);
+    project_one(params, n_pad, D, k, W, H, i, f, tight != 0);
     is_cand[i] = f.cand ? 1 : 0;
     flags[i] = f.flags;
     double* r = rec + i * OR_REC;
@@ -400,6 +410,14 @@ int64_t or_project(const double* params, int64_t n, int64_t n_pad, int32_t D,
     depth_key[i] = bits;
   }
   return count;
+}
+
+int64_t or_project(const double* params, int64_t n, int64_t n_pad, int32_t D,
+                   const double* cam, int32_t W, int32_t H, uint8_t* is_cand,
+                   double* rec, int32_t* rect, uint32_t* depth_key,
+                   uint8_t* flags) {
+  return or_project_rects(params, n, n_pad, D, cam, W, H, 1, is_cand, rec,
+                          rect, depth_key, flags);
 }
 
 int64_t or_tile_lists_scan(int64_t C, const int32_t* rect, const uint32_t* key,

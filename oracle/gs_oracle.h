@@ -49,6 +49,15 @@ int64_t or_project(const double* params, int64_t n, int64_t n_pad, int32_t D,
                    double* rec, int32_t* rect, uint32_t* depth_key,
                    uint8_t* flags);
 
+/* The same with the rect chosen by `tight`: 1 = the tiles of the 3-sigma
+ * square whose pixel-centre box meets the inflated alpha >= 1/255 box (and
+ * Gaussians that cannot reach 1/255 culled), as or_project; 0 = the plain
+ * closed 3-sigma square clamped to the grid. */
+int64_t or_project_rects(const double* params, int64_t n, int64_t n_pad,
+                         int32_t D, const double* cam, int32_t W, int32_t H,
+                         int32_t tight, uint8_t* is_cand, double* rec,
+                         int32_t* rect, uint32_t* depth_key, uint8_t* flags);
+
 /* Real SH basis (degree <= 3, 16 values) and its gradient (16 x 3) at a unit
  * direction d. */
 void or_sh_basis(const double* d, double* Y, double* dY);

@@ -75,6 +75,9 @@ def lib():
         i64, i32 = C.c_int64, C.c_int32
         L.or_project.restype = i64
         L.or_project.argtypes = [p, i64, i64, i32, p, i32, i32, p, p, p, p, p]
+        L.or_project_rects.restype = i64
+        L.or_project_rects.argtypes = [p, i64, i64, i32, p, i32, i32, i32, p,
+                                       p, p, p, p]
         L.or_sh_basis.argtypes = [p, p, p]
         L.or_tile_lists_scan.restype = i64
         L.or_tile_lists_scan.argtypes = [i64, p, p, i32, p, i64, p, p]
@@ -116,9 +119,13 @@ def grid(cam):
 # stage wrappers
 # ---------------------------------------------------------------------------
 
-def project(params: np.ndarray, n: int, sh_degree: int, cam):
+def project(params: np.ndarray, n: int, sh_degree: int, cam, tight=True):
     """Cull + project all Gaussians.  Returns per-Gaussian arrays and the
-    candidate view (ascending Gaussian index)."""
+    candidate view (ascending Gaussian index).  `tight` selects the tile
+    rect: the tiles of the 3-sigma square that meet the alpha >= 1/255 box
+    (the binning the library uses), or with False the plain closed 3-sigma
+    square, in which case a Gaussian that can never reach 1/255 is still a
+    candidate."""
     par = np.ascontiguousarray(params, np.float64)
     n_pad = par.shape[1]
     is_c = np.zeros(n, np.uint8)
@@ -127,8 +134,9 @@ def project(params: np.ndarray, n: int, sh_degree: int, cam):
     key = np.zeros(n, np.uint32)
     flags = np.zeros(n, np.uint8)
     ca = cam_array(cam)
-    lib().or_project(_p(par), n, n_pad, sh_degree, _p(ca), cam.width,
-                     cam.height, _p(is_c), _p(rec), _p(rect), _p(key), _p(flags))
+    lib().or_project_rects(_p(par), n, n_pad, sh_degree, _p(ca), cam.width,
+                           cam.height, 1 if tight else 0, _p(is_c), _p(rec),
+                           _p(rect), _p(key), _p(flags))
     cand = np.nonzero(is_c)[0].astype(np.int32)
     return dict(is_cand=is_c.astype(bool), rec_all=rec, rect_all=rect,
                 key_all=key, flags_all=flags, cand_idx=cand, rec=rec[cand],
@@ -416,16 +424,21 @@ def render(params, n, sh_degree, cam):
 
 
 def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
-         lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, t=1, ssim_lambda=None):
+         lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, t=1, ssim_lambda=None,
+         tight=True):
     """One training step for one view: project, per-Leaf raster forward +
     loss + raster backward (summed over Leaves), projection backward, one
     Adam update.  `leaves` is a list of tile rects; None = whole image.
     The loss is L1, or with `ssim_lambda` the composite
     (1 - lambda) L1 + lambda (1 - SSIM), SSIM over each Leaf's pixel
-    rectangle (loss_ssim), both normalised by 3 W H."""
+    rectangle (loss_ssim), both normalised by 3 W H.  `tight` is passed to
+    `project`.  Besides the list position `last`, the result holds
+    `last_id`: the Gaussian index of each pixel's last composited entry
+    (-1 if none), which does not depend on which skipped entries a list
+    holds."""
     W, H = cam.width, cam.height
     TW, TH = grid(cam)
-    pr = project(params, n, sh_degree, cam)
+    pr = project(params, n, sh_degree, cam, tight=tight)
     if leaves is None:
         leaves = [(0, 0, TW, TH)]
     Cn = len(pr["cand_idx"])
@@ -435,6 +448,7 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
     img = np.zeros((3, TH * 16, TW * 16))
     Tfin = np.ones((TH * 16, TW * 16))
     last = np.zeros((TH * 16, TW * 16), np.int32)
+    last_id = np.full((TH * 16, TW * 16), -1, np.int64)
     pflags = np.zeros((TH * 16, TW * 16), np.uint8)
     n_eval = 0
     n_isect = 0
@@ -474,6 +488,11 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
             img[(slice(None),) + sl] = fw["img"][j].reshape(3, 16, 16)
             Tfin[sl] = fw["T"][j].reshape(16, 16)
             last[sl] = fw["last"][j].reshape(16, 16)
+            lj = fw["last"][j].astype(np.int64)
+            lid = np.full(256, -1, np.int64)
+            hit = lj > 0
+            lid[hit] = pr["cand_idx"][vals[off[j] + lj[hit] - 1]]
+            last_id[sl] = lid.reshape(16, 16)
             pflags[sl] = fw["flags"][j].reshape(16, 16)
     g3d = project_bwd(params, sh_degree, cam, pr["cand_idx"], g2d)
     P, n_pad = params.shape
@@ -488,7 +507,8 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
     m_new[:, n:] = 0
     v_new[:, n:] = 0
     return dict(proj=pr, g2d=g2d, grad=grad, loss=loss, img=img[:, :H, :W],
-                T=Tfin[:H, :W], last=last[:H, :W], pflags=pflags[:H, :W],
+                T=Tfin[:H, :W], last=last[:H, :W], last_id=last_id[:H, :W],
+                pflags=pflags[:H, :W],
                 params=p_new, m=m_new, v=v_new, n_eval=n_eval,
                 n_isect=n_isect)
 

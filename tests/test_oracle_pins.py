@@ -199,67 +199,173 @@ def test_cull_rules(oracle_mod):
         assert oracle_mod.project(p, 1, 0, cam)["is_cand"][0] == expect, mean
 
 
-def _alpha_box(rec):
-    """Half extents of the inflated alpha >= 1/255 box (the reading's bound)."""
-    lq = np.log(255.0 * rec[:, 7])
-    q = np.maximum(lq, 0.0) * 1.0001 + 1e-4
-    return np.sqrt(2 * q * rec[:, 11]) + 0.01, np.sqrt(2 * q * rec[:, 13]) + 0.01
+def _square_bruteforce(u, v, r, TW, TH):
+    """Tiles (tx, ty) of the grid that meet the closed square [u-r, u+r] x
+    [v-r, v+r], by enumeration."""
+    return {(tx, ty) for ty in range(TH) for tx in range(TW)
+            if tx * 16 <= u + r and (tx + 1) * 16 > u - r
+            and ty * 16 <= v + r and (ty + 1) * 16 > v - r}
 
 
-def test_rect_and_depth_key_bruteforce(oracle_mod):
-    sc, cams = synth.tiny_oracle_scene(0)
+def _alpha_at_centres(rec, tiles, W, H):
+    """alpha = min(0.99, o exp(-q)) of one record at every in-image pixel
+    centre of the given tiles, with q = (a dx^2 + c dy^2)/2 + b dx dy,
+    d = mean - centre (the compositing definition, evaluated directly)."""
+    out = []
+    for tx, ty in tiles:
+        ys, xs = np.mgrid[ty * 16:ty * 16 + 16, tx * 16:tx * 16 + 16]
+        keep = (xs < W) & (ys < H)
+        dx = rec[0] - (xs[keep] + 0.5)
+        dy = rec[1] - (ys[keep] + 0.5)
+        q = 0.5 * (rec[4] * dx * dx + rec[6] * dy * dy) + rec[5] * dx * dy
+        out.append(np.minimum(0.99, rec[7] * np.exp(-q)))
+    return np.concatenate(out) if out else np.zeros(0)
+
+
+def _rect_tiles(r):
+    return {(tx, ty) for ty in range(r[1], r[3]) for tx in range(r[0], r[2])}
+
+
+def _pin_scenes():
+    """Seeded scenes for the rect pins: SH degree 3 spread, large splats,
+    opacities near the 0.99 clamp, opacities around 1/255, needle-thin
+    Gaussians across the image border, and the 2,000-Gaussian scene."""
+    return {
+        "sh3_spread": synth.tiny_scene(n=60, width=96, height=80, sh_degree=3, seed=0,
+                                       scale_px=(1.0, 9.0), opacity=(0.01, 0.99)),
+        "sh3_large": synth.tiny_scene(n=40, width=80, height=64, sh_degree=3, seed=1,
+                                      scale_px=(3.0, 14.0), opacity=(0.05, 0.95)),
+        "near_clamp": synth.tiny_scene(n=60, width=80, height=64, sh_degree=3, seed=2,
+                                       scale_px=(3.0, 10.0), opacity=(0.97, 0.9999)),
+        "near_skip": synth.tiny_scene(n=80, width=80, height=64, sh_degree=0, seed=3,
+                                      scale_px=(1.0, 8.0), opacity=(0.0025, 0.008)),
+        "needles_edge": synth.edge_needle_scene(n=48, width=96, height=80, seed=4),
+        "needles_edge_faint": synth.edge_needle_scene(n=48, width=96, height=80, seed=5,
+                                                      opacity=(0.003, 0.05)),
+        "tiny_2k": synth.tiny_oracle_scene(0),
+    }
+
+
+@pytest.mark.parametrize("name", list(_pin_scenes()))
+def test_rects_and_removed_tiles_bruteforce(oracle_mod, name):
+    """The plain rect is the 3-sigma square by enumeration; the tight rect
+    lies inside it; every tile the tight rect drops (all of the square for a
+    Gaussian the tight projection culls) has alpha below 1/255 at every
+    in-image pixel centre, with a margin far above fp32 rounding.  The
+    depth key is the fp32 bit pattern of t_z; records do not depend on the
+    rect mode."""
+    sc, cams = _pin_scenes()[name]
     cam = cams[0]
-    pr = oracle_mod.project(sc.params, sc.n, 0, cam)
+    W, H = cam.width, cam.height
     TW, TH = oracle_mod.grid(cam)
-    rec, rect = pr["rec"], pr["rect"]
-    hx, hy = _alpha_box(rec)
-    for j in range(0, len(rec), 7):
-        u, v, r = rec[j, 0], rec[j, 1], rec[j, 3]
-        # tiles meeting the closed 3-sigma square AND whose pixel-centre box
-        # meets the alpha box
-        tiles = [(tx, ty) for ty in range(TH) for tx in range(TW)
-                 if tx * 16 <= u + r and (tx + 1) * 16 > u - r
-                 and ty * 16 <= v + r and (ty + 1) * 16 > v - r
-                 and tx * 16 + 0.5 <= u + hx[j] and tx * 16 + 15.5 >= u - hx[j]
-                 and ty * 16 + 0.5 <= v + hy[j] and ty * 16 + 15.5 >= v - hy[j]]
-        xs = [a for a, _ in tiles]
-        ys = [b for _, b in tiles]
-        assert (rect[j] == [min(xs), min(ys), max(xs) + 1, max(ys) + 1]).all()
-        assert len(tiles) == (rect[j, 2] - rect[j, 0]) * (rect[j, 3] - rect[j, 1])
-        square = [(tx, ty) for ty in range(TH) for tx in range(TW)
-                  if tx * 16 <= u + r and (tx + 1) * 16 > u - r
-                  and ty * 16 <= v + r and (ty + 1) * 16 > v - r]
-        assert rec[j, 14] == len(square)
-    keys = np.float32(rec[:, 2]).view(np.uint32)
-    assert (keys == pr["key"]).all()
-    # candidates = the Gaussians that pass; ascending index
-    assert (np.diff(pr["cand_idx"]) > 0).all()
+    p = sc.params.astype(np.float64)
+    tight = oracle_mod.project(p, sc.n, sc.sh_degree, cam, tight=True)
+    sq = oracle_mod.project(p, sc.n, sc.sh_degree, cam, tight=False)
+    assert not (tight["is_cand"] & ~sq["is_cand"]).any()
+    worst = 0.0
+    n_removed = 0
+    for g in np.nonzero(sq["is_cand"])[0]:
+        rec = sq["rec_all"][g]
+        square = _square_bruteforce(rec[0], rec[1], rec[3], TW, TH)
+        assert square == _rect_tiles(sq["rect_all"][g])
+        assert rec[14] == len(square)
+        if tight["is_cand"][g]:
+            assert (tight["rec_all"][g] == rec).all()
+            assert tight["key_all"][g] == sq["key_all"][g]
+            kept = _rect_tiles(tight["rect_all"][g])
+            assert kept <= square
+        else:
+            kept = set()
+        removed = square - kept
+        n_removed += len(removed)
+        a = _alpha_at_centres(rec, sorted(removed), W, H)
+        if a.size:
+            worst = max(worst, float(a.max()) * 255.0)
+    assert n_removed > 0
+    # the inflation of the alpha box (1e-4 in q) leaves every removed pixel
+    # at least ~1e-4 relative below the threshold
+    assert worst < 1.0 - 5e-5, worst
+    keys = np.float32(sq["rec"][:, 2]).view(np.uint32)
+    assert (keys == sq["key"]).all()
+    assert (np.diff(sq["cand_idx"]) > 0).all() and (np.diff(tight["cand_idx"]) > 0).all()
 
 
-@pytest.mark.parametrize("seed", [0, 1])
-def test_tight_rect_leaves_image_unchanged(oracle_mod, seed):
-    """Reading: dropping the tiles of the 3-sigma square that the alpha box
-    misses changes neither image nor transmittance (those tiles skip the
-    Gaussian at every pixel); only the list positions (`last`) move."""
-    sc, cams = synth.tiny_scene(n=60, width=96, height=80, sh_degree=3, seed=seed,
-                                scale_px=(1.0, 9.0), opacity=(0.01, 0.99))
+@pytest.mark.parametrize("name", list(_pin_scenes()))
+def test_tight_rects_give_the_plain_square_step(oracle_mod, name):
+    """Reading (tight tile rects): binning each candidate into only the
+    tiles of its 3-sigma square that meet its alpha >= 1/255 box, and culling
+    the Gaussians that cannot reach 1/255, gives the step of the plain
+    3-sigma-square binning: the same image, transmittance, last composited
+    Gaussian per pixel, loss, 2D gradients (zero for every Gaussian the
+    tight binning drops), 3D gradients and Adam update.  Checked with two
+    Leaves and a non-trivial Adam state (t = 5), so that the update depends
+    on the gradient's magnitude."""
+    sc, cams = _pin_scenes()[name]
     cam = cams[0]
+    W, H = cam.width, cam.height
     TW, TH = oracle_mod.grid(cam)
-    pr = oracle_mod.project(sc.params.astype(np.float64), sc.n, 3, cam)
-    rec = pr["rec"]
-    u, v, r = rec[:, 0], rec[:, 1], rec[:, 3]
-    square = np.stack([np.floor((u - r) / 16), np.floor((v - r) / 16),
-                       np.floor((u + r) / 16) + 1, np.floor((v + r) / 16) + 1], 1)
-    square = np.clip(square, 0, [TW, TH, TW, TH]).astype(np.int32)
-    assert ((pr["rect"][:, :2] >= square[:, :2]) & (pr["rect"][:, 2:] <= square[:, 2:])).all()
-    tiles = np.arange(TW * TH, dtype=np.int32)
-    outs = []
-    for rc in (pr["rect"], square):
-        off, vals = oracle_mod.tile_lists(rc, pr["key"], TW, tiles)
-        outs.append((len(vals), oracle_mod.raster_fwd(rec, TW, cam.width, cam.height, tiles, off, vals)))
-    (n_tight, a), (n_sq, b) = outs
-    assert n_tight < n_sq
+    p = sc.params.astype(np.float64)
+    target = synth.random_image(W, H, seed=11).astype(np.float64)
+    rng = np.random.default_rng(12)
+    m0 = rng.normal(0, 1e-3, p.shape)
+    v0 = rng.uniform(0, 1e-6, p.shape)
+    m0[:, sc.n:] = 0
+    v0[:, sc.n:] = 0
+    leaves = [(0, 0, TW // 2, TH), (TW // 2, 0, TW, TH)]
+    a = oracle_mod.step(p, sc.n, sc.sh_degree, cam, target, leaves=leaves,
+                        m=m0, v=v0, t=5, tight=True)
+    b = oracle_mod.step(p, sc.n, sc.sh_degree, cam, target, leaves=leaves,
+                        m=m0, v=v0, t=5, tight=False)
+    assert a["n_isect"] < b["n_isect"]
     assert (a["img"] == b["img"]).all() and (a["T"] == b["T"]).all()
+    assert (a["last_id"] == b["last_id"]).all()
+    assert (a["last_id"] >= 0).any()
+    assert abs(a["loss"] - b["loss"]) <= 1e-14 * abs(b["loss"])
+    # 2D gradients: per candidate of the tight binning equal, zero elsewhere
+    ca, cb = a["proj"]["cand_idx"], b["proj"]["cand_idx"]
+    pos = np.searchsorted(cb, ca)
+    assert (cb[pos] == ca).all()
+    g_sq = b["g2d"]
+    scale = np.abs(g_sq).max()
+    assert scale > 0
+    assert np.abs(a["g2d"] - g_sq[pos]).max() <= 1e-12 * scale
+    dropped = np.ones(len(cb), bool)
+    dropped[pos] = False
+    assert (g_sq[dropped] == 0).all()
+    # dense 3D gradients and the Adam update
+    gs = np.abs(b["grad"]).max()
+    assert np.abs(a["grad"] - b["grad"]).max() <= 1e-12 * gs
+    for key in ("params", "m", "v"):
+        ref = b[key]
+        assert np.abs(a[key] - ref).max() <= 1e-12 * max(np.abs(ref).max(), 1e-30), key
+
+
+def test_pin_scenes_reach_the_thresholds(oracle_mod):
+    """The rect pins' scenes do exercise the decisions the tight rects
+    touch: the 0.99 clamp, Gaussians under 1/255 everywhere, the T stop, and
+    needles that cross the image border."""
+    sc_ = _pin_scenes()
+    hit = {}
+    for name in ("near_clamp", "near_skip", "needles_edge", "sh3_large"):
+        sc, cams = sc_[name]
+        cam = cams[0]
+        p = sc.params.astype(np.float64)
+        tight = oracle_mod.project(p, sc.n, sc.sh_degree, cam, tight=True)
+        sq = oracle_mod.project(p, sc.n, sc.sh_degree, cam, tight=False)
+        r = oracle_mod.render(p, sc.n, sc.sh_degree, cam)
+        o = sq["rec"][:, 7]
+        hit[name] = dict(n_faint=int((o < 1 / 255).sum()),
+                         n_culled=int(sq["is_cand"].sum() - tight["is_cand"].sum()),
+                         clamp=bool((o > 0.99).any()),
+                         # a pixel stopped iff it visited fewer entries than its list
+                         stop=bool((r["fwd"]["n_eval"] < np.diff(r["off"])[:, None])
+                                   [(r["fwd"]["flags"] & oracle_mod.P_INVALID) == 0].any()),
+                         cross=int(((sq["rec"][:, 0] < 0) | (sq["rec"][:, 0] > cam.width)
+                                    | (sq["rec"][:, 1] < 0) | (sq["rec"][:, 1] > cam.height)).sum()))
+    assert hit["near_clamp"]["clamp"]
+    assert hit["near_skip"]["n_faint"] > 0 and hit["near_skip"]["n_culled"] > 0
+    assert hit["needles_edge"]["cross"] > 0
+    assert hit["near_clamp"]["stop"]
 
 
 # ---------------------------------------------------------------------------
