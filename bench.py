@@ -92,7 +92,7 @@ def workload_name(a):
             f"SH3, {a.views} views on a radius-4 circle, {a.budget_mib:g} MiB Leaf budget")
 
 
-def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_peak, W, H,
+def step_roofline(a, model, stats, ops_fwd, ops_bwd, per_step, peaks, alu_peak, W, H,
                   step_ms):
     """Roofline time of the step: for each stage the larger of its compulsory
     HBM bytes / measured copy bandwidth and its lane-ops / ALU issue peak,
@@ -120,8 +120,8 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
                    (g2d, record, fp64 geometric scratch) + N*4 (slot map)
     (E_blk = block-list entries, R_blk = their reads over the Leaves, I =
     tile-list entries, C = candidates, N = Gaussians.)  The raster stages'
-    lane-ops are E k (K_FWD, K_BWD) from the accounting view, scaled to each
-    view's I."""
+    lane-ops are E k (K_FWD, K_BWD), E counted on the same views the stage
+    times are averaged over."""
     hbm = peaks["hbm_gbs"] * 1e9
     n, P = model.n, model.P
     k = len(stats)
@@ -141,8 +141,7 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
         "raster_bwd": C * 96 + px * 20,
         "project_bwd": n * P * 24 + C * 208 + n * 4,
     }
-    scale = I / max(acc.n_isect, 1)
-    ops = {"raster_fwd": ops_fwd * scale, "raster_bwd": ops_bwd * scale}
+    ops = {"raster_fwd": ops_fwd, "raster_bwd": ops_bwd}
     if a.loss == "l1_ssim":
         byt["ssim"] = px * 48
         ops["ssim"] = px * 3 * K_SSIM
@@ -159,6 +158,16 @@ def step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks, alu_p
     return {"roofline_ms": round(total, 4), "stages_ms": round(measured, 4),
             "step_ms": round(step_ms, 4),
             "frac": round(total / step_ms, 4) if step_ms > 0 else None, "stages": stages}
+
+
+def alu_roofline(kernel, lane_ops, stage_ms, alu_peak):
+    """Roofline of an issue-bound kernel: achieved = its algorithmic lane-ops
+    per step / its device time per step, against the ALU issue peak.  The
+    same lane-ops enter the step roofline's stage, so the two agree."""
+    ach = lane_ops / (stage_ms / 1e3) / 1e12
+    return {"bound": "alu", "kernel": kernel, "achieved": round(ach, 3),
+            "peak": round(alu_peak / 1e12, 3), "unit": "Tlane-op/s",
+            "frac": round(ach / (alu_peak / 1e12), 4), "lane_ops_per_step": round(lane_ops)}
 
 
 def profile_traffic(kernel):
@@ -440,6 +449,7 @@ def main():
     value = isect_all / (ms_max / 1e3)
     n_steps = a.steps
     stage_src = "timed region"
+    stage_views = [view_of(a.warmup + k) for k in range(a.steps)]
     overlapped = None
     if a.leaf_streams == 2:
         # two Leaves in flight: a stage's events span the other stream's
@@ -458,14 +468,18 @@ def main():
         stage_n = {name: len(timing.get(name, [])) for name in STAGES}
         n_steps = a.stage_steps
         stage_src = f"serialized pass of {a.stage_steps} steps (Leaves on one stream)"
+        stage_views = [view_of(a.warmup + k) for k in range(a.stage_steps)]
 
-    # ---- accounting step (untimed): work counters per launch -----------------
-    counters = torch.zeros(6, dtype=torch.int64, device="cuda")
-    acc_timing = {}
-    v = view_of(a.warmup + a.steps)
-    acc = stp.run_view(cams[v], targets[v], counters=counters, timing=acc_timing)
-    torch.cuda.synchronize()
-    cnt = [int(x) for x in counters.cpu()]
+    # ---- accounting (untimed): the work counters of every view whose stage
+    # times are averaged, so the raster stages' lane-ops per step are the mean
+    # over exactly those views (no update: the counts are the views' own) --
+    cnt_view = {}
+    for v in sorted(set(stage_views)):
+        counters = torch.zeros(6, dtype=torch.int64, device="cuda")
+        stp.run_view(cams[v], targets[v], counters=counters, update=False)
+        torch.cuda.synchronize()
+        cnt_view[v] = [int(x) for x in counters.cpu()]
+    cnt = [statistics.mean(cnt_view[v][j] for v in stage_views) for j in range(6)]
     ops_fwd = cnt[2] * K_FWD
     ops_bwd = cnt[3] * K_BWD
 
@@ -477,17 +491,14 @@ def main():
     per_step = {s: stage_ms[s] / n_steps for s in STAGES}
     if dom in ("raster_bwd", "raster_fwd"):
         ops = ops_bwd if dom == "raster_bwd" else ops_fwd
-        ach = ops / (per_step[dom] / 1e3) / 1e12
         traffic, traffic_src = profile_traffic(f"k_{dom}")
-        roof = {"bound": "alu", "kernel": f"k_{dom}", "achieved": round(ach, 3),
-                "peak": round(alu_peak / 1e12, 3), "unit": "Tlane-op/s",
-                "frac": round(ach / (alu_peak / 1e12), 4), "traffic": traffic,
-                "traffic_source": traffic_src,
-                "peak_source": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {sm_mhz:g} MHz "
-                               f"(sm_max_mhz of {peak_src})"}
+        roof = alu_roofline(f"k_{dom}", ops, per_step[dom], alu_peak)
+        roof.update(traffic=traffic, traffic_source=traffic_src,
+                    peak_source=f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {sm_mhz:g} MHz "
+                                f"(sm_max_mhz of {peak_src})")
     else:
         P = model.P
-        C = acc.n_cand
+        C = statistics.mean(s.n_cand for s in stats)
         byt = scene.n * P * 24 + C * (48 + 16) + scene.n * 4
         ach = byt / (per_step[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": round(ach, 1),
@@ -495,7 +506,7 @@ def main():
                 "traffic": None}
 
     # ---- step roofline: per stage max(algorithmic bytes / HBM, lane-ops / ALU)
-    step_roof = step_roofline(a, model, stats, acc, ops_fwd, ops_bwd, per_step, peaks,
+    step_roof = step_roofline(a, model, stats, ops_fwd, ops_bwd, per_step, peaks,
                               alu_peak, W, H, ms_max / a.steps)
 
     # ---- end to end through host buffers --------------------------------------
@@ -570,9 +581,11 @@ def main():
             "stage_ms_source": stage_src,
             "stage_ms_per_step_overlapped": overlapped,
             "stage_launches_per_step": {s: stage_n[s] / n_steps for s in STAGES},
-            "work": {"method_fwd_evaluations": cnt[2], "method_bwd_evaluations": cnt[3],
-                     "fwd_pairs_evaluated": cnt[0], "fwd_pairs_composited": cnt[1],
-                     "bwd_pairs_evaluated": cnt[4], "bwd_pairs_differentiated": cnt[5]},
+            "work": {"per": "mean over the views the stage times average "
+                            f"({len(stage_views)} steps, views {sorted(set(stage_views))})",
+                     "method_fwd_evaluations": round(cnt[2]), "method_bwd_evaluations": round(cnt[3]),
+                     "fwd_pairs_evaluated": round(cnt[0]), "fwd_pairs_composited": round(cnt[1]),
+                     "bwd_pairs_evaluated": round(cnt[4]), "bwd_pairs_differentiated": round(cnt[5])},
             "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk,
         }

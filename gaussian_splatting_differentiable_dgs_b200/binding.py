@@ -282,6 +282,7 @@ def gs_sort_tiles(tile_keys, vals, n, ranges, n_tiles, ws, dev_status, stream=No
 
 
 SORT_NOALLOC_MAX_N = 1 << 18
+SORT_NOALLOC_SCRATCH_BYTES = 3 << 20
 
 
 def gs_sort_keys32_noalloc(keys_in, keys, vals, n, begin_bit, end_bit, flags, dev_status,

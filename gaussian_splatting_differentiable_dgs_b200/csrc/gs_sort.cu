@@ -10,7 +10,6 @@
 // and per Leaf a sort of the duplicated (tile << 32 | depth) keys on the
 // tile bits only.  Because the keys are emitted in depth order, the stable
 // tile-bit sort yields the same order as a full 64-bit sort.
-#include <mutex>
 
 #include "gs_internal.cuh"
 
@@ -704,26 +703,33 @@ extern "C" gs_status gs_sort_keys32(const uint32_t* keys_in, uint32_t* keys, int
 namespace gs {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = (size_t)3 << 20;  // 3 MiB
+constexpr size_t kNoAllocScratchBytes = GS_SORT_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_sort_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+// Upper bound of carve_sort<uint32_t>'s layout (each region rounded up to
+// 256 bytes, the look-back / per-tile count region at its largest, 4 passes
+// of 8-bit digits for 32-bit keys), so that a build with other tile sizes
+// cannot make a call with n <= the maximum run out of scratch.
+constexpr size_t ru256(size_t x) { return (x + 255) / 256 * 256; }
+constexpr size_t noalloc_plan_bound(size_t n) {
+  return ru256(n * 4) + ru256(n * 4) + ru256(8 * kRadix * 8) + ru256(8 * kRadix * 8) +
+         ru256(64 * 4) + 4 * ((n + kSortTile - 1) / kSortTile) * kRadix * 8;
+}
+static_assert(noalloc_plan_bound(GS_SORT_NOALLOC_MAX_N) <= kNoAllocScratchBytes,
+              "the allocation-free sort's array must hold the plan of its largest size");
 
-// Device address of g_sort_scratch for the current device, looked up once
-// per device (the host-side name of the array is not a device address).
+// Device address of g_sort_scratch in the current device's context.  It is
+// looked up on every call (a cheap host-side lookup once the module is
+// loaded) rather than cached, because a cached address would go stale if
+// the context were destroyed and recreated (cudaDeviceReset).  The first
+// call on a device may load the module; make it before any stream capture.
 gs_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GS_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return GS_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_sort_scratch) != cudaSuccess || !p) return GS_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_sort_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();  // leave no sticky error for the next call
+    return GS_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return GS_OK;
 }
 
@@ -734,7 +740,9 @@ extern "C" gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* k
                                             int32_t* vals, int64_t n, int32_t begin_bit,
                                             int32_t end_bit, uint32_t flags, int32_t* dev_status,
                                             gs_stream stream) {
-  if (flags & ~(GS_SORT_IOTA | GS_SORT_ONESWEEP | GS_SORT_TEST_STALL)) return GS_ERR_ARG;
+  // the stall hook of the bounded-wait test is not accepted here: a stalled
+  // call would leave the shared array mid look-back
+  if (flags & ~(GS_SORT_IOTA | GS_SORT_ONESWEEP)) return GS_ERR_ARG;
   if (n < 0) return GS_ERR_ARG;
   if (n > GS_SORT_NOALLOC_MAX_N) return GS_ERR_CAPACITY;
   if (n == 0) return GS_OK;
@@ -744,8 +752,7 @@ extern "C" gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* k
   // the whole plan must fit the array (it does for every n <= the maximum)
   if (gs_sort_workspace_size(n, 4, begin_bit, end_bit) > kNoAllocScratchBytes)
     return GS_ERR_CAPACITY;
-  return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0,
-                             (flags & GS_SORT_TEST_STALL) != 0, n, begin_bit, end_bit, scratch,
-                             kNoAllocScratchBytes, dev_status, to_stream(stream), nullptr, 0,
-                             (flags & GS_SORT_ONESWEEP) != 0);
+  return sort_impl<uint32_t>(keys_in, keys, vals, (flags & GS_SORT_IOTA) != 0, false, n,
+                             begin_bit, end_bit, scratch, kNoAllocScratchBytes, dev_status,
+                             to_stream(stream), nullptr, 0, (flags & GS_SORT_ONESWEEP) != 0);
 }

@@ -285,16 +285,21 @@ gs_status gs_sort_tiles(uint32_t* tile_keys, int32_t* vals, int64_t n,
  * memory when they need the sort, e.g. code inside a host application whose
  * allocator owns the whole device, or a latency-critical loop that must not
  * risk an allocation's implicit device synchronisation.  Same arguments and
- * result as gs_sort_keys32 without the workspace: the scratch is a 3 MiB
- * array inside the library that every GPU loading the library holds until
- * the process exits.  n > GS_SORT_NOALLOC_MAX_N returns GS_ERR_CAPACITY and
- * launches nothing.  The first call on a device looks up the array's device
- * address (make that first call before any stream capture).  It never
- * calls cudaMalloc or cudaFree.  All calls share the one array: calls that
- * overlap on the GPU (e.g. on two streams) race and give wrong results;
- * serialise them.  The parts of the array that must start at zero are
- * cleared by every call, so a call does not depend on the previous one. */
+ * result as gs_sort_keys32 without the workspace: the scratch is an array
+ * of GS_SORT_NOALLOC_SCRATCH_BYTES (3 MiB) inside the library that every
+ * GPU loading the library holds until the process exits.  n >
+ * GS_SORT_NOALLOC_MAX_N returns GS_ERR_CAPACITY and launches nothing;
+ * flags other than GS_SORT_IOTA and GS_SORT_ONESWEEP return GS_ERR_ARG.
+ * Every call looks up the array's address in the current device's context
+ * (cudaGetSymbolAddress; GS_ERR_CUDA if that fails); the first call on a
+ * device may load the library's device code, so make it before any stream
+ * capture.  It never calls cudaMalloc or cudaFree.  All calls share the one
+ * array: calls that overlap on the GPU (e.g. on two streams) race and give
+ * wrong results; serialise them.  The parts of the array that must start
+ * at zero are cleared by every call, so a call does not depend on the
+ * previous one. */
 #define GS_SORT_NOALLOC_MAX_N (1 << 18)
+#define GS_SORT_NOALLOC_SCRATCH_BYTES ((size_t)3 << 20)
 gs_status gs_sort_keys32_noalloc(const uint32_t* keys_in, uint32_t* keys,
                                  int32_t* vals, int64_t n, int32_t begin_bit,
                                  int32_t end_bit, uint32_t flags,

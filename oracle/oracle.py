@@ -435,7 +435,9 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
     `project`.  Besides the list position `last`, the result holds
     `last_id`: the Gaussian index of each pixel's last composited entry
     (-1 if none), which does not depend on which skipped entries a list
-    holds."""
+    holds; `n_eval_px`: the list entries each pixel visits (up to and
+    including the one it stops at, else its whole list), `list_len`: the
+    length of each pixel's tile list."""
     W, H = cam.width, cam.height
     TW, TH = grid(cam)
     pr = project(params, n, sh_degree, cam, tight=tight)
@@ -449,6 +451,8 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
     Tfin = np.ones((TH * 16, TW * 16))
     last = np.zeros((TH * 16, TW * 16), np.int32)
     last_id = np.full((TH * 16, TW * 16), -1, np.int64)
+    n_eval_px = np.zeros((TH * 16, TW * 16), np.int64)
+    list_len = np.zeros((TH * 16, TW * 16), np.int64)
     pflags = np.zeros((TH * 16, TW * 16), np.uint8)
     n_eval = 0
     n_isect = 0
@@ -493,6 +497,8 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
             hit = lj > 0
             lid[hit] = pr["cand_idx"][vals[off[j] + lj[hit] - 1]]
             last_id[sl] = lid.reshape(16, 16)
+            n_eval_px[sl] = fw["n_eval"][j].reshape(16, 16)
+            list_len[sl] = off[j + 1] - off[j]
             pflags[sl] = fw["flags"][j].reshape(16, 16)
     g3d = project_bwd(params, sh_degree, cam, pr["cand_idx"], g2d)
     P, n_pad = params.shape
@@ -508,6 +514,7 @@ def step(params, n, sh_degree, cam, target, leaves=None, m=None, v=None,
     v_new[:, n:] = 0
     return dict(proj=pr, g2d=g2d, grad=grad, loss=loss, img=img[:, :H, :W],
                 T=Tfin[:H, :W], last=last[:H, :W], last_id=last_id[:H, :W],
+                n_eval_px=n_eval_px[:H, :W], list_len=list_len[:H, :W],
                 pflags=pflags[:H, :W],
                 params=p_new, m=m_new, v=v_new, n_eval=n_eval,
                 n_isect=n_isect)

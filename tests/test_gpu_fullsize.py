@@ -1,14 +1,21 @@
-"""Parity at the full size of the 6M-Gaussian outdoor workload (5000x3300,
-384 MiB Leaf budget) in the configuration bench.py times, against the
-oracle's own computation:
+"""Parity at full size against the oracle's own computation:
 
-- the projection's integer outputs for every Gaussian (candidate set, tile
-  rects, depth keys) bit-exactly, records within their rounding bounds;
-- on sampled tiles (random ones plus every tile of a sample of small
-  candidates) the oracle's lists, compositing and reverse blend: image, T
-  and last per pixel, the sampled candidates' 2D gradients (complete, since
-  all their tiles are sampled), and their parameters after the one Adam
-  update of the view.
+- the 6M-Gaussian outdoor workload (5000x3300, 384 MiB Leaf budget) in the
+  configuration bench.py times (two Leaves in flight);
+- the whole-image configuration (BoundedGS page, Fig. A and ablation A: one
+  Leaf covering the image, dense projection state, raster buffers alive
+  through projection backward) at 16000x10667, where a view's tile lists
+  hold more than 2^31 entries, so counts, table entries and list offsets
+  need 64 bits.
+
+Each checks the projection's integer outputs for every Gaussian (candidate
+set, tile rects, depth keys, the tile SAT) bit-exactly, records within
+their rounding bounds, and on sampled tiles (random ones plus every tile of
+a sample of small candidates) the oracle's lists, compositing and reverse
+blend: image, T and last per pixel, the sampled candidates' 2D gradients
+(complete, since all their tiles are sampled), their 3D gradients (read from
+Adam's first moment) and their parameters after the one Adam update of the
+view.
 
 The target is a seeded random image, so no oracle input comes from the CUDA
 path."""
@@ -58,45 +65,72 @@ class Grab:
         self.g2d = ctx["g2d"][:12 * self.C].cpu().numpy().reshape(-1, 12)
 
 
-def test_full_size_step_sampled(oracle_mod):
-    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
-    O = oracle_mod
-    sc, cams = synth.outdoor_scene(6_000_000, seed=0, width=5000, height=3300, n_views=8)
-    cam = cams[0]
-    W, H = cam.width, cam.height
-    TW, TH = O.grid(cam)
-    target = (synth.random_image(W, H, 11) * 0.6).astype(np.float32)
+def check_sat(O, sat_gpu, pr, near, TW, TH):
+    """The GPU's tile SAT against the oracle's counts.  A candidate the oracle
+    flags (a rect edge within rounding of a tile boundary) may take either
+    side, so a tile's count may differ from the oracle's by at most the
+    flagged candidates whose 3-sigma square covers it; every other tile
+    matches exactly."""
+    sat_gpu = np.asarray(sat_gpu, np.int64)
+    got = np.diff(np.diff(sat_gpu, axis=0), axis=1)
+    exp = O.tile_counts_fast(pr["rect"], TW, TH)
+    ro = pr["rec"][near]
+    sq = np.stack([np.floor((ro[:, 0] - ro[:, 3]) / 16), np.floor((ro[:, 1] - ro[:, 3]) / 16),
+                   np.floor((ro[:, 0] + ro[:, 3]) / 16) + 1,
+                   np.floor((ro[:, 1] + ro[:, 3]) / 16) + 1], 1)
+    sq = np.clip(sq, 0, [TW, TH, TW, TH]).astype(np.int64)
+    slack = O.tile_counts_fast(sq, TW, TH) if len(sq) else np.zeros_like(exp)
+    diff = np.abs(got - exp)
+    assert (diff <= slack).all(), int((diff > slack).sum())
+    assert sat_gpu[0].max() == 0 and sat_gpu[:, 0].max() == 0
+    return int((diff > 0).sum())
 
-    # ---- the GPU step, as bench.py runs it (two Leaves in flight) ------------
+
+def run_gpu_step(sc, cam, target, **stepper_kw):
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=384 << 20, leaf_streams=2)
-    grab = Grab(W, H)
+    stp = Stepper(model, **stepper_kw)
+    grab = Grab(cam.width, cam.height)
     stats = stp.run_view(cam, torch.as_tensor(target).cuda(), hooks=grab)
     stp.check()
-    assert stats.n_leaves > 1
-    p_after = model.params.cpu().numpy()
+    grab.p_after = model.params.cpu().numpy()
+    grab.m_after = model.m.cpu().numpy()
     del model, stp
     torch.cuda.empty_cache()
+    return stats, grab
 
-    # ---- projection: every Gaussian -----------------------------------------
+
+def check_against_oracle(O, sc, cam, target, grab, dense):
+    """Every check of the module docstring.  dense: the GPU's candidate state
+    is indexed by Gaussian (whole-image configuration) instead of by
+    candidate."""
+    W, H = cam.width, cam.height
+    TW, TH = O.grid(cam)
     p64 = sc.params.astype(np.float64)
     pr = O.project(p64, sc.n, sc.sh_degree, cam)
     C = len(pr["cand_idx"])
-    assert grab.C == C
-    assert (grab.cand_idx == pr["cand_idx"]).all()
-    assert (grab.key == pr["key"]).all()
-    near = (pr["flags"] & 1) != 0      # radius within rounding of a tile boundary
+    if dense:
+        assert grab.C == sc.n and (grab.cand_idx == np.arange(sc.n)).all()
+        rows = pr["cand_idx"]          # GPU row of each oracle candidate
+        culled = np.ones(sc.n, bool)
+        culled[rows] = False
+        assert (grab.rect[culled] == 0).all()
+    else:
+        assert grab.C == C and (grab.cand_idx == pr["cand_idx"]).all()
+        rows = np.arange(C)
+    assert (grab.key[rows] == pr["key"]).all()
+    near = (pr["flags"] & 1) != 0      # a rect edge within rounding of a tile boundary
     assert near.sum() <= max(1, C // 10000)
-    assert (grab.rect[~near] == pr["rect"][~near]).all()
+    assert (grab.rect[rows][~near] == pr["rect"][~near]).all()
     exp = encode_records(pr["rec"])
-    d = decode_records(grab.rec)
+    rec = grab.rec[rows]
+    d = decode_records(rec)
     ro = pr["rec"]
     assert np.abs(d["u"] - ro[:, 0]).max() <= 2.5e-7 + 1e-12 * np.abs(ro[:, 0]).max()
     assert np.abs(d["v"] - ro[:, 1]).max() <= 2.5e-7 + 1e-12 * np.abs(ro[:, 1]).max()
     for col in (4, 5, 6, 7, 8, 9, 10, 11):
-        assert rel_err(grab.rec[:, col], exp[:, col], floor=1e-30).max() <= 2.4e-7, col
-    if (grab.rect == pr["rect"]).all():
-        assert (grab.sat == O.sat(O.tile_counts_fast(pr["rect"], TW, TH))).all()
+        assert rel_err(rec[:, col], exp[:, col], floor=1e-30).max() <= 2.4e-7, col
+    check_sat(O, grab.sat, pr, near, TW, TH)
 
     # ---- sampled tiles: lists, compositing, reverse blend --------------------
     rng = np.random.default_rng(5)
@@ -128,7 +162,7 @@ def test_full_size_step_sampled(oracle_mod):
     valid = (fw["flags"] & 0x80) == 0
     dL = np.where(valid[:, None, :], np.sign(fw["img"] - tg) / (3.0 * W * H), 0.0)
     g2d_o = O.raster_bwd(pr["rec"], TW, W, H, tiles, off, vals, dL)
-    gs = grab.g2d[pick, :9].astype(np.float64)
+    gs = grab.g2d[rows[pick], :9].astype(np.float64)
     go = g2d_o[pick]
     for f in range(9):
         assert rel_l2(gs[:, f], go[:, f]) <= GRAD_TOL, f
@@ -138,9 +172,42 @@ def test_full_size_step_sampled(oracle_mod):
     g3d = O.project_bwd(p64, sc.sh_degree, cam, gi, go)
     zeros = np.zeros_like(p64[:, gi])
     pe, _, _ = O.adam(p64[:, gi], zeros, zeros, g3d, step=1)
-    got = p_after[:, gi]
+    # the gradient with its magnitude: after the first update m = (1 - b1) g
+    g_impl = grab.m_after[:, gi].astype(np.float64) / float(np.float32(0.1))
+    for a_, e_ in ((0, 3), (3, 6), (6, 10), (10, 11), (11, 14), (14, sc.P)):
+        assert rel_l2(g_impl[a_:e_], g3d[a_:e_]) <= GRAD_TOL, (a_, e_)
+    got = grab.p_after[:, gi]
     gg = np.abs(g3d)
     mask = gg > 1e-3 * gg.max(axis=1, keepdims=True)
     diff = np.abs(got - pe)
     assert diff[mask].max() <= 1e-5
     assert diff.max() <= 2.1e-3  # at most one sign flip of a ~zero gradient
+    return pr
+
+
+def test_full_size_step_sampled(oracle_mod):
+    sc, cams = synth.outdoor_scene(6_000_000, seed=0, width=5000, height=3300, n_views=8)
+    cam = cams[0]
+    target = (synth.random_image(cam.width, cam.height, 11) * 0.6).astype(np.float32)
+    stats, grab = run_gpu_step(sc, cam, target, budget=384 << 20, leaf_streams=2)
+    assert stats.n_leaves > 1
+    check_against_oracle(oracle_mod, sc, cam, target, grab, dense=False)
+
+
+def test_whole_image_16k_int64(oracle_mod):
+    """The whole-image configuration at 16000x10667 (camera 0 of the outdoor
+    scene at the resolution sweep's widest width): more than 2^31 tile-list
+    entries in one Leaf, so the SAT, the per-tile ranges and the list
+    offsets run past 32 bits.  Checked against the oracle as the 5K case
+    is."""
+    W = 16000
+    cam = synth.sweep_camera(W)
+    H = cam.height
+    sc, _ = synth.outdoor_scene(6_000_000, seed=0, width=W, height=H, n_views=1)
+    target = (synth.random_image(W, H, 13) * 0.6).astype(np.float32)
+    stats, grab = run_gpu_step(sc, cam, target, budget=384 << 20, mode="original")
+    assert stats.n_leaves == 1
+    assert stats.n_isect > 2 ** 31 and stats.n_isect_square > 2 ** 31
+    assert int(grab.sat[-1, -1]) == stats.n_isect
+    pr = check_against_oracle(oracle_mod, sc, cam, target, grab, dense=True)
+    assert int(pr["rec"][:, 14].sum()) == stats.n_isect_square

@@ -65,6 +65,11 @@ def test_workspace_sizes(gsb):
     assert s2 > s1 > 12 << 20
     assert b.gs_bin_workspace_size(1 << 20) >= 8 * (1 << 20) // 1024
     assert b.gs_depth_order_workspace_size(1 << 20) > 12 << 20
+    # the allocation-free sort's array holds the plan of its largest size
+    # for every bit range (32-bit keys)
+    for lo, hi in ((0, 32), (0, 16), (5, 29), (0, 1)):
+        need = b.gs_sort_workspace_size(b.SORT_NOALLOC_MAX_N, 4, lo, hi)
+        assert 0 < need <= b.SORT_NOALLOC_SCRATCH_BYTES, (lo, hi, need)
 
 
 def test_load_model_matches_buffers(gsb):
@@ -139,13 +144,12 @@ def test_step_roofline_properties():
     model = types.SimpleNamespace(n=1_000_000, P=59)
     st = types.SimpleNamespace(n_cand=800_000, n_isect=50_000_000, n_block_entries=3_000_000,
                                n_block_reads=0, n_leaves=2)
-    acc = types.SimpleNamespace(n_isect=50_000_000)
     per_step = {"project": 0.2, "raster_bwd": 0.5, "project_bwd": 0.4}
     peaks = {"hbm_gbs": 6000.0}
     alu = 37e12
 
     def run(peaks, alu, step_ms, ops_bwd=4e10):
-        return bench.step_roofline(a, model, [st], acc, 1e10, ops_bwd, per_step, peaks, alu,
+        return bench.step_roofline(a, model, [st], 1e10, ops_bwd, per_step, peaks, alu,
                                    2000, 1000, step_ms)
 
     r = run(peaks, alu, 2.0)
@@ -164,3 +168,9 @@ def test_step_roofline_properties():
     assert abs(r2["stages"]["project_bwd"]["roofline_ms"] * 2
                - s["project_bwd"]["roofline_ms"]) <= 1e-3
     assert r2["stages"]["raster_bwd"]["roofline_ms"] == s["raster_bwd"]["roofline_ms"]
+    # the dominant kernel's roofline object and the step roofline's stage take
+    # the same lane-ops, so an ALU-bound stage's fraction is the same in both
+    k = bench.alu_roofline("k_raster_bwd", 4e10, per_step["raster_bwd"], alu)
+    st_b = s["raster_bwd"]
+    assert abs(k["frac"] - st_b["roofline_ms"] / st_b["measured_ms"]) <= 1e-3
+    assert k["lane_ops_per_step"] == st_b["lane_ops"]
