@@ -241,6 +241,12 @@ gs_status gs_project_region(const gs_model* model, const gs_camera* cam,
                             int32_t* dev_status, gs_stream stream);
 
 /* ---- 2. radix sorts ------------------------------------------------------
+ * The per-tile depth order of the tile rasteriser: its duplicated 64-bit
+ * keys (tile << 32 | depth bits) sorted ascending, ties in candidate order
+ * (the sort the SkipGS paper notes' differentiable tile rasteriser rests
+ * on, "research background"; the BoundedGS page sorts each Leaf's entries,
+ * section 02 B -> C).  This library sorts the candidates once by depth and
+ * then only the tile bits, which gives the same order.
  * Stable LSD radix sort of (key, value) pairs on key bits [begin_bit,
  * end_bit), 8-bit digits, an even number of passes: a histogram of every
  * digit in one pass over the keys, then per digit either three kernels
@@ -412,6 +418,10 @@ gs_status gs_expand_tiles(const gs_proj* proj, const int32_t* block_vals,
                           int32_t* dev_status, gs_stream stream);
 
 /* ---- 5. raster forward ---------------------------------------------------
+ * Front-to-back alpha compositing of the projected Gaussians (SkipGS paper
+ * notes, "research background" and "loss function / training strategy":
+ * differentiable rasterisation through the transmittance accumulation;
+ * BoundedGS page, section 02 B -> C: one Leaf's pixels at a time).
  * Per pixel p of the Leaf, over its tile's list in order: d = (u, v) - p;
  * q = (a d_x^2 + c d_y^2)/2 + b d_x d_y; alpha = min(0.99, o exp(-q)); skip
  * if alpha < 1/255; T' = T (1 - alpha); stop (without compositing) if
@@ -545,6 +555,10 @@ gs_status gs_grad_accumulate(const float* g3d, int64_t g3d_stride,
                              float* G, int64_t n_pad, gs_stream stream);
 
 /* ---- 9. Adam -------------------------------------------------------------
+ * One Adam update per view on the view's summed gradient (BoundedGS page,
+ * section 01: every region's gradient is summed over the whole view, then
+ * the parameters are updated once; Kingma & Ba's Adam with bias
+ * correction, the optimiser of 3DGS training):
  * m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
  * p -= lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps), for i < n, all P
  * planes.  If slot is NULL, g is dense [P][n_pad]; else g is compact
