@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=48)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3],
+                    help="1: 2,000 Gaussians SH0 256x256; 2: 100,000 Gaussians SH3 1920x1080; "
+                         "3: the outdoor scene (--gaussians, --width, --height, --views)")
     ap.add_argument("--gaussians", type=int, default=6_000_000)
     ap.add_argument("--width", type=int, default=5000)
     ap.add_argument("--height", type=int, default=3300)
@@ -88,8 +91,39 @@ def parse():
 
 
 def workload_name(a):
+    if a.config == 1:
+        return ("tiny_2k_256x256: 2,000 Gaussians SH0, one camera at the origin, f 300, "
+                f"{a.budget_mib:g} MiB Leaf budget")
+    if a.config == 2:
+        return ("hd_100k_1920x1080: 100,000 Gaussians SH3 in 64 clusters, one camera, f 1500, "
+                f"{a.budget_mib:g} MiB Leaf budget")
     return (f"outdoor_{a.gaussians / 1e6:g}m_{a.width}x{a.height}: {a.gaussians:,} Gaussians "
             f"SH3, {a.views} views on a radius-4 circle, {a.budget_mib:g} MiB Leaf budget")
+
+
+def make_workload(a, synth):
+    """(scene, cameras) of the selected configuration; the small ones fit in
+    L2, so their timed steps are preceded by an L2 flush."""
+    if a.config == 1:
+        return synth.tiny_oracle_scene(0)
+    if a.config == 2:
+        return synth.hd_cluster_scene(0)
+    return synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
+                               n_views=a.views)
+
+
+def cpu_model():
+    """The host CPU's model name (/proc/cpuinfo) and its logical core count."""
+    name = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return name or "unknown", os.cpu_count()
 
 
 def step_roofline(a, model, stats, ops_fwd, ops_bwd, per_step, peaks, alu_peak, W, H,
@@ -300,15 +334,20 @@ class OracleSample:
         # projection of 1/8 of the Gaussians
         sub = np.sort(self.rng.choice(n, n // 8, replace=False))
         ps = np.ascontiguousarray(p64[:, sub])
+        measured = 0.0
         t0 = time.perf_counter()
         O.project(ps, len(sub), sc.sh_degree, cam)
-        t_proj = (time.perf_counter() - t0) * n / len(sub)
+        dt = time.perf_counter() - t0
+        measured += dt
+        t_proj = dt * n / len(sub)
         # tile lists: scatter + per-tile stable sort for 1/16 of the candidates
         C = len(pr["cand_idx"])
         cs = np.sort(self.rng.choice(C, max(C // 16, 1), replace=False))
         t0 = time.perf_counter()
         O.tile_lists_all(pr["rect"][cs], pr["key"][cs], TW, TH)
-        t_lists = (time.perf_counter() - t0) * C / len(cs)
+        dt = time.perf_counter() - t0
+        measured += dt
+        t_lists = dt * C / len(cs)
         # raster forward + L1 + raster backward on uniformly random tiles
         tiles = np.sort(self.rng.choice(TW * TH, self.n_tiles, replace=False)).astype(np.int32)
         off, vals = O.tile_lists(pr["rect"], pr["key"], TW, tiles)
@@ -321,22 +360,28 @@ class OracleSample:
         d = np.where(valid[:, None, :], fw["img"] - tg, 0.0)
         dL = np.sign(d) / (3.0 * W * H)
         O.raster_bwd(pr["rec"], TW, W, H, tiles, off, vals, dL)
-        t_raster = (time.perf_counter() - t0) * (TW * TH) / self.n_tiles
+        dt = time.perf_counter() - t0
+        measured += dt
+        t_raster = dt * (TW * TH) / self.n_tiles
         I_s = int(off[-1])
         # projection backward on 1/16 of the candidates
         g2d = self.rng.normal(size=(len(cs), 9)) * 1e-3
         t0 = time.perf_counter()
         O.project_bwd(p64, sc.sh_degree, cam, pr["cand_idx"][cs], g2d)
-        t_pbwd = (time.perf_counter() - t0) * C / len(cs)
+        dt = time.perf_counter() - t0
+        measured += dt
+        t_pbwd = dt * C / len(cs)
         # Adam on 1/64 of the Gaussians (all planes)
         k = max(n // 64, 1)
         pa = p64[:, :k]
         g = self.rng.normal(size=pa.shape)
         t0 = time.perf_counter()
         O.adam(pa, np.zeros_like(pa), np.zeros_like(pa), g, step=1)
-        t_adam = (time.perf_counter() - t0) * n / k
+        dt = time.perf_counter() - t0
+        measured += dt
+        t_adam = dt * n / k
         est = t_proj + t_lists + t_raster + t_pbwd + t_adam
-        return dict(est_step_s=est, I_total=I_total, sample_isect=I_s,
+        return dict(est_step_s=est, measured_s=measured, I_total=I_total, sample_isect=I_s,
                     parts=dict(project=t_proj, lists=t_lists, raster=t_raster,
                                project_bwd=t_pbwd, adam=t_adam))
 
@@ -346,6 +391,20 @@ class OracleSample:
                 f"uniformly random tiles (x tiles/{self.n_tiles}), projection bwd on 1/16 of the "
                 f"candidates (x16), Adam on 1/64 of the Gaussians (x64); value = the view's "
                 f"intersections / estimated step time")
+
+
+def oracle_full_step(O, scene, cam, target, reps=1):
+    """The oracle's whole step of one view (projection, lists, raster forward,
+    L1, raster backward, projection backward, one Adam update), timed on the
+    host cores: the fastest of `reps` runs."""
+    p64 = scene.params.astype(np.float64)
+    best, r = None, None
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        r = O.step(p64, scene.n, scene.sh_degree, cam, target)
+        dt = time.perf_counter() - t0
+        best = dt if best is None else min(best, dt)
+    return dict(step_s=best, I_total=int(r["proj"]["rec"][:, 14].sum()), loss=r["loss"])
 
 
 # ---------------------------------------------------------------------------
@@ -396,10 +455,14 @@ def main():
                                 device_id=torch.device("cuda", local))
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper, STAGES
 
-    scene, cams = synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
-                                      n_views=a.views)
-    W, H = a.width, a.height
+    scene, cams = make_workload(a, synth)
+    W, H = cams[0].width, cams[0].height
     budget = int(a.budget_mib * (1 << 20))
+    # a workload that fits in L2 gets it flushed before every timed step
+    # (outside the step's events); the outdoor scene's 4.25 GB of parameters
+    # and moments stream through HBM every step
+    flush = (torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+             if a.config in (1, 2) else None)
     # targets: renders of the jittered copy (means N(0, 0.02), colour N(0, 0.05))
     jit = synth.jittered(scene, seed=1)
     jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
@@ -427,18 +490,29 @@ def main():
     wall0 = time.time()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
     stats = []
-    for k in range(a.steps):
-        v = view_of(a.warmup + k)
-        stats.append(stp.run_view(cams[v], targets[v], timing=timing))
-    e1.record()
-    torch.cuda.synchronize()
+    if flush is None:
+        e0.record()
+        for k in range(a.steps):
+            v = view_of(a.warmup + k)
+            stats.append(stp.run_view(cams[v], targets[v], timing=timing))
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+    else:
+        ms = 0.0
+        for k in range(a.steps):
+            v = view_of(a.warmup + k)
+            flush.fill_(k & 255)          # evicts the step's inputs from L2
+            e0.record()
+            stats.append(stp.run_view(cams[v], targets[v], timing=timing))
+            e1.record()
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1)
     if dist:
         dist.barrier()
     clk = clocks.stop(wall0, time.time())
     stp.check()
-    ms = e0.elapsed_time(e1)
     isect = sum(s.n_isect_square for s in stats)   # conventional 3-sigma-square count
     entries = sum(s.n_isect for s in stats)         # entries of the tight tile lists
     launches = sum(s.launches for s in stats)
@@ -551,13 +625,25 @@ def main():
                 tg_host[v] = targets[v].cpu().numpy().astype(np.float64)
             return tg_host[v]
 
-        osm = OracleSample(scene, cams, target_fn, n_tiles=a.cpu_tiles)
-        r = osm.step(0)
         from oracle import oracle as O
-        cpu = {"value": r["I_total"] / r["est_step_s"], "unit": UNIT,
-               "cores": O.num_threads(), "kind": "oracle", "sample": osm.describe(),
-               "est_step_s": round(r["est_step_s"], 2),
-               "parts_s": {k: round(x, 2) for k, x in r["parts"].items()}}
+        model_name, ncpu = cpu_model()
+        if a.config in (1, 2):
+            # the whole oracle step, measured (no sampling)
+            r = oracle_full_step(O, scene, cams[0], target_fn(0), reps=3 if a.config == 1 else 1)
+            cpu = {"value": r["I_total"] / r["step_s"], "unit": UNIT, "cores": O.num_threads(),
+                   "cpu_model": model_name, "logical_cpus": ncpu, "kind": "oracle",
+                   "sample": "the whole step of the view (projection, lists, raster forward, "
+                             "L1, raster backward, projection backward, Adam), measured",
+                   "estimated": False, "step_s": round(r["step_s"], 4)}
+        else:
+            osm = OracleSample(scene, cams, target_fn, n_tiles=a.cpu_tiles)
+            r = osm.step(0)
+            cpu = {"value": r["I_total"] / r["est_step_s"], "unit": UNIT,
+                   "cores": O.num_threads(), "cpu_model": model_name, "logical_cpus": ncpu,
+                   "kind": "oracle", "sample": osm.describe(),
+                   "estimated": True, "est_step_s": round(r["est_step_s"], 2),
+                   "measured_s": round(r["measured_s"], 2),
+                   "parts_s": {k: round(x, 2) for k, x in r["parts"].items()}}
 
     if rank == 0:
         out = {
@@ -565,12 +651,15 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded generator; targets = renders of a jittered copy)",
-            "config": {"workload": workload_name(a), "gaussians": a.gaussians, "sh_degree": 3,
+            "config": {"workload": workload_name(a), "gaussians": scene.n,
+                       "sh_degree": scene.sh_degree,
                        "width": W, "height": H, "views": nv, "leaf_budget_mib": a.budget_mib,
                        "binning": a.binning, "loss": a.loss, "leaf_streams": a.leaf_streams,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (4.25 GB of params + Adam moments "
-                             "stream every step)"},
+                       "l2": ("inputs larger than L2 (4.25 GB of params + Adam moments "
+                              "stream every step)") if flush is None else
+                             ("L2 flushed before every timed step (512 MiB fill outside the "
+                              "step's CUDA events; the step's inputs fit in L2)")},
             "peak_ws_gib": peak_ws / 2 ** 30,
             "isect_per_view": isect / a.steps,
             "list_entries_per_view": entries / a.steps,
@@ -611,6 +700,8 @@ def run_sweep(a):
     jit = synth.jittered(scene, seed=1)
     budget = int(a.budget_mib * (1 << 20))
     rows = []
+    clocks = ClockSampler(0)
+    wall0 = time.time()
     for width in [int(w) for w in a.sweep.split(",")]:
         cam = synth.sweep_camera(width)
         jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
@@ -659,8 +750,10 @@ def run_sweep(a):
         print(json.dumps(rows[-1]), flush=True)
         del target, target_dev, target_host
         torch.cuda.empty_cache()
+    clk = clocks.stop(wall0, time.time())
     diffs = [r["l1_rel_diff"] for r in rows if "l1_rel_diff" in r]
     print(json.dumps({"sweep": "resolution", "summary": True, "max_l1_rel_diff": max(diffs),
+                      "clocks": clk,
                       "workload": workload_name(a) + ", camera 0 pose, fixed field of view"}))
 
 
@@ -765,12 +858,42 @@ def run_skipgs(a):
 
 
 def run_reference(a, rank, world):
-    """The oracle, as it stands, timed on the host cores (rank 0 only)."""
+    """The oracle, as it stands, timed on the host cores (rank 0 only).  The
+    small configurations run its whole step; the outdoor scene runs bounded
+    samples of each step, scaled to the step (an estimate, marked so)."""
     if rank != 0:
         return
     from gaussian_splatting_differentiable_dgs_b200 import synth
-    scene, cams = synth.outdoor_scene(a.gaussians, seed=0, width=a.width, height=a.height,
-                                      n_views=a.views)
+    from oracle import oracle as O
+    model_name, ncpu = cpu_model()
+    scene, cams = make_workload(a, synth)
+    if a.config in (1, 2):
+        cam = cams[0]
+        target = synth.random_image(cam.width, cam.height, 100).astype(np.float64)
+        for _ in range(a.warmup if a.config == 1 else min(a.warmup, 1)):
+            oracle_full_step(O, scene, cam, target)
+        steps = a.steps if a.config == 1 else min(a.steps, 3)
+        t0 = time.perf_counter()
+        times, isect = [], 0
+        for _ in range(steps):
+            r = oracle_full_step(O, scene, cam, target)
+            times.append(r["step_s"])
+            isect += r["I_total"]
+        wall = time.perf_counter() - t0
+        value = isect / sum(times)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": steps, "warmup": a.warmup,
+            "ms_per_step": 1e3 * sum(times) / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(a)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.num_threads(),
+                             "cpu_model": model_name, "logical_cpus": ncpu, "kind": "oracle",
+                             "sample": "the whole step, measured", "estimated": False},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "estimated": False, "wall_s": round(wall, 3)}))
+        return
     jit = synth.jittered(scene, seed=1)
     cache = {}
 
@@ -786,23 +909,28 @@ def run_reference(a, rank, world):
     for k in range(a.warmup):
         osm.step(k % len(cams))
     t0 = time.perf_counter()
-    ests, isects = [], []
+    ests, isects, measured = [], [], 0.0
     for k in range(a.steps):
         r = osm.step(k % len(cams))
         ests.append(r["est_step_s"])
         isects.append(r["I_total"])
+        measured += r["measured_s"]
     wall = time.perf_counter() - t0
-    from oracle import oracle as O
     value = sum(isects) / sum(ests)
+    # ms_per_step is the estimate of a whole oracle step from its samples; the
+    # samples themselves took measured_sample_s (the run took wall_s)
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(ests) / a.steps,
+           "estimated": True, "measured_sample_s": round(measured, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic", "config": {"workload": workload_name(a)},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.num_threads(),
-                            "kind": "oracle", "sample": osm.describe()},
+                            "cpu_model": model_name, "logical_cpus": ncpu,
+                            "kind": "oracle", "sample": osm.describe(), "estimated": True,
+                            "measured_sample_s": round(measured, 3)},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0},
-           "wall_s": wall}
+           "wall_s": round(wall, 3)}
     print(json.dumps(out))
 
 
