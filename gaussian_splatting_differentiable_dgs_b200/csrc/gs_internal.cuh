@@ -143,16 +143,23 @@ constexpr unsigned long long kFlagAgg = 1ull << 62;
 constexpr unsigned long long kFlagInc = 2ull << 62;
 constexpr unsigned long long kValMask = (1ull << 62) - 1;
 
-// Called by one full warp.  Publishes `agg` for block `b` and returns the
-// exclusive prefix (sum of the aggregates of blocks 0..b-1) to every lane.
-__device__ __forceinline__ int64_t lookback_warp(unsigned long long* status, int64_t b,
-                                                 int64_t agg, int32_t* dev_status) {
+// Decoupled look-back over the status words of ordered units (blocks or
+// warps).  lookback_publish makes unit b's aggregate visible (unit 0's is
+// its inclusive prefix); lookback_resolve then returns the exclusive prefix
+// (sum of the aggregates of units 0..b-1) to every lane and publishes b's
+// inclusive prefix.  Both are called by one full warp.  A unit waits only
+// on lower-numbered units, so units must be numbered in an order in which
+// they are guaranteed to start (an atomic ticket).
+__device__ __forceinline__ void lookback_publish(unsigned long long* status, int64_t b,
+                                                 int64_t agg) {
+  if ((threadIdx.x & 31) == 0)
+    st_relaxed(&status[b], (b == 0 ? kFlagInc : kFlagAgg) | (unsigned long long)agg);
+}
+
+__device__ __forceinline__ int64_t lookback_resolve(unsigned long long* status, int64_t b,
+                                                    int64_t agg, int32_t* dev_status) {
   const int lane = threadIdx.x & 31;
-  if (b == 0) {
-    if (lane == 0) st_relaxed(&status[0], kFlagInc | (unsigned long long)agg);
-    return 0;
-  }
-  if (lane == 0) st_relaxed(&status[b], kFlagAgg | (unsigned long long)agg);
+  if (b == 0) return 0;
   int64_t excl = 0;
   int64_t end = b - 1;  // window covers end, end-1, ..., end-31
   int spins = 0;
@@ -179,6 +186,13 @@ __device__ __forceinline__ int64_t lookback_warp(unsigned long long* status, int
   }
   if (lane == 0) st_relaxed(&status[b], kFlagInc | (unsigned long long)(excl + agg));
   return excl;
+}
+
+// Publishes `agg` for unit `b` and returns its exclusive prefix.
+__device__ __forceinline__ int64_t lookback_warp(unsigned long long* status, int64_t b,
+                                                 int64_t agg, int32_t* dev_status) {
+  lookback_publish(status, b, agg);
+  return lookback_resolve(status, b, agg, dev_status);
 }
 
 

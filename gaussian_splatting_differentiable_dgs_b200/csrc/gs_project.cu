@@ -20,10 +20,16 @@
 namespace gs {
 namespace {
 
-constexpr int kProjThreads = 256;
+#ifndef GS_PROJ_THREADS
+#define GS_PROJ_THREADS 256
+#endif
+#ifndef GS_PROJ_MINB
+#define GS_PROJ_MINB 4
+#endif
+constexpr int kProjThreads = GS_PROJ_THREADS;
 // blocks between a block and the one whose geometric planes it prefetches:
-// about one wave of resident blocks (148 SMs x 3)
-constexpr int kProjAhead = 444;
+// about one wave of resident blocks (148 SMs x GS_PROJ_MINB)
+constexpr int kProjAhead = 148 * GS_PROJ_MINB * 256 / GS_PROJ_THREADS;
 
 struct ProjCam {
   double R[9], t[3];
@@ -242,10 +248,11 @@ __device__ __forceinline__ void sh_record(const float* __restrict__ P, int64_t n
                    depth);
 }
 
-// 3 CTAs per SM: the degree-3 instance fits in 85 registers with a few bytes
-// of spill, faster than 2 CTAs at 92
+// 4 CTAs of 256 per SM (64 registers, a few spilled): on the 6M view the
+// kernel takes 0.615 ms, against 0.665 ms at 3 CTAs (80 registers) and
+// 0.632 ms with 8 CTAs of 128
 template <int D>
-__global__ void __launch_bounds__(kProjThreads, 3)
+__global__ void __launch_bounds__(kProjThreads, GS_PROJ_MINB)
 k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam cam,
           int32_t* __restrict__ cand_idx, int32_t* __restrict__ slot_map, float4* __restrict__ rec,
           short4* __restrict__ rect, uint32_t* __restrict__ depth_key, int32_t* __restrict__ diff,
@@ -254,8 +261,6 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
           unsigned long long* __restrict__ square_isect, bool dense, bool prefetch,
           int32_t* dev_status) {
   __shared__ unsigned int s_b;
-  __shared__ int s_scan[kProjThreads / 32 + 1];
-  __shared__ long long s_prefix;
   if (threadIdx.x == 0) s_b = atomicAdd(ticket, 1u);
   __syncthreads();
   const int64_t b = s_b;
@@ -315,19 +320,21 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
     }
     return;
   }
-  int total;
-  const int rank = block_exclusive_scan<int, kProjThreads / 32>(cand ? 1 : 0, s_scan, &total);
-  // warp 0 resolves the block's prefix while every warp forms its
-  // candidates' records (which do not depend on the slot), so the look-back
-  // latency hides behind the SH reads and arithmetic
-  if (threadIdx.x < 32) {
-    int64_t ex = lookback_warp(lb, b, total, dev_status);
-    if (threadIdx.x == 0) s_prefix = ex;
-  }
+  // ordered compaction by warps: each warp publishes its candidate count,
+  // forms its candidates' records (which do not depend on the slot), and
+  // only then resolves its prefix from the warps before it (numbered by the
+  // block ticket, so a warp waits only on warps that have started); no CTA
+  // barrier, so a warp never waits for its block's slowest warp
+  const unsigned lane = threadIdx.x & 31;
+  const unsigned bal = __ballot_sync(0xffffffffu, cand);
+  const int total = __popc(bal);
+  const int rank = __popc(bal & ((1u << lane) - 1u));
+  const int64_t wid = b * (kProjThreads / 32) + (threadIdx.x >> 5);
+  lookback_publish(lb, wid, total);
   float4 r0, r1, r2;
   if (cand) sh_record<D>(params, n_pad, i, cam, o, r0, r1, r2);
-  __syncthreads();
-  const int64_t slot = s_prefix + rank;
+  const int64_t prefix = lookback_resolve(lb, wid, total, dev_status);
+  const int64_t slot = prefix + rank;
   const bool fits = slot < capacity;  // false beyond the caller's capacity (it retries)
   if (cand && !fits) dev_flag(dev_status, GS_DEV_BOUNDS);
   if (i < n) slot_map[i] = (cand && fits) ? (int32_t)slot : -1;
@@ -344,7 +351,7 @@ k_project(const float* __restrict__ params, int64_t n, int64_t n_pad, ProjCam ca
     atomicAdd(&diff[o.rect.w * s + o.rect.x], -1);
     atomicAdd(&diff[o.rect.w * s + o.rect.z], 1);
   }
-  if (b == n_blocks - 1 && threadIdx.x == 0) *n_cand = (int32_t)(s_prefix + total);
+  if (wid == n_blocks * (kProjThreads / 32) - 1 && lane == 0) *n_cand = (int32_t)(prefix + total);
   if (square_isect) {
     unsigned long long sq = counted ? (unsigned long long)o.square_tiles : 0ull;
     sq = warp_sum(sq);
@@ -455,7 +462,7 @@ ProjWs carve_proj(void* ws, size_t cap, int64_t n, int32_t W, int32_t H) {
   const int64_t nb = (n + kProjThreads - 1) / kProjThreads;
   ProjWs p;
   p.ticket = cv.take<unsigned int>(64);
-  p.lb = cv.take<unsigned long long>(nb > 0 ? nb : 1);
+  p.lb = cv.take<unsigned long long>(nb > 0 ? nb * (kProjThreads / 32) : 1);  // per warp
   p.diff = cv.take<int32_t>((TW + 1) * (TH + 1));
   p.tmp = cv.take<int64_t>(TW * TH);
   p.bytes = cv.off;
