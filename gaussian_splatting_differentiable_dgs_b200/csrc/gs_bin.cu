@@ -413,18 +413,269 @@ k_expand_write(const short4* __restrict__ rect, const int32_t* __restrict__ bloc
   if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
 }
 
+// ---------------------------------------------------------------------------
+// Block lists by a counting scatter (no sort), for grids of up to
+// kScatMaxBlocks blocks.  The candidates in depth order are cut into chunks
+// of `chunk` candidates.  (A) k_blk_count: per chunk, its entries per block
+// (a candidate has one entry in each block its tile rect meets).  (S)
+// k_blk_scan: per block, the exclusive scan of those counts over the chunks,
+// offset by the block's start in the block lists (from the block SAT), so
+// offs[c][b] is where chunk c's first entry of block b goes.  (B)
+// k_blk_scatter: one warp per chunk walks its candidates in depth order and
+// writes each entry to offs[c][b] + the entries of block b it has written
+// so far (a cursor per block in shared memory, advanced by match_any
+// groups), so every block list is in depth order with ties by candidate
+// position: the order of a stable sort of (block, depth) keys.
+// ---------------------------------------------------------------------------
+#ifndef GS_SCAT_MAX_BLOCKS
+#define GS_SCAT_MAX_BLOCKS 4096
+#endif
+constexpr int kScatMaxBlocks = GS_SCAT_MAX_BLOCKS;
+constexpr int64_t kScatCountBudget = 4 << 20;  // counts per view (16 MB)
+
+int64_t scat_chunk(int64_t n_cand, int64_t nblocks) {
+  int64_t c = (n_cand * nblocks + kScatCountBudget - 1) / kScatCountBudget;
+  c = c < 1024 ? 1024 : c;
+  return (c + 31) / 32 * 32;
+}
+
+struct BlockRect {
+  int bx0, by0, bw, n;  // first block, width in blocks, number of blocks (0 = none)
+};
+
+__device__ __forceinline__ BlockRect block_rect(short4 r, int BW, int BH) {
+  BlockRect b{0, 0, 1, 0};
+  if (r.z <= r.x || r.w <= r.y) return b;  // empty (a culled Gaussian of the dense layout)
+  const int bx0 = r.x / GS_TILE_BLOCK, by0 = r.y / GS_TILE_BLOCK;
+  const int bx1 = min((r.z - 1) / GS_TILE_BLOCK + 1, BW), by1 = min((r.w - 1) / GS_TILE_BLOCK + 1, BH);
+  if (bx1 <= bx0 || by1 <= by0) return b;
+  b.bx0 = bx0;
+  b.by0 = by0;
+  b.bw = bx1 - bx0;
+  b.n = b.bw * (by1 - by0);
+  return b;
+}
+
+constexpr int kScatSeg = 64;  // chunk segments of the offsets' scan
+
+// Per chunk, its entries per block through a 2D difference grid in shared
+// memory: 4 atomics per candidate at its block rect's corners, then a 2D
+// prefix sum (rows, then columns), so a candidate costs the same whatever
+// its size.
+__global__ void __launch_bounds__(256)
+k_blk_count(const short4* __restrict__ drect, int64_t n_cand, int64_t chunk, int BW, int BH,
+            uint32_t* __restrict__ counts) {
+  extern __shared__ int32_t s_d[];  // [(BH + 1) * (BW + 1)]
+  const int sw = BW + 1, cells = (BH + 1) * sw;
+  for (int b = threadIdx.x; b < cells; b += 256) s_d[b] = 0;
+  __syncthreads();
+  const int64_t c = blockIdx.x;
+  const int64_t j1 = min(n_cand, (c + 1) * chunk);
+  for (int64_t base = c * chunk; base < j1; base += 4 * 256) {
+    short4 r[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {  // four loads in flight per thread
+      const int64_t j = base + k * 256 + threadIdx.x;
+      r[k] = j < j1 ? drect[j] : make_short4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const BlockRect br = block_rect(r[k], BW, BH);
+      if (br.n == 0) continue;
+      const int bx1 = br.bx0 + br.bw, by1 = br.by0 + br.n / br.bw;
+      atomicAdd(&s_d[br.by0 * sw + br.bx0], 1);
+      atomicAdd(&s_d[br.by0 * sw + bx1], -1);
+      atomicAdd(&s_d[by1 * sw + br.bx0], -1);
+      atomicAdd(&s_d[by1 * sw + bx1], 1);
+    }
+  }
+  __syncthreads();
+  for (int y = threadIdx.x; y < BH; y += 256) {  // prefix along each row
+    int run = 0;
+    for (int x = 0; x < BW; ++x) {
+      run += s_d[y * sw + x];
+      s_d[y * sw + x] = run;
+    }
+  }
+  __syncthreads();
+  for (int x = threadIdx.x; x < BW; x += 256) {  // then down each column
+    int run = 0;
+    for (int y = 0; y < BH; ++y) {
+      run += s_d[y * sw + x];
+      s_d[y * sw + x] = run;
+    }
+  }
+  __syncthreads();
+  const int nbk = BW * BH;
+  for (int b = threadIdx.x; b < nbk; b += 256) counts[c * nbk + b] = (uint32_t)s_d[(b / BW) * sw + b % BW];
+}
+
+// Offsets in two levels over kScatSeg segments of chunks.  One CTA per
+// (32 blocks, segment): lane = block, the 8 warps split the segment.
+// k_blk_segsum: the segment's total per block.
+__global__ void __launch_bounds__(256)
+k_blk_segsum(const uint32_t* __restrict__ counts, int64_t n_chunks, int nbk,
+             uint32_t* __restrict__ segtot) {
+  __shared__ uint32_t s_tot[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int b = blockIdx.x * 32 + lane;
+  const int64_t L = (n_chunks + kScatSeg - 1) / kScatSeg;
+  const int64_t c0 = min(n_chunks, blockIdx.y * L), c1 = min(n_chunks, c0 + L);
+  const int64_t l = (c1 - c0 + 7) / 8;
+  const int64_t a0 = min(c1, c0 + w * l), a1 = min(c1, a0 + l);
+  uint32_t tot = 0;
+  if (b < nbk) {
+#pragma unroll 4
+    for (int64_t c = a0; c < a1; ++c) tot += counts[c * nbk + b];
+  }
+  s_tot[w][lane] = tot;
+  __syncthreads();
+  if (w == 0 && b < nbk) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) t += s_tot[ww][lane];
+    segtot[(int64_t)blockIdx.y * nbk + b] = t;
+  }
+}
+
+// k_blk_offs: counts[c][b] <- the block list position of chunk c's first
+// entry of block b (exclusive scan over the chunks, from the block's start).
+__global__ void __launch_bounds__(256)
+k_blk_offs(uint32_t* __restrict__ counts, int64_t n_chunks, int nbk,
+           const uint32_t* __restrict__ segtot, const int64_t* __restrict__ block_ranges,
+           int32_t* dev_status) {
+  __shared__ uint32_t s_tot[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int b = blockIdx.x * 32 + lane;
+  const int64_t L = (n_chunks + kScatSeg - 1) / kScatSeg;
+  const int64_t c0 = min(n_chunks, blockIdx.y * L), c1 = min(n_chunks, c0 + L);
+  const int64_t l = (c1 - c0 + 7) / 8;
+  const int64_t a0 = min(c1, c0 + w * l), a1 = min(c1, a0 + l);
+  uint32_t tot = 0;
+  if (b < nbk) {
+#pragma unroll 4
+    for (int64_t c = a0; c < a1; ++c) tot += counts[c * nbk + b];
+  }
+  s_tot[w][lane] = tot;
+  __syncthreads();
+  if (b >= nbk) return;
+  int64_t run = block_ranges[2 * b];
+  for (int s = 0; s < (int)blockIdx.y; ++s) run += segtot[(int64_t)s * nbk + b];
+  for (int ww = 0; ww < w; ++ww) run += s_tot[ww][lane];
+  for (int64_t c = a0; c < a1; ++c) {
+    const uint32_t v = counts[c * nbk + b];
+    counts[c * nbk + b] = (uint32_t)run;
+    run += v;
+  }
+  // the last chunk of the last segment ends at the block's end
+  if (blockIdx.y == gridDim.y - 1 && w == 7 && run != block_ranges[2 * b + 1])
+    dev_flag(dev_status, GS_DEV_BOUNDS);
+}
+
+// One warp per chunk: a cursor per block in shared memory; each round of 32
+// candidates (inputs prefetched one round ahead) emits its entries in
+// (candidate, block row-major) order, 32 at a time.  The row of entry q of
+// a w-block-wide rect is floor((q + 0.5) / w) in fp32: exact, since
+// q + w < 2^21 keeps the error of the product below 0.5 / w.
+__global__ void __launch_bounds__(32)
+k_blk_scatter(const short4* __restrict__ drect, const int32_t* __restrict__ order,
+              int64_t n_cand, int64_t chunk, int BW, int BH, const uint32_t* __restrict__ offs,
+              int32_t* __restrict__ block_vals, int64_t capacity, int32_t* dev_status) {
+  extern __shared__ uint32_t s_cur[];  // [nbk]
+  __shared__ int s_ex[32], s_bx[32], s_by[32], s_bw[32], s_slot[32];
+  __shared__ float s_rw[32];
+  const int lane = threadIdx.x;
+  const int nbk = BW * BH;
+  const int64_t c = blockIdx.x;
+#pragma unroll 4
+  for (int b = lane; b < nbk; b += 32) s_cur[b] = offs[c * nbk + b];
+  const int64_t j0 = c * chunk, j1 = min(n_cand, j0 + chunk);
+  const unsigned lt = (1u << lane) - 1u;
+  bool bad = false;
+  short4 nr = make_short4(0, 0, 0, 0);
+  int32_t nsl = 0;
+  if (j0 + lane < j1) {
+    nr = drect[j0 + lane];
+    nsl = order[j0 + lane];
+  }
+  __syncwarp();
+  for (int64_t base = j0; base < j1; base += 32) {
+    const short4 r = nr;
+    const int32_t slot = nsl;
+    const bool valid = base + lane < j1;
+    if (base + 32 + lane < j1) {  // the next round's inputs
+      nr = drect[base + 32 + lane];
+      nsl = order[base + 32 + lane];
+    }
+    BlockRect br{0, 0, 1, 0};
+    if (valid) br = block_rect(r, BW, BH);
+    int incl = br.n;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    s_ex[lane] = incl - br.n;
+    s_bx[lane] = br.bx0;
+    s_by[lane] = br.by0;
+    s_bw[lane] = br.bw;
+    s_rw[lane] = 1.0f / (float)br.bw;
+    s_slot[lane] = slot;
+    __syncwarp();
+    for (int e0 = 0; e0 < total; e0 += 32) {
+      const int e = e0 + lane;
+      int b = -1, sl = 0;
+      if (e < total) {
+        int lo = 0;  // the last candidate whose first entry is <= e
+#pragma unroll
+        for (int step = 16; step > 0; step >>= 1)
+          if (s_ex[lo + step] <= e) lo += step;
+        const int q = e - s_ex[lo], bw = s_bw[lo];
+        const int row = (int)(((float)q + 0.5f) * s_rw[lo]);
+        b = (s_by[lo] + row) * BW + s_bx[lo] + (q - row * bw);
+        sl = s_slot[lo];
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, b);
+      if (b >= 0) {
+        const uint32_t cur = s_cur[b];
+        const int64_t pos = (int64_t)cur + __popc(peers & lt);
+        if (pos < capacity) block_vals[pos] = sl;
+        else bad = true;
+        __syncwarp(peers);
+        if (lane == __ffs(peers) - 1) s_cur[b] = cur + (uint32_t)__popc(peers);
+      }
+      __syncwarp();
+    }
+  }
+  if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
+}
+
 struct BlockBinWs {
   unsigned int* ticket;
   unsigned long long* lb;
   uint32_t* keys;
   void* sort_ws;
   size_t sort_bytes;
+  uint32_t* counts;   // counting scatter: [n_chunks][nblocks]
+  uint32_t* segtot;   // [kScatSeg][nblocks]
+  int64_t chunk, n_chunks;
+  bool scatter;
   size_t bytes;
 };
 
 BlockBinWs carve_block_bin(void* ws, size_t cap, int64_t n_cand, int64_t n_entries, int64_t nblocks) {
   Carver cv(ws, cap);
-  BlockBinWs w;
+  BlockBinWs w{};
+  w.scatter = nblocks <= kScatMaxBlocks;
+  if (w.scatter) {
+    w.chunk = scat_chunk(n_cand, nblocks);
+    w.n_chunks = (n_cand + w.chunk - 1) / w.chunk;
+    w.counts = cv.take<uint32_t>(w.n_chunks > 0 ? w.n_chunks * nblocks : 1);
+    w.segtot = cv.take<uint32_t>(kScatSeg * nblocks);
+    w.bytes = cv.off;
+    return w;
+  }
   w.ticket = cv.take<unsigned int>(64);
   const int64_t nb = (n_cand + kBinChunk - 1) / kBinChunk;
   w.lb = cv.take<unsigned long long>(nb > 0 ? nb : 1);
@@ -599,6 +850,24 @@ extern "C" gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand, const in
   k_ranges<<<(unsigned)((nblocks + 255) / 256), 256, 0, s>>>(block_sat, grid, BW, block_ranges);
   GS_LAUNCH_CHECK();
   if (n_cand == 0 || n_entries == 0) return GS_OK;
+  if (w.scatter) {
+    const int nbk = (int)nblocks;
+    const size_t smem = (size_t)nbk * sizeof(uint32_t);  // <= 16 KB
+    const size_t smem_d = (size_t)(BW + 1) * (BH + 1) * sizeof(int32_t);
+    k_blk_count<<<(unsigned)w.n_chunks, 256, smem_d, s>>>(
+        reinterpret_cast<const short4*>(depth_rect), n_cand, w.chunk, BW, BH, w.counts);
+    GS_LAUNCH_CHECK();
+    const dim3 sg((unsigned)((nbk + 31) / 32), kScatSeg);
+    k_blk_segsum<<<sg, 256, 0, s>>>(w.counts, w.n_chunks, nbk, w.segtot);
+    GS_LAUNCH_CHECK();
+    k_blk_offs<<<sg, 256, 0, s>>>(w.counts, w.n_chunks, nbk, w.segtot, block_ranges, dev_status);
+    GS_LAUNCH_CHECK();
+    k_blk_scatter<<<(unsigned)w.n_chunks, 32, smem, s>>>(
+        reinterpret_cast<const short4*>(depth_rect), depth_order, n_cand, w.chunk, BW, BH,
+        w.counts, block_vals, capacity, dev_status);
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+  }
   GS_TRY(cudaMemsetAsync(ws, 0, (size_t)((char*)w.keys - (char*)ws), s));
   const int64_t nb = (n_cand + kBinChunk - 1) / kBinChunk;
   k_bin<kBlk><<<(unsigned)nb, kBinThreads, 0, s>>>(

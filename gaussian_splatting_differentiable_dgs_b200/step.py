@@ -250,12 +250,12 @@ class Stepper:
         nc_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
         sq_h = torch.empty(1, dtype=torch.int64, pin_memory=True)
         while True:
-            n_cand_d = torch.zeros(1, dtype=torch.int32, device=dev)
+            n_cand_d = torch.empty(1, dtype=torch.int32, device=dev)   # written by gs_project
             cand_idx = torch.empty(cap, dtype=torch.int32, device=dev)
             rec = torch.empty(cap * 12, dtype=torch.float32, device=dev)
             rect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
             dkey = torch.empty(cap, dtype=torch.int32, device=dev)
-            sq_d = torch.zeros(1, dtype=torch.int64, device=dev)
+            sq_d = torch.empty(1, dtype=torch.int64, device=dev)       # cleared by gs_project
             proj = B.gs_proj(cap, n_cand_d.data_ptr(), cand_idx.data_ptr(), slot.data_ptr(),
                              rec.data_ptr(), rect.data_ptr(), dkey.data_ptr(), sq_d.data_ptr())
             if region is None:
@@ -344,7 +344,12 @@ class Stepper:
 
         # ---- per-Leaf raster: forward + L1 + backward into compact g2d ------
         g2d = torch.zeros(max(C, 1) * 12, dtype=torch.float32, device=dev)
-        loss_tiles = torch.zeros(T, dtype=torch.float32, device=dev)
+        # every tile's loss partial is written by its Leaf's forward when the
+        # planned Leaves cover the grid; a region or caller-given Leaves may
+        # leave tiles out, which must then count zero
+        zero_tiles = region is not None or leaves is not None
+        loss_tiles = (torch.zeros if zero_tiles else torch.empty)(T, dtype=torch.float32,
+                                                                    device=dev)
         if fused:
             bin_ws = torch.empty(256, dtype=torch.uint8, device=dev)
         elif expand:
@@ -509,10 +514,11 @@ class Stepper:
         # with their backward; the projection and lists are reused)
         if gate is not None and backward:
             leaf_pass(False)
-            pre = torch.zeros(1, dtype=torch.float64, device=dev)
+            pre = torch.empty(1, dtype=torch.float64, device=dev)  # written by gs_loss_total
             B.gs_loss_total(loss_tiles, T, pre)
             if gate(float(pre.item())):
-                loss_tiles.zero_()
+                if zero_tiles:
+                    loss_tiles.zero_()
                 leaf_pass(True)
             else:
                 backward = update = False
@@ -527,7 +533,8 @@ class Stepper:
             if host_target:
                 del crops
 
-        loss_d = torch.zeros(1, dtype=torch.float64, device=dev)
+        loss_d = torch.zeros(1, dtype=torch.float64, device=dev) if target is None else \
+            torch.empty(1, dtype=torch.float64, device=dev)
         if target is not None:
             B.gs_loss_total(loss_tiles, T, loss_d)
         self._last_loss = loss_d

@@ -1095,42 +1095,59 @@ def test_grouped_step_matches_oracle(oracle_mod):
     assert d.max() <= 2.1e-3  # at most one sign flip of a ~zero gradient
 
 
-@pytest.mark.parametrize("blocks", [(2, 2), (3, 3)])
-def test_fixed_block_schedule_matches_oracle(oracle_mod, blocks):
-    """The fixed-block schedule (BoundedGS page, Figs. 5-6): the view cut into
-    a fixed grid, each block a step of its own (its candidates, the view's
-    loss normaliser) with its own Adam update, t = 1 .. B.  The oracle
-    composes the same schedule from its step restricted to each block's
-    tiles, block after block from the updated parameters.  Compared: the
-    summed loss, Adam's moments (magnitude of every block's gradient) and
-    the parameters."""
-    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
-    sc, cam = scene("hd")
-    tgt = synth.random_image(cam.width, cam.height, 4) * 0.5
-    TW, TH = oracle_mod.grid(cam)
-    model = GaussianModel(sc.params, sc.n, sc.sh_degree)
-    stp = Stepper(model, budget=4 << 20)
-    stats = stp.run_view_blocks(cam, torch.as_tensor(tgt).cuda(), blocks=blocks)
-    stp.check()
-    regions = Stepper.split_regions(TW, TH, *blocks)
-    nb = len(regions)
-    assert model.step == nb and nb == blocks[0] * blocks[1]
+def _oracle_blocks(oracle_mod, sc, cam, tgt, regions, lr):
+    """The oracle's fixed-block schedule: its step restricted to each block's
+    tiles, block after block from the updated parameters, Adam t = 1 .. B."""
     p = sc.params.astype(np.float64)
     m = np.zeros_like(p)
     v = np.zeros_like(p)
     loss = 0.0
     for k, r in enumerate(regions):
         ref = oracle_mod.step(p, sc.n, sc.sh_degree, cam, tgt.astype(np.float64),
-                              leaves=[r], m=m, v=v, t=k + 1)
+                              leaves=[r], m=m, v=v, t=k + 1, lr=lr)
         p, m, v, loss = ref["params"], ref["m"], ref["v"], loss + ref["loss"]
+    return p, m, v, loss
+
+
+@pytest.mark.parametrize("blocks", [(2, 2), (3, 3)])
+@pytest.mark.parametrize("lr", [0.0, 1e-3])
+def test_fixed_block_schedule_matches_oracle(oracle_mod, blocks, lr):
+    """The fixed-block schedule (BoundedGS page, Figs. 5-6): the view cut into
+    a fixed grid, each block a step of its own (its candidates, the view's
+    loss normaliser) with its own Adam update, t = 1 .. B, against the oracle
+    composing the same schedule.
+
+    With lr = 0 every block's gradient is taken at the same parameters on
+    both sides, so Adam's moments (the decayed sum of the blocks' gradients
+    and of their squares) meet the gradient tolerance.  With lr = 1e-3 a
+    later block sees parameters that differ from the oracle's by the fp32
+    rounding of the earlier updates, which can move a pixel across a
+    threshold decision; the moments then get a ten times looser bound, and
+    the parameters the per-update bound of the single-step tests."""
+    from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
+    sc, cam = scene("hd")
+    tgt = synth.random_image(cam.width, cam.height, 4) * 0.5
+    TW, TH = oracle_mod.grid(cam)
+    model = GaussianModel(sc.params, sc.n, sc.sh_degree)
+    stp = Stepper(model, budget=4 << 20, lr=lr)
+    stp.run_view_blocks(cam, torch.as_tensor(tgt).cuda(), blocks=blocks)
+    stp.check()
+    regions = Stepper.split_regions(TW, TH, *blocks)
+    nb = len(regions)
+    assert model.step == nb and nb == blocks[0] * blocks[1]
+    p, m, v, loss = _oracle_blocks(oracle_mod, sc, cam, tgt, regions, lr)
     assert abs(stp.last_loss() - loss) <= IMG_TOL * loss
     n = sc.n
+    tol = GRAD_TOL if lr == 0.0 else 10 * GRAD_TOL
     mg, vg = model.m.cpu().numpy(), model.v.cpu().numpy()
     for gname, a, e in GROUPS:
         e = sc.P if e is None else e
-        assert rel_l2(mg[a:e, :n], m[a:e, :n]) <= GRAD_TOL, gname
-        assert rel_l2(vg[a:e, :n], v[a:e, :n]) <= 2 * GRAD_TOL, gname
+        assert rel_l2(mg[a:e, :n], m[a:e, :n]) <= tol, gname
+        assert rel_l2(vg[a:e, :n], v[a:e, :n]) <= 2 * tol, gname
     pg = model.params.cpu().numpy()
+    if lr == 0.0:
+        assert (pg == sc.params).all()
+        return
     dp = np.abs(pg[:, :n] - p[:, :n])
     big = np.abs(m[:, :n]) > 1e-3 * np.abs(m[:, :n]).max(axis=1, keepdims=True)
     assert dp[big].max() <= 1e-5 * nb
