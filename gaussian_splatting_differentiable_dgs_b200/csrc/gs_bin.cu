@@ -431,6 +431,7 @@ k_expand_write(const short4* __restrict__ rect, const int32_t* __restrict__ bloc
 #define GS_SCAT_MAX_BLOCKS 4096
 #endif
 constexpr int kScatMaxBlocks = GS_SCAT_MAX_BLOCKS;
+constexpr size_t kScatMaxSmem = 160 << 10;  // the scatter's per-warp count grids
 constexpr int64_t kScatCountBudget = 4 << 20;  // counts per view (16 MB)
 
 int64_t scat_chunk(int64_t n_cand, int64_t nblocks) {
@@ -572,43 +573,78 @@ k_blk_offs(uint32_t* __restrict__ counts, int64_t n_chunks, int nbk,
     dev_flag(dev_status, GS_DEV_BOUNDS);
 }
 
-// One warp per chunk: a cursor per block in shared memory; each round of 32
-// candidates (inputs prefetched one round ahead) emits its entries in
-// (candidate, block row-major) order, 32 at a time.  The row of entry q of
-// a w-block-wide rect is floor((q + 0.5) / w) in fp32: exact, since
-// q + w < 2^21 keeps the error of the product below 0.5 / w.
-__global__ void __launch_bounds__(32)
+// One CTA of kScatWarps warps per chunk; warp w takes the w-th contiguous
+// part of the chunk.  Each warp counts its part per block in its own 2D
+// difference grid in shared memory; the prefix sums turn the grids into
+// counts, and the CTA turns those into each warp's start per block (the
+// chunk's offset plus the counts of the warps before it).  Each warp then
+// emits its part in rounds of 32 candidates, entries in (candidate, block
+// row-major) order, 32 at a time, advancing its cursors by match_any groups.
+// The row of entry q of a w-block-wide rect is floor((q + 0.5) / w) in
+// fp32: exact, since q + w < 2^21 keeps the product's error below 0.5 / w.
+constexpr int kScatWarps = 8;
+
+__global__ void __launch_bounds__(kScatWarps * 32)
 k_blk_scatter(const short4* __restrict__ drect, const int32_t* __restrict__ order,
               int64_t n_cand, int64_t chunk, int BW, int BH, const uint32_t* __restrict__ offs,
               int32_t* __restrict__ block_vals, int64_t capacity, int32_t* dev_status) {
-  extern __shared__ uint32_t s_cur[];  // [nbk]
-  __shared__ int s_ex[32], s_bx[32], s_by[32], s_bw[32], s_slot[32];
-  __shared__ float s_rw[32];
-  const int lane = threadIdx.x;
-  const int nbk = BW * BH;
+  extern __shared__ int32_t s_g[];  // [kScatWarps][(BH + 1) * (BW + 1)]
+  __shared__ int s_ex[kScatWarps][32], s_bx[kScatWarps][32], s_by[kScatWarps][32],
+      s_bw[kScatWarps][32], s_slot[kScatWarps][32];
+  __shared__ float s_rw[kScatWarps][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int sw = BW + 1, cells = (BH + 1) * sw, nbk = BW * BH;
+  int32_t* g = s_g + w * cells;
   const int64_t c = blockIdx.x;
-#pragma unroll 4
-  for (int b = lane; b < nbk; b += 32) s_cur[b] = offs[c * nbk + b];
-  const int64_t j0 = c * chunk, j1 = min(n_cand, j0 + chunk);
-  const unsigned lt = (1u << lane) - 1u;
-  bool bad = false;
-  short4 nr = make_short4(0, 0, 0, 0);
-  int32_t nsl = 0;
-  if (j0 + lane < j1) {
-    nr = drect[j0 + lane];
-    nsl = order[j0 + lane];
+  const int64_t cj0 = c * chunk, cj1 = min(n_cand, cj0 + chunk);
+  const int64_t part = (cj1 - cj0 + kScatWarps - 1) / kScatWarps;
+  const int64_t j0 = min(cj1, cj0 + w * part), j1 = min(cj1, j0 + part);
+  for (int b = threadIdx.x; b < kScatWarps * cells; b += kScatWarps * 32) s_g[b] = 0;
+  __syncthreads();
+  // (1) this warp's counts per block
+  for (int64_t j = j0 + lane; j < j1; j += 32) {
+    const BlockRect br = block_rect(drect[j], BW, BH);
+    if (br.n == 0) continue;
+    const int bx1 = br.bx0 + br.bw, by1 = br.by0 + br.n / br.bw;
+    atomicAdd(&g[br.by0 * sw + br.bx0], 1);
+    atomicAdd(&g[br.by0 * sw + bx1], -1);
+    atomicAdd(&g[by1 * sw + br.bx0], -1);
+    atomicAdd(&g[by1 * sw + bx1], 1);
   }
   __syncwarp();
-  for (int64_t base = j0; base < j1; base += 32) {
-    const short4 r = nr;
-    const int32_t slot = nsl;
-    const bool valid = base + lane < j1;
-    if (base + 32 + lane < j1) {  // the next round's inputs
-      nr = drect[base + 32 + lane];
-      nsl = order[base + 32 + lane];
+  for (int y = lane; y < BH; y += 32) {
+    int run = 0;
+    for (int x = 0; x < BW; ++x) run = (g[y * sw + x] += run);
+  }
+  __syncwarp();
+  for (int x = lane; x < BW; x += 32) {
+    int run = 0;
+    for (int y = 0; y < BH; ++y) run = (g[y * sw + x] += run);
+  }
+  __syncthreads();
+  // (2) counts -> each warp's first position per block
+  for (int b = threadIdx.x; b < nbk; b += kScatWarps * 32) {
+    const int cell = (b / BW) * sw + b % BW;
+    int32_t run = (int32_t)offs[c * nbk + b];
+#pragma unroll
+    for (int ww = 0; ww < kScatWarps; ++ww) {
+      const int32_t v = s_g[ww * cells + cell];
+      s_g[ww * cells + cell] = run;
+      run += v;
     }
+  }
+  __syncthreads();
+  // (3) emission
+  const unsigned lt = (1u << lane) - 1u;
+  bool bad = false;
+  for (int64_t base = j0; base < j1; base += 32) {
+    const int64_t j = base + lane;
     BlockRect br{0, 0, 1, 0};
-    if (valid) br = block_rect(r, BW, BH);
+    int32_t slot = 0;
+    if (j < j1) {
+      br = block_rect(drect[j], BW, BH);
+      slot = order[j];
+    }
     int incl = br.n;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -616,39 +652,44 @@ k_blk_scatter(const short4* __restrict__ drect, const int32_t* __restrict__ orde
       if (lane >= d) incl += v;
     }
     const int total = __shfl_sync(0xffffffffu, incl, 31);
-    s_ex[lane] = incl - br.n;
-    s_bx[lane] = br.bx0;
-    s_by[lane] = br.by0;
-    s_bw[lane] = br.bw;
-    s_rw[lane] = 1.0f / (float)br.bw;
-    s_slot[lane] = slot;
+    __syncwarp();
+    s_ex[w][lane] = incl - br.n;
+    s_bx[w][lane] = br.bx0;
+    s_by[w][lane] = br.by0;
+    s_bw[w][lane] = br.bw;
+    s_rw[w][lane] = 1.0f / (float)br.bw;
+    s_slot[w][lane] = slot;
     __syncwarp();
     for (int e0 = 0; e0 < total; e0 += 32) {
       const int e = e0 + lane;
-      int b = -1, sl = 0;
+      int cell = -1, sl = 0;
       if (e < total) {
         int lo = 0;  // the last candidate whose first entry is <= e
 #pragma unroll
         for (int step = 16; step > 0; step >>= 1)
-          if (s_ex[lo + step] <= e) lo += step;
-        const int q = e - s_ex[lo], bw = s_bw[lo];
-        const int row = (int)(((float)q + 0.5f) * s_rw[lo]);
-        b = (s_by[lo] + row) * BW + s_bx[lo] + (q - row * bw);
-        sl = s_slot[lo];
+          if (s_ex[w][lo + step] <= e) lo += step;
+        const int q = e - s_ex[w][lo], bw = s_bw[w][lo];
+        const int row = (int)(((float)q + 0.5f) * s_rw[w][lo]);
+        cell = (s_by[w][lo] + row) * sw + s_bx[w][lo] + (q - row * bw);
+        sl = s_slot[w][lo];
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, b);
-      if (b >= 0) {
-        const uint32_t cur = s_cur[b];
+      const unsigned peers = __match_any_sync(0xffffffffu, cell);
+      if (cell >= 0) {
+        const int32_t cur = g[cell];
         const int64_t pos = (int64_t)cur + __popc(peers & lt);
         if (pos < capacity) block_vals[pos] = sl;
         else bad = true;
         __syncwarp(peers);
-        if (lane == __ffs(peers) - 1) s_cur[b] = cur + (uint32_t)__popc(peers);
+        if (lane == __ffs(peers) - 1) g[cell] = cur + __popc(peers);
       }
       __syncwarp();
     }
   }
   if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
+}
+
+size_t scat_smem(int64_t BW, int64_t BH) {
+  return (size_t)kScatWarps * (BW + 1) * (BH + 1) * sizeof(int32_t);
 }
 
 struct BlockBinWs {
@@ -664,10 +705,12 @@ struct BlockBinWs {
   size_t bytes;
 };
 
-BlockBinWs carve_block_bin(void* ws, size_t cap, int64_t n_cand, int64_t n_entries, int64_t nblocks) {
+BlockBinWs carve_block_bin(void* ws, size_t cap, int64_t n_cand, int64_t n_entries, int64_t TWB,
+                           int64_t THB) {
+  const int64_t nblocks = TWB * THB;
   Carver cv(ws, cap);
   BlockBinWs w{};
-  w.scatter = nblocks <= kScatMaxBlocks;
+  w.scatter = nblocks <= kScatMaxBlocks && scat_smem(TWB, THB) <= kScatMaxSmem;
   if (w.scatter) {
     w.chunk = scat_chunk(n_cand, nblocks);
     w.n_chunks = (n_cand + w.chunk - 1) / w.chunk;
@@ -818,8 +861,8 @@ extern "C" gs_status gs_bin_tiles(const gs_proj* proj, int64_t n_cand, const int
 extern "C" size_t gs_bin_blocks_workspace_size(int64_t n_cand, int64_t n_entries, int32_t TW,
                                                int32_t TH) {
   if (n_cand < 0 || n_entries < 0 || TW <= 0 || TH <= 0) return 0;
-  const int64_t nblocks = (int64_t)((TW + kBlk - 1) / kBlk) * ((TH + kBlk - 1) / kBlk);
-  return carve_block_bin(nullptr, 0, n_cand, n_entries, nblocks).bytes;
+  return carve_block_bin(nullptr, 0, n_cand, n_entries, (TW + kBlk - 1) / kBlk,
+                         (TH + kBlk - 1) / kBlk).bytes;
 }
 
 extern "C" gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand, const int32_t* depth_order,
@@ -839,7 +882,7 @@ extern "C" gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand, const in
   if (n_entries > 0 && !block_vals) return GS_ERR_ARG;
   const int32_t BW = (TW + kBlk - 1) / kBlk, BH = (TH + kBlk - 1) / kBlk;
   const int64_t nblocks = (int64_t)BW * BH;
-  BlockBinWs w = carve_block_bin(ws, ws_bytes, n_cand, n_entries, nblocks);
+  BlockBinWs w = carve_block_bin(ws, ws_bytes, n_cand, n_entries, BW, BH);
   if (!ws || w.bytes > ws_bytes) {
     if (needed) *needed = (int64_t)w.bytes;
     return GS_ERR_CAPACITY;
@@ -852,7 +895,6 @@ extern "C" gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand, const in
   if (n_cand == 0 || n_entries == 0) return GS_OK;
   if (w.scatter) {
     const int nbk = (int)nblocks;
-    const size_t smem = (size_t)nbk * sizeof(uint32_t);  // <= 16 KB
     const size_t smem_d = (size_t)(BW + 1) * (BH + 1) * sizeof(int32_t);
     k_blk_count<<<(unsigned)w.n_chunks, 256, smem_d, s>>>(
         reinterpret_cast<const short4*>(depth_rect), n_cand, w.chunk, BW, BH, w.counts);
@@ -862,7 +904,12 @@ extern "C" gs_status gs_bin_blocks(const gs_proj* proj, int64_t n_cand, const in
     GS_LAUNCH_CHECK();
     k_blk_offs<<<sg, 256, 0, s>>>(w.counts, w.n_chunks, nbk, w.segtot, block_ranges, dev_status);
     GS_LAUNCH_CHECK();
-    k_blk_scatter<<<(unsigned)w.n_chunks, 32, smem, s>>>(
+    const size_t smem_sc = scat_smem(BW, BH);  // <= kScatMaxSmem
+    {
+      static std::atomic<unsigned long long> done{0};
+      GS_TRY(smem_attrs_once((const void*)k_blk_scatter, (int)kScatMaxSmem, &done));
+    }
+    k_blk_scatter<<<(unsigned)w.n_chunks, kScatWarps * 32, smem_sc, s>>>(
         reinterpret_cast<const short4*>(depth_rect), depth_order, n_cand, w.chunk, BW, BH,
         w.counts, block_vals, capacity, dev_status);
     GS_LAUNCH_CHECK();
