@@ -138,8 +138,8 @@ def step_roofline(a, model, stats, ops_fwd, ops_bwd, per_step, peaks, alu_peak, 
                    parameters; record, rect, depth key, candidate index)
       sort_depth   4 passes x C x 16 (keys + values in and out) + C*4
                    (histogram read) + C*20 (rect gather)
-      bin          C*8 (block counts) + C*12 (order + rects) + E_blk*8
-                   (keys + values) + 2 passes x E_blk x 20 (block sort)
+      bin          C*12 (rects + slots in depth order) + E_blk*4 (the block
+                   lists written once: they are built by a counting scatter)
       sort_tiles   2 passes x I x 20 (the bin + sort path only)
       expand       2 passes x R_blk x 12 (block entries + rect gathers) +
                    I*4 (the Leaf lists)
@@ -168,7 +168,7 @@ def step_roofline(a, model, stats, ops_fwd, ops_bwd, per_step, peaks, alu_peak, 
     byt = {
         "project": n * 12 + n * 4 + C * ((P - 3) * 4 + 64),
         "sort_depth": C * (4 * 16 + 4 + 20),
-        "bin": (C * 8 + C * 12 + E * 8 + E * 40) if expand else C * 12 * max(1, stats[0].n_leaves) + I * 8,
+        "bin": (C * 12 + E * 4) if expand else C * 12 * max(1, stats[0].n_leaves) + I * 8,
         "sort_tiles": 0.0 if expand else I * 40,
         "expand": (R * 24 + I * 4) if a.binning == "expand" else 0.0,
         "raster_fwd": C * 48 + px * 44,
