@@ -476,6 +476,289 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
 }
 
 // ---------------------------------------------------------------------------
+// forward, warp-specialised (the block-list path): one producer warp builds
+// the tile's list from its block list and stages the records; the NC
+// consumer warps composite them.  No CTA barrier separates the two roles:
+//
+// - producer: reads kWsU x 32 block-list entries per fill (kWsU loads in
+//   flight per lane), keeps the hits ("tile inside the candidate's rect"),
+//   in list order, in a circular queue s_q and in the Leaf's vals, and
+//   stages up to 32 queued records at a time into stage k % kWsS of a ring
+//   (the record's fields, its per-warp mask, the count and the list position
+//   of its first record), completing the stage's "full" mbarrier;
+// - consumers: each waits for stage k, walks the records whose mask bit is
+//   set for it, and arrives on the stage's "empty" mbarrier.  A warp whose
+//   pixels are all done counts itself in s_ndone once and from then on only
+//   releases stages; the producer stops filling once every consumer warp is
+//   done or the block list is exhausted and then publishes a terminal stage
+//   (count -1).
+//
+// Every wait is bounded: on expiry the waiter sets s_abort and
+// GS_DEV_TIMEOUT, and both roles leave.  The list prefix the producer
+// writes covers every position a consumer composited (positions < last).
+// ---------------------------------------------------------------------------
+constexpr int kWsS = 8;      // ring stages of 32 records
+constexpr int kWsQ = 512;    // hit queue (circular)
+constexpr int kWsU = 8;      // block-list entries per producer lane per fill
+
+// A shared flag read once for the whole warp (lane 0's value), so that the
+// warp takes the same branch.
+__device__ __forceinline__ int warp_flag(const int* f) {
+  return __shfl_sync(0xffffffffu, *(const volatile int*)f, 0);
+}
+
+// mbar_wait by every lane, true only if every lane saw the phase complete.
+__device__ __forceinline__ bool warp_mbar_wait(unsigned long long* bar, unsigned parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+template <int PPT, bool COUNT>
+__global__ void __launch_bounds__(TileGeom<PPT>::NT + 32, PPT == 2 ? 6 : 8)
+k_raster_fwd_ws(const float4* __restrict__ rec, gs_rect leaf, int W, int H, int TW, PixArgs px,
+                BlockSrc bsrc, int32_t* dev_status) {
+  using G = TileGeom<PPT>;
+  constexpr int NC = G::NW;
+  __shared__ float4 sA[kWsS][32], sB[kWsS][32];
+  __shared__ float sC[kWsS][32];
+  __shared__ uint8_t sM[kWsS][32];
+  __shared__ int sCnt[kWsS], sPos[kWsS];
+  __shared__ unsigned long long s_full[kWsS], s_empty[kWsS];
+  __shared__ int32_t s_q[kWsQ];
+  __shared__ int s_ndone, s_abort;
+  __shared__ float s_red[NC];
+  const int lw = leaf.x1 - leaf.x0;
+  const int ltile = blockIdx.x;
+  const int tx = leaf.x0 + ltile % lw, ty = leaf.y0 + ltile / lw;
+  const int64_t begin = bsrc.ranges_io[2 * ltile], end = bsrc.ranges_io[2 * ltile + 1];
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  if (t == 0) {
+    for (int st = 0; st < kWsS; ++st) {
+      mbar_init(&s_full[st], 32);
+      mbar_init(&s_empty[st], NC);
+    }
+    s_ndone = 0;
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (w == NC) {  // ---- producer warp ----
+    const int64_t b = (int64_t)(ty / GS_TILE_BLOCK) * bsrc.BW + tx / GS_TILE_BLOCK;
+    int64_t bp = bsrc.block_ranges[2 * b];
+    const int64_t be = bsrc.block_ranges[2 * b + 1];
+    const unsigned ltm = (1u << lane) - 1u;
+    unsigned qh = 0, qt = 0;  // staged / queued hits (list positions)
+    bool exhausted = bp >= be, bad = false, ok = true;
+    int k = 0;
+    for (;;) {
+      // every consumer warp done: stop (the hits queued so far are in vals)
+      if (warp_flag(&s_ndone) == NC) break;
+      while (!exhausted && qt - qh < 32u) {
+        int32_t sl[kWsU];
+        short4 rc[kWsU];
+#pragma unroll
+        for (int u = 0; u < kWsU; ++u) {
+          const int64_t q = bp + u * 32 + lane;
+          sl[u] = q < be ? bsrc.block_vals[q] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kWsU; ++u)
+          rc[u] = sl[u] >= 0 ? bsrc.rect[sl[u]] : make_short4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < kWsU; ++u) {
+          const bool hit = sl[u] >= 0 && (rc[u].x <= tx) & (tx < rc[u].z) & (rc[u].y <= ty) &
+                                             (ty < rc[u].w);
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
+          if (hit) {
+            const unsigned pos = qt + __popc(bal & ltm);
+            s_q[pos & (kWsQ - 1)] = sl[u];
+            const int64_t o = begin + pos;
+            if (o < end) bsrc.vals_out[o] = sl[u];
+            else bad = true;
+          }
+          qt += __popc(bal);
+        }
+        bp += kWsU * 32;
+        exhausted = bp >= be;
+      }
+      const int m = (int)min(32u, qt - qh);
+      if (m == 0) break;
+      const int st = k % kWsS;
+      if (k >= kWsS && !warp_mbar_wait(&s_empty[st], (unsigned)((k / kWsS - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      __syncwarp();  // the queue entries written by other lanes are visible
+      if (lane < m) {
+        const Staged g = stage_record(rec, s_q[(qh + lane) & (kWsQ - 1)], tx, ty);
+        sM[st][lane] = (uint8_t)warp_mask<PPT>(g);
+        sA[st][lane] = make_float4(g.gx, g.gy, g.beta, g.ns1);
+        sB[st][lane] = make_float4(g.ns2, g.lo2, g.r, g.g);
+        sC[st][lane] = g.b;
+      }
+      if (lane == 0) {
+        sCnt[st] = m;
+        sPos[st] = (int)qh;
+      }
+      qh += m;
+      mbar_arrive(&s_full[st]);
+      ++k;
+      if (warp_flag(&s_abort)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok) {  // terminal stage
+      const int st = k % kWsS;
+      if (k >= kWsS && !warp_mbar_wait(&s_empty[st], (unsigned)((k / kWsS - 1) & 1))) ok = false;
+      if (ok) {
+        if (lane == 0) sCnt[st] = -1;
+        mbar_arrive(&s_full[st]);
+      }
+    }
+    if (!ok) {
+      *(volatile int*)&s_abort = 1;
+      if (lane == 0) dev_flag(dev_status, GS_DEV_TIMEOUT);
+    }
+    if (bad) dev_flag(dev_status, GS_DEV_BOUNDS);
+    if (lane == 0)
+      bsrc.ranges_io[2 * ltile + 1] = begin + ((int64_t)qt < end - begin ? (int64_t)qt : end - begin);
+    return;
+  }
+
+  // ---- consumer warps ----
+  const WarpPix wp = warp_pixels<PPT>(t);
+  const float fpx = (float)wp.lx + 0.5f;
+  float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
+  int lastp[PPT];
+  int stopn[PPT];  // COUNT: 1-based list position of the stopping entry, 0 = none
+  bool done[PPT], inside[PPT];
+  unsigned n_vis = 0, n_kept = 0;
+#pragma unroll
+  for (int k = 0; k < PPT; ++k) {
+    const int ly = wp.ly0 + k * G::LROWS;
+    fpy[k] = (float)ly + 0.5f;
+    inside[k] = (tx * kTile + wp.lx < W) && (ty * kTile + ly < H);
+    done[k] = !inside[k];
+    T[k] = 1.0f;
+    Cr[k] = Cg[k] = Cb[k] = 0.0f;
+    lastp[k] = 0;
+    stopn[k] = 0;
+  }
+  bool counted = false;
+  for (int ks = 0;; ++ks) {
+    const int st = ks % kWsS;
+    if (!warp_mbar_wait(&s_full[st], (unsigned)((ks / kWsS) & 1))) {
+      *(volatile int*)&s_abort = 1;
+      if (lane == 0) dev_flag(dev_status, GS_DEV_TIMEOUT);
+      break;
+    }
+    const int cnt = sCnt[st];
+    if (cnt < 0 || warp_flag(&s_abort)) break;
+    bool d_all = true;
+#pragma unroll
+    for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
+    if (!__all_sync(0xffffffffu, d_all)) {
+      const int pos1 = sPos[st] + 1;
+      unsigned bits = __ballot_sync(0xffffffffu, lane < cnt && ((sM[st][lane] >> w) & 1u));
+      while (bits) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        const float4 A = sA[st][j];
+        const float4 B = sB[st][j];
+        const float Bb = sC[st][j];
+        const int posn = pos1 + j;
+        const float dx = __fsub_rn(A.x, fpx);
+#pragma unroll
+        for (int k = 0; k < PPT; ++k) {
+          const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
+          if (COUNT) n_vis += done[k] ? 0u : 1u;
+          const bool use = !done[k] && ev.alpha >= kAlphaMin;
+          const float Tn = __fmaf_rn(-ev.alpha, T[k], T[k]);  // T (1 - alpha), one rounding
+          const bool stop = use && Tn < kTMin;
+          const bool comp = use && !stop;
+          if (COUNT) {
+            stopn[k] = stop ? posn : stopn[k];
+            n_kept += comp ? 1u : 0u;
+          }
+          done[k] = done[k] || stop;
+          const float wgt = comp ? ev.alpha * T[k] : 0.0f;
+          Cr[k] = fmaf(B.z, wgt, Cr[k]);
+          Cg[k] = fmaf(B.w, wgt, Cg[k]);
+          Cb[k] = fmaf(Bb, wgt, Cb[k]);
+          T[k] = comp ? Tn : T[k];
+          lastp[k] = comp ? posn : lastp[k];
+        }
+      }
+      d_all = true;
+#pragma unroll
+      for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
+      d_all = __all_sync(0xffffffffu, d_all);
+    }
+    if (d_all && !counted) {
+      counted = true;
+      if (lane == 0) atomicAdd(&s_ndone, 1);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s_empty[st]);
+  }
+  if (COUNT) {  // one atomic per warp: per-thread ones on one word serialise
+    unsigned long long e_f = 0, e_b = 0;
+#pragma unroll
+    for (int k = 0; k < PPT; ++k)
+      if (inside[k]) {
+        e_f += stopn[k] ? (unsigned long long)stopn[k] : (unsigned long long)(end - begin);
+        e_b += (unsigned long long)lastp[k];
+      }
+    const unsigned long long a = warp_sum((unsigned long long)n_vis);
+    const unsigned long long bq = warp_sum((unsigned long long)n_kept);
+    const unsigned long long c = warp_sum(e_f);
+    const unsigned long long d = warp_sum(e_b);
+    if (lane == 0) {
+      atomicAdd(&px.counters[0], a);
+      atomicAdd(&px.counters[1], bq);
+      atomicAdd(&px.counters[2], c);
+      atomicAdd(&px.counters[3], d);
+    }
+  }
+  // epilogue: outputs and the fused L1 terms
+  float lsum = 0.0f;
+#pragma unroll
+  for (int k = 0; k < PPT; ++k) {
+    if (!inside[k]) continue;
+    const int x = tx * kTile + wp.lx, y = ty * kTile + wp.ly0 + k * G::LROWS;
+    const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
+    if (px.img) {
+      px.img[o] = Cr[k];
+      px.img[o + px.plane] = Cg[k];
+      px.img[o + 2 * px.plane] = Cb[k];
+    }
+    px.T_final[o] = T[k];
+    px.last[o] = lastp[k];
+    if (px.target) {
+      const float c[3] = {Cr[k], Cg[k], Cb[k]};
+      const int64_t ot = (int64_t)(y - px.ty0) * px.tpitch + (x - px.tx0);
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) {
+        const float d = c[ch] - px.target[ot + ch * px.tplane];
+        px.dL[o + ch * px.plane] = d > 0.0f ? px.norm : (d < 0.0f ? -px.norm : 0.0f);
+        lsum += fabsf(d);
+      }
+    }
+  }
+  if (px.target && px.loss_tiles) {
+    lsum = warp_sum(lsum);
+    if (lane == 0) s_red[w] = lsum;
+    asm volatile("bar.sync 1, %0;" ::"r"(NC * 32) : "memory");  // the consumer warps only
+    if (t == 0) {
+      float tot = 0.0f;
+      for (int ww = 0; ww < NC; ++ww) tot += s_red[ww];
+      px.loss_tiles[(int64_t)ty * TW + tx] = tot * px.norm;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // standalone L1 over a Leaf
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
@@ -822,6 +1105,18 @@ extern "C" gs_status gs_raster_fwd_blocks(const gs_proj* proj, const int32_t* bl
   const bool cnt = px->counters != nullptr;
   const BlockSrc src{reinterpret_cast<const short4*>(proj->rect), block_vals, block_ranges,
                      (TW + GS_TILE_BLOCK - 1) / GS_TILE_BLOCK, vals, ranges};
+  if (flags & GS_RASTER_WS) {
+    // warp-specialised: a producer warp fills and stages, NC warps composite
+#define GS_FWD(P, C) \
+  k_raster_fwd_ws<P, C><<<nb, 256 / P + 32, 0, s>>>(rec, leaf, W, H, TW, a, src, dev_status)
+    switch (pick_ppt(flags, 2)) {
+      case 4: if (cnt) GS_FWD(4, true); else GS_FWD(4, false); break;
+      default: if (cnt) GS_FWD(2, true); else GS_FWD(2, false); break;
+    }
+#undef GS_FWD
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+  }
 #define GS_FWD(P, C) \
   k_raster_fwd<P, C, true><<<nb, 256 / P, 0, s>>>(rec, vals, ranges, leaf, W, H, TW, a, src, dev_status)
   switch (pick_ppt(flags, 2)) {

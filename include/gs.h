@@ -429,8 +429,10 @@ gs_status gs_expand_tiles(const gs_proj* proj, const int32_t* block_vals,
  * T_final, last; if px->target is set, also the L1 loss terms (as
  * gs_loss_l1).  fp32 arithmetic.
  * flags & 7 selects the pixels per thread (1, 2 or 4; 0 = the default, 2
- * here and 4 in gs_raster_bwd, the faster shapes on B200); the result does
- * not depend on it.  The same flag applies to gs_raster_bwd. */
+ * here and 4 in gs_raster_bwd, the faster shapes on B200); img, T_final,
+ * last and dL_dimg do not depend on it, the fp32 summation order of a
+ * tile's loss partial (over the tile's warps) does.  The same flag applies
+ * to gs_raster_bwd. */
 gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals,
                         const int64_t* ranges, gs_rect leaf,
                         const gs_camera* cam, const gs_pixels* px,
@@ -449,7 +451,16 @@ gs_status gs_raster_fwd(const gs_proj* proj, const int32_t* vals,
  * number of list entries consumed, and vals[begin .. end) = that prefix of
  * the tile's list (everything gs_raster_bwd reads: positions < last).
  * Image, T_final, last and loss are identical to gs_raster_fwd on the full
- * lists.  n_isect: the Leaf's count (host SAT), must be <= capacity. */
+ * lists.  n_isect: the Leaf's count (host SAT), must be <= capacity.
+ * By default all threads of a tile build its list, stage the records and
+ * composite them in turn, meeting at CTA barriers; flags & GS_RASTER_WS
+ * selects a warp-specialised form in which one warp per tile builds the list
+ * and stages the records through an mbarrier ring while the others
+ * composite (pixels per thread 2, or 4 with flags & 7 == 4).  Both give
+ * identical results; on B200 the default is faster (the forward is bound by
+ * its instruction issue, and the producer warp lowers the resident
+ * compositing warps). */
+#define GS_RASTER_WS 0x20u
 gs_status gs_tile_ranges(const int64_t* tile_sat, int32_t TW, int32_t TH,
                          gs_rect leaf, int64_t* ranges, gs_stream stream);
 gs_status gs_raster_fwd_blocks(const gs_proj* proj, const int32_t* block_vals,

@@ -189,10 +189,14 @@ def test_two_level_binning_leaf_without_entries(oracle_mod):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "hd"])
-def test_fused_forward_matches_oracle(oracle_mod, name):
+@pytest.mark.parametrize("flags", [0, 4, 0x20, 0x20 | 4])
+def test_fused_forward_matches_oracle(oracle_mod, name, flags):
     """gs_raster_fwd_blocks: image, T, last and loss as the oracle's
     compositing of the full lists; vals holds an exact prefix of each tile's
-    list that covers every position the backward reads (< last)."""
+    list that covers every position the backward reads (< last).  Both forms:
+    all threads filling, staging and compositing in turn (default), and a
+    producer warp filling and staging for the compositing warps (0x20); 2 or
+    4 pixels per thread."""
     sc, cams = {"tiny": synth.tiny_oracle_scene, "hd": synth.hd_cluster_scene}.get(
         name, lambda s: synth.tiny_scene(n=80, width=83, height=61, sh_degree=3, seed=4))(0)
     cam = cams[0]
@@ -227,7 +231,7 @@ def test_fused_forward_matches_oracle(oracle_mod, name):
         ranges = torch.zeros(2 * len(tiles), dtype=torch.int64, device="cuda")
         b.gs_tile_ranges(case.sat_d, TW, TH, L, ranges)
         b.gs_raster_fwd_blocks(case.pb.struct, case.bvals, case.branges, L, b.camera_struct(cam),
-                               px, vals, max(I, 1), I, ranges, case.st)
+                               px, vals, max(I, 1), I, ranges, case.st, flags=flags)
         assert b.gs_check(case.st) == 0
         # the same outputs as the full-list forward on the oracle's lists
         ref_img = torch.zeros_like(img)
@@ -240,7 +244,10 @@ def test_fused_forward_matches_oracle(oracle_mod, name):
                        loss_tiles=ref_lt, norm=1.0 / (3.0 * W * H))
         vals_full = torch.as_tensor(vals_o if I else np.zeros(1, np.int32)).cuda()
         rg_full = torch.as_tensor(np.stack([off[:-1], off[1:]], 1).astype(np.int64).reshape(-1)).cuda()
-        b.gs_raster_fwd(case.pb.struct, vals_full, rg_full, L, b.camera_struct(cam), pxr, case.st)
+        # the same pixels per thread: the per-tile loss partial's fp32 sum
+        # runs over the tile's warps in order
+        b.gs_raster_fwd(case.pb.struct, vals_full, rg_full, L, b.camera_struct(cam), pxr, case.st,
+                        flags & 7)
         assert b.gs_check(case.st) == 0
         assert torch.equal(img, ref_img) and torch.equal(Tf, ref_T) and torch.equal(last, ref_last)
         assert torch.equal(dL, ref_dL) and torch.equal(loss_tiles, ref_lt)
