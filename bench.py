@@ -204,10 +204,14 @@ def alu_roofline(kernel, lane_ops, stage_ms, alu_peak):
             "frac": round(ach / (alu_peak / 1e12), 4), "lane_ops_per_step": round(lane_ops)}
 
 
-def profile_traffic(kernel):
+def profile_traffic(kernel, alg_bytes_per_launch=None):
     """DRAM bytes per launch of `kernel` from the committed ncu summary
     (profiles/<kernel>_*_dram.json), or None when there is none or the
-    kernel's source file has changed since it was taken."""
+    kernel's source file has changed since it was taken.  A summary taken on
+    a smaller case records that case's algorithmic bytes per launch; its
+    traffic is then scaled to this workload's launch by the ratio of the
+    algorithmic bytes (the kernel's DRAM traffic is its compulsory bytes
+    times a waste factor that does not depend on the size)."""
     import glob
     import hashlib
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*_dram.json"))):
@@ -219,9 +223,23 @@ def profile_traffic(kernel):
                 digest = hashlib.sha256(f.read()).hexdigest()
         except (OSError, KeyError, ValueError):
             continue
-        if digest == rec.get("source_sha256"):
-            return rec["dram_bytes_per_launch"], os.path.relpath(path, ROOT)
+        if digest != rec.get("source_sha256"):
+            continue
+        t = rec["dram_bytes_per_launch"]
+        base = rec.get("alg_bytes_per_launch")
+        if base and alg_bytes_per_launch:
+            return round(t * alg_bytes_per_launch / base), (
+                f"{os.path.relpath(path, ROOT)}, scaled by algorithmic bytes per launch "
+                f"{alg_bytes_per_launch:.4g} / {base:.4g}")
+        return t, os.path.relpath(path, ROOT)
     return None, None
+
+
+def raster_bwd_alg_bytes(n_cand, pixels):
+    """Compulsory DRAM bytes of the raster backward over a region: each
+    record fetched once (48 B), the gradient reductions (48 B per candidate),
+    and T, last and dL/dcolour per pixel (20 B); as in step_roofline."""
+    return n_cand * 96 + pixels * 20
 
 
 def load_peaks():
@@ -565,7 +583,10 @@ def main():
     per_step = {s: stage_ms[s] / n_steps for s in STAGES}
     if dom in ("raster_bwd", "raster_fwd"):
         ops = ops_bwd if dom == "raster_bwd" else ops_fwd
-        traffic, traffic_src = profile_traffic(f"k_{dom}")
+        # per launch (one Leaf): the view's compulsory bytes over its Leaves
+        leaves = statistics.mean(st.n_leaves for st in stats)
+        alg = raster_bwd_alg_bytes(statistics.mean(st.n_cand for st in stats), W * H) / leaves
+        traffic, traffic_src = profile_traffic(f"k_{dom}", alg if dom == "raster_bwd" else None)
         roof = alu_roofline(f"k_{dom}", ops, per_step[dom], alu_peak)
         roof.update(traffic=traffic, traffic_source=traffic_src,
                     peak_source=f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {sm_mhz:g} MHz "
@@ -778,6 +799,8 @@ def run_schedules(a):
              ("groups3x3_128MiB", dict(budget=128 << 20), (3, 3)),
              ("blocks8x8", dict(budget=1 << 40), (8, 8))]
     for name, kw, split in plans:
+        clocks = ClockSampler(0)
+        wall0 = time.time()
         model = GaussianModel(scene.params, scene.n, scene.sh_degree)
         stp = Stepper(model, **kw)
         jm = GaussianModel(jit.params, jit.n, jit.sh_degree)
@@ -803,11 +826,12 @@ def run_schedules(a):
             peak = max(peak, st.peak_ws_bytes)
             leaves += st.n_leaves
             del target
+        clk = clocks.stop(wall0, time.time())
         print(json.dumps({"schedule": name, "views": len(cams), "ms_per_view": total_ms / len(cams),
                           "pass_s": total_ms / 1e3, "working_set_gib": peak / 2 ** 30,
                           "mean_loss": float(np.mean(losses)),
                           "adam_updates": model.step - updates0,
-                          "leaves_per_view": leaves / len(cams),
+                          "leaves_per_view": leaves / len(cams), "clocks": clk,
                           "workload": workload_name(a)}), flush=True)
         del stp, model, renderer, jm
         torch.cuda.empty_cache()
