@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--raster-ppt", type=int, default=0)
     # 2: consecutive Leaves alternate between two streams and two raster
     # arenas (one Leaf's kernels fill the SMs the other's tail leaves idle)
-    ap.add_argument("--leaf-streams", type=int, default=2, choices=[1, 2])
+    ap.add_argument("--leaf-streams", type=int, default=2, choices=[1, 2, 3, 4])
     # steps of the serialized pass (Leaves on one stream) whose per-stage
     # CUDA-event times give the kernels' own durations when the timed region
     # overlaps Leaves
@@ -543,8 +543,8 @@ def main():
     stage_src = "timed region"
     stage_views = [view_of(a.warmup + k) for k in range(a.steps)]
     overlapped = None
-    if a.leaf_streams == 2:
-        # two Leaves in flight: a stage's events span the other stream's
+    if a.leaf_streams > 1:
+        # several Leaves in flight: a stage's events span the other streams'
         # kernels too, so the kernels' own durations come from a serialized
         # pass of the same workload (same views, Leaves on one stream)
         overlapped = {s: round(stage_ms[s] / a.steps, 3) for s in STAGES}
@@ -554,7 +554,7 @@ def main():
             v = view_of(a.warmup + k)
             stp.run_view(cams[v], targets[v], timing=timing)
         torch.cuda.synchronize()
-        stp.leaf_streams = 2
+        stp.leaf_streams = a.leaf_streams
         stage_ms = {name: sum(x.elapsed_time(y) for x, y in timing.get(name, []))
                     for name in STAGES}
         stage_n = {name: len(timing.get(name, [])) for name in STAGES}

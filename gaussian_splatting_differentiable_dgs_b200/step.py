@@ -133,7 +133,7 @@ class Stepper:
     gradients and a separate Adam), binning ("fused", "expand", "sort": the
     three list builders), mode ("bounded" or the whole-image "original"),
     loss ("l1" or "l1_ssim" with weight ssim_lambda), leaf_streams (1: one
-    Leaf at a time; 2: consecutive Leaves on two streams with two raster
+    Leaf at a time; k = 2..4: consecutive Leaves on k streams with k raster
     arenas)."""
 
     def __init__(self, model: GaussianModel, budget: int = DEFAULT_BUDGET, lr=1e-3,
@@ -151,12 +151,12 @@ class Stepper:
         # alive through the projection backward, dense gradients)
         if loss not in ("l1", "l1_ssim"):
             raise ValueError(f"loss must be 'l1' or 'l1_ssim', not {loss!r}")
-        # leaf_streams = 2: consecutive Leaves alternate between two streams
-        # and two raster arenas, so one Leaf's kernels fill the SMs that the
-        # other's last CTAs leave idle (two Leaves' raster buffers in flight,
+        # leaf_streams = k > 1: consecutive Leaves rotate over k streams and
+        # k raster arenas, so one Leaf's kernels fill the SMs that another's
+        # last CTAs leave idle (k Leaves' raster buffers in flight,
         # each within the budget)
-        if leaf_streams not in (1, 2):
-            raise ValueError(f"leaf_streams must be 1 or 2, not {leaf_streams!r}")
+        if leaf_streams not in (1, 2, 3, 4):
+            raise ValueError(f"leaf_streams must be 1 to 4, not {leaf_streams!r}")
         # l1: the L1 photometric loss; l1_ssim: the composite
         # (1 - lambda) L1 + lambda (1 - SSIM) of 3DGS training (SkipGS notes,
         # "loss function / training strategy"), SSIM windows local to each Leaf
@@ -174,7 +174,7 @@ class Stepper:
         self._last_loss = None
         self._copy_stream = None
         self.leaf_streams = leaf_streams
-        self._leaf_stream = None
+        self._side_streams = []
         self._cap_hint = {}  # region -> candidate capacity for the next view
 
     def check(self):
@@ -379,16 +379,16 @@ class Stepper:
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
         arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
-        two = self.leaf_streams == 2 and len(lv) > 1 and not original
+        n_ls = 1 if original else max(1, min(self.leaf_streams, len(lv)))
         main = torch.cuda.current_stream(dev)
         arenas, lstreams = [arena], [main]
         bin_wss = [bin_ws]
-        if two:
+        while len(self._side_streams) < n_ls - 1:
+            self._side_streams.append(torch.cuda.Stream(device=dev))
+        for k in range(n_ls - 1):
             arenas.append(torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev))
             bin_wss.append(torch.empty_like(bin_ws))  # the list builders' scratch, per stream
-            if self._leaf_stream is None:
-                self._leaf_stream = torch.cuda.Stream(device=dev)
-            lstreams.append(self._leaf_stream)
+            lstreams.append(self._side_streams[k])
         norm = 1.0 / (3.0 * W * H)
         # with the SSIM term the forward's L1 part carries (1 - lambda)
         norm_l1 = (1.0 - self.ssim_lambda) * norm if ssim else norm
@@ -408,8 +408,8 @@ class Stepper:
 
         def leaf_pass(with_bwd):
             """Every Leaf: lists, forward (+ L1) and, if with_bwd, backward."""
-            if two:
-                lstreams[1].wait_stream(main)  # g2d, lists and tables are ready
+            for side in lstreams[1:]:
+                side.wait_stream(main)  # g2d, lists and tables are ready
             if host_target:
                 up = [torch.cuda.Event() for _ in lv]
                 freed = [None, None]
@@ -429,8 +429,8 @@ class Stepper:
             for li_k, (L, I) in enumerate(zip(lv, li)):
                 with torch.cuda.stream(lstreams[li_k % len(lstreams)]):
                     leaf_one(li_k, L, I, with_bwd)
-            if two:
-                main.wait_stream(lstreams[1])
+            for side in lstreams[1:]:
+                main.wait_stream(side)
 
         def leaf_one(li_k, L, I, with_bwd):
             """One Leaf on the current stream, with its arena."""

@@ -127,7 +127,7 @@ def test_stepper_rejects_unknown_options():
     from gaussian_splatting_differentiable_dgs_b200.step import GaussianModel, Stepper
     sc, _ = synth.tiny_scene(n=4)
     model = GaussianModel(np.asarray(sc.params), sc.n, sc.sh_degree, device="cpu")
-    for kw in ({"leaf_streams": 3}, {"leaf_streams": 0}, {"binning": "tiles"},
+    for kw in ({"leaf_streams": 5}, {"leaf_streams": 0}, {"binning": "tiles"},
                {"mode": "whole"}, {"loss": "l2"}):
         with pytest.raises(ValueError):
             Stepper(model, device="cpu", **kw)
