@@ -175,6 +175,7 @@ class Stepper:
         self._copy_stream = None
         self.leaf_streams = leaf_streams
         self._side_streams = []
+        self._fill_stream = None
         self._cap_hint = {}  # region -> candidate capacity for the next view
 
     def check(self):
@@ -289,6 +290,18 @@ class Stepper:
         if hooks is not None and hasattr(hooks, "on_project"):
             hooks.on_project(ctx)
 
+        # the compact 2D gradient, zeroed on a side stream so that the fill
+        # runs beside the depth sort and binning (the raster backward, its
+        # first user, waits for it)
+        g2d = torch.empty(max(C, 1) * 12, dtype=torch.float32, device=dev)
+        if self._fill_stream is None:
+            self._fill_stream = torch.cuda.Stream(device=dev)
+        self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(self._fill_stream):
+            g2d.zero_()
+        g2d_ready = torch.cuda.Event()
+        g2d_ready.record(self._fill_stream)
+
         # ---- depth presort (+ rects gathered in depth order) ------------------
         order = torch.empty(max(C, 1), dtype=torch.int32, device=dev)
         drect = torch.empty(max(C, 1) * 4, dtype=torch.int16, device=dev)
@@ -343,7 +356,6 @@ class Stepper:
             ov = np.zeros(len(lv), bool)
 
         # ---- per-Leaf raster: forward + L1 + backward into compact g2d ------
-        g2d = torch.zeros(max(C, 1) * 12, dtype=torch.float32, device=dev)
         # every tile's loss partial is written by its Leaf's forward when the
         # planned Leaves cover the grid; a region or caller-given Leaves may
         # leave tiles out, which must then count zero
@@ -405,6 +417,8 @@ class Stepper:
             cs = self._copy_stream
 
         hstate = {}  # the host target's upload state, shared by leaf_pass and leaf_one
+
+        main.wait_event(g2d_ready)
 
         def leaf_pass(with_bwd):
             """Every Leaf: lists, forward (+ L1) and, if with_bwd, backward."""
