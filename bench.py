@@ -85,6 +85,8 @@ def parse():
     ap.add_argument("--schedules", action="store_true",
                     help="schedule comparison: Leaves, 3x3 groups at 128 MiB, fixed 8x8 blocks")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-mode", default="prefetch", choices=["prefetch", "crops"],
+                    help="how the e2e run supplies the targets from pinned host memory")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
     return ap.parse_args()
@@ -607,9 +609,13 @@ def main():
     # ---- end to end through host buffers --------------------------------------
     e2e = None
     if not a.no_e2e:
-        # the step's public call with the view's target in pinned host memory:
-        # each Leaf's crop is uploaded on a copy stream, overlapped with compute
+        # the step's public calls with the views' targets in pinned host
+        # memory: "prefetch" uploads each view's target during the previous
+        # view's step (TargetPrefetcher); "crops" uploads each Leaf's crop on
+        # a copy stream during the view's own Leaves (two crops resident)
+        from gaussian_splatting_differentiable_dgs_b200.step import TargetPrefetcher
         host_t = [t.cpu().pin_memory() for t in targets]
+        feeder = TargetPrefetcher(host_t) if a.e2e_mode == "prefetch" else None
         loss_h = torch.empty(1, dtype=torch.float64, pin_memory=True)
         if dist:
             dist.barrier()
@@ -618,9 +624,10 @@ def main():
         f1 = torch.cuda.Event(enable_timing=True)
         f0.record()
         e2e_isect = 0
-        for k in range(a.steps):
-            v = view_of(k)
-            s = stp.run_view(cams[v], host_t[v])
+        order = [view_of(k) for k in range(a.steps)]
+        supply = feeder.iterate(order) if feeder else ((v, host_t[v]) for v in order)
+        for v, tgt in supply:
+            s = stp.run_view(cams[v], tgt)
             loss_h.copy_(stp._last_loss, non_blocking=True)
             e2e_isect += s.n_isect_square
         f1.record()
@@ -634,7 +641,11 @@ def main():
         if a.binning in ("expand", "fused"):
             d2h += (BW + 1) * (BH + 1) * 8
         e2e = {"value": e2e_isect / (ems / 1e3), "unit": UNIT, "ms_per_step": ems / a.steps,
-               "h2d_bytes_per_step": 3 * W * H * 4, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": 3 * W * H * 4, "d2h_bytes_per_step": d2h,
+               "supply": ("prefetch: each view's target uploaded during the previous view's "
+                          "step, two device targets resident") if feeder else
+                         ("crops: each Leaf's crop uploaded during the view's Leaves, "
+                          "two crops resident")}
 
     # ---- CPU baseline (rank 0, one GPU) ---------------------------------------
     cpu = None

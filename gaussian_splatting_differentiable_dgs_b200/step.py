@@ -102,6 +102,59 @@ class GaussianModel:
         return B.gs_model(self.n, self.n_pad, self.sh_degree, 0, self.params.data_ptr())
 
 
+class TargetPrefetcher:
+    """Supplies views' targets to the device one view ahead.  While the step
+    of view k runs, the target of the next view in the order is copied from
+    pinned host memory on a copy stream into the other of two device buffers,
+    so its upload overlaps the step instead of the Leaves' compute.  Holds
+    two device targets (2 x 3 x H x W fp32); the per-Leaf crop supply of
+    `Stepper.run_view` with a host target holds two Leaf crops instead.
+
+        for v, target in TargetPrefetcher(host_targets).iterate(order):
+            stepper.run_view(cams[v], target)
+    """
+
+    def __init__(self, host_targets, device="cuda"):
+        self.host = host_targets          # indexable: view -> pinned [3][H][W] fp32
+        self.device = torch.device(device)
+        self.stream = torch.cuda.Stream(device=self.device)
+        self._bufs = None
+
+    def iterate(self, order):
+        order = list(order)
+        if not order:
+            return
+        shape = tuple(self.host[order[0]].shape)
+        if self._bufs is None or tuple(self._bufs[0].shape) != shape:
+            self._bufs = [torch.empty(shape, dtype=torch.float32, device=self.device)
+                          for _ in range(2)]
+        main = torch.cuda.current_stream(self.device)
+        ready, free = [None, None], [None, None]
+
+        def upload(slot, v):
+            # the buffer's previous reader (two steps back) must be done with it
+            if free[slot] is not None:
+                self.stream.wait_event(free[slot])
+            else:
+                self.stream.wait_stream(main)
+            with torch.cuda.stream(self.stream):
+                self._bufs[slot].copy_(self.host[v], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(self.stream)
+            ready[slot] = ev
+
+        upload(0, order[0])
+        for i, v in enumerate(order):
+            slot = i & 1
+            if i + 1 < len(order):
+                upload(1 - slot, order[i + 1])
+            main.wait_event(ready[slot])
+            yield v, self._bufs[slot]
+            ev = torch.cuda.Event()
+            ev.record(main)   # after the step's work on this buffer
+            free[slot] = ev
+
+
 class _Timer:
     def __init__(self, timing):
         self.timing = timing
