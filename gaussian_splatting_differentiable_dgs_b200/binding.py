@@ -24,6 +24,7 @@ GS_ERR_UNSUPPORTED = -6
 GS_SORT_IOTA = 1
 GS_SORT_ONESWEEP = 2
 GS_RASTER_WS = 0x20
+GS_COUNT_ON_DEVICE = -1
 GS_SORT_TEST_STALL = 0x80000000
 TILE = 16
 

@@ -27,7 +27,8 @@ constexpr int kBinChunk = kBinThreads * kBinItems; // candidates per block
 
 __global__ void __launch_bounds__(256)
 k_gather_rects(const short4* __restrict__ rect, const int32_t* __restrict__ order, int64_t n,
-               short4* __restrict__ out) {
+               short4* __restrict__ out, const int32_t* __restrict__ n_dev) {
+  if (n_dev) n = min(n, (int64_t)*n_dev);
   const int64_t j = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (j < n) out[j] = rect[order[j]];
 }
@@ -797,18 +798,25 @@ extern "C" size_t gs_depth_order_workspace_size(int64_t n_cand) {
 extern "C" gs_status gs_depth_order(const gs_proj* proj, int64_t n_cand, int32_t* depth_order,
                                     int16_t* depth_rect, void* ws, size_t ws_bytes,
                                     int32_t* dev_status, gs_stream stream) {
-  if (!proj || n_cand < 0 || n_cand > proj->capacity) return GS_ERR_ARG;
-  if (n_cand == 0) return GS_OK;
+  if (!proj || n_cand < GS_COUNT_ON_DEVICE || n_cand > proj->capacity) return GS_ERR_ARG;
+  // the count on the device (proj->n_cand, at most the capacity): the call
+  // can be issued before the host has read the projection's count
+  const bool dev = n_cand == GS_COUNT_ON_DEVICE;
+  const int64_t n = dev ? proj->capacity : n_cand;
+  if (dev && !proj->n_cand) return GS_ERR_ARG;
+  if (n == 0) return GS_OK;
   if (!depth_order || !depth_rect || !proj->depth_key || !proj->rect) return GS_ERR_ARG;
   if (!aligned(depth_rect, 8) || !aligned(ws, 256)) return GS_ERR_ARG;
-  OrderWs w = carve_order(ws, ws_bytes, n_cand);
+  OrderWs w = carve_order(ws, ws_bytes, n);
   if (!ws || w.bytes > ws_bytes) return GS_ERR_CAPACITY;
-  const gs_status st = gs_sort_keys32(proj->depth_key, w.keys, depth_order, n_cand, 0, 32,
-                                      GS_SORT_IOTA, w.sort_ws, w.sort_bytes, dev_status, stream);
+  const int32_t* n_dev = dev ? proj->n_cand : nullptr;
+  const gs_status st = sort32_iota_devcount(proj->depth_key, w.keys, depth_order, n, n_dev,
+                                            w.sort_ws, w.sort_bytes, dev_status,
+                                            to_stream(stream));
   if (st != GS_OK) return st;
-  k_gather_rects<<<(unsigned)((n_cand + 255) / 256), 256, 0, to_stream(stream)>>>(
-      reinterpret_cast<const short4*>(proj->rect), depth_order, n_cand,
-      reinterpret_cast<short4*>(depth_rect));
+  k_gather_rects<<<(unsigned)((n + 255) / 256), 256, 0, to_stream(stream)>>>(
+      reinterpret_cast<const short4*>(proj->rect), depth_order, n,
+      reinterpret_cast<short4*>(depth_rect), n_dev);
   GS_LAUNCH_CHECK();
   return GS_OK;
 }

@@ -288,4 +288,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 32-bit key sort with values 0..count-1, the count read on the device (at
+// most n) (gs_sort.cu; library-internal).
+gs_status sort32_iota_devcount(const uint32_t* keys_in, uint32_t* keys, int32_t* vals, int64_t n,
+                               const int32_t* n_dev, void* ws, size_t ws_bytes,
+                               int32_t* dev_status, cudaStream_t s);
+
 }  // namespace gs

@@ -68,7 +68,9 @@ __device__ __forceinline__ unsigned digit_of(K key, int shift, unsigned mask) {
 
 template <class K>
 __global__ void __launch_bounds__(kSortThreads)
-k_hist(const K* __restrict__ keys, int64_t n, SortPlan plan, unsigned long long* __restrict__ hist) {
+k_hist(const K* __restrict__ keys, int64_t n, SortPlan plan, unsigned long long* __restrict__ hist,
+       const int32_t* __restrict__ n_dev) {
+  if (n_dev) n = min(n, (int64_t)*n_dev);  // the count on the device, at most n
   __shared__ unsigned int sh[8][kRadix];
   for (int e = threadIdx.x; e < 8 * kRadix; e += kSortThreads) (&sh[0][0])[e] = 0;
   __syncthreads();
@@ -285,7 +287,8 @@ k_onesweep(const K* __restrict__ src_k, const int32_t* __restrict__ src_v, bool 
 template <class K>
 __global__ void __launch_bounds__(kSortThreads)
 k_upsweep(const K* __restrict__ keys, int64_t n, int shift, int bits, int64_t tiles,
-          unsigned int* __restrict__ counts) {
+          unsigned int* __restrict__ counts, const int32_t* __restrict__ n_dev) {
+  if (n_dev) n = min(n, (int64_t)*n_dev);  // tiles past the count write zero counts
   __shared__ unsigned int sh[kRadix];
   const unsigned mask = (1u << bits) - 1u;
   for (int d = threadIdx.x; d < kRadix; d += kSortThreads) sh[d] = 0;
@@ -430,7 +433,9 @@ struct DownSmem32 {
 __global__ void __launch_bounds__(kSortThreads, GS_SORT_MINB)
 k_downsweep32(const uint32_t* __restrict__ src_k, const int32_t* __restrict__ src_v, bool iota,
               uint32_t* __restrict__ dst_k, int32_t* __restrict__ dst_v, int n, int shift,
-              int bits, const unsigned int* __restrict__ offsets, int tiles, int32_t* dev_status) {
+              int bits, const unsigned int* __restrict__ offsets, int tiles, int32_t* dev_status,
+              const int32_t* __restrict__ n_dev) {
+  if (n_dev) n = min(n, *n_dev);  // tiles past the count write nothing
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DownSmem32& S = *reinterpret_cast<DownSmem32*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -566,8 +571,11 @@ template <class K>
 gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool stall, int64_t n,
                     int begin_bit, int end_bit, void* ws, size_t ws_bytes, int32_t* dev_status,
                     cudaStream_t s, const int64_t* ranges = nullptr, int64_t n_tiles = 0,
-                    bool chained = false) {
+                    bool chained = false, const int32_t* n_dev = nullptr) {
+  // n_dev: the number of pairs is read on the device (at most n); only the
+  // lean 32-bit passes take it
   chained = chained || stall;
+  if (n_dev && (chained || sizeof(K) != 4 || ranges)) return GS_ERR_UNSUPPORTED;
   const int kbits = (int)(8 * sizeof(K));
   if (n < 0 || begin_bit < 0 || end_bit > kbits || begin_bit > end_bit) return GS_ERR_ARG;
   if (n == 0) return GS_OK;
@@ -592,7 +600,7 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
         ranges, n_tiles, plan, w.hist);
   } else {
     const int hist_blocks = (int)(tiles < 1184 ? tiles : 1184);
-    k_hist<K><<<hist_blocks, kSortThreads, 0, s>>>(first_k, n, plan, w.hist);
+    k_hist<K><<<hist_blocks, kSortThreads, 0, s>>>(first_k, n, plan, w.hist, n_dev);
   }
   GS_LAUNCH_CHECK();
   k_hist_scan<<<plan.passes, kRadix, 0, s>>>(w.hist, w.hstart);
@@ -628,14 +636,14 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
       continue;
     }
     k_upsweep<K><<<(unsigned)tiles, kSortThreads, 0, s>>>(sk, n, plan.shift[p], plan.bits[p], tiles,
-                                                            w.counts);
+                                                            w.counts, n_dev);
     GS_LAUNCH_CHECK();
     k_scan_tiles<<<kRadix, 1024, 0, s>>>(w.counts, tiles, w.hstart + (size_t)p * kRadix);
     GS_LAUNCH_CHECK();
     if (use32) {
       k_downsweep32<<<(unsigned)tiles, kSortThreads, sizeof(DownSmem32), s>>>(
           reinterpret_cast<const uint32_t*>(sk), sv, siota, reinterpret_cast<uint32_t*>(dk), dv,
-          (int)n, plan.shift[p], plan.bits[p], w.counts, (int)tiles, dev_status);
+          (int)n, plan.shift[p], plan.bits[p], w.counts, (int)tiles, dev_status, n_dev);
     } else {
       k_downsweep<K><<<(unsigned)tiles, kSortThreads, smem, s>>>(
           sk, sv, siota, dk, dv, n, plan.shift[p], plan.bits[p], w.counts, tiles, dev_status);
@@ -649,6 +657,17 @@ gs_status sort_impl(const K* keys_in, K* keys, int32_t* vals, bool iota, bool st
 }
 
 }  // namespace
+
+// The depth order's sort: 32-bit keys, values 0..count-1, the count read on
+// the device (at most n).  Library-internal (hidden), used by gs_depth_order.
+__attribute__((visibility("hidden")))
+gs_status sort32_iota_devcount(const uint32_t* keys_in, uint32_t* keys, int32_t* vals, int64_t n,
+                               const int32_t* n_dev, void* ws, size_t ws_bytes,
+                               int32_t* dev_status, cudaStream_t s) {
+  return sort_impl<uint32_t>(keys_in, keys, vals, true, false, n, 0, 32, ws, ws_bytes, dev_status,
+                             s, nullptr, 0, false, n_dev);
+}
+
 }  // namespace gs
 
 using namespace gs;

@@ -322,14 +322,37 @@ class Stepper:
             sat_h.copy_(sat, non_blocking=True)
             nc_h.copy_(n_cand_d, non_blocking=True)
             sq_h.copy_(sq_d, non_blocking=True)
-            torch.cuda.current_stream(dev).synchronize()   # the one sync per view
+            clk.toc(tk)
+            tables_ready = torch.cuda.Event()
+            tables_ready.record()
+            # what needs no host decision is issued before the host waits, so
+            # the GPU works while the host reads the tables and plans: the
+            # compact 2D gradient, zeroed on a side stream (the raster
+            # backward, its first user, waits for it), and the depth presort
+            # on the candidate count the projection left on the device
+            g2d = torch.empty(cap * 12, dtype=torch.float32, device=dev)
+            if self._fill_stream is None:
+                self._fill_stream = torch.cuda.Stream(device=dev)
+            self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(self._fill_stream):
+                g2d.zero_()
+            g2d_ready = torch.cuda.Event()
+            g2d_ready.record(self._fill_stream)
+            order = torch.empty(cap, dtype=torch.int32, device=dev)
+            drect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
+            ows = torch.empty(B.gs_depth_order_workspace_size(cap), dtype=torch.uint8, device=dev)
+            tk = clk.tic("sort_depth")
+            B.gs_depth_order(proj, B.GS_COUNT_ON_DEVICE, order, drect, ows, st)
+            clk.toc(tk)
+            del ows
+            tables_ready.synchronize()   # the one host wait per view
             if int(nc_h[0]) <= cap:
                 break
             # more candidates than the capacity hint: the kernel skipped (and
             # flagged) those beyond it; clear the flag and project again
             B.gs_check(st)
             cap = int(nc_h[0])
-        clk.toc(tk)
+            tk = clk.tic("project")
         del ws
         if expand:
             del bws
@@ -343,27 +366,6 @@ class Stepper:
         if hooks is not None and hasattr(hooks, "on_project"):
             hooks.on_project(ctx)
 
-        # the compact 2D gradient, zeroed on a side stream so that the fill
-        # runs beside the depth sort and binning (the raster backward, its
-        # first user, waits for it)
-        g2d = torch.empty(max(C, 1) * 12, dtype=torch.float32, device=dev)
-        if self._fill_stream is None:
-            self._fill_stream = torch.cuda.Stream(device=dev)
-        self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(self._fill_stream):
-            g2d.zero_()
-        g2d_ready = torch.cuda.Event()
-        g2d_ready.record(self._fill_stream)
-
-        # ---- depth presort (+ rects gathered in depth order) ------------------
-        order = torch.empty(max(C, 1), dtype=torch.int32, device=dev)
-        drect = torch.empty(max(C, 1) * 4, dtype=torch.int16, device=dev)
-        if C > 0:
-            ws = torch.empty(B.gs_depth_order_workspace_size(C), dtype=torch.uint8, device=dev)
-            tk = clk.tic("sort_depth")
-            B.gs_depth_order(proj, C, order, drect, ws, st)
-            clk.toc(tk)
-            del ws
         ctx["depth_order"] = order
         ctx["depth_rect"] = drect
 

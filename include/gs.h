@@ -343,8 +343,11 @@ gs_status gs_leaf_partition(const int64_t* sat_host, int32_t TW, int32_t TH,
  * gs_depth_order (once per view): depth_order[0..n_cand) = candidate slots
  * sorted by the fp32 bits of their depth (stable: equal depths keep the
  * ascending Gaussian index), and depth_rect[j] = rect[depth_order[j]].
- *
- * gs_bin_tiles (per Leaf): for the candidates in depth order, one entry per
+ * n_cand = GS_COUNT_ON_DEVICE reads the count from proj->n_cand on the
+ * device (at most proj->capacity; buffers and workspace sized for the
+ * capacity), so the call can be issued before the host has read it. */
+#define GS_COUNT_ON_DEVICE (-1)
+/* gs_bin_tiles (per Leaf): for the candidates in depth order, one entry per
  * tile of rect ∩ leaf, written in depth order: vals = candidate slot,
  * tile_keys = Leaf-local tile index (ly * leaf width + lx), and, if keys64
  * is not NULL, the duplicated 64-bit key (tile id << 32) | depth_key.  A

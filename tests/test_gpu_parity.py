@@ -304,21 +304,27 @@ def _bin_leaf(pb, C, order_d, drect_d, L, TW, TH, sat_d, I, tile_bits):
     return emitted, tkeys, vals, k64, v64, ranges
 
 
-def test_depth_order(oracle_mod):
-    sc, cam = scene("hd")
+@pytest.mark.parametrize("name,on_device", [("hd", False), ("hd", True), ("tiny", True)])
+def test_depth_order(oracle_mod, name, on_device):
+    """gs_depth_order against numpy's stable argsort of the oracle's depth
+    keys, with the count given by the host or read on the device
+    (GS_COUNT_ON_DEVICE: buffers sized for a capacity above the count)."""
+    sc, cam = scene(name)
     pr = oracle_mod.project(sc.params.astype(np.float64), sc.n, sc.sh_degree, cam)
     C = len(pr["cand_idx"])
     pb = ProjBuffers.from_oracle(pr, sc.n)
     b = B()
-    order = torch.zeros(C, dtype=torch.int32, device="cuda")
-    drect = torch.zeros(4 * C, dtype=torch.int16, device="cuda")
-    ws = torch.empty(b.gs_depth_order_workspace_size(C), dtype=torch.uint8, device="cuda")
+    cap = pb.cap if on_device else C
+    assert cap >= C
+    order = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    drect = torch.zeros(4 * cap, dtype=torch.int16, device="cuda")
+    ws = torch.empty(b.gs_depth_order_workspace_size(cap), dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    b.gs_depth_order(pb.struct, C, order, drect, ws, st)
+    b.gs_depth_order(pb.struct, b.GS_COUNT_ON_DEVICE if on_device else C, order, drect, ws, st)
     assert b.gs_check(st) == 0
     exp = np.argsort(pr["key"], kind="stable")
-    assert (order.cpu().numpy() == exp).all()
-    assert (drect.cpu().numpy().reshape(-1, 4) == pr["rect"][exp]).all()
+    assert (order[:C].cpu().numpy() == exp).all()
+    assert (drect[:4 * C].cpu().numpy().reshape(-1, 4) == pr["rect"][exp]).all()
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "hd"])
