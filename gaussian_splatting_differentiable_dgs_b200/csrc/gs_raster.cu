@@ -74,31 +74,60 @@ __device__ __forceinline__ Staged stage_record(const float4* __restrict__ rec, i
   return s;
 }
 
+// A staged record as the forward's pixel pairs read it: every field twice,
+// so that one packed fp32x2 operation applies it to both pixels; the
+// colours negated (they multiply the negated weight).
+struct __align__(16) Packed {
+  float2 gy, beta;
+  float2 ns1, ns2;
+  float2 lo2, nr;
+  float2 ng, nb;
+  float2 gx;
+};
+
+__device__ __forceinline__ Packed pack_record(const Staged& st) {
+  Packed q;
+  q.gx = make_float2(st.gx, st.gx);
+  q.gy = make_float2(st.gy, st.gy);
+  q.beta = make_float2(st.beta, st.beta);
+  q.ns1 = make_float2(st.ns1, st.ns1);
+  q.ns2 = make_float2(st.ns2, st.ns2);
+  q.lo2 = make_float2(st.lo2, st.lo2);
+  q.nr = make_float2(-st.r, -st.r);
+  q.ng = make_float2(-st.g, -st.g);
+  q.nb = make_float2(-st.b, -st.b);
+  return q;
+}
+
+// The backward's form: colours as they are.
+struct __align__(16) PackedB {
+  float2 gy, beta;
+  float2 ns1, ns2;
+  float2 lo2, r;
+  float2 g, b;
+  float2 gx;
+};
+
+__device__ __forceinline__ PackedB pack_record_bwd(const Staged& st) {
+  PackedB q;
+  q.gx = make_float2(st.gx, st.gx);
+  q.gy = make_float2(st.gy, st.gy);
+  q.beta = make_float2(st.beta, st.beta);
+  q.ns1 = make_float2(st.ns1, st.ns1);
+  q.ns2 = make_float2(st.ns2, st.ns2);
+  q.lo2 = make_float2(st.lo2, st.lo2);
+  q.r = make_float2(st.r, st.r);
+  q.g = make_float2(st.g, st.g);
+  q.b = make_float2(st.b, st.b);
+  return q;
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-struct Eval {
-  float dx, dy, t1, araw, alpha;
-};
-
-// alpha = min(0.99, o e^-q) = min(0.99, 2^(log2 o - q log2 e)),
-// q = s1 (dx + beta dy)^2 + s2 dy^2, with dx = gx - px given (a lane's
-// pixels share their column); araw = o e^-q is the unclamped value
-__device__ __forceinline__ Eval eval_alpha(float dx, float gy, float beta, float ns1, float ns2,
-                                           float lo2, float py) {
-  Eval e;
-  e.dx = dx;
-  e.dy = __fsub_rn(gy, py);
-  e.t1 = __fmaf_rn(beta, e.dy, e.dx);
-  const float qa = __fmul_rn(ns1, e.t1);
-  const float qb = __fmaf_rn(__fmul_rn(ns2, e.dy), e.dy, lo2);
-  e.araw = ex2_approx(__fmaf_rn(qa, e.t1, qb));
-  e.alpha = fminf(e.araw, kAlphaMax);
-  return e;
-}
 
 struct PixArgs {
   int32_t x0, y0, w, h;
@@ -199,6 +228,58 @@ __device__ __forceinline__ unsigned warp_mask(const Staged& st) {
   return m;
 }
 
+// One staged entry composited into a lane's pixel pairs, front to back.
+// alpha = min(0.99, o e^-q) = min(0.99, 2^(log2 o - q log2 e)) with
+// q = s1 (dx + beta dy)^2 + s2 dy^2, dx = gx - px, dy = gy - py, each step
+// one rounded operation (dx and dy once per pixel, t = beta dy + dx as one
+// fma, q log2 e as ns1 t^2 + ns2 dy^2 from one product and two fmas).
+// Branch-free: every pixel evaluates.  A pixel that is done, skips the
+// entry or stops at it composites with a zero alpha, which leaves T and the
+// colour sums exactly as they were.  A packed fp32x2 operation rounds each
+// of its two pixels as the scalar operation would; T (1 - alpha) is one
+// fma, and the negated alpha and colours make every product exact to negate.
+template <int NP, bool COUNT>
+__device__ __forceinline__ void composite_entry(const Packed& R, int posn, float2 nfpx2,
+                                                const float2 (&npy2)[NP], float2 (&T2)[NP],
+                                                float2 (&Cr2)[NP], float2 (&Cg2)[NP],
+                                                float2 (&Cb2)[NP], bool (&done)[2 * NP],
+                                                int (&lastp)[2 * NP], int (&stopn)[2 * NP],
+                                                unsigned& n_vis, unsigned& n_kept) {
+  const float2 dx2 = __fadd2_rn(R.gx, nfpx2);  // gx - px
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const float2 dy = __fadd2_rn(R.gy, npy2[p]);
+    const float2 t1 = __ffma2_rn(R.beta, dy, dx2);
+    const float2 qa = __fmul2_rn(R.ns1, t1);
+    const float2 qb = __ffma2_rn(__fmul2_rn(R.ns2, dy), dy, R.lo2);
+    const float2 e = __ffma2_rn(qa, t1, qb);
+    float na[2] = {fmaxf(-ex2_approx(e.x), -kAlphaMax), fmaxf(-ex2_approx(e.y), -kAlphaMax)};
+    const float2 Tn = __ffma2_rn(make_float2(na[0], na[1]), T2[p], T2[p]);
+    const float tn[2] = {Tn.x, Tn.y};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = 2 * p + h;
+      if (COUNT) n_vis += done[k] ? 0u : 1u;
+      const bool use = !done[k] && na[h] <= -kAlphaMin;
+      const bool stop = use && tn[h] < kTMin;
+      const bool comp = use && !stop;
+      if (COUNT) {
+        stopn[k] = stop ? posn : stopn[k];
+        n_kept += comp ? 1u : 0u;
+      }
+      done[k] = done[k] || stop;
+      na[h] = comp ? na[h] : 0.0f;
+      lastp[k] = comp ? posn : lastp[k];
+    }
+    const float2 na2 = make_float2(na[0], na[1]);
+    const float2 nw = __fmul2_rn(na2, T2[p]);  // -alpha T
+    T2[p] = __ffma2_rn(na2, T2[p], T2[p]);
+    Cr2[p] = __ffma2_rn(R.nr, nw, Cr2[p]);
+    Cg2[p] = __ffma2_rn(R.ng, nw, Cg2[p]);
+    Cb2[p] = __ffma2_rn(R.nb, nw, Cb2[p]);
+  }
+}
+
 // The batch positions j in [j0, cnt) whose record meets warp w's pixels, in
 // ascending order, into list[0..n); returns n (warp-uniform).
 template <class LT>
@@ -250,8 +331,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   constexpr int CAP = NT;
   using LT = std::conditional_t<(CAP <= 256), uint8_t, uint16_t>;
   constexpr int HCAP = BLK ? kFillU * NT : 1;
-  __shared__ float4 sA[CAP], sB[CAP];
-  __shared__ float sC[CAP];
+  __shared__ Packed sPk[CAP];
   __shared__ uint8_t s_mask[CAP];
   __shared__ LT s_list[G::NW][CAP];
   __shared__ float s_red[G::NW];
@@ -271,29 +351,38 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   }
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const WarpPix wp = warp_pixels<PPT>(t);
+  // the lane's pixels in pairs (NP of them; with an odd PPT the last pair's
+  // second pixel is a placeholder that starts done): the per-pixel state of
+  // a pair lives in float2s that packed fp32x2 operations update together
+  constexpr int NP = (PPT + 1) / 2;
   const float fpx = (float)wp.lx + 0.5f;
-  float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
-  int lastp[PPT];
-  int stopn[PPT];  // COUNT: 1-based list position of the stopping entry, 0 = none
-  bool done[PPT], inside[PPT];
+  const float2 nfpx2 = make_float2(-fpx, -fpx);
+  float2 npy2[NP], T2[NP], Cr2[NP], Cg2[NP], Cb2[NP];
+  int lastp[2 * NP];
+  int stopn[2 * NP];  // COUNT: 1-based list position of the stopping entry, 0 = none
+  bool done[2 * NP], inside[2 * NP];
   unsigned n_vis = 0, n_kept = 0;
 #pragma unroll
-  for (int k = 0; k < PPT; ++k) {
+  for (int k = 0; k < 2 * NP; ++k) {
     const int ly = wp.ly0 + k * G::LROWS;
-    fpy[k] = (float)ly + 0.5f;
-    inside[k] = (tx * kTile + wp.lx < W) && (ty * kTile + ly < H);
+    const float npy = -((float)ly + 0.5f);
+    if (k & 1) npy2[k >> 1].y = npy; else npy2[k >> 1].x = npy;
+    inside[k] = k < PPT && (tx * kTile + wp.lx < W) && (ty * kTile + ly < H);
     done[k] = !inside[k];
-    T[k] = 1.0f;
-    Cr[k] = Cg[k] = Cb[k] = 0.0f;
     lastp[k] = 0;
     stopn[k] = 0;
+  }
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    T2[p] = make_float2(1.0f, 1.0f);
+    Cr2[p] = Cg2[p] = Cb2[p] = make_float2(0.0f, 0.0f);
   }
   bool bad = false;
   for (int64_t base = begin;; base += NT) {
     if (!BLK && base >= end) break;
     bool mine_done = true;
 #pragma unroll
-    for (int k = 0; k < PPT; ++k) mine_done = mine_done && done[k];
+    for (int k = 0; k < 2 * NP; ++k) mine_done = mine_done && done[k];
     if (__syncthreads_count(mine_done) == NT) break;
     int cnt, pos1;
     if (BLK) {
@@ -348,9 +437,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       if (t < cnt) {
         const Staged st = stage_record(rec, s_hits[hp + t], tx, ty);
         s_mask[t] = (uint8_t)warp_mask<PPT>(st);
-        sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-        sB[t] = make_float4(st.ns2, st.lo2, st.r, st.g);
-        sC[t] = st.b;
+        sPk[t] = pack_record(st);
       }
       __syncthreads();
       pos1 = (int)n_staged + 1;
@@ -361,9 +448,7 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       if (e < end) {
         const Staged st = stage_record(rec, vals[e], tx, ty);
         s_mask[t] = (uint8_t)warp_mask<PPT>(st);
-        sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-        sB[t] = make_float4(st.ns2, st.lo2, st.r, st.g);
-        sC[t] = st.b;
+        sPk[t] = pack_record(st);
       }
       __syncthreads();
       cnt = (int)min((int64_t)NT, end - base);
@@ -375,40 +460,16 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       if (i0 > 0) {
         bool d_all = true;
 #pragma unroll
-        for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
+        for (int k = 0; k < 2 * NP; ++k) d_all = d_all && done[k];
         if (__all_sync(0xffffffffu, d_all)) break;
       }
       const int i1 = min(nl, i0 + 32);
       for (int i = i0; i < i1; ++i) {
-      const int j = s_list[w][i];
-      const float4 A = sA[j];
-      const float4 B = sB[j];
-      const float Bb = sC[j];
-      const int posn = pos1 + j;
-      const float dx = __fsub_rn(A.x, fpx);
-      // branch-free: every pixel evaluates, and selects keep the state of
-      // a pixel that is done, skips the entry or stops at it (a zero weight
-      // leaves the colour sums unchanged)
-#pragma unroll
-      for (int k = 0; k < PPT; ++k) {
-        const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
-        if (COUNT) n_vis += done[k] ? 0u : 1u;
-        const bool use = !done[k] && ev.alpha >= kAlphaMin;
-        const float Tn = __fmaf_rn(-ev.alpha, T[k], T[k]);  // T (1 - alpha), one rounding
-        const bool stop = use && Tn < kTMin;
-        const bool comp = use && !stop;
-        if (COUNT) {
-          stopn[k] = stop ? posn : stopn[k];
-          n_kept += comp ? 1u : 0u;
-        }
-        done[k] = done[k] || stop;
-        const float wgt = comp ? ev.alpha * T[k] : 0.0f;
-        Cr[k] = fmaf(B.z, wgt, Cr[k]);
-        Cg[k] = fmaf(B.w, wgt, Cg[k]);
-        Cb[k] = fmaf(Bb, wgt, Cb[k]);
-        T[k] = comp ? Tn : T[k];
-        lastp[k] = comp ? posn : lastp[k];
-      }
+        const int j = s_list[w][i];
+        const Packed R = sPk[j];
+        const int posn = pos1 + j;
+        composite_entry<NP, COUNT>(R, posn, nfpx2, npy2, T2, Cr2, Cg2, Cb2, done, lastp, stopn,
+                                   n_vis, n_kept);
       }
     }
   }
@@ -445,15 +506,16 @@ k_raster_fwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     if (!inside[k]) continue;
     const int x = tx * kTile + wp.lx, y = ty * kTile + wp.ly0 + k * G::LROWS;
     const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
+    const float2 T_ = T2[k >> 1], r_ = Cr2[k >> 1], g_ = Cg2[k >> 1], b_ = Cb2[k >> 1];
+    const float c[3] = {(k & 1) ? r_.y : r_.x, (k & 1) ? g_.y : g_.x, (k & 1) ? b_.y : b_.x};
     if (px.img) {
-      px.img[o] = Cr[k];
-      px.img[o + px.plane] = Cg[k];
-      px.img[o + 2 * px.plane] = Cb[k];
+      px.img[o] = c[0];
+      px.img[o + px.plane] = c[1];
+      px.img[o + 2 * px.plane] = c[2];
     }
-    px.T_final[o] = T[k];
+    px.T_final[o] = (k & 1) ? T_.y : T_.x;
     px.last[o] = lastp[k];
     if (px.target) {
-      const float c[3] = {Cr[k], Cg[k], Cb[k]};
       const int64_t ot = (int64_t)(y - px.ty0) * px.tpitch + (x - px.tx0);
 #pragma unroll
       for (int ch = 0; ch < 3; ++ch) {
@@ -518,8 +580,7 @@ k_raster_fwd_ws(const float4* __restrict__ rec, gs_rect leaf, int W, int H, int 
                 BlockSrc bsrc, int32_t* dev_status) {
   using G = TileGeom<PPT>;
   constexpr int NC = G::NW;
-  __shared__ float4 sA[kWsS][32], sB[kWsS][32];
-  __shared__ float sC[kWsS][32];
+  __shared__ Packed sPk[kWsS][32];
   __shared__ uint8_t sM[kWsS][32];
   __shared__ int sCnt[kWsS], sPos[kWsS];
   __shared__ unsigned long long s_full[kWsS], s_empty[kWsS];
@@ -592,9 +653,7 @@ k_raster_fwd_ws(const float4* __restrict__ rec, gs_rect leaf, int W, int H, int 
       if (lane < m) {
         const Staged g = stage_record(rec, s_q[(qh + lane) & (kWsQ - 1)], tx, ty);
         sM[st][lane] = (uint8_t)warp_mask<PPT>(g);
-        sA[st][lane] = make_float4(g.gx, g.gy, g.beta, g.ns1);
-        sB[st][lane] = make_float4(g.ns2, g.lo2, g.r, g.g);
-        sC[st][lane] = g.b;
+        sPk[st][lane] = pack_record(g);
       }
       if (lane == 0) {
         sCnt[st] = m;
@@ -628,22 +687,31 @@ k_raster_fwd_ws(const float4* __restrict__ rec, gs_rect leaf, int W, int H, int 
 
   // ---- consumer warps ----
   const WarpPix wp = warp_pixels<PPT>(t);
+  // the lane's pixels in pairs (NP of them; with an odd PPT the last pair's
+  // second pixel is a placeholder that starts done): the per-pixel state of
+  // a pair lives in float2s that packed fp32x2 operations update together
+  constexpr int NP = (PPT + 1) / 2;
   const float fpx = (float)wp.lx + 0.5f;
-  float fpy[PPT], T[PPT], Cr[PPT], Cg[PPT], Cb[PPT];
-  int lastp[PPT];
-  int stopn[PPT];  // COUNT: 1-based list position of the stopping entry, 0 = none
-  bool done[PPT], inside[PPT];
+  const float2 nfpx2 = make_float2(-fpx, -fpx);
+  float2 npy2[NP], T2[NP], Cr2[NP], Cg2[NP], Cb2[NP];
+  int lastp[2 * NP];
+  int stopn[2 * NP];  // COUNT: 1-based list position of the stopping entry, 0 = none
+  bool done[2 * NP], inside[2 * NP];
   unsigned n_vis = 0, n_kept = 0;
 #pragma unroll
-  for (int k = 0; k < PPT; ++k) {
+  for (int k = 0; k < 2 * NP; ++k) {
     const int ly = wp.ly0 + k * G::LROWS;
-    fpy[k] = (float)ly + 0.5f;
-    inside[k] = (tx * kTile + wp.lx < W) && (ty * kTile + ly < H);
+    const float npy = -((float)ly + 0.5f);
+    if (k & 1) npy2[k >> 1].y = npy; else npy2[k >> 1].x = npy;
+    inside[k] = k < PPT && (tx * kTile + wp.lx < W) && (ty * kTile + ly < H);
     done[k] = !inside[k];
-    T[k] = 1.0f;
-    Cr[k] = Cg[k] = Cb[k] = 0.0f;
     lastp[k] = 0;
     stopn[k] = 0;
+  }
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    T2[p] = make_float2(1.0f, 1.0f);
+    Cr2[p] = Cg2[p] = Cb2[p] = make_float2(0.0f, 0.0f);
   }
   bool counted = false;
   for (int ks = 0;; ++ks) {
@@ -657,42 +725,20 @@ k_raster_fwd_ws(const float4* __restrict__ rec, gs_rect leaf, int W, int H, int 
     if (cnt < 0 || warp_flag(&s_abort)) break;
     bool d_all = true;
 #pragma unroll
-    for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
+    for (int k = 0; k < 2 * NP; ++k) d_all = d_all && done[k];
     if (!__all_sync(0xffffffffu, d_all)) {
       const int pos1 = sPos[st] + 1;
       unsigned bits = __ballot_sync(0xffffffffu, lane < cnt && ((sM[st][lane] >> w) & 1u));
       while (bits) {
         const int j = __ffs(bits) - 1;
         bits &= bits - 1u;
-        const float4 A = sA[st][j];
-        const float4 B = sB[st][j];
-        const float Bb = sC[st][j];
-        const int posn = pos1 + j;
-        const float dx = __fsub_rn(A.x, fpx);
-#pragma unroll
-        for (int k = 0; k < PPT; ++k) {
-          const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
-          if (COUNT) n_vis += done[k] ? 0u : 1u;
-          const bool use = !done[k] && ev.alpha >= kAlphaMin;
-          const float Tn = __fmaf_rn(-ev.alpha, T[k], T[k]);  // T (1 - alpha), one rounding
-          const bool stop = use && Tn < kTMin;
-          const bool comp = use && !stop;
-          if (COUNT) {
-            stopn[k] = stop ? posn : stopn[k];
-            n_kept += comp ? 1u : 0u;
-          }
-          done[k] = done[k] || stop;
-          const float wgt = comp ? ev.alpha * T[k] : 0.0f;
-          Cr[k] = fmaf(B.z, wgt, Cr[k]);
-          Cg[k] = fmaf(B.w, wgt, Cg[k]);
-          Cb[k] = fmaf(Bb, wgt, Cb[k]);
-          T[k] = comp ? Tn : T[k];
-          lastp[k] = comp ? posn : lastp[k];
-        }
+        const Packed R = sPk[st][j];
+        composite_entry<NP, COUNT>(R, pos1 + j, nfpx2, npy2, T2, Cr2, Cg2, Cb2, done, lastp,
+                                   stopn, n_vis, n_kept);
       }
       d_all = true;
 #pragma unroll
-      for (int k = 0; k < PPT; ++k) d_all = d_all && done[k];
+      for (int k = 0; k < 2 * NP; ++k) d_all = d_all && done[k];
       d_all = __all_sync(0xffffffffu, d_all);
     }
     if (d_all && !counted) {
@@ -728,15 +774,16 @@ k_raster_fwd_ws(const float4* __restrict__ rec, gs_rect leaf, int W, int H, int 
     if (!inside[k]) continue;
     const int x = tx * kTile + wp.lx, y = ty * kTile + wp.ly0 + k * G::LROWS;
     const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
+    const float2 T_ = T2[k >> 1], r_ = Cr2[k >> 1], g_ = Cg2[k >> 1], b_ = Cb2[k >> 1];
+    const float c[3] = {(k & 1) ? r_.y : r_.x, (k & 1) ? g_.y : g_.x, (k & 1) ? b_.y : b_.x};
     if (px.img) {
-      px.img[o] = Cr[k];
-      px.img[o + px.plane] = Cg[k];
-      px.img[o + 2 * px.plane] = Cb[k];
+      px.img[o] = c[0];
+      px.img[o + px.plane] = c[1];
+      px.img[o + 2 * px.plane] = c[2];
     }
-    px.T_final[o] = T[k];
+    px.T_final[o] = (k & 1) ? T_.y : T_.x;
     px.last[o] = lastp[k];
     if (px.target) {
-      const float c[3] = {Cr[k], Cg[k], Cb[k]};
       const int64_t ot = (int64_t)(y - px.ty0) * px.tpitch + (x - px.tx0);
 #pragma unroll
       for (int ch = 0; ch < 3; ++ch) {
@@ -841,12 +888,11 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
              float* __restrict__ g2d, int32_t* dev_status) {
   using G = TileGeom<PPT>;
   constexpr int NT = G::NT;
-  __shared__ float4 sA[NT], sB[NT];
-  __shared__ float4 sC[NT];       // {b, 2 s1, 2 s2, slot bits}
+  __shared__ PackedB sPk[NT];
+  __shared__ float4 sF[NT];  // {2 s1, 2 s2, slot bits, beta}
   __shared__ uint8_t s_mask[NT];
   __shared__ uint8_t s_list[G::NW][NT];
-  __shared__ float sg[NT][12];
-  __shared__ int s_touched[NT];
+  __shared__ float sg[NT][12];  // the record's 9 sums; word 9: "touched" flag (int)
   __shared__ float s_red[G::NW][32 * 9];
   __shared__ int s_maxlast;
   const int lw = leaf.x1 - leaf.x0;
@@ -856,40 +902,50 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const int rv = lane / 3, rp = lane - 3 * (lane / 3);  // reduction role (warp_reduce9_smem)
   const WarpPix wp = warp_pixels<PPT>(t);
+  // the lane's pixels in pairs (an odd PPT's last pair has a placeholder
+  // second pixel with last = 0, which never takes part), their state in
+  // float2s for packed fp32x2 operations.  NS = -S, S = sum_c g_c A_c with
+  // A_c the colour composited behind the current entry.
+  constexpr int NP = (PPT + 1) / 2;
   const float fpx = (float)wp.lx + 0.5f;
-  // S = sum_c g_c A_c, A_c = colour composited behind the current entry
-  float fpy[PPT], T[PPT], S[PPT], gr[PPT], gg[PPT], gb[PPT];
-  int lastp[PPT];
+  const float2 nfpx2 = make_float2(-fpx, -fpx);
+  float2 npy2[NP], T2[NP], NS2[NP], gr2[NP], gg2[NP], gb2[NP];
+  int lastp[2 * NP];
   if (t == 0) s_maxlast = 0;
   for (int e = t; e < NT * 12; e += NT) (&sg[0][0])[e] = 0.0f;
-  s_touched[t] = 0;
   __syncthreads();
   int mylast = 0;
 #pragma unroll
-  for (int k = 0; k < PPT; ++k) {
+  for (int k = 0; k < 2 * NP; ++k) {
     const int ly = wp.ly0 + k * G::LROWS;
-    fpy[k] = (float)ly + 0.5f;
     const int x = tx * kTile + wp.lx, y = ty * kTile + ly;
-    S[k] = 0.0f;
-    if (x < W && y < H) {
+    float Tk = 1.0f, r = 0.0f, g = 0.0f, b = 0.0f;
+    int lk = 0;
+    if (k < PPT && x < W && y < H) {
       const int64_t o = (int64_t)(y - px.y0) * px.pitch + (x - px.x0);
-      T[k] = px.T_final[o];
-      lastp[k] = px.last[o];
-      gr[k] = px.dL[o];
-      gg[k] = px.dL[o + px.plane];
-      gb[k] = px.dL[o + 2 * px.plane];
-    } else {
-      T[k] = 1.0f;
-      lastp[k] = 0;
-      gr[k] = gg[k] = gb[k] = 0.0f;
+      Tk = px.T_final[o];
+      lk = px.last[o];
+      r = px.dL[o];
+      g = px.dL[o + px.plane];
+      b = px.dL[o + 2 * px.plane];
     }
-    mylast = max(mylast, lastp[k]);
+    const float npy = -((float)ly + 0.5f);
+    if (k & 1) {
+      npy2[k >> 1].y = npy; T2[k >> 1].y = Tk; NS2[k >> 1].y = 0.0f;
+      gr2[k >> 1].y = r; gg2[k >> 1].y = g; gb2[k >> 1].y = b;
+    } else {
+      npy2[k >> 1].x = npy; T2[k >> 1].x = Tk; NS2[k >> 1].x = 0.0f;
+      gr2[k >> 1].x = r; gg2[k >> 1].x = g; gb2[k >> 1].x = b;
+    }
+    lastp[k] = lk;
+    mylast = max(mylast, lk);
   }
   const int warp_last = __reduce_max_sync(0xffffffffu, mylast);
   if (lane == 0) atomicMax(&s_maxlast, warp_last);
   __syncthreads();
   const int tile_last = s_maxlast;
   unsigned n_vis = 0, n_kept = 0;
+  const float2 one2 = make_float2(1.0f, 1.0f), zero2 = make_float2(0.0f, 0.0f);
 
   for (int bend = tile_last; bend > 0; bend -= NT) {
     const int bstart = max(0, bend - NT);
@@ -898,9 +954,8 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
       const int pos = bend - 1 - t;
       const Staged st = stage_record(rec, vals[begin + pos], tx, ty);
       s_mask[t] = (uint8_t)warp_mask<PPT>(st);
-      sA[t] = make_float4(st.gx, st.gy, st.beta, st.ns1);
-      sB[t] = make_float4(st.ns2, st.lo2, st.r, st.g);
-      sC[t] = make_float4(st.b, 2.0f * st.s1, 2.0f * st.s2, __int_as_float(st.slot));
+      sPk[t] = pack_record_bwd(st);
+      sF[t] = make_float4(2.0f * st.s1, 2.0f * st.s2, __int_as_float(st.slot), st.beta);
     }
     __syncthreads();
     // positions at or beyond every lane's `last` need no work in this warp
@@ -909,91 +964,108 @@ k_raster_bwd(const float4* __restrict__ rec, const int32_t* __restrict__ vals,
     for (int i = 0; i < nl; ++i) {
       const int j = s_list[w][i];
       const int pos = bend - 1 - j;
-      const float4 A = sA[j];
-      const float4 B = sB[j];
-      const float4 Cc = sC[j];
-      float acc[9];
-#pragma unroll
-      for (int q = 0; q < 9; ++q) acc[q] = 0.0f;
-      // the lane's pixels share dx, so the geometric terms need only
-      // sum dq, sum dq dy and sum dq dy^2 over them
-      float sq = 0.0f, sqy = 0.0f, sqyy = 0.0f;
+      const PackedB R = sPk[j];
+      // per pair: m6..m8 = -sum alpha T_before g_c, and the dq moments (the
+      // lane's pixels share dx, so the geometric terms need only sum dq,
+      // sum dq dy and sum dq dy^2 over them)
+      float2 m6 = zero2, m7 = zero2, m8 = zero2, sq2 = zero2, sqy2 = zero2, sqyy2 = zero2;
       bool any = false;
-      const float dx = __fsub_rn(A.x, fpx);
+      const float2 dx2 = __fadd2_rn(R.gx, nfpx2);  // gx - px
       // branch-free: an entry at or beyond the pixel's last, or below 1/255,
       // enters with alpha = 0, which leaves T, S and every sum unchanged
 #pragma unroll
-      for (int k = 0; k < PPT; ++k) {
-        const bool inl = pos < lastp[k];
-        const Eval ev = eval_alpha(dx, A.y, A.z, A.w, B.x, B.y, fpy[k]);
-        const bool use = inl && ev.alpha >= kAlphaMin;
-        if (COUNT) {
-          n_vis += inl ? 1u : 0u;
-          n_kept += use ? 1u : 0u;
+      for (int p = 0; p < NP; ++p) {
+        const float2 dy = __fadd2_rn(R.gy, npy2[p]);
+        const float2 t1 = __ffma2_rn(R.beta, dy, dx2);
+        const float2 qa = __fmul2_rn(R.ns1, t1);
+        const float2 qb = __ffma2_rn(__fmul2_rn(R.ns2, dy), dy, R.lo2);
+        const float2 e = __ffma2_rn(qa, t1, qb);
+        const float raw[2] = {ex2_approx(e.x), ex2_approx(e.y)};  // o e^-q
+        float nau[2], nua[2];
+        bool use[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const bool inl = pos < lastp[2 * p + h];
+          const float na = fmaxf(-raw[h], -kAlphaMax);  // -alpha
+          use[h] = inl && na <= -kAlphaMin;
+          if (COUNT) {
+            n_vis += inl ? 1u : 0u;
+            n_kept += use[h] ? 1u : 0u;
+          }
+          any = any || use[h];
+          nau[h] = use[h] ? na : 0.0f;
+          // unclamped entries (alpha = araw = o e^-q): dL/dq (natural
+          // units) = -alpha dL/dalpha, and o dL/dopacity = alpha dL/dalpha
+          nua[h] = raw[h] <= kAlphaMax ? nau[h] : 0.0f;
         }
-        any = any || use;
-        const float au = use ? ev.alpha : 0.0f;
+        const float2 nau2 = make_float2(nau[0], nau[1]);
         // T only scales gradient values here (no decision depends on it), so
         // the hardware reciprocal (about 1 ulp) is enough
-        const float inv = rcp_approx(1.0f - au);
-        const float Tb = T[k] * inv;          // transmittance before this entry
-        const float wgt = au * Tb;
-        acc[6] = fmaf(wgt, gr[k], acc[6]);
-        acc[7] = fmaf(wgt, gg[k], acc[7]);
-        acc[8] = fmaf(wgt, gb[k], acc[8]);
-        // dL/dalpha = sum_c g_c (rgb_c T_i - A_c / (1 - alpha))
-        //           = T_i (g . rgb) - S / (1 - alpha)
-        const float grgb = fmaf(gb[k], Cc.x, fmaf(gg[k], B.w, gr[k] * B.z));
-        const float da = fmaf(Tb, grgb, -S[k] * inv);
-        S[k] = fmaf(wgt, grgb, S[k]);
-        T[k] = use ? Tb : T[k];
-        // unclamped entries (where alpha = araw = o e^-q): dL/dq (natural
-        // units) = -alpha dL/dalpha, and o dL/dopacity = alpha dL/dalpha
-        const float ua = ev.araw <= kAlphaMax ? au : 0.0f;
-        const float dq = -ua * da;
-        acc[5] = fmaf(ua, da, acc[5]);  // 1/o at the flush
-        sq += dq;
-        const float dqy = dq * ev.dy;
-        sqy += dqy;
-        sqyy = fmaf(dqy, ev.dy, sqyy);
+        const float2 om = __fadd2_rn(one2, nau2);  // 1 - alpha
+        const float2 inv = make_float2(rcp_approx(om.x), rcp_approx(om.y));
+        const float2 Tb = __fmul2_rn(T2[p], inv);  // transmittance before this entry
+        const float2 nwgt = __fmul2_rn(nau2, Tb);   // -alpha T_before
+        m6 = __ffma2_rn(nwgt, gr2[p], m6);
+        m7 = __ffma2_rn(nwgt, gg2[p], m7);
+        m8 = __ffma2_rn(nwgt, gb2[p], m8);
+        // dL/dalpha = sum_c g_c (rgb_c T_before - A_c / (1 - alpha))
+        //           = T_before (g . rgb) - S / (1 - alpha)
+        const float2 grgb =
+            __ffma2_rn(gb2[p], R.b, __ffma2_rn(gg2[p], R.g, __fmul2_rn(gr2[p], R.r)));
+        const float2 da = __ffma2_rn(Tb, grgb, __fmul2_rn(NS2[p], inv));
+        NS2[p] = __ffma2_rn(nwgt, grgb, NS2[p]);
+        T2[p].x = use[0] ? Tb.x : T2[p].x;
+        T2[p].y = use[1] ? Tb.y : T2[p].y;
+        const float2 dq = __fmul2_rn(make_float2(nua[0], nua[1]), da);
+        sq2 = __fadd2_rn(sq2, dq);
+        const float2 dqy = __fmul2_rn(dq, dy);
+        sqy2 = __fadd2_rn(sqy2, dqy);
+        sqyy2 = __ffma2_rn(dqy, dy, sqyy2);
       }
       // the geometric gradients are linear in five moments of dq over the
       // warp's pixels: sum dx dq, sum dx^2 dq, sum dq dy, sum dx dq dy and
       // sum dq dy^2 (turned into du, dv, da, db, dc once per record at the
-      // flush below)
+      // flush below); o dL/do = sum alpha dL/dalpha = -sum dq
+      const float dx = dx2.x;
+      const float sq = sq2.x + sq2.y, sqy = sqy2.x + sqy2.y;
+      float acc[9];
       const float dxq = dx * sq;
       acc[0] = dxq;
       acc[1] = dx * dxq;
       acc[2] = sqy;
       acc[3] = dx * sqy;
-      acc[4] = sqyy;
+      acc[4] = sqyy2.x + sqyy2.y;
+      acc[5] = -sq;
+      acc[6] = -(m6.x + m6.y);
+      acc[7] = -(m7.x + m7.y);
+      acc[8] = -(m8.x + m8.y);
       // reduce first: per-lane shared atomics on the same 9 words cost more
       // than the reduction, even with only 2 lanes kept
       if (__any_sync(0xffffffffu, any)) {
         const float tot = warp_reduce9_smem(acc, s_red[w], lane, rv, rp);
         if (lane < 27 && rp == 0) atomicAdd(&sg[j][rv], tot);
-        if (lane == 0) s_touched[j] = 1;
+        if (lane == 0) reinterpret_cast<int*>(sg[j])[9] = 1;
       }
     }
     __syncthreads();
-    if (t < cnt && s_touched[t]) {
-      const float4 Cc = sC[t];
-      const int32_t slot = __float_as_int(Cc.w);
-      const float beta = sA[t].z;
+    if (t < cnt && reinterpret_cast<const int*>(sg[t])[9]) {
+      const float4 F = sF[t];
+      const int32_t slot = __float_as_int(F.z);
+      const float beta = F.w;
       // q = (a dx^2 + c dy^2) / 2 + b dx dy with a = 2 s1, b = beta a,
       // c = 2 s2 + beta b: dq/du = a dx + b dy, dq/dv = b dx + c dy
       // = beta dq/du + 2 s2 dy, dq/da = dx^2 / 2, dq/db = dx dy, dq/dc = dy^2 / 2
-      const float du = Cc.y * fmaf(beta, sg[t][2], sg[t][0]);
-      const float dv = fmaf(beta, du, Cc.z * sg[t][2]);
+      const float du = F.x * fmaf(beta, sg[t][2], sg[t][0]);
+      const float dv = fmaf(beta, du, F.y * sg[t][2]);
       float4* dst = reinterpret_cast<float4*>(g2d + (int64_t)slot * 12);
       atomicAdd(dst, make_float4(du, dv, 0.5f * sg[t][1], sg[t][3]));
       // dL/do = sum e^-q dL/dalpha = (sum o e^-q dL/dalpha) / o, 1/o = 2^-log2 o
-      const float inv_o = ex2_approx(-sB[t].y);
+      const float inv_o = ex2_approx(-sPk[t].lo2.x);
       atomicAdd(dst + 1, make_float4(0.5f * sg[t][4], sg[t][5] * inv_o, sg[t][6], sg[t][7]));
       atomicAdd(dst + 2, make_float4(sg[t][8], 0.0f, 0.0f, 0.0f));
 #pragma unroll
       for (int q = 0; q < 9; ++q) sg[t][q] = 0.0f;
-      s_touched[t] = 0;
+      reinterpret_cast<int*>(sg[t])[9] = 0;
     }
     __syncthreads();
   }
