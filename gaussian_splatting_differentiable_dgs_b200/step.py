@@ -445,7 +445,13 @@ class Stepper:
 
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
-        arena = torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev)
+        # a bounded run's arenas take the whole Leaf budget (more only for an
+        # over-budget Leaf): every view then reuses the same cached blocks,
+        # where arenas sized to the view's largest Leaf would need a new
+        # device allocation (a host stall of up to tens of milliseconds) on
+        # the first view whose largest Leaf beats every earlier one
+        alloc_bytes = arena_bytes if original else max(arena_bytes, self.budget)
+        arena = torch.empty(max(alloc_bytes, 256), dtype=torch.uint8, device=dev)
         n_ls = 1 if original else max(1, min(self.leaf_streams, len(lv)))
         main = torch.cuda.current_stream(dev)
         arenas, lstreams = [arena], [main]
@@ -453,7 +459,7 @@ class Stepper:
         while len(self._side_streams) < n_ls - 1:
             self._side_streams.append(torch.cuda.Stream(device=dev))
         for k in range(n_ls - 1):
-            arenas.append(torch.empty(max(arena_bytes, 256), dtype=torch.uint8, device=dev))
+            arenas.append(torch.empty(max(alloc_bytes, 256), dtype=torch.uint8, device=dev))
             bin_wss.append(torch.empty_like(bin_ws))  # the list builders' scratch, per stream
             lstreams.append(self._side_streams[k])
         norm = 1.0 / (3.0 * W * H)
