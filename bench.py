@@ -615,7 +615,7 @@ def main():
         # a copy stream during the view's own Leaves (two crops resident)
         from gaussian_splatting_differentiable_dgs_b200.step import TargetPrefetcher
         host_t = [t.cpu().pin_memory() for t in targets]
-        feeder = TargetPrefetcher(host_t) if a.e2e_mode == "prefetch" else None
+        feeder = TargetPrefetcher(host_t, stepper=stp) if a.e2e_mode == "prefetch" else None
         loss_h = torch.empty(1, dtype=torch.float64, pin_memory=True)
         if dist:
             dist.barrier()
@@ -643,7 +643,8 @@ def main():
         e2e = {"value": e2e_isect / (ems / 1e3), "unit": UNIT, "ms_per_step": ems / a.steps,
                "h2d_bytes_per_step": 3 * W * H * 4, "d2h_bytes_per_step": d2h,
                "supply": ("prefetch: each view's target uploaded during the previous view's "
-                          "step, two device targets resident") if feeder else
+                          "step (issued once that step's projection tables reached the host), "
+                          "two device targets resident") if feeder else
                          ("crops: each Leaf's crop uploaded during the view's Leaves, "
                           "two crops resident")}
 

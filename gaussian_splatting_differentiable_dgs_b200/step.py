@@ -110,14 +110,21 @@ class TargetPrefetcher:
     two device targets (2 x 3 x H x W fp32); the per-Leaf crop supply of
     `Stepper.run_view` with a host target holds two Leaf crops instead.
 
-        for v, target in TargetPrefetcher(host_targets).iterate(order):
+    Given the Stepper that consumes the targets, the next upload is issued
+    once the current view's projection tables have reached the host: a
+    device-to-host copy queued behind a 200 MB upload would hold back the
+    host's Leaf planning (0.12 ms per step on the 5000x3300 views).
+
+        feeder = TargetPrefetcher(host_targets, stepper=stepper)
+        for v, target in feeder.iterate(order):
             stepper.run_view(cams[v], target)
     """
 
-    def __init__(self, host_targets, device="cuda"):
+    def __init__(self, host_targets, device="cuda", stepper=None):
         self.host = host_targets          # indexable: view -> pinned [3][H][W] fp32
         self.device = torch.device(device)
         self.stream = torch.cuda.Stream(device=self.device)
+        self.stepper = stepper
         self._bufs = None
 
     def iterate(self, order):
@@ -132,11 +139,12 @@ class TargetPrefetcher:
         ready, free = [None, None], [None, None]
 
         def upload(slot, v):
-            # the buffer's previous reader (two steps back) must be done with it
+            # after the work issued on the main stream so far (with a Stepper:
+            # the current view's projection and its tables' read-back), and
+            # after the buffer's previous reader (two views back)
+            self.stream.wait_stream(main)
             if free[slot] is not None:
                 self.stream.wait_event(free[slot])
-            else:
-                self.stream.wait_stream(main)
             with torch.cuda.stream(self.stream):
                 self._bufs[slot].copy_(self.host[v], non_blocking=True)
             ev = torch.cuda.Event()
@@ -147,9 +155,18 @@ class TargetPrefetcher:
         for i, v in enumerate(order):
             slot = i & 1
             if i + 1 < len(order):
-                upload(1 - slot, order[i + 1])
+                nxt = (1 - slot, order[i + 1])
+                if self.stepper is not None:
+                    self.stepper._after_tables.append(lambda nxt=nxt: upload(*nxt))
+                else:
+                    upload(*nxt)
             main.wait_event(ready[slot])
             yield v, self._bufs[slot]
+            if self.stepper is not None and self.stepper._after_tables:
+                # the view was not stepped through this Stepper: upload now
+                calls, self.stepper._after_tables = self.stepper._after_tables, []
+                for f in calls:
+                    f()
             ev = torch.cuda.Event()
             ev.record(main)   # after the step's work on this buffer
             free[slot] = ev
@@ -229,6 +246,10 @@ class Stepper:
         self.leaf_streams = leaf_streams
         self._side_streams = []
         self._fill_stream = None
+        # one-shot callables run once the view's projection tables are on the
+        # host, before its Leaves are issued (TargetPrefetcher starts the next
+        # view's target upload there, after the tables' device-to-host copies)
+        self._after_tables = []
         self._cap_hint = {}  # region -> candidate capacity for the next view
 
     def check(self):
@@ -365,6 +386,9 @@ class Stepper:
                    sat=sat, sat_host=sat_np, n_cand=C, TW=TW, TH=TH, cam=cam)
         if hooks is not None and hasattr(hooks, "on_project"):
             hooks.on_project(ctx)
+        calls, self._after_tables = self._after_tables, []
+        for f in calls:
+            f()
 
         ctx["depth_order"] = order
         ctx["depth_rect"] = drect

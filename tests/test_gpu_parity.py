@@ -939,11 +939,13 @@ def test_host_target_matches_resident_target(streams):
     assert np.abs(p1 - p0).max() <= 2.1e-3
 
 
-def test_target_prefetcher_matches_resident_targets():
+@pytest.mark.parametrize("bound", [False, True])
+def test_target_prefetcher_matches_resident_targets(bound):
     """Views fed by TargetPrefetcher (each target uploaded from pinned host
     memory during the previous view's step, two device buffers) take the same
     steps as views whose targets are resident, over a sequence that reuses
-    both buffers."""
+    both buffers; bound: the prefetcher knows the Stepper and issues each
+    upload after the current view's projection tables reached the host."""
     from gaussian_splatting_differentiable_dgs_b200.step import (GaussianModel, Stepper,
                                                                   TargetPrefetcher)
     sc, cam = scene("small3")
@@ -956,7 +958,7 @@ def test_target_prefetcher_matches_resident_targets():
         losses = []
         if prefetch:
             host = [torch.as_tensor(t).pin_memory() for t in tg]
-            supply = TargetPrefetcher(host).iterate(order)
+            supply = TargetPrefetcher(host, stepper=stp if bound else None).iterate(order)
         else:
             dev = [torch.as_tensor(t).cuda() for t in tg]
             supply = ((v, dev[v]) for v in order)
