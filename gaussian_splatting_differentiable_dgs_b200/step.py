@@ -125,7 +125,15 @@ class TargetPrefetcher:
         self.device = torch.device(device)
         self.stream = torch.cuda.Stream(device=self.device)
         self.stepper = stepper
+        # the two device buffers are allocated here, not in the first step
+        # of an iteration (where a new device allocation would stall it)
         self._bufs = None
+        if len(host_targets):
+            self._alloc(tuple(host_targets[0].shape))
+
+    def _alloc(self, shape):
+        self._bufs = [torch.empty(shape, dtype=torch.float32, device=self.device)
+                      for _ in range(2)]
 
     def iterate(self, order):
         order = list(order)
@@ -133,8 +141,7 @@ class TargetPrefetcher:
             return
         shape = tuple(self.host[order[0]].shape)
         if self._bufs is None or tuple(self._bufs[0].shape) != shape:
-            self._bufs = [torch.empty(shape, dtype=torch.float32, device=self.device)
-                          for _ in range(2)]
+            self._alloc(shape)
         main = torch.cuda.current_stream(self.device)
         ready, free = [None, None], [None, None]
 
@@ -250,6 +257,7 @@ class Stepper:
         # host, before its Leaves are issued (TargetPrefetcher starts the next
         # view's target upload there, after the tables' device-to-host copies)
         self._after_tables = []
+        self._arena_hint = 0  # bytes per Leaf arena (bounded runs), see run_view
         self._cap_hint = {}  # region -> candidate capacity for the next view
 
     def check(self):
@@ -469,12 +477,16 @@ class Stepper:
 
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
-        # a bounded run's arenas take the whole Leaf budget (more only for an
-        # over-budget Leaf): every view then reuses the same cached blocks,
-        # where arenas sized to the view's largest Leaf would need a new
-        # device allocation (a host stall of up to tens of milliseconds) on
-        # the first view whose largest Leaf beats every earlier one
-        alloc_bytes = arena_bytes if original else max(arena_bytes, self.budget)
+        # a bounded run's arenas keep 25 % headroom over the largest Leaf seen
+        # (up to the Leaf budget; more only for an over-budget Leaf): later
+        # views then reuse the same cached blocks, where arenas sized to each
+        # view's largest Leaf would need a new device allocation (a host stall
+        # of up to tens of milliseconds) on the first view whose largest Leaf
+        # beats every earlier one
+        if not original:
+            self._arena_hint = max(self._arena_hint,
+                                   min(self.budget, arena_bytes + arena_bytes // 4))
+        alloc_bytes = arena_bytes if original else max(arena_bytes, self._arena_hint)
         arena = torch.empty(max(alloc_bytes, 256), dtype=torch.uint8, device=dev)
         n_ls = 1 if original else max(1, min(self.leaf_streams, len(lv)))
         main = torch.cuda.current_stream(dev)
