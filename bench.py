@@ -497,6 +497,9 @@ def main():
     nv = len(cams)
     view_of = lambda k: rank_view(k, rank, nv)
 
+    # the Leaf arenas sized for every view of the run (projection and Leaf
+    # planning only, before the warm-up), so that no timed step allocates
+    stp.reserve(cams)
     clocks = ClockSampler(local)
     for k in range(a.warmup):
         stp.run_view(cams[view_of(k)], targets[view_of(k)])
@@ -748,6 +751,8 @@ def run_sweep(a):
             target = target_dev if mode == "original" else target_host
             model = GaussianModel(scene.params, scene.n, scene.sh_degree)
             stp = Stepper(model, budget=budget, mode=mode, binning=a.binning)
+            if mode == "bounded":
+                stp.reserve([cam])  # candidate capacity and arena sized for the view
             torch.cuda.synchronize()
             torch.cuda.reset_peak_memory_stats()
             base = torch.cuda.memory_allocated()

@@ -260,6 +260,15 @@ class Stepper:
         self._arena_hint = 0  # bytes per Leaf arena (bounded runs), see run_view
         self._cap_hint = {}  # region -> candidate capacity for the next view
 
+    def reserve(self, cams, region=None):
+        """Sizes the Leaf arenas for the views a run will step through: each
+        view is projected and its Leaves planned (no raster, no update), and
+        later steps' arenas take the largest Leaf over these views plus 1/16
+        (at most the Leaf budget), so that no step needs a new device
+        allocation for them.  Also seeds the candidate-capacity hint."""
+        for cam in cams:
+            self.run_view(cam, None, region=region, plan_only=True)
+
     def check(self):
         st = B.gs_check(self.dev_status)
         if st < 0:
@@ -274,7 +283,7 @@ class Stepper:
     # ------------------------------------------------------------------
     def run_view(self, cam, target, leaves=None, hooks=None, update=True, backward=True,
                  timing=None, counters=None, region=None, grad_out=None,
-                 gate=None) -> ViewStats:
+                 gate=None, plan_only=False) -> ViewStats:
         """One view.  target: [3][H][W] fp32, a device tensor (the whole view
         resident, read in place) or a pinned host tensor (each Leaf's crop is
         uploaded before its forward); None renders only (no loss, backward or
@@ -286,7 +295,8 @@ class Stepper:
         grid).  grad_out: dense [P][n_pad] gradient the view's gradient is
         added to instead of taking the Adam step.  gate: callable(loss) ->
         bool asked with the view's forward loss (skipgs.BackwardGate); False
-        skips the backward and the update."""
+        skips the backward and the update.  plan_only: project and plan the
+        Leaves, size later arenas by them, and return None (`reserve`)."""
         dev = self.device
         if target is None:
             backward = update = False
@@ -359,14 +369,16 @@ class Stepper:
             # compact 2D gradient, zeroed on a side stream (the raster
             # backward, its first user, waits for it), and the depth presort
             # on the candidate count the projection left on the device
-            g2d = torch.empty(cap * 12, dtype=torch.float32, device=dev)
-            if self._fill_stream is None:
-                self._fill_stream = torch.cuda.Stream(device=dev)
-            self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
-            with torch.cuda.stream(self._fill_stream):
-                g2d.zero_()
-            g2d_ready = torch.cuda.Event()
-            g2d_ready.record(self._fill_stream)
+            g2d = g2d_ready = None
+            if not plan_only:
+                g2d = torch.empty(cap * 12, dtype=torch.float32, device=dev)
+                if self._fill_stream is None:
+                    self._fill_stream = torch.cuda.Stream(device=dev)
+                self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
+                with torch.cuda.stream(self._fill_stream):
+                    g2d.zero_()
+                g2d_ready = torch.cuda.Event()
+                g2d_ready.record(self._fill_stream)
             order = torch.empty(cap, dtype=torch.int32, device=dev)
             drect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
             ows = torch.empty(B.gs_depth_order_workspace_size(cap), dtype=torch.uint8, device=dev)
@@ -394,9 +406,10 @@ class Stepper:
                    sat=sat, sat_host=sat_np, n_cand=C, TW=TW, TH=TH, cam=cam)
         if hooks is not None and hasattr(hooks, "on_project"):
             hooks.on_project(ctx)
-        calls, self._after_tables = self._after_tables, []
-        for f in calls:
-            f()
+        if not plan_only:
+            calls, self._after_tables = self._after_tables, []
+            for f in calls:
+                f()
 
         ctx["depth_order"] = order
         ctx["depth_rect"] = drect
@@ -418,7 +431,7 @@ class Stepper:
                        block_ranges=branges, n_block_entries=n_blk)
 
         # ---- Leaf plan ------------------------------------------------------
-        ssim = self.loss == "l1_ssim" and target is not None
+        ssim = self.loss == "l1_ssim" and (target is not None or plan_only)
         lm = B.gs_leaf_load_model(tile_bits, (B.GS_BIN_EXPAND if expand else B.GS_BIN_SORT) |
                                   (B.GS_LOAD_SSIM if ssim else 0))
         if leaves is None and original:
@@ -477,15 +490,17 @@ class Stepper:
 
         arena_bytes = max((_carved_bytes(leaf_sizes(L, int(I))[0]) for L, I in zip(lv, li)),
                           default=0)
-        # a bounded run's arenas keep 25 % headroom over the largest Leaf seen
-        # (up to the Leaf budget; more only for an over-budget Leaf): later
-        # views then reuse the same cached blocks, where arenas sized to each
-        # view's largest Leaf would need a new device allocation (a host stall
-        # of up to tens of milliseconds) on the first view whose largest Leaf
-        # beats every earlier one
+        # a bounded run's arenas keep 1/16 headroom over the largest Leaf seen
+        # (up to the Leaf budget; more only for an over-budget Leaf), so that
+        # later views reuse the same cached blocks: an arena sized to each
+        # view's largest Leaf needs a new device allocation (a host stall of
+        # up to tens of milliseconds) on the first view whose largest Leaf
+        # beats every earlier one.  `reserve` plans a set of views up front.
         if not original:
             self._arena_hint = max(self._arena_hint,
-                                   min(self.budget, arena_bytes + arena_bytes // 4))
+                                   min(self.budget, arena_bytes + arena_bytes // 16))
+        if plan_only:
+            return None
         alloc_bytes = arena_bytes if original else max(arena_bytes, self._arena_hint)
         arena = torch.empty(max(alloc_bytes, 256), dtype=torch.uint8, device=dev)
         n_ls = 1 if original else max(1, min(self.leaf_streams, len(lv)))
