@@ -269,6 +269,32 @@ class Stepper:
         for cam in cams:
             self.run_view(cam, None, region=region, plan_only=True)
 
+    def _zeroed_g2d(self, rows):
+        """The compact 2D gradient [rows][12], zeroed on a side stream; the
+        event marks the end of the fill."""
+        dev = self.device
+        g2d = torch.empty(rows * 12, dtype=torch.float32, device=dev)
+        if self._fill_stream is None:
+            self._fill_stream = torch.cuda.Stream(device=dev)
+        self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(self._fill_stream):
+            g2d.zero_()
+        ready = torch.cuda.Event()
+        ready.record(self._fill_stream)
+        return g2d, ready
+
+    def _depth_order(self, proj, count, cap, clk):
+        """Candidates in depth order and their rects (gs_depth_order), for
+        `count` candidates (or GS_COUNT_ON_DEVICE) in buffers of `cap`."""
+        dev = self.device
+        order = torch.empty(cap, dtype=torch.int32, device=dev)
+        drect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
+        ows = torch.empty(B.gs_depth_order_workspace_size(cap), dtype=torch.uint8, device=dev)
+        tk = clk.tic("sort_depth")
+        B.gs_depth_order(proj, count, order, drect, ows, self.dev_status)
+        clk.toc(tk)
+        return order, drect
+
     def check(self):
         st = B.gs_check(self.dev_status)
         if st < 0:
@@ -368,24 +394,16 @@ class Stepper:
             # the GPU works while the host reads the tables and plans: the
             # compact 2D gradient, zeroed on a side stream (the raster
             # backward, its first user, waits for it), and the depth presort
-            # on the candidate count the projection left on the device
-            g2d = g2d_ready = None
-            if not plan_only:
-                g2d = torch.empty(cap * 12, dtype=torch.float32, device=dev)
-                if self._fill_stream is None:
-                    self._fill_stream = torch.cuda.Stream(device=dev)
-                self._fill_stream.wait_stream(torch.cuda.current_stream(dev))
-                with torch.cuda.stream(self._fill_stream):
-                    g2d.zero_()
-                g2d_ready = torch.cuda.Event()
-                g2d_ready.record(self._fill_stream)
-            order = torch.empty(cap, dtype=torch.int32, device=dev)
-            drect = torch.empty(cap * 4, dtype=torch.int16, device=dev)
-            ows = torch.empty(B.gs_depth_order_workspace_size(cap), dtype=torch.uint8, device=dev)
-            tk = clk.tic("sort_depth")
-            B.gs_depth_order(proj, B.GS_COUNT_ON_DEVICE, order, drect, ows, st)
-            clk.toc(tk)
-            del ows
+            # on the candidate count the projection left on the device.  Both
+            # are sized by the capacity; without a capacity hint (a region's
+            # first view, whose capacity is every Gaussian) they wait for the
+            # count instead, so that they are sized by it.
+            early = hint is not None or original
+            g2d = g2d_ready = order = drect = None
+            if early:
+                if not plan_only:
+                    g2d, g2d_ready = self._zeroed_g2d(cap)
+                order, drect = self._depth_order(proj, B.GS_COUNT_ON_DEVICE, cap, clk)
             tables_ready.synchronize()   # the one host wait per view
             if int(nc_h[0]) <= cap:
                 break
@@ -398,6 +416,10 @@ class Stepper:
         if expand:
             del bws
         C = int(nc_h[0])
+        if not early:
+            if not plan_only:
+                g2d, g2d_ready = self._zeroed_g2d(max(C, 1))
+            order, drect = self._depth_order(proj, C, max(C, 1), clk)
         if not original:
             self._cap_hint[hint_key] = C + C // 20 + 1024
         n_square = int(sq_h[0])
