@@ -239,8 +239,8 @@ __device__ __forceinline__ unsigned warp_mask(const Staged& st) {
 // One staged entry composited into a lane's pixel pairs, front to back.
 // alpha = min(0.99, o e^-q) = min(0.99, 2^(log2 o - q log2 e)) with
 // q = s1 (dx + beta dy)^2 + s2 dy^2, dx = gx - px, dy = gy - py, each step
-// one rounded operation (dx and dy once per pixel, t = beta dy + dx as one
-// fma, q log2 e as ns1 t^2 + ns2 dy^2 from one product and two fmas).
+// one rounded operation: dx and dy, t = fma(beta, dy, dx), and the exponent
+// fma(ns1 t, t, fma(ns2 dy, dy, log2 o)) with ns = -s log2 e.
 // Branch-free: every pixel evaluates.  A pixel that is done, skips the
 // entry or stops at it composites with a zero alpha, which leaves T and the
 // colour sums exactly as they were.  A packed fp32x2 operation rounds each
