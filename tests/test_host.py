@@ -174,3 +174,25 @@ def test_step_roofline_properties():
     st_b = s["raster_bwd"]
     assert abs(k["frac"] - st_b["roofline_ms"] / st_b["measured_ms"]) <= 1e-3
     assert k["lane_ops_per_step"] == st_b["lane_ops"]
+
+
+def test_committed_dram_record_matches_its_kernel_source():
+    """bench.py reports the dominant kernel's DRAM traffic from the committed
+    ncu record only while the kernel's source file is the one the counters
+    were taken on (else the traffic is null); the record in profiles/ is
+    current, and its scaling to another launch follows the algorithmic
+    bytes."""
+    import hashlib
+    import json
+    import bench
+    path = os.path.join(ROOT, "profiles", "k_raster_bwd_outdoor_3m_2k5_dram.json")
+    rec = json.load(open(path))
+    src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    assert hashlib.sha256(src).hexdigest() == rec["source_sha256"]
+    t, where = bench.profile_traffic("k_raster_bwd")
+    assert t == rec["dram_bytes_per_launch"] and where.endswith("_dram.json")
+    half = rec["alg_bytes_per_launch"] // 2
+    t2, _ = bench.profile_traffic("k_raster_bwd", half)
+    assert abs(t2 - rec["dram_bytes_per_launch"] * half / rec["alg_bytes_per_launch"]) <= 1
+    assert bench.raster_bwd_alg_bytes(1000, 100) == 1000 * 96 + 100 * 20
+    assert bench.profile_traffic("k_no_such_kernel") == (None, None)
